@@ -1,0 +1,447 @@
+#!/usr/bin/env python3
+"""Decode-attention throughput on B200: one JSON line on rank 0.
+
+A step is one decode step of one layer for the whole batch: for the c4a
+layer (the default workload) dsv4kv_index_topk followed by
+dsv4kv_sparse_decode; for the c128a layer dsv4kv_dense_decode.  The caches
+are resident in HBM (a KV cache is state, not a per-step input); two input
+replicas alternate so every step streams from DRAM rather than L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs its own batch (weak scaling, no collective on
+the data path); the time is the max over ranks.  `--impl reference` times the
+float64 CPU oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn steps/s per layer type; HBM GB/s vs ~8 TB/s peak, 1 B200"
+WORKLOADS = {
+    # name: (kind, batch, t, heads)
+    "c4a_b32": ("c4a", 32, 131072, 64),
+    "c128a_b8": ("c128a", 8, 131072, 64),
+    "c128a_b32": ("c128a", 32, 131072, 64),
+}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops", 1671.7)), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    def __init__(self, dev_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self._stop, self._t = period_s, threading.Event(), None
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            self.N, self.h = N, N.nvmlDeviceGetHandleByIndex(dev_index)
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM)
+        except Exception:
+            self.N = None
+
+    _NAMES = {0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+              0x80: "hw_power_brake_slowdown", 0x4: "sw_power_cap", 0x1: "gpu_idle", 0x2: "applications_clocks_setting"}
+
+    def _sample(self):
+        N = self.N
+        self.samples.append(N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM))
+        try:
+            r = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            r = N.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        for bit, name in self._NAMES.items():
+            if r & bit and name != "gpu_idle":
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.N:
+            self._sample()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.N:
+            self._stop.set()
+            self._t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ our arm
+class Layer:
+    """One layer's resident caches (R replicas) and per-step buffers on the GPU."""
+
+    def __init__(self, kind, batch, t, heads, seed, replicas):
+        import torch
+        import compressed_sparse_kv_b200 as K
+        import datagen.gpu as G
+        from datagen import workloads as WL
+        self.K, self.torch = K, torch
+        self.kind, self.batch, self.t, self.heads = kind, batch, t, heads
+        self.window, self.k = 128, 512
+        stride = 4 if kind == "c4a" else 128
+        self.n = (t - self.window) // stride
+        dev = "cuda"
+        self.reps = []
+        for r in range(replicas):
+            keys = WL.keys_for(seed, 1000 * r)
+            rep = {}
+            rep["comp"] = G.normal_bf16_(torch.empty(batch, self.n, 512, dtype=torch.bfloat16, device=dev), keys["comp"])
+            rep["win"] = G.normal_bf16_(torch.empty(batch, self.window, 512, dtype=torch.bfloat16, device=dev), keys["win"])
+            if kind == "c4a":
+                rep["kidx"] = G.int_bf16_(torch.empty(batch, self.n, 128, dtype=torch.bfloat16, device=dev), keys["kidx"])
+            self.reps.append(rep)
+        keys = WL.keys_for(seed, 0)
+        self.q = G.normal_bf16_(torch.empty(batch, heads, 512, dtype=torch.bfloat16, device=dev), keys["q"])
+        self.qidx = G.int_bf16_(torch.empty(batch, 128, dtype=torch.bfloat16, device=dev), keys["qidx"])
+        self.idx = torch.empty(batch, self.k, dtype=torch.int32, device=dev)
+        self.cnt = torch.empty(batch, dtype=torch.int32, device=dev)
+        self.out = torch.empty(batch, heads, 512, dtype=torch.bfloat16, device=dev)
+        if kind == "c4a":
+            self.ws_idx = K.new_workspace(K.index_topk_workspace_bytes(batch, self.n, self.k))
+            self.ws_dec = K.new_workspace(K.sparse_decode_workspace_bytes(batch, heads, self.k, self.window))
+        else:
+            self.ws_dec = K.new_workspace(K.dense_decode_workspace_bytes(batch, heads, self.n, self.window))
+
+    # algorithmic bytes of one step (indexer keys + rows read), and the q/out bytes
+    def alg_bytes(self):
+        rows = (self.k + self.window) if self.kind == "c4a" else (self.n + self.window)
+        b = self.batch * rows * 1024
+        if self.kind == "c4a":
+            b += self.batch * self.n * 256
+        return b
+
+    def index_bytes(self):
+        return self.batch * self.n * 256 + self.batch * 256
+
+    def launches_per_step(self):
+        return 4 if self.kind == "c4a" else 2
+
+    def index(self, r):
+        rep = self.reps[r]
+        self.K.index_topk(self.qidx, self.K.Cache(0, rep["kidx"], None, 128), self.n, self.k, idx_out=self.idx,
+                          count_out=self.cnt, ws=self.ws_idx)
+
+    def decode(self, r, q=None, out=None):
+        rep = self.reps[r]
+        K = self.K
+        q = self.q if q is None else q
+        out = self.out if out is None else out
+        if self.kind == "c4a":
+            K.sparse_decode(q, K.Cache(0, rep["comp"]), K.Cache(0, rep["win"]), self.idx, self.n, self.window, self.t,
+                            out=out, ws=self.ws_dec)
+        else:
+            K.dense_decode(q, K.Cache(0, rep["comp"]), K.Cache(0, rep["win"]), self.n, self.window, self.t, out=out,
+                           ws=self.ws_dec)
+
+
+def time_layer(layer, steps, warmup, dist_max, dev_index, sample_clocks):
+    """Device time of exactly `steps` steps (CUDA graphs per call, events per call)."""
+    torch = layer.torch
+    R = len(layer.reps)
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for i in range(max(warmup, 1)):
+            if layer.kind == "c4a":
+                layer.index(i % R)
+            layer.decode(i % R)
+    stream.synchronize()
+    # capture each call of each replica into its own graph
+    g_idx, g_dec = [], []
+    for r in range(R):
+        if layer.kind == "c4a":
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                layer.index(r)
+            g_idx.append(g)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            layer.decode(r)
+        g_dec.append(g)
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            if g_idx:
+                g_idx[i % R].replay()
+            g_dec[i % R].replay()
+    stream.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    dist_barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev_index) if sample_clocks else None
+    if sampler:
+        sampler.__enter__()
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            ev[i][0].record(stream)
+            if g_idx:
+                g_idx[i % R].replay()
+            ev[i][1].record(stream)
+            g_dec[i % R].replay()
+            ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.__exit__()
+    dist_barrier()
+    total_ms = ev[0][0].elapsed_time(ev[-1][2])
+    idx_ms = [e[0].elapsed_time(e[1]) for e in ev] if g_idx else [0.0]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = dist_max(total_ms)
+    return {"total_ms": total_ms, "index_ms": float(np.mean(idx_ms)), "decode_ms": float(np.mean(dec_ms)),
+            "clocks": sampler.summary() if sampler else None}
+
+
+def time_e2e(layer, steps):
+    """Same steps through the public API with host buffers: H2D of the step's
+    queries, the calls, D2H of the outputs, all inside the timed region."""
+    torch = layer.torch
+    R = len(layer.reps)
+    q_host = layer.q.cpu().pin_memory()
+    qi_host = layer.qidx.cpu().pin_memory()
+    out_host = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
+    q_dev, qi_dev = torch.empty_like(layer.q), torch.empty_like(layer.qidx)
+    stream = torch.cuda.Stream()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def step(i):
+        q_dev.copy_(q_host, non_blocking=True)
+        if layer.kind == "c4a":
+            qi_dev.copy_(qi_host, non_blocking=True)
+            layer.K.index_topk(qi_dev, layer.K.Cache(0, layer.reps[i % R]["kidx"], None, 128), layer.n, layer.k,
+                               idx_out=layer.idx, count_out=layer.cnt, ws=layer.ws_idx)
+        layer.decode(i % R, q=q_dev)
+        out_host.copy_(layer.out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            step(i)
+        stream.synchronize()
+        start.record(stream)
+        for i in range(steps):
+            step(i)
+        stop.record(stream)
+    stop.synchronize()
+    ms = start.elapsed_time(stop)
+    h2d = layer.q.numel() * 2 + (layer.qidx.numel() * 2 if layer.kind == "c4a" else 0)
+    return ms, h2d, layer.out.numel() * 2
+
+
+# ------------------------------------------------------------------ oracle arm
+def oracle_sample(kind, batch, t, heads, budget_s=12.0, seed=7):
+    """Seconds per sequence of the float64 oracle on one layer step (one
+    sequence of the batch, repeated within a time budget)."""
+    import datagen as D
+    from datagen import workloads as WL
+    from oracle import attention as OA
+    from oracle import formats as OF
+    from oracle import indexer as OI
+    window, k = 128, 512
+    n = (t - window) // (4 if kind == "c4a" else 128)
+    keys = WL.keys_for(seed, 0)
+    q = OF.bf16_bits_to_f64(D.rows_normal_bf16(keys["q"], np.arange(heads), 512))
+    win = OF.bf16_bits_to_f64(D.rows_normal_bf16(keys["win"], np.arange(window), 512))
+    if kind == "c4a":
+        kr = OF.bf16_bits_to_f64(D.rows_int_bf16(keys["kidx"], np.arange(n), 128))
+        qi = OF.bf16_bits_to_f64(D.rows_int_bf16(keys["qidx"], np.array([0]), 128)[0])
+        comp = None
+    else:
+        comp = OF.bf16_bits_to_f64(D.rows_normal_bf16(keys["comp"], np.arange(n), 512))
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        if kind == "c4a":
+            idx, cnt = OI.index_topk(qi, kr, k)
+            sel = OF.bf16_bits_to_f64(D.rows_normal_bf16(keys["comp"], idx[:cnt].astype(np.uint64), 512))
+            rows = np.concatenate([sel, win])
+            OA.shared_kv_decode(q, rows, 512 ** -0.5, t)
+        else:
+            OA.dense_decode(q[None], comp[None], win[None], t, 512 ** -0.5)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el > budget_s or reps >= 200:
+            break
+    return el / reps, reps
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:
+        return 1
+
+
+def cpu_baseline(kind, batch, t, heads, budget_s):
+    per_seq, reps = oracle_sample(kind, batch, t, heads, budget_s)
+    return {"value": 1.0 / (per_seq * batch), "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{reps} x one sequence of the {batch}-sequence step (float64 NumPy oracle), scaled to a step"}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+_dist = {"on": False}
+
+
+def dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        _dist.update(on=True, rank=dist.get_rank(), world=ws, local=int(os.environ.get("LOCAL_RANK", "0")))
+    else:
+        _dist.update(on=False, rank=0, world=1, local=0)
+    return _dist
+
+
+def dist_barrier():
+    if _dist["on"]:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def dist_max(x: float) -> float:
+    if not _dist["on"]:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="c4a_b32")
+    ap.add_argument("--secondary", default="c128a_b8,c128a_b32", help="extra per-layer-type workloads ('' = none)")
+    ap.add_argument("--replicas", type=int, default=2)
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    d = dist_init()
+    kind, batch, t, heads = WORKLOADS[args.workload]
+    wl_name = f"{kind} layer decode B={batch} t={t} H={heads} k=512 W=128 bf16 caches"
+
+    if args.impl == "reference":
+        if d["rank"] != 0:
+            return
+        per_seq, reps = oracle_sample(kind, batch, t, heads, budget_s=max(5.0, args.cpu_budget))
+        v = 1.0 / (per_seq * batch)
+        cb = {"value": v, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+              "sample": f"{reps} x one sequence of the {batch}-sequence step, scaled to a step"}
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": args.gpus,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / v,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                          "data": "synthetic", "config": {"workload": wl_name, "parallelism": f"dp{args.gpus}"},
+                          "cpu_baseline": cb,
+                          "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+              flush=True)
+        return
+
+    import torch
+    import compressed_sparse_kv_b200 as K
+    K.lib()
+    torch.cuda.set_device(d["local"])
+    hbm_peak, tf_peak, peak_src = measured_peaks()
+    seed = 1234 + d["rank"]
+    layer = Layer(kind, batch, t, heads, seed, args.replicas)
+    res = time_layer(layer, args.steps, args.warmup, dist_max, d["local"], sample_clocks=(d["rank"] == 0))
+    ms = res["total_ms"] / args.steps
+    steps_per_s = d["world"] * 1e3 / ms            # whole job: every rank ran `steps` steps
+    alg = layer.alg_bytes()
+    e2e_ms, h2d, d2h = time_e2e(layer, args.steps)
+    e2e_ms = dist_max(e2e_ms)
+    e2e_v = d["world"] * args.steps * 1e3 / e2e_ms
+
+    # roofline of the dominant call (the indexer for c4a, the dense decode for c128a)
+    if kind == "c4a":
+        dom_bytes, dom_ms, dom_name = layer.index_bytes(), res["index_ms"], "dsv4kv_index_topk (index_score + index_filter_select)"
+    else:
+        dom_bytes, dom_ms, dom_name = alg, res["decode_ms"], "dsv4kv_dense_decode (decode_kernel + decode_combine)"
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "kernel": dom_name, "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+            "frac": round(achieved / hbm_peak, 4), "peak_source": peak_src, "traffic": None,
+            "bytes_per_launch": dom_bytes, "avg_launch_ms": round(dom_ms, 5)}
+
+    per_type = {kind: {"workload": wl_name, "steps_per_s": round(steps_per_s, 1),
+                       "tokens_per_s": round(steps_per_s * batch, 1),
+                       "hbm_gbs": round(alg / (ms * 1e-3) / 1e9, 1),
+                       "frac_of_measured_hbm": round(alg / (ms * 1e-3) / 1e9 / hbm_peak, 4),
+                       "frac_of_8tbs": round(alg / (ms * 1e-3) / 8e12, 4),
+                       "index_ms": round(res["index_ms"], 5), "decode_ms": round(res["decode_ms"], 5)}}
+    for name in [s for s in args.secondary.split(",") if s and s != args.workload]:
+        k2, b2, t2, h2 = WORKLOADS[name]
+        L2 = Layer(k2, b2, t2, h2, seed + 99, max(args.replicas, 4 if b2 * t2 < 2 ** 21 else 2))
+        r2 = time_layer(L2, args.steps, args.warmup, dist_max, d["local"], sample_clocks=False)
+        ms2 = r2["total_ms"] / args.steps
+        a2 = L2.alg_bytes()
+        per_type.setdefault(k2 if k2 not in per_type else name, {}).update({
+            "workload": f"{k2} layer decode B={b2} t={t2} H={h2} W=128 bf16 caches",
+            "steps_per_s": round(d["world"] * 1e3 / ms2, 1), "hbm_gbs": round(a2 / (ms2 * 1e-3) / 1e9, 1),
+            "frac_of_measured_hbm": round(a2 / (ms2 * 1e-3) / 1e9 / hbm_peak, 4)})
+        del L2
+        torch.cuda.empty_cache()
+
+    line = {"metric": METRIC, "value": round(steps_per_s, 2), "unit": "steps/s", "n_gpus": d["world"],
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl_name, "batch_per_gpu": batch, "context": t, "heads": heads,
+                       "parallelism": f"dp{d['world']}",
+                       "l2": f"{args.replicas} cache replicas alternate; {alg / 1e6:.0f} MB read per step (> 126 MB L2)"},
+            "hbm_gbs": round(alg / (ms * 1e-3) / 1e9, 1), "alg_bytes_per_step": alg,
+            "per_layer_type": per_type, "roofline": roof,
+            "e2e": {"value": round(e2e_v, 2), "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": layer.launches_per_step() * args.steps,
+            "clocks": res["clocks"]}
+    if d["rank"] == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(kind, batch, t, heads, args.cpu_budget)
+    if d["rank"] == 0:
+        print(json.dumps(line), flush=True)
+    if _dist["on"]:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,221 @@
+"""Python binding of libdsv4kv (C ABI in include/dsv4kv.h).
+
+Argument marshalling only: every step of the path runs in the library's
+sm_100a kernels.  PyTorch provides device memory and the current stream.
+The binding raises if the shared library is missing or a call fails; there is
+no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdsv4kv.so")
+
+BF16, FP8_E4M3_ROW, FP4_E2M1_G16 = 0, 1, 2
+DEV_BAD_INDEX, DEV_TIMEOUT, DEV_INCONSISTENT = 0x1, 0x2, 0x4
+STATUS_NAMES = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED", 3: "ERR_WORKSPACE", 4: "ERR_CUDA"}
+
+
+class Dsv4kvError(RuntimeError):
+    def __init__(self, status: int, where: str, text: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {text}")
+        self.status = status
+
+
+class CacheDesc(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("dim", ctypes.c_int32), ("rows", ctypes.c_int64),
+                ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+_c = ctypes
+_SIGS = {
+    "dsv4kv_last_error": (_c.c_char_p, []),
+    "dsv4kv_version": (_c.c_char_p, []),
+    "dsv4kv_compress_entries": (_c.c_int64, [_c.c_int64, _c.c_int32, _c.c_int32]),
+    "dsv4kv_compress": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_int64, _c.c_int32, _c.c_int32,
+                                   _c.c_int32, _c.c_int32, _c.c_int64, _c.c_int32, _c.c_double, _c.c_int32,
+                                   _c.c_void_p, _c.c_void_p]),
+    "dsv4kv_quantize": (_c.c_int, [_c.c_void_p, _c.c_int32, _c.c_int64, _c.c_int32, _c.c_int32, _c.c_void_p,
+                                   _c.c_void_p, _c.c_void_p]),
+    "dsv4kv_index_topk_workspace_bytes": (_c.c_size_t, [_c.c_int32, _c.c_int64, _c.c_int32]),
+    "dsv4kv_index_topk": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.c_int32, _c.c_int64, _c.c_int32,
+                                     _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "dsv4kv_sparse_decode_workspace_bytes": (_c.c_size_t, [_c.c_int32, _c.c_int32, _c.c_int32, _c.c_int32,
+                                                           _c.c_int32]),
+    "dsv4kv_sparse_decode": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.POINTER(CacheDesc), _c.c_void_p,
+                                        _c.c_int32, _c.c_int32, _c.c_int64, _c.c_int32, _c.c_int32, _c.c_int64,
+                                        _c.c_float, _c.c_int32, _c.c_double, _c.c_int32, _c.c_void_p,
+                                        _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "dsv4kv_dense_decode_workspace_bytes": (_c.c_size_t, [_c.c_int32, _c.c_int32, _c.c_int32, _c.c_int64,
+                                                          _c.c_int32]),
+    "dsv4kv_dense_decode": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.POINTER(CacheDesc), _c.c_int32,
+                                       _c.c_int32, _c.c_int64, _c.c_int32, _c.c_int64, _c.c_float, _c.c_int32,
+                                       _c.c_double, _c.c_int32, _c.c_void_p, _c.c_void_p, _c.c_size_t,
+                                       _c.c_void_p]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libdsv4kv.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m compressed_sparse_kv_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise Dsv4kvError(status, where, lib().dsv4kv_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+@dataclass
+class Cache:
+    """A cache tensor [B][rows][dim] in one of the three formats."""
+    fmt: int
+    codes: torch.Tensor                      # bf16/u16 [B][rows][dim], u8 [B][rows][dim] or [B][rows][dim/2]
+    scales: Optional[torch.Tensor] = None    # None, f32 [B][rows], u8 [B][rows][dim/16]
+    dim: int = 512
+
+    @property
+    def rows(self) -> int:
+        return int(self.codes.shape[1]) if self.codes.dim() >= 2 else 0
+
+    def desc(self) -> CacheDesc:
+        return CacheDesc(self.fmt, self.dim, self.rows, _ptr(self.codes), _ptr(self.scales))
+
+
+def new_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """Zero-filled workspace (the library leaves it zeroed after each call)."""
+    return torch.zeros(max(int(nbytes), 16), dtype=torch.uint8, device=device or "cuda")
+
+
+def workspace_status(ws: torch.Tensor) -> int:
+    """The sticky device status word of a workspace (DEV_* flags)."""
+    return int(ws[:4].view(torch.int32).item())
+
+
+def compress_entries(t: int, window: int, stride: int) -> int:
+    return int(lib().dsv4kv_compress_entries(t, window, stride))
+
+
+def compress(s_raw: torch.Tensor, w: torch.Tensor, stride: int, window: int, pos0: int = 0, rope_dim: int = 64,
+             rope_base: float = 10000.0, out_fp32: bool = False, out: Optional[torch.Tensor] = None,
+             stream=None) -> torch.Tensor:
+    """s_raw bf16 [B][t][D], w f32 [K][D] -> entries [B][N][D] (bf16 or f32)."""
+    b, t, d = s_raw.shape
+    n = compress_entries(t, window, stride)
+    if out is None:
+        out = torch.empty((b, n, d), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=s_raw.device)
+    _check(lib().dsv4kv_compress(_ptr(s_raw), _ptr(w), b, t, d, int(w.shape[0]), stride, window, pos0, rope_dim,
+                                 rope_base, int(out_fp32), _ptr(out), _stream(stream)), "dsv4kv_compress")
+    return out
+
+
+def quantize(x: torch.Tensor, fmt: int, codes: Optional[torch.Tensor] = None,
+             scales: Optional[torch.Tensor] = None, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Rows x [..., D] (bf16 or f32) -> (codes, scales) in the fp8 or fp4 cache format."""
+    d = int(x.shape[-1])
+    rows = x.numel() // d
+    lead = tuple(x.shape[:-1])
+    if codes is None:
+        codes = torch.empty(lead + ((d,) if fmt == FP8_E4M3_ROW else (d // 2,)), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = (torch.empty(lead, dtype=torch.float32, device=x.device) if fmt == FP8_E4M3_ROW
+                  else torch.empty(lead + (d // 16,), dtype=torch.uint8, device=x.device))
+    _check(lib().dsv4kv_quantize(_ptr(x), int(x.dtype == torch.float32), rows, d, fmt, _ptr(codes), _ptr(scales),
+                                 _stream(stream)), "dsv4kv_quantize")
+    return codes, scales
+
+
+def index_topk_workspace_bytes(batch: int, n: int, k: int) -> int:
+    return int(lib().dsv4kv_index_topk_workspace_bytes(batch, n, k))
+
+
+def index_topk(qidx: torch.Tensor, keys: Cache, n: int, k: int, idx_out: Optional[torch.Tensor] = None,
+               count_out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+               stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """qidx bf16 [B][128], keys [B][>=n][128] -> (idx int32 [B][k] ascending, -1 padded; count int32 [B])."""
+    b = int(qidx.shape[0])
+    dev = qidx.device
+    if idx_out is None:
+        idx_out = torch.empty((b, k), dtype=torch.int32, device=dev)
+    if count_out is None:
+        count_out = torch.empty((b,), dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = new_workspace(index_topk_workspace_bytes(b, n, k), dev)
+    d = keys.desc()
+    _check(lib().dsv4kv_index_topk(_ptr(qidx), ctypes.byref(d), b, n, k, _ptr(idx_out), _ptr(count_out), _ptr(ws),
+                                   ws.numel(), _stream(stream)), "dsv4kv_index_topk")
+    return idx_out, count_out
+
+
+def sparse_decode_workspace_bytes(batch: int, heads: int, k: int, window: int, dim: int = 512) -> int:
+    return int(lib().dsv4kv_sparse_decode_workspace_bytes(batch, heads, dim, k, window))
+
+
+def dense_decode_workspace_bytes(batch: int, heads: int, n: int, window: int, dim: int = 512) -> int:
+    return int(lib().dsv4kv_dense_decode_workspace_bytes(batch, heads, dim, n, window))
+
+
+def sparse_decode(q: torch.Tensor, comp: Cache, win: Cache, idx: torch.Tensor, n: int, window: int, t: int,
+                  sm_scale: Optional[float] = None, rope_dim: int = 64, rope_base: float = 10000.0,
+                  out_fp32: bool = False, out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
+    """q bf16 [B][H][512] -> out [B][H][512]; idx int32 [B][k] from index_topk."""
+    b, h, d = q.shape
+    k = int(idx.shape[1])
+    if sm_scale is None:
+        sm_scale = d ** -0.5
+    if out is None:
+        out = torch.empty((b, h, d), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=q.device)
+    if ws is None:
+        ws = new_workspace(sparse_decode_workspace_bytes(b, h, k, window, d), q.device)
+    cd, wd = comp.desc(), win.desc()
+    _check(lib().dsv4kv_sparse_decode(_ptr(q), ctypes.byref(cd), ctypes.byref(wd), _ptr(idx), b, h, n, window, k, t,
+                                      sm_scale, rope_dim, rope_base, int(out_fp32), _ptr(out), _ptr(ws), ws.numel(),
+                                      _stream(stream)), "dsv4kv_sparse_decode")
+    return out
+
+
+def dense_decode(q: torch.Tensor, comp: Cache, win: Cache, n: int, window: int, t: int,
+                 sm_scale: Optional[float] = None, rope_dim: int = 64, rope_base: float = 10000.0,
+                 out_fp32: bool = False, out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """q bf16 [B][H][512] -> out [B][H][512] over all n compressed rows plus the window."""
+    b, h, d = q.shape
+    if sm_scale is None:
+        sm_scale = d ** -0.5
+    if out is None:
+        out = torch.empty((b, h, d), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=q.device)
+    if ws is None:
+        ws = new_workspace(dense_decode_workspace_bytes(b, h, n, window, d), q.device)
+    cd, wd = comp.desc(), win.desc()
+    _check(lib().dsv4kv_dense_decode(_ptr(q), ctypes.byref(cd), ctypes.byref(wd), b, h, n, window, t, sm_scale,
+                                     rope_dim, rope_base, int(out_fp32), _ptr(out), _ptr(ws), ws.numel(),
+                                     _stream(stream)), "dsv4kv_dense_decode")
+    return out

@@ -1,0 +1,238 @@
+// Exported C ABI of libdsv4kv: argument validation, workspace sizing and
+// kernel launches on the caller's stream.  No allocation, no host sync.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+#define DSV4KV_API extern "C" __attribute__((visibility("default")))
+
+namespace dsv4kv {
+
+static thread_local char g_err[512] = "";
+
+dsv4kv_status set_error(dsv4kv_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+dsv4kv_status check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(DSV4KV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return DSV4KV_OK;
+}
+
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t d0, uint64_t d1,
+                    uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2,
+                    CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  const cuuint32_t box[3] = {b0, b1, b2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static dsv4kv_status check_cache(const dsv4kv_cache* c, const char* what, int64_t need_rows, int dim) {
+  if (!c) return set_error(DSV4KV_ERR_INVALID_ARG, "%s: cache descriptor is null", what);
+  if (c->dim != dim) return set_error(DSV4KV_ERR_UNSUPPORTED, "%s: dim %d, expected %d", what, c->dim, dim);
+  if (c->rows < need_rows)
+    return set_error(DSV4KV_ERR_INVALID_ARG, "%s: %lld rows per sequence < %lld needed", what, (long long)c->rows,
+                     (long long)need_rows);
+  if (need_rows == 0) return DSV4KV_OK;
+  if (!c->codes || !aligned16(c->codes))
+    return set_error(DSV4KV_ERR_INVALID_ARG, "%s: codes pointer null or not 16-byte aligned", what);
+  if (c->fmt == DSV4KV_BF16) return DSV4KV_OK;
+  if (c->fmt == DSV4KV_FP8_E4M3_ROW || c->fmt == DSV4KV_FP4_E2M1_G16) {
+    if (!c->scales || !aligned16(c->scales))
+      return set_error(DSV4KV_ERR_INVALID_ARG, "%s: scales pointer null or not 16-byte aligned", what);
+    return DSV4KV_OK;
+  }
+  return set_error(DSV4KV_ERR_UNSUPPORTED, "%s: unknown format %d", what, c->fmt);
+}
+
+}  // namespace dsv4kv
+
+using namespace dsv4kv;
+
+DSV4KV_API const char* dsv4kv_last_error(void) { return g_err; }
+
+DSV4KV_API const char* dsv4kv_version(void) { return "dsv4kv 0.1 (sm_100a)"; }
+
+DSV4KV_API int64_t dsv4kv_compress_entries(int64_t t, int32_t window, int32_t stride) {
+  if (stride <= 0 || t < window) return 0;
+  return (t - window) / stride;
+}
+
+DSV4KV_API dsv4kv_status dsv4kv_compress(const void* s_raw, const float* w, int32_t batch, int64_t t, int32_t dim,
+                                         int32_t k_taps, int32_t stride, int32_t window, int64_t pos0,
+                                         int32_t rope_dim, double rope_base, int32_t out_fp32, void* out,
+                                         void* stream) {
+  g_err[0] = 0;
+  if (batch < 0 || t < 0 || k_taps < 1 || stride < 1 || window < 0)
+    return set_error(DSV4KV_ERR_INVALID_ARG, "compress: bad sizes");
+  if (rope_dim < 0 || rope_dim > dim || (rope_dim & 1))
+    return set_error(DSV4KV_ERR_INVALID_ARG, "compress: rope_dim must be even and <= dim");
+  if (!(rope_base > 0.0)) return set_error(DSV4KV_ERR_INVALID_ARG, "compress: rope_base must be > 0");
+  const int64_t n = dsv4kv_compress_entries(t, window, stride);
+  if (batch == 0 || n == 0) return DSV4KV_OK;
+  if (!s_raw || !w || !out || !aligned16(s_raw) || !aligned16(w) || !aligned16(out))
+    return set_error(DSV4KV_ERR_INVALID_ARG, "compress: null or misaligned pointer");
+  return compress_launch(s_raw, w, batch, t, dim, k_taps, stride, window, pos0, rope_dim, rope_base, out_fp32, out,
+                         static_cast<cudaStream_t>(stream));
+}
+
+DSV4KV_API dsv4kv_status dsv4kv_quantize(const void* in, int32_t in_fp32, int64_t rows, int32_t dim, int32_t fmt,
+                                         void* codes, void* scales, void* stream) {
+  g_err[0] = 0;
+  if (rows < 0) return set_error(DSV4KV_ERR_INVALID_ARG, "quantize: rows < 0");
+  if (fmt != DSV4KV_FP8_E4M3_ROW && fmt != DSV4KV_FP4_E2M1_G16)
+    return set_error(DSV4KV_ERR_UNSUPPORTED, "quantize: format %d is not a quantised format", fmt);
+  if (rows == 0) return DSV4KV_OK;
+  if (!in || !codes || !scales || !aligned16(in) || !aligned16(codes) || !aligned16(scales))
+    return set_error(DSV4KV_ERR_INVALID_ARG, "quantize: null or misaligned pointer");
+  return quantize_launch(in, in_fp32, rows, dim, fmt, codes, scales, static_cast<cudaStream_t>(stream));
+}
+
+DSV4KV_API size_t dsv4kv_index_topk_workspace_bytes(int32_t batch, int64_t n, int32_t k) {
+  if (batch < 0 || n < 0 || k < 1) return 0;
+  return index_topk_ws_bytes(batch, n, k);
+}
+
+DSV4KV_API dsv4kv_status dsv4kv_index_topk(const void* qidx, const dsv4kv_cache* keys, int32_t batch, int64_t n,
+                                           int32_t k, int32_t* idx_out, int32_t* count_out, void* ws,
+                                           size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  if (batch < 0 || n < 0) return set_error(DSV4KV_ERR_INVALID_ARG, "index_topk: bad sizes");
+  if (k < 1 || k > 2048) return set_error(DSV4KV_ERR_UNSUPPORTED, "index_topk: k must be in [1, 2048]");
+  if (batch == 0) return DSV4KV_OK;
+  if (!idx_out) return set_error(DSV4KV_ERR_INVALID_ARG, "index_topk: idx_out is null");
+  if (!keys) return set_error(DSV4KV_ERR_INVALID_ARG, "index_topk: keys is null");
+  if (keys->fmt != DSV4KV_BF16 && keys->fmt != DSV4KV_FP4_E2M1_G16)
+    return set_error(DSV4KV_ERR_UNSUPPORTED, "index_topk: keys must be bf16 or fp4");
+  dsv4kv_status st = check_cache(keys, "index_topk keys", n, 128);
+  if (st != DSV4KV_OK) return st;
+  if (n > k) {
+    if (!qidx || !aligned16(qidx)) return set_error(DSV4KV_ERR_INVALID_ARG, "index_topk: qidx null or misaligned");
+    if (int64_t(batch) * n > (int64_t(1) << 40)) return set_error(DSV4KV_ERR_UNSUPPORTED, "index_topk: too large");
+    if (!ws || ws_bytes < index_topk_ws_bytes(batch, n, k))
+      return set_error(DSV4KV_ERR_WORKSPACE, "index_topk: workspace null or too small");
+  }
+  return index_topk_launch(static_cast<const uint16_t*>(qidx), *keys, batch, n, k, idx_out, count_out, ws, ws_bytes,
+                           static_cast<cudaStream_t>(stream));
+}
+
+static dsv4kv_status check_decode(const void* q, const dsv4kv_cache* comp, const dsv4kv_cache* win, int32_t batch,
+                                  int32_t heads, int64_t n, int32_t window, int64_t need_comp_rows, const void* out) {
+  if (batch < 1) return set_error(DSV4KV_ERR_INVALID_ARG, "decode: batch must be >= 1");
+  if (heads < 1 || heads > 64) return set_error(DSV4KV_ERR_UNSUPPORTED, "decode: heads must be in [1, 64]");
+  if (n < 0 || window < 0) return set_error(DSV4KV_ERR_INVALID_ARG, "decode: negative sizes");
+  if (!q || !aligned16(q) || !out || !aligned16(out))
+    return set_error(DSV4KV_ERR_INVALID_ARG, "decode: q/out null or misaligned");
+  if (!comp || !win) return set_error(DSV4KV_ERR_INVALID_ARG, "decode: cache descriptor is null");
+  dsv4kv_status st = check_cache(comp, "decode comp", need_comp_rows, 512);
+  if (st != DSV4KV_OK) return st;
+  st = check_cache(win, "decode window", window, 512);
+  if (st != DSV4KV_OK) return st;
+  if (int64_t(batch) * std::max<int64_t>(comp->rows, 1) >= (int64_t(1) << 31) ||
+      int64_t(batch) * std::max<int64_t>(win->rows, 1) >= (int64_t(1) << 31))
+    return set_error(DSV4KV_ERR_UNSUPPORTED, "decode: batch x rows must be < 2^31");
+  return DSV4KV_OK;
+}
+
+DSV4KV_API size_t dsv4kv_sparse_decode_workspace_bytes(int32_t batch, int32_t heads, int32_t dim, int32_t k,
+                                                       int32_t window) {
+  if (batch < 1 || heads < 1 || k < 0 || window < 0) return 0;
+  return decode_ws_bytes(batch, heads, dim, int64_t(k) + window);
+}
+
+DSV4KV_API size_t dsv4kv_dense_decode_workspace_bytes(int32_t batch, int32_t heads, int32_t dim, int64_t n,
+                                                      int32_t window) {
+  if (batch < 1 || heads < 1 || n < 0 || window < 0) return 0;
+  return decode_ws_bytes(batch, heads, dim, n + window);
+}
+
+DSV4KV_API dsv4kv_status dsv4kv_sparse_decode(const void* q, const dsv4kv_cache* comp, const dsv4kv_cache* win,
+                                              const int32_t* idx, int32_t batch, int32_t heads, int64_t n,
+                                              int32_t window, int32_t k, int64_t t, float sm_scale,
+                                              int32_t rope_dim, double rope_base, int32_t out_fp32, void* out,
+                                              void* ws, size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  if (k < 0 || k > 2048) return set_error(DSV4KV_ERR_UNSUPPORTED, "sparse_decode: k must be in [0, 2048]");
+  dsv4kv_status st = check_decode(q, comp, win, batch, heads, n, window, n, out);
+  if (st != DSV4KV_OK) return st;
+  if (k > 0 && n > 0 && !idx) return set_error(DSV4KV_ERR_INVALID_ARG, "sparse_decode: idx is null");
+  if (rope_dim < 0 || rope_dim > 512 || (rope_dim & 1))
+    return set_error(DSV4KV_ERR_INVALID_ARG, "sparse_decode: bad rope_dim");
+  if (!ws || ws_bytes < dsv4kv_sparse_decode_workspace_bytes(batch, heads, 512, k, window))
+    return set_error(DSV4KV_ERR_WORKSPACE, "sparse_decode: workspace null or too small");
+  DecodeArgs a{q, *comp, *win, idx, batch, heads, 512, n, window, k, t, sm_scale, rope_dim, rope_base, out_fp32, out};
+  return decode_launch(a, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+DSV4KV_API dsv4kv_status dsv4kv_dense_decode(const void* q, const dsv4kv_cache* comp, const dsv4kv_cache* win,
+                                             int32_t batch, int32_t heads, int64_t n, int32_t window, int64_t t,
+                                             float sm_scale, int32_t rope_dim, double rope_base, int32_t out_fp32,
+                                             void* out, void* ws, size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  dsv4kv_status st = check_decode(q, comp, win, batch, heads, n, window, n, out);
+  if (st != DSV4KV_OK) return st;
+  if (rope_dim < 0 || rope_dim > 512 || (rope_dim & 1))
+    return set_error(DSV4KV_ERR_INVALID_ARG, "dense_decode: bad rope_dim");
+  if (n > (int64_t(1) << 30)) return set_error(DSV4KV_ERR_UNSUPPORTED, "dense_decode: n too large");
+  if (!ws || ws_bytes < dsv4kv_dense_decode_workspace_bytes(batch, heads, 512, n, window))
+    return set_error(DSV4KV_ERR_WORKSPACE, "dense_decode: workspace null or too small");
+  DecodeArgs a{q, *comp, *win, nullptr, batch, heads, 512, n, window, 0, t, sm_scale, rope_dim, rope_base, out_fp32, out};
+  return decode_launch(a, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}

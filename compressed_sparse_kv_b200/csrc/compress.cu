@@ -1,0 +1,125 @@
+// c4a / c128a compressors.
+//
+// [P1] "c4a (the milder scheme)": each compressed entry is a learned weighted
+// sum of 8 states, the next entry shifted by 4; "c128a (the aggressive
+// scheme)": 128 states at stride 128.  [P2] Step 4: C4A[1] = mix(S0..S7),
+// C4A[2] = mix(S4..S11), C128A[0] = mix(S0..S127).  Entry i of stride s with
+// K taps mixes positions s*i + s - K + j (j < K; positions < 0 contribute 0),
+// per channel, then rotates its rotary channel pairs at position pos0 + s*i.
+//
+// Layout of the work: one warp per entry, each lane owns 16 consecutive
+// channels (two 16-byte bf16 loads per tap row), so a tap row is one fully
+// coalesced 1 KB read.  The K tap loads are unrolled by 4 to keep several
+// rows in flight; c4a entries overlap by 4 rows, which the L1/L2 absorb.
+#include <cmath>
+#include <cstdint>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dsv4kv {
+
+namespace {
+
+constexpr int kWarpsPerBlock = 8;
+
+template <int PER>  // channels per lane (dim / 32)
+__global__ void __launch_bounds__(32 * kWarpsPerBlock)
+    compress_kernel(const uint16_t* __restrict__ s_raw, const float* __restrict__ w, int64_t t, int k_taps,
+                    int stride, int64_t n_entries, int64_t pos0, int rope_dim, double rope_base, int out_fp32,
+                    void* __restrict__ out) {
+  constexpr int D = 32 * PER;
+  const int lane = threadIdx.x & 31;
+  const int b = blockIdx.y;
+  const int64_t i = int64_t(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5);
+  if (i >= n_entries) return;
+  const int c0 = PER * lane;
+  const uint16_t* sb = s_raw + size_t(b) * size_t(t) * D + c0;
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  const int64_t first = int64_t(stride) * i + stride - k_taps;
+  const int j0 = first < 0 ? int(-first) : 0;  // skip taps before position 0
+#pragma unroll 4
+  for (int j = j0; j < k_taps; ++j) {
+    const uint16_t* row = sb + size_t(first + j) * D;
+    const float* wr = w + size_t(j) * D + c0;
+#pragma unroll
+    for (int v = 0; v < PER / 8; ++v) {
+      const uint4 x = *reinterpret_cast<const uint4*>(row + 8 * v);
+      const float4 wa = *reinterpret_cast<const float4*>(wr + 8 * v);
+      const float4 wb = *reinterpret_cast<const float4*>(wr + 8 * v + 4);
+      acc[8 * v + 0] = fmaf(wa.x, bf16lo(x.x), acc[8 * v + 0]);
+      acc[8 * v + 1] = fmaf(wa.y, bf16hi(x.x), acc[8 * v + 1]);
+      acc[8 * v + 2] = fmaf(wa.z, bf16lo(x.y), acc[8 * v + 2]);
+      acc[8 * v + 3] = fmaf(wa.w, bf16hi(x.y), acc[8 * v + 3]);
+      acc[8 * v + 4] = fmaf(wb.x, bf16lo(x.z), acc[8 * v + 4]);
+      acc[8 * v + 5] = fmaf(wb.y, bf16hi(x.z), acc[8 * v + 5]);
+      acc[8 * v + 6] = fmaf(wb.z, bf16lo(x.w), acc[8 * v + 6]);
+      acc[8 * v + 7] = fmaf(wb.w, bf16hi(x.w), acc[8 * v + 7]);
+    }
+  }
+  // RoPE at the block's first position (fp64 angle; the pair index m of
+  // channel c is (c - (D - rope_dim)) / 2).
+  const int r0 = D - rope_dim;
+  if (c0 + PER > r0) {
+    const double pos = double(pos0 + int64_t(stride) * i);
+#pragma unroll
+    for (int e = 0; e < PER; e += 2) {
+      const int c = c0 + e;
+      if (c >= r0) {
+        const int m = (c - r0) >> 1;
+        const double theta = pow(rope_base, -2.0 * double(m) / double(rope_dim));
+        double sn, cs;
+        sincos(pos * theta, &sn, &cs);
+        const float x = acc[e], y = acc[e + 1];
+        acc[e] = float(double(x) * cs - double(y) * sn);
+        acc[e + 1] = float(double(x) * sn + double(y) * cs);
+      }
+    }
+  }
+  const size_t o = (size_t(b) * size_t(n_entries) + size_t(i)) * D + c0;
+  if (out_fp32) {
+    float* op = static_cast<float*>(out) + o;
+#pragma unroll
+    for (int v = 0; v < PER / 4; ++v)
+      *reinterpret_cast<float4*>(op + 4 * v) = make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+  } else {
+    uint16_t* op = static_cast<uint16_t*>(out) + o;
+#pragma unroll
+    for (int v = 0; v < PER / 8; ++v)
+      *reinterpret_cast<uint4*>(op + 8 * v) =
+          make_uint4(pack_bf16x2(acc[8 * v], acc[8 * v + 1]), pack_bf16x2(acc[8 * v + 2], acc[8 * v + 3]),
+                     pack_bf16x2(acc[8 * v + 4], acc[8 * v + 5]), pack_bf16x2(acc[8 * v + 6], acc[8 * v + 7]));
+  }
+}
+
+}  // namespace
+
+dsv4kv_status compress_launch(const void* s_raw, const float* w, int batch, int64_t t, int dim, int k_taps,
+                              int stride, int window, int64_t pos0, int rope_dim, double rope_base,
+                              int out_fp32, void* out, cudaStream_t stream) {
+  const int64_t n = std::max<int64_t>(0, (t - window) / stride);
+  if (n == 0) return DSV4KV_OK;
+  dim3 grid(unsigned((n + kWarpsPerBlock - 1) / kWarpsPerBlock), unsigned(batch));
+  const uint16_t* s = static_cast<const uint16_t*>(s_raw);
+  switch (dim) {
+    case 256:
+      compress_kernel<8><<<grid, 32 * kWarpsPerBlock, 0, stream>>>(s, w, t, k_taps, stride, n, pos0, rope_dim,
+                                                                  rope_base, out_fp32, out);
+      break;
+    case 512:
+      compress_kernel<16><<<grid, 32 * kWarpsPerBlock, 0, stream>>>(s, w, t, k_taps, stride, n, pos0, rope_dim,
+                                                                   rope_base, out_fp32, out);
+      break;
+    case 1024:
+      compress_kernel<32><<<grid, 32 * kWarpsPerBlock, 0, stream>>>(s, w, t, k_taps, stride, n, pos0, rope_dim,
+                                                                   rope_base, out_fp32, out);
+      break;
+    default:
+      return set_error(DSV4KV_ERR_UNSUPPORTED, "compress: dim must be 256, 512 or 1024 (got %d)", dim);
+  }
+  return check_launch("compress_kernel");
+}
+
+}  // namespace dsv4kv

@@ -1,0 +1,57 @@
+// Host-side declarations shared by the dsv4kv translation units (not exported).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "dsv4kv.h"
+
+namespace dsv4kv {
+
+dsv4kv_status set_error(dsv4kv_status st, const char* fmt, ...);
+dsv4kv_status check_launch(const char* what);
+int sm_count();
+
+// Driver entry point for cuTensorMapEncodeTiled (resolved once through the runtime).
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                    uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                    CUtensorMapSwizzle swizzle);
+bool encode_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t d0, uint64_t d1,
+                    uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1,
+                    uint32_t b2, CUtensorMapSwizzle swizzle);
+
+size_t index_topk_ws_bytes(int batch, int64_t n, int k);
+dsv4kv_status index_topk_launch(const uint16_t* qidx, const dsv4kv_cache& keys, int batch, int64_t n, int k,
+                                int32_t* idx_out, int32_t* count_out, void* ws, size_t ws_bytes,
+                                cudaStream_t stream);
+
+struct DecodeArgs {
+  const void* q;
+  dsv4kv_cache comp;
+  dsv4kv_cache win;
+  const int32_t* idx;  // null for dense
+  int batch, heads, dim;
+  int64_t n;
+  int window;
+  int k;  // sparse only
+  int64_t t;
+  float sm_scale;
+  int rope_dim;
+  double rope_base;
+  int out_fp32;
+  void* out;
+};
+size_t decode_ws_bytes(int batch, int heads, int dim, int64_t rows_per_seq);
+dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+dsv4kv_status compress_launch(const void* s_raw, const float* w, int batch, int64_t t, int dim, int k_taps,
+                              int stride, int window, int64_t pos0, int rope_dim, double rope_base,
+                              int out_fp32, void* out, cudaStream_t stream);
+
+dsv4kv_status quantize_launch(const void* in, int in_fp32, int64_t rows, int dim, int fmt, void* codes,
+                              void* scales, cudaStream_t stream);
+
+}  // namespace dsv4kv

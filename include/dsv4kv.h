@@ -1,0 +1,187 @@
+/*
+ * dsv4kv — decode attention over DeepSeek-V4-style hybrid compressed KV caches
+ * on NVIDIA B200 (sm_100a).  C ABI.
+ *
+ * Sources the operations follow (web pages, cited by title and section):
+ *  [P1] "How DeepSeek V4 Uses Less Memory: KV Cache Explained"
+ *  [P2] "DeepSeek V4 KV Cache" visual walkthrough
+ *  [P3] "KV cache at 890 bytes per token: how DeepSeek squeezed attention memory"
+ *
+ * Conventions shared by every call
+ *  - Every pointer argument that names tensor data is DEVICE memory owned by
+ *    the caller (for example allocated through PyTorch).  The library keeps
+ *    no pointer after a call returns and allocates no device memory on any
+ *    call path; scratch memory is the caller's workspace.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream) and never synchronises the host.
+ *  - Tensors are dense and row-major with the shapes given below.
+ *  - bf16 data is passed as 16-bit words (IEEE binary32 upper halves).
+ *  - Return value: DSV4KV_OK or an error code; on an error nothing was
+ *    launched (DSV4KV_ERR_CUDA: a launch failed — the text is in
+ *    dsv4kv_last_error(), and the workspace must be zero-filled again).
+ *  - Workspaces: `*_workspace_bytes` gives the size; a workspace must be
+ *    zero-filled once before its first use and is left in that state by every
+ *    successful call, so it can be reused by the next call on the same stream.
+ *    Calls that run concurrently need separate workspaces.  The first 4 bytes
+ *    of a workspace are a sticky device status word: kernels OR the
+ *    DSV4KV_DEV_* flags below into it and never trap or hang; the caller
+ *    reads and clears it.
+ */
+#ifndef DSV4KV_H_
+#define DSV4KV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSV4KV_OK = 0,
+  DSV4KV_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer  */
+  DSV4KV_ERR_UNSUPPORTED = 2,  /* a format or dimension this build lacks      */
+  DSV4KV_ERR_WORKSPACE = 3,    /* workspace null or smaller than required     */
+  DSV4KV_ERR_CUDA = 4          /* CUDA runtime/driver error at launch         */
+} dsv4kv_status;
+
+/* Device status flags (OR-ed into the first word of a workspace). */
+#define DSV4KV_DEV_BAD_INDEX 0x1u  /* a selected index was outside [0, n): row skipped */
+#define DSV4KV_DEV_TIMEOUT 0x2u    /* a bounded wait gave up: outputs are invalid       */
+#define DSV4KV_DEV_INCONSISTENT 0x4u /* selection counts disagreed: outputs are invalid */
+
+/* Cache row formats.
+ *  DSV4KV_BF16:          codes = bf16 [B][rows][dim]; scales = NULL.
+ *  DSV4KV_FP8_E4M3_ROW:  codes = u8 [B][rows][dim] (OCP E4M3); scales = float [B][rows];
+ *                        value = E4M3(code) * scale.  ([P1] "the attention cache uses fp8",
+ *                        "decode uses partly token-wise fp8")
+ *  DSV4KV_FP4_E2M1_G16:  codes = u8 [B][rows][dim/2], two OCP E2M1 codes per byte, the
+ *                        even channel in the low nibble; scales = u8 [B][rows][dim/16] E4M3,
+ *                        one per 16 channels; value = E2M1(code) * E4M3(scale).
+ *                        ([P3] "storing the main KV in FP4"; [P1] "indexer cache uses fp4")
+ */
+typedef enum {
+  DSV4KV_BF16 = 0,
+  DSV4KV_FP8_E4M3_ROW = 1,
+  DSV4KV_FP4_E2M1_G16 = 2
+} dsv4kv_format;
+
+/* A cache tensor of `batch` sequences x `rows` rows x `dim` channels.
+ * `rows` is the per-sequence row capacity (the batch stride in rows). */
+typedef struct {
+  int32_t fmt;          /* dsv4kv_format */
+  int32_t dim;          /* channels per row */
+  int64_t rows;         /* rows per sequence */
+  const void* codes;    /* device pointer, layout per format, 16-byte aligned */
+  const void* scales;   /* device pointer or NULL for bf16, 16-byte aligned   */
+} dsv4kv_cache;
+
+/* ---------------------------------------------------------------------------
+ * Compressor.  [P1] "c4a (the milder scheme)": each entry is a weighted sum of
+ * 8 states with stride 4; "c128a (the aggressive scheme)": 128 states, stride
+ * 128.  [P2] Step 4: C4A[1] mixes S0..S7, C4A[2] mixes S4..S11, C128A[0] is
+ * S0..S127.
+ *
+ * For entry i < N = max(0, floor((t - window) / stride)) and channel c:
+ *   out[b][i][c] = rope( sum_{j<k_taps} w[j][c] * s_raw[b][stride*i + stride - k_taps + j][c] )
+ * where taps at a position < 0 contribute nothing, and rope rotates channel
+ * pairs (dim-rope_dim+2m, dim-rope_dim+2m+1) by the angle
+ * (pos0 + stride*i) * rope_base^(-2m/rope_dim)  ([P1] "Shared key and value").
+ *   s_raw : bf16 [batch][t][dim]   (row 0 is at position pos0)
+ *   w     : float [k_taps][dim]
+ *   out   : bf16 or (out_fp32 != 0) float, [batch][N][dim]
+ * Requirements: dim in {256, 512, 1024}, rope_dim even, 0 <= rope_dim <= dim,
+ * 1 <= k_taps, 1 <= stride, window >= 0.  N == 0 launches nothing.
+ * ------------------------------------------------------------------------ */
+int64_t dsv4kv_compress_entries(int64_t t, int32_t window, int32_t stride);
+
+dsv4kv_status dsv4kv_compress(const void* s_raw, const float* w, int32_t batch, int64_t t,
+                              int32_t dim, int32_t k_taps, int32_t stride, int32_t window,
+                              int64_t pos0, int32_t rope_dim, double rope_base,
+                              int32_t out_fp32, void* out, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Quantiser.  [P1] quantisation paragraphs (fp8 attention cache, fp4 indexer
+ * cache); [P3] fp4 E2M1 main cache with one E4M3 scale per 16 channels.
+ *   DSV4KV_FP8_E4M3_ROW: scale = fp32(amax / 448) (1 if amax == 0),
+ *       code = E4M3(fp32(x / scale)), round to nearest even, saturating.
+ *   DSV4KV_FP4_E2M1_G16: s = E4M3(fp32(amax16 / 6)) (nearest even,
+ *       saturating), code = E2M1(fp32(x / s)) nearest even, saturating;
+ *       codes are 0 when s == 0.
+ *   in     : bf16 or (in_fp32 != 0) float, [rows][dim]
+ *   codes  : u8 [rows][dim] (fp8) or [rows][dim/2] (fp4)
+ *   scales : float [rows] (fp8) or u8 [rows][dim/16] (fp4)
+ * Requirements: dim in {128, 256, 512, 1024}; fmt != DSV4KV_BF16.
+ * ------------------------------------------------------------------------ */
+dsv4kv_status dsv4kv_quantize(const void* in, int32_t in_fp32, int64_t rows, int32_t dim,
+                              int32_t fmt, void* codes, void* scales, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Lightning indexer + top-k.  [P1] "c4a": DeepSeek Sparse Attention picks the
+ * top-k compressed entries per query (k = 512); [P2] Step 5: a learned indexer
+ * scores the compressed blocks.
+ *   score[b][n] = sum_d qidx[b][d] * key[b][n][d]     (fp32 accumulation)
+ * The selected set is the first min(k, n) entries under (score descending,
+ * index ascending) — ties go to the lower index.  It is written in ascending
+ * index order to idx_out[b][0..count), and idx_out[b][count..k) = -1.
+ *   qidx     : bf16 [batch][dim]
+ *   keys     : cache of dim channels (BF16 or FP4_E2M1_G16), rows >= n
+ *   idx_out  : int32 [batch][k];  count_out : int32 [batch] (may be NULL)
+ * Requirements: dim == 128; 1 <= k <= 2048; n >= 0.  Scores are exact (and
+ * the selection bit-exact) when every product and partial sum is an integer
+ * below 2^24, as for the small-integer indexer inputs of the workloads.
+ * ------------------------------------------------------------------------ */
+size_t dsv4kv_index_topk_workspace_bytes(int32_t batch, int64_t n, int32_t k);
+
+dsv4kv_status dsv4kv_index_topk(const void* qidx, const dsv4kv_cache* keys, int32_t batch,
+                                int64_t n, int32_t k, int32_t* idx_out, int32_t* count_out,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Decode attention with shared K/V.  [P2] Step 3: one cached vector S_j is
+ * both key (score = Q.S_j) and value; [P1] "The sliding window": a 128-token
+ * exact window; [P1] "Shared key and value": inverse RoPE on the output.
+ *
+ * For each sequence b and head h, with rows R = {selected compressed rows}
+ * followed by the `window` window rows:
+ *   p   = softmax_r( sm_scale * q[b][h] . R[r] )          (one softmax over all rows)
+ *   o   = sum_r p[r] * R[r]
+ *   out = o with channel pairs (dim-rope_dim+2m, +1) rotated by -t * rope_base^(-2m/rope_dim)
+ *   q    : bf16 [batch][heads][dim], already rotated at position t
+ *   comp : compressed cache, rows >= n;  win : window cache, rows >= window
+ *   idx  : int32 [batch][k], ascending, -1 padded (dsv4kv_index_topk output);
+ *          an index outside [0, n) is skipped and flags DSV4KV_DEV_BAD_INDEX
+ *   out  : bf16 or (out_fp32 != 0) float, [batch][heads][dim]
+ * Requirements: dim == 512; 1 <= heads <= 64; comp and win of the same dim;
+ * 0 <= window; k <= 2048.  The dense call reads all n compressed rows
+ * ([P1] "c128a": full attention over the compressed entries).
+ * ------------------------------------------------------------------------ */
+size_t dsv4kv_sparse_decode_workspace_bytes(int32_t batch, int32_t heads, int32_t dim,
+                                            int32_t k, int32_t window);
+
+dsv4kv_status dsv4kv_sparse_decode(const void* q, const dsv4kv_cache* comp,
+                                   const dsv4kv_cache* win, const int32_t* idx, int32_t batch,
+                                   int32_t heads, int64_t n, int32_t window, int32_t k,
+                                   int64_t t, float sm_scale, int32_t rope_dim,
+                                   double rope_base, int32_t out_fp32, void* out, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+size_t dsv4kv_dense_decode_workspace_bytes(int32_t batch, int32_t heads, int32_t dim,
+                                           int64_t n, int32_t window);
+
+dsv4kv_status dsv4kv_dense_decode(const void* q, const dsv4kv_cache* comp,
+                                  const dsv4kv_cache* win, int32_t batch, int32_t heads,
+                                  int64_t n, int32_t window, int64_t t, float sm_scale,
+                                  int32_t rope_dim, double rope_base, int32_t out_fp32,
+                                  void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Text of the last error on the calling host thread ("" if none). */
+const char* dsv4kv_last_error(void);
+
+/* Library version string. */
+const char* dsv4kv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DSV4KV_H_ */

@@ -1,0 +1,31 @@
+"""Small helpers shared by the tests (tolerances, dtype conversion)."""
+import numpy as np
+import torch
+
+# Tolerances for floating-point outputs (compressor and attention) against
+# the float64 oracle: max-abs <= 1e-2 and relative L2 <= 5e-3.
+MAX_ABS = 1e-2
+REL_L2 = 5e-3
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def from_bits(bits: np.ndarray, device="cuda") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(torch.bfloat16)
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+def assert_close(got, ref, max_abs=MAX_ABS, rel_l2=REL_L2, what=""):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    err = np.abs(got - ref)
+    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert err.max() <= max_abs and rel <= rel_l2, f"{what}: max-abs {err.max():.3e} rel-L2 {rel:.3e}"
+    return float(err.max()), float(rel)

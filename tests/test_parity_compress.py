@@ -1,0 +1,57 @@
+"""dsv4kv_compress against the oracle (c4a and c128a, bf16 and fp32 outputs)."""
+import numpy as np
+import pytest
+import torch
+
+import compressed_sparse_kv_b200 as K
+import datagen as D
+from oracle import compress as OC
+from oracle import formats as OF
+from tests._util import assert_close, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _raw(seed, b, t, d=512):
+    import datagen.gpu as G
+    key = D.stream_key(seed, D.TID_RAW_S, 0)
+    return G.normal_bf16_(torch.empty(b, t, d, dtype=torch.bfloat16, device="cuda"), key), key
+
+
+@pytest.mark.parametrize("kind,b,t,window,pos0", [
+    ("c4a", 1, 2048, 128, 0),          # tiny c4a: 480 entries
+    ("c4a", 2, 1000 + 3, 128, 0),      # ragged t
+    ("c4a", 1, 4096, 0, 1 << 20),      # no window, large positions
+    ("c128a", 2, 128 * 20 + 128 + 50, 128, 0),
+    ("c128a", 1, 131072, 128, 0),      # c128a t=131072: 1023 entries
+])
+@pytest.mark.parametrize("out_fp32", [True, False])
+def test_compress(kind, b, t, window, pos0, out_fp32):
+    s, k = (4, 8) if kind == "c4a" else (128, 128)
+    raw, key = _raw(hash((kind, t)) % 1000, b, t)
+    w = D.compress_weights(5, 0, k, 512)
+    out = K.compress(raw, torch.from_numpy(w).cuda(), s, window, pos0=pos0, out_fp32=out_fp32)
+    n = OC.n_entries(t, window, s)
+    assert out.shape == (b, n, 512)
+    got = to_f64(out)
+    for bb in range(b):
+        r = OF.bf16_bits_to_f64(D.normal_bf16(key, t * 512, offset=bb * t * 512).reshape(t, 512))
+        ref = OC.compress(r, w.astype(np.float64), s, window, pos0=pos0)
+        if not out_fp32:
+            ref_stored = OF.round_bf16(ref)
+            assert_close(got[bb], ref_stored, what=f"{kind} seq {bb}")
+        assert_close(got[bb], ref, what=f"{kind} seq {bb}")
+        if out_fp32:
+            assert np.abs(got[bb] - ref).max() < 1e-4       # fp32 accumulation of <= 128 taps
+
+
+def test_window_rows_are_one_tap_compression():
+    """K = 1, stride 1, weight 1: the entries are the raw rows rotated at their positions."""
+    t, W = 3000, 128
+    raw, key = _raw(3, 1, t)
+    w = torch.ones(1, 512, dtype=torch.float32, device="cuda")
+    win = K.compress(raw[:, t - W:].contiguous(), w, 1, 0, pos0=t - W, out_fp32=True)
+    r = OF.bf16_bits_to_f64(D.normal_bf16(key, t * 512).reshape(t, 512))
+    from oracle import rope as OR
+    ref = OR.rope(r[t - W:], np.arange(t - W, t))
+    assert_close(to_f64(win)[0], ref, max_abs=1e-5, rel_l2=1e-6)
