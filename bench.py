@@ -409,7 +409,7 @@ def main():
                        "frac_of_measured_hbm": round(alg / (ms * 1e-3) / 1e9 / hbm_peak, 4),
                        "frac_of_8tbs": round(alg / (ms * 1e-3) / 8e12, 4),
                        "index_ms": round(res["index_ms"], 5), "decode_ms": round(res["decode_ms"], 5)}}
-    for name in [s for s in args.secondary.split(",") if s and s != args.workload]:
+    for name in [s for s in args.secondary.split(",") if s and s not in ("none", args.workload)]:
         k2, b2, t2, h2 = WORKLOADS[name]
         L2 = Layer(k2, b2, t2, h2, seed + 99, max(args.replicas, 4 if b2 * t2 < 2 ** 21 else 2))
         r2 = time_layer(L2, args.steps, args.warmup, dist_max, d["local"], sample_clocks=False)

@@ -35,19 +35,34 @@ namespace {
 constexpr int kTileRows = 64;
 constexpr int kStages = 2;
 constexpr int kDim = 512;
-constexpr int kChunks = kDim / 64;              // 64-channel (128-byte) column chunks
-constexpr int kChunkBytes = kTileRows * 128;    // 8 KB
+constexpr int kChunks = kDim / 64;                 // 64-channel (128-byte) column chunks
+constexpr int kChunkBytes = kTileRows * 128;       // 8 KB
 constexpr int kTileBytes = kChunks * kChunkBytes;  // 64 KB
-constexpr int kQBytes = kChunks * 64 * 128;     // 64 heads x 512 channels bf16
-constexpr int kPBytes = 64 * 128;               // 64 heads x 64 rows bf16
-constexpr int kThreads = 192;
+constexpr int kQBytes = kChunks * 64 * 128;        // 64 heads x 512 channels, 16-bit
+constexpr int kPBytes = 64 * 128;                  // 64 heads x 64 rows, 16-bit
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;    // O^T: 4 channel tiles x 64 heads
 constexpr uint32_t kColS = 256;  // scores: 2 buffers x 64 rows (M = 64 layout)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
+// Per-format configuration.  bf16 caches go straight from HBM to the MMA
+// operand tile by TMA gather and run kind::f16 with bf16 inputs.  Quantised
+// caches are dequantised in the load path by four converter warps (16-byte
+// loads straight from HBM, hardware cvt to f16, swizzled stores); every
+// E4M3 value and every E2M1 x E4M3 product is exact in f16, so those run
+// kind::f16 with f16 inputs (Q is converted to f16 once per CTA).
+template <int FMT>
+struct Cfg {
+  static constexpr bool kQuant = FMT != DSV4KV_BF16;
+  static constexpr bool kRowScale = FMT == DSV4KV_FP8_E4M3_ROW;
+  static constexpr int kThreads = kQuant ? 320 : 192;
+  static constexpr uint32_t kIdescQK = kQuant ? idesc_f16(64, 64, 0, 0) : idesc_bf16(64, 64, 0, 0);
+  static constexpr uint32_t kIdescPV = kQuant ? idesc_f16(128, 64, 1, 0) : idesc_bf16(128, 64, 1, 0);
+};
+
 struct __align__(8) Ctl {
   uint64_t q_full;
+  uint64_t q_ready;
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t s_full[2];
@@ -58,6 +73,7 @@ struct __align__(8) Ctl {
   uint32_t tmem_base;
   volatile int abort;
   float alpha[64];
+  float row_scale[kStages][kTileRows];
 };
 
 constexpr size_t kSmemBytes = 1024 + kQBytes + kStages * kTileBytes + 2 * kPBytes + sizeof(Ctl);
@@ -70,9 +86,13 @@ struct Params {
   int comp_tiles, tiles, splits, tiles_per_split;
   int64_t comp_rows, win_rows;  // per-sequence row capacity of each cache
   const int32_t* idx;           // [B][k] or null (dense)
+  const uint8_t* comp_codes;    // quantised caches (converter warps)
+  const void* comp_scales;
+  const uint8_t* win_codes;
+  const void* win_scales;
   float score_scale;            // sm_scale * log2(e)
   float* o_part;                // [B][splits][H][512]
-  float* ml_part;               // [B][splits][H][2]
+  float* ml_part;               // [B][splits][H][4]: (m_o, m_l, l, 0)
   uint32_t* status;
 };
 
@@ -99,6 +119,13 @@ __device__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ctl* ctl) {
   }
 }
 
+// Warp-uniform bounded wait: lane 0 polls, the result is broadcast.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Ctl* ctl, int lane) {
+  bool ok = true;
+  if (lane == 0) ok = wait_or_abort(bar, parity, ctl);
+  return __shfl_sync(kFull, ok, 0);
+}
+
 __device__ __forceinline__ bool named_bar_or(bool pred) {
   uint32_t r;
   asm volatile(
@@ -109,6 +136,36 @@ __device__ __forceinline__ bool named_bar_or(bool pred) {
   return r != 0;
 }
 __device__ __forceinline__ void named_bar_sync() { asm volatile("barrier.cta.sync 1, 128;" ::: "memory"); }
+
+// Source of row `r` of tile T: global row (b * rows + i) of the compressed
+// cache (from_win = false) or of the window cache; valid = false for padding
+// slots and for rejected indices (the row then reads nothing).
+struct RowSrc {
+  int64_t row;
+  bool valid, from_win;
+};
+__device__ __forceinline__ RowSrc row_source(const Params& p, int b, int T, int r) {
+  RowSrc s{0, false, false};
+  if (T < p.comp_tiles) {
+    const int slot = T * kTileRows + r;
+    int64_t i = -1;
+    if (p.idx) {
+      const int32_t v = slot < p.k ? p.idx[size_t(b) * p.k + slot] : -1;
+      if (v >= p.n) set_status(p.status, DSV4KV_DEV_BAD_INDEX);
+      i = v;
+    } else if (slot < p.n) {
+      i = slot;
+    }
+    s.valid = i >= 0 && i < p.n;
+    s.row = int64_t(b) * p.comp_rows + (s.valid ? i : 0);
+  } else {
+    const int wr = (T - p.comp_tiles) * kTileRows + r;
+    s.from_win = true;
+    s.valid = wr < p.window;
+    s.row = int64_t(b) * p.win_rows + (s.valid ? wr : 0);
+  }
+  return s;
+}
 
 // Row validity of tile T (rows lane and lane+32 of the tile), warp-wide.
 __device__ __forceinline__ uint64_t tile_valid_mask(const Params& p, int b, int T, int lane) {
@@ -132,9 +189,27 @@ __device__ __forceinline__ uint64_t tile_valid_mask(const Params& p, int b, int 
   return uint64_t(__ballot_sync(kFull, v0)) | (uint64_t(__ballot_sync(kFull, v1)) << 32);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__device__ __forceinline__ uint32_t pack_p(float a, float b, bool f16) {
+  return f16 ? f32x2_to_f16x2_sat(a, b) : pack_bf16x2(a, b);
+}
+__device__ __forceinline__ float p_lo(uint32_t v, bool f16) {
+  if (!f16) return bf16lo(v);
+  float f;
+  asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.f32.f16 %0, l;\n\t}" : "=f"(f) : "r"(v));
+  return f;
+}
+__device__ __forceinline__ float p_hi(uint32_t v, bool f16) {
+  if (!f16) return bf16hi(v);
+  float f;
+  asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.f32.f16 %0, h;\n\t}" : "=f"(f) : "r"(v));
+  return f;
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(Cfg<FMT>::kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_comp,
                   const __grid_constant__ CUtensorMap tm_win, const Params p) {
+  using C = Cfg<FMT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
@@ -149,8 +224,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl->q_full, 1);
+    mbar_init(&ctl->q_ready, 4);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->full[s], C::kQuant ? 4 : 1);
       mbar_init(&ctl->empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -169,8 +245,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_q);
-    prefetch_tmap(&tm_comp);
-    prefetch_tmap(&tm_win);
+    if (!C::kQuant) {
+      prefetch_tmap(&tm_comp);
+      prefetch_tmap(&tm_win);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -178,54 +256,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = ctl->tmem_base;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ producer (TMA)
     if (lane == 0) {
       mbar_arrive_expect_tx(&ctl->q_full, kQBytes);
       for (int c = 0; c < kChunks; ++c) tma_load_3d(sQ + c * kChunkBytes, &tm_q, &ctl->q_full, c * 64, 0, b);
     }
     int issued = 0;
-    for (int i = 0; i < nt; ++i) {
-      const int T = t0 + i, stage = i % kStages;
-      if (i >= kStages) {
-        bool ok = true;
-        if (lane == 0) ok = wait_or_abort(&ctl->empty[stage], ((i / kStages) - 1) & 1, ctl);
-        if (!__shfl_sync(kFull, ok, 0)) break;
-      }
-      if (lane == 0) mbar_arrive_expect_tx(&ctl->full[stage], kTileBytes);
-      __syncwarp();
-      const int g = lane & 15;  // 4-row group of this lane
-      int32_t r[4];
-      const CUtensorMap* tm;
-      if (T < p.comp_tiles) {
-        tm = &tm_comp;
+    if (!C::kQuant) {
+      for (int i = 0; i < nt; ++i) {
+        const int T = t0 + i, stage = i % kStages;
+        if (i >= kStages && !warp_wait(&ctl->empty[stage], ((i / kStages) - 1) & 1, ctl, lane)) break;
+        if (lane == 0) mbar_arrive_expect_tx(&ctl->full[stage], kTileBytes);
+        __syncwarp();
+        const int g = lane & 15;  // 4-row group of this lane
+        int32_t r[4];
+        bool from_win = false;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int slot = T * kTileRows + 4 * g + e;
-          int64_t row = 0;
-          if (p.idx) {
-            const int32_t v = slot < p.k ? p.idx[size_t(b) * p.k + slot] : -1;
-            if (v >= 0 && v < p.n) row = v;
-            else if (v >= p.n && (lane >> 4) == 0) set_status(p.status, DSV4KV_DEV_BAD_INDEX);
-          } else if (slot < p.n) {
-            row = slot;
-          }
-          r[e] = int32_t(int64_t(b) * p.comp_rows + row);
+          const RowSrc s = row_source(p, b, T, 4 * g + e);
+          r[e] = int32_t(s.row);
+          from_win = s.from_win;
         }
-      } else {
-        tm = &tm_win;
+        const CUtensorMap* tm = from_win ? &tm_win : &tm_comp;
+        uint8_t* dst = sR + stage * kTileBytes + g * 512;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int wr = (T - p.comp_tiles) * kTileRows + 4 * g + e;
-          r[e] = int32_t(int64_t(b) * p.win_rows + (wr < p.window ? wr : 0));
+        for (int cc = 0; cc < 4; ++cc) {
+          const int c = (lane >> 4) * 4 + cc;
+          tma_gather4(dst + c * kChunkBytes, tm, &ctl->full[stage], c * 64, r[0], r[1], r[2], r[3]);
         }
+        issued = i + 1;
       }
-      uint8_t* dst = sR + stage * kTileBytes + g * 512;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int c = (lane >> 4) * 4 + cc;
-        tma_gather4(dst + c * kChunkBytes, tm, &ctl->full[stage], c * 64, r[0], r[1], r[2], r[3]);
-      }
-      issued = i + 1;
     }
     // drain: never leave the CTA with copies in flight
     if (lane == 0) {
@@ -236,9 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16(64, 64, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16(128, 64, 1, 0);
-      bool ok = wait_or_abort(&ctl->q_full, 0, ctl);
+      bool ok = wait_or_abort(C::kQuant ? &ctl->q_ready : &ctl->q_full, 0, ctl);
       const uint32_t q_addr = smem_u32(sQ);
       for (int i = 0; ok && i <= nt; ++i) {
         if (i < nt) {
@@ -253,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < kDim / 16; ++kk) {
             const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
             mma_bf16_ss(d, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(r_addr + off, 16, 1024),
-                        idesc_qk, kk > 0);
+                        C::kIdescQK, kk > 0);
           }
           mma_commit(&ctl->s_full[sb]);
         }
@@ -270,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kr = 0; kr < kTileRows / 16; ++kr) {
               const uint64_t a = smem_desc_sw128(r_addr + 2 * ct * kChunkBytes + kr * 2048, kChunkBytes, 1024);
               const uint64_t bd = smem_desc_sw128(p_addr + kr * 32, 16, 1024);
-              mma_bf16_ss(tmem + kColO + 64 * ct, a, bd, idesc_pv, (j > 0 || kr > 0) ? 1u : 0u);
+              mma_bf16_ss(tmem + kColO + 64 * ct, a, bd, C::kIdescPV, (j > 0 || kr > 0) ? 1u : 0u);
             }
           }
           mma_commit(&ctl->empty[stage]);
@@ -279,22 +337,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       mma_commit(&ctl->o_done);  // completes once every issued MMA has finished
     }
-  } else {
+  } else if (warp < 6) {
     // ------------------------------------------------------------ softmax + epilogue (warps 2..5)
     // After a timed-out wait a warp turns `dead` (warp-uniform): it skips
     // every wait, TMEM and shared-memory access but still takes part in the
     // group's named barriers, so the other softmax warps cannot hang on them.
+    //
+    // Two running maxima: m_l for the softmax denominator l and m_o for the
+    // weights that multiply the stored rows.  With fp8 rows the per-row scale
+    // s_r is folded into the weights (w_r = p_r * s_r, y_r = x_r + log2 s_r),
+    // so the accumulator's weights stay <= 2^8 whatever the scales are; for
+    // other formats y == x and the two maxima coincide.
     const int wq = warp & 3;  // TMEM lane quadrant of this warp
     const uint32_t lane_base = uint32_t(32 * wq) << 16;
     const bool head_thread = lane < 16;
     const int h = 16 * wq + (lane & 15);
-    float m_used = -INFINITY, l = 0.f;
+    float m_o = -INFINITY, m_l = -INFINITY, l = 0.f;
     bool dead = false;
     for (int i = 0; i < nt; ++i) {
-      const int T = t0 + i, sb = i & 1;
-      if (!dead) dead = __any_sync(kFull, !wait_or_abort(&ctl->s_full[sb], (i >> 1) & 1, ctl));
+      const int T = t0 + i, sb = i & 1, stage = i % kStages;
+      if (!dead) dead = !warp_wait(&ctl->s_full[sb], (i >> 1) & 1, ctl, lane);
+      if (C::kRowScale && !dead) dead = !warp_wait(&ctl->full[stage], (i / kStages) & 1, ctl, lane);
       float x[64];
-      float tmax = -INFINITY;
+      float tmax = -INFINITY, ymax = -INFINITY;
       if (!dead) {
         tc_fence_after();
         uint32_t s0[32], s1[32];
@@ -306,20 +371,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&ctl->s_free[sb]);
         const uint64_t vmask = tile_valid_mask(p, b, T, lane);
 #pragma unroll
-        for (int r = 0; r < 32; ++r) {
-          x[r] = ((vmask >> r) & 1) ? __uint_as_float(s0[r]) * p.score_scale : -INFINITY;
-          x[r + 32] = ((vmask >> (r + 32)) & 1) ? __uint_as_float(s1[r]) * p.score_scale : -INFINITY;
-          tmax = fmaxf(tmax, fmaxf(x[r], x[r + 32]));
+        for (int r = 0; r < 64; ++r) {
+          const float raw = __uint_as_float(r < 32 ? s0[r] : s1[r - 32]);
+          const bool v = (vmask >> r) & 1;
+          if (C::kRowScale) {
+            const float sc = ctl->row_scale[stage][r];
+            x[r] = v ? raw * sc * p.score_scale : -INFINITY;
+            ymax = fmaxf(ymax, (v && sc > 0.f) ? x[r] + __log2f(sc) : -INFINITY);
+          } else {
+            x[r] = v ? raw * p.score_scale : -INFINITY;
+          }
+          tmax = fmaxf(tmax, x[r]);
         }
-        if (i >= 1) dead = __any_sync(kFull, !wait_or_abort(&ctl->pv_done, (i - 1) & 1, ctl));
+        if (!C::kRowScale) ymax = tmax;
+        if (i >= 1) dead = !warp_wait(&ctl->pv_done, (i - 1) & 1, ctl, lane);
       }
-      const bool need = !dead && head_thread && tmax > m_used + kRescaleThreshold;
+      if (!dead && tmax > m_l + kRescaleThreshold) {
+        l *= (m_l == -INFINITY) ? 0.f : exp2f(m_l - tmax);
+        m_l = tmax;
+      }
+      const bool need = !dead && head_thread && ymax > m_o + kRescaleThreshold;
       float alpha = 1.f;
       if (need) {
-        alpha = (m_used == -INFINITY) ? 0.f : exp2f(m_used - tmax);
-        m_used = tmax;
+        alpha = (m_o == -INFINITY) ? 0.f : exp2f(m_o - ymax);
+        m_o = ymax;
       }
-      l *= alpha;
       if (i >= 1 && named_bar_or(need)) {
         if (!dead && head_thread) ctl->alpha[h] = alpha;
         named_bar_sync();
@@ -352,10 +428,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int r = 8 * c16 + 2 * e;
-            const float pa = (m_used == -INFINITY) ? 0.f : exp2f(x[r] - m_used);
-            const float pb = (m_used == -INFINITY) ? 0.f : exp2f(x[r + 1] - m_used);
-            const uint32_t packed = pack_bf16x2(pa, pb);
-            l += bf16lo(packed) + bf16hi(packed);
+            float ya = x[r], yb = x[r + 1];
+            if (C::kRowScale) {  // y = x + log2(s_r): the weight of the stored row carries its scale
+              const float sa = ctl->row_scale[stage][r], sb2 = ctl->row_scale[stage][r + 1];
+              ya = sa > 0.f ? ya + __log2f(sa) : -INFINITY;
+              yb = sb2 > 0.f ? yb + __log2f(sb2) : -INFINITY;
+            }
+            const float wa = (m_o == -INFINITY) ? 0.f : exp2f(ya - m_o);
+            const float wb = (m_o == -INFINITY) ? 0.f : exp2f(yb - m_o);
+            const uint32_t packed = pack_p(wa, wb, C::kQuant);
+            if (C::kRowScale) {
+              if (m_l != -INFINITY) l += exp2f(x[r] - m_l) + exp2f(x[r + 1] - m_l);
+            } else {
+              l += p_lo(packed, C::kQuant) + p_hi(packed, C::kQuant);  // the weights the MMA uses
+            }
             w[e] = packed;
           }
           *reinterpret_cast<uint4*>(prow + ((c16 ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -366,8 +452,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->p_full[sb]);
     }
-    if (!dead) dead = __any_sync(kFull, !wait_or_abort(&ctl->o_done, 0, ctl));
-    float* ml = p.ml_part + ((size_t(b) * p.splits + split) * p.heads + h) * 2;
+    if (!dead) dead = !warp_wait(&ctl->o_done, 0, ctl, lane);
+    float* ml = p.ml_part + ((size_t(b) * p.splits + split) * p.heads + h) * 4;
     if (!dead) {
       tc_fence_after();
       float* op = p.o_part + (size_t(b) * p.splits + split) * size_t(p.heads) * kDim;
@@ -386,13 +472,85 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (head_thread && h < p.heads) {
-        ml[0] = m_used;
-        ml[1] = l;
-      }
+      if (head_thread && h < p.heads) *reinterpret_cast<float4*>(ml) = make_float4(m_o, m_l, l, 0.f);
     } else if (head_thread && h < p.heads) {
-      ml[0] = -INFINITY;  // an empty partial keeps the combine step finite
-      ml[1] = 0.f;
+      // an empty partial keeps the combine step finite
+      *reinterpret_cast<float4*>(ml) = make_float4(-INFINITY, -INFINITY, 0.f, 0.f);
+    }
+  } else if (C::kQuant) {
+    // ------------------------------------------------------------ converters (warps 6..9)
+    const int cw = warp - 6;
+    const int tid = threadIdx.x - 192;
+    // (1) Q: bf16 -> f16 in place (saturating), once per CTA
+    if (warp_wait(&ctl->q_full, 0, ctl, lane)) {
+      for (int v = tid; v < kQBytes / 16; v += 128) {
+        uint4 x = *reinterpret_cast<const uint4*>(sQ + 16 * v);
+        x = make_uint4(f32x2_to_f16x2_sat(bf16lo(x.x), bf16hi(x.x)), f32x2_to_f16x2_sat(bf16lo(x.y), bf16hi(x.y)),
+                       f32x2_to_f16x2_sat(bf16lo(x.z), bf16hi(x.z)), f32x2_to_f16x2_sat(bf16lo(x.w), bf16hi(x.w)));
+        *reinterpret_cast<uint4*>(sQ + 16 * v) = x;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->q_ready);
+    }
+    // (2) rows: warp cw converts rows 16*cw .. 16*cw+15 of every tile; lane
+    // `lane` owns channels [16*lane, 16*lane+16) = half of a 64-channel chunk.
+    const int chunk = lane >> 2, u0 = (lane & 3) * 2;
+    for (int i = 0; i < nt; ++i) {
+      const int T = t0 + i, stage = i % kStages;
+      if (i >= kStages && !warp_wait(&ctl->empty[stage], ((i / kStages) - 1) & 1, ctl, lane)) break;
+      // lane j < 16 resolves row 16*cw + j, then every lane reads all 16 answers
+      const RowSrc mine = row_source(p, b, T, 16 * cw + (lane & 15));
+      const bool from_win = mine.from_win;  // uniform within a tile
+      const uint8_t* codes = from_win ? p.win_codes : p.comp_codes;
+      const void* scales = from_win ? p.win_scales : p.comp_scales;
+      if (C::kRowScale && lane < 16)
+        ctl->row_scale[stage][16 * cw + lane] = mine.valid ? static_cast<const float*>(scales)[mine.row] : 0.f;
+      uint4 raw[16];
+      uint32_t sgrp[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int64_t row = __shfl_sync(kFull, mine.row, j);
+        const bool valid = __shfl_sync(kFull, mine.valid, j);
+        if (C::kRowScale) {
+          raw[j] = valid ? ld_stream_v4(codes + size_t(row) * kDim + 16 * lane) : make_uint4(0, 0, 0, 0);
+          sgrp[j] = 0;
+        } else {
+          if (valid) {
+            const uint2 c8 = *reinterpret_cast<const uint2*>(codes + size_t(row) * (kDim / 2) + 8 * lane);
+            raw[j] = make_uint4(c8.x, c8.y, 0, 0);
+            sgrp[j] = static_cast<const uint8_t*>(scales)[size_t(row) * (kDim / 16) + lane];
+          } else {
+            raw[j] = make_uint4(0, 0, 0, 0);
+            sgrp[j] = 0;
+          }
+        }
+      }
+      uint8_t* tile = sR + stage * kTileBytes + chunk * kChunkBytes;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int r = 16 * cw + j;
+        uint32_t hv[8];
+        if (C::kRowScale) {
+          const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            hv[2 * e] = e4m3x2_to_f16x2(w[e] & 0xffffu);
+            hv[2 * e + 1] = e4m3x2_to_f16x2(w[e] >> 16);
+          }
+        } else {
+          const uint32_t s2 = e4m3x2_to_f16x2(sgrp[j] | (sgrp[j] << 8));  // (scale, scale) as f16x2
+          const uint32_t w[2] = {raw[j].x, raw[j].y};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) hv[e] = hmul2(e2m1x2_to_f16x2((w[e >> 2] >> (8 * (e & 3))) & 0xffu), s2);
+        }
+        uint8_t* line = tile + r * 128;
+        *reinterpret_cast<uint4*>(line + ((u0 ^ (r & 7)) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        *reinterpret_cast<uint4*>(line + (((u0 + 1) ^ (r & 7)) << 4)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->full[stage]);
     }
   }
   tc_fence_before();
@@ -404,7 +562,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0 && ctl->abort) set_status(p.status, DSV4KV_DEV_TIMEOUT);
 }
 
-// Merge split partials (log2-domain max m, sum l), normalise, inverse RoPE.
+// Merge split partials, normalise, inverse RoPE.  Per split: O_s (weights
+// relative to 2^m_o), l_s (relative to 2^m_l):
+//   out = [sum_s O_s 2^(m_o,s - Mo)] / [sum_s l_s 2^(m_l,s - Ml)] * 2^(Mo - Ml).
 __global__ void __launch_bounds__(128) decode_combine(const float* __restrict__ o_part,
                                                       const float* __restrict__ ml_part, int splits, int heads,
                                                       int64_t t, int rope_dim, double rope_base, int out_fp32,
@@ -412,22 +572,26 @@ __global__ void __launch_bounds__(128) decode_combine(const float* __restrict__ 
   const int bh = blockIdx.x;
   const int b = bh / heads, h = bh % heads;
   const int c = 4 * threadIdx.x;
-  float M = -INFINITY;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, ml_part[((size_t(b) * splits + s) * heads + h) * 2]);
+  float Mo = -INFINITY, Ml = -INFINITY;
+  for (int s = 0; s < splits; ++s) {
+    const float4 ml = *reinterpret_cast<const float4*>(ml_part + ((size_t(b) * splits + s) * heads + h) * 4);
+    Mo = fmaxf(Mo, ml.x);
+    Ml = fmaxf(Ml, ml.y);
+  }
   float L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s = 0; s < splits; ++s) {
-    const float* ml = ml_part + ((size_t(b) * splits + s) * heads + h) * 2;
-    const float w = (ml[0] == -INFINITY) ? 0.f : exp2f(ml[0] - M);
-    if (w == 0.f) continue;
-    L += w * ml[1];
+    const float4 ml = *reinterpret_cast<const float4*>(ml_part + ((size_t(b) * splits + s) * heads + h) * 4);
+    if (ml.y != -INFINITY) L += ml.z * exp2f(ml.y - Ml);
+    if (ml.x == -INFINITY) continue;
+    const float w = exp2f(ml.x - Mo);
     const float4 o = *reinterpret_cast<const float4*>(o_part + ((size_t(b) * splits + s) * heads + h) * kDim + c);
     acc.x += w * o.x;
     acc.y += w * o.y;
     acc.z += w * o.z;
     acc.w += w * o.w;
   }
-  const float inv = 1.f / L;
+  const float inv = (Mo == -INFINITY) ? 0.f : exp2f(Mo - Ml) / L;
   float v[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
   const int r0 = kDim - rope_dim;
   if (c >= r0) {
@@ -483,7 +647,7 @@ DecodeWs decode_ws_layout(char* base, int batch, int heads, const Plan& pl) {
   };
   w.status = reinterpret_cast<uint32_t*>(take(16));
   w.o_part = reinterpret_cast<float*>(take(sizeof(float) * size_t(batch) * pl.splits * heads * kDim));
-  w.ml_part = reinterpret_cast<float*>(take(sizeof(float) * size_t(batch) * pl.splits * heads * 2));
+  w.ml_part = reinterpret_cast<float*>(take(sizeof(float) * size_t(batch) * pl.splits * heads * 4));
   w.bytes = off;
   return w;
 }
@@ -499,16 +663,32 @@ size_t decode_ws_bytes(int batch, int heads, int dim, int64_t rows_per_seq) {
   return decode_ws_layout(nullptr, batch, heads, pl).bytes;
 }
 
+template <int FMT>
+dsv4kv_status launch_fmt(const CUtensorMap& tq, const CUtensorMap& tc, const CUtensorMap& tw, const Params& p,
+                         int grid, cudaStream_t stream) {
+  static bool attr_set = false;  // per instantiation
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(decode_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes)) !=
+        cudaSuccess)
+      return check_launch("decode: cudaFuncSetAttribute");
+    attr_set = true;
+  }
+  decode_kernel<FMT><<<grid, Cfg<FMT>::kThreads, kSmemBytes, stream>>>(tq, tc, tw, p);
+  return check_launch("decode_kernel");
+}
+
 dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream) {
   if (a.dim != kDim) return set_error(DSV4KV_ERR_UNSUPPORTED, "decode: dim must be 512 (got %d)", a.dim);
-  if (a.comp.fmt != DSV4KV_BF16 || a.win.fmt != DSV4KV_BF16)
-    return set_error(DSV4KV_ERR_UNSUPPORTED, "decode: only bf16 caches in this build");
+  const int fmt = a.comp.fmt;
+  if (a.win.fmt != fmt)
+    return set_error(DSV4KV_ERR_UNSUPPORTED, "decode: the window cache must have the compressed cache's format");
+  if (fmt != DSV4KV_BF16 && fmt != DSV4KV_FP8_E4M3_ROW && fmt != DSV4KV_FP4_E2M1_G16)
+    return set_error(DSV4KV_ERR_UNSUPPORTED, "decode: unknown cache format %d", fmt);
   const int slots = a.idx ? a.k : int(a.n);
   const int comp_tiles = (a.n > 0 && slots > 0) ? (slots + kTileRows - 1) / kTileRows : 0;
   const int win_tiles = (a.window + kTileRows - 1) / kTileRows;
   if (comp_tiles + win_tiles == 0) return set_error(DSV4KV_ERR_INVALID_ARG, "decode: no rows to attend");
   const Plan pl = make_plan(a.batch, comp_tiles, win_tiles);
-  // workspace sized for the worst split count of this tile count
   const DecodeWs w = decode_ws_layout(static_cast<char*>(ws), a.batch, a.heads, pl);
   if (ws_bytes < w.bytes) return set_error(DSV4KV_ERR_WORKSPACE, "decode: workspace too small");
 
@@ -517,16 +697,22 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
                       uint64_t(kDim) * 2, uint64_t(a.heads) * kDim * 2, 64, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B))
     return set_error(DSV4KV_ERR_INVALID_ARG, "decode: cannot encode the query tensor map");
   const dsv4kv_cache& cc = a.comp;
-  const void* comp_base = cc.codes ? cc.codes : a.win.codes;
-  const uint64_t comp_rows_total = std::max<uint64_t>(1, uint64_t(a.batch) * uint64_t(std::max<int64_t>(cc.rows, 1)));
-  if (!encode_tmap_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, comp_base, kDim, comp_rows_total, uint64_t(kDim) * 2, 64,
-                      1, CU_TENSOR_MAP_SWIZZLE_128B))
-    return set_error(DSV4KV_ERR_INVALID_ARG, "decode: cannot encode the compressed-cache tensor map");
-  const void* win_base = a.win.codes ? a.win.codes : comp_base;
-  const uint64_t win_rows_total = std::max<uint64_t>(1, uint64_t(a.batch) * uint64_t(std::max<int64_t>(a.win.rows, 1)));
-  if (!encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, win_base, kDim, win_rows_total, uint64_t(kDim) * 2, 64, 1,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
-    return set_error(DSV4KV_ERR_INVALID_ARG, "decode: cannot encode the window tensor map");
+  if (fmt == DSV4KV_BF16) {
+    // row gathers (box: 64 channels x 1 row, 128-byte swizzle)
+    const void* comp_base = cc.codes ? cc.codes : a.win.codes;
+    const uint64_t comp_rows_total = std::max<uint64_t>(1, uint64_t(a.batch) * uint64_t(std::max<int64_t>(cc.rows, 1)));
+    if (!encode_tmap_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, comp_base, kDim, comp_rows_total, uint64_t(kDim) * 2,
+                        64, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+      return set_error(DSV4KV_ERR_INVALID_ARG, "decode: cannot encode the compressed-cache tensor map");
+    const void* win_base = a.win.codes ? a.win.codes : comp_base;
+    const uint64_t win_rows_total = std::max<uint64_t>(1, uint64_t(a.batch) * uint64_t(std::max<int64_t>(a.win.rows, 1)));
+    if (!encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, win_base, kDim, win_rows_total, uint64_t(kDim) * 2, 64,
+                        1, CU_TENSOR_MAP_SWIZZLE_128B))
+      return set_error(DSV4KV_ERR_INVALID_ARG, "decode: cannot encode the window tensor map");
+  } else {
+    tc = tq;  // unused: quantised rows are loaded by the converter warps
+    tw = tq;
+  }
 
   Params p{};
   p.heads = a.heads;
@@ -540,20 +726,22 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
   p.comp_rows = cc.rows;
   p.win_rows = a.win.rows;
   p.idx = a.idx;
+  p.comp_codes = static_cast<const uint8_t*>(cc.codes);
+  p.comp_scales = cc.scales;
+  p.win_codes = static_cast<const uint8_t*>(a.win.codes);
+  p.win_scales = a.win.scales;
   p.score_scale = a.sm_scale * 1.4426950408889634f;
   p.o_part = w.o_part;
   p.ml_part = w.ml_part;
   p.status = w.status;
 
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes)) !=
-        cudaSuccess)
-      return check_launch("decode: cudaFuncSetAttribute");
-    attr_set = true;
+  const int grid = a.batch * pl.splits;
+  dsv4kv_status st;
+  switch (fmt) {
+    case DSV4KV_BF16: st = launch_fmt<DSV4KV_BF16>(tq, tc, tw, p, grid, stream); break;
+    case DSV4KV_FP8_E4M3_ROW: st = launch_fmt<DSV4KV_FP8_E4M3_ROW>(tq, tc, tw, p, grid, stream); break;
+    default: st = launch_fmt<DSV4KV_FP4_E2M1_G16>(tq, tc, tw, p, grid, stream); break;
   }
-  decode_kernel<<<a.batch * pl.splits, kThreads, kSmemBytes, stream>>>(tq, tc, tw, p);
-  dsv4kv_status st = check_launch("decode_kernel");
   if (st != DSV4KV_OK) return st;
   decode_combine<<<a.batch * a.heads, kDim / 4, 0, stream>>>(w.o_part, w.ml_part, pl.splits, a.heads, a.t,
                                                               a.rope_dim, a.rope_base, a.out_fp32, a.out);
