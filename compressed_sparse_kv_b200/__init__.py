@@ -48,6 +48,9 @@ _SIGS = {
     "dsv4kv_index_topk_workspace_bytes": (_c.c_size_t, [_c.c_int32, _c.c_int64, _c.c_int32]),
     "dsv4kv_index_topk": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.c_int32, _c.c_int64, _c.c_int32,
                                      _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "dsv4kv_index_topk_noalloc_max_scratch_bytes": (_c.c_size_t, []),
+    "dsv4kv_index_topk_noalloc": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.c_int32, _c.c_int64, _c.c_int32,
+                                             _c.c_void_p, _c.c_void_p, _c.c_void_p]),
     "dsv4kv_sparse_decode_workspace_bytes": (_c.c_size_t, [_c.c_int32, _c.c_int32, _c.c_int32, _c.c_int32,
                                                            _c.c_int32]),
     "dsv4kv_sparse_decode": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.POINTER(CacheDesc), _c.c_void_p,
@@ -171,6 +174,21 @@ def index_topk(qidx: torch.Tensor, keys: Cache, n: int, k: int, idx_out: Optiona
     d = keys.desc()
     _check(lib().dsv4kv_index_topk(_ptr(qidx), ctypes.byref(d), b, n, k, _ptr(idx_out), _ptr(count_out), _ptr(ws),
                                    ws.numel(), _stream(stream)), "dsv4kv_index_topk")
+    return idx_out, count_out
+
+
+def index_topk_noalloc(qidx: torch.Tensor, keys: Cache, n: int, k: int, idx_out: Optional[torch.Tensor] = None,
+                       count_out: Optional[torch.Tensor] = None, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """index_topk with the library's static device scratch instead of a workspace (for callers that
+    cannot allocate device memory; concurrent calls on the GPU race)."""
+    b = int(qidx.shape[0])
+    if idx_out is None:
+        idx_out = torch.empty((b, k), dtype=torch.int32, device=qidx.device)
+    if count_out is None:
+        count_out = torch.empty((b,), dtype=torch.int32, device=qidx.device)
+    d = keys.desc()
+    _check(lib().dsv4kv_index_topk_noalloc(_ptr(qidx), ctypes.byref(d), b, n, k, _ptr(idx_out), _ptr(count_out),
+                                           _stream(stream)), "dsv4kv_index_topk_noalloc")
     return idx_out, count_out
 
 

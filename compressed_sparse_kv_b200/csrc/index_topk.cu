@@ -537,6 +537,13 @@ static IndexWs index_ws_layout(char* base, int batch, int64_t n, int k) {
 
 size_t index_topk_ws_bytes(int batch, int64_t n, int k) { return index_ws_layout(nullptr, batch, n, k).bytes; }
 
+// Bytes at the start of the workspace that must be zero before a call (status
+// word, counters, histograms): everything before the scores.
+size_t index_topk_zero_prefix_bytes(int batch) {
+  const IndexWs w = index_ws_layout(nullptr, batch, 1, 1);
+  return size_t(reinterpret_cast<char*>(w.scores) - static_cast<char*>(nullptr));
+}
+
 dsv4kv_status index_topk_launch(const uint16_t* qidx, const dsv4kv_cache& keys, int batch, int64_t n, int k,
                                 int32_t* idx_out, int32_t* count_out, void* ws, size_t ws_bytes,
                                 cudaStream_t stream) {

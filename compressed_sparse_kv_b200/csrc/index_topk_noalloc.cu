@@ -1,0 +1,87 @@
+// dsv4kv_index_topk_noalloc: the indexer top-k with its scratch in a
+// file-scope device array instead of a caller workspace.
+//
+// Some callers cannot allocate device memory for a workspace: for example a
+// serving engine whose memory manager has already reserved nearly all of HBM
+// for its KV block pool, a plugin host that forbids device allocations, or a
+// latency-critical path that must not pay for cudaMalloc's implicit
+// synchronisation.  They still pass the inputs and outputs; the scratch comes
+// from `g_index_scratch` below, which every GPU that loads this library keeps
+// until the process exits.
+//
+// Set-up: the first call on a device, with that device current, looks up the
+// array's device address with cudaGetSymbolAddress (in host code the symbol
+// is only a stand-in, never a device pointer) and caches it; make that first
+// call before any stream capture.  Every call shares the array, so calls that
+// overlap on the GPU (other streams, other threads) race; the counters and
+// histograms that must start at zero are cleared on the stream at the start
+// of every call.
+#include <cstdio>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dsv4kv {
+
+// Maximum scratch: 8 MiB (fits, e.g., batch 32 x 32736 entries with k = 512).
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;
+
+static __device__ __align__(256) unsigned char g_index_scratch[kStaticScratchBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void* g_addr[kMaxDevices] = {nullptr};
+
+dsv4kv_status scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return set_error(DSV4KV_ERR_CUDA, "index_topk_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return set_error(DSV4KV_ERR_UNSUPPORTED, "index_topk_noalloc: device %d", dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_index_scratch);
+    if (e != cudaSuccess || !p)
+      return set_error(DSV4KV_ERR_CUDA, "index_topk_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    g_addr[dev] = p;
+  }
+  *out = g_addr[dev];
+  return DSV4KV_OK;
+}
+
+}  // namespace
+}  // namespace dsv4kv
+
+using namespace dsv4kv;
+
+extern "C" __attribute__((visibility("default"))) size_t dsv4kv_index_topk_noalloc_max_scratch_bytes(void) {
+  return kStaticScratchBytes;
+}
+
+extern "C" __attribute__((visibility("default"))) dsv4kv_status dsv4kv_index_topk_noalloc(
+    const void* qidx, const dsv4kv_cache* keys, int32_t batch, int64_t n, int32_t k, int32_t* idx_out,
+    int32_t* count_out, void* stream) {
+  if (batch < 0 || n < 0) return set_error(DSV4KV_ERR_INVALID_ARG, "index_topk_noalloc: bad sizes");
+  if (k < 1 || k > 2048) return set_error(DSV4KV_ERR_UNSUPPORTED, "index_topk_noalloc: k must be in [1, 2048]");
+  const size_t need = dsv4kv_index_topk_workspace_bytes(batch, n, k);
+  if (need > kStaticScratchBytes)
+    return set_error(DSV4KV_ERR_UNSUPPORTED,
+                     "index_topk_noalloc: this call needs %zu bytes of scratch, above the %zu-byte static maximum "
+                     "(use dsv4kv_index_topk with a workspace)",
+                     need, kStaticScratchBytes);
+  void* ws = nullptr;
+  if (batch > 0 && n > k) {
+    dsv4kv_status st = scratch_address(&ws);
+    if (st != DSV4KV_OK) return st;
+    // The workspace layout starts with the status word, the per-sequence
+    // ticket and candidate counters and the two histograms; clear that prefix.
+    const size_t zero_bytes = index_topk_zero_prefix_bytes(batch);
+    const cudaError_t e = cudaMemsetAsync(ws, 0, zero_bytes, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+      return set_error(DSV4KV_ERR_CUDA, "index_topk_noalloc: clearing scratch: %s", cudaGetErrorString(e));
+  }
+  return dsv4kv_index_topk(qidx, keys, batch, n, k, idx_out, count_out, ws, kStaticScratchBytes, stream);
+}

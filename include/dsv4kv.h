@@ -138,6 +138,31 @@ dsv4kv_status dsv4kv_index_topk(const void* qidx, const dsv4kv_cache* keys, int3
                                 void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * dsv4kv_index_topk without a caller workspace.  The pages have no
+ * counterpart: this exists for callers that cannot allocate device memory for
+ * a workspace — a serving engine whose memory manager has already reserved
+ * nearly all of HBM for its KV block pool, a plugin host that forbids device
+ * allocations, or a latency-critical path that must not pay for cudaMalloc's
+ * implicit synchronisation.  Same inputs, outputs and results as
+ * dsv4kv_index_topk.
+ *
+ * The scratch is a library-owned static device array of
+ * dsv4kv_index_topk_noalloc_max_scratch_bytes() bytes (8 MiB) that every GPU
+ * which loads the library holds until the process exits.  A call whose
+ * scratch need (dsv4kv_index_topk_workspace_bytes) exceeds it returns
+ * DSV4KV_ERR_UNSUPPORTED; batch 32 x 32736 entries with k = 512 fits.  The
+ * first call on a device (with that device current) looks up the array's
+ * device address; make it before any stream capture.  Each call clears the
+ * scratch counters on `stream` first.  All calls share the one array, so
+ * calls that overlap on the GPU race.  Nothing here allocates memory.
+ * ------------------------------------------------------------------------ */
+size_t dsv4kv_index_topk_noalloc_max_scratch_bytes(void);
+
+dsv4kv_status dsv4kv_index_topk_noalloc(const void* qidx, const dsv4kv_cache* keys, int32_t batch,
+                                        int64_t n, int32_t k, int32_t* idx_out, int32_t* count_out,
+                                        void* stream);
+
+/* ---------------------------------------------------------------------------
  * Decode attention with shared K/V.  [P2] Step 3: one cached vector S_j is
  * both key (score = Q.S_j) and value; [P1] "The sliding window": a 128-token
  * exact window; [P1] "Shared key and value": inverse RoPE on the output.
