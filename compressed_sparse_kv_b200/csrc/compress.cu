@@ -69,9 +69,11 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock)
       const int c = c0 + e;
       if (c >= r0) {
         const int m = (c - r0) >> 1;
-        const double theta = pow(rope_base, -2.0 * double(m) / double(rope_dim));
+        // angle pos*theta in units of pi, reduced exactly modulo 2 before sincospi
+        const double ang = pos * (pow(rope_base, -2.0 * double(m) / double(rope_dim)) / 3.141592653589793);
+        const double xr = ang - 2.0 * rint(0.5 * ang);
         double sn, cs;
-        sincos(pos * theta, &sn, &cs);
+        sincospi(xr, &sn, &cs);
         const float x = acc[e], y = acc[e + 1];
         acc[e] = float(double(x) * cs - double(y) * sn);
         acc[e + 1] = float(double(x) * sn + double(y) * cs);

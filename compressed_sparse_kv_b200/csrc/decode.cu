@@ -189,6 +189,14 @@ __device__ __forceinline__ uint64_t tile_valid_mask(const Params& p, int b, int 
   return uint64_t(__ballot_sync(kFull, v0)) | (uint64_t(__ballot_sync(kFull, v1)) << 32);
 }
 
+// 2^x with the hardware approximation (max relative error ~2^-22, far below
+// the 16-bit rounding of P); ex2(-inf) = +0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_p(float a, float b, bool f16) {
   return f16 ? f32x2_to_f16x2_sat(a, b) : pack_bf16x2(a, b);
 }
@@ -434,11 +442,11 @@ __global__ void __launch_bounds__(Cfg<FMT>::kThreads, 1)
               ya = sa > 0.f ? ya + __log2f(sa) : -INFINITY;
               yb = sb2 > 0.f ? yb + __log2f(sb2) : -INFINITY;
             }
-            const float wa = (m_o == -INFINITY) ? 0.f : exp2f(ya - m_o);
-            const float wb = (m_o == -INFINITY) ? 0.f : exp2f(yb - m_o);
+            const float wa = (m_o == -INFINITY) ? 0.f : fast_exp2(ya - m_o);
+            const float wb = (m_o == -INFINITY) ? 0.f : fast_exp2(yb - m_o);
             const uint32_t packed = pack_p(wa, wb, C::kQuant);
             if (C::kRowScale) {
-              if (m_l != -INFINITY) l += exp2f(x[r] - m_l) + exp2f(x[r + 1] - m_l);
+              if (m_l != -INFINITY) l += fast_exp2(x[r] - m_l) + fast_exp2(x[r + 1] - m_l);
             } else {
               l += p_lo(packed, C::kQuant) + p_hi(packed, C::kQuant);  // the weights the MMA uses
             }
@@ -598,9 +606,11 @@ __global__ void __launch_bounds__(128) decode_combine(const float* __restrict__ 
 #pragma unroll
     for (int e = 0; e < 4; e += 2) {
       const int m = (c + e - r0) >> 1;
-      const double theta = pow(rope_base, -2.0 * double(m) / double(rope_dim));
+      // angle -t*theta in units of pi, reduced exactly modulo 2 before sincospi
+      const double ang = double(t) * (pow(rope_base, -2.0 * double(m) / double(rope_dim)) / 3.141592653589793);
+      const double xr = ang - 2.0 * rint(0.5 * ang);
       double sn, cs;
-      sincos(-double(t) * theta, &sn, &cs);
+      sincospi(-xr, &sn, &cs);
       const float x = v[e], y = v[e + 1];
       v[e] = float(x * cs - y * sn);
       v[e + 1] = float(x * sn + y * cs);
@@ -624,7 +634,8 @@ Plan make_plan(int batch, int comp_tiles, int win_tiles) {
   pl.comp_tiles = comp_tiles;
   pl.tiles = comp_tiles + win_tiles;
   const int sms = sm_count();
-  int splits = std::max(1, std::min(pl.tiles, (sms + batch - 1) / batch));
+  // one CTA per SM at most (shared memory), so at most one wave
+  int splits = std::max(1, std::min(pl.tiles, sms / std::max(batch, 1)));
   pl.tiles_per_split = (pl.tiles + splits - 1) / splits;
   pl.splits = (pl.tiles + pl.tiles_per_split - 1) / pl.tiles_per_split;
   return pl;
@@ -659,7 +670,7 @@ size_t decode_ws_bytes(int batch, int heads, int dim, int64_t rows_per_seq) {
   // rows_per_seq = compressed slots + window rows; the split plan only depends on the tile count
   const int tiles = int((rows_per_seq + kTileRows - 1) / kTileRows) + 1;
   Plan pl{};
-  pl.splits = std::max(1, std::min(tiles, (sm_count() + batch - 1) / batch));  // upper bound of make_plan
+  pl.splits = std::max(1, std::min(tiles, sm_count() / std::max(batch, 1)));  // upper bound of make_plan
   return decode_ws_layout(nullptr, batch, heads, pl).bytes;
 }
 

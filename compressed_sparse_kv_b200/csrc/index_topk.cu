@@ -32,77 +32,129 @@ namespace dsv4kv {
 constexpr int kHistBins = 4096;  // 12-bit digits
 
 // ------------------------------------------------------------------ scoring
-// bf16 keys, dim 128: a key is 256 B = 16 lanes x 16 B.  A warp iteration
-// covers 16 keys: half-warp h reads keys base+8h+u, u = 0..7 (8 independent
-// 16-byte loads per lane in flight), then a transposing butterfly reduces the
-// 8 partial sums over the 16 lanes with 8 shuffles (instead of 32).
+// Transposing butterfly: lane l16 of a 16-lane group holds U partial sums
+// (one per key); after log2 steps each lane holds the full 16-lane sum of one
+// key.  U = 16: key l16 (15 shuffles for 16 keys).  U = 8: key (l16 >> 1) & 7,
+// duplicated on lanes 2i and 2i+1 (8 shuffles for 8 keys).
+template <int U>
+__device__ __forceinline__ float reduce16_transposed(const float (&p)[U], int l16) {
+  float a[8], c[4], d[2];
+  if constexpr (U == 16) {
+    const bool b3 = l16 & 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      a[i] = (b3 ? p[8 + i] : p[i]) + __shfl_xor_sync(kFull, b3 ? p[i] : p[8 + i], 8);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = p[i];
+  }
+  const int sh = U == 16 ? 0 : 1;  // lane bit that selects in the next step
+  const bool x2 = (l16 >> (2 + sh)) & 1, x1 = (l16 >> (1 + sh)) & 1, x0 = (l16 >> sh) & 1;
+  const int o2 = 4 << sh, o1 = 2 << sh, o0 = 1 << sh;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) c[i] = (x2 ? a[4 + i] : a[i]) + __shfl_xor_sync(kFull, x2 ? a[i] : a[4 + i], o2);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) d[i] = (x1 ? c[2 + i] : c[i]) + __shfl_xor_sync(kFull, x1 ? c[i] : c[2 + i], o1);
+  float s = (x0 ? d[1] : d[0]) + __shfl_xor_sync(kFull, x0 ? d[0] : d[1], o0);
+  if constexpr (U == 8) s += __shfl_xor_sync(kFull, s, 1);
+  return s;
+}
+
+__device__ __forceinline__ float dot8_bf16(const uint4& v, const float (&q)[8]) {
+  float a = q[0] * bf16lo(v.x);
+  a = fmaf(q[1], bf16hi(v.x), a);
+  a = fmaf(q[2], bf16lo(v.y), a);
+  a = fmaf(q[3], bf16hi(v.y), a);
+  a = fmaf(q[4], bf16lo(v.z), a);
+  a = fmaf(q[5], bf16hi(v.z), a);
+  a = fmaf(q[6], bf16lo(v.w), a);
+  return fmaf(q[7], bf16hi(v.w), a);
+}
+
+// bf16 keys, dim 128: a key is 256 B = 16 lanes x 16 B.  The flattened
+// (sequence, entry) range of all B*n keys is split evenly over the grid; a
+// CTA walks its range one sequence segment at a time.  A warp iteration
+// covers 2U keys: half-warp h reads keys 2U*j + U*h + u (u < U), U
+// independent 16-byte loads per lane; with DB the next iteration's loads are
+// issued before the current iteration is reduced, so loads stay in flight.
+template <int U, bool DB>
 __global__ void __launch_bounds__(256) index_score_bf16(const uint16_t* __restrict__ qidx,
                                                         const uint16_t* __restrict__ keys, int64_t key_rows,
-                                                        int64_t n, int64_t chunk, float* __restrict__ scores,
-                                                        uint32_t* __restrict__ hist) {
+                                                        int64_t n, int batch, int64_t per_cta,
+                                                        float* __restrict__ scores, uint32_t* __restrict__ hist) {
   __shared__ uint32_t sh[kHistBins];
-  const int b = blockIdx.y;
-  const int64_t n0 = int64_t(blockIdx.x) * chunk;
-  const int64_t n1 = min(n, n0 + chunk);
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0;
+  const int64_t total = int64_t(batch) * n;
+  const int64_t g0 = int64_t(blockIdx.x) * per_cta;
+  const int64_t g1 = min(total, g0 + per_cta);
+  if (g0 >= g1) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int half = lane >> 4, l16 = lane & 15;
-  float q[8];
-  {
-    const uint4 v = *reinterpret_cast<const uint4*>(qidx + size_t(b) * 128 + 8 * l16);
-    q[0] = bf16lo(v.x); q[1] = bf16hi(v.x); q[2] = bf16lo(v.y); q[3] = bf16hi(v.y);
-    q[4] = bf16lo(v.z); q[5] = bf16hi(v.z); q[6] = bf16lo(v.w); q[7] = bf16hi(v.w);
+  const int my_key = U == 16 ? l16 : ((l16 >> 1) & 7);
+  const bool writer = U == 16 || !(lane & 1);
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0;
+  for (int64_t s0 = g0; s0 < g1;) {
+    const int b = int(s0 / n);
+    const int64_t s1 = min(g1, int64_t(b + 1) * n);
+    const int64_t i0 = s0 - int64_t(b) * n, cnt = s1 - s0;
+    float q[8];
+    {
+      const uint4 v = *reinterpret_cast<const uint4*>(qidx + size_t(b) * 128 + 8 * l16);
+      q[0] = bf16lo(v.x); q[1] = bf16hi(v.x); q[2] = bf16lo(v.y); q[3] = bf16hi(v.y);
+      q[4] = bf16lo(v.z); q[5] = bf16hi(v.z); q[6] = bf16lo(v.w); q[7] = bf16hi(v.w);
+    }
+    __syncthreads();  // histogram cleared
+    const uint16_t* kb = keys + (size_t(b) * size_t(key_rows) + size_t(i0)) * 128 + 8 * l16;
+    float* sc = scores + size_t(b) * size_t(n) + size_t(i0);
+    auto load = [&](int64_t j, uint4 (&v)[U]) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t key = 2 * U * j + U * half + u;
+        v[u] = key < cnt ? ld_stream_v4(kb + key * 128) : make_uint4(0, 0, 0, 0);
+      }
+    };
+    auto process = [&](int64_t j, const uint4 (&v)[U]) {
+      float p[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) p[u] = dot8_bf16(v[u], q);
+      const float s = reduce16_transposed<U>(p, l16) + 0.0f;  // -0 -> +0
+      const int64_t key = 2 * U * j + U * half + my_key;
+      if (writer && key < cnt) {
+        sc[key] = s;
+        atomicAdd(&sh[ord_f32(s) >> 20], 1u);
+      }
+    };
+    const int64_t ngroups = (cnt + 2 * U - 1) / (2 * U);
+    if constexpr (DB) {
+      uint4 va[U], vb[U];
+      int64_t j = warp;
+      if (j < ngroups) load(j, va);
+      while (j < ngroups) {
+        if (j + nwarps < ngroups) load(j + nwarps, vb);
+        process(j, va);
+        j += nwarps;
+        if (j >= ngroups) break;
+        if (j + nwarps < ngroups) load(j + nwarps, va);
+        process(j, vb);
+        j += nwarps;
+      }
+    } else {
+      for (int64_t j = warp; j < ngroups; j += nwarps) {
+        uint4 v[U];
+        load(j, v);
+        process(j, v);
+      }
+    }
+    __syncthreads();
+    uint32_t* hb = hist + size_t(b) * kHistBins;
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
+      const uint32_t c = sh[i];
+      if (c) {
+        atomicAdd(&hb[i], c);
+        sh[i] = 0;
+      }
+    }
+    s0 = s1;
   }
-  __syncthreads();
-  const uint16_t* kb = keys + size_t(b) * size_t(key_rows) * 128 + 8 * l16;
-  float* sc = scores + size_t(b) * size_t(n);
-  const bool b3 = l16 & 8, b2 = l16 & 4, b1 = l16 & 2;
-  for (int64_t base = n0 + 16 * warp; base < n1; base += 16 * nwarps) {
-    uint4 v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int64_t key = base + 8 * half + u;
-      v[u] = key < n1 ? ld_stream_v4(kb + key * 128) : make_uint4(0, 0, 0, 0);
-    }
-    float p[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      float a = q[0] * bf16lo(v[u].x);
-      a = fmaf(q[1], bf16hi(v[u].x), a);
-      a = fmaf(q[2], bf16lo(v[u].y), a);
-      a = fmaf(q[3], bf16hi(v[u].y), a);
-      a = fmaf(q[4], bf16lo(v[u].z), a);
-      a = fmaf(q[5], bf16hi(v[u].z), a);
-      a = fmaf(q[6], bf16lo(v[u].w), a);
-      a = fmaf(q[7], bf16hi(v[u].w), a);
-      p[u] = a;
-    }
-    float k4[4], k2[2];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float keep = b3 ? p[4 + i] : p[i];
-      const float send = b3 ? p[i] : p[4 + i];
-      k4[i] = keep + __shfl_xor_sync(kFull, send, 8);
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const float keep = b2 ? k4[2 + i] : k4[i];
-      const float send = b2 ? k4[i] : k4[2 + i];
-      k2[i] = keep + __shfl_xor_sync(kFull, send, 4);
-    }
-    float s = (b1 ? k2[1] : k2[0]) + __shfl_xor_sync(kFull, b1 ? k2[0] : k2[1], 2);
-    s += __shfl_xor_sync(kFull, s, 1);
-    const int64_t key = base + 8 * half + ((l16 >> 1) & 7);
-    if (!(lane & 1) && key < n1) {
-      s += 0.0f;  // -0 -> +0
-      sc[key] = s;
-      atomicAdd(&sh[ord_f32(s) >> 20], 1u);
-    }
-  }
-  __syncthreads();
-  uint32_t* hb = hist + size_t(b) * kHistBins;
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
-    if (sh[i]) atomicAdd(&hb[i], sh[i]);
 }
 
 // fp4 keys, dim 128: codes 64 B + 8 E4M3 scale bytes per key.  A quarter warp
@@ -236,41 +288,58 @@ __global__ void __launch_bounds__(256) index_score_fp4(const uint16_t* __restric
 }
 
 // ------------------------------------------------------------------ selection helpers
-// Block-wide: find the bin where the descending cumulative count of `h`
-// (kHistBins entries in smem) first reaches `need` (1 <= need <= total).
-// Returns the bin; *above = count of entries in higher bins.
-template <int NT>
-__device__ int find_threshold_bin(const uint32_t* h, uint32_t need, uint32_t* above, uint32_t* scratch) {
-  constexpr int PER = kHistBins / NT;
-  const int t = threadIdx.x;
-  // thread t owns bins [kHistBins-1 - PER*t - (PER-1), kHistBins-1 - PER*t] (descending)
-  uint32_t local = 0;
-  const int top = kHistBins - 1 - PER * t;
+constexpr int kSelThreads = 512;
+constexpr int kTieCap = 2048;
+constexpr int64_t kMaxBitmapN = 262144;  // entries covered by the shared-memory bitmaps (8192 words each)
+
+// Block-wide exclusive prefix sum of one value per thread (kSelThreads threads).
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* total) {
+  __shared__ uint32_t wsum[kSelThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = v;
 #pragma unroll
-  for (int i = 0; i < PER; ++i) local += h[top - i];
-  // inclusive scan over threads (ascending thread id = descending bins)
-  scratch[t] = local;
-  __syncthreads();
-  for (int off = 1; off < NT; off <<= 1) {
-    const uint32_t add = t >= off ? scratch[t - off] : 0u;
-    __syncthreads();
-    scratch[t] += add;
-    __syncthreads();
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t x = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += x;
   }
-  const uint32_t incl = scratch[t];
-  const uint32_t excl = incl - local;
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  uint32_t base = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < kSelThreads / 32; ++w) {
+    const uint32_t x = wsum[w];
+    base += w < warp ? x : 0u;
+    all += x;
+  }
+  __syncthreads();
+  if (total) *total = all;
+  return base + incl - v;
+}
+
+// The bin where the descending cumulative count of the 4096-bin histogram h
+// (shared memory) first reaches `need` (1 <= need <= sum h); *above = count in
+// higher bins.  Thread t owns bins 4095-8t .. 4088-8t.
+__device__ int find_threshold_bin(const uint32_t* h, uint32_t need, uint32_t* above) {
+  static_assert(kSelThreads * 8 == kHistBins, "8 bins per thread");
   __shared__ int s_bin;
   __shared__ uint32_t s_above;
-  if (excl < need && incl >= need) {
+  const int top = kHistBins - 1 - 8 * int(threadIdx.x);
+  uint32_t v[8], local = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[i] = h[top - i];
+    local += v[i];
+  }
+  const uint32_t excl = block_exclusive_scan(local, nullptr);
+  if (excl < need && excl + local >= need) {
     uint32_t c = excl;
-    for (int i = 0; i < PER; ++i) {
-      const uint32_t v = h[top - i];
-      if (c + v >= need) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (c < need && c + v[i] >= need) {
         s_bin = top - i;
         s_above = c;
-        break;
       }
-      c += v;
+      c += v[i];
     }
   }
   __syncthreads();
@@ -300,19 +369,38 @@ __device__ void bitonic_sort_smem(T* a, int n_pow2) {
   }
 }
 
-constexpr int kSelThreads = 512;
-constexpr int kTieCap = 2048;
+// Ordered walk of a bitmap of `words` words: calls emit(index, rank) for
+// every set bit in ascending index order (rank = 0, 1, ...).  Returns the count.
+template <typename F>
+__device__ uint32_t bitmap_ordered_walk(const uint32_t* bm, int words, F emit) {
+  const int per = (words + kSelThreads - 1) / kSelThreads;
+  const int w0 = min(words, int(threadIdx.x) * per), w1 = min(words, w0 + per);
+  uint32_t local = 0;
+  for (int w = w0; w < w1; ++w) local += __popc(bm[w]);
+  uint32_t total;
+  uint32_t rank = block_exclusive_scan(local, &total);
+  for (int w = w0; w < w1; ++w) {
+    uint32_t x = bm[w];
+    while (x) {
+      const int bit = __ffs(x) - 1;
+      x &= x - 1;
+      emit(uint32_t(w) * 32u + uint32_t(bit), rank++);
+    }
+  }
+  return total;
+}
 
 // ------------------------------------------------------------------ filter + select
+// Dynamic shared memory: two bitmaps of ceil(n/32) words when n <= kMaxBitmapN.
 __global__ void __launch_bounds__(kSelThreads) index_filter_select(
     const float* __restrict__ scores, int64_t n, int k, int64_t chunk, uint32_t* __restrict__ hist,
     uint32_t* __restrict__ hist2, uint32_t* __restrict__ done, uint32_t* __restrict__ cand_count,
     uint64_t* __restrict__ cand, int64_t cap, int32_t* __restrict__ idx_out, int32_t* __restrict__ count_out,
     uint32_t* __restrict__ status) {
+  extern __shared__ uint32_t dyn_bm[];
   __shared__ uint32_t sh[kHistBins];
-  __shared__ uint32_t scratch[kSelThreads];
   __shared__ int s_last;
-  __shared__ uint32_t s_nsel, s_ntie;
+  __shared__ uint32_t s_ntie, s_tie_min, s_tie_max, s_taken;
   __shared__ int32_t sel[2048];
   __shared__ uint64_t ties[kTieCap];
 
@@ -322,19 +410,20 @@ __global__ void __launch_bounds__(kSelThreads) index_filter_select(
   uint32_t* h2 = hist2 + size_t(b) * kHistBins;
   const float* sc = scores + size_t(b) * size_t(n);
   uint64_t* cb = cand + size_t(b) * size_t(cap);
+  const int lane = threadIdx.x & 31;
 
   // 1) threshold bin of the top-12-bit histogram
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = hb[i];
   __syncthreads();
   uint32_t above1;
-  const int bin1 = find_threshold_bin<kSelThreads>(sh, kk, &above1, scratch);
+  const int bin1 = find_threshold_bin(sh, kk, &above1);
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0;
   __syncthreads();
 
-  // 2) filter this CTA's chunk
+  // 2) filter this CTA's chunk: candidates (bin >= bin1) and the next-12-bit
+  //    histogram of the entries in bin1
   const int64_t n0 = int64_t(blockIdx.x) * chunk;
   const int64_t n1 = min(n, n0 + chunk);
-  const int lane = threadIdx.x & 31;
   for (int64_t base = n0; base < n1; base += blockDim.x) {
     const int64_t i = base + threadIdx.x;
     uint32_t o = 0;
@@ -370,45 +459,78 @@ __global__ void __launch_bounds__(kSelThreads) index_filter_select(
 
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = __ldcg(&h2[i]);
   if (threadIdx.x == 0) {
-    s_nsel = 0;
     s_ntie = 0;
+    s_tie_min = 0xffffffffu;
+    s_tie_max = 0;
+    s_taken = 0;
   }
   __syncthreads();
   uint32_t above2;
   const uint32_t need1 = kk - above1;  // still needed from bin1 (>= 1)
-  const int bin2 = find_threshold_bin<kSelThreads>(sh, need1, &above2, scratch);
+  const int bin2 = find_threshold_bin(sh, need1, &above2);
   const uint32_t prefix = (uint32_t(bin1) << 12) | uint32_t(bin2);  // 24-bit threshold prefix
   const uint32_t need_tie = need1 - above2;                           // >= 1
-  const uint32_t n_tie = sh[bin2];
   const uint32_t total = __ldcg(&cand_count[b]);
+  int32_t* ob = idx_out + size_t(b) * k;
 
-  const bool fast = total <= uint64_t(cap) && n_tie <= kTieCap;
-  if (fast) {
+  bool done_out = false;
+  if (total <= uint64_t(cap) && n <= kMaxBitmapN) {
+    // bitmap path: entries above the prefix into `selbm`, entries at the prefix into `tiebm`
+    const int words = int((n + 31) / 32);
+    uint32_t* selbm = dyn_bm;
+    uint32_t* tiebm = dyn_bm + words;
+    for (int w = threadIdx.x; w < 2 * words; w += blockDim.x) dyn_bm[w] = 0;
+    __syncthreads();
     for (uint32_t c = threadIdx.x; c < total; c += blockDim.x) {
       const uint64_t key = __ldcg(&cb[c]);
-      const uint32_t pre = uint32_t(key >> 40);
+      const uint32_t o = uint32_t(key >> 32), i = 0xffffffffu - uint32_t(key);
+      const uint32_t pre = o >> 8;
       if (pre > prefix) {
-        sel[atomicAdd(&s_nsel, 1u)] = int32_t(0xffffffffu - uint32_t(key));
+        atomicOr(&selbm[i >> 5], 1u << (i & 31));
       } else if (pre == prefix) {
-        ties[atomicAdd(&s_ntie, 1u)] = key;
+        atomicOr(&tiebm[i >> 5], 1u << (i & 31));
+        atomicMin(&s_tie_min, o);
+        atomicMax(&s_tie_max, o);
+        const uint32_t slot = atomicAdd(&s_ntie, 1u);
+        if (slot < kTieCap) ties[slot] = key;
       }
     }
     __syncthreads();
-    // order the ties by (score desc, index asc) == key desc; take need_tie
-    int np2 = 1;
-    while (np2 < int(n_tie)) np2 <<= 1;
-    for (int i = int(n_tie) + threadIdx.x; i < np2; i += blockDim.x) ties[i] = 0;
+    const uint32_t n_tie = s_ntie;
+    bool ties_ok = true;
+    if (s_tie_min == s_tie_max) {
+      // every entry at the prefix has the same score: the lowest indices win
+      bitmap_ordered_walk(tiebm, words, [&](uint32_t i, uint32_t rank) {
+        if (rank < need_tie) atomicOr(&selbm[i >> 5], 1u << (i & 31));
+      });
+    } else if (n_tie <= uint32_t(kTieCap)) {
+      // distinct scores share the prefix: order those entries by (score desc, index asc)
+      int np2 = 1;
+      while (np2 < int(n_tie)) np2 <<= 1;
+      for (int i = int(n_tie) + threadIdx.x; i < np2; i += blockDim.x) ties[i] = 0;
+      __syncthreads();
+      bitonic_sort_smem<uint64_t, false>(ties, np2);
+      for (uint32_t t = threadIdx.x; t < need_tie; t += blockDim.x) {
+        const uint32_t i = 0xffffffffu - uint32_t(ties[t]);
+        atomicOr(&selbm[i >> 5], 1u << (i & 31));
+      }
+    } else {
+      ties_ok = false;
+    }
     __syncthreads();
-    bitonic_sort_smem<uint64_t, false>(ties, np2);
-    const uint32_t base_sel = above1 + above2;
-    if (threadIdx.x == 0 && (s_nsel != base_sel || s_ntie != n_tie)) set_status(status, DSV4KV_DEV_INCONSISTENT);
-    for (uint32_t i = threadIdx.x; i < need_tie; i += blockDim.x)
-      sel[base_sel + i] = int32_t(0xffffffffu - uint32_t(ties[i]));
-    __syncthreads();
-  } else {
-    // General path (adversarial ties): exact threshold code o* from the low
-    // 8 bits of the entries at the prefix, then one ordered scan over all
-    // scores keeps codes > o* and the first r codes == o* (lowest indices).
+    if (ties_ok) {
+      const uint32_t got = bitmap_ordered_walk(selbm, words, [&](uint32_t i, uint32_t rank) {
+        if (rank < kk) ob[rank] = int32_t(i);
+      });
+      if (threadIdx.x == 0 && got != kk) set_status(status, DSV4KV_DEV_INCONSISTENT);
+      done_out = true;
+    }
+  }
+  if (!done_out) {
+    // General path (huge n, candidate overflow or massive heterogeneous ties):
+    // exact threshold code o* from the low 8 bits of the entries at the
+    // prefix, then one ordered scan over all scores keeps codes > o* and the
+    // first r codes == o* (lowest indices).
     for (int i = threadIdx.x; i < 256; i += blockDim.x) sh[i] = 0;
     __syncthreads();
     for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
@@ -432,57 +554,34 @@ __global__ void __launch_bounds__(kSelThreads) index_filter_select(
     const uint32_t ostar = (prefix << 8) | s_low;
     const uint32_t r_eq = need_tie - s_above3;  // entries equal to o* to keep
     __shared__ uint32_t s_gt_seen, s_eq_seen;
-    __shared__ uint32_t wgt[kSelThreads / 32], weq[kSelThreads / 32];
     if (threadIdx.x == 0) {
       s_gt_seen = 0;
       s_eq_seen = 0;
     }
     __syncthreads();
-    const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    const uint32_t lt = (1u << lane) - 1u;
     for (int64_t base = 0; base < n; base += blockDim.x) {
       const int64_t i = base + threadIdx.x;
       const uint32_t o = i < n ? ord_f32(sc[i]) : 0u;
       const bool gt = i < n && o > ostar;
       const bool eq = i < n && o == ostar;
-      const uint32_t mgt = __ballot_sync(kFull, gt), meq = __ballot_sync(kFull, eq);
-      if (lane == 0) {
-        wgt[warp] = __popc(mgt);
-        weq[warp] = __popc(meq);
-      }
-      __syncthreads();
-      uint32_t gt_before = s_gt_seen + __popc(mgt & lt), eq_before = s_eq_seen + __popc(meq & lt);
-      for (int w = 0; w < warp; ++w) {
-        gt_before += wgt[w];
-        eq_before += weq[w];
-      }
+      uint32_t ngt, neq;
+      const uint32_t gt_before = s_gt_seen + block_exclusive_scan(gt ? 1u : 0u, &ngt);
+      const uint32_t eq_before = s_eq_seen + block_exclusive_scan(eq ? 1u : 0u, &neq);
       // index order is preserved: kept entries before this one = gt_before + min(eq_before, r_eq)
       const uint32_t pos = gt_before + min(eq_before, r_eq);
-      if ((gt || (eq && eq_before < r_eq)) && pos < 2048u) sel[pos] = int32_t(i);
-      __syncthreads();
+      if ((gt || (eq && eq_before < r_eq)) && pos < kk) ob[pos] = int32_t(i);
       if (threadIdx.x == 0) {
-        for (int w = 0; w < nw; ++w) {
-          s_gt_seen += wgt[w];
-          s_eq_seen += weq[w];
-        }
+        s_gt_seen += ngt;
+        s_eq_seen += neq;
       }
       __syncthreads();
     }
     if (threadIdx.x == 0 && s_gt_seen + min(s_eq_seen, r_eq) != kk) set_status(status, DSV4KV_DEV_INCONSISTENT);
-    __syncthreads();
   }
-
-  // 4) sort the kk selected indices ascending and write them
-  int np2 = 1;
-  while (np2 < int(kk)) np2 <<= 1;
-  for (int i = int(kk) + threadIdx.x; i < np2; i += blockDim.x) sel[i] = 0x7fffffff;
-  __syncthreads();
-  if (fast) bitonic_sort_smem<int32_t, true>(sel, np2);
-  int32_t* ob = idx_out + size_t(b) * k;
-  for (int i = threadIdx.x; i < k; i += blockDim.x) ob[i] = i < int(kk) ? sel[i] : -1;
+  for (int i = int(kk) + threadIdx.x; i < k; i += blockDim.x) ob[i] = -1;
   if (threadIdx.x == 0 && count_out) count_out[b] = int32_t(kk);
 
-  // 5) leave the workspace zeroed for the next call
+  // 4) leave the workspace zeroed for the next call
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
     hb[i] = 0;
     h2[i] = 0;
@@ -555,20 +654,28 @@ dsv4kv_status index_topk_launch(const uint16_t* qidx, const dsv4kv_cache& keys, 
   const IndexWs w = index_ws_layout(static_cast<char*>(ws), batch, n, k);
   if (ws_bytes < w.bytes) return set_error(DSV4KV_ERR_WORKSPACE, "index_topk: workspace too small");
   const int sms = sm_count();
-  // scoring: about 4 resident CTAs of 256 threads per SM, one wave
-  const int64_t target = int64_t(sms) * 4;
-  int64_t splits = std::max<int64_t>(1, (target + batch - 1) / batch);
-  int64_t chunk = (n + splits - 1) / splits;
-  chunk = std::max<int64_t>(256, (chunk + 31) / 32 * 32);
-  splits = (n + chunk - 1) / chunk;
-  const dim3 g1((unsigned)splits, (unsigned)batch);
   if (keys.fmt == DSV4KV_BF16) {
-    index_score_bf16<<<g1, 256, 0, stream>>>(qidx, static_cast<const uint16_t*>(keys.codes), keys.rows, n,
-                                             chunk, w.scores, w.hist);
+    // one wave (resident CTAs per SM x SMs) over the flattened (sequence, entry) range
+    static int occ = 0;
+    if (occ == 0 &&
+        (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, index_score_bf16<8, true>, 256, 0) != cudaSuccess ||
+         occ < 1))
+      occ = 1;
+    const int64_t total = int64_t(batch) * n;
+    const int64_t grid = int64_t(sms) * occ;
+    const int64_t per_cta = std::max<int64_t>(64, (total + grid - 1) / grid);
+    index_score_bf16<8, true><<<unsigned((total + per_cta - 1) / per_cta), 256, 0, stream>>>(
+        qidx, static_cast<const uint16_t*>(keys.codes), keys.rows, n, batch, per_cta, w.scores, w.hist);
   } else {
+    const int64_t target = int64_t(sms) * 4;
+    int64_t splits = std::max<int64_t>(1, (target + batch - 1) / batch);
+    int64_t chunk = (n + splits - 1) / splits;
+    chunk = std::max<int64_t>(256, (chunk + 31) / 32 * 32);
+    splits = (n + chunk - 1) / chunk;
+    const dim3 g1((unsigned)splits, (unsigned)batch);
     index_score_fp4<<<g1, 256, 0, stream>>>(qidx, static_cast<const uint8_t*>(keys.codes),
-                                            static_cast<const uint8_t*>(keys.scales), keys.rows, n, chunk,
-                                            w.scores, w.hist);
+                                            static_cast<const uint8_t*>(keys.scales), keys.rows, n, chunk, w.scores,
+                                            w.hist);
   }
   dsv4kv_status st = check_launch("index_score");
   if (st != DSV4KV_OK) return st;
@@ -576,9 +683,17 @@ dsv4kv_status index_topk_launch(const uint16_t* qidx, const dsv4kv_cache& keys, 
   int64_t chunk2 = 4096;
   int64_t splits2 = (n + chunk2 - 1) / chunk2;
   const dim3 g2((unsigned)splits2, (unsigned)batch);
-  index_filter_select<<<g2, kSelThreads, 0, stream>>>(w.scores, n, k, chunk2, w.hist, w.hist2, w.done,
-                                                      w.cand_count, w.cand, w.cap, idx_out, count_out,
-                                                      w.status);
+  const size_t dyn = n <= kMaxBitmapN ? size_t(2) * size_t((n + 31) / 32) * sizeof(uint32_t) : 0;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(index_filter_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(2 * (kMaxBitmapN / 32) * sizeof(uint32_t))) != cudaSuccess)
+      return check_launch("index_filter_select: cudaFuncSetAttribute");
+    attr_set = true;
+  }
+  index_filter_select<<<g2, kSelThreads, dyn, stream>>>(w.scores, n, k, chunk2, w.hist, w.hist2, w.done,
+                                                        w.cand_count, w.cand, w.cap, idx_out, count_out,
+                                                        w.status);
   return check_launch("index_filter_select");
 }
 
