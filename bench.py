@@ -30,11 +30,16 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode-attn steps/s per layer type; HBM GB/s vs ~8 TB/s peak, 1 B200"
 WORKLOADS = {
-    # name: (kind, batch, t, heads)
-    "c4a_b32": ("c4a", 32, 131072, 64),
-    "c128a_b8": ("c128a", 8, 131072, 64),
-    "c128a_b32": ("c128a", 32, 131072, 64),
+    # name: (kind, batch, t, heads, main_fmt, index_fmt)
+    "c4a_b32": ("c4a", 32, 131072, 64, 0, 0),
+    "c128a_b8": ("c128a", 8, 131072, 64, 0, 0),
+    "c128a_b32": ("c128a", 32, 131072, 64, 0, 0),
+    "q_c4a_fp8": ("c4a", 64, 262144, 64, 1, 2),
+    "q_c4a_fp4": ("c4a", 64, 262144, 64, 2, 2),
+    "q_c128a_fp8": ("c128a", 64, 262144, 64, 1, 0),
+    "q_c128a_fp4": ("c128a", 64, 262144, 64, 2, 0),
 }
+FMT_NAME = {0: "bf16", 1: "fp8", 2: "fp4"}
 
 
 def measured_peaks():
@@ -100,59 +105,88 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ our arm
+ROW_BYTES = {0: 1024, 1: 516, 2: 288}     # one 512-channel cache row: bf16, fp8 + scale, fp4 + scales
+KEY_BYTES = {0: 256, 2: 72}               # one 128-channel indexer key: bf16, fp4 + scales
+
+
 class Layer:
     """One layer's resident caches (R replicas) and per-step buffers on the GPU."""
 
-    def __init__(self, kind, batch, t, heads, seed, replicas):
+    def __init__(self, kind, batch, t, heads, seed, replicas, main_fmt=0, index_fmt=0, layer_id=0, shared=None):
         import torch
         import compressed_sparse_kv_b200 as K
         import datagen.gpu as G
         from datagen import workloads as WL
         self.K, self.torch = K, torch
         self.kind, self.batch, self.t, self.heads = kind, batch, t, heads
+        self.main_fmt, self.index_fmt = main_fmt, index_fmt
         self.window, self.k = 128, 512
         stride = 4 if kind == "c4a" else 128
         self.n = (t - self.window) // stride
         dev = "cuda"
+
+        def rows(key, count):
+            x = G.normal_bf16_(torch.empty(batch, count, 512, dtype=torch.bfloat16, device=dev), key)
+            if main_fmt == 0:
+                return K.Cache(0, x)
+            codes, scales = K.quantize(x, main_fmt)
+            del x
+            return K.Cache(main_fmt, codes, scales)
+
         self.reps = []
         for r in range(replicas):
-            keys = WL.keys_for(seed, 1000 * r)
-            rep = {}
-            rep["comp"] = G.normal_bf16_(torch.empty(batch, self.n, 512, dtype=torch.bfloat16, device=dev), keys["comp"])
-            rep["win"] = G.normal_bf16_(torch.empty(batch, self.window, 512, dtype=torch.bfloat16, device=dev), keys["win"])
+            keys = WL.keys_for(seed, 1000 * r + layer_id)
+            rep = {"comp": rows(keys["comp"], self.n), "win": rows(keys["win"], self.window)}
             if kind == "c4a":
-                rep["kidx"] = G.int_bf16_(torch.empty(batch, self.n, 128, dtype=torch.bfloat16, device=dev), keys["kidx"])
+                if index_fmt == 0:
+                    kt = G.int_bf16_(torch.empty(batch, self.n, 128, dtype=torch.bfloat16, device=dev), keys["kidx"])
+                    rep["kidx"] = K.Cache(0, kt, None, 128)
+                else:
+                    codes = torch.empty(batch, self.n, 64, dtype=torch.uint8, device=dev)
+                    scales = torch.empty(batch, self.n, 8, dtype=torch.uint8, device=dev)
+                    G.fp4_index_keys_(codes, scales, keys["kidx_fp4"])
+                    rep["kidx"] = K.Cache(2, codes, scales, 128)
             self.reps.append(rep)
-        keys = WL.keys_for(seed, 0)
+        keys = WL.keys_for(seed, layer_id)
         self.q = G.normal_bf16_(torch.empty(batch, heads, 512, dtype=torch.bfloat16, device=dev), keys["q"])
         self.qidx = G.int_bf16_(torch.empty(batch, 128, dtype=torch.bfloat16, device=dev), keys["qidx"])
-        self.idx = torch.empty(batch, self.k, dtype=torch.int32, device=dev)
-        self.cnt = torch.empty(batch, dtype=torch.int32, device=dev)
+        sh = shared if shared is not None else {}
+        self.idx = sh.setdefault("idx", torch.empty(batch, self.k, dtype=torch.int32, device=dev))
+        self.cnt = sh.setdefault("cnt", torch.empty(batch, dtype=torch.int32, device=dev))
         self.out = torch.empty(batch, heads, 512, dtype=torch.bfloat16, device=dev)
         if kind == "c4a":
-            self.ws_idx = K.new_workspace(K.index_topk_workspace_bytes(batch, self.n, self.k))
-            self.ws_dec = K.new_workspace(K.sparse_decode_workspace_bytes(batch, heads, self.k, self.window))
+            need_i = K.index_topk_workspace_bytes(batch, self.n, self.k)
+            need_d = K.sparse_decode_workspace_bytes(batch, heads, self.k, self.window)
+            if "ws_idx" not in sh or sh["ws_idx"].numel() < need_i:
+                sh["ws_idx"] = K.new_workspace(need_i)
+            self.ws_idx = sh["ws_idx"]
         else:
-            self.ws_dec = K.new_workspace(K.dense_decode_workspace_bytes(batch, heads, self.n, self.window))
+            need_d = K.dense_decode_workspace_bytes(batch, heads, self.n, self.window)
+        if "ws_dec" not in sh or sh["ws_dec"].numel() < need_d:
+            sh["ws_dec"] = K.new_workspace(need_d)
+        self.ws_dec = sh["ws_dec"]
 
-    # algorithmic bytes of one step (indexer keys + rows read), and the q/out bytes
+    # algorithmic bytes of one step: indexer keys + rows read (queries/outputs excluded)
     def alg_bytes(self):
         rows = (self.k + self.window) if self.kind == "c4a" else (self.n + self.window)
-        b = self.batch * rows * 1024
+        b = self.batch * rows * ROW_BYTES[self.main_fmt]
         if self.kind == "c4a":
-            b += self.batch * self.n * 256
+            b += self.batch * self.n * KEY_BYTES[self.index_fmt]
         return b
 
     def index_bytes(self):
-        return self.batch * self.n * 256 + self.batch * 256
+        return self.batch * self.n * KEY_BYTES[self.index_fmt] + self.batch * 256
+
+    def flops(self):
+        rows = (self.k + self.window) if self.kind == "c4a" else (self.n + self.window)
+        return self.batch * rows * 4 * self.heads * 512
 
     def launches_per_step(self):
         return 4 if self.kind == "c4a" else 2
 
     def index(self, r):
-        rep = self.reps[r]
-        self.K.index_topk(self.qidx, self.K.Cache(0, rep["kidx"], None, 128), self.n, self.k, idx_out=self.idx,
-                          count_out=self.cnt, ws=self.ws_idx)
+        self.K.index_topk(self.qidx, self.reps[r]["kidx"], self.n, self.k, idx_out=self.idx, count_out=self.cnt,
+                          ws=self.ws_idx)
 
     def decode(self, r, q=None, out=None):
         rep = self.reps[r]
@@ -160,64 +194,167 @@ class Layer:
         q = self.q if q is None else q
         out = self.out if out is None else out
         if self.kind == "c4a":
-            K.sparse_decode(q, K.Cache(0, rep["comp"]), K.Cache(0, rep["win"]), self.idx, self.n, self.window, self.t,
-                            out=out, ws=self.ws_dec)
+            K.sparse_decode(q, rep["comp"], rep["win"], self.idx, self.n, self.window, self.t, out=out, ws=self.ws_dec)
         else:
-            K.dense_decode(q, K.Cache(0, rep["comp"]), K.Cache(0, rep["win"]), self.n, self.window, self.t, out=out,
-                           ws=self.ws_dec)
+            K.dense_decode(q, rep["comp"], rep["win"], self.n, self.window, self.t, out=out, ws=self.ws_dec)
+
+    def step(self, r):
+        if self.kind == "c4a":
+            self.index(r)
+        self.decode(r)
+
+
+def time_stack(steps, warmup, seed, dist_max):
+    """The 61-layer stack at t = 2^20, B = 1 (layer l: c128a if l is even,
+    c4a if odd), one decode step = every layer once, captured as one graph."""
+    import torch
+    from datagen import workloads as WL
+    shared = {}
+    layers = [Layer(WL.stack_layer_kind(l), 1, 1 << 20, 64, seed, 1, layer_id=l, shared=shared)
+              for l in range(WL.STACK_LAYERS)]
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for _ in range(max(warmup, 1)):
+            for L in layers:
+                L.step(0)
+    stream.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * len(layers) + 1)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        ev[0].record(stream)
+        for i, L in enumerate(layers):
+            if L.kind == "c4a":
+                L.index(0)
+            ev[2 * i + 1].record(stream)
+            L.decode(0)
+            ev[2 * i + 2].record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+    stream.synchronize()
+    # one replay for the per-call breakdown
+    with torch.cuda.stream(stream):
+        g.replay()
+    stream.synchronize()
+    idx_ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i, L in enumerate(layers) if L.kind == "c4a")
+    c4a_dec = sum(ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i, L in enumerate(layers) if L.kind == "c4a")
+    c128a_ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 2]) for i, L in enumerate(layers) if L.kind == "c128a")
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(steps):
+            g.replay()
+        stop.record(stream)
+    stop.synchronize()
+    ms = dist_max(start.elapsed_time(stop)) / steps
+    alg = sum(L.alg_bytes() for L in layers)
+    n4 = sum(1 for L in layers if L.kind == "c4a")
+    res = {"workload": "61-layer stack decode step B=1 t=1048576 H=64 (30 c4a + 31 c128a), bf16, one CUDA graph",
+           "steps_per_s": round(1e3 / ms, 2), "ms_per_step": round(ms, 4), "alg_bytes_per_step": alg,
+           "hbm_gbs": round(alg / (ms * 1e-3) / 1e9, 1),
+           "c4a_layer_us": round((idx_ms + c4a_dec) / n4 * 1e3, 2),
+           "c4a_index_us": round(idx_ms / n4 * 1e3, 2),
+           "c128a_layer_us": round(c128a_ms / (len(layers) - n4) * 1e3, 2),
+           "launches_per_step": sum(L.launches_per_step() for L in layers)}
+    del g, layers
+    torch.cuda.empty_cache()
+    return res
+
+
+def time_bulk(seed):
+    """Bulk throughput of the compressor and the quantiser."""
+    import torch
+    import compressed_sparse_kv_b200 as K
+    import datagen as D
+    import datagen.gpu as G
+    out = {}
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    raw = G.normal_bf16_(torch.empty(8, 131072, 512, dtype=torch.bfloat16, device="cuda"), D.stream_key(seed, D.TID_RAW_S))
+    for kind, st, k in (("c4a", 4, 8), ("c128a", 128, 128)):
+        w = torch.from_numpy(D.compress_weights(seed, 0, k, 512)).cuda()
+        n = K.compress_entries(131072, 128, st)
+        o = torch.empty(8, n, 512, dtype=torch.bfloat16, device="cuda")
+        for _ in range(3):
+            K.compress(raw, w, st, 128, out=o)
+        s.record()
+        for _ in range(10):
+            K.compress(raw, w, st, 128, out=o)
+        e.record()
+        e.synchronize()
+        ms = s.elapsed_time(e) / 10
+        byts = raw.numel() * 2 + o.numel() * 2
+        out[f"compress_{kind}"] = {"workload": f"B=8 t=131072 -> {n} entries, bf16 out", "us": round(ms * 1e3, 1),
+                                   "gbs": round(byts / (ms * 1e-3) / 1e9, 1)}
+    x = raw.view(-1, 512)[: 64 * 2175]
+    for fmt, name, rb in ((1, "fp8", 516), (2, "fp4", 288)):
+        codes, scales = K.quantize(x, fmt)
+        s.record()
+        for _ in range(10):
+            K.quantize(x, fmt, codes, scales)
+        e.record()
+        e.synchronize()
+        ms = s.elapsed_time(e) / 10
+        byts = x.shape[0] * (1024 + rb)
+        out[f"quantize_{name}"] = {"workload": f"{x.shape[0]} rows x 512 bf16", "us": round(ms * 1e3, 1),
+                                   "gbs": round(byts / (ms * 1e-3) / 1e9, 1)}
+    del raw
+    torch.cuda.empty_cache()
+    return out
 
 
 def time_layer(layer, steps, warmup, dist_max, dev_index, sample_clocks):
-    """Device time of exactly `steps` steps (CUDA graphs per call, events per call)."""
+    """Device time of exactly `steps` steps.  All steps (replicas alternating)
+    are captured into one CUDA graph with event nodes between the calls, so
+    the host launches once and the per-call device times come from the
+    events of the timed replay itself."""
     torch = layer.torch
     R = len(layer.reps)
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
         for i in range(max(warmup, 1)):
-            if layer.kind == "c4a":
-                layer.index(i % R)
-            layer.decode(i % R)
+            layer.step(i % R)
     stream.synchronize()
-    # capture each call of each replica into its own graph
-    g_idx, g_dec = [], []
-    for r in range(R):
-        if layer.kind == "c4a":
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                layer.index(r)
-            g_idx.append(g)
+    # external=True: records inside the capture become event nodes of the graph
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(steps)]
+
+    def capture(n_steps, events):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            layer.decode(r)
-        g_dec.append(g)
+            for i in range(n_steps):
+                if events:
+                    events[i][0].record(stream)
+                if layer.kind == "c4a":
+                    layer.index(i % R)
+                if events:
+                    events[i][1].record(stream)
+                layer.decode(i % R)
+                if events:
+                    events[i][2].record(stream)
+        return g
+
+    g_warm = capture(max(warmup, 1), None)
+    g_main = capture(steps, ev)
     with torch.cuda.stream(stream):
-        for i in range(3):
-            if g_idx:
-                g_idx[i % R].replay()
-            g_dec[i % R].replay()
+        g_warm.replay()
     stream.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     dist_barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(dev_index) if sample_clocks else None
     if sampler:
         sampler.__enter__()
     with torch.cuda.stream(stream):
-        for i in range(steps):
-            ev[i][0].record(stream)
-            if g_idx:
-                g_idx[i % R].replay()
-            ev[i][1].record(stream)
-            g_dec[i % R].replay()
-            ev[i][2].record(stream)
+        g_main.replay()
     torch.cuda.synchronize()
     if sampler:
         sampler.__exit__()
     dist_barrier()
     total_ms = ev[0][0].elapsed_time(ev[-1][2])
-    idx_ms = [e[0].elapsed_time(e[1]) for e in ev] if g_idx else [0.0]
+    idx_ms = [e[0].elapsed_time(e[1]) for e in ev] if layer.kind == "c4a" else [0.0]
     dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
     total_ms = dist_max(total_ms)
+    del g_warm, g_main
     return {"total_ms": total_ms, "index_ms": float(np.mean(idx_ms)), "decode_ms": float(np.mean(dec_ms)),
             "clocks": sampler.summary() if sampler else None}
 
@@ -238,8 +375,8 @@ def time_e2e(layer, steps):
         q_dev.copy_(q_host, non_blocking=True)
         if layer.kind == "c4a":
             qi_dev.copy_(qi_host, non_blocking=True)
-            layer.K.index_topk(qi_dev, layer.K.Cache(0, layer.reps[i % R]["kidx"], None, 128), layer.n, layer.k,
-                               idx_out=layer.idx, count_out=layer.cnt, ws=layer.ws_idx)
+            layer.K.index_topk(qi_dev, layer.reps[i % R]["kidx"], layer.n, layer.k, idx_out=layer.idx,
+                               count_out=layer.cnt, ws=layer.ws_idx)
         layer.decode(i % R, q=q_dev)
         out_host.copy_(layer.out, non_blocking=True)
 
@@ -351,7 +488,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="c4a_b32")
-    ap.add_argument("--secondary", default="c128a_b8,c128a_b32", help="extra per-layer-type workloads ('' = none)")
+    ap.add_argument("--secondary", default="c128a_b8,c128a_b32,q_c4a_fp8,q_c4a_fp4,q_c128a_fp8,q_c128a_fp4",
+                    help="extra per-layer-type workloads (comma list, 'none' = none)")
+    ap.add_argument("--no-stack", action="store_true", help="skip the 61-layer stack step")
+    ap.add_argument("--no-bulk", action="store_true", help="skip compressor/quantiser throughput")
     ap.add_argument("--replicas", type=int, default=2)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -359,13 +499,18 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
     d = dist_init()
-    kind, batch, t, heads = WORKLOADS[args.workload]
-    wl_name = f"{kind} layer decode B={batch} t={t} H={heads} k=512 W=128 bf16 caches"
+    kind, batch, t, heads, mfmt, ifmt = WORKLOADS[args.workload]
+
+    def wl_desc(kind, batch, t, heads, mfmt, ifmt):
+        idx = f", {FMT_NAME[ifmt]} indexer" if kind == "c4a" else ""
+        return f"{kind} layer decode B={batch} t={t} H={heads} k=512 W=128 {FMT_NAME[mfmt]} main cache{idx}"
+
+    wl_name = wl_desc(kind, batch, t, heads, mfmt, ifmt)
 
     if args.impl == "reference":
         if d["rank"] != 0:
             return
-        per_seq, reps = oracle_sample(kind, batch, t, heads, budget_s=max(5.0, args.cpu_budget))
+        per_seq, reps = oracle_sample(kind, batch, t, heads, budget_s=max(5.0, args.cpu_budget))  # bf16 rows
         v = 1.0 / (per_seq * batch)
         cb = {"value": v, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
               "sample": f"{reps} x one sequence of the {batch}-sequence step, scaled to a step"}
@@ -384,7 +529,7 @@ def main():
     torch.cuda.set_device(d["local"])
     hbm_peak, tf_peak, peak_src = measured_peaks()
     seed = 1234 + d["rank"]
-    layer = Layer(kind, batch, t, heads, seed, args.replicas)
+    layer = Layer(kind, batch, t, heads, seed, args.replicas, mfmt, ifmt)
     res = time_layer(layer, args.steps, args.warmup, dist_max, d["local"], sample_clocks=(d["rank"] == 0))
     ms = res["total_ms"] / args.steps
     steps_per_s = d["world"] * 1e3 / ms            # whole job: every rank ran `steps` steps
@@ -410,21 +555,29 @@ def main():
                        "frac_of_8tbs": round(alg / (ms * 1e-3) / 8e12, 4),
                        "index_ms": round(res["index_ms"], 5), "decode_ms": round(res["decode_ms"], 5)}}
     for name in [s for s in args.secondary.split(",") if s and s not in ("none", args.workload)]:
-        k2, b2, t2, h2 = WORKLOADS[name]
-        L2 = Layer(k2, b2, t2, h2, seed + 99, max(args.replicas, 4 if b2 * t2 < 2 ** 21 else 2))
+        spec = WORKLOADS[name]
+        big = spec[1] * spec[2] >= 2 ** 22
+        L2 = Layer(*spec[:4], seed + 99, 2 if big else 4, spec[4], spec[5])
         r2 = time_layer(L2, args.steps, args.warmup, dist_max, d["local"], sample_clocks=False)
         ms2 = r2["total_ms"] / args.steps
         a2 = L2.alg_bytes()
-        per_type.setdefault(k2 if k2 not in per_type else name, {}).update({
-            "workload": f"{k2} layer decode B={b2} t={t2} H={h2} W=128 bf16 caches",
-            "steps_per_s": round(d["world"] * 1e3 / ms2, 1), "hbm_gbs": round(a2 / (ms2 * 1e-3) / 1e9, 1),
-            "frac_of_measured_hbm": round(a2 / (ms2 * 1e-3) / 1e9 / hbm_peak, 4)})
+        per_type[name] = {"workload": wl_desc(*spec), "steps_per_s": round(d["world"] * 1e3 / ms2, 1),
+                          "us_per_step": round(ms2 * 1e3, 2),
+                          "hbm_gbs": round(a2 / (ms2 * 1e-3) / 1e9, 1),
+                          "frac_of_measured_hbm": round(a2 / (ms2 * 1e-3) / 1e9 / hbm_peak, 4),
+                          "tflops": round(L2.flops() / (ms2 * 1e-3) / 1e12, 1),
+                          "frac_of_measured_bf16": round(L2.flops() / (ms2 * 1e-3) / 1e12 / tf_peak, 4)}
+        if spec[0] == "c4a":
+            per_type[name]["index_us"] = round(r2["index_ms"] * 1e3, 2)
+            per_type[name]["decode_us"] = round(r2["decode_ms"] * 1e3, 2)
         del L2
         torch.cuda.empty_cache()
+    stack = None if args.no_stack else time_stack(max(10, args.steps // 20), args.warmup, seed + 7, dist_max)
+    bulk = None if args.no_bulk else time_bulk(seed + 11)
 
     line = {"metric": METRIC, "value": round(steps_per_s, 2), "unit": "steps/s", "n_gpus": d["world"],
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": FMT_NAME[mfmt], "data": "synthetic",
             "config": {"workload": wl_name, "batch_per_gpu": batch, "context": t, "heads": heads,
                        "parallelism": f"dp{d['world']}",
                        "l2": f"{args.replicas} cache replicas alternate; {alg / 1e6:.0f} MB read per step (> 126 MB L2)"},
@@ -433,6 +586,10 @@ def main():
             "e2e": {"value": round(e2e_v, 2), "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": layer.launches_per_step() * args.steps,
             "clocks": res["clocks"]}
+    if stack:
+        line["stack"] = stack
+    if bulk:
+        line["bulk"] = bulk
     if d["rank"] == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(kind, batch, t, heads, args.cpu_budget)
     if d["rank"] == 0:

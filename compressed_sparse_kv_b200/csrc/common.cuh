@@ -44,6 +44,16 @@ __device__ __forceinline__ void set_status(uint32_t* status, uint32_t flag) {
   if (status) atomicOr(status, flag);
 }
 
+// ----------------------------------------------------------------- programmatic dependent launch
+// Every kernel of the library is launched with programmatic stream
+// serialisation: it may start while the previous kernel in the stream is
+// finishing.  Each kernel therefore runs only private set-up (shared memory,
+// TMEM, barriers) before pdl_wait(), which returns once the previous grid has
+// completed and its memory is visible; completion is then transitive along
+// the whole chain.  pdl_trigger() lets the next kernel start its set-up.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ----------------------------------------------------------------- smem / mbarrier
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

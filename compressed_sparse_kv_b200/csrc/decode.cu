@@ -229,6 +229,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::kThreads, 1)
   const int b = blockIdx.x / p.splits, split = blockIdx.x % p.splits;
   const int t0 = split * p.tiles_per_split;
   const int nt = max(0, min(p.tiles, t0 + p.tiles_per_split) - t0);
+  pdl_trigger();
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl->q_full, 1);
@@ -262,6 +263,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
+  pdl_wait();  // everything above touched only shared memory, TMEM and the tensor maps
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (TMA)
@@ -577,6 +579,8 @@ __global__ void __launch_bounds__(128) decode_combine(const float* __restrict__ 
                                                       const float* __restrict__ ml_part, int splits, int heads,
                                                       int64_t t, int rope_dim, double rope_base, int out_fp32,
                                                       void* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   const int bh = blockIdx.x;
   const int b = bh / heads, h = bh % heads;
   const int c = 4 * threadIdx.x;
@@ -684,7 +688,7 @@ dsv4kv_status launch_fmt(const CUtensorMap& tq, const CUtensorMap& tc, const CUt
       return check_launch("decode: cudaFuncSetAttribute");
     attr_set = true;
   }
-  decode_kernel<FMT><<<grid, Cfg<FMT>::kThreads, kSmemBytes, stream>>>(tq, tc, tw, p);
+  launch_pdl(decode_kernel<FMT>, dim3(grid), dim3(Cfg<FMT>::kThreads), kSmemBytes, stream, tq, tc, tw, p);
   return check_launch("decode_kernel");
 }
 
@@ -754,8 +758,8 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
     default: st = launch_fmt<DSV4KV_FP4_E2M1_G16>(tq, tc, tw, p, grid, stream); break;
   }
   if (st != DSV4KV_OK) return st;
-  decode_combine<<<a.batch * a.heads, kDim / 4, 0, stream>>>(w.o_part, w.ml_part, pl.splits, a.heads, a.t,
-                                                              a.rope_dim, a.rope_base, a.out_fp32, a.out);
+  launch_pdl(decode_combine, dim3(a.batch * a.heads), dim3(kDim / 4), 0, stream, (const float*)w.o_part,
+             (const float*)w.ml_part, pl.splits, a.heads, a.t, a.rope_dim, a.rope_base, a.out_fp32, a.out);
   return check_launch("decode_combine");
 }
 

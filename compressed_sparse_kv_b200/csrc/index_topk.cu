@@ -83,10 +83,12 @@ __global__ void __launch_bounds__(256) index_score_bf16(const uint16_t* __restri
                                                         int64_t n, int batch, int64_t per_cta,
                                                         float* __restrict__ scores, uint32_t* __restrict__ hist) {
   __shared__ uint32_t sh[kHistBins];
+  pdl_trigger();
   const int64_t total = int64_t(batch) * n;
   const int64_t g0 = int64_t(blockIdx.x) * per_cta;
   const int64_t g1 = min(total, g0 + per_cta);
   if (g0 >= g1) return;
+  pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int half = lane >> 4, l16 = lane & 15;
   const int my_key = U == 16 ? l16 : ((l16 >> 1) & 7);
@@ -215,10 +217,12 @@ __global__ void __launch_bounds__(256) index_score_fp4(const uint16_t* __restric
                                                        int64_t n, int64_t chunk, float* __restrict__ scores,
                                                        uint32_t* __restrict__ hist) {
   __shared__ uint32_t sh[kHistBins];
+  pdl_trigger();
   const int b = blockIdx.y;
   const int64_t n0 = int64_t(blockIdx.x) * chunk;
   const int64_t n1 = min(n, n0 + chunk);
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0;
+  pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int quad = lane >> 2, l4 = lane & 3;  // key slot in the warp, segment in the key
   // Lane l4 covers channels [32*l4, 32*l4+32).  Word j of its 16 B holds
@@ -411,6 +415,8 @@ __global__ void __launch_bounds__(kSelThreads) index_filter_select(
   const float* sc = scores + size_t(b) * size_t(n);
   uint64_t* cb = cand + size_t(b) * size_t(cap);
   const int lane = threadIdx.x & 31;
+  pdl_trigger();
+  pdl_wait();
 
   // 1) threshold bin of the top-12-bit histogram
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = hb[i];
@@ -593,6 +599,8 @@ __global__ void __launch_bounds__(kSelThreads) index_filter_select(
 }
 
 __global__ void index_fill_all(int64_t n, int k, int32_t* __restrict__ idx_out, int32_t* __restrict__ count_out) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.y;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < k; i += gridDim.x * blockDim.x)
     idx_out[size_t(b) * k + i] = i < n ? i : -1;
@@ -648,7 +656,8 @@ dsv4kv_status index_topk_launch(const uint16_t* qidx, const dsv4kv_cache& keys, 
                                 cudaStream_t stream) {
   if (n <= k) {
     const dim3 grid((unsigned)((k + 255) / 256), (unsigned)batch);
-    index_fill_all<<<grid, 256, 0, stream>>>(n, k, idx_out, count_out);
+    if (launch_pdl(index_fill_all, grid, dim3(256), 0, stream, n, k, idx_out, count_out) != cudaSuccess)
+      return check_launch("index_fill_all");
     return check_launch("index_fill_all");
   }
   const IndexWs w = index_ws_layout(static_cast<char*>(ws), batch, n, k);
@@ -664,8 +673,8 @@ dsv4kv_status index_topk_launch(const uint16_t* qidx, const dsv4kv_cache& keys, 
     const int64_t total = int64_t(batch) * n;
     const int64_t grid = int64_t(sms) * occ;
     const int64_t per_cta = std::max<int64_t>(64, (total + grid - 1) / grid);
-    index_score_bf16<8, true><<<unsigned((total + per_cta - 1) / per_cta), 256, 0, stream>>>(
-        qidx, static_cast<const uint16_t*>(keys.codes), keys.rows, n, batch, per_cta, w.scores, w.hist);
+    launch_pdl(index_score_bf16<8, true>, dim3(unsigned((total + per_cta - 1) / per_cta)), dim3(256), 0, stream, qidx,
+               static_cast<const uint16_t*>(keys.codes), keys.rows, n, batch, per_cta, w.scores, w.hist);
   } else {
     const int64_t target = int64_t(sms) * 4;
     int64_t splits = std::max<int64_t>(1, (target + batch - 1) / batch);
@@ -673,9 +682,8 @@ dsv4kv_status index_topk_launch(const uint16_t* qidx, const dsv4kv_cache& keys, 
     chunk = std::max<int64_t>(256, (chunk + 31) / 32 * 32);
     splits = (n + chunk - 1) / chunk;
     const dim3 g1((unsigned)splits, (unsigned)batch);
-    index_score_fp4<<<g1, 256, 0, stream>>>(qidx, static_cast<const uint8_t*>(keys.codes),
-                                            static_cast<const uint8_t*>(keys.scales), keys.rows, n, chunk, w.scores,
-                                            w.hist);
+    launch_pdl(index_score_fp4, g1, dim3(256), 0, stream, qidx, static_cast<const uint8_t*>(keys.codes),
+               static_cast<const uint8_t*>(keys.scales), keys.rows, n, chunk, w.scores, w.hist);
   }
   dsv4kv_status st = check_launch("index_score");
   if (st != DSV4KV_OK) return st;
@@ -691,9 +699,8 @@ dsv4kv_status index_topk_launch(const uint16_t* qidx, const dsv4kv_cache& keys, 
       return check_launch("index_filter_select: cudaFuncSetAttribute");
     attr_set = true;
   }
-  index_filter_select<<<g2, kSelThreads, dyn, stream>>>(w.scores, n, k, chunk2, w.hist, w.hist2, w.done,
-                                                        w.cand_count, w.cand, w.cap, idx_out, count_out,
-                                                        w.status);
+  launch_pdl(index_filter_select, g2, dim3(kSelThreads), dyn, stream, w.scores, n, k, chunk2, w.hist, w.hist2, w.done,
+             w.cand_count, w.cand, w.cap, idx_out, count_out, w.status);
   return check_launch("index_filter_select");
 }
 
