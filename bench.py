@@ -149,6 +149,7 @@ class Layer:
             self.reps.append(rep)
         keys = WL.keys_for(seed, layer_id)
         self.q = G.normal_bf16_(torch.empty(batch, heads, 512, dtype=torch.bfloat16, device=dev), keys["q"])
+        # the inputs are generated on the current stream; the timed work runs on its own stream
         self.qidx = G.int_bf16_(torch.empty(batch, 128, dtype=torch.bfloat16, device=dev), keys["qidx"])
         sh = shared if shared is not None else {}
         self.idx = sh.setdefault("idx", torch.empty(batch, self.k, dtype=torch.int32, device=dev))
@@ -165,6 +166,7 @@ class Layer:
         if "ws_dec" not in sh or sh["ws_dec"].numel() < need_d:
             sh["ws_dec"] = K.new_workspace(need_d)
         self.ws_dec = sh["ws_dec"]
+        torch.cuda.synchronize()  # inputs and zeroed workspaces are complete before any other stream uses them
 
     # algorithmic bytes of one step: indexer keys + rows read (queries/outputs excluded)
     def alg_bytes(self):

@@ -6,22 +6,28 @@
 // output; [P1] "c4a" / "c128a" and [P2] Step 5: c4a reads the top-k selected
 // entries, c128a reads all of them.
 //
-// One CTA per (sequence, split) runs over a contiguous range of 64-row tiles
-// of that sequence's row list (selected or all compressed rows, then window
-// rows).  Per tile:
-//   * warp 0 gathers the 64 rows into shared memory with TMA tile::gather4
-//     (4 rows x 64 channels per copy, 128-byte swizzle);
+// One CTA per (sequence, split) walks a contiguous range of 64-row tiles of
+// the sequence's row list (selected or all compressed rows, then the window
+// rows).  Roles (10 warps):
+//   * warp 0 loads Q (TMA, 128-byte swizzle) and every tile whose rows are
+//     contiguous in HBM (dense compressed rows, window rows) with 2D TMA
+//     tiles: 8 copies of 64 rows x 64 channels per tile;
+//   * warps 6-9 load the tiles that are not: gathered bf16 rows with 16-byte
+//     cp.async straight into the swizzled tile, and quantised rows
+//     (fp8 / fp4) with 16-byte loads and hardware cvt to f16 (exact);
 //   * warp 1 (one thread) issues tcgen05.mma: S = Q . R^T (M = 64 heads,
-//     N = 64 rows, K = 512) into TMEM, then O^T += R^T . P^T (M = 128 channels
-//     x 4 tiles, N = 64 heads, K = 64 rows) — the SAME shared-memory tile is
-//     the K-major B operand of the first product and the MN-major A operand
-//     of the second, which is the shared-K/V saving;
-//   * warps 2-5 run the online softmax out of TMEM (one thread per head),
-//     write P (bf16) to shared memory, and rescale the O^T accumulator in TMEM
-//     only when a head's running max grows by more than 2^8.
-// Partial (O, m, l) per split go to the workspace; decode_combine merges the
-// splits with their log-sum-exp weights, normalises, applies the inverse RoPE
-// to the rotary channels and stores bf16 or fp32.
+//     N = 64 rows, 32 K-steps of 16 channels; head h lands in TMEM lane
+//     32*(h/16) + h%16, row r in column r), and O^T += R^T . P^T
+//     (M = 128 channels x 4, N = 64 heads, K = 64 rows) from the SAME
+//     shared-memory tile — the shared-K/V saving.  It issues whichever
+//     product is ready first;
+//   * warps 2-5 run the online softmax out of TMEM with 16-lane loads: a
+//     quad of threads shares two heads, each thread 16 rows of both; they
+//     write P (16-bit) to shared memory and rescale the O^T accumulator in
+//     TMEM only when a head's running max grows by > 2^8.
+// With one split per sequence the CTA normalises, applies the inverse RoPE
+// and stores the output itself; otherwise partial (O, m, l) go to the
+// workspace and decode_combine merges them with log-sum-exp weights.
 #include <cmath>
 #include <cstdint>
 
@@ -40,22 +46,20 @@ constexpr int kChunkBytes = kTileRows * 128;       // 8 KB
 constexpr int kTileBytes = kChunks * kChunkBytes;  // 64 KB
 constexpr int kQBytes = kChunks * 64 * 128;        // 64 heads x 512 channels, 16-bit
 constexpr int kPBytes = 64 * 128;                  // 64 heads x 64 rows, 16-bit
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;    // O^T: 4 channel tiles x 64 heads
-constexpr uint32_t kColS = 256;  // scores: 2 buffers x 64 rows (M = 64 layout)
+constexpr uint32_t kColS = 256;  // scores: 2 buffers x 64 columns
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-// Per-format configuration.  bf16 caches go straight from HBM to the MMA
-// operand tile by TMA gather and run kind::f16 with bf16 inputs.  Quantised
-// caches are dequantised in the load path by four converter warps (16-byte
-// loads straight from HBM, hardware cvt to f16, swizzled stores); every
-// E4M3 value and every E2M1 x E4M3 product is exact in f16, so those run
-// kind::f16 with f16 inputs (Q is converted to f16 once per CTA).
+// Per-format configuration.  bf16 rows feed kind::f16 MMAs with bf16 inputs.
+// Quantised rows are dequantised in the load path; every E4M3 value and every
+// E2M1 x E4M3 product is exact in f16, so those run kind::f16 with f16 inputs
+// (Q is converted to f16 once per CTA).
 template <int FMT>
 struct Cfg {
   static constexpr bool kQuant = FMT != DSV4KV_BF16;
   static constexpr bool kRowScale = FMT == DSV4KV_FP8_E4M3_ROW;
-  static constexpr int kThreads = kQuant ? 320 : 192;
   static constexpr uint32_t kIdescQK = kQuant ? idesc_f16(64, 64, 0, 0) : idesc_bf16(64, 64, 0, 0);
   static constexpr uint32_t kIdescPV = kQuant ? idesc_f16(128, 64, 1, 0) : idesc_bf16(128, 64, 1, 0);
 };
@@ -73,7 +77,11 @@ struct __align__(8) Ctl {
   uint32_t tmem_base;
   volatile int abort;
   float alpha[64];
+  float fin[64];
   float row_scale[kStages][kTileRows];
+  uint32_t vmask[kStages][4];  // row validity of a gathered tile, 16 rows per loader warp
+  float rope_cs[kDim / 2];  // inverse-RoPE rotation of pair m: cos / sin of -t * theta_m
+  float rope_sn[kDim / 2];
 };
 
 constexpr size_t kSmemBytes = 1024 + kQBytes + kStages * kTileBytes + 2 * kPBytes + sizeof(Ctl);
@@ -86,14 +94,21 @@ struct Params {
   int comp_tiles, tiles, splits, tiles_per_split;
   int64_t comp_rows, win_rows;  // per-sequence row capacity of each cache
   const int32_t* idx;           // [B][k] or null (dense)
-  const uint8_t* comp_codes;    // quantised caches (converter warps)
+  const uint8_t* comp_codes;
   const void* comp_scales;
   const uint8_t* win_codes;
   const void* win_scales;
-  float score_scale;            // sm_scale * log2(e)
-  float* o_part;                // [B][splits][H][512]
-  float* ml_part;               // [B][splits][H][4]: (m_o, m_l, l, 0)
+  float score_scale;  // sm_scale * log2(e)
+  float* o_part;      // [B][splits][H][512]
+  float* ml_part;     // [B][splits][H][4]: (m_o, m_l, l, 0)
+  float* rope_tab;    // [2][256]: the rotation table for decode_combine (written by CTA 0)
   uint32_t* status;
+  // direct output when splits == 1
+  int64_t t;
+  int rope_dim;
+  double rope_base;
+  int out_fp32;
+  void* out;
 };
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -102,8 +117,10 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 
-// Bounded wait (about one second); on timeout or when another role gave up,
-// returns false and raises the CTA's abort flag.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // one second
+
+// Bounded wait; on timeout or when another role gave up, returns false and
+// raises the CTA's abort flag.
 __device__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ctl* ctl) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
@@ -112,7 +129,7 @@ __device__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ctl* ctl) {
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (ctl->abort) return false;
-    if (globaltimer() - t0 > 1000000000ull) {
+    if (globaltimer() - t0 > kWaitLimitNs) {
       ctl->abort = 1;
       return false;
     }
@@ -137,9 +154,22 @@ __device__ __forceinline__ bool named_bar_or(bool pred) {
 }
 __device__ __forceinline__ void named_bar_sync() { asm volatile("barrier.cta.sync 1, 128;" ::: "memory"); }
 
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// Whether tile T is a run of contiguous rows (TMA tile) rather than a gather.
+__device__ __forceinline__ bool tile_contiguous(const Params& p, int T) {
+  return T >= p.comp_tiles || p.idx == nullptr;
+}
+
 // Source of row `r` of tile T: global row (b * rows + i) of the compressed
 // cache (from_win = false) or of the window cache; valid = false for padding
-// slots and for rejected indices (the row then reads nothing).
+// slots and rejected indices (the row then reads row 0 of the sequence, which
+// is finite, and is masked in the softmax).
 struct RowSrc {
   int64_t row;
   bool valid, from_win;
@@ -167,26 +197,23 @@ __device__ __forceinline__ RowSrc row_source(const Params& p, int b, int T, int 
   return s;
 }
 
-// Row validity of tile T (rows lane and lane+32 of the tile), warp-wide.
-__device__ __forceinline__ uint64_t tile_valid_mask(const Params& p, int b, int T, int lane) {
-  bool v0, v1;
-  if (T < p.comp_tiles) {
-    const int s0 = T * kTileRows + lane, s1 = s0 + 32;
-    if (p.idx) {
-      const int32_t* ib = p.idx + size_t(b) * p.k;
-      const int32_t i0 = s0 < p.k ? ib[s0] : -1, i1 = s1 < p.k ? ib[s1] : -1;
-      v0 = i0 >= 0 && i0 < p.n;
-      v1 = i1 >= 0 && i1 < p.n;
-    } else {
-      v0 = s0 < p.n;
-      v1 = s1 < p.n;
-    }
-  } else {
-    const int w0 = (T - p.comp_tiles) * kTileRows + lane;
-    v0 = w0 < p.window;
-    v1 = w0 + 32 < p.window;
-  }
-  return uint64_t(__ballot_sync(kFull, v0)) | (uint64_t(__ballot_sync(kFull, v1)) << 32);
+// Row validity of a contiguous tile: the first n - 64T compressed rows, or
+// the first window - 64(T - comp_tiles) window rows.
+__device__ __forceinline__ uint64_t contiguous_mask(const Params& p, int T) {
+  const int64_t lim = T < p.comp_tiles ? p.n - int64_t(T) * kTileRows
+                                       : int64_t(p.window) - int64_t(T - p.comp_tiles) * kTileRows;
+  return lim >= kTileRows ? ~0ull : (lim <= 0 ? 0ull : ((1ull << lim) - 1ull));
+}
+
+// cos / sin of the inverse-RoPE angle -t * rope_base^(-2m/rope_dim): the
+// angle in units of pi is reduced exactly modulo 2 before sincospi.
+__device__ __forceinline__ void inv_rope_rotation(int64_t t, int m, int rope_dim, double rope_base, float* cs,
+                                                  float* sn) {
+  const double ang = double(t) * (pow(rope_base, -2.0 * double(m) / double(rope_dim)) / 3.141592653589793);
+  double sd, cd;
+  sincospi(-(ang - 2.0 * rint(0.5 * ang)), &sd, &cd);
+  *cs = float(cd);
+  *sn = float(sd);
 }
 
 // 2^x with the hardware approximation (max relative error ~2^-22, far below
@@ -214,7 +241,7 @@ __device__ __forceinline__ float p_hi(uint32_t v, bool f16) {
 }
 
 template <int FMT>
-__global__ void __launch_bounds__(Cfg<FMT>::kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_comp,
                   const __grid_constant__ CUtensorMap tm_win, const Params p) {
   using C = Cfg<FMT>;
@@ -235,7 +262,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::kThreads, 1)
     mbar_init(&ctl->q_full, 1);
     mbar_init(&ctl->q_ready, 4);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&ctl->full[s], C::kQuant ? 4 : 1);
+      mbar_init(&ctl->full[s], 5);  // warp 0 + the four loader warps, every tile
       mbar_init(&ctl->empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -266,39 +293,28 @@ __global__ void __launch_bounds__(Cfg<FMT>::kThreads, 1)
   pdl_wait();  // everything above touched only shared memory, TMEM and the tensor maps
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer (TMA)
+    // ------------------------------------------------------------ TMA: Q and contiguous tiles
     if (lane == 0) {
       mbar_arrive_expect_tx(&ctl->q_full, kQBytes);
       for (int c = 0; c < kChunks; ++c) tma_load_3d(sQ + c * kChunkBytes, &tm_q, &ctl->q_full, c * 64, 0, b);
-    }
-    int issued = 0;
-    if (!C::kQuant) {
+      int issued = 0;
       for (int i = 0; i < nt; ++i) {
         const int T = t0 + i, stage = i % kStages;
-        if (i >= kStages && !warp_wait(&ctl->empty[stage], ((i / kStages) - 1) & 1, ctl, lane)) break;
-        if (lane == 0) mbar_arrive_expect_tx(&ctl->full[stage], kTileBytes);
-        __syncwarp();
-        const int g = lane & 15;  // 4-row group of this lane
-        int32_t r[4];
-        bool from_win = false;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const RowSrc s = row_source(p, b, T, 4 * g + e);
-          r[e] = int32_t(s.row);
-          from_win = s.from_win;
-        }
-        const CUtensorMap* tm = from_win ? &tm_win : &tm_comp;
-        uint8_t* dst = sR + stage * kTileBytes + g * 512;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int c = (lane >> 4) * 4 + cc;
-          tma_gather4(dst + c * kChunkBytes, tm, &ctl->full[stage], c * 64, r[0], r[1], r[2], r[3]);
+        if (i >= kStages && !wait_or_abort(&ctl->empty[stage], ((i / kStages) - 1) & 1, ctl)) break;
+        if (!C::kQuant && tile_contiguous(p, T)) {
+          const RowSrc s0 = row_source(p, b, T, 0);  // first row of the run
+          const CUtensorMap* tm = s0.from_win ? &tm_win : &tm_comp;
+          const int32_t row0 = int32_t(s0.from_win ? int64_t(b) * p.win_rows + (T - p.comp_tiles) * kTileRows
+                                                   : int64_t(b) * p.comp_rows + int64_t(T) * kTileRows);
+          mbar_arrive_expect_tx(&ctl->full[stage], kTileBytes);
+          uint8_t* dst = sR + stage * kTileBytes;
+          for (int c = 0; c < kChunks; ++c) tma_load_2d(dst + c * kChunkBytes, tm, &ctl->full[stage], c * 64, row0);
+        } else {
+          mbar_arrive(&ctl->full[stage]);
         }
         issued = i + 1;
       }
-    }
-    // drain: never leave the CTA with copies in flight
-    if (lane == 0) {
+      // drain: never leave the CTA with copies in flight
       wait_or_abort(&ctl->q_full, 0, ctl);
       for (int i = max(0, issued - kStages); i < issued; ++i)
         wait_or_abort(&ctl->full[i % kStages], (i / kStages) & 1, ctl);
@@ -307,28 +323,13 @@ __global__ void __launch_bounds__(Cfg<FMT>::kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = wait_or_abort(C::kQuant ? &ctl->q_ready : &ctl->q_full, 0, ctl);
-      const uint32_t q_addr = smem_u32(sQ);
-      for (int i = 0; ok && i <= nt; ++i) {
-        if (i < nt) {
-          const int stage = i % kStages, sb = i & 1;
-          ok = wait_or_abort(&ctl->full[stage], (i / kStages) & 1, ctl);
-          if (ok && i >= 2) ok = wait_or_abort(&ctl->s_free[sb], ((i - 2) >> 1) & 1, ctl);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t r_addr = smem_u32(sR + stage * kTileBytes);
-          const uint32_t d = tmem + kColS + 64 * sb;
-#pragma unroll
-          for (int kk = 0; kk < kDim / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-            mma_bf16_ss(d, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(r_addr + off, 16, 1024),
-                        C::kIdescQK, kk > 0);
-          }
-          mma_commit(&ctl->s_full[sb]);
-        }
-        if (i >= 1) {
-          const int j = i - 1, stage = j % kStages, pb = j & 1;
-          ok = wait_or_abort(&ctl->p_full[pb], (j >> 1) & 1, ctl);
-          if (!ok) break;
+      const uint64_t qd = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+      int next_qk = 0, next_pv = 0;
+      uint64_t idle_since = 0;
+      while (ok && next_pv < nt) {
+        bool progressed = false;
+        if (next_pv < next_qk && mbar_try_wait(&ctl->p_full[next_pv & 1], (next_pv >> 1) & 1)) {
+          const int j = next_pv, stage = j % kStages, pb = j & 1;
           tc_fence_after();
           const uint32_t r_addr = smem_u32(sR + stage * kTileBytes);
           const uint32_t p_addr = smem_u32(sP + pb * kPBytes);
@@ -343,71 +344,144 @@ __global__ void __launch_bounds__(Cfg<FMT>::kThreads, 1)
           }
           mma_commit(&ctl->empty[stage]);
           mma_commit(&ctl->pv_done);
+          ++next_pv;
+          progressed = true;
+        } else if (next_qk < nt && next_qk < next_pv + 2) {
+          const int i = next_qk, stage = i % kStages, sb = i & 1;
+          if (mbar_try_wait(&ctl->full[stage], (i / kStages) & 1) &&
+              (i < 2 || mbar_try_wait(&ctl->s_free[sb], ((i - 2) >> 1) & 1))) {
+            tc_fence_after();
+            const uint64_t rd = smem_desc_sw128(smem_u32(sR + stage * kTileBytes), 16, 1024);
+            const uint32_t d = tmem + kColS + 64 * sb;
+#pragma unroll
+            for (int kk = 0; kk < kDim / 16; ++kk) {
+              const uint32_t off16 = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;  // descriptor address units
+              mma_bf16_ss(d, qd + off16, rd + off16, C::kIdescQK, kk > 0);
+            }
+            mma_commit(&ctl->s_full[sb]);
+            ++next_qk;
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          idle_since = 0;
+        } else {
+          const uint64_t now = globaltimer();
+          if (idle_since == 0) idle_since = now;
+          if (ctl->abort || now - idle_since > kWaitLimitNs) {
+            ctl->abort = 1;
+            ok = false;
+          }
         }
       }
       mma_commit(&ctl->o_done);  // completes once every issued MMA has finished
     }
   } else if (warp < 6) {
     // ------------------------------------------------------------ softmax + epilogue (warps 2..5)
-    // After a timed-out wait a warp turns `dead` (warp-uniform): it skips
-    // every wait, TMEM and shared-memory access but still takes part in the
-    // group's named barriers, so the other softmax warps cannot hang on them.
+    // Warp w reads TMEM lane quarter wq = w % 4 (heads 16wq .. 16wq+15).  A
+    // 16x256b.x8 load gives thread i the scores of heads hA = 16wq + i/4 and
+    // hB = hA + 8 at rows 8j + 2(i%4) + {0, 1} (j < 8): the four threads of a
+    // quad share two heads and reduce over the quad.  After a timed-out wait a
+    // warp turns `dead` (warp-uniform): it skips every wait, TMEM and
+    // shared-memory access but still takes part in the group's named barriers.
     //
-    // Two running maxima: m_l for the softmax denominator l and m_o for the
-    // weights that multiply the stored rows.  With fp8 rows the per-row scale
-    // s_r is folded into the weights (w_r = p_r * s_r, y_r = x_r + log2 s_r),
-    // so the accumulator's weights stay <= 2^8 whatever the scales are; for
-    // other formats y == x and the two maxima coincide.
-    const int wq = warp & 3;  // TMEM lane quadrant of this warp
+    // Two running maxima per head: m_l for the softmax denominator l and m_o
+    // for the weights that multiply the stored rows.  With fp8 rows the
+    // per-row scale s_r is folded into the weights (w_r = p_r * s_r,
+    // y_r = x_r + log2 s_r), so the accumulator's weights stay <= 2^8 whatever
+    // the scales are; for other formats y == x and the two maxima coincide.
+    const int wq = warp & 3;  // TMEM lane quarter of this warp
     const uint32_t lane_base = uint32_t(32 * wq) << 16;
-    const bool head_thread = lane < 16;
-    const int h = 16 * wq + (lane & 15);
-    float m_o = -INFINITY, m_l = -INFINITY, l = 0.f;
+    const int g = lane >> 2, c2 = lane & 3;
+    const int hd[2] = {16 * wq + g, 16 * wq + 8 + g};
+    // the inverse-RoPE table, while the first tile is still in flight
+    for (int m = threadIdx.x - 64; m < p.rope_dim / 2; m += 128) {
+      float cs, sn;
+      inv_rope_rotation(p.t, m, p.rope_dim, p.rope_base, &cs, &sn);
+      ctl->rope_cs[m] = cs;
+      ctl->rope_sn[m] = sn;
+      if (p.splits > 1 && blockIdx.x == 0) {
+        p.rope_tab[m] = cs;
+        p.rope_tab[kDim / 2 + m] = sn;
+      }
+    }
+    float m_o[2] = {-INFINITY, -INFINITY}, m_l[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
     bool dead = false;
     for (int i = 0; i < nt; ++i) {
       const int T = t0 + i, sb = i & 1, stage = i % kStages;
+      const bool gathered = C::kQuant || !tile_contiguous(p, T);
       if (!dead) dead = !warp_wait(&ctl->s_full[sb], (i >> 1) & 1, ctl, lane);
-      if (C::kRowScale && !dead) dead = !warp_wait(&ctl->full[stage], (i / kStages) & 1, ctl, lane);
-      float x[64];
-      float tmax = -INFINITY, ymax = -INFINITY;
+      // the loaders' row mask and row scales (complete: the MMA already consumed this tile)
+      if ((gathered || C::kRowScale) && !dead) dead = !warp_wait(&ctl->full[stage], (i / kStages) & 1, ctl, lane);
+      float x[2][16];
+      float tmax[2] = {-INFINITY, -INFINITY}, ymax[2] = {-INFINITY, -INFINITY};
       if (!dead) {
         tc_fence_after();
-        uint32_t s0[32], s1[32];
-        tmem_ld32(tmem + lane_base + kColS + 64 * sb, s0);
-        tmem_ld32(tmem + lane_base + kColS + 64 * sb + 32, s1);
+        uint32_t sc[32];
+        tmem_ld_16x256b_x8(tmem + lane_base + kColS + 64 * sb, sc);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->s_free[sb]);
-        const uint64_t vmask = tile_valid_mask(p, b, T, lane);
+        const uint64_t vm = gathered ? (uint64_t(ctl->vmask[stage][0]) | (uint64_t(ctl->vmask[stage][1]) << 16) |
+                                        (uint64_t(ctl->vmask[stage][2]) << 32) | (uint64_t(ctl->vmask[stage][3]) << 48))
+                                     : contiguous_mask(p, T);
 #pragma unroll
-        for (int r = 0; r < 64; ++r) {
-          const float raw = __uint_as_float(r < 32 ? s0[r] : s1[r - 32]);
-          const bool v = (vmask >> r) & 1;
-          if (C::kRowScale) {
-            const float sc = ctl->row_scale[stage][r];
-            x[r] = v ? raw * sc * p.score_scale : -INFINITY;
-            ymax = fmaxf(ymax, (v && sc > 0.f) ? x[r] + __log2f(sc) : -INFINITY);
-          } else {
-            x[r] = v ? raw * p.score_scale : -INFINITY;
+        for (int j = 0; j < 8; ++j) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int r = 8 * j + 2 * c2 + e;
+            const bool v = (vm >> r) & 1;
+            float ls = 0.f;
+            bool sok = true;
+            if (C::kRowScale) {
+              const float s = ctl->row_scale[stage][r];
+              sok = s > 0.f;
+              ls = sok ? __log2f(s) : 0.f;
+            }
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              float xv = v ? __uint_as_float(sc[4 * j + 2 * hh + e]) * p.score_scale : -INFINITY;
+              if (C::kRowScale) {
+                xv = v ? xv * ctl->row_scale[stage][r] : -INFINITY;
+                ymax[hh] = fmaxf(ymax[hh], (v && sok) ? xv + ls : -INFINITY);
+              }
+              x[hh][2 * j + e] = xv;
+              tmax[hh] = fmaxf(tmax[hh], xv);
+            }
           }
-          tmax = fmaxf(tmax, x[r]);
         }
-        if (!C::kRowScale) ymax = tmax;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          if (!C::kRowScale) ymax[hh] = tmax[hh];
+#pragma unroll
+          for (int o = 1; o <= 2; o <<= 1) {
+            tmax[hh] = fmaxf(tmax[hh], __shfl_xor_sync(kFull, tmax[hh], o));
+            if (C::kRowScale) ymax[hh] = fmaxf(ymax[hh], __shfl_xor_sync(kFull, ymax[hh], o));
+          }
+          if (!C::kRowScale) ymax[hh] = tmax[hh];
+        }
         if (i >= 1) dead = !warp_wait(&ctl->pv_done, (i - 1) & 1, ctl, lane);
       }
-      if (!dead && tmax > m_l + kRescaleThreshold) {
-        l *= (m_l == -INFINITY) ? 0.f : exp2f(m_l - tmax);
-        m_l = tmax;
-      }
-      const bool need = !dead && head_thread && ymax > m_o + kRescaleThreshold;
-      float alpha = 1.f;
-      if (need) {
-        alpha = (m_o == -INFINITY) ? 0.f : exp2f(m_o - ymax);
-        m_o = ymax;
+      bool need = false;
+      float alpha[2] = {1.f, 1.f};
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        if (!dead && tmax[hh] > m_l[hh] + kRescaleThreshold) {
+          l[hh] *= (m_l[hh] == -INFINITY) ? 0.f : fast_exp2(m_l[hh] - tmax[hh]);
+          m_l[hh] = tmax[hh];
+        }
+        if (!dead && ymax[hh] > m_o[hh] + kRescaleThreshold) {
+          alpha[hh] = (m_o[hh] == -INFINITY) ? 0.f : fast_exp2(m_o[hh] - ymax[hh]);
+          m_o[hh] = ymax[hh];
+          need = true;
+        }
       }
       if (i >= 1 && named_bar_or(need)) {
-        if (!dead && head_thread) ctl->alpha[h] = alpha;
+        if (!dead && c2 == 0) {
+          ctl->alpha[hd[0]] = alpha[0];
+          ctl->alpha[hd[1]] = alpha[1];
+        }
         named_bar_sync();
         if (!dead) {
           tc_fence_after();
@@ -430,31 +504,29 @@ __global__ void __launch_bounds__(Cfg<FMT>::kThreads, 1)
         named_bar_sync();  // alpha[] is rewritten only after everyone read it
       }
       if (dead) continue;
-      if (head_thread) {
-        uint8_t* prow = sP + sb * kPBytes + (h >> 3) * 1024 + (h & 7) * 128;
 #pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16) {
-          uint32_t w[4];
+      for (int hh = 0; hh < 2; ++hh) {
+        const int h = hd[hh];
+        uint8_t* prow = sP + sb * kPBytes + (h >> 3) * 1024 + (h & 7) * 128 + 4 * c2;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int r = 8 * c16 + 2 * e;
-            float ya = x[r], yb = x[r + 1];
-            if (C::kRowScale) {  // y = x + log2(s_r): the weight of the stored row carries its scale
-              const float sa = ctl->row_scale[stage][r], sb2 = ctl->row_scale[stage][r + 1];
-              ya = sa > 0.f ? ya + __log2f(sa) : -INFINITY;
-              yb = sb2 > 0.f ? yb + __log2f(sb2) : -INFINITY;
-            }
-            const float wa = (m_o == -INFINITY) ? 0.f : fast_exp2(ya - m_o);
-            const float wb = (m_o == -INFINITY) ? 0.f : fast_exp2(yb - m_o);
-            const uint32_t packed = pack_p(wa, wb, C::kQuant);
-            if (C::kRowScale) {
-              if (m_l != -INFINITY) l += fast_exp2(x[r] - m_l) + fast_exp2(x[r + 1] - m_l);
-            } else {
-              l += p_lo(packed, C::kQuant) + p_hi(packed, C::kQuant);  // the weights the MMA uses
-            }
-            w[e] = packed;
+        for (int j = 0; j < 8; ++j) {
+          const int r = 8 * j + 2 * c2;
+          float ya = x[hh][2 * j], yb = x[hh][2 * j + 1];
+          if (C::kRowScale) {  // y = x + log2(s_r): the weight of the stored row carries its scale
+            const float sa = ctl->row_scale[stage][r], sb2 = ctl->row_scale[stage][r + 1];
+            ya = sa > 0.f ? ya + __log2f(sa) : -INFINITY;
+            yb = sb2 > 0.f ? yb + __log2f(sb2) : -INFINITY;
           }
-          *reinterpret_cast<uint4*>(prow + ((c16 ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          const float wa = (m_o[hh] == -INFINITY) ? 0.f : fast_exp2(ya - m_o[hh]);
+          const float wb = (m_o[hh] == -INFINITY) ? 0.f : fast_exp2(yb - m_o[hh]);
+          const uint32_t packed = pack_p(wa, wb, C::kQuant);
+          if (C::kRowScale) {
+            if (m_l[hh] != -INFINITY) l[hh] += fast_exp2(x[hh][2 * j] - m_l[hh]) + fast_exp2(x[hh][2 * j + 1] - m_l[hh]);
+          } else {
+            l[hh] += p_lo(packed, C::kQuant) + p_hi(packed, C::kQuant);  // the weights the MMA uses
+          }
+          // rows 8j .. 8j+7 form 16-byte chunk j of the head's 128-byte row (128-byte swizzle)
+          *reinterpret_cast<uint32_t*>(prow + ((j ^ (h & 7)) << 4)) = packed;
         }
       }
       fence_proxy_async_smem();
@@ -463,102 +535,176 @@ __global__ void __launch_bounds__(Cfg<FMT>::kThreads, 1)
       if (lane == 0) mbar_arrive(&ctl->p_full[sb]);
     }
     if (!dead) dead = !warp_wait(&ctl->o_done, 0, ctl, lane);
-    float* ml = p.ml_part + ((size_t(b) * p.splits + split) * p.heads + h) * 4;
-    if (!dead) {
-      tc_fence_after();
-      float* op = p.o_part + (size_t(b) * p.splits + split) * size_t(p.heads) * kDim;
-#pragma unroll 1
-      for (int ct = 0; ct < kDim / 128; ++ct) {
-        const int c = 128 * ct + 32 * wq + lane;
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          uint32_t o[32];
-          tmem_ld32(tmem + lane_base + kColO + 64 * ct + 32 * half, o);
-          tmem_wait_ld();
+    float l_tot[2];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int hh = 32 * half + e;
-            if (hh < p.heads) op[size_t(hh) * kDim + c] = __uint_as_float(o[e]);
+    for (int hh = 0; hh < 2; ++hh) {
+      l_tot[hh] = l[hh] + __shfl_xor_sync(kFull, l[hh], 1);
+      l_tot[hh] += __shfl_xor_sync(kFull, l_tot[hh], 2);
+    }
+    if (p.splits > 1) {
+      if (!dead) {
+        tc_fence_after();
+        float* op = p.o_part + (size_t(b) * p.splits + split) * size_t(p.heads) * kDim;
+#pragma unroll 1
+        for (int ct = 0; ct < kDim / 128; ++ct) {
+          const int c = 128 * ct + 32 * wq + lane;
+#pragma unroll 1
+          for (int half = 0; half < 2; ++half) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_base + kColO + 64 * ct + 32 * half, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int hh = 32 * half + e;
+              if (hh < p.heads) op[size_t(hh) * kDim + c] = __uint_as_float(o[e]);
+            }
           }
         }
       }
-      if (head_thread && h < p.heads) *reinterpret_cast<float4*>(ml) = make_float4(m_o, m_l, l, 0.f);
-    } else if (head_thread && h < p.heads) {
-      // an empty partial keeps the combine step finite
-      *reinterpret_cast<float4*>(ml) = make_float4(-INFINITY, -INFINITY, 0.f, 0.f);
-    }
-  } else if (C::kQuant) {
-    // ------------------------------------------------------------ converters (warps 6..9)
-    const int cw = warp - 6;
-    const int tid = threadIdx.x - 192;
-    // (1) Q: bf16 -> f16 in place (saturating), once per CTA
-    if (warp_wait(&ctl->q_full, 0, ctl, lane)) {
-      for (int v = tid; v < kQBytes / 16; v += 128) {
-        uint4 x = *reinterpret_cast<const uint4*>(sQ + 16 * v);
-        x = make_uint4(f32x2_to_f16x2_sat(bf16lo(x.x), bf16hi(x.x)), f32x2_to_f16x2_sat(bf16lo(x.y), bf16hi(x.y)),
-                       f32x2_to_f16x2_sat(bf16lo(x.z), bf16hi(x.z)), f32x2_to_f16x2_sat(bf16lo(x.w), bf16hi(x.w)));
-        *reinterpret_cast<uint4*>(sQ + 16 * v) = x;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int h = hd[hh];
+        if (c2 == 0 && h < p.heads) {
+          float* ml = p.ml_part + ((size_t(b) * p.splits + split) * p.heads + h) * 4;
+          *reinterpret_cast<float4*>(ml) = dead ? make_float4(-INFINITY, -INFINITY, 0.f, 0.f)  // empty partial
+                                                : make_float4(m_o[hh], m_l[hh], l_tot[hh], 0.f);
+        }
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->q_ready);
+    } else {
+      // one split: normalise, inverse RoPE, store.  out = O * 2^(m_o - m_l) / l
+      if (c2 == 0) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          ctl->fin[hd[hh]] = (!dead && m_o[hh] != -INFINITY && l_tot[hh] > 0.f)
+                                 ? fast_exp2(m_o[hh] - m_l[hh]) / l_tot[hh] : 0.f;
+      }
+      named_bar_sync();
+      if (!dead) {
+        tc_fence_after();
+        const int r0 = kDim - p.rope_dim;
+#pragma unroll 1
+        for (int ct = 0; ct < kDim / 128; ++ct) {
+          const int c = 128 * ct + 32 * wq + lane;
+          const bool rot = c >= r0;
+          const float cs = rot ? ctl->rope_cs[(c - r0) >> 1] : 1.f;
+          const float sn = rot ? ctl->rope_sn[(c - r0) >> 1] : 0.f;
+#pragma unroll 1
+          for (int half = 0; half < 2; ++half) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_base + kColO + 64 * ct + 32 * half, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int hh = 32 * half + e;
+              float v = __uint_as_float(o[e]) * ctl->fin[hh];
+              const float partner = __shfl_xor_sync(kFull, v, 1);  // channel c ^ 1 of the same head
+              if (rot) v = (c & 1) ? partner * sn + v * cs : v * cs - partner * sn;
+              if (hh < p.heads) {
+                const size_t oi = (size_t(b) * p.heads + hh) * kDim + c;
+                if (p.out_fp32) static_cast<float*>(p.out)[oi] = v;
+                else static_cast<uint16_t*>(p.out)[oi] = f2bf(v);
+              }
+            }
+          }
+        }
+      }
     }
-    // (2) rows: warp cw converts rows 16*cw .. 16*cw+15 of every tile; lane
-    // `lane` owns channels [16*lane, 16*lane+16) = half of a 64-channel chunk.
-    const int chunk = lane >> 2, u0 = (lane & 3) * 2;
+  } else {
+    // ------------------------------------------------------------ loaders (warps 6..9)
+    const int lw = warp - 6;
+    if (C::kQuant) {
+      // Q: bf16 -> f16 in place (saturating), once per CTA
+      if (warp_wait(&ctl->q_full, 0, ctl, lane)) {
+        for (int v = threadIdx.x - 192; v < kQBytes / 16; v += 128) {
+          uint4 x = *reinterpret_cast<const uint4*>(sQ + 16 * v);
+          x = make_uint4(f32x2_to_f16x2_sat(bf16lo(x.x), bf16hi(x.x)), f32x2_to_f16x2_sat(bf16lo(x.y), bf16hi(x.y)),
+                         f32x2_to_f16x2_sat(bf16lo(x.z), bf16hi(x.z)), f32x2_to_f16x2_sat(bf16lo(x.w), bf16hi(x.w)));
+          *reinterpret_cast<uint4*>(sQ + 16 * v) = x;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->q_ready);
+      }
+    }
+    // rows: warp lw covers rows 16*lw .. 16*lw+15 of every tile
     for (int i = 0; i < nt; ++i) {
       const int T = t0 + i, stage = i % kStages;
       if (i >= kStages && !warp_wait(&ctl->empty[stage], ((i / kStages) - 1) & 1, ctl, lane)) break;
-      // lane j < 16 resolves row 16*cw + j, then every lane reads all 16 answers
-      const RowSrc mine = row_source(p, b, T, 16 * cw + (lane & 15));
-      const bool from_win = mine.from_win;  // uniform within a tile
-      const uint8_t* codes = from_win ? p.win_codes : p.comp_codes;
-      const void* scales = from_win ? p.win_scales : p.comp_scales;
-      if (C::kRowScale && lane < 16)
-        ctl->row_scale[stage][16 * cw + lane] = mine.valid ? static_cast<const float*>(scales)[mine.row] : 0.f;
-      uint4 raw[16];
-      uint32_t sgrp[16];
+      uint8_t* tile = sR + stage * kTileBytes;
+      if (!C::kQuant && tile_contiguous(p, T)) {
+        // warp 0 brings this tile by TMA
+      } else {
+        // lane j < 16 resolves row 16*lw + j; every lane reads all 16 answers
+        const RowSrc mine = row_source(p, b, T, 16 * lw + (lane & 15));
+        const uint32_t vb = __ballot_sync(kFull, mine.valid) & 0xffffu;
+        if (lane == 0) ctl->vmask[stage][lw] = vb;
+        if (!C::kQuant) {
+          // gathered bf16 rows: 16-byte cp.async into the 128-byte-swizzled tile
+          const uint8_t* base = static_cast<const uint8_t*>(mine.from_win ? p.win_codes : p.comp_codes);
+#pragma unroll 4
+          for (int j = 0; j < 16; ++j) {
+            const int r = 16 * lw + j;
+            const int64_t row = __shfl_sync(kFull, mine.row, j);
+            const uint8_t* src = base + size_t(row) * (kDim * 2);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int64_t row = __shfl_sync(kFull, mine.row, j);
-        const bool valid = __shfl_sync(kFull, mine.valid, j);
-        if (C::kRowScale) {
-          raw[j] = valid ? ld_stream_v4(codes + size_t(row) * kDim + 16 * lane) : make_uint4(0, 0, 0, 0);
-          sgrp[j] = 0;
+            for (int hh = 0; hh < 2; ++hh) {
+              const int u_all = 32 * hh + lane;  // 16-byte unit of the 1 KB row
+              const int c = u_all >> 3, u = u_all & 7;
+              cp_async16(tile + c * kChunkBytes + r * 128 + ((u ^ (r & 7)) << 4), src + 16 * u_all);
+            }
+          }
+          cp_async_wait_all();
         } else {
-          if (valid) {
-            const uint2 c8 = *reinterpret_cast<const uint2*>(codes + size_t(row) * (kDim / 2) + 8 * lane);
-            raw[j] = make_uint4(c8.x, c8.y, 0, 0);
-            sgrp[j] = static_cast<const uint8_t*>(scales)[size_t(row) * (kDim / 16) + lane];
-          } else {
-            raw[j] = make_uint4(0, 0, 0, 0);
-            sgrp[j] = 0;
+          const uint8_t* codes = mine.from_win ? p.win_codes : p.comp_codes;
+          const void* scales = mine.from_win ? p.win_scales : p.comp_scales;
+          if (C::kRowScale && lane < 16)
+            ctl->row_scale[stage][16 * lw + lane] = mine.valid ? static_cast<const float*>(scales)[mine.row] : 0.f;
+          const int chunk = lane >> 2, u0 = (lane & 3) * 2;  // lane owns channels [16*lane, 16*lane+16)
+          uint4 raw[16];
+          uint32_t sgrp[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int64_t row = __shfl_sync(kFull, mine.row, j);
+            const bool valid = __shfl_sync(kFull, mine.valid, j);
+            if (C::kRowScale) {
+              raw[j] = valid ? ld_stream_v4(codes + size_t(row) * kDim + 16 * lane) : make_uint4(0, 0, 0, 0);
+              sgrp[j] = 0;
+            } else {
+              if (valid) {
+                const uint2 c8 = *reinterpret_cast<const uint2*>(codes + size_t(row) * (kDim / 2) + 8 * lane);
+                raw[j] = make_uint4(c8.x, c8.y, 0, 0);
+                sgrp[j] = static_cast<const uint8_t*>(scales)[size_t(row) * (kDim / 16) + lane];
+              } else {
+                raw[j] = make_uint4(0, 0, 0, 0);
+                sgrp[j] = 0;
+              }
+            }
+          }
+          uint8_t* ctile = tile + chunk * kChunkBytes;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int r = 16 * lw + j;
+            uint32_t hv[8];
+            if (C::kRowScale) {
+              const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                hv[2 * e] = e4m3x2_to_f16x2(w[e] & 0xffffu);
+                hv[2 * e + 1] = e4m3x2_to_f16x2(w[e] >> 16);
+              }
+            } else {
+              const uint32_t s2 = e4m3x2_to_f16x2(sgrp[j] | (sgrp[j] << 8));  // (scale, scale) as f16x2
+              const uint32_t w[2] = {raw[j].x, raw[j].y};
+#pragma unroll
+              for (int e = 0; e < 8; ++e) hv[e] = hmul2(e2m1x2_to_f16x2((w[e >> 2] >> (8 * (e & 3))) & 0xffu), s2);
+            }
+            uint8_t* line = ctile + r * 128;
+            *reinterpret_cast<uint4*>(line + ((u0 ^ (r & 7)) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+            *reinterpret_cast<uint4*>(line + (((u0 + 1) ^ (r & 7)) << 4)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
           }
         }
+        fence_proxy_async_smem();
       }
-      uint8_t* tile = sR + stage * kTileBytes + chunk * kChunkBytes;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int r = 16 * cw + j;
-        uint32_t hv[8];
-        if (C::kRowScale) {
-          const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            hv[2 * e] = e4m3x2_to_f16x2(w[e] & 0xffffu);
-            hv[2 * e + 1] = e4m3x2_to_f16x2(w[e] >> 16);
-          }
-        } else {
-          const uint32_t s2 = e4m3x2_to_f16x2(sgrp[j] | (sgrp[j] << 8));  // (scale, scale) as f16x2
-          const uint32_t w[2] = {raw[j].x, raw[j].y};
-#pragma unroll
-          for (int e = 0; e < 8; ++e) hv[e] = hmul2(e2m1x2_to_f16x2((w[e >> 2] >> (8 * (e & 3))) & 0xffu), s2);
-        }
-        uint8_t* line = tile + r * 128;
-        *reinterpret_cast<uint4*>(line + ((u0 ^ (r & 7)) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-        *reinterpret_cast<uint4*>(line + (((u0 + 1) ^ (r & 7)) << 4)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
-      }
-      fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->full[stage]);
     }
@@ -575,57 +721,92 @@ __global__ void __launch_bounds__(Cfg<FMT>::kThreads, 1)
 // Merge split partials, normalise, inverse RoPE.  Per split: O_s (weights
 // relative to 2^m_o), l_s (relative to 2^m_l):
 //   out = [sum_s O_s 2^(m_o,s - Mo)] / [sum_s l_s 2^(m_l,s - Ml)] * 2^(Mo - Ml).
-__global__ void __launch_bounds__(128) decode_combine(const float* __restrict__ o_part,
-                                                      const float* __restrict__ ml_part, int splits, int heads,
-                                                      int64_t t, int rope_dim, double rope_base, int out_fp32,
-                                                      void* __restrict__ out) {
+// One warp per (sequence, head), four per block.  Lane j owns channels
+// 4j + 128q (q < 4) as float4s, so both channels of a rotary pair sit in one
+// lane; lane s also owns split s's (m, l) terms, which the warp shares by
+// shuffles.  The split loop's loads do not depend on each other.
+constexpr int kCombWarps = 4;
+
+__global__ void __launch_bounds__(32 * kCombWarps) decode_combine(const float* __restrict__ o_part,
+                                                                  const float* __restrict__ ml_part,
+                                                                  const float* __restrict__ rope_tab, int splits,
+                                                                  int heads, int bh_total, int rope_dim, int out_fp32,
+                                                                  void* __restrict__ out) {
   pdl_trigger();
   pdl_wait();
-  const int bh = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x * kCombWarps + warp;
+  if (bh >= bh_total) return;
   const int b = bh / heads, h = bh % heads;
-  const int c = 4 * threadIdx.x;
-  float Mo = -INFINITY, Ml = -INFINITY;
-  for (int s = 0; s < splits; ++s) {
-    const float4 ml = *reinterpret_cast<const float4*>(ml_part + ((size_t(b) * splits + s) * heads + h) * 4);
-    Mo = fmaxf(Mo, ml.x);
-    Ml = fmaxf(Ml, ml.y);
+  const size_t ml_stride = size_t(heads) * 4, o_stride = size_t(heads) * kDim;
+  const float* mlb = ml_part + (size_t(b) * splits * heads + h) * 4;
+  const float* ob = o_part + (size_t(b) * splits * heads + h) * kDim + 4 * lane;
+  float mo = -INFINITY, ml = -INFINITY;
+  for (int s = lane; s < splits; s += 32) {
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(mlb + s * ml_stride));
+    mo = fmaxf(mo, v.x);
+    ml = fmaxf(ml, v.y);
   }
-  float L = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < splits; ++s) {
-    const float4 ml = *reinterpret_cast<const float4*>(ml_part + ((size_t(b) * splits + s) * heads + h) * 4);
-    if (ml.y != -INFINITY) L += ml.z * exp2f(ml.y - Ml);
-    if (ml.x == -INFINITY) continue;
-    const float w = exp2f(ml.x - Mo);
-    const float4 o = *reinterpret_cast<const float4*>(o_part + ((size_t(b) * splits + s) * heads + h) * kDim + c);
-    acc.x += w * o.x;
-    acc.y += w * o.y;
-    acc.z += w * o.z;
-    acc.w += w * o.w;
-  }
-  const float inv = (Mo == -INFINITY) ? 0.f : exp2f(Mo - Ml) / L;
-  float v[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
-  const int r0 = kDim - rope_dim;
-  if (c >= r0) {
 #pragma unroll
-    for (int e = 0; e < 4; e += 2) {
-      const int m = (c + e - r0) >> 1;
-      // angle -t*theta in units of pi, reduced exactly modulo 2 before sincospi
-      const double ang = double(t) * (pow(rope_base, -2.0 * double(m) / double(rope_dim)) / 3.141592653589793);
-      const double xr = ang - 2.0 * rint(0.5 * ang);
-      double sn, cs;
-      sincospi(-xr, &sn, &cs);
-      const float x = v[e], y = v[e + 1];
-      v[e] = float(x * cs - y * sn);
-      v[e + 1] = float(x * sn + y * cs);
+  for (int o = 16; o > 0; o >>= 1) {
+    mo = fmaxf(mo, __shfl_xor_sync(kFull, mo, o));
+    ml = fmaxf(ml, __shfl_xor_sync(kFull, ml, o));
+  }
+  float4 acc[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float L = 0.f;
+  for (int s0 = 0; s0 < splits; s0 += 32) {
+    float w = 0.f;
+    if (s0 + lane < splits) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(mlb + (s0 + lane) * ml_stride));
+      w = v.x == -INFINITY ? 0.f : exp2f(v.x - mo);
+      if (v.y != -INFINITY) L += v.z * exp2f(v.y - ml);
+    }
+    const int cnt = min(32, splits - s0);
+#pragma unroll 4
+    for (int j = 0; j < cnt; ++j) {
+      const float wj = __shfl_sync(kFull, w, j);
+      const float* os = ob + size_t(s0 + j) * o_stride;
+      float4 v[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) v[q] = __ldcg(reinterpret_cast<const float4*>(os + 128 * q));
+      if (wj != 0.f) {  // an empty partial's O is never read
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          acc[q].x = fmaf(wj, v[q].x, acc[q].x);
+          acc[q].y = fmaf(wj, v[q].y, acc[q].y);
+          acc[q].z = fmaf(wj, v[q].z, acc[q].z);
+          acc[q].w = fmaf(wj, v[q].w, acc[q].w);
+        }
+      }
     }
   }
-  const size_t o = (size_t(b) * heads + h) * kDim + c;
-  if (out_fp32) {
-    *reinterpret_cast<float4*>(static_cast<float*>(out) + o) = make_float4(v[0], v[1], v[2], v[3]);
-  } else {
-    *reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + o) =
-        make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(kFull, L, o);
+  const float inv = (mo == -INFINITY || L <= 0.f) ? 0.f : exp2f(mo - ml) / L;
+  const int r0 = kDim - rope_dim;
+  const size_t ob_out = (size_t(b) * heads + h) * kDim;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int c = 128 * q + 4 * lane;
+    float v[4] = {acc[q].x * inv, acc[q].y * inv, acc[q].z * inv, acc[q].w * inv};
+#pragma unroll
+    for (int e = 0; e < 4; e += 2) {
+      if (c + e >= r0) {
+        const int m = (c + e - r0) >> 1;
+        const float cs = __ldcg(rope_tab + m), sn = __ldcg(rope_tab + kDim / 2 + m);
+        const float x = v[e], y = v[e + 1];
+        v[e] = x * cs - y * sn;
+        v[e + 1] = x * sn + y * cs;
+      }
+    }
+    if (out_fp32) {
+      *reinterpret_cast<float4*>(static_cast<float*>(out) + ob_out + c) = make_float4(v[0], v[1], v[2], v[3]);
+    } else {
+      *reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + ob_out + c) =
+          make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+    }
   }
 }
 
@@ -649,6 +830,7 @@ struct DecodeWs {
   uint32_t* status;
   float* o_part;
   float* ml_part;
+  float* rope_tab;
   size_t bytes;
 };
 
@@ -663,6 +845,7 @@ DecodeWs decode_ws_layout(char* base, int batch, int heads, const Plan& pl) {
   w.status = reinterpret_cast<uint32_t*>(take(16));
   w.o_part = reinterpret_cast<float*>(take(sizeof(float) * size_t(batch) * pl.splits * heads * kDim));
   w.ml_part = reinterpret_cast<float*>(take(sizeof(float) * size_t(batch) * pl.splits * heads * 4));
+  w.rope_tab = reinterpret_cast<float*>(take(sizeof(float) * kDim));
   w.bytes = off;
   return w;
 }
@@ -688,7 +871,7 @@ dsv4kv_status launch_fmt(const CUtensorMap& tq, const CUtensorMap& tc, const CUt
       return check_launch("decode: cudaFuncSetAttribute");
     attr_set = true;
   }
-  launch_pdl(decode_kernel<FMT>, dim3(grid), dim3(Cfg<FMT>::kThreads), kSmemBytes, stream, tq, tc, tw, p);
+  launch_pdl(decode_kernel<FMT>, dim3(grid), dim3(kThreads), kSmemBytes, stream, tq, tc, tw, p);
   return check_launch("decode_kernel");
 }
 
@@ -713,19 +896,19 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
     return set_error(DSV4KV_ERR_INVALID_ARG, "decode: cannot encode the query tensor map");
   const dsv4kv_cache& cc = a.comp;
   if (fmt == DSV4KV_BF16) {
-    // row gathers (box: 64 channels x 1 row, 128-byte swizzle)
+    // contiguous row runs: boxes of 64 channels x 64 rows, 128-byte swizzle
     const void* comp_base = cc.codes ? cc.codes : a.win.codes;
     const uint64_t comp_rows_total = std::max<uint64_t>(1, uint64_t(a.batch) * uint64_t(std::max<int64_t>(cc.rows, 1)));
     if (!encode_tmap_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, comp_base, kDim, comp_rows_total, uint64_t(kDim) * 2,
-                        64, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+                        64, kTileRows, CU_TENSOR_MAP_SWIZZLE_128B))
       return set_error(DSV4KV_ERR_INVALID_ARG, "decode: cannot encode the compressed-cache tensor map");
     const void* win_base = a.win.codes ? a.win.codes : comp_base;
     const uint64_t win_rows_total = std::max<uint64_t>(1, uint64_t(a.batch) * uint64_t(std::max<int64_t>(a.win.rows, 1)));
     if (!encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, win_base, kDim, win_rows_total, uint64_t(kDim) * 2, 64,
-                        1, CU_TENSOR_MAP_SWIZZLE_128B))
+                        kTileRows, CU_TENSOR_MAP_SWIZZLE_128B))
       return set_error(DSV4KV_ERR_INVALID_ARG, "decode: cannot encode the window tensor map");
   } else {
-    tc = tq;  // unused: quantised rows are loaded by the converter warps
+    tc = tq;  // unused: quantised rows are loaded by the loader warps
     tw = tq;
   }
 
@@ -748,7 +931,13 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
   p.score_scale = a.sm_scale * 1.4426950408889634f;
   p.o_part = w.o_part;
   p.ml_part = w.ml_part;
+  p.rope_tab = w.rope_tab;
   p.status = w.status;
+  p.t = a.t;
+  p.rope_dim = a.rope_dim;
+  p.rope_base = a.rope_base;
+  p.out_fp32 = a.out_fp32;
+  p.out = a.out;
 
   const int grid = a.batch * pl.splits;
   dsv4kv_status st;
@@ -757,9 +946,11 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
     case DSV4KV_FP8_E4M3_ROW: st = launch_fmt<DSV4KV_FP8_E4M3_ROW>(tq, tc, tw, p, grid, stream); break;
     default: st = launch_fmt<DSV4KV_FP4_E2M1_G16>(tq, tc, tw, p, grid, stream); break;
   }
-  if (st != DSV4KV_OK) return st;
-  launch_pdl(decode_combine, dim3(a.batch * a.heads), dim3(kDim / 4), 0, stream, (const float*)w.o_part,
-             (const float*)w.ml_part, pl.splits, a.heads, a.t, a.rope_dim, a.rope_base, a.out_fp32, a.out);
+  if (st != DSV4KV_OK || pl.splits == 1) return st;  // one split: the decode kernel stored the output
+  const int bh_total = a.batch * a.heads;
+  launch_pdl(decode_combine, dim3((bh_total + kCombWarps - 1) / kCombWarps), dim3(32 * kCombWarps), 0, stream,
+             (const float*)w.o_part, (const float*)w.ml_part, (const float*)w.rope_tab, pl.splits, a.heads, bh_total,
+             a.rope_dim, a.out_fp32, a.out);
   return check_launch("decode_combine");
 }
 

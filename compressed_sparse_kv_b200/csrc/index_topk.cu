@@ -5,21 +5,17 @@
 // cache holds 128 values per entry and may be fp4; [P2] Step 5: the learned
 // indexer scores compressed blocks and the query reads the selected ones.
 //
-// Three launches per call (all on the caller's stream):
+// Two launches per call (both on the caller's stream):
 //  1. index_score_*: streams the keys once (16-byte vector loads, half a warp
 //     per bf16 key / a quarter warp per fp4 key), writes one fp32 score per
 //     entry to the workspace and builds a per-sequence histogram of the top
 //     12 bits of the order-preserving score code.
-//  2. index_filter_select: every CTA finds the threshold bin b1 of its
-//     sequence from that histogram, appends every entry whose bin is >= b1 to
-//     a candidate list, and builds a second-level histogram (next 12 bits) of
-//     the entries in bin b1.  The last CTA of a sequence to finish (atomic
-//     ticket, no waiting) resolves the exact selection from the candidates:
-//     entries above the 24-bit threshold prefix are in; among the entries at
-//     the prefix it orders by (score desc, index asc) and takes what is
-//     missing; it sorts the selection by index, writes it, and re-zeroes the
-//     sequence's histograms and counters.
-//  3. (only when n <= k) index_fill_all writes 0..n-1 directly.
+//  2. index_select: several CTAs per sequence filter the scores against the
+//     threshold bin of that histogram into a candidate list; the last of them
+//     resolves the exact selection from the candidates (second-level
+//     histogram, ranked ties, index-ordered output) and re-zeroes the
+//     sequence's counters.
+//  (only when n <= k) index_fill_all writes 0..n-1 directly.
 // The order (score desc, index asc) is a total order, so the result is the
 // same for every split of the entries (exact, not approximate).
 #include <cstdint>
@@ -211,94 +207,138 @@ __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
   return d;
 }
 
+// fp4 keys, dim 128: 64 B of codes + 8 E4M3 scale bytes per key.  A quarter
+// warp (4 lanes x 16 B) covers one key; lane l4 holds channels
+// [32*l4, 32*l4+32) = two 16-channel scale groups.  Same flattened, evenly
+// split, double-buffered structure as the bf16 kernel; each warp iteration
+// covers 32 keys (U = 4 per quad).  Each code byte is decoded to a packed f16
+// pair with cvt.rn.f16x2.e2m1x2 and accumulated with packed f16 FMAs per
+// group (exact for integer queries: |partial| <= 8*8*6 per half at a
+// resolution of 0.5), then scaled by the group's E4M3 scale in fp32.
 __global__ void __launch_bounds__(256) index_score_fp4(const uint16_t* __restrict__ qidx,
                                                        const uint8_t* __restrict__ codes,
                                                        const uint8_t* __restrict__ scales, int64_t key_rows,
-                                                       int64_t n, int64_t chunk, float* __restrict__ scores,
-                                                       uint32_t* __restrict__ hist) {
+                                                       int64_t n, int batch, int64_t per_cta,
+                                                       float* __restrict__ scores, uint32_t* __restrict__ hist) {
+  constexpr int U = 4;
   __shared__ uint32_t sh[kHistBins];
   pdl_trigger();
-  const int b = blockIdx.y;
-  const int64_t n0 = int64_t(blockIdx.x) * chunk;
-  const int64_t n1 = min(n, n0 + chunk);
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0;
+  const int64_t total = int64_t(batch) * n;
+  const int64_t g0 = int64_t(blockIdx.x) * per_cta;
+  const int64_t g1 = min(total, g0 + per_cta);
+  if (g0 >= g1) return;
   pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int quad = lane >> 2, l4 = lane & 3;  // key slot in the warp, segment in the key
-  // Lane l4 covers channels [32*l4, 32*l4+32).  Word j of its 16 B holds
-  // channels 32*l4 + 8j .. +8 (nibble e = channel 8j+e); the decode pairs
-  // nibbles (i, i+4), so q is packed the same way: qp[j][i] = (q[8j+i], q[8j+i+4]).
-  uint32_t qp[4][4];
-  {
-    const uint16_t* qb = qidx + size_t(b) * 128 + 32 * l4;
+  const int quad = lane >> 2, l4 = lane & 3;
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0;
+  for (int64_t s0 = g0; s0 < g1;) {
+    const int b = int(s0 / n);
+    const int64_t s1 = min(g1, int64_t(b + 1) * n);
+    const int64_t i0 = s0 - int64_t(b) * n, cnt = s1 - s0;
+    uint32_t qp[16];  // (q[2j], q[2j+1]) as f16x2 for this lane's 32 channels
+    {
+      const uint16_t* qb = qidx + size_t(b) * 128 + 32 * l4;
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) qp[j][i] = f32x2_to_f16x2(bf16f(qb[8 * j + i]), bf16f(qb[8 * j + i + 4]));
-  }
-  __syncthreads();
-  const uint8_t* cb = codes + size_t(b) * size_t(key_rows) * 64 + 16 * l4;
-  const uint8_t* sb = scales + size_t(b) * size_t(key_rows) * 8 + 2 * l4;
-  float* sc = scores + size_t(b) * size_t(n);
-  constexpr int U = 4;  // keys per quad per iteration (32 keys per warp)
-  for (int64_t base = n0 + 32 * warp; base < n1; base += 32 * nwarps) {
-    uint4 v[U];
-    uint32_t s2[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t key = base + 8 * u + quad;
-      const bool ok = key < n1;
-      v[u] = ok ? ld_stream_v4(cb + key * 64) : make_uint4(0, 0, 0, 0);
-      s2[u] = ok ? *reinterpret_cast<const uint16_t*>(sb + key * 8) : 0u;
+      for (int j = 0; j < 16; ++j) qp[j] = f32x2_to_f16x2(bf16f(qb[2 * j]), bf16f(qb[2 * j + 1]));
     }
-    float p[U];
+    __syncthreads();  // histogram cleared
+    const uint8_t* cb = codes + (size_t(b) * size_t(key_rows) + size_t(i0)) * 64 + 16 * l4;
+    const uint8_t* sb = scales + (size_t(b) * size_t(key_rows) + size_t(i0)) * 8 + 2 * l4;
+    float* sc = scores + size_t(b) * size_t(n) + size_t(i0);
+    auto load = [&](int64_t j, uint4 (&v)[U], uint32_t (&s2)[U]) {
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-      uint32_t acc0 = 0, acc1 = 0;  // f16x2 accumulators of group 0 (words 0,1) and group 1 (words 2,3)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t h[4];
-        e2m1x8_to_f16x2(w[j], h);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          if (j < 2) acc0 = hfma2(qp[j][i], h[i], acc0);
-          else acc1 = hfma2(qp[j][i], h[i], acc1);
-        }
+      for (int u = 0; u < U; ++u) {
+        const int64_t key = 8 * U * j + 8 * u + quad;
+        const bool ok = key < cnt;
+        v[u] = ok ? ld_stream_v4(cb + key * 64) : make_uint4(0, 0, 0, 0);
+        s2[u] = ok ? *reinterpret_cast<const uint16_t*>(sb + key * 8) : 0u;
       }
-      p[u] = f16x2_sum(acc0) * e4m3_to_f32(s2[u] & 0xffu) + f16x2_sum(acc1) * e4m3_to_f32(s2[u] >> 8);
-    }
-    // reduce over the 4 lanes of the quad: 4 values -> transposing butterfly
-    const bool bb1 = l4 & 2, bb0 = l4 & 1;
-    float k2[2];
+    };
+    auto process = [&](int64_t j, const uint4 (&v)[U], const uint32_t (&s2)[U]) {
+      float p[U];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const float keep = bb1 ? p[2 + i] : p[i];
-      const float send = bb1 ? p[i] : p[2 + i];
-      k2[i] = keep + __shfl_xor_sync(kFull, send, 2);
+      for (int u = 0; u < U; ++u) {
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        uint32_t acc0 = 0, acc1 = 0;  // f16x2 sums of group 0 (words 0, 1) and group 1 (words 2, 3)
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+#pragma unroll
+          for (int by = 0; by < 4; ++by) {
+            const uint32_t h = e2m1x2_to_f16x2((w[wi] >> (8 * by)) & 0xffu);
+            if (wi < 2) acc0 = hfma2(qp[4 * wi + by], h, acc0);
+            else acc1 = hfma2(qp[4 * wi + by], h, acc1);
+          }
+        }
+        p[u] = f16x2_sum(acc0) * e4m3_to_f32(s2[u] & 0xffu) + f16x2_sum(acc1) * e4m3_to_f32(s2[u] >> 8);
+      }
+      // reduce over the 4 lanes of the quad: 4 values -> transposing butterfly
+      const bool bb1 = l4 & 2, bb0 = l4 & 1;
+      float k2[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) k2[i] = (bb1 ? p[2 + i] : p[i]) + __shfl_xor_sync(kFull, bb1 ? p[i] : p[2 + i], 2);
+      const float s = (bb0 ? k2[1] : k2[0]) + __shfl_xor_sync(kFull, bb0 ? k2[0] : k2[1], 1) + 0.0f;
+      const int64_t key = 8 * U * j + 8 * l4 + quad;  // lane l4 ends with key u = l4
+      if (key < cnt) {
+        sc[key] = s;
+        atomicAdd(&sh[ord_f32(s) >> 20], 1u);
+      }
+    };
+    const int64_t ngroups = (cnt + 8 * U - 1) / (8 * U);
+    uint4 va[U], vb[U];
+    uint32_t sa[U], sb2[U];
+    int64_t j = warp;
+    if (j < ngroups) load(j, va, sa);
+    while (j < ngroups) {
+      if (j + nwarps < ngroups) load(j + nwarps, vb, sb2);
+      process(j, va, sa);
+      j += nwarps;
+      if (j >= ngroups) break;
+      if (j + nwarps < ngroups) load(j + nwarps, va, sa);
+      process(j, vb, sb2);
+      j += nwarps;
     }
-    const float s = (bb0 ? k2[1] : k2[0]) + __shfl_xor_sync(kFull, bb0 ? k2[0] : k2[1], 1);
-    const int64_t key = base + 8 * (2 * (l4 >> 1) + (l4 & 1)) + quad;
-    if (key < n1) {
-      const float sz = s + 0.0f;
-      sc[key] = sz;
-      atomicAdd(&sh[ord_f32(sz) >> 20], 1u);
+    __syncthreads();
+    uint32_t* hb = hist + size_t(b) * kHistBins;
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
+      const uint32_t c = sh[i];
+      if (c) {
+        atomicAdd(&hb[i], c);
+        sh[i] = 0;
+      }
     }
+    s0 = s1;
   }
-  __syncthreads();
-  uint32_t* hb = hist + size_t(b) * kHistBins;
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
-    if (sh[i]) atomicAdd(&hb[i], sh[i]);
 }
 
-// ------------------------------------------------------------------ selection helpers
+// ------------------------------------------------------------------ selection
+// index_select runs one thread-block cluster of C CTAs per sequence (grid
+// C x B).  Every CTA finds the threshold bin b1 of its sequence in the score
+// kernel's histogram and filters its chunk of scores (the loads of a batch in
+// flight before any is inspected) into a shared-memory list of candidates
+// (top-12-bit bin >= b1), kept in index order.  After a cluster barrier the
+// leader CTA reads every CTA's list through distributed shared memory, in
+// chunk order, so the candidates arrive sorted by index; the other CTAs wait
+// at a second barrier until it has, then exit.  The leader resolves the exact
+// selection from the candidates alone: the second-level histogram of the
+// entries in b1 gives the 24-bit threshold prefix; entries above it are in;
+// the entries at it are ranked by (score desc, index asc) and the best fill
+// what is missing; an ordered compaction writes the result in ascending index
+// order.  It re-zeroes the sequence's histogram for the next call.
 constexpr int kSelThreads = 512;
+constexpr int kSelBatch = 8;                           // scores per thread and batch
+constexpr int kSelBatchSpan = kSelThreads * kSelBatch;  // 4096 scores per CTA batch
+constexpr int kSelStage = 4096;                        // candidates a CTA can hold
+constexpr int kCandCap = 8192;                         // candidates per sequence the leader can resolve
+constexpr int kResPer = kCandCap / kSelThreads;        // candidates per leader thread
 constexpr int kTieCap = 2048;
-constexpr int64_t kMaxBitmapN = 262144;  // entries covered by the shared-memory bitmaps (8192 words each)
+constexpr int kMaxClusterSel = 16;
+constexpr size_t kSelDyn = size_t(kSelStage) * sizeof(uint64_t);
+static_assert(kTieCap * (sizeof(uint64_t) + sizeof(uint32_t)) <= kSelDyn, "the tie list reuses the list area");
 
-// Block-wide exclusive prefix sum of one value per thread (kSelThreads threads).
+// Block-wide exclusive prefix sum of one value per thread (NT threads).
+template <int NT>
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* total) {
-  __shared__ uint32_t wsum[kSelThreads / 32];
+  __shared__ uint32_t wsum[NT / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t incl = v;
 #pragma unroll
@@ -310,7 +350,7 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* t
   __syncthreads();
   uint32_t base = 0, all = 0;
 #pragma unroll
-  for (int w = 0; w < kSelThreads / 32; ++w) {
+  for (int w = 0; w < NT / 32; ++w) {
     const uint32_t x = wsum[w];
     base += w < warp ? x : 0u;
     all += x;
@@ -320,30 +360,57 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* t
   return base + incl - v;
 }
 
+__device__ __forceinline__ uint32_t warp_inclusive_scan(uint32_t v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(kFull, v, o);
+    if (lane >= o) v += y;
+  }
+  return v;
+}
+
 // The bin where the descending cumulative count of the 4096-bin histogram h
 // (shared memory) first reaches `need` (1 <= need <= sum h); *above = count in
-// higher bins.  Thread t owns bins 4095-8t .. 4088-8t.
+// higher bins.  Warp w owns the bins [4096 - S(w+1), 4096 - Sw), S = 4096/warps,
+// and its lanes read consecutive bins from the top (no bank conflicts); the
+// warp that holds the crossing walks its bins 32 at a time with warp scans.
+template <int NT>
 __device__ int find_threshold_bin(const uint32_t* h, uint32_t need, uint32_t* above) {
-  static_assert(kSelThreads * 8 == kHistBins, "8 bins per thread");
+  constexpr int NW = NT / 32, SPAN = kHistBins / NW, STEPS = SPAN / 32;
+  static_assert(STEPS * 32 * NW == kHistBins, "bins per warp");
+  __shared__ uint32_t s_wtot[NW];
   __shared__ int s_bin;
   __shared__ uint32_t s_above;
-  const int top = kHistBins - 1 - 8 * int(threadIdx.x);
-  uint32_t v[8], local = 0;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int top = kHistBins - 1 - SPAN * warp;
+  uint32_t v[STEPS], sum = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    v[i] = h[top - i];
-    local += v[i];
+  for (int j = 0; j < STEPS; ++j) {
+    v[j] = h[top - 32 * j - lane];
+    sum += v[j];
   }
-  const uint32_t excl = block_exclusive_scan(local, nullptr);
-  if (excl < need && excl + local >= need) {
-    uint32_t c = excl;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (c < need && c + v[i] >= need) {
-        s_bin = top - i;
-        s_above = c;
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
+  if (lane == 0) s_wtot[warp] = sum;
+  __syncthreads();
+  uint32_t before = 0;
+  for (int w = 0; w < warp; ++w) before += s_wtot[w];
+  if (before < need && before + sum >= need) {  // this warp holds the crossing (warp-uniform)
+    uint32_t c = before;
+#pragma unroll
+    for (int j = 0; j < STEPS; ++j) {
+      const uint32_t incl = warp_inclusive_scan(v[j]);
+      const uint32_t tot = __shfl_sync(kFull, incl, 31);
+      if (c + tot >= need) {
+        const uint32_t ex = c + incl - v[j];
+        if (ex < need && ex + v[j] >= need) {  // exactly one lane
+          s_bin = top - 32 * j - lane;
+          s_above = ex;
+        }
+        break;
       }
-      c += v[i];
+      c += tot;
     }
   }
   __syncthreads();
@@ -353,249 +420,302 @@ __device__ int find_threshold_bin(const uint32_t* h, uint32_t need, uint32_t* ab
   return r;
 }
 
-template <typename T, bool ASC>
-__device__ void bitonic_sort_smem(T* a, int n_pow2) {
-  for (int size = 2; size <= n_pow2; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < n_pow2; i += blockDim.x) {
-        const int j = i ^ stride;
-        if (j > i) {
-          const bool up = ((i & size) == 0) == ASC;
-          const T x = a[i], y = a[j];
-          if ((x > y) == up) {
-            a[i] = y;
-            a[j] = x;
-          }
-        }
-      }
-      __syncthreads();
-    }
+// Ordered compaction offsets for BATCH elements per thread at positions
+// (j, warp, lane) in that lexicographic order: m[j] is the warp's ballot of
+// the predicate for element j; off[j] receives the number of true elements
+// before lane 0 of (j, warp).  Returns the total.  Block-wide (syncs).
+template <int NT, int BATCH>
+__device__ uint32_t ordered_offsets(const uint32_t (&m)[BATCH], uint32_t (&off)[BATCH]) {
+  constexpr int NW = NT / 32, E = BATCH * NW, PER = E / 32;
+  static_assert(PER * 32 == E, "entries per lane");
+  __shared__ uint32_t s_c[E];
+  __shared__ uint32_t s_total;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) {
+#pragma unroll
+    for (int j = 0; j < BATCH; ++j) s_c[j * NW + warp] = __popc(m[j]);
   }
-}
-
-// Ordered walk of a bitmap of `words` words: calls emit(index, rank) for
-// every set bit in ascending index order (rank = 0, 1, ...).  Returns the count.
-template <typename F>
-__device__ uint32_t bitmap_ordered_walk(const uint32_t* bm, int words, F emit) {
-  const int per = (words + kSelThreads - 1) / kSelThreads;
-  const int w0 = min(words, int(threadIdx.x) * per), w1 = min(words, w0 + per);
-  uint32_t local = 0;
-  for (int w = w0; w < w1; ++w) local += __popc(bm[w]);
-  uint32_t total;
-  uint32_t rank = block_exclusive_scan(local, &total);
-  for (int w = w0; w < w1; ++w) {
-    uint32_t x = bm[w];
-    while (x) {
-      const int bit = __ffs(x) - 1;
-      x &= x - 1;
-      emit(uint32_t(w) * 32u + uint32_t(bit), rank++);
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t x[PER], loc = 0;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      x[q] = s_c[PER * lane + q];
+      loc += x[q];
     }
+    const uint32_t incl = warp_inclusive_scan(loc);
+    uint32_t run = incl - loc;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      s_c[PER * lane + q] = run;
+      run += x[q];
+    }
+    if (lane == 31) s_total = incl;
   }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < BATCH; ++j) off[j] = s_c[j * NW + warp];
+  const uint32_t total = s_total;
+  __syncthreads();  // s_c is rewritten by the next call
   return total;
 }
 
-// ------------------------------------------------------------------ filter + select
-// Dynamic shared memory: two bitmaps of ceil(n/32) words when n <= kMaxBitmapN.
-__global__ void __launch_bounds__(kSelThreads) index_filter_select(
-    const float* __restrict__ scores, int64_t n, int k, int64_t chunk, uint32_t* __restrict__ hist,
-    uint32_t* __restrict__ hist2, uint32_t* __restrict__ done, uint32_t* __restrict__ cand_count,
-    uint64_t* __restrict__ cand, int64_t cap, int32_t* __restrict__ idx_out, int32_t* __restrict__ count_out,
-    uint32_t* __restrict__ status) {
-  extern __shared__ uint32_t dyn_bm[];
+template <int NT, int BATCH>
+__device__ __forceinline__ void load_codes(const float* __restrict__ sc, int64_t base, int64_t end,
+                                           uint32_t (&o)[BATCH]) {
+#pragma unroll
+  for (int j = 0; j < BATCH; ++j) {
+    const int64_t i = base + int64_t(j) * NT + threadIdx.x;
+    o[j] = i < end ? ord_f32(__ldcg(sc + i)) : 0u;
+  }
+}
+
+// Appends, in index order, the batch's entries whose top-12-bit bin is
+// >= bin1 to the CTA's list (u64 = code << 32 | ~index) after `count`
+// entries; returns the new count (entries beyond kSelStage are counted, not
+// stored).
+__device__ __forceinline__ uint32_t stage_batch(const uint32_t (&o)[kSelBatch], int64_t base, int64_t end, int bin1,
+                                                uint32_t count, uint64_t* list) {
+  const int lane = threadIdx.x & 31;
+  uint32_t m[kSelBatch], off[kSelBatch];
+#pragma unroll
+  for (int j = 0; j < kSelBatch; ++j) {
+    const int64_t i = base + int64_t(j) * kSelThreads + threadIdx.x;
+    m[j] = __ballot_sync(kFull, i < end && int(o[j] >> 20) >= bin1);
+  }
+  const uint32_t total = ordered_offsets<kSelThreads, kSelBatch>(m, off);
+  const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int j = 0; j < kSelBatch; ++j) {
+    if ((m[j] >> lane) & 1u) {
+      const uint32_t at = count + off[j] + __popc(m[j] & lt);
+      const int64_t i = base + int64_t(j) * kSelThreads + threadIdx.x;
+      if (at < uint32_t(kSelStage)) list[at] = (uint64_t(o[j]) << 32) | uint64_t(0xffffffffu - uint32_t(i));
+    }
+  }
+  return count + total;
+}
+
+// Exact selection with no candidate list (overflow, or more than kTieCap
+// entries at the prefix): the threshold code o* from the low 8 bits of the
+// entries at the 24-bit prefix, then one ordered scan of all scores keeps
+// codes > o* and the first r codes == o* (the lowest indices), in index order.
+template <int NT>
+__device__ void select_by_scan(const float* __restrict__ sc, int64_t n, uint32_t prefix, uint32_t need_tie,
+                               uint32_t kk, int32_t* __restrict__ ob, uint32_t* sh256, uint32_t* status) {
+  __shared__ uint32_t s_low, s_above3, s_gt_seen, s_eq_seen;
+  for (int i = threadIdx.x; i < 256; i += NT) sh256[i] = 0;
+  __syncthreads();
+  for (int64_t i = threadIdx.x; i < n; i += NT) {
+    const uint32_t o = ord_f32(sc[i]);
+    if ((o >> 8) == prefix) atomicAdd(&sh256[o & 0xffu], 1u);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t c = 0;
+    for (int v = 255; v >= 0; --v) {
+      if (c + sh256[v] >= need_tie) {
+        s_low = uint32_t(v);
+        s_above3 = c;
+        break;
+      }
+      c += sh256[v];
+    }
+    s_gt_seen = 0;
+    s_eq_seen = 0;
+  }
+  __syncthreads();
+  const uint32_t ostar = (prefix << 8) | s_low;
+  const uint32_t r_eq = need_tie - s_above3;  // entries equal to o* to keep
+  for (int64_t base = 0; base < n; base += NT) {
+    const int64_t i = base + threadIdx.x;
+    const uint32_t o = i < n ? ord_f32(sc[i]) : 0u;
+    const bool gt = i < n && o > ostar;
+    const bool eq = i < n && o == ostar;
+    uint32_t ngt, neq;
+    const uint32_t gt_before = s_gt_seen + block_exclusive_scan<NT>(gt ? 1u : 0u, &ngt);
+    const uint32_t eq_before = s_eq_seen + block_exclusive_scan<NT>(eq ? 1u : 0u, &neq);
+    // index order is preserved: kept entries before this one = gt_before + min(eq_before, r_eq)
+    const uint32_t pos = gt_before + min(eq_before, r_eq);
+    if ((gt || (eq && eq_before < r_eq)) && pos < kk) ob[pos] = int32_t(i);
+    if (threadIdx.x == 0) {
+      s_gt_seen += ngt;
+      s_eq_seen += neq;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0 && s_gt_seen + min(s_eq_seen, r_eq) != kk) set_status(status, DSV4KV_DEV_INCONSISTENT);
+}
+
+__global__ void __launch_bounds__(kSelThreads) index_select(const float* __restrict__ scores, int64_t n, int k,
+                                                            int64_t chunk, uint32_t* __restrict__ hist,
+                                                            int32_t* __restrict__ idx_out,
+                                                            int32_t* __restrict__ count_out,
+                                                            uint32_t* __restrict__ status) {
+  extern __shared__ __align__(16) uint64_t stage[];  // kSelStage: this CTA's candidates, in index order
   __shared__ uint32_t sh[kHistBins];
-  __shared__ int s_last;
-  __shared__ uint32_t s_ntie, s_tie_min, s_tie_max, s_taken;
-  __shared__ int32_t sel[2048];
-  __shared__ uint64_t ties[kTieCap];
+  __shared__ uint32_t s_count, s_ntie;
+  __shared__ uint32_t s_keep[kCandCap / 32];  // tie verdicts by candidate position
+  __shared__ uint32_t s_pre[kMaxClusterSel + 1];
 
   const int b = blockIdx.y;
+  const uint32_t rank = cluster_rank();
+  const uint32_t csize = gridDim.x;  // one cluster spans the sequence's CTAs
   const uint32_t kk = uint32_t(int64_t(k) < n ? int64_t(k) : n);
   uint32_t* hb = hist + size_t(b) * kHistBins;
-  uint32_t* h2 = hist2 + size_t(b) * kHistBins;
   const float* sc = scores + size_t(b) * size_t(n);
-  uint64_t* cb = cand + size_t(b) * size_t(cap);
+  const int64_t n0 = int64_t(rank) * chunk, n1 = min(n, n0 + chunk);
   const int lane = threadIdx.x & 31;
   pdl_trigger();
   pdl_wait();
 
-  // 1) threshold bin of the top-12-bit histogram
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = hb[i];
+  // 1) the first batch of scores is in flight while the histogram is read
+  uint32_t oa[kSelBatch], ob2[kSelBatch];
+  load_codes<kSelThreads, kSelBatch>(sc, n0, n1, oa);
+  for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) sh[i] = __ldcg(hb + i);
   __syncthreads();
   uint32_t above1;
-  const int bin1 = find_threshold_bin(sh, kk, &above1);
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0;
-  __syncthreads();
+  const int bin1 = find_threshold_bin<kSelThreads>(sh, kk, &above1);
 
-  // 2) filter this CTA's chunk: candidates (bin >= bin1) and the next-12-bit
-  //    histogram of the entries in bin1
-  const int64_t n0 = int64_t(blockIdx.x) * chunk;
-  const int64_t n1 = min(n, n0 + chunk);
-  for (int64_t base = n0; base < n1; base += blockDim.x) {
-    const int64_t i = base + threadIdx.x;
-    uint32_t o = 0;
-    bool take = false;
-    if (i < n1) {
-      o = ord_f32(sc[i]);
-      const int bin = int(o >> 20);
-      take = bin >= bin1;
-      if (bin == bin1) atomicAdd(&sh[(o >> 8) & 0xfffu], 1u);
+  // 2) this CTA's candidates, in index order; batches double-buffered
+  uint32_t count = 0;
+  for (int64_t base = n0; base < n1; base += 2 * kSelBatchSpan) {
+    if (base + kSelBatchSpan < n1) load_codes<kSelThreads, kSelBatch>(sc, base + kSelBatchSpan, n1, ob2);
+    count = stage_batch(oa, base, n1, bin1, count, stage);
+    if (base + kSelBatchSpan >= n1) break;
+    if (base + 2 * kSelBatchSpan < n1) load_codes<kSelThreads, kSelBatch>(sc, base + 2 * kSelBatchSpan, n1, oa);
+    count = stage_batch(ob2, base + kSelBatchSpan, n1, bin1, count, stage);
+  }
+  if (threadIdx.x == 0) s_count = count;
+  cluster_sync();  // every list of the cluster is complete
+
+  // 3) the leader gathers the lists in chunk order (= index order)
+  uint64_t c[kResPer];
+  uint32_t total = 0;
+  bool fits = true;
+  if (rank == 0) {
+    if (threadIdx.x == 0) {
+      uint32_t run = 0;
+      for (uint32_t r = 0; r < csize; ++r) {
+        s_pre[r] = run;
+        const uint32_t cnt = ld_dsmem_u32(dsmem_addr(&s_count, r));
+        if (cnt > uint32_t(kSelStage)) fits = false;
+        run += cnt;
+      }
+      s_pre[csize] = fits ? run : 0xffffffffu;
     }
-    const uint32_t m = __ballot_sync(kFull, take);
-    if (m) {
-      uint32_t pos0 = 0;
-      if (lane == __ffs(m) - 1) pos0 = atomicAdd(&cand_count[b], uint32_t(__popc(m)));
-      pos0 = __shfl_sync(kFull, pos0, __ffs(m) - 1);
-      if (take) {
-        const uint64_t pos = uint64_t(pos0) + __popc(m & ((1u << lane) - 1u));
-        if (pos < uint64_t(cap)) cb[pos] = (uint64_t(o) << 32) | uint64_t(0xffffffffu - uint32_t(i));
+    __syncthreads();
+    total = s_pre[csize];
+    fits = total <= uint32_t(kCandCap);
+    if (fits) {
+#pragma unroll
+      for (int j = 0; j < kResPer; ++j) {
+        const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
+        c[j] = 0ull;
+        if (g < total) {
+          uint32_t r = 0;
+          while (r + 1 < csize && s_pre[r + 1] <= g) ++r;
+          c[j] = ld_dsmem_u64(dsmem_addr(&stage[g - s_pre[r]], r));
+        }
       }
     }
   }
-  __syncthreads();
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
-    if (sh[i]) atomicAdd(&h2[i], sh[i]);
+  cluster_sync();  // the other CTAs' lists are no longer read
+  if (rank != 0) return;
 
-  // 3) ticket: the last CTA of this sequence resolves the selection
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) s_last = (atomicAdd(&done[b], 1u) == gridDim.x - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = __ldcg(&h2[i]);
-  if (threadIdx.x == 0) {
-    s_ntie = 0;
-    s_tie_min = 0xffffffffu;
-    s_tie_max = 0;
-    s_taken = 0;
-  }
-  __syncthreads();
-  uint32_t above2;
+  // 4) resolve
+  int32_t* out = idx_out + size_t(b) * k;
   const uint32_t need1 = kk - above1;  // still needed from bin1 (>= 1)
-  const int bin2 = find_threshold_bin(sh, need1, &above2);
-  const uint32_t prefix = (uint32_t(bin1) << 12) | uint32_t(bin2);  // 24-bit threshold prefix
-  const uint32_t need_tie = need1 - above2;                           // >= 1
-  const uint32_t total = __ldcg(&cand_count[b]);
-  int32_t* ob = idx_out + size_t(b) * k;
-
-  bool done_out = false;
-  if (total <= uint64_t(cap) && n <= kMaxBitmapN) {
-    // bitmap path: entries above the prefix into `selbm`, entries at the prefix into `tiebm`
-    const int words = int((n + 31) / 32);
-    uint32_t* selbm = dyn_bm;
-    uint32_t* tiebm = dyn_bm + words;
-    for (int w = threadIdx.x; w < 2 * words; w += blockDim.x) dyn_bm[w] = 0;
+  uint64_t* ties = stage;              // the leader's list is in registers now
+  bool ok = false;
+  uint32_t prefix = 0, need_tie = 0;
+  for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) sh[i] = 0;
+  for (int i = threadIdx.x; i < kCandCap / 32; i += kSelThreads) s_keep[i] = 0;
+  if (threadIdx.x == 0) s_ntie = 0;
+  __syncthreads();
+  if (fits) {
+    // second-level histogram of bin1 (every entry of bin1 is a candidate)
+#pragma unroll
+    for (int j = 0; j < kResPer; ++j) {
+      const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
+      const uint32_t o = uint32_t(c[j] >> 32);
+      if (g < total && int(o >> 20) == bin1) atomicAdd(&sh[(o >> 8) & 0xfffu], 1u);
+    }
     __syncthreads();
-    for (uint32_t c = threadIdx.x; c < total; c += blockDim.x) {
-      const uint64_t key = __ldcg(&cb[c]);
-      const uint32_t o = uint32_t(key >> 32), i = 0xffffffffu - uint32_t(key);
-      const uint32_t pre = o >> 8;
-      if (pre > prefix) {
-        atomicOr(&selbm[i >> 5], 1u << (i & 31));
-      } else if (pre == prefix) {
-        atomicOr(&tiebm[i >> 5], 1u << (i & 31));
-        atomicMin(&s_tie_min, o);
-        atomicMax(&s_tie_max, o);
+    uint32_t above2;
+    const int bin2 = find_threshold_bin<kSelThreads>(sh, need1, &above2);
+    prefix = (uint32_t(bin1) << 12) | uint32_t(bin2);  // 24-bit threshold prefix
+    need_tie = need1 - above2;                          // >= 1
+    // the entries at the prefix: (key, position) into the tie list
+#pragma unroll
+    for (int j = 0; j < kResPer; ++j) {
+      const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
+      if (g < total && uint32_t(c[j] >> 40) == prefix) {
         const uint32_t slot = atomicAdd(&s_ntie, 1u);
-        if (slot < kTieCap) ties[slot] = key;
+        if (slot < uint32_t(kTieCap)) {
+          ties[slot] = c[j];
+          reinterpret_cast<uint32_t*>(ties + kTieCap)[slot] = g;
+        }
       }
     }
     __syncthreads();
     const uint32_t n_tie = s_ntie;
-    bool ties_ok = true;
-    if (s_tie_min == s_tie_max) {
-      // every entry at the prefix has the same score: the lowest indices win
-      bitmap_ordered_walk(tiebm, words, [&](uint32_t i, uint32_t rank) {
-        if (rank < need_tie) atomicOr(&selbm[i >> 5], 1u << (i & 31));
-      });
-    } else if (n_tie <= uint32_t(kTieCap)) {
-      // distinct scores share the prefix: order those entries by (score desc, index asc)
-      int np2 = 1;
-      while (np2 < int(n_tie)) np2 <<= 1;
-      for (int i = int(n_tie) + threadIdx.x; i < np2; i += blockDim.x) ties[i] = 0;
-      __syncthreads();
-      bitonic_sort_smem<uint64_t, false>(ties, np2);
-      for (uint32_t t = threadIdx.x; t < need_tie; t += blockDim.x) {
-        const uint32_t i = 0xffffffffu - uint32_t(ties[t]);
-        atomicOr(&selbm[i >> 5], 1u << (i & 31));
-      }
-    } else {
-      ties_ok = false;
-    }
-    __syncthreads();
-    if (ties_ok) {
-      const uint32_t got = bitmap_ordered_walk(selbm, words, [&](uint32_t i, uint32_t rank) {
-        if (rank < kk) ob[rank] = int32_t(i);
-      });
-      if (threadIdx.x == 0 && got != kk) set_status(status, DSV4KV_DEV_INCONSISTENT);
-      done_out = true;
-    }
-  }
-  if (!done_out) {
-    // General path (huge n, candidate overflow or massive heterogeneous ties):
-    // exact threshold code o* from the low 8 bits of the entries at the
-    // prefix, then one ordered scan over all scores keeps codes > o* and the
-    // first r codes == o* (lowest indices).
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) sh[i] = 0;
-    __syncthreads();
-    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
-      const uint32_t o = ord_f32(sc[i]);
-      if ((o >> 8) == prefix) atomicAdd(&sh[o & 0xffu], 1u);
-    }
-    __syncthreads();
-    __shared__ uint32_t s_low, s_above3;
-    if (threadIdx.x == 0) {
-      uint32_t c = 0;
-      for (int v = 255; v >= 0; --v) {
-        if (c + sh[v] >= need_tie) {
-          s_low = uint32_t(v);
-          s_above3 = c;
-          break;
+    if (n_tie <= uint32_t(kTieCap)) {
+      ok = true;
+      // a tie is kept when fewer than need_tie keys (score desc, index asc) exceed its own
+      for (uint32_t t = threadIdx.x; t < n_tie; t += kSelThreads) {
+        const uint64_t key = ties[t];
+        uint32_t r = 0;
+        for (uint32_t u = 0; u < n_tie; ++u) r += ties[u] > key ? 1u : 0u;
+        if (r < need_tie) {
+          const uint32_t g = reinterpret_cast<const uint32_t*>(ties + kTieCap)[t];
+          atomicOr(&s_keep[g >> 5], 1u << (g & 31));
         }
-        c += sh[v];
-      }
-    }
-    __syncthreads();
-    const uint32_t ostar = (prefix << 8) | s_low;
-    const uint32_t r_eq = need_tie - s_above3;  // entries equal to o* to keep
-    __shared__ uint32_t s_gt_seen, s_eq_seen;
-    if (threadIdx.x == 0) {
-      s_gt_seen = 0;
-      s_eq_seen = 0;
-    }
-    __syncthreads();
-    for (int64_t base = 0; base < n; base += blockDim.x) {
-      const int64_t i = base + threadIdx.x;
-      const uint32_t o = i < n ? ord_f32(sc[i]) : 0u;
-      const bool gt = i < n && o > ostar;
-      const bool eq = i < n && o == ostar;
-      uint32_t ngt, neq;
-      const uint32_t gt_before = s_gt_seen + block_exclusive_scan(gt ? 1u : 0u, &ngt);
-      const uint32_t eq_before = s_eq_seen + block_exclusive_scan(eq ? 1u : 0u, &neq);
-      // index order is preserved: kept entries before this one = gt_before + min(eq_before, r_eq)
-      const uint32_t pos = gt_before + min(eq_before, r_eq);
-      if ((gt || (eq && eq_before < r_eq)) && pos < kk) ob[pos] = int32_t(i);
-      if (threadIdx.x == 0) {
-        s_gt_seen += ngt;
-        s_eq_seen += neq;
       }
       __syncthreads();
+      // ordered compaction of the kept candidates
+      uint32_t m[kResPer], off[kResPer];
+#pragma unroll
+      for (int j = 0; j < kResPer; ++j) {
+        const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
+        const uint32_t pre = uint32_t(c[j] >> 40);
+        const bool keep = g < total && (pre > prefix || (pre == prefix && ((s_keep[g >> 5] >> (g & 31)) & 1u)));
+        m[j] = __ballot_sync(kFull, keep);
+      }
+      const uint32_t got = ordered_offsets<kSelThreads, kResPer>(m, off);
+      const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+      for (int j = 0; j < kResPer; ++j) {
+        if ((m[j] >> lane) & 1u) {
+          const uint32_t at = off[j] + __popc(m[j] & lt);
+          if (at < kk) out[at] = int32_t(0xffffffffu - uint32_t(c[j]));
+        }
+      }
+      if (threadIdx.x == 0 && got != kk) set_status(status, DSV4KV_DEV_INCONSISTENT);
     }
-    if (threadIdx.x == 0 && s_gt_seen + min(s_eq_seen, r_eq) != kk) set_status(status, DSV4KV_DEV_INCONSISTENT);
   }
-  for (int i = int(kk) + threadIdx.x; i < k; i += blockDim.x) ob[i] = -1;
+  __syncthreads();
+  if (!ok) {
+    if (!fits) {
+      // the candidates did not fit: the second-level threshold from all scores
+      for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) sh[i] = 0;
+      __syncthreads();
+      for (int64_t i = threadIdx.x; i < n; i += kSelThreads) {
+        const uint32_t o = ord_f32(sc[i]);
+        if (int(o >> 20) == bin1) atomicAdd(&sh[(o >> 8) & 0xfffu], 1u);
+      }
+      __syncthreads();
+      uint32_t above2;
+      const int bin2 = find_threshold_bin<kSelThreads>(sh, need1, &above2);
+      prefix = (uint32_t(bin1) << 12) | uint32_t(bin2);
+      need_tie = need1 - above2;
+    }
+    select_by_scan<kSelThreads>(sc, n, prefix, need_tie, kk, out, sh, status);
+  }
+  for (int i = int(kk) + threadIdx.x; i < k; i += kSelThreads) out[i] = -1;
   if (threadIdx.x == 0 && count_out) count_out[b] = int32_t(kk);
-
-  // 4) leave the workspace zeroed for the next call
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
-    hb[i] = 0;
-    h2[i] = 0;
-  }
-  if (threadIdx.x == 0) {
-    cand_count[b] = 0;
-    done[b] = 0;
-  }
+  // 5) leave the histogram zeroed for the next call (every CTA of the cluster has read it)
+  for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) hb[i] = 0;
 }
 
 __global__ void index_fill_all(int64_t n, int k, int32_t* __restrict__ idx_out, int32_t* __restrict__ count_out) {
@@ -610,19 +730,15 @@ __global__ void index_fill_all(int64_t n, int k, int32_t* __restrict__ idx_out, 
 // ------------------------------------------------------------------ host side
 struct IndexWs {
   uint32_t* status;
-  uint32_t* done;
-  uint32_t* cand_count;
   uint32_t* hist;
-  uint32_t* hist2;
   float* scores;
-  uint64_t* cand;
-  int64_t cap;
   size_t bytes;
 };
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 static IndexWs index_ws_layout(char* base, int batch, int64_t n, int k) {
+  (void)k;
   IndexWs w{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -631,13 +747,8 @@ static IndexWs index_ws_layout(char* base, int batch, int64_t n, int k) {
     return p;
   };
   w.status = reinterpret_cast<uint32_t*>(take(16));
-  w.done = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * batch));
-  w.cand_count = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * batch));
   w.hist = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * kHistBins * size_t(batch)));
-  w.hist2 = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * kHistBins * size_t(batch)));
   w.scores = reinterpret_cast<float*>(take(sizeof(float) * size_t(batch) * size_t(n)));
-  w.cap = std::max<int64_t>(8192, 2 * int64_t(k));
-  w.cand = reinterpret_cast<uint64_t*>(take(sizeof(uint64_t) * size_t(batch) * size_t(w.cap)));
   w.bytes = off;
   return w;
 }
@@ -676,32 +787,51 @@ dsv4kv_status index_topk_launch(const uint16_t* qidx, const dsv4kv_cache& keys, 
     launch_pdl(index_score_bf16<8, true>, dim3(unsigned((total + per_cta - 1) / per_cta)), dim3(256), 0, stream, qidx,
                static_cast<const uint16_t*>(keys.codes), keys.rows, n, batch, per_cta, w.scores, w.hist);
   } else {
-    const int64_t target = int64_t(sms) * 4;
-    int64_t splits = std::max<int64_t>(1, (target + batch - 1) / batch);
-    int64_t chunk = (n + splits - 1) / splits;
-    chunk = std::max<int64_t>(256, (chunk + 31) / 32 * 32);
-    splits = (n + chunk - 1) / chunk;
-    const dim3 g1((unsigned)splits, (unsigned)batch);
-    launch_pdl(index_score_fp4, g1, dim3(256), 0, stream, qidx, static_cast<const uint8_t*>(keys.codes),
-               static_cast<const uint8_t*>(keys.scales), keys.rows, n, chunk, w.scores, w.hist);
+    static int occ4 = 0;
+    if (occ4 == 0 &&
+        (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ4, index_score_fp4, 256, 0) != cudaSuccess || occ4 < 1))
+      occ4 = 1;
+    const int64_t total = int64_t(batch) * n;
+    const int64_t grid = int64_t(sms) * occ4;
+    const int64_t per_cta = std::max<int64_t>(64, (total + grid - 1) / grid);
+    launch_pdl(index_score_fp4, dim3(unsigned((total + per_cta - 1) / per_cta)), dim3(256), 0, stream, qidx,
+               static_cast<const uint8_t*>(keys.codes), static_cast<const uint8_t*>(keys.scales), keys.rows, n,
+               batch, per_cta, w.scores, w.hist);
   }
   dsv4kv_status st = check_launch("index_score");
   if (st != DSV4KV_OK) return st;
-  // filter/select: chunks of 4096 scores
-  int64_t chunk2 = 4096;
-  int64_t splits2 = (n + chunk2 - 1) / chunk2;
-  const dim3 g2((unsigned)splits2, (unsigned)batch);
-  const size_t dyn = n <= kMaxBitmapN ? size_t(2) * size_t((n + 31) / 32) * sizeof(uint32_t) : 0;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(index_filter_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(2 * (kMaxBitmapN / 32) * sizeof(uint32_t))) != cudaSuccess)
-      return check_launch("index_filter_select: cudaFuncSetAttribute");
-    attr_set = true;
+  // selection: one cluster of C CTAs per sequence, chunks of whole 4096-score batches
+  static int max_cluster = 0;
+  if (max_cluster == 0) {
+    if (cudaFuncSetAttribute(index_select, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSelDyn)) != cudaSuccess)
+      return check_launch("index_select: cudaFuncSetAttribute");
+    max_cluster = 8;
+    if (cudaFuncSetAttribute(index_select, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(kMaxClusterSel, 1);
+      cfg.blockDim = dim3(kSelThreads);
+      cfg.dynamicSmemBytes = kSelDyn;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = kMaxClusterSel;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, index_select, &cfg) == cudaSuccess && clusters > 0)
+        max_cluster = kMaxClusterSel;
+    }
+    cudaGetLastError();  // a refused query only means the portable size
   }
-  launch_pdl(index_filter_select, g2, dim3(kSelThreads), dyn, stream, w.scores, n, k, chunk2, w.hist, w.hist2, w.done,
-             w.cand_count, w.cand, w.cap, idx_out, count_out, w.status);
-  return check_launch("index_filter_select");
+  // at most one CTA per SM in all (the leader's registers allow one per SM)
+  const int64_t per_seq = std::max<int64_t>(1, std::min<int64_t>(max_cluster, sms / std::max(batch, 1)));
+  const int64_t batches_per_cta = std::max<int64_t>(1, (n + per_seq * kSelBatchSpan - 1) / (per_seq * kSelBatchSpan));
+  const int64_t chunk = batches_per_cta * kSelBatchSpan;
+  const unsigned ctas = unsigned((n + chunk - 1) / chunk);
+  launch_pdl_cluster(index_select, dim3(ctas, unsigned(batch)), dim3(kSelThreads), kSelDyn, ctas, stream,
+                     (const float*)w.scores, n, k, chunk, w.hist, idx_out, count_out, w.status);
+  return check_launch("index_select");
 }
 
 }  // namespace dsv4kv
