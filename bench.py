@@ -40,6 +40,10 @@ WORKLOADS = {
     "q_c128a_fp4": ("c128a", 64, 262144, 64, 2, 0),
 }
 FMT_NAME = {0: "bf16", 1: "fp8", 2: "fp4"}
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
+# capture of that kernel in this workload (profiles/ holds the summary and the
+# command); cleared whenever the kernel changes
+TRAFFIC = {("c4a_b32", "index_score_bf16"): 273290752}
 
 
 def measured_peaks():
@@ -190,6 +194,13 @@ class Layer:
         self.K.index_topk(self.qidx, self.reps[r]["kidx"], self.n, self.k, idx_out=self.idx, count_out=self.cnt,
                           ws=self.ws_idx)
 
+    # the same call in its two steps (dsv4kv_index_score; dsv4kv_index_select)
+    def index_score(self, r):
+        self.K.index_score(self.qidx, self.reps[r]["kidx"], self.n, self.k, self.ws_idx)
+
+    def index_select(self):
+        self.K.index_select(self.batch, self.n, self.k, self.idx, self.cnt, self.ws_idx)
+
     def decode(self, r, q=None, out=None):
         rep = self.reps[r]
         K = self.K
@@ -308,9 +319,10 @@ def time_bulk(seed):
 
 def time_layer(layer, steps, warmup, dist_max, dev_index, sample_clocks):
     """Device time of exactly `steps` steps.  All steps (replicas alternating)
-    are captured into one CUDA graph with event nodes between the calls, so
-    the host launches once and the per-call device times come from the
-    events of the timed replay itself."""
+    are captured into one CUDA graph and timed with events on the launching
+    stream around its replay.  A second graph of the same steps with event
+    nodes between the calls (which cost the programmatic-launch overlap at
+    each event) gives the per-call device times."""
     torch = layer.torch
     R = len(layer.reps)
     stream = torch.cuda.Stream()
@@ -319,25 +331,31 @@ def time_layer(layer, steps, warmup, dist_max, dev_index, sample_clocks):
             layer.step(i % R)
     stream.synchronize()
     # external=True: records inside the capture become event nodes of the graph
-    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(steps)]
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(steps)]
 
     def capture(n_steps, events):
+        # events: step start | after index_score | after index_select | after decode
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for i in range(n_steps):
                 if events:
                     events[i][0].record(stream)
                 if layer.kind == "c4a":
-                    layer.index(i % R)
+                    layer.index_score(i % R)
                 if events:
                     events[i][1].record(stream)
-                layer.decode(i % R)
+                if layer.kind == "c4a":
+                    layer.index_select()
                 if events:
                     events[i][2].record(stream)
+                layer.decode(i % R)
+                if events:
+                    events[i][3].record(stream)
         return g
 
     g_warm = capture(max(warmup, 1), None)
-    g_main = capture(steps, ev)
+    g_main = capture(steps, None)
+    g_inst = capture(steps, ev)
     with torch.cuda.stream(stream):
         g_warm.replay()
     stream.synchronize()
@@ -346,18 +364,26 @@ def time_layer(layer, steps, warmup, dist_max, dev_index, sample_clocks):
     sampler = ClockSampler(dev_index) if sample_clocks else None
     if sampler:
         sampler.__enter__()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
+        start.record(stream)
         g_main.replay()
+        stop.record(stream)
     torch.cuda.synchronize()
     if sampler:
         sampler.__exit__()
     dist_barrier()
-    total_ms = ev[0][0].elapsed_time(ev[-1][2])
-    idx_ms = [e[0].elapsed_time(e[1]) for e in ev] if layer.kind == "c4a" else [0.0]
-    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = start.elapsed_time(stop)
+    with torch.cuda.stream(stream):
+        g_inst.replay()
+    torch.cuda.synchronize()
+    score_ms = [e[0].elapsed_time(e[1]) for e in ev] if layer.kind == "c4a" else [0.0]
+    select_ms = [e[1].elapsed_time(e[2]) for e in ev] if layer.kind == "c4a" else [0.0]
+    dec_ms = [e[2].elapsed_time(e[3]) for e in ev]
     total_ms = dist_max(total_ms)
-    del g_warm, g_main
-    return {"total_ms": total_ms, "index_ms": float(np.mean(idx_ms)), "decode_ms": float(np.mean(dec_ms)),
+    del g_warm, g_main, g_inst
+    return {"total_ms": total_ms, "score_ms": float(np.mean(score_ms)), "select_ms": float(np.mean(select_ms)),
+            "index_ms": float(np.mean(score_ms) + np.mean(select_ms)), "decode_ms": float(np.mean(dec_ms)),
             "clocks": sampler.summary() if sampler else None}
 
 
@@ -540,14 +566,17 @@ def main():
     e2e_ms = dist_max(e2e_ms)
     e2e_v = d["world"] * args.steps * 1e3 / e2e_ms
 
-    # roofline of the dominant call (the indexer for c4a, the dense decode for c128a)
+    # roofline of the dominant kernel: the indexer score kernel for c4a (one
+    # launch per dsv4kv_index_score call), the dense decode call for c128a
     if kind == "c4a":
-        dom_bytes, dom_ms, dom_name = layer.index_bytes(), res["index_ms"], "dsv4kv_index_topk (index_score + index_filter_select)"
+        dom_bytes, dom_ms = layer.index_bytes(), res["score_ms"]
+        dom_name = "index_score_bf16" if ifmt == 0 else "index_score_fp4"
     else:
         dom_bytes, dom_ms, dom_name = alg, res["decode_ms"], "dsv4kv_dense_decode (decode_kernel + decode_combine)"
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     roof = {"bound": "hbm", "kernel": dom_name, "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-            "frac": round(achieved / hbm_peak, 4), "peak_source": peak_src, "traffic": None,
+            "frac": round(achieved / hbm_peak, 4), "peak_source": peak_src,
+            "traffic": TRAFFIC.get((args.workload, dom_name)),
             "bytes_per_launch": dom_bytes, "avg_launch_ms": round(dom_ms, 5)}
 
     per_type = {kind: {"workload": wl_name, "steps_per_s": round(steps_per_s, 1),
@@ -555,7 +584,8 @@ def main():
                        "hbm_gbs": round(alg / (ms * 1e-3) / 1e9, 1),
                        "frac_of_measured_hbm": round(alg / (ms * 1e-3) / 1e9 / hbm_peak, 4),
                        "frac_of_8tbs": round(alg / (ms * 1e-3) / 8e12, 4),
-                       "index_ms": round(res["index_ms"], 5), "decode_ms": round(res["decode_ms"], 5)}}
+                       "index_ms": round(res["index_ms"], 5), "score_ms": round(res["score_ms"], 5),
+                       "select_ms": round(res["select_ms"], 5), "decode_ms": round(res["decode_ms"], 5)}}
     for name in [s for s in args.secondary.split(",") if s and s not in ("none", args.workload)]:
         spec = WORKLOADS[name]
         big = spec[1] * spec[2] >= 2 ** 22
@@ -571,6 +601,8 @@ def main():
                           "frac_of_measured_bf16": round(L2.flops() / (ms2 * 1e-3) / 1e12 / tf_peak, 4)}
         if spec[0] == "c4a":
             per_type[name]["index_us"] = round(r2["index_ms"] * 1e3, 2)
+            per_type[name]["score_us"] = round(r2["score_ms"] * 1e3, 2)
+            per_type[name]["select_us"] = round(r2["select_ms"] * 1e3, 2)
             per_type[name]["decode_us"] = round(r2["decode_ms"] * 1e3, 2)
         del L2
         torch.cuda.empty_cache()

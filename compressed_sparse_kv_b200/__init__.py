@@ -48,6 +48,10 @@ _SIGS = {
     "dsv4kv_index_topk_workspace_bytes": (_c.c_size_t, [_c.c_int32, _c.c_int64, _c.c_int32]),
     "dsv4kv_index_topk": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.c_int32, _c.c_int64, _c.c_int32,
                                      _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "dsv4kv_index_score": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.c_int32, _c.c_int64, _c.c_int32,
+                                      _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "dsv4kv_index_select": (_c.c_int, [_c.c_int32, _c.c_int64, _c.c_int32, _c.c_void_p, _c.c_void_p, _c.c_void_p,
+                                       _c.c_size_t, _c.c_void_p]),
     "dsv4kv_index_topk_noalloc_max_scratch_bytes": (_c.c_size_t, []),
     "dsv4kv_index_topk_noalloc": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.c_int32, _c.c_int64, _c.c_int32,
                                              _c.c_void_p, _c.c_void_p, _c.c_void_p]),
@@ -174,6 +178,21 @@ def index_topk(qidx: torch.Tensor, keys: Cache, n: int, k: int, idx_out: Optiona
     d = keys.desc()
     _check(lib().dsv4kv_index_topk(_ptr(qidx), ctypes.byref(d), b, n, k, _ptr(idx_out), _ptr(count_out), _ptr(ws),
                                    ws.numel(), _stream(stream)), "dsv4kv_index_topk")
+    return idx_out, count_out
+
+
+def index_score(qidx: torch.Tensor, keys: Cache, n: int, k: int, ws: torch.Tensor, stream=None) -> None:
+    """The scoring half of index_topk: scores and histogram into ws (index_topk_workspace_bytes sized)."""
+    d = keys.desc()
+    _check(lib().dsv4kv_index_score(_ptr(qidx), ctypes.byref(d), int(qidx.shape[0]), n, k, _ptr(ws), ws.numel(),
+                                    _stream(stream)), "dsv4kv_index_score")
+
+
+def index_select(batch: int, n: int, k: int, idx_out: torch.Tensor, count_out: Optional[torch.Tensor],
+                 ws: torch.Tensor, stream=None) -> tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """The selection half of index_topk, from the workspace index_score filled."""
+    _check(lib().dsv4kv_index_select(batch, n, k, _ptr(idx_out), _ptr(count_out) if count_out is not None else None,
+                                     _ptr(ws), ws.numel(), _stream(stream)), "dsv4kv_index_select")
     return idx_out, count_out
 
 

@@ -150,27 +150,55 @@ DSV4KV_API size_t dsv4kv_index_topk_workspace_bytes(int32_t batch, int64_t n, in
   return index_topk_ws_bytes(batch, n, k);
 }
 
+// Shared checks of the indexer calls (what = the call's name for messages).
+static dsv4kv_status check_index(const char* what, const void* qidx, const dsv4kv_cache* keys, int32_t batch,
+                                 int64_t n, int32_t k, bool need_keys, bool need_out, const int32_t* idx_out,
+                                 const void* ws, size_t ws_bytes) {
+  if (batch < 0 || n < 0) return set_error(DSV4KV_ERR_INVALID_ARG, "%s: bad sizes", what);
+  if (k < 1 || k > 2048) return set_error(DSV4KV_ERR_UNSUPPORTED, "%s: k must be in [1, 2048]", what);
+  if (batch == 0) return DSV4KV_OK;
+  if (need_out && !idx_out) return set_error(DSV4KV_ERR_INVALID_ARG, "%s: idx_out is null", what);
+  if (need_keys) {
+    if (!keys) return set_error(DSV4KV_ERR_INVALID_ARG, "%s: keys is null", what);
+    if (keys->fmt != DSV4KV_BF16 && keys->fmt != DSV4KV_FP4_E2M1_G16)
+      return set_error(DSV4KV_ERR_UNSUPPORTED, "%s: keys must be bf16 or fp4", what);
+    dsv4kv_status st = check_cache(keys, what, n, 128);
+    if (st != DSV4KV_OK) return st;
+    if (n > k && (!qidx || !aligned16(qidx))) return set_error(DSV4KV_ERR_INVALID_ARG, "%s: qidx null or misaligned", what);
+  }
+  if (n > k) {
+    if (int64_t(batch) * n > (int64_t(1) << 40)) return set_error(DSV4KV_ERR_UNSUPPORTED, "%s: too large", what);
+    if (!ws || ws_bytes < index_topk_ws_bytes(batch, n, k))
+      return set_error(DSV4KV_ERR_WORKSPACE, "%s: workspace null or too small", what);
+  }
+  return DSV4KV_OK;
+}
+
 DSV4KV_API dsv4kv_status dsv4kv_index_topk(const void* qidx, const dsv4kv_cache* keys, int32_t batch, int64_t n,
                                            int32_t k, int32_t* idx_out, int32_t* count_out, void* ws,
                                            size_t ws_bytes, void* stream) {
   g_err[0] = 0;
-  if (batch < 0 || n < 0) return set_error(DSV4KV_ERR_INVALID_ARG, "index_topk: bad sizes");
-  if (k < 1 || k > 2048) return set_error(DSV4KV_ERR_UNSUPPORTED, "index_topk: k must be in [1, 2048]");
-  if (batch == 0) return DSV4KV_OK;
-  if (!idx_out) return set_error(DSV4KV_ERR_INVALID_ARG, "index_topk: idx_out is null");
-  if (!keys) return set_error(DSV4KV_ERR_INVALID_ARG, "index_topk: keys is null");
-  if (keys->fmt != DSV4KV_BF16 && keys->fmt != DSV4KV_FP4_E2M1_G16)
-    return set_error(DSV4KV_ERR_UNSUPPORTED, "index_topk: keys must be bf16 or fp4");
-  dsv4kv_status st = check_cache(keys, "index_topk keys", n, 128);
-  if (st != DSV4KV_OK) return st;
-  if (n > k) {
-    if (!qidx || !aligned16(qidx)) return set_error(DSV4KV_ERR_INVALID_ARG, "index_topk: qidx null or misaligned");
-    if (int64_t(batch) * n > (int64_t(1) << 40)) return set_error(DSV4KV_ERR_UNSUPPORTED, "index_topk: too large");
-    if (!ws || ws_bytes < index_topk_ws_bytes(batch, n, k))
-      return set_error(DSV4KV_ERR_WORKSPACE, "index_topk: workspace null or too small");
-  }
+  dsv4kv_status st = check_index("index_topk", qidx, keys, batch, n, k, true, true, idx_out, ws, ws_bytes);
+  if (st != DSV4KV_OK || batch == 0) return st;
   return index_topk_launch(static_cast<const uint16_t*>(qidx), *keys, batch, n, k, idx_out, count_out, ws, ws_bytes,
                            static_cast<cudaStream_t>(stream));
+}
+
+DSV4KV_API dsv4kv_status dsv4kv_index_score(const void* qidx, const dsv4kv_cache* keys, int32_t batch, int64_t n,
+                                            int32_t k, void* ws, size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  dsv4kv_status st = check_index("index_score", qidx, keys, batch, n, k, true, false, nullptr, ws, ws_bytes);
+  if (st != DSV4KV_OK || batch == 0) return st;
+  return index_score_launch(static_cast<const uint16_t*>(qidx), *keys, batch, n, k, ws, ws_bytes,
+                            static_cast<cudaStream_t>(stream));
+}
+
+DSV4KV_API dsv4kv_status dsv4kv_index_select(int32_t batch, int64_t n, int32_t k, int32_t* idx_out,
+                                             int32_t* count_out, void* ws, size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  dsv4kv_status st = check_index("index_select", nullptr, nullptr, batch, n, k, false, true, idx_out, ws, ws_bytes);
+  if (st != DSV4KV_OK || batch == 0) return st;
+  return index_select_launch(batch, n, k, idx_out, count_out, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 static dsv4kv_status check_decode(const void* q, const dsv4kv_cache* comp, const dsv4kv_cache* win, int32_t batch,

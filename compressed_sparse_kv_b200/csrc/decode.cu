@@ -51,6 +51,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;    // O^T: 4 channel tiles x 64 heads
 constexpr uint32_t kColS = 256;  // scores: 2 buffers x 64 columns
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kIdxSmem = 2048;             // selected indices a CTA keeps in shared memory (k <= 2048)
 
 // Per-format configuration.  bf16 rows feed kind::f16 MMAs with bf16 inputs.
 // Quantised rows are dequantised in the load path; every E4M3 value and every
@@ -80,11 +81,13 @@ struct __align__(8) Ctl {
   float fin[64];
   float row_scale[kStages][kTileRows];
   uint32_t vmask[kStages][4];  // row validity of a gathered tile, 16 rows per loader warp
+  int32_t idx_s[kIdxSmem];     // the selected indices of this CTA's compressed tiles
   float rope_cs[kDim / 2];  // inverse-RoPE rotation of pair m: cos / sin of -t * theta_m
   float rope_sn[kDim / 2];
 };
 
 constexpr size_t kSmemBytes = 1024 + kQBytes + kStages * kTileBytes + 2 * kPBytes + sizeof(Ctl);
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 struct Params {
   int heads;
@@ -153,6 +156,7 @@ __device__ __forceinline__ bool named_bar_or(bool pred) {
   return r != 0;
 }
 __device__ __forceinline__ void named_bar_sync() { asm volatile("barrier.cta.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void loader_bar_sync() { asm volatile("barrier.cta.sync 2, 128;" ::: "memory"); }
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
@@ -174,13 +178,14 @@ struct RowSrc {
   int64_t row;
   bool valid, from_win;
 };
-__device__ __forceinline__ RowSrc row_source(const Params& p, int b, int T, int r) {
+__device__ __forceinline__ RowSrc row_source(const Params& p, int b, int T, int r, const int32_t* idx_s = nullptr,
+                                             int slot0 = 0) {
   RowSrc s{0, false, false};
   if (T < p.comp_tiles) {
     const int slot = T * kTileRows + r;
     int64_t i = -1;
     if (p.idx) {
-      const int32_t v = slot < p.k ? p.idx[size_t(b) * p.k + slot] : -1;
+      const int32_t v = slot >= p.k ? -1 : (idx_s ? idx_s[slot - slot0] : p.idx[size_t(b) * p.k + slot]);
       if (v >= p.n) set_status(p.status, DSV4KV_DEV_BAD_INDEX);
       i = v;
     } else if (slot < p.n) {
@@ -612,6 +617,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ loaders (warps 6..9)
     const int lw = warp - 6;
+    // the CTA's selected indices, once, into shared memory
+    const int slot0 = t0 * kTileRows;
+    const int nslots = p.idx ? min(max(0, min(p.k, (t0 + nt) * kTileRows) - slot0), kIdxSmem) : 0;
+    for (int i = threadIdx.x - 192; i < nslots; i += 128) ctl->idx_s[i] = __ldg(p.idx + size_t(b) * p.k + slot0 + i);
+    loader_bar_sync();
     if (C::kQuant) {
       // Q: bf16 -> f16 in place (saturating), once per CTA
       if (warp_wait(&ctl->q_full, 0, ctl, lane)) {
@@ -635,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // warp 0 brings this tile by TMA
       } else {
         // lane j < 16 resolves row 16*lw + j; every lane reads all 16 answers
-        const RowSrc mine = row_source(p, b, T, 16 * lw + (lane & 15));
+        const RowSrc mine = row_source(p, b, T, 16 * lw + (lane & 15), ctl->idx_s, slot0);
         const uint32_t vb = __ballot_sync(kFull, mine.valid) & 0xffffu;
         if (lane == 0) ctl->vmask[stage][lw] = vb;
         if (!C::kQuant) {

@@ -67,13 +67,76 @@ __device__ __forceinline__ float dot8_bf16(const uint4& v, const float (&q)[8]) 
   return fmaf(q[7], bf16hi(v.w), a);
 }
 
-// bf16 keys, dim 128: a key is 256 B = 16 lanes x 16 B.  The flattened
-// (sequence, entry) range of all B*n keys is split evenly over the grid; a
-// CTA walks its range one sequence segment at a time.  A warp iteration
-// covers 2U keys: half-warp h reads keys 2U*j + U*h + u (u < U), U
-// independent 16-byte loads per lane; with DB the next iteration's loads are
-// issued before the current iteration is reduced, so loads stay in flight.
-template <int U, bool DB>
+// bf16 keys, dim 128: a key is 256 B = 16 lanes x 16 B.  score_segment_bf16
+// scores the keys [0, cnt) of one sequence segment (kb: the segment's first
+// key, this lane's 16 bytes): a warp iteration covers 2U keys, half-warp h
+// reading keys 2U*j + U*h + u (u < U), U independent 16-byte loads per lane;
+// the next iteration's loads are issued before the current one is reduced,
+// so loads stay in flight.  Scores go to sc (global) and, when ssc is not
+// null, to shared memory; the top-12-bit histogram of the codes to sh.
+template <int U>
+__device__ __forceinline__ void score_segment_bf16(const uint16_t* __restrict__ qrow, const uint16_t* kb,
+                                                   int64_t cnt, float* sc, float* ssc, uint32_t* sh, uint64_t pol) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int half = lane >> 4, l16 = lane & 15;
+  const int my_key = U == 16 ? l16 : ((l16 >> 1) & 7);
+  const bool writer = U == 16 || !(lane & 1);
+  float q[8];
+  {
+    const uint4 v = *reinterpret_cast<const uint4*>(qrow + 8 * l16);
+    q[0] = bf16lo(v.x); q[1] = bf16hi(v.x); q[2] = bf16lo(v.y); q[3] = bf16hi(v.y);
+    q[4] = bf16lo(v.z); q[5] = bf16hi(v.z); q[6] = bf16lo(v.w); q[7] = bf16hi(v.w);
+  }
+  kb += 8 * l16;
+  auto load = [&](int64_t j, uint4 (&v)[U]) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t key = 2 * U * j + U * half + u;
+      v[u] = key < cnt ? ld_once_v4(kb + key * 128, pol) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  auto process = [&](int64_t j, const uint4 (&v)[U]) {
+    float p[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) p[u] = dot8_bf16(v[u], q);
+    const float s = reduce16_transposed<U>(p, l16) + 0.0f;  // -0 -> +0
+    const int64_t key = 2 * U * j + U * half + my_key;
+    if (writer && key < cnt) {
+      sc[key] = s;
+      if (ssc) ssc[key] = s;
+      atomicAdd(&sh[ord_f32(s) >> 20], 1u);
+    }
+  };
+  const int64_t ngroups = (cnt + 2 * U - 1) / (2 * U);
+  uint4 va[U], vb[U];
+  int64_t j = warp;
+  if (j < ngroups) load(j, va);
+  while (j < ngroups) {
+    if (j + nwarps < ngroups) load(j + nwarps, vb);
+    process(j, va);
+    j += nwarps;
+    if (j >= ngroups) break;
+    if (j + nwarps < ngroups) load(j + nwarps, va);
+    process(j, vb);
+    j += nwarps;
+  }
+}
+
+// Adds the CTA's histogram sh to the sequence's global histogram and clears it.
+__device__ __forceinline__ void flush_histogram(uint32_t* sh, uint32_t* hb) {
+  __syncthreads();
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
+    const uint32_t c = sh[i];
+    if (c) {
+      atomicAdd(&hb[i], c);
+      sh[i] = 0;
+    }
+  }
+}
+
+// The flattened (sequence, entry) range of all B*n keys split evenly over the
+// grid; a CTA walks its range one sequence segment at a time.
+template <int U>
 __global__ void __launch_bounds__(256) index_score_bf16(const uint16_t* __restrict__ qidx,
                                                         const uint16_t* __restrict__ keys, int64_t key_rows,
                                                         int64_t n, int batch, int64_t per_cta,
@@ -85,72 +148,17 @@ __global__ void __launch_bounds__(256) index_score_bf16(const uint16_t* __restri
   const int64_t g1 = min(total, g0 + per_cta);
   if (g0 >= g1) return;
   pdl_wait();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int half = lane >> 4, l16 = lane & 15;
-  const int my_key = U == 16 ? l16 : ((l16 >> 1) & 7);
-  const bool writer = U == 16 || !(lane & 1);
+  const uint64_t pol = l2_evict_first_policy();  // keys are read once
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0;
+  __syncthreads();
   for (int64_t s0 = g0; s0 < g1;) {
     const int b = int(s0 / n);
     const int64_t s1 = min(g1, int64_t(b + 1) * n);
-    const int64_t i0 = s0 - int64_t(b) * n, cnt = s1 - s0;
-    float q[8];
-    {
-      const uint4 v = *reinterpret_cast<const uint4*>(qidx + size_t(b) * 128 + 8 * l16);
-      q[0] = bf16lo(v.x); q[1] = bf16hi(v.x); q[2] = bf16lo(v.y); q[3] = bf16hi(v.y);
-      q[4] = bf16lo(v.z); q[5] = bf16hi(v.z); q[6] = bf16lo(v.w); q[7] = bf16hi(v.w);
-    }
-    __syncthreads();  // histogram cleared
-    const uint16_t* kb = keys + (size_t(b) * size_t(key_rows) + size_t(i0)) * 128 + 8 * l16;
-    float* sc = scores + size_t(b) * size_t(n) + size_t(i0);
-    auto load = [&](int64_t j, uint4 (&v)[U]) {
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t key = 2 * U * j + U * half + u;
-        v[u] = key < cnt ? ld_stream_v4(kb + key * 128) : make_uint4(0, 0, 0, 0);
-      }
-    };
-    auto process = [&](int64_t j, const uint4 (&v)[U]) {
-      float p[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) p[u] = dot8_bf16(v[u], q);
-      const float s = reduce16_transposed<U>(p, l16) + 0.0f;  // -0 -> +0
-      const int64_t key = 2 * U * j + U * half + my_key;
-      if (writer && key < cnt) {
-        sc[key] = s;
-        atomicAdd(&sh[ord_f32(s) >> 20], 1u);
-      }
-    };
-    const int64_t ngroups = (cnt + 2 * U - 1) / (2 * U);
-    if constexpr (DB) {
-      uint4 va[U], vb[U];
-      int64_t j = warp;
-      if (j < ngroups) load(j, va);
-      while (j < ngroups) {
-        if (j + nwarps < ngroups) load(j + nwarps, vb);
-        process(j, va);
-        j += nwarps;
-        if (j >= ngroups) break;
-        if (j + nwarps < ngroups) load(j + nwarps, va);
-        process(j, vb);
-        j += nwarps;
-      }
-    } else {
-      for (int64_t j = warp; j < ngroups; j += nwarps) {
-        uint4 v[U];
-        load(j, v);
-        process(j, v);
-      }
-    }
+    const int64_t i0 = s0 - int64_t(b) * n;
+    score_segment_bf16<U>(qidx + size_t(b) * 128, keys + (size_t(b) * size_t(key_rows) + size_t(i0)) * 128, s1 - s0,
+                          scores + size_t(b) * size_t(n) + size_t(i0), nullptr, sh, pol);
+    flush_histogram(sh, hist + size_t(b) * kHistBins);
     __syncthreads();
-    uint32_t* hb = hist + size_t(b) * kHistBins;
-    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
-      const uint32_t c = sh[i];
-      if (c) {
-        atomicAdd(&hb[i], c);
-        sh[i] = 0;
-      }
-    }
     s0 = s1;
   }
 }
@@ -209,18 +217,86 @@ __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
 
 // fp4 keys, dim 128: 64 B of codes + 8 E4M3 scale bytes per key.  A quarter
 // warp (4 lanes x 16 B) covers one key; lane l4 holds channels
-// [32*l4, 32*l4+32) = two 16-channel scale groups.  Same flattened, evenly
-// split, double-buffered structure as the bf16 kernel; each warp iteration
-// covers 32 keys (U = 4 per quad).  Each code byte is decoded to a packed f16
-// pair with cvt.rn.f16x2.e2m1x2 and accumulated with packed f16 FMAs per
-// group (exact for integer queries: |partial| <= 8*8*6 per half at a
-// resolution of 0.5), then scaled by the group's E4M3 scale in fp32.
+// [32*l4, 32*l4+32) = two 16-channel scale groups.  Same segment structure as
+// the bf16 path; each warp iteration covers 32 keys (U = 4 per quad).  Each
+// code byte is decoded to a packed f16 pair with cvt.rn.f16x2.e2m1x2 and
+// accumulated with packed f16 FMAs per group (exact for integer queries:
+// |partial| <= 8*8*6 per half at a resolution of 0.5), then scaled by the
+// group's E4M3 scale in fp32.
+__device__ __forceinline__ void score_segment_fp4(const uint16_t* __restrict__ qrow, const uint8_t* cb,
+                                                  const uint8_t* sb, int64_t cnt, float* sc, float* ssc,
+                                                  uint32_t* sh, uint64_t pol) {
+  constexpr int U = 4;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int quad = lane >> 2, l4 = lane & 3;
+  uint32_t qp[16];  // (q[2j], q[2j+1]) as f16x2 for this lane's 32 channels
+  {
+    const uint16_t* qb = qrow + 32 * l4;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) qp[j] = f32x2_to_f16x2(bf16f(qb[2 * j]), bf16f(qb[2 * j + 1]));
+  }
+  cb += 16 * l4;
+  sb += 2 * l4;
+  auto load = [&](int64_t j, uint4 (&v)[U], uint32_t (&s2)[U]) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t key = 8 * U * j + 8 * u + quad;
+      const bool ok = key < cnt;
+      v[u] = ok ? ld_once_v4(cb + key * 64, pol) : make_uint4(0, 0, 0, 0);
+      s2[u] = ok ? ld_once_u16(sb + key * 8, pol) : 0u;
+    }
+  };
+  auto process = [&](int64_t j, const uint4 (&v)[U], const uint32_t (&s2)[U]) {
+    float p[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      uint32_t acc0 = 0, acc1 = 0;  // f16x2 sums of group 0 (words 0, 1) and group 1 (words 2, 3)
+#pragma unroll
+      for (int wi = 0; wi < 4; ++wi) {
+#pragma unroll
+        for (int by = 0; by < 4; ++by) {
+          const uint32_t h = e2m1x2_to_f16x2((w[wi] >> (8 * by)) & 0xffu);
+          if (wi < 2) acc0 = hfma2(qp[4 * wi + by], h, acc0);
+          else acc1 = hfma2(qp[4 * wi + by], h, acc1);
+        }
+      }
+      p[u] = f16x2_sum(acc0) * e4m3_to_f32(s2[u] & 0xffu) + f16x2_sum(acc1) * e4m3_to_f32(s2[u] >> 8);
+    }
+    // reduce over the 4 lanes of the quad: 4 values -> transposing butterfly
+    const bool bb1 = l4 & 2, bb0 = l4 & 1;
+    float k2[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) k2[i] = (bb1 ? p[2 + i] : p[i]) + __shfl_xor_sync(kFull, bb1 ? p[i] : p[2 + i], 2);
+    const float s = (bb0 ? k2[1] : k2[0]) + __shfl_xor_sync(kFull, bb0 ? k2[0] : k2[1], 1) + 0.0f;
+    const int64_t key = 8 * U * j + 8 * l4 + quad;  // lane l4 ends with key u = l4
+    if (key < cnt) {
+      sc[key] = s;
+      if (ssc) ssc[key] = s;
+      atomicAdd(&sh[ord_f32(s) >> 20], 1u);
+    }
+  };
+  const int64_t ngroups = (cnt + 8 * U - 1) / (8 * U);
+  uint4 va[U], vb[U];
+  uint32_t sa[U], sb2[U];
+  int64_t j = warp;
+  if (j < ngroups) load(j, va, sa);
+  while (j < ngroups) {
+    if (j + nwarps < ngroups) load(j + nwarps, vb, sb2);
+    process(j, va, sa);
+    j += nwarps;
+    if (j >= ngroups) break;
+    if (j + nwarps < ngroups) load(j + nwarps, va, sa);
+    process(j, vb, sb2);
+    j += nwarps;
+  }
+}
+
 __global__ void __launch_bounds__(256) index_score_fp4(const uint16_t* __restrict__ qidx,
                                                        const uint8_t* __restrict__ codes,
                                                        const uint8_t* __restrict__ scales, int64_t key_rows,
                                                        int64_t n, int batch, int64_t per_cta,
                                                        float* __restrict__ scores, uint32_t* __restrict__ hist) {
-  constexpr int U = 4;
   __shared__ uint32_t sh[kHistBins];
   pdl_trigger();
   const int64_t total = int64_t(batch) * n;
@@ -228,84 +304,18 @@ __global__ void __launch_bounds__(256) index_score_fp4(const uint16_t* __restric
   const int64_t g1 = min(total, g0 + per_cta);
   if (g0 >= g1) return;
   pdl_wait();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int quad = lane >> 2, l4 = lane & 3;
+  const uint64_t pol = l2_evict_first_policy();  // keys are read once
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0;
+  __syncthreads();
   for (int64_t s0 = g0; s0 < g1;) {
     const int b = int(s0 / n);
     const int64_t s1 = min(g1, int64_t(b + 1) * n);
-    const int64_t i0 = s0 - int64_t(b) * n, cnt = s1 - s0;
-    uint32_t qp[16];  // (q[2j], q[2j+1]) as f16x2 for this lane's 32 channels
-    {
-      const uint16_t* qb = qidx + size_t(b) * 128 + 32 * l4;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) qp[j] = f32x2_to_f16x2(bf16f(qb[2 * j]), bf16f(qb[2 * j + 1]));
-    }
-    __syncthreads();  // histogram cleared
-    const uint8_t* cb = codes + (size_t(b) * size_t(key_rows) + size_t(i0)) * 64 + 16 * l4;
-    const uint8_t* sb = scales + (size_t(b) * size_t(key_rows) + size_t(i0)) * 8 + 2 * l4;
-    float* sc = scores + size_t(b) * size_t(n) + size_t(i0);
-    auto load = [&](int64_t j, uint4 (&v)[U], uint32_t (&s2)[U]) {
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t key = 8 * U * j + 8 * u + quad;
-        const bool ok = key < cnt;
-        v[u] = ok ? ld_stream_v4(cb + key * 64) : make_uint4(0, 0, 0, 0);
-        s2[u] = ok ? *reinterpret_cast<const uint16_t*>(sb + key * 8) : 0u;
-      }
-    };
-    auto process = [&](int64_t j, const uint4 (&v)[U], const uint32_t (&s2)[U]) {
-      float p[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-        uint32_t acc0 = 0, acc1 = 0;  // f16x2 sums of group 0 (words 0, 1) and group 1 (words 2, 3)
-#pragma unroll
-        for (int wi = 0; wi < 4; ++wi) {
-#pragma unroll
-          for (int by = 0; by < 4; ++by) {
-            const uint32_t h = e2m1x2_to_f16x2((w[wi] >> (8 * by)) & 0xffu);
-            if (wi < 2) acc0 = hfma2(qp[4 * wi + by], h, acc0);
-            else acc1 = hfma2(qp[4 * wi + by], h, acc1);
-          }
-        }
-        p[u] = f16x2_sum(acc0) * e4m3_to_f32(s2[u] & 0xffu) + f16x2_sum(acc1) * e4m3_to_f32(s2[u] >> 8);
-      }
-      // reduce over the 4 lanes of the quad: 4 values -> transposing butterfly
-      const bool bb1 = l4 & 2, bb0 = l4 & 1;
-      float k2[2];
-#pragma unroll
-      for (int i = 0; i < 2; ++i) k2[i] = (bb1 ? p[2 + i] : p[i]) + __shfl_xor_sync(kFull, bb1 ? p[i] : p[2 + i], 2);
-      const float s = (bb0 ? k2[1] : k2[0]) + __shfl_xor_sync(kFull, bb0 ? k2[0] : k2[1], 1) + 0.0f;
-      const int64_t key = 8 * U * j + 8 * l4 + quad;  // lane l4 ends with key u = l4
-      if (key < cnt) {
-        sc[key] = s;
-        atomicAdd(&sh[ord_f32(s) >> 20], 1u);
-      }
-    };
-    const int64_t ngroups = (cnt + 8 * U - 1) / (8 * U);
-    uint4 va[U], vb[U];
-    uint32_t sa[U], sb2[U];
-    int64_t j = warp;
-    if (j < ngroups) load(j, va, sa);
-    while (j < ngroups) {
-      if (j + nwarps < ngroups) load(j + nwarps, vb, sb2);
-      process(j, va, sa);
-      j += nwarps;
-      if (j >= ngroups) break;
-      if (j + nwarps < ngroups) load(j + nwarps, va, sa);
-      process(j, vb, sb2);
-      j += nwarps;
-    }
+    const int64_t i0 = s0 - int64_t(b) * n;
+    const size_t r0 = size_t(b) * size_t(key_rows) + size_t(i0);
+    score_segment_fp4(qidx + size_t(b) * 128, codes + r0 * 64, scales + r0 * 8, s1 - s0,
+                      scores + size_t(b) * size_t(n) + size_t(i0), nullptr, sh, pol);
+    flush_histogram(sh, hist + size_t(b) * kHistBins);
     __syncthreads();
-    uint32_t* hb = hist + size_t(b) * kHistBins;
-    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
-      const uint32_t c = sh[i];
-      if (c) {
-        atomicAdd(&hb[i], c);
-        sh[i] = 0;
-      }
-    }
     s0 = s1;
   }
 }
@@ -460,6 +470,19 @@ __device__ uint32_t ordered_offsets(const uint32_t (&m)[BATCH], uint32_t (&off)[
   return total;
 }
 
+// Copies a sequence's 4096-bin histogram from the workspace (L2) into shared
+// memory with every load of a thread issued before its stores.
+template <int NT>
+__device__ __forceinline__ void load_histogram(const uint32_t* __restrict__ hb, uint32_t* sh) {
+  constexpr int V = kHistBins / 4 / NT;  // uint4 per thread
+  static_assert(V * 4 * NT == kHistBins, "histogram split");
+  uint4 v[V];
+#pragma unroll
+  for (int j = 0; j < V; ++j) v[j] = __ldcg(reinterpret_cast<const uint4*>(hb) + threadIdx.x + j * NT);
+#pragma unroll
+  for (int j = 0; j < V; ++j) reinterpret_cast<uint4*>(sh)[threadIdx.x + j * NT] = v[j];
+}
+
 template <int NT, int BATCH>
 __device__ __forceinline__ void load_codes(const float* __restrict__ sc, int64_t base, int64_t end,
                                            uint32_t (&o)[BATCH]) {
@@ -553,7 +576,7 @@ __global__ void __launch_bounds__(kSelThreads) index_select(const float* __restr
                                                             int32_t* __restrict__ count_out,
                                                             uint32_t* __restrict__ status) {
   extern __shared__ __align__(16) uint64_t stage[];  // kSelStage: this CTA's candidates, in index order
-  __shared__ uint32_t sh[kHistBins];
+  __shared__ __align__(16) uint32_t sh[kHistBins];
   __shared__ uint32_t s_count, s_ntie;
   __shared__ uint32_t s_keep[kCandCap / 32];  // tie verdicts by candidate position
   __shared__ uint32_t s_pre[kMaxClusterSel + 1];
@@ -572,7 +595,7 @@ __global__ void __launch_bounds__(kSelThreads) index_select(const float* __restr
   // 1) the first batch of scores is in flight while the histogram is read
   uint32_t oa[kSelBatch], ob2[kSelBatch];
   load_codes<kSelThreads, kSelBatch>(sc, n0, n1, oa);
-  for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) sh[i] = __ldcg(hb + i);
+  load_histogram<kSelThreads>(hb, sh);
   __syncthreads();
   uint32_t above1;
   const int bin1 = find_threshold_bin<kSelThreads>(sh, kk, &above1);
@@ -608,15 +631,19 @@ __global__ void __launch_bounds__(kSelThreads) index_select(const float* __restr
     total = s_pre[csize];
     fits = total <= uint32_t(kCandCap);
     if (fits) {
+      // the source of every position first, then all the loads
+      uint32_t src[kResPer];
 #pragma unroll
       for (int j = 0; j < kResPer; ++j) {
         const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
-        c[j] = 0ull;
-        if (g < total) {
-          uint32_t r = 0;
-          while (r + 1 < csize && s_pre[r + 1] <= g) ++r;
-          c[j] = ld_dsmem_u64(dsmem_addr(&stage[g - s_pre[r]], r));
-        }
+        uint32_t r = 0;
+        while (r + 1 < csize && s_pre[r + 1] <= g) ++r;
+        src[j] = dsmem_addr(&stage[g < total ? g - s_pre[r] : 0], r);
+      }
+#pragma unroll
+      for (int j = 0; j < kResPer; ++j) {
+        const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
+        c[j] = g < total ? ld_dsmem_u64(src[j]) : 0ull;
       }
     }
   }
@@ -762,29 +789,30 @@ size_t index_topk_zero_prefix_bytes(int batch) {
   return size_t(reinterpret_cast<char*>(w.scores) - static_cast<char*>(nullptr));
 }
 
-dsv4kv_status index_topk_launch(const uint16_t* qidx, const dsv4kv_cache& keys, int batch, int64_t n, int k,
-                                int32_t* idx_out, int32_t* count_out, void* ws, size_t ws_bytes,
-                                cudaStream_t stream) {
-  if (n <= k) {
-    const dim3 grid((unsigned)((k + 255) / 256), (unsigned)batch);
-    if (launch_pdl(index_fill_all, grid, dim3(256), 0, stream, n, k, idx_out, count_out) != cudaSuccess)
-      return check_launch("index_fill_all");
-    return check_launch("index_fill_all");
-  }
+static dsv4kv_status index_fill_launch(int batch, int64_t n, int k, int32_t* idx_out, int32_t* count_out,
+                                       cudaStream_t stream) {
+  const dim3 grid((unsigned)((k + 255) / 256), (unsigned)batch);
+  launch_pdl(index_fill_all, grid, dim3(256), 0, stream, n, k, idx_out, count_out);
+  return check_launch("index_fill_all");
+}
+
+dsv4kv_status index_score_launch(const uint16_t* qidx, const dsv4kv_cache& keys, int batch, int64_t n, int k,
+                                 void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (n <= k) return DSV4KV_OK;  // every entry is selected: nothing to score
   const IndexWs w = index_ws_layout(static_cast<char*>(ws), batch, n, k);
-  if (ws_bytes < w.bytes) return set_error(DSV4KV_ERR_WORKSPACE, "index_topk: workspace too small");
+  if (ws_bytes < w.bytes) return set_error(DSV4KV_ERR_WORKSPACE, "index_score: workspace too small");
   const int sms = sm_count();
   if (keys.fmt == DSV4KV_BF16) {
     // one wave (resident CTAs per SM x SMs) over the flattened (sequence, entry) range
     static int occ = 0;
     if (occ == 0 &&
-        (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, index_score_bf16<8, true>, 256, 0) != cudaSuccess ||
+        (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, index_score_bf16<8>, 256, 0) != cudaSuccess ||
          occ < 1))
       occ = 1;
     const int64_t total = int64_t(batch) * n;
     const int64_t grid = int64_t(sms) * occ;
     const int64_t per_cta = std::max<int64_t>(64, (total + grid - 1) / grid);
-    launch_pdl(index_score_bf16<8, true>, dim3(unsigned((total + per_cta - 1) / per_cta)), dim3(256), 0, stream, qidx,
+    launch_pdl(index_score_bf16<8>, dim3(unsigned((total + per_cta - 1) / per_cta)), dim3(256), 0, stream, qidx,
                static_cast<const uint16_t*>(keys.codes), keys.rows, n, batch, per_cta, w.scores, w.hist);
   } else {
     static int occ4 = 0;
@@ -798,8 +826,15 @@ dsv4kv_status index_topk_launch(const uint16_t* qidx, const dsv4kv_cache& keys, 
                static_cast<const uint8_t*>(keys.codes), static_cast<const uint8_t*>(keys.scales), keys.rows, n,
                batch, per_cta, w.scores, w.hist);
   }
-  dsv4kv_status st = check_launch("index_score");
-  if (st != DSV4KV_OK) return st;
+  return check_launch("index_score");
+}
+
+dsv4kv_status index_select_launch(int batch, int64_t n, int k, int32_t* idx_out, int32_t* count_out, void* ws,
+                                  size_t ws_bytes, cudaStream_t stream) {
+  if (n <= k) return index_fill_launch(batch, n, k, idx_out, count_out, stream);
+  const IndexWs w = index_ws_layout(static_cast<char*>(ws), batch, n, k);
+  if (ws_bytes < w.bytes) return set_error(DSV4KV_ERR_WORKSPACE, "index_select: workspace too small");
+  const int sms = sm_count();
   // selection: one cluster of C CTAs per sequence, chunks of whole 4096-score batches
   static int max_cluster = 0;
   if (max_cluster == 0) {
@@ -832,6 +867,15 @@ dsv4kv_status index_topk_launch(const uint16_t* qidx, const dsv4kv_cache& keys, 
   launch_pdl_cluster(index_select, dim3(ctas, unsigned(batch)), dim3(kSelThreads), kSelDyn, ctas, stream,
                      (const float*)w.scores, n, k, chunk, w.hist, idx_out, count_out, w.status);
   return check_launch("index_select");
+}
+
+
+dsv4kv_status index_topk_launch(const uint16_t* qidx, const dsv4kv_cache& keys, int batch, int64_t n, int k,
+                                int32_t* idx_out, int32_t* count_out, void* ws, size_t ws_bytes,
+                                cudaStream_t stream) {
+  const dsv4kv_status st = index_score_launch(qidx, keys, batch, n, k, ws, ws_bytes, stream);
+  if (st != DSV4KV_OK) return st;
+  return index_select_launch(batch, n, k, idx_out, count_out, ws, ws_bytes, stream);
 }
 
 }  // namespace dsv4kv

@@ -63,6 +63,10 @@ bool encode_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* bas
 
 size_t index_topk_ws_bytes(int batch, int64_t n, int k);
 size_t index_topk_zero_prefix_bytes(int batch);
+dsv4kv_status index_score_launch(const uint16_t* qidx, const dsv4kv_cache& keys, int batch, int64_t n, int k,
+                                 void* ws, size_t ws_bytes, cudaStream_t stream);
+dsv4kv_status index_select_launch(int batch, int64_t n, int k, int32_t* idx_out, int32_t* count_out, void* ws,
+                                  size_t ws_bytes, cudaStream_t stream);
 dsv4kv_status index_topk_launch(const uint16_t* qidx, const dsv4kv_cache& keys, int batch, int64_t n, int k,
                                 int32_t* idx_out, int32_t* count_out, void* ws, size_t ws_bytes,
                                 cudaStream_t stream);

@@ -138,6 +138,24 @@ dsv4kv_status dsv4kv_index_topk(const void* qidx, const dsv4kv_cache* keys, int3
                                 void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * dsv4kv_index_topk in its two steps, for callers that time or schedule them
+ * apart.  dsv4kv_index_score computes the scores of all n entries ([P2] Step
+ * 5: the learned indexer scores the compressed blocks) and a histogram of
+ * them into `ws`; dsv4kv_index_select then picks the top-k from that
+ * workspace ([P1] "c4a": the top-k entries per query) and leaves it ready for
+ * the next dsv4kv_index_score.  The pair, on one workspace with the same
+ * batch, n and k and nothing else on that workspace in between, is exactly
+ * dsv4kv_index_topk (same arguments, requirements, results and errors).
+ * When n <= k dsv4kv_index_score does nothing and dsv4kv_index_select writes
+ * 0..n-1.  The workspace contents between the two calls are opaque.
+ * ------------------------------------------------------------------------ */
+dsv4kv_status dsv4kv_index_score(const void* qidx, const dsv4kv_cache* keys, int32_t batch,
+                                 int64_t n, int32_t k, void* ws, size_t ws_bytes, void* stream);
+
+dsv4kv_status dsv4kv_index_select(int32_t batch, int64_t n, int32_t k, int32_t* idx_out,
+                                  int32_t* count_out, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * dsv4kv_index_topk without a caller workspace.  The pages have no
  * counterpart: this exists for callers that cannot allocate device memory for
  * a workspace — a serving engine whose memory manager has already reserved

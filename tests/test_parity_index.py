@@ -114,3 +114,22 @@ def test_index_topk_full_size_fp4_sampled():
         qr = OF.bf16_bits_to_f64(D.rows_int_bf16(kq, np.array([s]), 128)[0])
         ref, _ = OI.index_topk(qr, OF.dequant_fp4_rows(hc, hs), k)
         assert np.array_equal(idx[s], ref)
+
+
+@pytest.mark.parametrize("b,n,k", [(2, 300, 512), (3, 5000, 512), (32, 32736, 512)])
+def test_index_score_then_select_equals_index_topk(b, n, k):
+    """The two-step form (dsv4kv_index_score; dsv4kv_index_select) on one
+    workspace gives index_topk's result, call after call."""
+    q, keys, kk, kq = _bf16_keys(300 + n, b, n)
+    cache = K.Cache(0, keys, None, 128)
+    ref_idx, ref_cnt = K.index_topk(q, cache, n, k)
+    ws = K.new_workspace(K.index_topk_workspace_bytes(b, n, k))
+    idx = torch.empty(b, k, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(b, dtype=torch.int32, device="cuda")
+    for _ in range(3):
+        idx.fill_(-7)
+        K.index_score(q, cache, n, k, ws)
+        K.index_select(b, n, k, idx, cnt, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(idx, ref_idx) and torch.equal(cnt, ref_cnt)
+        assert K.workspace_status(ws) == 0
