@@ -381,46 +381,46 @@ __device__ __forceinline__ uint32_t warp_inclusive_scan(uint32_t v) {
 }
 
 // The bin where the descending cumulative count of the 4096-bin histogram h
-// (shared memory) first reaches `need` (1 <= need <= sum h); *above = count in
-// higher bins.  Warp w owns the bins [4096 - S(w+1), 4096 - Sw), S = 4096/warps,
-// and its lanes read consecutive bins from the top (no bank conflicts); the
-// warp that holds the crossing walks its bins 32 at a time with warp scans.
+// (shared memory, 16-byte aligned) first reaches `need` (1 <= need <= sum h);
+// *above = count in higher bins.  Warp w owns the S = 4096/warps highest bins
+// below those of warp w-1; lane l of it owns a contiguous run of PER = S/32
+// bins (highest run on lane 0), read with 16-byte loads.  One warp scan over
+// the lanes' run sums finds the crossing lane, which walks its own run.
 template <int NT>
 __device__ int find_threshold_bin(const uint32_t* h, uint32_t need, uint32_t* above) {
-  constexpr int NW = NT / 32, SPAN = kHistBins / NW, STEPS = SPAN / 32;
-  static_assert(STEPS * 32 * NW == kHistBins, "bins per warp");
+  constexpr int NW = NT / 32, SPAN = kHistBins / NW, PER = SPAN / 32;
+  static_assert(PER % 4 == 0 && PER * 32 * NW == kHistBins, "bins per lane");
   __shared__ uint32_t s_wtot[NW];
   __shared__ int s_bin;
   __shared__ uint32_t s_above;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int top = kHistBins - 1 - SPAN * warp;
-  uint32_t v[STEPS], sum = 0;
+  const int lo = kHistBins - SPAN * warp - PER * (lane + 1);  // lowest bin of this lane's run
+  uint32_t v[PER], sum = 0;
 #pragma unroll
-  for (int j = 0; j < STEPS; ++j) {
-    v[j] = h[top - 32 * j - lane];
-    sum += v[j];
+  for (int q = 0; q < PER / 4; ++q) {
+    const uint4 x = *reinterpret_cast<const uint4*>(h + lo + 4 * q);
+    v[4 * q] = x.x;
+    v[4 * q + 1] = x.y;
+    v[4 * q + 2] = x.z;
+    v[4 * q + 3] = x.w;
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
-  if (lane == 0) s_wtot[warp] = sum;
+  for (int i = 0; i < PER; ++i) sum += v[i];
+  const uint32_t incl = warp_inclusive_scan(sum);  // lane order = descending bins
+  if (lane == 31) s_wtot[warp] = incl;
   __syncthreads();
   uint32_t before = 0;
   for (int w = 0; w < warp; ++w) before += s_wtot[w];
-  if (before < need && before + sum >= need) {  // this warp holds the crossing (warp-uniform)
-    uint32_t c = before;
+  const uint32_t ex = before + incl - sum;  // entries in higher bins than this run
+  if (ex < need && ex + sum >= need) {      // exactly one lane: walk its run from the top
+    uint32_t c = ex;
 #pragma unroll
-    for (int j = 0; j < STEPS; ++j) {
-      const uint32_t incl = warp_inclusive_scan(v[j]);
-      const uint32_t tot = __shfl_sync(kFull, incl, 31);
-      if (c + tot >= need) {
-        const uint32_t ex = c + incl - v[j];
-        if (ex < need && ex + v[j] >= need) {  // exactly one lane
-          s_bin = top - 32 * j - lane;
-          s_above = ex;
-        }
-        break;
+    for (int i = PER - 1; i >= 0; --i) {
+      if (c < need && c + v[i] >= need) {
+        s_bin = lo + i;
+        s_above = c;
       }
-      c += tot;
+      c += v[i];
     }
   }
   __syncthreads();

@@ -133,3 +133,26 @@ def test_index_score_then_select_equals_index_topk(b, n, k):
         torch.cuda.synchronize()
         assert torch.equal(idx, ref_idx) and torch.equal(cnt, ref_cnt)
         assert K.workspace_status(ws) == 0
+
+
+@pytest.mark.parametrize("n_hot", [60, 1000])
+def test_index_topk_hot_entries_with_exact_ties(n_hot):
+    """n_hot evenly spaced entries score far above everything else, all with
+    exactly the same score: with 60 of them the rest of the selection comes
+    from the bulk of the scores; with 1000 the top-k is 512 of the equal hot
+    entries, which the tie rule resolves to the lowest indices."""
+    b, n, k = 2, 40000, 512
+    q, keys, kk, kq = _bf16_keys(4242 + n_hot, b, n, -1, 1)
+    qsign = torch.where(q.float() >= 0, 1.0, -1.0).to(torch.bfloat16)
+    hot = [(j * n) // 1024 for j in range(n_hot)]
+    assert n_hot <= 1024 and max(hot) < n
+    pos = torch.tensor(hot, device="cuda")
+    for s in range(b):
+        keys[s, pos] = 8 * qsign[s]
+    idx, cnt = K.index_topk(q, K.Cache(0, keys, None, 128), n, k)
+    qh = q.float().cpu().double().numpy()
+    kh = keys.float().cpu().double().numpy()
+    for s in range(b):
+        ref_idx, ref_cnt = OI.index_topk(qh[s], kh[s], k)
+        assert np.array_equal(idx[s].cpu().numpy(), ref_idx), f"seq {s}"
+        assert int(cnt[s]) == ref_cnt
