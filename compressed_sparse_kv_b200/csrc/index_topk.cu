@@ -163,31 +163,15 @@ __global__ void __launch_bounds__(256) index_score_bf16(const uint16_t* __restri
   }
 }
 
-// fp4 keys, dim 128: codes 64 B + 8 E4M3 scale bytes per key.  A quarter warp
-// (4 lanes x 16 B) covers one key; each lane holds 32 channels = 2 scale
-// groups.  E2M1 codes are decoded to packed f16 pairs with byte permutes
-// (a PRMT table of the eight magnitudes) and the sign bit OR-ed in; each
-// 16-channel group is accumulated with packed f16 FMAs (exact for integer
-// queries: |partial| <= 16*8*6 = 768 at a resolution of 0.5 needs 11 bits)
-// and the group sum is scaled in fp32.
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
-}
-// High bytes of the f16 encodings of 0, .5, 1, 1.5, 2, 3, 4, 6.
-constexpr uint32_t kE2M1HiLo = 0x3E3C3800u;  // codes 3..0
-constexpr uint32_t kE2M1HiHi = 0x46444240u;  // codes 7..4
-
-// Decode the 8 nibbles of w into four f16x2: out[i] = (nibble i, nibble i+4).
-__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&out)[4]) {
-  const uint32_t mlo = prmt(kE2M1HiLo, kE2M1HiHi, w & 0x7777u);          // mags of nibbles 0..3
-  const uint32_t mhi = prmt(kE2M1HiLo, kE2M1HiHi, (w >> 16) & 0x7777u);  // mags of nibbles 4..7
-  // selector nibble 8 (sign-replicate of a byte whose top bit is 0) yields 0x00
-  out[0] = prmt(mlo, mhi, 0x4808u) | ((w << 12) & 0x80008000u);
-  out[1] = prmt(mlo, mhi, 0x5818u) | ((w << 8) & 0x80008000u);
-  out[2] = prmt(mlo, mhi, 0x6828u) | ((w << 4) & 0x80008000u);
-  out[3] = prmt(mlo, mhi, 0x7838u) | (w & 0x80008000u);
+// The four code bytes of w (byte 0 = lowest) decoded to four f16x2 pairs by
+// cvt.rn.f16x2.e2m1x2 straight from the unpacked bytes (no shifts or masks);
+// each pair holds (low nibble, high nibble) = (even, odd) channel.
+__device__ __forceinline__ void e2m1x8_unpack(uint32_t w, uint32_t (&h)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(w));
 }
 
 __device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
@@ -254,11 +238,12 @@ __device__ __forceinline__ void score_segment_fp4(const uint16_t* __restrict__ q
       uint32_t acc0 = 0, acc1 = 0;  // f16x2 sums of group 0 (words 0, 1) and group 1 (words 2, 3)
 #pragma unroll
       for (int wi = 0; wi < 4; ++wi) {
+        uint32_t h[4];
+        e2m1x8_unpack(w[wi], h);
 #pragma unroll
         for (int by = 0; by < 4; ++by) {
-          const uint32_t h = e2m1x2_to_f16x2((w[wi] >> (8 * by)) & 0xffu);
-          if (wi < 2) acc0 = hfma2(qp[4 * wi + by], h, acc0);
-          else acc1 = hfma2(qp[4 * wi + by], h, acc1);
+          if (wi < 2) acc0 = hfma2(qp[4 * wi + by], h[by], acc0);
+          else acc1 = hfma2(qp[4 * wi + by], h[by], acc1);
         }
       }
       p[u] = f16x2_sum(acc0) * e4m3_to_f32(s2[u] & 0xffu) + f16x2_sum(acc1) * e4m3_to_f32(s2[u] >> 8);
