@@ -245,6 +245,31 @@ __device__ __forceinline__ float p_hi(uint32_t v, bool f16) {
   return f;
 }
 
+// Writes channel tiles [ct0, ct1) of the CTA's partial O^T (TMEM lanes of
+// quarter wq, i.e. channels 128ct + 32wq + lane) to o_part, heads as rows.
+// The epilogue warps and the loader warps that share a lane quarter each
+// write half of the channel tiles.
+__device__ __forceinline__ void store_partial(const Params& p, int b, int split, uint32_t tmem, int wq, int lane,
+                                              int ct0, int ct1) {
+  const uint32_t lane_base = uint32_t(32 * wq) << 16;
+  float* op = p.o_part + (size_t(b) * p.splits + split) * size_t(p.heads) * kDim;
+#pragma unroll 1
+  for (int ct = ct0; ct < ct1; ++ct) {
+    const int c = 128 * ct + 32 * wq + lane;
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+      uint32_t o[32];
+      tmem_ld32(tmem + lane_base + kColO + 64 * ct + 32 * half, o);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int hh = 32 * half + e;
+        if (hh < p.heads) op[size_t(hh) * kDim + c] = __uint_as_float(o[e]);
+      }
+    }
+  }
+}
+
 template <int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_comp,
@@ -547,24 +572,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       l_tot[hh] += __shfl_xor_sync(kFull, l_tot[hh], 2);
     }
     if (p.splits > 1) {
-      if (!dead) {
+      if (!dead) {  // channel tiles 0-1; the loader warp of the same lane quarter writes 2-3
         tc_fence_after();
-        float* op = p.o_part + (size_t(b) * p.splits + split) * size_t(p.heads) * kDim;
-#pragma unroll 1
-        for (int ct = 0; ct < kDim / 128; ++ct) {
-          const int c = 128 * ct + 32 * wq + lane;
-#pragma unroll 1
-          for (int half = 0; half < 2; ++half) {
-            uint32_t o[32];
-            tmem_ld32(tmem + lane_base + kColO + 64 * ct + 32 * half, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int hh = 32 * half + e;
-              if (hh < p.heads) op[size_t(hh) * kDim + c] = __uint_as_float(o[e]);
-            }
-          }
-        }
+        store_partial(p, b, split, tmem, wq, lane, 0, kDim / 256);
       }
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
@@ -718,6 +728,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->full[stage]);
     }
+    // the other half of the partial O^T (this warp's TMEM lane quarter is warp % 4)
+    if (p.splits > 1 && warp_wait(&ctl->o_done, 0, ctl, lane)) {
+      tc_fence_after();
+      store_partial(p, b, split, tmem, warp & 3, lane, kDim / 256, kDim / 128);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -736,6 +751,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // lane; lane s also owns split s's (m, l) terms, which the warp shares by
 // shuffles.  The split loop's loads do not depend on each other.
 constexpr int kCombWarps = 4;
+constexpr int kCombFast = 4;  // splits up to which a warp issues all its loads at once
 
 __global__ void __launch_bounds__(32 * kCombWarps) decode_combine(const float* __restrict__ o_part,
                                                                   const float* __restrict__ ml_part,
@@ -751,43 +767,90 @@ __global__ void __launch_bounds__(32 * kCombWarps) decode_combine(const float* _
   const size_t ml_stride = size_t(heads) * 4, o_stride = size_t(heads) * kDim;
   const float* mlb = ml_part + (size_t(b) * splits * heads + h) * 4;
   const float* ob = o_part + (size_t(b) * splits * heads + h) * kDim + 4 * lane;
-  float mo = -INFINITY, ml = -INFINITY;
-  for (int s = lane; s < splits; s += 32) {
-    const float4 v = __ldcg(reinterpret_cast<const float4*>(mlb + s * ml_stride));
-    mo = fmaxf(mo, v.x);
-    ml = fmaxf(ml, v.y);
-  }
+  // the rotation of this lane's rotary pairs (channels 128q + 4 lane + {0, 2}), read up front
+  const int r0 = kDim - rope_dim;
+  float cs[4][2], sn[4][2];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    mo = fmaxf(mo, __shfl_xor_sync(kFull, mo, o));
-    ml = fmaxf(ml, __shfl_xor_sync(kFull, ml, o));
-  }
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int c = 128 * q + 4 * lane + 2 * e;
+      const bool rot = c >= r0;
+      cs[q][e] = rot ? __ldcg(rope_tab + ((c - r0) >> 1)) : 1.f;
+      sn[q][e] = rot ? __ldcg(rope_tab + kDim / 2 + ((c - r0) >> 1)) : 0.f;
+    }
   float4 acc[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-  float L = 0.f;
-  for (int s0 = 0; s0 < splits; s0 += 32) {
-    float w = 0.f;
-    if (s0 + lane < splits) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(mlb + (s0 + lane) * ml_stride));
-      w = v.x == -INFINITY ? 0.f : exp2f(v.x - mo);
-      if (v.y != -INFINITY) L += v.z * exp2f(v.y - ml);
-    }
-    const int cnt = min(32, splits - s0);
-#pragma unroll 4
-    for (int j = 0; j < cnt; ++j) {
-      const float wj = __shfl_sync(kFull, w, j);
-      const float* os = ob + size_t(s0 + j) * o_stride;
-      float4 v[4];
+  float mo = -INFINITY, ml = -INFINITY, L = 0.f;
+  if (splits <= kCombFast) {
+    // every load of the warp in one round trip: lane s holds split s's (m, l),
+    // every lane its 16 channels of each split
+    const float4 v = lane < splits ? __ldcg(reinterpret_cast<const float4*>(mlb + lane * ml_stride))
+                                   : make_float4(-INFINITY, -INFINITY, 0.f, 0.f);
+    float4 x[kCombFast][4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) v[q] = __ldcg(reinterpret_cast<const float4*>(os + 128 * q));
-      if (wj != 0.f) {  // an empty partial's O is never read
+    for (int s = 0; s < kCombFast; ++s)
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        x[s][q] = s < splits ? __ldcg(reinterpret_cast<const float4*>(ob + size_t(s) * o_stride + 128 * q))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+    mo = v.x;
+    ml = v.y;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mo = fmaxf(mo, __shfl_xor_sync(kFull, mo, o));
+      ml = fmaxf(ml, __shfl_xor_sync(kFull, ml, o));
+    }
+    const float w = v.x == -INFINITY ? 0.f : exp2f(v.x - mo);
+    L = v.y == -INFINITY ? 0.f : v.z * exp2f(v.y - ml);
+#pragma unroll
+    for (int s = 0; s < kCombFast; ++s) {
+      const float ws = __shfl_sync(kFull, w, s);
+      if (ws != 0.f) {  // an empty partial's O is never read (lanes >= splits carry w = 0)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          acc[q].x = fmaf(wj, v[q].x, acc[q].x);
-          acc[q].y = fmaf(wj, v[q].y, acc[q].y);
-          acc[q].z = fmaf(wj, v[q].z, acc[q].z);
-          acc[q].w = fmaf(wj, v[q].w, acc[q].w);
+          acc[q].x = fmaf(ws, x[s][q].x, acc[q].x);
+          acc[q].y = fmaf(ws, x[s][q].y, acc[q].y);
+          acc[q].z = fmaf(ws, x[s][q].z, acc[q].z);
+          acc[q].w = fmaf(ws, x[s][q].w, acc[q].w);
+        }
+      }
+    }
+  } else {
+    for (int s = lane; s < splits; s += 32) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(mlb + s * ml_stride));
+      mo = fmaxf(mo, v.x);
+      ml = fmaxf(ml, v.y);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mo = fmaxf(mo, __shfl_xor_sync(kFull, mo, o));
+      ml = fmaxf(ml, __shfl_xor_sync(kFull, ml, o));
+    }
+    for (int s0 = 0; s0 < splits; s0 += 32) {
+      float w = 0.f;
+      if (s0 + lane < splits) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(mlb + (s0 + lane) * ml_stride));
+        w = v.x == -INFINITY ? 0.f : exp2f(v.x - mo);
+        if (v.y != -INFINITY) L += v.z * exp2f(v.y - ml);
+      }
+      const int cnt = min(32, splits - s0);
+#pragma unroll 4
+      for (int j = 0; j < cnt; ++j) {
+        const float wj = __shfl_sync(kFull, w, j);
+        const float* os = ob + size_t(s0 + j) * o_stride;
+        float4 v[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) v[q] = __ldcg(reinterpret_cast<const float4*>(os + 128 * q));
+        if (wj != 0.f) {  // an empty partial's O is never read
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            acc[q].x = fmaf(wj, v[q].x, acc[q].x);
+            acc[q].y = fmaf(wj, v[q].y, acc[q].y);
+            acc[q].z = fmaf(wj, v[q].z, acc[q].z);
+            acc[q].w = fmaf(wj, v[q].w, acc[q].w);
+          }
         }
       }
     }
@@ -795,21 +858,16 @@ __global__ void __launch_bounds__(32 * kCombWarps) decode_combine(const float* _
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(kFull, L, o);
   const float inv = (mo == -INFINITY || L <= 0.f) ? 0.f : exp2f(mo - ml) / L;
-  const int r0 = kDim - rope_dim;
   const size_t ob_out = (size_t(b) * heads + h) * kDim;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int c = 128 * q + 4 * lane;
     float v[4] = {acc[q].x * inv, acc[q].y * inv, acc[q].z * inv, acc[q].w * inv};
 #pragma unroll
-    for (int e = 0; e < 4; e += 2) {
-      if (c + e >= r0) {
-        const int m = (c + e - r0) >> 1;
-        const float cs = __ldcg(rope_tab + m), sn = __ldcg(rope_tab + kDim / 2 + m);
-        const float x = v[e], y = v[e + 1];
-        v[e] = x * cs - y * sn;
-        v[e + 1] = x * sn + y * cs;
-      }
+    for (int e = 0; e < 2; ++e) {  // identity rotation outside the rotary channels
+      const float x = v[2 * e], y = v[2 * e + 1];
+      v[2 * e] = x * cs[q][e] - y * sn[q][e];
+      v[2 * e + 1] = x * sn[q][e] + y * cs[q][e];
     }
     if (out_fp32) {
       *reinterpret_cast<float4*>(static_cast<float*>(out) + ob_out + c) = make_float4(v[0], v[1], v[2], v[3]);

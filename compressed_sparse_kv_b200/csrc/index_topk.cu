@@ -31,9 +31,20 @@ constexpr int kHistBins = 4096;  // 12-bit digits
 // Transposing butterfly: lane l16 of a 16-lane group holds U partial sums
 // (one per key); after log2 steps each lane holds the full 16-lane sum of one
 // key.  U = 16: key l16 (15 shuffles for 16 keys).  U = 8: key (l16 >> 1) & 7,
-// duplicated on lanes 2i and 2i+1 (8 shuffles for 8 keys).
+// duplicated on lanes 2i and 2i+1 (8 shuffles for 8 keys).  U = 4: key
+// (l16 >> 2) & 3 on lanes 4i..4i+3 (4 shuffles for 4 keys).
 template <int U>
 __device__ __forceinline__ float reduce16_transposed(const float (&p)[U], int l16) {
+  if constexpr (U == 4) {
+    const bool b3 = l16 & 8, b2 = l16 & 4;
+    float c[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) c[i] = (b3 ? p[2 + i] : p[i]) + __shfl_xor_sync(kFull, b3 ? p[i] : p[2 + i], 8);
+    float s = (b2 ? c[1] : c[0]) + __shfl_xor_sync(kFull, b2 ? c[0] : c[1], 4);
+    s += __shfl_xor_sync(kFull, s, 2);
+    return s + __shfl_xor_sync(kFull, s, 1);
+  }
+  static_assert(U == 8 || U == 16 || U == 4, "keys per half-warp");
   float a[8], c[4], d[2];
   if constexpr (U == 16) {
     const bool b3 = l16 & 8;
@@ -79,8 +90,8 @@ __device__ __forceinline__ void score_segment_bf16(const uint16_t* __restrict__ 
                                                    int64_t cnt, float* sc, float* ssc, uint32_t* sh, uint64_t pol) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int half = lane >> 4, l16 = lane & 15;
-  const int my_key = U == 16 ? l16 : ((l16 >> 1) & 7);
-  const bool writer = U == 16 || !(lane & 1);
+  const int my_key = U == 16 ? l16 : (U == 8 ? ((l16 >> 1) & 7) : ((l16 >> 2) & 3));
+  const bool writer = U == 16 || (U == 8 ? !(lane & 1) : !(lane & 3));
   float q[8];
   {
     const uint4 v = *reinterpret_cast<const uint4*>(qrow + 8 * l16);
