@@ -878,6 +878,106 @@ __global__ void __launch_bounds__(32 * kCombWarps) decode_combine(const float* _
   }
 }
 
+// The same merge for many splits: one block of kWideWarps warps per
+// (sequence, head); warp w takes splits w, w + kWideWarps, ...; lanes own 16
+// channels (4 float4); the warps' sums meet in shared memory (rows of 512
+// channels, lane-contiguous float4s: no bank conflicts) and thread t
+// finishes channels 2t, 2t+1 (a rotary pair).
+constexpr int kWideWarps = 8;
+
+__global__ void __launch_bounds__(32 * kWideWarps) decode_combine_wide(const float* __restrict__ o_part,
+                                                                       const float* __restrict__ ml_part,
+                                                                       const float* __restrict__ rope_tab, int splits,
+                                                                       int heads, int rope_dim, int out_fp32,
+                                                                       void* __restrict__ out) {
+  __shared__ __align__(16) float red[kWideWarps][kDim];
+  __shared__ float s_mo[kWideWarps], s_ml[kWideWarps], s_l[kWideWarps];
+  pdl_trigger();
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x / heads, h = blockIdx.x % heads;
+  const size_t ml_stride = size_t(heads) * 4, o_stride = size_t(heads) * kDim;
+  const float* mlb = ml_part + (size_t(b) * splits * heads + h) * 4;
+  const float* ob = o_part + (size_t(b) * splits * heads + h) * kDim + 4 * lane;
+  // maxima over all splits
+  float mo = -INFINITY, ml = -INFINITY;
+  for (int s = threadIdx.x; s < splits; s += 32 * kWideWarps) {
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(mlb + s * ml_stride));
+    mo = fmaxf(mo, v.x);
+    ml = fmaxf(ml, v.y);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mo = fmaxf(mo, __shfl_xor_sync(kFull, mo, o));
+    ml = fmaxf(ml, __shfl_xor_sync(kFull, ml, o));
+  }
+  if (lane == 0) {
+    s_mo[warp] = mo;
+    s_ml[warp] = ml;
+  }
+  __syncthreads();
+  mo = s_mo[0];
+  ml = s_ml[0];
+#pragma unroll
+  for (int w = 1; w < kWideWarps; ++w) {
+    mo = fmaxf(mo, s_mo[w]);
+    ml = fmaxf(ml, s_ml[w]);
+  }
+  // this warp's splits
+  float4 acc[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float L = 0.f;
+#pragma unroll 2
+  for (int s = warp; s < splits; s += kWideWarps) {
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(mlb + s * ml_stride));
+    float4 x[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) x[q] = __ldcg(reinterpret_cast<const float4*>(ob + size_t(s) * o_stride + 128 * q));
+    if (v.y != -INFINITY) L += v.z * exp2f(v.y - ml);
+    const float w = v.x == -INFINITY ? 0.f : exp2f(v.x - mo);
+    if (w != 0.f) {  // an empty partial's O is never read
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc[q].x = fmaf(w, x[q].x, acc[q].x);
+        acc[q].y = fmaf(w, x[q].y, acc[q].y);
+        acc[q].z = fmaf(w, x[q].z, acc[q].z);
+        acc[q].w = fmaf(w, x[q].w, acc[q].w);
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) *reinterpret_cast<float4*>(&red[warp][128 * q + 4 * lane]) = acc[q];
+  if (lane == 0) s_l[warp] = L;  // every lane carries the same L
+  __syncthreads();
+  float Lt = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWideWarps; ++w) Lt += s_l[w];
+  const float inv = (mo == -INFINITY || Lt <= 0.f) ? 0.f : exp2f(mo - ml) / Lt;
+  const int c = 2 * threadIdx.x;  // 256 threads x 2 channels
+  float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWideWarps; ++w) {
+    const float2 x = *reinterpret_cast<const float2*>(&red[w][c]);
+    v0 += x.x;
+    v1 += x.y;
+  }
+  v0 *= inv;
+  v1 *= inv;
+  const int r0 = kDim - rope_dim;
+  if (c >= r0) {
+    const int m = (c - r0) >> 1;
+    const float cs = __ldcg(rope_tab + m), sn = __ldcg(rope_tab + kDim / 2 + m);
+    const float x = v0, y = v1;
+    v0 = x * cs - y * sn;
+    v1 = x * sn + y * cs;
+  }
+  const size_t o = (size_t(b) * heads + h) * kDim + c;
+  if (out_fp32) *reinterpret_cast<float2*>(static_cast<float*>(out) + o) = make_float2(v0, v1);
+  else static_cast<uint32_t*>(out)[o / 2] = pack_bf16x2(v0, v1);
+}
+static_assert(2 * 32 * kWideWarps == kDim, "two channels per thread");
+
 struct Plan {
   int comp_tiles, tiles, splits, tiles_per_split;
 };
@@ -1016,9 +1116,14 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
   }
   if (st != DSV4KV_OK || pl.splits == 1) return st;  // one split: the decode kernel stored the output
   const int bh_total = a.batch * a.heads;
-  launch_pdl(decode_combine, dim3((bh_total + kCombWarps - 1) / kCombWarps), dim3(32 * kCombWarps), 0, stream,
-             (const float*)w.o_part, (const float*)w.ml_part, (const float*)w.rope_tab, pl.splits, a.heads, bh_total,
-             a.rope_dim, a.out_fp32, a.out);
+  if (pl.splits <= kCombFast)
+    launch_pdl(decode_combine, dim3((bh_total + kCombWarps - 1) / kCombWarps), dim3(32 * kCombWarps), 0, stream,
+               (const float*)w.o_part, (const float*)w.ml_part, (const float*)w.rope_tab, pl.splits, a.heads,
+               bh_total, a.rope_dim, a.out_fp32, a.out);
+  else
+    launch_pdl(decode_combine_wide, dim3(bh_total), dim3(32 * kWideWarps), 0, stream, (const float*)w.o_part,
+               (const float*)w.ml_part, (const float*)w.rope_tab, pl.splits, a.heads, a.rope_dim, a.out_fp32,
+               a.out);
   return check_launch("decode_combine");
 }
 
