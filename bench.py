@@ -4,8 +4,9 @@
 A step is one decode step of one layer for the whole batch: for the c4a
 layer (the default workload) dsv4kv_index_topk followed by
 dsv4kv_sparse_decode; for the c128a layer dsv4kv_dense_decode.  The caches
-are resident in HBM (a KV cache is state, not a per-step input); two input
-replicas alternate so every step streams from DRAM rather than L2.
+are resident in HBM (a KV cache is state, not a per-step input); the steps
+cycle through enough cache replicas that the bytes read between two reads of
+one replica exceed twice the L2, so every step streams from DRAM.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -40,6 +41,7 @@ WORKLOADS = {
     "q_c128a_fp4": ("c128a", 64, 262144, 64, 2, 0),
 }
 FMT_NAME = {0: "bf16", 1: "fp8", 2: "fp4"}
+L2_BYTES = 126 * 2 ** 20
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
 # capture of that kernel in this workload (profiles/ holds the summary and the
 # command); cleared whenever the kernel changes
@@ -113,6 +115,25 @@ ROW_BYTES = {0: 1024, 1: 516, 2: 288}     # one 512-channel cache row: bf16, fp8
 KEY_BYTES = {0: 256, 2: 72}               # one 128-channel indexer key: bf16, fp4 + scales
 
 
+def step_bytes(kind, batch, t, main_fmt, index_fmt, k=512, window=128):
+    """Algorithmic bytes one step reads from one cache replica: indexer keys
+    (c4a) + the attended rows.  Queries and outputs are excluded."""
+    n = (t - window) // (4 if kind == "c4a" else 128)
+    rows = (k + window) if kind == "c4a" else (n + window)
+    b = batch * rows * ROW_BYTES[main_fmt]
+    if kind == "c4a":
+        b += batch * n * KEY_BYTES[index_fmt]
+    return b
+
+
+def replicas_for(kind, batch, t, main_fmt, index_fmt, at_least):
+    """Cache replicas the timed steps cycle through: enough that the bytes
+    read between two reads of the same replica exceed twice the L2, so every
+    step streams its rows from DRAM."""
+    per = step_bytes(kind, batch, t, main_fmt, index_fmt)
+    return max(at_least, -(-2 * L2_BYTES // per))
+
+
 class Layer:
     """One layer's resident caches (R replicas) and per-step buffers on the GPU."""
 
@@ -174,11 +195,7 @@ class Layer:
 
     # algorithmic bytes of one step: indexer keys + rows read (queries/outputs excluded)
     def alg_bytes(self):
-        rows = (self.k + self.window) if self.kind == "c4a" else (self.n + self.window)
-        b = self.batch * rows * ROW_BYTES[self.main_fmt]
-        if self.kind == "c4a":
-            b += self.batch * self.n * KEY_BYTES[self.index_fmt]
-        return b
+        return step_bytes(self.kind, self.batch, self.t, self.main_fmt, self.index_fmt, self.k, self.window)
 
     def index_bytes(self):
         return self.batch * self.n * KEY_BYTES[self.index_fmt] + self.batch * 256
@@ -277,7 +294,7 @@ def time_stack(steps, warmup, seed, dist_max):
 
 
 def time_bulk(seed):
-    """Bulk throughput of the compressor and the quantiser."""
+    """Bulk throughput of the c4a / c128a compressors and the fp8 / fp4 quantiser."""
     import torch
     import compressed_sparse_kv_b200 as K
     import datagen as D
@@ -326,36 +343,42 @@ def time_layer(layer, steps, warmup, dist_max, dev_index, sample_clocks):
     torch = layer.torch
     R = len(layer.reps)
     stream = torch.cuda.Stream()
+    # one full cycle over the replicas first, so no replica is still in L2
+    # from its creation; every graph then continues the cycle where the
+    # previous one stopped
+    n_eager = max(warmup, R)
     with torch.cuda.stream(stream):
-        for i in range(max(warmup, 1)):
+        for i in range(n_eager):
             layer.step(i % R)
     stream.synchronize()
     # external=True: records inside the capture become event nodes of the graph
     ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(steps)]
 
-    def capture(n_steps, events):
+    def capture(first, n_steps, events):
         # events: step start | after index_score | after index_select | after decode
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for i in range(n_steps):
+                r = (first + i) % R
                 if events:
                     events[i][0].record(stream)
                 if layer.kind == "c4a":
-                    layer.index_score(i % R)
+                    layer.index_score(r)
                 if events:
                     events[i][1].record(stream)
                 if layer.kind == "c4a":
                     layer.index_select()
                 if events:
                     events[i][2].record(stream)
-                layer.decode(i % R)
+                layer.decode(r)
                 if events:
                     events[i][3].record(stream)
         return g
 
-    g_warm = capture(max(warmup, 1), None)
-    g_main = capture(steps, None)
-    g_inst = capture(steps, ev)
+    n_warm = max(warmup, 1)
+    g_warm = capture(n_eager, n_warm, None)
+    g_main = capture(n_eager + n_warm, steps, None)
+    g_inst = capture(n_eager + n_warm + steps, steps, ev)
     with torch.cuda.stream(stream):
         g_warm.replay()
     stream.synchronize()
@@ -543,7 +566,7 @@ def main():
                     help="extra per-layer-type workloads (comma list, 'none' = none)")
     ap.add_argument("--no-stack", action="store_true", help="skip the 61-layer stack step")
     ap.add_argument("--no-bulk", action="store_true", help="skip compressor/quantiser throughput")
-    ap.add_argument("--replicas", type=int, default=2)
+    ap.add_argument("--replicas", type=int, default=2, help="minimum cache replicas (raised until they exceed 2x L2)")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -580,7 +603,8 @@ def main():
     torch.cuda.set_device(d["local"])
     hbm_peak, tf_peak, peak_src = measured_peaks()
     seed = 1234 + d["rank"]
-    layer = Layer(kind, batch, t, heads, seed, args.replicas, mfmt, ifmt)
+    reps = replicas_for(kind, batch, t, mfmt, ifmt, args.replicas)
+    layer = Layer(kind, batch, t, heads, seed, reps, mfmt, ifmt)
     res = time_layer(layer, args.steps, args.warmup, dist_max, d["local"], sample_clocks=(d["rank"] == 0))
     ms = res["total_ms"] / args.steps
     steps_per_s = d["world"] * 1e3 / ms            # whole job: every rank ran `steps` steps
@@ -611,13 +635,13 @@ def main():
                        "select_ms": round(res["select_ms"], 5), "decode_ms": round(res["decode_ms"], 5)}}
     for name in [s for s in args.secondary.split(",") if s and s not in ("none", args.workload)]:
         spec = WORKLOADS[name]
-        big = spec[1] * spec[2] >= 2 ** 22
-        L2 = Layer(*spec[:4], seed + 99, 2 if big else 4, spec[4], spec[5])
+        r2n = replicas_for(spec[0], spec[1], spec[2], spec[4], spec[5], 2)
+        L2 = Layer(*spec[:4], seed + 99, r2n, spec[4], spec[5])
         r2 = time_layer(L2, args.steps, args.warmup, dist_max, d["local"], sample_clocks=False)
         ms2 = r2["total_ms"] / args.steps
         a2 = L2.alg_bytes()
         per_type[name] = {"workload": wl_desc(*spec), "steps_per_s": round(d["world"] * 1e3 / ms2, 1),
-                          "us_per_step": round(ms2 * 1e3, 2),
+                          "us_per_step": round(ms2 * 1e3, 2), "cache_replicas": r2n,
                           "hbm_gbs": round(a2 / (ms2 * 1e-3) / 1e9, 1),
                           "frac_of_measured_hbm": round(a2 / (ms2 * 1e-3) / 1e9 / hbm_peak, 4),
                           "tflops": round(L2.flops() / (ms2 * 1e-3) / 1e12, 1),
@@ -637,7 +661,8 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": FMT_NAME[mfmt], "data": "synthetic",
             "config": {"workload": wl_name, "batch_per_gpu": batch, "context": t, "heads": heads,
                        "parallelism": f"dp{d['world']}",
-                       "l2": f"{args.replicas} cache replicas alternate; {alg / 1e6:.0f} MB read per step (> 126 MB L2)"},
+                       "l2": f"inputs larger than L2: {reps} cache replicas cycle, {alg / 1e6:.0f} MB read per step, "
+                             f"{reps * alg / 1e6:.0f} MB between two reads of one replica (L2 126 MB)"},
             "hbm_gbs": round(alg / (ms * 1e-3) / 1e9, 1), "alg_bytes_per_step": alg,
             "per_layer_type": per_type, "roofline": roof,
             "e2e": {"value": round(e2e_v, 2), "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
