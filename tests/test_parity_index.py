@@ -31,6 +31,7 @@ def _bf16_keys(seed, b, n, lo=-8, hi=8, rows=None):
     (1, 70000, 70000, 64),
     (2, 9000, 9000, 1),
     (2, 9000, 9000, 2048),
+    (150, 1000, 1003, 512),    # many short sequences: a CTA's keys span several sequences
 ])
 def test_index_topk_bf16_small(b, n, rows, k):
     q, keys, kk, kq = _bf16_keys(100 + n + k, b, n, rows=rows)
