@@ -427,15 +427,19 @@ __global__ void __launch_bounds__(256) index_score_fp4(const uint16_t* __restric
 // what is missing; an ordered compaction writes the result in ascending index
 // order.  It re-zeroes the sequence's histogram for the next call.
 constexpr int kSelThreads = 512;
-constexpr int kSelBatch = 8;                           // scores per thread and batch
-constexpr int kSelBatchSpan = kSelThreads * kSelBatch;  // 4096 scores per CTA batch
+constexpr int kSelBatch = 8;                           // scores per lane and warp batch
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelWarpSpan = 32 * kSelBatch;           // 256 scores per warp batch
+constexpr int kSelChunkUnit = 4096;                    // CTA chunks are multiples of this
 constexpr int kSelStage = 4096;                        // candidates a CTA can hold
 constexpr int kCandCap = 8192;                         // candidates per sequence the leader can resolve
 constexpr int kResPer = kCandCap / kSelThreads;        // candidates per leader thread
 constexpr int kTieCap = 2048;
 constexpr int kMaxClusterSel = 16;
-constexpr size_t kSelDyn = size_t(kSelStage) * sizeof(uint64_t);
-static_assert(kTieCap * (sizeof(uint64_t) + sizeof(uint32_t)) <= kSelDyn, "the tie list reuses the list area");
+constexpr int kWarpCap = kSelStage / kSelWarps;       // candidates a warp's list can hold
+// dynamic shared memory: the CTA's list (kSelStage) + the warps' lists (kSelStage)
+constexpr size_t kSelDyn = 2 * size_t(kSelStage) * sizeof(uint64_t);
+static_assert(kTieCap * (sizeof(uint64_t) + sizeof(uint32_t)) <= kSelDyn / 2, "the tie list reuses the list area");
 
 // Block-wide exclusive prefix sum of one value per thread (NT threads).
 template <int NT>
@@ -575,40 +579,37 @@ __device__ __forceinline__ void load_histogram(const uint32_t* __restrict__ hb, 
   for (int j = 0; j < V; ++j) reinterpret_cast<uint4*>(sh)[threadIdx.x + j * NT] = v[j];
 }
 
-template <int NT, int BATCH>
-__device__ __forceinline__ void load_codes(const float* __restrict__ sc, int64_t base, int64_t end,
-                                           uint32_t (&o)[BATCH]) {
+// One warp batch of score codes: lane l takes positions base + 32 v + l.
+__device__ __forceinline__ void warp_load_codes(const float* __restrict__ sc, int64_t base, int64_t end,
+                                                uint32_t (&o)[kSelBatch]) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int j = 0; j < BATCH; ++j) {
-    const int64_t i = base + int64_t(j) * NT + threadIdx.x;
-    o[j] = i < end ? ord_f32(__ldcg(sc + i)) : 0u;
+  for (int v = 0; v < kSelBatch; ++v) {
+    const int64_t i = base + 32 * v + lane;
+    o[v] = i < end ? ord_f32(__ldcg(sc + i)) : 0u;
   }
 }
 
-// Appends, in index order, the batch's entries whose top-12-bit bin is
-// >= bin1 to the CTA's list (u64 = code << 32 | ~index) after `count`
-// entries; returns the new count (entries beyond kSelStage are counted, not
-// stored).
-__device__ __forceinline__ uint32_t stage_batch(const uint32_t (&o)[kSelBatch], int64_t base, int64_t end, int bin1,
-                                                uint32_t count, uint64_t* list) {
+// Appends, in index order, the warp batch's entries whose top-12-bit bin is
+// >= bin1 to the warp's list (u64 = code << 32 | ~index) after `count`
+// entries; returns the new count (entries beyond kWarpCap are counted, not
+// stored).  Warp-synchronous: ballots give the order, no block barrier.
+__device__ __forceinline__ uint32_t warp_stage_batch(const uint32_t (&o)[kSelBatch], int64_t base, int64_t end,
+                                                     int bin1, uint32_t count, uint64_t* list) {
   const int lane = threadIdx.x & 31;
-  uint32_t m[kSelBatch], off[kSelBatch];
-#pragma unroll
-  for (int j = 0; j < kSelBatch; ++j) {
-    const int64_t i = base + int64_t(j) * kSelThreads + threadIdx.x;
-    m[j] = __ballot_sync(kFull, i < end && int(o[j] >> 20) >= bin1);
-  }
-  const uint32_t total = ordered_offsets<kSelThreads, kSelBatch>(m, off);
   const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll
-  for (int j = 0; j < kSelBatch; ++j) {
-    if ((m[j] >> lane) & 1u) {
-      const uint32_t at = count + off[j] + __popc(m[j] & lt);
-      const int64_t i = base + int64_t(j) * kSelThreads + threadIdx.x;
-      if (at < uint32_t(kSelStage)) list[at] = (uint64_t(o[j]) << 32) | uint64_t(0xffffffffu - uint32_t(i));
+  for (int v = 0; v < kSelBatch; ++v) {
+    const int64_t i = base + 32 * v + lane;
+    const bool keep = i < end && int(o[v] >> 20) >= bin1;
+    const uint32_t m = __ballot_sync(kFull, keep);
+    if (keep) {
+      const uint32_t at = count + __popc(m & lt);
+      if (at < uint32_t(kWarpCap)) list[at] = (uint64_t(o[v]) << 32) | uint64_t(0xffffffffu - uint32_t(i));
     }
+    count += __popc(m);
   }
-  return count + total;
+  return count;
 }
 
 // Exact selection with no candidate list (overflow, or more than kTieCap
@@ -662,13 +663,15 @@ __device__ void select_by_scan(const float* __restrict__ sc, int64_t n, uint32_t
   if (threadIdx.x == 0 && s_gt_seen + min(s_eq_seen, r_eq) != kk) set_status(status, DSV4KV_DEV_INCONSISTENT);
 }
 
-__global__ void __launch_bounds__(kSelThreads) index_select(const float* __restrict__ scores, int64_t n, int k,
+__global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __restrict__ scores, int64_t n, int k,
                                                             int64_t chunk, uint32_t* __restrict__ hist,
                                                             int32_t* __restrict__ idx_out,
                                                             int32_t* __restrict__ count_out,
                                                             uint32_t* __restrict__ status,
                                                             uint32_t* __restrict__ tail_ctr) {
-  extern __shared__ __align__(16) uint64_t stage[];  // kSelStage: this CTA's candidates, in index order
+  extern __shared__ __align__(16) uint64_t stage[];  // kSelStage: this CTA's candidates, in index order;
+                                                     // then kSelWarps lists of kWarpCap (the warps' runs)
+  __shared__ uint32_t s_wcnt[kSelWarps];
   __shared__ __align__(16) uint32_t sh[kHistBins];
   __shared__ uint32_t s_count, s_ntie;
   __shared__ uint32_t s_keep[kCandCap / 32];  // tie verdicts by candidate position
@@ -686,24 +689,48 @@ __global__ void __launch_bounds__(kSelThreads) index_select(const float* __restr
   pdl_wait();
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *tail_ctr = 0;  // the score kernel's queue, for the next call
 
-  // 1) the first batch of scores is in flight while the histogram is read
+  // 1) every warp owns a contiguous run of the CTA's chunk; its first batch
+  //    of scores is in flight while the histogram is read
+  const int warp = threadIdx.x >> 5;
+  const int64_t wspan = ((n1 - n0 + kSelWarps - 1) / kSelWarps + 31) / 32 * 32;
+  const int64_t w0 = min(n1, n0 + int64_t(warp) * wspan), w1 = min(n1, w0 + wspan);
   uint32_t oa[kSelBatch], ob2[kSelBatch];
-  load_codes<kSelThreads, kSelBatch>(sc, n0, n1, oa);
+  warp_load_codes(sc, w0, w1, oa);
   load_histogram<kSelThreads>(hb, sh);
   __syncthreads();
   uint32_t above1;
   const int bin1 = find_threshold_bin<kSelThreads>(sh, kk, &above1);
 
-  // 2) this CTA's candidates, in index order; batches double-buffered
-  uint32_t count = 0;
-  for (int64_t base = n0; base < n1; base += 2 * kSelBatchSpan) {
-    if (base + kSelBatchSpan < n1) load_codes<kSelThreads, kSelBatch>(sc, base + kSelBatchSpan, n1, ob2);
-    count = stage_batch(oa, base, n1, bin1, count, stage);
-    if (base + kSelBatchSpan >= n1) break;
-    if (base + 2 * kSelBatchSpan < n1) load_codes<kSelThreads, kSelBatch>(sc, base + 2 * kSelBatchSpan, n1, oa);
-    count = stage_batch(ob2, base + kSelBatchSpan, n1, bin1, count, stage);
+  // 2) each warp filters its run into its own index-ordered list (batches
+  //    double-buffered, no block barrier); the lists are then concatenated in
+  //    warp order into the CTA's list, which is therefore in index order
+  uint64_t* wl = stage + kSelStage + warp * kWarpCap;
+  uint32_t wc = 0;
+  for (int64_t base = w0; base < w1; base += 2 * kSelWarpSpan) {
+    if (base + kSelWarpSpan < w1) warp_load_codes(sc, base + kSelWarpSpan, w1, ob2);
+    wc = warp_stage_batch(oa, base, w1, bin1, wc, wl);
+    if (base + kSelWarpSpan >= w1) break;
+    if (base + 2 * kSelWarpSpan < w1) warp_load_codes(sc, base + 2 * kSelWarpSpan, w1, oa);
+    wc = warp_stage_batch(ob2, base + kSelWarpSpan, w1, bin1, wc, wl);
   }
-  if (threadIdx.x == 0) s_count = count;
+  if (lane == 0) s_wcnt[warp] = wc;
+  __syncthreads();
+  {
+    uint32_t off = 0, tot = 0;
+    bool over = false;
+#pragma unroll
+    for (int w = 0; w < kSelWarps; ++w) {
+      const uint32_t c = s_wcnt[w];
+      off += w < warp ? c : 0u;
+      tot += c;
+      over |= c > uint32_t(kWarpCap);
+    }
+    const uint32_t mine = min(wc, uint32_t(kWarpCap));
+    for (uint32_t i = lane; i < mine; i += 32)
+      if (off + i < uint32_t(kSelStage)) stage[off + i] = wl[i];
+    // a list that overflowed sends the sequence to the exact fallback
+    if (threadIdx.x == 0) s_count = over ? uint32_t(kSelStage) + 1u : tot;
+  }
   cluster_sync();  // every list of the cluster is complete
 
   // 3) the leader gathers the lists in chunk order (= index order)
@@ -962,8 +989,8 @@ dsv4kv_status index_select_launch(int batch, int64_t n, int k, int32_t* idx_out,
   }
   // at most one CTA per SM in all (the leader's registers allow one per SM)
   const int64_t per_seq = std::max<int64_t>(1, std::min<int64_t>(max_cluster, sms / std::max(batch, 1)));
-  const int64_t batches_per_cta = std::max<int64_t>(1, (n + per_seq * kSelBatchSpan - 1) / (per_seq * kSelBatchSpan));
-  const int64_t chunk = batches_per_cta * kSelBatchSpan;
+  const int64_t units_per_cta = std::max<int64_t>(1, (n + per_seq * kSelChunkUnit - 1) / (per_seq * kSelChunkUnit));
+  const int64_t chunk = units_per_cta * kSelChunkUnit;
   const unsigned ctas = unsigned((n + chunk - 1) / chunk);
   launch_pdl_cluster(index_select, dim3(ctas, unsigned(batch)), dim3(kSelThreads), kSelDyn, ctas, stream,
                      (const float*)w.scores, n, k, chunk, w.hist, idx_out, count_out, w.status, w.tail_ctr);
