@@ -437,9 +437,12 @@ constexpr int kResPer = kCandCap / kSelThreads;        // candidates per leader 
 constexpr int kTieCap = 2048;
 constexpr int kMaxClusterSel = 16;
 constexpr int kWarpCap = kSelStage / kSelWarps;       // candidates a warp's list can hold
-// dynamic shared memory: the CTA's list (kSelStage) + the warps' lists (kSelStage)
-constexpr size_t kSelDyn = 2 * size_t(kSelStage) * sizeof(uint64_t);
-static_assert(kTieCap * (sizeof(uint64_t) + sizeof(uint32_t)) <= kSelDyn / 2, "the tie list reuses the list area");
+// dynamic shared memory: the tie list (kSelStage u64), the warps' lists
+// (kSelStage), and the leader's receive buffer (kCandCap): CTA r of the
+// cluster pushes its list into region r (kCandCap / C entries)
+constexpr size_t kSelDyn = (2 * size_t(kSelStage) + kCandCap) * sizeof(uint64_t);
+static_assert(kTieCap * (sizeof(uint64_t) + sizeof(uint32_t)) <= size_t(kSelStage) * sizeof(uint64_t),
+              "the tie list fits its area");
 
 // Block-wide exclusive prefix sum of one value per thread (NT threads).
 template <int NT>
@@ -669,11 +672,12 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
                                                             int32_t* __restrict__ count_out,
                                                             uint32_t* __restrict__ status,
                                                             uint32_t* __restrict__ tail_ctr) {
-  extern __shared__ __align__(16) uint64_t stage[];  // kSelStage: this CTA's candidates, in index order;
-                                                     // then kSelWarps lists of kWarpCap (the warps' runs)
+  extern __shared__ __align__(16) uint64_t stage[];  // the tie list; kSelWarps lists of kWarpCap (the
+                                                     // warps' runs); the leader's receive buffer
   __shared__ uint32_t s_wcnt[kSelWarps];
+  __shared__ uint32_t s_rcnt[kMaxClusterSel];  // leader: the count each CTA pushed (~0u: overflow)
   __shared__ __align__(16) uint32_t sh[kHistBins];
-  __shared__ uint32_t s_count, s_ntie;
+  __shared__ uint32_t s_ntie;
   __shared__ uint32_t s_keep[kCandCap / 32];  // tie verdicts by candidate position
   __shared__ uint32_t s_pre[kMaxClusterSel + 1];
 
@@ -715,6 +719,12 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
   }
   if (lane == 0) s_wcnt[warp] = wc;
   __syncthreads();
+  // 3) every CTA pushes its warps' lists, concatenated in warp order, into
+  //    its region of the leader's receive buffer (remote shared-memory stores),
+  //    and its count; a list or region that overflowed sends the sequence to
+  //    the exact fallback
+  const uint32_t regcap = uint32_t(kCandCap) / csize;
+  uint64_t* recv = stage + 2 * kSelStage;
   {
     uint32_t off = 0, tot = 0;
     bool over = false;
@@ -725,62 +735,61 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
       tot += c;
       over |= c > uint32_t(kWarpCap);
     }
+    over |= tot > regcap;
     const uint32_t mine = min(wc, uint32_t(kWarpCap));
-    for (uint32_t i = lane; i < mine; i += 32)
-      if (off + i < uint32_t(kSelStage)) stage[off + i] = wl[i];
-    // a list that overflowed sends the sequence to the exact fallback
-    if (threadIdx.x == 0) s_count = over ? uint32_t(kSelStage) + 1u : tot;
+    const uint32_t dst = dsmem_addr(recv + size_t(rank) * regcap, 0);
+    if (!over)
+      for (uint32_t i = lane; i < mine; i += 32) st_dsmem_u64(dst + 8u * (off + i), wl[i]);
+    if (threadIdx.x == 0) st_dsmem_u32(dsmem_addr(&s_rcnt[rank], 0), over ? 0xffffffffu : tot);
   }
-  cluster_sync();  // every list of the cluster is complete
+  if (rank == 0) {  // the leader's resolve state, cleared while the other CTAs finish
+    for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) sh[i] = 0;
+    for (int i = threadIdx.x; i < kCandCap / 32; i += kSelThreads) s_keep[i] = 0;
+    if (threadIdx.x == 0) s_ntie = 0;
+  }
+  cluster_sync();  // every list is in the leader's shared memory
+  if (rank != 0) return;
 
-  // 3) the leader gathers the lists in chunk order (= index order)
+  // 4) the leader reads the regions in rank order (= index order)
   uint64_t c[kResPer];
   uint32_t total = 0;
   bool fits = true;
-  if (rank == 0) {
-    if (threadIdx.x == 0) {
-      uint32_t run = 0;
-      for (uint32_t r = 0; r < csize; ++r) {
-        s_pre[r] = run;
-        const uint32_t cnt = ld_dsmem_u32(dsmem_addr(&s_count, r));
-        if (cnt > uint32_t(kSelStage)) fits = false;
-        run += cnt;
-      }
-      s_pre[csize] = fits ? run : 0xffffffffu;
-    }
-    __syncthreads();
-    total = s_pre[csize];
-    fits = total <= uint32_t(kCandCap);
-    if (fits) {
-      // the source of every position first, then all the loads
-      uint32_t src[kResPer];
+  if (threadIdx.x < 32) {  // one warp scan of the counts gives the offsets
+    const uint32_t cnt = threadIdx.x < csize ? s_rcnt[threadIdx.x] : 0u;
+    const bool bad = __any_sync(kFull, cnt == 0xffffffffu);
+    const uint32_t incl = warp_inclusive_scan(bad ? 0u : cnt);
+    if (threadIdx.x < csize) s_pre[threadIdx.x] = incl - (bad ? 0u : cnt);
+    if (threadIdx.x == csize - 1) s_pre[csize] = bad ? 0xffffffffu : incl;
+  }
+  __syncthreads();
+  total = s_pre[csize];
+  fits = total <= uint32_t(kCandCap);
+  if (fits) {
+    // the region of every position (offsets in registers, a branch-free
+    // search: offsets are non-decreasing, the last one <= g holds g)
+    uint32_t pre[kMaxClusterSel];
 #pragma unroll
-      for (int j = 0; j < kResPer; ++j) {
-        const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
-        uint32_t r = 0;
-        while (r + 1 < csize && s_pre[r + 1] <= g) ++r;
-        src[j] = dsmem_addr(&stage[g < total ? g - s_pre[r] : 0], r);
-      }
+    for (int i = 0; i < kMaxClusterSel; ++i) pre[i] = i < int(csize) ? s_pre[i] : 0xffffffffu;
 #pragma unroll
-      for (int j = 0; j < kResPer; ++j) {
-        const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
-        c[j] = g < total ? ld_dsmem_u64(src[j]) : 0ull;
+    for (int j = 0; j < kResPer; ++j) {
+      const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
+      uint32_t r = 0, base = 0;
+#pragma unroll
+      for (int i = 1; i < kMaxClusterSel; ++i) {
+        const bool past = pre[i] <= g;
+        r = past ? uint32_t(i) : r;
+        base = past ? pre[i] : base;
       }
+      c[j] = g < total ? recv[size_t(r) * regcap + (g - base)] : 0ull;
     }
   }
-  cluster_sync();  // the other CTAs' lists are no longer read
-  if (rank != 0) return;
 
-  // 4) resolve
+  // 5) resolve
   int32_t* out = idx_out + size_t(b) * k;
   const uint32_t need1 = kk - above1;  // still needed from bin1 (>= 1)
   uint64_t* ties = stage;              // the leader's list is in registers now
   bool ok = false;
   uint32_t prefix = 0, need_tie = 0;
-  for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) sh[i] = 0;
-  for (int i = threadIdx.x; i < kCandCap / 32; i += kSelThreads) s_keep[i] = 0;
-  if (threadIdx.x == 0) s_ntie = 0;
-  __syncthreads();
   if (fits) {
     // second-level histogram of bin1 (every entry of bin1 is a candidate)
 #pragma unroll
@@ -794,40 +803,48 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
     const int bin2 = find_threshold_bin<kSelThreads>(sh, need1, &above2);
     prefix = (uint32_t(bin1) << 12) | uint32_t(bin2);  // 24-bit threshold prefix
     need_tie = need1 - above2;                          // >= 1
-    // the entries at the prefix: (key, position) into the tie list
+    // every entry at the prefix is needed (the usual case: one entry at a
+    // 24-bit prefix) -> no ranking; else rank the entries at the prefix
+    const bool all_at = sh[bin2] == need_tie;
+    if (!all_at) {
+      // the entries at the prefix: (key, position) into the tie list
 #pragma unroll
-    for (int j = 0; j < kResPer; ++j) {
-      const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
-      if (g < total && uint32_t(c[j] >> 40) == prefix) {
-        const uint32_t slot = atomicAdd(&s_ntie, 1u);
-        if (slot < uint32_t(kTieCap)) {
-          ties[slot] = c[j];
-          reinterpret_cast<uint32_t*>(ties + kTieCap)[slot] = g;
-        }
-      }
-    }
-    __syncthreads();
-    const uint32_t n_tie = s_ntie;
-    if (n_tie <= uint32_t(kTieCap)) {
-      ok = true;
-      // a tie is kept when fewer than need_tie keys (score desc, index asc) exceed its own
-      for (uint32_t t = threadIdx.x; t < n_tie; t += kSelThreads) {
-        const uint64_t key = ties[t];
-        uint32_t r = 0;
-        for (uint32_t u = 0; u < n_tie; ++u) r += ties[u] > key ? 1u : 0u;
-        if (r < need_tie) {
-          const uint32_t g = reinterpret_cast<const uint32_t*>(ties + kTieCap)[t];
-          atomicOr(&s_keep[g >> 5], 1u << (g & 31));
+      for (int j = 0; j < kResPer; ++j) {
+        const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
+        if (g < total && uint32_t(c[j] >> 40) == prefix) {
+          const uint32_t slot = atomicAdd(&s_ntie, 1u);
+          if (slot < uint32_t(kTieCap)) {
+            ties[slot] = c[j];
+            reinterpret_cast<uint32_t*>(ties + kTieCap)[slot] = g;
+          }
         }
       }
       __syncthreads();
+    }
+    const uint32_t n_tie = all_at ? 0u : s_ntie;
+    if (n_tie <= uint32_t(kTieCap)) {
+      ok = true;
+      // a tie is kept when fewer than need_tie keys (score desc, index asc) exceed its own
+      if (!all_at) {
+        for (uint32_t t = threadIdx.x; t < n_tie; t += kSelThreads) {
+          const uint64_t key = ties[t];
+          uint32_t r = 0;
+          for (uint32_t u = 0; u < n_tie; ++u) r += ties[u] > key ? 1u : 0u;
+          if (r < need_tie) {
+            const uint32_t g = reinterpret_cast<const uint32_t*>(ties + kTieCap)[t];
+            atomicOr(&s_keep[g >> 5], 1u << (g & 31));
+          }
+        }
+        __syncthreads();
+      }
       // ordered compaction of the kept candidates
       uint32_t m[kResPer], off[kResPer];
 #pragma unroll
       for (int j = 0; j < kResPer; ++j) {
         const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
         const uint32_t pre = uint32_t(c[j] >> 40);
-        const bool keep = g < total && (pre > prefix || (pre == prefix && ((s_keep[g >> 5] >> (g & 31)) & 1u)));
+        const bool keep =
+            g < total && (pre > prefix || (pre == prefix && (all_at || ((s_keep[g >> 5] >> (g & 31)) & 1u))));
         m[j] = __ballot_sync(kFull, keep);
       }
       const uint32_t got = ordered_offsets<kSelThreads, kResPer>(m, off);
@@ -862,7 +879,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
   }
   for (int i = int(kk) + threadIdx.x; i < k; i += kSelThreads) out[i] = -1;
   if (threadIdx.x == 0 && count_out) count_out[b] = int32_t(kk);
-  // 5) leave the histogram zeroed for the next call (every CTA of the cluster has read it)
+  // 6) leave the histogram zeroed for the next call (every CTA of the cluster has read it)
   for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) hb[i] = 0;
 }
 
