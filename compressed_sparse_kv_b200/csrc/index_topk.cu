@@ -27,6 +27,10 @@ namespace dsv4kv {
 
 constexpr int kHistBins = 4096;  // 12-bit digits
 
+// Row stride of the fp32 score rows in the workspace: n rounded up to 4, so
+// every row starts on a 16-byte boundary.
+__host__ __device__ __forceinline__ int64_t score_stride(int64_t n) { return (n + 3) & ~int64_t(3); }
+
 // ------------------------------------------------------------------ scoring
 // Transposing butterfly: lane l16 of a 16-lane group holds U partial sums
 // (one per key); after log2 steps each lane holds the full 16-lane sum of one
@@ -194,7 +198,7 @@ __device__ __forceinline__ void score_tail_bf16(const uint16_t* __restrict__ qid
     const float sc = reduce16_transposed<U>(p, l16) + 0.0f;  // -0 -> +0
     const int64_t key = i0 + 16 * g + U * half + my_key;
     if (writer && key < n) {
-      scores[size_t(b) * size_t(n) + size_t(key)] = sc;
+      scores[size_t(b) * size_t(score_stride(n)) + size_t(key)] = sc;
       atomicAdd(&hist[size_t(b) * kHistBins + (ord_f32(sc) >> 20)], 1u);
     }
   };
@@ -262,7 +266,7 @@ __global__ void __launch_bounds__(256) index_score_bf16(const uint16_t* __restri
       __syncthreads();
     }
     score_segment_bf16<U>(qidx + size_t(b) * 128, keys + (size_t(b) * size_t(key_rows) + size_t(i0)) * 128, s1 - s0,
-                          scores + size_t(b) * size_t(n) + size_t(i0), nullptr, sh, pol);
+                          scores + size_t(b) * size_t(score_stride(n)) + size_t(i0), nullptr, sh, pol);
     b_last = b;
     s0 = s1;
   }
@@ -405,7 +409,7 @@ __global__ void __launch_bounds__(256) index_score_fp4(const uint16_t* __restric
     const int64_t i0 = s0 - int64_t(b) * n;
     const size_t r0 = size_t(b) * size_t(key_rows) + size_t(i0);
     score_segment_fp4(qidx + size_t(b) * 128, codes + r0 * 64, scales + r0 * 8, s1 - s0,
-                      scores + size_t(b) * size_t(n) + size_t(i0), nullptr, sh, pol);
+                      scores + size_t(b) * size_t(score_stride(n)) + size_t(i0), nullptr, sh, pol);
     flush_histogram(sh, hist + size_t(b) * kHistBins);
     __syncthreads();
     s0 = s1;
@@ -437,12 +441,17 @@ constexpr int kResPer = kCandCap / kSelThreads;        // candidates per leader 
 constexpr int kTieCap = 2048;
 constexpr int kMaxClusterSel = 16;
 constexpr int kWarpCap = kSelStage / kSelWarps;       // candidates a warp's list can hold
-// dynamic shared memory: the tie list (kSelStage u64), the warps' lists
-// (kSelStage), and the leader's receive buffer (kCandCap): CTA r of the
-// cluster pushes its list into region r (kCandCap / C entries)
-constexpr size_t kSelDyn = (2 * size_t(kSelStage) + kCandCap) * sizeof(uint64_t);
-static_assert(kTieCap * (sizeof(uint64_t) + sizeof(uint32_t)) <= size_t(kSelStage) * sizeof(uint64_t),
-              "the tie list fits its area");
+// Every warp streams its run of scores through its own ring of kRing slots
+// of one warp batch (256 fp32 = 1 KB) in shared memory, filled by 16-byte
+// cp.async copies kRing - 1 batches ahead of the one it filters.
+constexpr int kRing = 4;
+constexpr size_t kRingBytes = size_t(kSelWarps) * kRing * kSelWarpSpan * sizeof(float);  // 64 KB
+// dynamic shared memory: the rings (whose first bytes the leader's tie list
+// reuses after the filter), the warps' lists (kSelStage u64), and the
+// leader's receive buffer (kCandCap): CTA r of the cluster pushes its list
+// into region r (kCandCap / C entries)
+constexpr size_t kSelDyn = kRingBytes + (size_t(kSelStage) + kCandCap) * sizeof(uint64_t);
+static_assert(kTieCap * (sizeof(uint64_t) + sizeof(uint32_t)) <= kRingBytes, "the tie list fits the ring area");
 
 // Block-wide exclusive prefix sum of one value per thread (NT threads).
 template <int NT>
@@ -582,15 +591,28 @@ __device__ __forceinline__ void load_histogram(const uint32_t* __restrict__ hb, 
   for (int j = 0; j < V; ++j) reinterpret_cast<uint4*>(sh)[threadIdx.x + j * NT] = v[j];
 }
 
-// One warp batch of score codes: lane l takes positions base + 32 v + l.
-__device__ __forceinline__ void warp_load_codes(const float* __restrict__ sc, int64_t base, int64_t end,
-                                                uint32_t (&o)[kSelBatch]) {
+// Issues the copy of one warp batch (scores [base, base + 256) of the row,
+// those at or beyond `end` zero-filled and not read) into a ring slot: lane l
+// copies 16-byte pieces l and l + 32.  base is a multiple of 32 and the row
+// 16-byte aligned, so every piece is aligned.
+__device__ __forceinline__ void warp_issue_batch(const float* __restrict__ sc, int64_t base, int64_t end,
+                                                 float* slot) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int v = 0; v < kSelBatch; ++v) {
-    const int64_t i = base + 32 * v + lane;
-    o[v] = i < end ? ord_f32(__ldcg(sc + i)) : 0u;
+  for (int h = 0; h < 2; ++h) {
+    const int piece = lane + 32 * h;
+    const int64_t i = base + 4 * piece;
+    const int64_t left = end - i;
+    const uint32_t bytes = left >= 4 ? 16u : (left > 0 ? uint32_t(left) * 4u : 0u);
+    cp_async16_zfill(slot + 4 * piece, bytes ? sc + i : sc, bytes);
   }
+}
+
+// The codes of a landed warp batch: lane l takes positions 32 v + l.
+__device__ __forceinline__ void warp_read_batch(const float* slot, uint32_t (&o)[kSelBatch]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int v = 0; v < kSelBatch; ++v) o[v] = ord_f32(slot[32 * v + lane]);
 }
 
 // Appends, in index order, the warp batch's entries whose top-12-bit bin is
@@ -686,37 +708,47 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
   const uint32_t csize = gridDim.x;  // one cluster spans the sequence's CTAs
   const uint32_t kk = uint32_t(int64_t(k) < n ? int64_t(k) : n);
   uint32_t* hb = hist + size_t(b) * kHistBins;
-  const float* sc = scores + size_t(b) * size_t(n);
+  const float* sc = scores + size_t(b) * size_t(score_stride(n));
   const int64_t n0 = int64_t(rank) * chunk, n1 = min(n, n0 + chunk);
   const int lane = threadIdx.x & 31;
   pdl_trigger();
   pdl_wait();
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *tail_ctr = 0;  // the score kernel's queue, for the next call
 
-  // 1) every warp owns a contiguous run of the CTA's chunk; its first batch
-  //    of scores is in flight while the histogram is read
+  // 1) every warp owns a contiguous run of the CTA's chunk; the first
+  //    batches of its run are in flight while the histogram is read
   const int warp = threadIdx.x >> 5;
   const int64_t wspan = ((n1 - n0 + kSelWarps - 1) / kSelWarps + 31) / 32 * 32;
   const int64_t w0 = min(n1, n0 + int64_t(warp) * wspan), w1 = min(n1, w0 + wspan);
-  uint32_t oa[kSelBatch], ob2[kSelBatch];
-  warp_load_codes(sc, w0, w1, oa);
+  const int64_t nbat = (w1 - w0 + kSelWarpSpan - 1) / kSelWarpSpan;
+  float* ring = reinterpret_cast<float*>(stage) + size_t(warp) * kRing * kSelWarpSpan;
+#pragma unroll
+  for (int t = 0; t < kRing - 1; ++t) {
+    if (t < nbat) warp_issue_batch(sc, w0 + int64_t(t) * kSelWarpSpan, w1, ring + t * kSelWarpSpan);
+    cp_async_commit();
+  }
   load_histogram<kSelThreads>(hb, sh);
   __syncthreads();
   uint32_t above1;
   const int bin1 = find_threshold_bin<kSelThreads>(sh, kk, &above1);
 
-  // 2) each warp filters its run into its own index-ordered list (batches
-  //    double-buffered, no block barrier); the lists are then concatenated in
-  //    warp order into the CTA's list, which is therefore in index order
-  uint64_t* wl = stage + kSelStage + warp * kWarpCap;
+  // 2) each warp filters its run into its own index-ordered list (no block
+  //    barrier); the lists are then concatenated in warp order, which is
+  //    index order
+  uint64_t* wl = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(stage) + kRingBytes) + warp * kWarpCap;
   uint32_t wc = 0;
-  for (int64_t base = w0; base < w1; base += 2 * kSelWarpSpan) {
-    if (base + kSelWarpSpan < w1) warp_load_codes(sc, base + kSelWarpSpan, w1, ob2);
-    wc = warp_stage_batch(oa, base, w1, bin1, wc, wl);
-    if (base + kSelWarpSpan >= w1) break;
-    if (base + 2 * kSelWarpSpan < w1) warp_load_codes(sc, base + 2 * kSelWarpSpan, w1, oa);
-    wc = warp_stage_batch(ob2, base + kSelWarpSpan, w1, bin1, wc, wl);
+  for (int64_t t = 0; t < nbat; ++t) {
+    if (t + kRing - 1 < nbat)
+      warp_issue_batch(sc, w0 + (t + kRing - 1) * kSelWarpSpan, w1, ring + ((t + kRing - 1) % kRing) * kSelWarpSpan);
+    cp_async_commit();
+    cp_async_wait_group<kRing - 1>();  // batch t has landed (this lane's pieces)
+    __syncwarp();                      // ... and every lane's
+    uint32_t o[kSelBatch];
+    warp_read_batch(ring + (t % kRing) * kSelWarpSpan, o);
+    __syncwarp();  // the slot is read before it is refilled
+    wc = warp_stage_batch(o, w0 + t * kSelWarpSpan, w1, bin1, wc, wl);
   }
+  cp_async_wait_group<0>();  // nothing left in flight (batches past the run were never issued)
   if (lane == 0) s_wcnt[warp] = wc;
   __syncthreads();
   // 3) every CTA pushes its warps' lists, concatenated in warp order, into
@@ -724,7 +756,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
   //    and its count; a list or region that overflowed sends the sequence to
   //    the exact fallback
   const uint32_t regcap = uint32_t(kCandCap) / csize;
-  uint64_t* recv = stage + 2 * kSelStage;
+  uint64_t* recv = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(stage) + kRingBytes) + kSelStage;
   {
     uint32_t off = 0, tot = 0;
     bool over = false;
@@ -748,7 +780,12 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
     if (threadIdx.x == 0) s_ntie = 0;
   }
   cluster_sync();  // every list is in the leader's shared memory
-  if (rank != 0) return;
+  if (rank != 0) {
+    // leave the histogram zeroed for the next call (every CTA read it before the barrier)
+    if (rank == 1)
+      for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) hb[i] = 0;
+    return;
+  }
 
   // 4) the leader reads the regions in rank order (= index order)
   uint64_t c[kResPer];
@@ -879,8 +916,9 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
   }
   for (int i = int(kk) + threadIdx.x; i < k; i += kSelThreads) out[i] = -1;
   if (threadIdx.x == 0 && count_out) count_out[b] = int32_t(kk);
-  // 6) leave the histogram zeroed for the next call (every CTA of the cluster has read it)
-  for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) hb[i] = 0;
+  // 6) leave the histogram zeroed for the next call (a one-CTA cluster has no helper)
+  if (csize == 1)
+    for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) hb[i] = 0;
 }
 
 __global__ void index_fill_all(int64_t n, int k, int32_t* __restrict__ idx_out, int32_t* __restrict__ count_out) {
@@ -915,7 +953,7 @@ static IndexWs index_ws_layout(char* base, int batch, int64_t n, int k) {
   w.status = reinterpret_cast<uint32_t*>(take(16));
   w.hist = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * kHistBins * size_t(batch)));
   w.tail_ctr = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t)));
-  w.scores = reinterpret_cast<float*>(take(sizeof(float) * size_t(batch) * size_t(n)));
+  w.scores = reinterpret_cast<float*>(take(sizeof(float) * size_t(batch) * size_t(score_stride(n))));
   w.bytes = off;
   return w;
 }
