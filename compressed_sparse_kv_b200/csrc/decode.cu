@@ -878,27 +878,35 @@ __global__ void __launch_bounds__(32 * kCombWarps) decode_combine(const float* _
   }
 }
 
-// The same merge for many splits: one block of kWideWarps warps per
-// (sequence, head); warp w takes splits w, w + kWideWarps, ...; lanes own 16
-// channels (4 float4); the warps' sums meet in shared memory (rows of 512
-// channels, lane-contiguous float4s: no bank conflicts) and thread t
-// finishes channels 2t, 2t+1 (a rotary pair).
+// Merge for more than kCombFast splits.  Block (sequence, head, channel
+// block cb) covers the CB-th part of the channels, [cb D/CB, (cb+1) D/CB):
+// lane l of every warp owns channels cb D/CB + 128 q + 4l .. + 3 (float4s,
+// q < 4/CB; both channels of a rotary pair sit in one float4), warp w the
+// splits s = w mod kWideWarps, taken 2 CB at a time (one when CB = 1) with all their loads in
+// flight before any is used.  The maxima come first from one pass over the
+// (m, l) terms; the warps' sums meet in shared memory.  CB is chosen per
+// launch so that the grid stays within a few blocks per SM.
 constexpr int kWideWarps = 8;
 
-__global__ void __launch_bounds__(32 * kWideWarps) decode_combine_wide(const float* __restrict__ o_part,
+template <int CB>
+__global__ void __launch_bounds__(32 * kWideWarps, CB == 1 ? 4 : 2) decode_combine_wide(const float* __restrict__ o_part,
                                                                        const float* __restrict__ ml_part,
                                                                        const float* __restrict__ rope_tab, int splits,
                                                                        int heads, int rope_dim, int out_fp32,
                                                                        void* __restrict__ out) {
-  __shared__ __align__(16) float red[kWideWarps][kDim];
+  constexpr int CW = kDim / CB;  // channels per block
+  constexpr int Q = 4 / CB;      // float4s per lane and split
+  constexpr int U = CB == 1 ? 1 : 2 * CB;  // splits per warp and round
+  __shared__ __align__(16) float red[kWideWarps][CW];
   __shared__ float s_mo[kWideWarps], s_ml[kWideWarps], s_l[kWideWarps];
   pdl_trigger();
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.x / heads, h = blockIdx.x % heads;
+  const int bh = blockIdx.x / CB, cb = blockIdx.x % CB;
+  const int b = bh / heads, h = bh % heads;
   const size_t ml_stride = size_t(heads) * 4, o_stride = size_t(heads) * kDim;
   const float* mlb = ml_part + (size_t(b) * splits * heads + h) * 4;
-  const float* ob = o_part + (size_t(b) * splits * heads + h) * kDim + 4 * lane;
+  const float* ob = o_part + (size_t(b) * splits * heads + h) * kDim + CW * cb + 4 * lane;
   // maxima over all splits
   float mo = -INFINITY, ml = -INFINITY;
   for (int s = threadIdx.x; s < splits; s += 32 * kWideWarps) {
@@ -923,42 +931,56 @@ __global__ void __launch_bounds__(32 * kWideWarps) decode_combine_wide(const flo
     mo = fmaxf(mo, s_mo[w]);
     ml = fmaxf(ml, s_ml[w]);
   }
-  // this warp's splits
-  float4 acc[4];
+  // this warp's splits, U per round
+  float4 acc[Q];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int q = 0; q < Q; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
   float L = 0.f;
-#pragma unroll 2
-  for (int s = warp; s < splits; s += kWideWarps) {
-    const float4 v = __ldcg(reinterpret_cast<const float4*>(mlb + s * ml_stride));
-    float4 x[4];
+  for (int s0 = warp; s0 < splits; s0 += kWideWarps * U) {
+    float4 v[U], x[U][Q];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) x[q] = __ldcg(reinterpret_cast<const float4*>(ob + size_t(s) * o_stride + 128 * q));
-    if (v.y != -INFINITY) L += v.z * exp2f(v.y - ml);
-    const float w = v.x == -INFINITY ? 0.f : exp2f(v.x - mo);
-    if (w != 0.f) {  // an empty partial's O is never read
+    for (int u = 0; u < U; ++u) {
+      const int s = s0 + u * kWideWarps;
+      v[u] = s < splits ? __ldcg(reinterpret_cast<const float4*>(mlb + s * ml_stride))
+                        : make_float4(-INFINITY, -INFINITY, 0.f, 0.f);
+    }
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        acc[q].x = fmaf(w, x[q].x, acc[q].x);
-        acc[q].y = fmaf(w, x[q].y, acc[q].y);
-        acc[q].z = fmaf(w, x[q].z, acc[q].z);
-        acc[q].w = fmaf(w, x[q].w, acc[q].w);
+    for (int u = 0; u < U; ++u) {
+      const int s = s0 + u * kWideWarps;
+#pragma unroll
+      for (int q = 0; q < Q; ++q)
+        x[u][q] = s < splits ? __ldcg(reinterpret_cast<const float4*>(ob + size_t(s) * o_stride + 128 * q))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (v[u].y != -INFINITY) L += v[u].z * exp2f(v[u].y - ml);
+      if (v[u].x != -INFINITY) {  // an empty partial's O (m_o = -inf) is not used
+        const float w = exp2f(v[u].x - mo);
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+          acc[q].x = fmaf(w, x[u][q].x, acc[q].x);
+          acc[q].y = fmaf(w, x[u][q].y, acc[q].y);
+          acc[q].z = fmaf(w, x[u][q].z, acc[q].z);
+          acc[q].w = fmaf(w, x[u][q].w, acc[q].w);
+        }
       }
     }
   }
 #pragma unroll
-  for (int q = 0; q < 4; ++q) *reinterpret_cast<float4*>(&red[warp][128 * q + 4 * lane]) = acc[q];
+  for (int q = 0; q < Q; ++q) *reinterpret_cast<float4*>(&red[warp][128 * q + 4 * lane]) = acc[q];
   if (lane == 0) s_l[warp] = L;  // every lane carries the same L
   __syncthreads();
+  if (threadIdx.x >= CW / 2) return;
   float Lt = 0.f;
 #pragma unroll
   for (int w = 0; w < kWideWarps; ++w) Lt += s_l[w];
   const float inv = (mo == -INFINITY || Lt <= 0.f) ? 0.f : exp2f(mo - ml) / Lt;
-  const int c = 2 * threadIdx.x;  // 256 threads x 2 channels
+  const int cl = 2 * threadIdx.x, c = CW * cb + cl;  // CW/2 threads x 2 channels
   float v0 = 0.f, v1 = 0.f;
 #pragma unroll
   for (int w = 0; w < kWideWarps; ++w) {
-    const float2 x = *reinterpret_cast<const float2*>(&red[w][c]);
+    const float2 x = *reinterpret_cast<const float2*>(&red[w][cl]);
     v0 += x.x;
     v1 += x.y;
   }
@@ -976,7 +998,7 @@ __global__ void __launch_bounds__(32 * kWideWarps) decode_combine_wide(const flo
   if (out_fp32) *reinterpret_cast<float2*>(static_cast<float*>(out) + o) = make_float2(v0, v1);
   else static_cast<uint32_t*>(out)[o / 2] = pack_bf16x2(v0, v1);
 }
-static_assert(2 * 32 * kWideWarps == kDim, "two channels per thread");
+static_assert(32 * kWideWarps >= kDim / 2, "enough threads to finish one channel pair each");
 
 struct Plan {
   int comp_tiles, tiles, splits, tiles_per_split;
@@ -1120,10 +1142,15 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
     launch_pdl(decode_combine, dim3((bh_total + kCombWarps - 1) / kCombWarps), dim3(32 * kCombWarps), 0, stream,
                (const float*)w.o_part, (const float*)w.ml_part, (const float*)w.rope_tab, pl.splits, a.heads,
                bh_total, a.rope_dim, a.out_fp32, a.out);
-  else
-    launch_pdl(decode_combine_wide, dim3(bh_total), dim3(32 * kWideWarps), 0, stream, (const float*)w.o_part,
+  else {
+    // channel blocks per (sequence, head): as many as keep the grid within ~3 blocks per SM
+    const int sms = sm_count();
+    const int cb = bh_total * 4 <= 3 * sms ? 4 : (bh_total * 2 <= 3 * sms ? 2 : 1);
+    auto kern = cb == 4 ? decode_combine_wide<4> : (cb == 2 ? decode_combine_wide<2> : decode_combine_wide<1>);
+    launch_pdl(kern, dim3(bh_total * cb), dim3(32 * kWideWarps), 0, stream, (const float*)w.o_part,
                (const float*)w.ml_part, (const float*)w.rope_tab, pl.splits, a.heads, a.rope_dim, a.out_fp32,
                a.out);
+  }
   return check_launch("decode_combine");
 }
 
