@@ -21,6 +21,13 @@ rounding rule; the reading used here (and fixed for the CUDA side too) is:
   even, saturating to +-6; all codes 0 when s == 0.  Nibbles are packed two
   per byte, the even channel in the low nibble.
 * The sign of a value that rounds to zero is kept (IEEE conversion rule).
+* fp8 with bf16 rotary channels (the layout [P1] describes for the attention
+  cache: "fp8 for most dimensions", the RoPE dimensions kept in bf16): the
+  first D - 64 channels of a row are quantised as an fp8 row (amax, scale and
+  codes over those channels only); the last 64 (rotary) channels are stored as
+  bf16 (nearest even from fp32 input, unchanged bits from bf16 input).  A row
+  is D - 64 code bytes followed by the 64 bf16 values (little-endian, 128
+  bytes), D + 64 bytes in all, plus the fp32 scale.
 """
 from __future__ import annotations
 
@@ -157,7 +164,35 @@ def dequant_fp4_rows(codes, scale_codes) -> np.ndarray:
     return vals * np.repeat(sc, 16, axis=-1)
 
 
-FMT_BF16, FMT_FP8, FMT_FP4 = 0, 1, 2
+ROPE_BF16_CHANNELS = 64  # rotary channels kept in bf16 by the fp8 + bf16-rotary layout
+
+
+def quantize_fp8_rope_rows(x) -> tuple[np.ndarray, np.ndarray]:
+    """fp32 rows [R][D] -> (row bytes u8 [R][D + 64], scales f32 [R]): the
+    first D - 64 channels as fp8 codes under one scale from their own amax,
+    then the last 64 channels as bf16 (2 bytes each, little-endian)."""
+    x = np.asarray(x, dtype=np.float32)
+    r, d = x.shape
+    nr = d - ROPE_BF16_CHANNELS
+    body = x[:, :nr]
+    amax = np.max(np.abs(body), axis=-1)
+    scale = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+    codes = e4m3_encode((body / scale[..., None]).astype(np.float32))
+    rope = f64_to_bf16_bits(x[:, nr:].astype(np.float64)).astype("<u2").view(np.uint8).reshape(r, 2 * ROPE_BF16_CHANNELS)
+    return np.concatenate([codes, rope], axis=1), scale
+
+
+def dequant_fp8_rope_rows(row_bytes, scales) -> np.ndarray:
+    """Row bytes u8 [R][D + 64] + scales f32 [R] -> float64 [R][D]."""
+    b = np.ascontiguousarray(np.asarray(row_bytes, dtype=np.uint8))
+    d = b.shape[-1] - ROPE_BF16_CHANNELS
+    nr = d - ROPE_BF16_CHANNELS
+    body = E4M3_TABLE[b[..., :nr]] * np.asarray(scales, dtype=np.float64)[..., None]
+    rope = bf16_bits_to_f64(np.ascontiguousarray(b[..., nr:]).view("<u2"))
+    return np.concatenate([body, rope], axis=-1)
+
+
+FMT_BF16, FMT_FP8, FMT_FP4, FMT_FP8_ROPE_BF16 = 0, 1, 2, 3
 
 
 def dequant(fmt: int, codes, scales=None) -> np.ndarray:
@@ -168,4 +203,6 @@ def dequant(fmt: int, codes, scales=None) -> np.ndarray:
         return dequant_fp8_rows(codes, scales)
     if fmt == FMT_FP4:
         return dequant_fp4_rows(codes, scales)
+    if fmt == FMT_FP8_ROPE_BF16:
+        return dequant_fp8_rope_rows(codes, scales)
     raise ValueError(f"unknown format {fmt}")

@@ -146,3 +146,50 @@ def test_fp4_zero_group_and_underflowing_scale():
     x[0, 16:] = 1e-6                     # amax/6 underflows E4M3 (min 2^-9)
     codes, sc = F.quantize_fp4_rows(x)
     assert np.all(sc == 0) and np.all(codes == 0)
+
+
+# ------------------------------------------------ fp8 body + bf16 rotary channels
+def test_fp8_rope_worked_example():
+    """A row worked by hand: body amax 224 -> scale 0.5; 224 / 0.5 = 448 is
+    code 0x7E, 1 / 0.5 = 2 is code 0x40; rotary 1.5 is bf16 0x3FC0 and -2 is
+    0xC000, stored little-endian after the 448 code bytes."""
+    x = np.zeros((1, 512), dtype=np.float32)
+    x[0, 0], x[0, 1], x[0, 447] = 224.0, 1.0, -0.25
+    x[0, 448], x[0, 511] = 1.5, -2.0
+    codes, scales = F.quantize_fp8_rope_rows(x)
+    assert codes.shape == (1, 576) and codes.dtype == np.uint8
+    assert scales[0] == np.float32(0.5)
+    assert codes[0, 0] == 0x7E and codes[0, 1] == 0x40
+    assert codes[0, 447] == 0xB0                      # -0.5 = -(1.0 * 2^-1): S=1, E=6, M=0
+    assert list(codes[0, 448:450]) == [0xC0, 0x3F]     # 1.5 -> 0x3FC0
+    assert list(codes[0, 574:576]) == [0x00, 0xC0]     # -2.0 -> 0xC000
+    assert np.all(codes[0, 2:447] == 0) and np.all(codes[0, 450:574] == 0)
+    back = F.dequant_fp8_rope_rows(codes, scales)
+    assert back[0, 0] == 224.0 and back[0, 1] == 1.0 and back[0, 447] == -0.25
+    assert back[0, 448] == 1.5 and back[0, 511] == -2.0
+
+
+def test_fp8_rope_rotary_channels_do_not_set_the_scale():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((8, 512)).astype(np.float32)
+    x[:, 448:] *= 1000.0                                # large rotary values
+    codes, scales = F.quantize_fp8_rope_rows(x)
+    amax = np.max(np.abs(x[:, :448]), axis=1)
+    assert np.array_equal(scales, (amax / np.float32(448.0)).astype(np.float32))
+    back = F.dequant_fp8_rope_rows(codes, scales)
+    ref = torch.from_numpy(x[:, 448:]).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(back[:, 448:], ref)           # rotary: bf16, nearest even (torch cast)
+
+
+def test_fp8_rope_body_error_bound_and_zero_rows():
+    rng = np.random.default_rng(6)
+    x = (rng.standard_normal((64, 512)) * rng.uniform(0.01, 50, (64, 1))).astype(np.float32)
+    x[3, :448] = 0.0
+    codes, scales = F.quantize_fp8_rope_rows(x)
+    assert scales[3] == 1.0 and np.all(codes[3, :448] == 0)
+    back = F.dequant_fp8_rope_rows(codes, scales)
+    # |q - x/s| <= half the E4M3 spacing at |x/s| (2^(e-3) / 2 for normals, 2^-10 below 2^-6)
+    q = x[:, :448] / scales[:, None]
+    e = np.floor(np.log2(np.maximum(np.abs(q), 2.0 ** -6)))
+    half = 2.0 ** (e - 4)
+    assert np.all(np.abs(back[:, :448] / scales[:, None].astype(np.float64) - q) <= half * (1 + 1e-12))
