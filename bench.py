@@ -39,8 +39,10 @@ WORKLOADS = {
     "q_c4a_fp4": ("c4a", 64, 262144, 64, 2, 2),
     "q_c128a_fp8": ("c128a", 64, 262144, 64, 1, 0),
     "q_c128a_fp4": ("c128a", 64, 262144, 64, 2, 0),
+    "q_c4a_fp8rope": ("c4a", 64, 262144, 64, 3, 2),
+    "q_c128a_fp8rope": ("c128a", 64, 262144, 64, 3, 0),
 }
-FMT_NAME = {0: "bf16", 1: "fp8", 2: "fp4"}
+FMT_NAME = {0: "bf16", 1: "fp8", 2: "fp4", 3: "fp8+bf16rope"}
 L2_BYTES = 126 * 2 ** 20
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
 # capture of that kernel in this workload (profiles/ holds the summary and the
@@ -111,7 +113,8 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ our arm
-ROW_BYTES = {0: 1024, 1: 516, 2: 288}     # one 512-channel cache row: bf16, fp8 + scale, fp4 + scales
+ROW_BYTES = {0: 1024, 1: 516, 2: 288, 3: 580}  # one 512-channel cache row: bf16, fp8 + scale, fp4 + scales,
+                                              # fp8 body + bf16 rotary channels + scale
 KEY_BYTES = {0: 256, 2: 72}               # one 128-channel indexer key: bf16, fp4 + scales
 
 
@@ -627,7 +630,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="c4a_b32")
-    ap.add_argument("--secondary", default="c128a_b8,c128a_b32,q_c4a_fp8,q_c4a_fp4,q_c128a_fp8,q_c128a_fp4",
+    ap.add_argument("--secondary", default="c128a_b8,c128a_b32,q_c4a_fp8,q_c4a_fp4,q_c128a_fp8,q_c128a_fp4,"
+                                           "q_c4a_fp8rope,q_c128a_fp8rope",
                     help="extra per-layer-type workloads (comma list, 'none' = none)")
     ap.add_argument("--no-stack", action="store_true", help="skip the 61-layer stack step")
     ap.add_argument("--no-bulk", action="store_true", help="skip compressor/quantiser throughput")

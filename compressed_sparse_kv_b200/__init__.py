@@ -17,7 +17,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libdsv4kv.so")
 
-BF16, FP8_E4M3_ROW, FP4_E2M1_G16 = 0, 1, 2
+BF16, FP8_E4M3_ROW, FP4_E2M1_G16, FP8_E4M3_ROW_ROPE_BF16 = 0, 1, 2, 3
 DEV_BAD_INDEX, DEV_TIMEOUT, DEV_INCONSISTENT = 0x1, 0x2, 0x4
 STATUS_NAMES = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED", 3: "ERR_WORKSPACE", 4: "ERR_CUDA"}
 
@@ -145,15 +145,18 @@ def compress(s_raw: torch.Tensor, w: torch.Tensor, stride: int, window: int, pos
 
 def quantize(x: torch.Tensor, fmt: int, codes: Optional[torch.Tensor] = None,
              scales: Optional[torch.Tensor] = None, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
-    """Rows x [..., D] (bf16 or f32) -> (codes, scales) in the fp8 or fp4 cache format."""
+    """Rows x [..., D] (bf16 or f32) -> (codes, scales) in a quantised cache format: fp8 rows
+    (codes [..., D], scales f32 [...]), fp4 (codes [..., D/2], E4M3 scales [..., D/16]) or fp8
+    with the last 64 channels in bf16 (row bytes [..., D + 64], scales f32 [...])."""
     d = int(x.shape[-1])
     rows = x.numel() // d
     lead = tuple(x.shape[:-1])
+    row_bytes = {FP8_E4M3_ROW: d, FP4_E2M1_G16: d // 2, FP8_E4M3_ROW_ROPE_BF16: d + 64}.get(fmt, d)
     if codes is None:
-        codes = torch.empty(lead + ((d,) if fmt == FP8_E4M3_ROW else (d // 2,)), dtype=torch.uint8, device=x.device)
+        codes = torch.empty(lead + (row_bytes,), dtype=torch.uint8, device=x.device)
     if scales is None:
-        scales = (torch.empty(lead, dtype=torch.float32, device=x.device) if fmt == FP8_E4M3_ROW
-                  else torch.empty(lead + (d // 16,), dtype=torch.uint8, device=x.device))
+        scales = (torch.empty(lead + (d // 16,), dtype=torch.uint8, device=x.device) if fmt == FP4_E2M1_G16
+                  else torch.empty(lead, dtype=torch.float32, device=x.device))
     _check(lib().dsv4kv_quantize(_ptr(x), int(x.dtype == torch.float32), rows, d, fmt, _ptr(codes), _ptr(scales),
                                  _stream(stream)), "dsv4kv_quantize")
     return codes, scales

@@ -94,7 +94,7 @@ static dsv4kv_status check_cache(const dsv4kv_cache* c, const char* what, int64_
   if (!c->codes || !aligned16(c->codes))
     return set_error(DSV4KV_ERR_INVALID_ARG, "%s: codes pointer null or not 16-byte aligned", what);
   if (c->fmt == DSV4KV_BF16) return DSV4KV_OK;
-  if (c->fmt == DSV4KV_FP8_E4M3_ROW || c->fmt == DSV4KV_FP4_E2M1_G16) {
+  if (c->fmt == DSV4KV_FP8_E4M3_ROW || c->fmt == DSV4KV_FP4_E2M1_G16 || c->fmt == DSV4KV_FP8_E4M3_ROW_ROPE_BF16) {
     if (!c->scales || !aligned16(c->scales))
       return set_error(DSV4KV_ERR_INVALID_ARG, "%s: scales pointer null or not 16-byte aligned", what);
     return DSV4KV_OK;
@@ -137,7 +137,7 @@ DSV4KV_API dsv4kv_status dsv4kv_quantize(const void* in, int32_t in_fp32, int64_
                                          void* codes, void* scales, void* stream) {
   g_err[0] = 0;
   if (rows < 0) return set_error(DSV4KV_ERR_INVALID_ARG, "quantize: rows < 0");
-  if (fmt != DSV4KV_FP8_E4M3_ROW && fmt != DSV4KV_FP4_E2M1_G16)
+  if (fmt != DSV4KV_FP8_E4M3_ROW && fmt != DSV4KV_FP4_E2M1_G16 && fmt != DSV4KV_FP8_E4M3_ROW_ROPE_BF16)
     return set_error(DSV4KV_ERR_UNSUPPORTED, "quantize: format %d is not a quantised format", fmt);
   if (rows == 0) return DSV4KV_OK;
   if (!in || !codes || !scales || !aligned16(in) || !aligned16(codes) || !aligned16(scales))

@@ -60,7 +60,7 @@ constexpr int kIdxSmem = 2048;             // selected indices a CTA keeps in sh
 template <int FMT>
 struct Cfg {
   static constexpr bool kQuant = FMT != DSV4KV_BF16;
-  static constexpr bool kRowScale = FMT == DSV4KV_FP8_E4M3_ROW;
+  static constexpr bool kRowScale = FMT == DSV4KV_FP8_E4M3_ROW || FMT == DSV4KV_FP8_E4M3_ROW_ROPE_BF16;
   static constexpr uint32_t kIdescQK = kQuant ? idesc_f16(64, 64, 0, 0) : idesc_bf16(64, 64, 0, 0);
   static constexpr uint32_t kIdescPV = kQuant ? idesc_f16(128, 64, 1, 0) : idesc_bf16(128, 64, 1, 0);
 };
@@ -674,6 +674,63 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           cp_async_wait_all();
+        } else if constexpr (FMT == DSV4KV_FP8_E4M3_ROW_ROPE_BF16) {
+          // rows of kDim + 64 bytes: lanes < 28 own 16 fp8 channels (16 code
+          // bytes), lanes 28..31 16 of the 64 bf16 rotary channels (32 bytes),
+          // stored as f16 of value / scale so that the row scale folds into
+          // the softmax weights exactly as for plain fp8 rows; two rounds of
+          // 8 rows keep the loads of a round in flight together
+          const uint8_t* codes = mine.from_win ? p.win_codes : p.comp_codes;
+          const float* scales = static_cast<const float*>(mine.from_win ? p.win_scales : p.comp_scales);
+          const float my_scale = (lane < 16 && mine.valid) ? scales[mine.row] : 0.f;
+          if (lane < 16) ctl->row_scale[stage][16 * lw + lane] = my_scale;
+          const bool rope_lane = lane >= 28;
+          const int chunk = lane >> 2, u0 = (lane & 3) * 2;  // lane owns channels [16*lane, 16*lane+16)
+          uint8_t* ctile = tile + chunk * kChunkBytes;
+#pragma unroll
+          for (int hb = 0; hb < 2; ++hb) {
+            uint4 ra[8], rb[8];
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+              const int j = 8 * hb + jj;
+              const int64_t row = __shfl_sync(kFull, mine.row, j);
+              const bool valid = __shfl_sync(kFull, mine.valid, j);
+              const uint8_t* rp = codes + size_t(row) * (kDim + 64);
+              if (!valid) {
+                ra[jj] = rb[jj] = make_uint4(0, 0, 0, 0);
+              } else if (rope_lane) {
+                const uint8_t* src = rp + (kDim - 64) + 32 * (lane - 28);
+                ra[jj] = ld_stream_v4(src);
+                rb[jj] = ld_stream_v4(src + 16);
+              } else {
+                ra[jj] = ld_stream_v4(rp + 16 * lane);
+                rb[jj] = make_uint4(0, 0, 0, 0);
+              }
+            }
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+              const int j = 8 * hb + jj;
+              const int r = 16 * lw + j;
+              const float s = __shfl_sync(kFull, my_scale, j);
+              uint32_t hv[8];
+              if (rope_lane) {
+                const float inv = s > 0.f ? 1.f / s : 0.f;
+                const uint32_t w[8] = {ra[jj].x, ra[jj].y, ra[jj].z, ra[jj].w, rb[jj].x, rb[jj].y, rb[jj].z, rb[jj].w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) hv[e] = f32x2_to_f16x2_sat(bf16lo(w[e]) * inv, bf16hi(w[e]) * inv);
+              } else {
+                const uint32_t w[4] = {ra[jj].x, ra[jj].y, ra[jj].z, ra[jj].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  hv[2 * e] = e4m3x2_to_f16x2(w[e] & 0xffffu);
+                  hv[2 * e + 1] = e4m3x2_to_f16x2(w[e] >> 16);
+                }
+              }
+              uint8_t* line = ctile + r * 128;
+              *reinterpret_cast<uint4*>(line + ((u0 ^ (r & 7)) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+              *reinterpret_cast<uint4*>(line + (((u0 + 1) ^ (r & 7)) << 4)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+            }
+          }
         } else {
           const uint8_t* codes = mine.from_win ? p.win_codes : p.comp_codes;
           const void* scales = mine.from_win ? p.win_scales : p.comp_scales;
@@ -1070,8 +1127,11 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
   const int fmt = a.comp.fmt;
   if (a.win.fmt != fmt)
     return set_error(DSV4KV_ERR_UNSUPPORTED, "decode: the window cache must have the compressed cache's format");
-  if (fmt != DSV4KV_BF16 && fmt != DSV4KV_FP8_E4M3_ROW && fmt != DSV4KV_FP4_E2M1_G16)
+  if (fmt != DSV4KV_BF16 && fmt != DSV4KV_FP8_E4M3_ROW && fmt != DSV4KV_FP4_E2M1_G16 &&
+      fmt != DSV4KV_FP8_E4M3_ROW_ROPE_BF16)
     return set_error(DSV4KV_ERR_UNSUPPORTED, "decode: unknown cache format %d", fmt);
+  if (fmt == DSV4KV_FP8_E4M3_ROW_ROPE_BF16 && a.rope_dim != 64)
+    return set_error(DSV4KV_ERR_UNSUPPORTED, "decode: fp8 rows with bf16 rotary channels need rope_dim == 64");
   const int slots = a.idx ? a.k : int(a.n);
   const int comp_tiles = (a.n > 0 && slots > 0) ? (slots + kTileRows - 1) / kTileRows : 0;
   const int win_tiles = (a.window + kTileRows - 1) / kTileRows;
@@ -1134,6 +1194,9 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
   switch (fmt) {
     case DSV4KV_BF16: st = launch_fmt<DSV4KV_BF16>(tq, tc, tw, p, grid, stream); break;
     case DSV4KV_FP8_E4M3_ROW: st = launch_fmt<DSV4KV_FP8_E4M3_ROW>(tq, tc, tw, p, grid, stream); break;
+    case DSV4KV_FP8_E4M3_ROW_ROPE_BF16:
+      st = launch_fmt<DSV4KV_FP8_E4M3_ROW_ROPE_BF16>(tq, tc, tw, p, grid, stream);
+      break;
     default: st = launch_fmt<DSV4KV_FP4_E2M1_G16>(tq, tc, tw, p, grid, stream); break;
   }
   if (st != DSV4KV_OK || pl.splits == 1) return st;  // one split: the decode kernel stored the output

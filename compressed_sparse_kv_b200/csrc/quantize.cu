@@ -9,6 +9,10 @@
 //             code = E4M3_rn_satfinite(fp32(x / scale)).
 //   fp4 group of 16: s = E4M3_rn_satfinite(fp32(amax / 6));
 //             code = E2M1_rn_satfinite(fp32(x / value(s))), 0 when value(s) == 0.
+//   fp8 with bf16 rotary channels ([P1]: the RoPE dimensions stay in bf16):
+//             the fp8 row rule over the first D - 64 channels (amax over
+//             those only), then the last 64 channels as bf16 (nearest even);
+//             a row is D - 64 code bytes followed by the 64 bf16 values.
 // Divisions are IEEE round-to-nearest (__fdiv_rn); conversions use the
 // hardware cvt.rn.satfinite instructions.  One warp per row.
 #include <cstdint>
@@ -70,7 +74,37 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock)
       x[4 * v + 3] = bf16hi(u.y);
     }
   }
-  if (FMT == DSV4KV_FP8_E4M3_ROW) {
+  if (FMT == DSV4KV_FP8_E4M3_ROW_ROPE_BF16) {
+    // lanes [0, BL) hold the fp8 body, lanes [BL, 32) the 64 rotary channels
+    constexpr int BL = 32 - 64 / PER;
+    const bool body = lane < BL;
+    float amax = 0.f;
+    if (body) {
+#pragma unroll
+      for (int e = 0; e < PER; ++e) amax = fmaxf(amax, fabsf(x[e]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+    const float scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    uint8_t* row_dst = codes + size_t(row) * (D + 64);
+    if (body) {
+      uint32_t packed[PER / 4];
+#pragma unroll
+      for (int v = 0; v < PER / 4; ++v) {
+        const uint32_t lo = cvt_e4m3x2(__fdiv_rn(x[4 * v + 1], scale), __fdiv_rn(x[4 * v], scale));
+        const uint32_t hi = cvt_e4m3x2(__fdiv_rn(x[4 * v + 3], scale), __fdiv_rn(x[4 * v + 2], scale));
+        packed[v] = lo | (hi << 16);
+      }
+#pragma unroll
+      for (int v = 0; v < PER / 4; ++v) reinterpret_cast<uint32_t*>(row_dst + PER * lane)[v] = packed[v];
+    } else {
+      // bf16 of fp32 input rounds to nearest even; bf16 input is reproduced exactly
+      uint32_t* dst = reinterpret_cast<uint32_t*>(row_dst + (D - 64) + 2 * PER * (lane - BL));
+#pragma unroll
+      for (int v = 0; v < PER / 2; ++v) dst[v] = pack_bf16x2(x[2 * v], x[2 * v + 1]);
+    }
+    if (lane == 0) static_cast<float*>(scales)[row] = scale;
+  } else if (FMT == DSV4KV_FP8_E4M3_ROW) {
     float amax = 0.f;
 #pragma unroll
     for (int e = 0; e < PER; ++e) amax = fmaxf(amax, fabsf(x[e]));
@@ -141,6 +175,11 @@ dsv4kv_status launch_per(const void* in, int in_fp32, int64_t rows, int fmt, voi
   if (fmt == DSV4KV_FP8_E4M3_ROW) {
     if (in_fp32) quantize_kernel<PER, true, DSV4KV_FP8_E4M3_ROW><<<grid, block, 0, stream>>>(in, rows, c, scales);
     else quantize_kernel<PER, false, DSV4KV_FP8_E4M3_ROW><<<grid, block, 0, stream>>>(in, rows, c, scales);
+  } else if (fmt == DSV4KV_FP8_E4M3_ROW_ROPE_BF16) {
+    if (in_fp32)
+      quantize_kernel<PER, true, DSV4KV_FP8_E4M3_ROW_ROPE_BF16><<<grid, block, 0, stream>>>(in, rows, c, scales);
+    else
+      quantize_kernel<PER, false, DSV4KV_FP8_E4M3_ROW_ROPE_BF16><<<grid, block, 0, stream>>>(in, rows, c, scales);
   } else {
     if (in_fp32) quantize_kernel<PER, true, DSV4KV_FP4_E2M1_G16><<<grid, block, 0, stream>>>(in, rows, c, scales);
     else quantize_kernel<PER, false, DSV4KV_FP4_E2M1_G16><<<grid, block, 0, stream>>>(in, rows, c, scales);

@@ -59,11 +59,20 @@ typedef enum {
  *                        even channel in the low nibble; scales = u8 [B][rows][dim/16] E4M3,
  *                        one per 16 channels; value = E2M1(code) * E4M3(scale).
  *                        ([P3] "storing the main KV in FP4"; [P1] "indexer cache uses fp4")
+ *  DSV4KV_FP8_E4M3_ROW_ROPE_BF16: the last 64 (rotary) channels kept in bf16, the other
+ *                        dim - 64 in fp8 under one fp32 scale per row.  codes = u8
+ *                        [B][rows][dim + 64]: dim - 64 OCP E4M3 codes, then the 64 bf16
+ *                        values (little-endian, 128 bytes); scales = float [B][rows];
+ *                        value = E4M3(code) * scale for channels < dim - 64, the bf16 value
+ *                        for the rest.  ([P1] quantisation paragraph: fp8 for most of the
+ *                        attention cache, the RoPE dimensions in bf16.)  With this format
+ *                        the decode calls require rope_dim == 64.
  */
 typedef enum {
   DSV4KV_BF16 = 0,
   DSV4KV_FP8_E4M3_ROW = 1,
-  DSV4KV_FP4_E2M1_G16 = 2
+  DSV4KV_FP4_E2M1_G16 = 2,
+  DSV4KV_FP8_E4M3_ROW_ROPE_BF16 = 3
 } dsv4kv_format;
 
 /* A cache tensor of `batch` sequences x `rows` rows x `dim` channels.
@@ -108,9 +117,13 @@ dsv4kv_status dsv4kv_compress(const void* s_raw, const float* w, int32_t batch, 
  *   DSV4KV_FP4_E2M1_G16: s = E4M3(fp32(amax16 / 6)) (nearest even,
  *       saturating), code = E2M1(fp32(x / s)) nearest even, saturating;
  *       codes are 0 when s == 0.
+ *   DSV4KV_FP8_E4M3_ROW_ROPE_BF16: the fp8 row rule over channels
+ *       [0, dim - 64) (amax over those channels only); channels
+ *       [dim - 64, dim) rounded to bf16 (nearest even; bf16 input is copied).
  *   in     : bf16 or (in_fp32 != 0) float, [rows][dim]
- *   codes  : u8 [rows][dim] (fp8) or [rows][dim/2] (fp4)
- *   scales : float [rows] (fp8) or u8 [rows][dim/16] (fp4)
+ *   codes  : u8 [rows][dim] (fp8), [rows][dim/2] (fp4) or [rows][dim + 64]
+ *            (fp8 with bf16 rotary channels)
+ *   scales : float [rows] (fp8 formats) or u8 [rows][dim/16] (fp4)
  * Requirements: dim in {128, 256, 512, 1024}; fmt != DSV4KV_BF16.
  * ------------------------------------------------------------------------ */
 dsv4kv_status dsv4kv_quantize(const void* in, int32_t in_fp32, int64_t rows, int32_t dim,

@@ -15,8 +15,11 @@ from tests._util import assert_close, to_f64
 
 pytestmark = pytest.mark.gpu
 SCALE = 512 ** -0.5
-QUANT = {K.FP8_E4M3_ROW: OF.quantize_fp8_rows, K.FP4_E2M1_G16: OF.quantize_fp4_rows}
-DEQ = {K.FP8_E4M3_ROW: OF.dequant_fp8_rows, K.FP4_E2M1_G16: OF.dequant_fp4_rows}
+QUANT = {K.FP8_E4M3_ROW: OF.quantize_fp8_rows, K.FP4_E2M1_G16: OF.quantize_fp4_rows,
+         K.FP8_E4M3_ROW_ROPE_BF16: OF.quantize_fp8_rope_rows}
+DEQ = {K.FP8_E4M3_ROW: OF.dequant_fp8_rows, K.FP4_E2M1_G16: OF.dequant_fp4_rows,
+       K.FP8_E4M3_ROW_ROPE_BF16: OF.dequant_fp8_rope_rows}
+FMTS = [K.FP8_E4M3_ROW, K.FP4_E2M1_G16, K.FP8_E4M3_ROW_ROPE_BF16]
 
 
 def _states(key, b, rows):
@@ -42,7 +45,7 @@ def _qh(kq, s, h):
     return OF.bf16_bits_to_f64(D.rows_normal_bf16(kq, np.arange(s * h, (s + 1) * h), 512))
 
 
-@pytest.mark.parametrize("fmt", [K.FP8_E4M3_ROW, K.FP4_E2M1_G16])
+@pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("b,h,n,window,t", [
     (1, 16, 0, 128, 128),
     (2, 64, 100, 128, 13000),
@@ -64,7 +67,7 @@ def test_dense_decode_quantised(fmt, b, h, n, window, t):
         assert_close(got[s], ref, what=f"fmt {fmt} seq {s}")
 
 
-@pytest.mark.parametrize("fmt", [K.FP8_E4M3_ROW, K.FP4_E2M1_G16])
+@pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("b,h,n,k,cnt,t", [
     (2, 64, 3000, 512, 512, 20000),
     (2, 16, 300, 512, 300, 2000),
@@ -110,3 +113,31 @@ def test_fp8_rows_with_large_scales():
         ref = OA.dense_decode(OF.bf16_bits_to_f64(qb[s])[None], cr[None], wr[None], t, SCALE)[0]
         mag = max(1.0, np.abs(ref).max())
         assert_close(got[s] / mag, ref / mag, what=f"seq {s}")
+
+
+def test_fp8_rope_rows_with_large_rotary_channels():
+    """fp8 rows with bf16 rotary channels whose rotary values are 50 times the
+    body's: the rotary channels are staged as f16 of value / row scale (here
+    up to ~2e4, inside the f16 range), so the output still matches."""
+    fmt = K.FP8_E4M3_ROW_ROPE_BF16
+    b, h, n, window, t = 2, 64, 700, 128, 9000
+    kq, kc, kw = (D.stream_key(91, x, 0) for x in (D.TID_Q, D.TID_STATES, D.TID_WIN))
+    import datagen.gpu as G
+    q = G.normal_bf16_(torch.empty(b, h, 512, dtype=torch.bfloat16, device="cuda"), kq)
+    q = (q.float() / 16).to(torch.bfloat16)        # keep the softmax from collapsing onto one row
+    st = _states(kc, b, n).float()
+    st[..., 448:] *= 50.0
+    st = st.to(torch.bfloat16)
+    cc, cs = K.quantize(st, fmt)
+    wc, wsc = K.quantize(_states(kw, b, window), fmt)
+    out = K.dense_decode(q, K.Cache(fmt, cc, cs), K.Cache(fmt, wc, wsc), n, window, t, SCALE, out_fp32=True)
+    got = to_f64(out)
+    qb = q.view(torch.int16).cpu().numpy().view(np.uint16)
+    sb = st.view(torch.int16).cpu().numpy().view(np.uint16)
+    for s in range(b):
+        cr = OF.dequant_fp8_rope_rows(*OF.quantize_fp8_rope_rows(OF.bf16_bits_to_f64(sb[s]).astype(np.float32)))
+        wr = _host_rows(fmt, kw, np.arange(s * window, (s + 1) * window))
+        ref = OA.dense_decode(OF.bf16_bits_to_f64(qb[s])[None], cr[None], wr[None], t, SCALE)[0]
+        # outputs of the rotary channels reach ~50x the usual magnitude: the
+        # absolute bound scales with them (the relative bound is unchanged)
+        assert_close(got[s], ref, max_abs=50 * 1e-2, what=f"seq {s}")

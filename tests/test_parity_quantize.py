@@ -20,7 +20,7 @@ def _special_rows(d):
     return np.stack(rows)
 
 
-@pytest.mark.parametrize("fmt", [K.FP8_E4M3_ROW, K.FP4_E2M1_G16])
+@pytest.mark.parametrize("fmt", [K.FP8_E4M3_ROW, K.FP4_E2M1_G16, K.FP8_E4M3_ROW_ROPE_BF16])
 @pytest.mark.parametrize("d", [128, 512])
 @pytest.mark.parametrize("in_fp32", [False, True])
 def test_quantize_bit_exact(fmt, d, in_fp32):
@@ -39,6 +39,10 @@ def test_quantize_bit_exact(fmt, d, in_fp32):
     codes, scales = K.quantize(xin, fmt)
     if fmt == K.FP8_E4M3_ROW:
         rc, rs = OF.quantize_fp8_rows(x32)
+        assert np.array_equal(scales.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    elif fmt == K.FP8_E4M3_ROW_ROPE_BF16:
+        rc, rs = OF.quantize_fp8_rope_rows(x32)
+        assert codes.shape[-1] == d + 64
         assert np.array_equal(scales.cpu().numpy().view(np.uint32), rs.view(np.uint32))
     else:
         rc, rs = OF.quantize_fp4_rows(x32)
