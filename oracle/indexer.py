@@ -35,3 +35,22 @@ def topk(score, k: int) -> tuple[np.ndarray, int]:
 
 def index_topk(q, keys, k: int) -> tuple[np.ndarray, int]:
     return topk(scores(q, keys), k)
+
+
+def index_topk_pool(q, keys, pool, k: int) -> tuple[np.ndarray, int]:
+    """Re-index inside a candidate pool ([P3] CSA2: "Reindex" layers keep their
+    indexing inside the candidate pool built by the first layer in Full mode;
+    layers share the indexer keys).  pool: entry indices (negative = no
+    entry).  Among the pool entries, the first min(k, |pool|) under (score
+    descending, entry index ascending), returned in ascending entry order,
+    padded with -1 to k.  Reading: the pool is a set of entry indices; its
+    size is the caller's choice (the pages give none)."""
+    pool = np.asarray(pool, dtype=np.int64)
+    ent = pool[pool >= 0]
+    s = scores(q, np.asarray(keys)[ent])
+    order = np.lexsort((ent, -s))                   # score desc, then entry index asc
+    cnt = min(k, ent.shape[0])
+    sel = np.sort(ent[order[:cnt]])
+    out = np.full(k, -1, dtype=np.int32)
+    out[:cnt] = sel
+    return out, cnt

@@ -59,3 +59,42 @@ def test_split_then_merge_equals_global():
     cand = np.array(sorted(cand))
     sub, c = I.topk(s[cand], 512)
     assert list(cand[sub[:c]]) == list(glob)
+
+
+# ------------------------------------------------------------ pool re-index
+def _int_data(seed, n, di=128):
+    rng = np.random.default_rng(seed)
+    return rng.integers(-8, 9, di).astype(np.float64), rng.integers(-8, 9, (n, di)).astype(np.float64)
+
+
+def test_pool_of_everything_is_the_full_selection():
+    q, keys = _int_data(3, 3000)
+    full, c1 = I.index_topk(q, keys, 512)
+    pooled, c2 = I.index_topk_pool(q, keys, np.arange(3000), 512)
+    assert c1 == c2 and np.array_equal(full, pooled)
+
+
+def test_pool_against_brute_force_and_padding():
+    q, keys = _int_data(4, 5000)
+    rng = np.random.default_rng(9)
+    pool = np.sort(rng.choice(5000, 1500, replace=False))
+    padded = np.concatenate([pool, -np.ones(548, dtype=np.int64)])
+    got, cnt = I.index_topk_pool(q, keys, padded, 512)
+    # brute force: rank every pool entry by (score desc, index asc) with Python tuples
+    s = {int(i): float(keys[i] @ q) for i in pool}
+    ranked = sorted(pool.tolist(), key=lambda i: (-s[i], i))
+    assert cnt == 512
+    assert got.tolist() == sorted(ranked[:512])
+    # a pool smaller than k: everything, ascending, padded
+    small, c = I.index_topk_pool(q, keys, pool[:100], 512)
+    assert c == 100 and small[:100].tolist() == pool[:100].tolist() and np.all(small[100:] == -1)
+
+
+def test_pool_order_and_duplicated_scores():
+    """The pool's order does not matter; equal scores go to the lower entry."""
+    keys = np.zeros((50, 128))
+    keys[[7, 3, 41, 12], 0] = 1.0                  # four equal top scores
+    q = np.zeros(128)
+    q[0] = 1.0
+    got, cnt = I.index_topk_pool(q, keys, np.array([41, 12, 7, 3, 20, 30]), 3)
+    assert cnt == 3 and got.tolist() == [3, 7, 12]
