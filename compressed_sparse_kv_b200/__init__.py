@@ -18,7 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libdsv4kv.so")
 
 BF16, FP8_E4M3_ROW, FP4_E2M1_G16, FP8_E4M3_ROW_ROPE_BF16 = 0, 1, 2, 3
-DEV_BAD_INDEX, DEV_TIMEOUT, DEV_INCONSISTENT = 0x1, 0x2, 0x4
+DEV_BAD_INDEX, DEV_TIMEOUT, DEV_INCONSISTENT, DEV_BAD_POOL = 0x1, 0x2, 0x4, 0x8
 STATUS_NAMES = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED", 3: "ERR_WORKSPACE", 4: "ERR_CUDA"}
 
 
@@ -50,6 +50,10 @@ _SIGS = {
                                      _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "dsv4kv_index_score": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.c_int32, _c.c_int64, _c.c_int32,
                                       _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "dsv4kv_index_topk_pool_workspace_bytes": (_c.c_size_t, [_c.c_int32, _c.c_int32, _c.c_int32]),
+    "dsv4kv_index_topk_pool": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.c_int32, _c.c_int64, _c.c_void_p,
+                                          _c.c_int32, _c.c_int32, _c.c_void_p, _c.c_void_p, _c.c_void_p,
+                                          _c.c_size_t, _c.c_void_p]),
     "dsv4kv_index_select": (_c.c_int, [_c.c_int32, _c.c_int64, _c.c_int32, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                        _c.c_size_t, _c.c_void_p]),
     "dsv4kv_index_topk_noalloc_max_scratch_bytes": (_c.c_size_t, []),
@@ -196,6 +200,26 @@ def index_select(batch: int, n: int, k: int, idx_out: torch.Tensor, count_out: O
     """The selection half of index_topk, from the workspace index_score filled."""
     _check(lib().dsv4kv_index_select(batch, n, k, _ptr(idx_out), _ptr(count_out) if count_out is not None else None,
                                      _ptr(ws), ws.numel(), _stream(stream)), "dsv4kv_index_select")
+    return idx_out, count_out
+
+
+def index_topk_pool(qidx: torch.Tensor, keys: Cache, n: int, pool: torch.Tensor, k: int,
+                    idx_out: Optional[torch.Tensor] = None, count_out: Optional[torch.Tensor] = None,
+                    ws: Optional[torch.Tensor] = None, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Top-k re-index inside a candidate pool: pool int32 [B][P] (ascending entries, negative = none)
+    -> (idx int32 [B][k] ascending, -1 padded; count int32 [B])."""
+    b = int(qidx.shape[0])
+    p = int(pool.shape[1]) if pool.dim() == 2 else 0
+    if idx_out is None:
+        idx_out = torch.empty((b, k), dtype=torch.int32, device=qidx.device)
+    if count_out is None:
+        count_out = torch.empty((b,), dtype=torch.int32, device=qidx.device)
+    if ws is None:
+        ws = new_workspace(int(lib().dsv4kv_index_topk_pool_workspace_bytes(b, p, k)), qidx.device)
+    d = keys.desc()
+    _check(lib().dsv4kv_index_topk_pool(_ptr(qidx), ctypes.byref(d), b, n, _ptr(pool), p, k, _ptr(idx_out),
+                                        _ptr(count_out), _ptr(ws), ws.numel(), _stream(stream)),
+           "dsv4kv_index_topk_pool")
     return idx_out, count_out
 
 

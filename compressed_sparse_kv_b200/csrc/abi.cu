@@ -201,6 +201,32 @@ DSV4KV_API dsv4kv_status dsv4kv_index_select(int32_t batch, int64_t n, int32_t k
   return index_select_launch(batch, n, k, idx_out, count_out, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
+DSV4KV_API size_t dsv4kv_index_topk_pool_workspace_bytes(int32_t batch, int32_t pool_cap, int32_t k) {
+  if (batch < 0 || pool_cap < 0 || k < 1) return 0;
+  return 16;  // the status word
+}
+
+DSV4KV_API dsv4kv_status dsv4kv_index_topk_pool(const void* qidx, const dsv4kv_cache* keys, int32_t batch, int64_t n,
+                                                const int32_t* pool, int32_t pool_cap, int32_t k, int32_t* idx_out,
+                                                int32_t* count_out, void* ws, size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  if (batch < 0 || n < 0 || pool_cap < 0) return set_error(DSV4KV_ERR_INVALID_ARG, "index_topk_pool: bad sizes");
+  if (k < 1 || k > 2048) return set_error(DSV4KV_ERR_UNSUPPORTED, "index_topk_pool: k must be in [1, 2048]");
+  if (pool_cap > 8192) return set_error(DSV4KV_ERR_UNSUPPORTED, "index_topk_pool: pool_cap must be <= 8192");
+  if (batch == 0) return DSV4KV_OK;
+  if (!idx_out) return set_error(DSV4KV_ERR_INVALID_ARG, "index_topk_pool: idx_out is null");
+  if (pool_cap > 0 && !pool) return set_error(DSV4KV_ERR_INVALID_ARG, "index_topk_pool: pool is null");
+  if (!keys) return set_error(DSV4KV_ERR_INVALID_ARG, "index_topk_pool: keys is null");
+  if (keys->fmt != DSV4KV_BF16 && keys->fmt != DSV4KV_FP4_E2M1_G16)
+    return set_error(DSV4KV_ERR_UNSUPPORTED, "index_topk_pool: keys must be bf16 or fp4");
+  dsv4kv_status st = check_cache(keys, "index_topk_pool", n, 128);
+  if (st != DSV4KV_OK) return st;
+  if (!qidx || !aligned16(qidx)) return set_error(DSV4KV_ERR_INVALID_ARG, "index_topk_pool: qidx null or misaligned");
+  if (!ws || ws_bytes < 16) return set_error(DSV4KV_ERR_WORKSPACE, "index_topk_pool: workspace null or too small");
+  return index_topk_pool_launch(static_cast<const uint16_t*>(qidx), *keys, batch, n, pool, pool_cap, k, idx_out,
+                                count_out, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
 static dsv4kv_status check_decode(const void* q, const dsv4kv_cache* comp, const dsv4kv_cache* win, int32_t batch,
                                   int32_t heads, int64_t n, int32_t window, int64_t need_comp_rows, const void* out) {
   if (batch < 1) return set_error(DSV4KV_ERR_INVALID_ARG, "decode: batch must be >= 1");

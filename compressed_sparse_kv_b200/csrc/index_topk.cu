@@ -930,6 +930,270 @@ __global__ void index_fill_all(int64_t n, int k, int32_t* __restrict__ idx_out, 
   if (count_out && blockIdx.x == 0 && threadIdx.x == 0) count_out[b] = int32_t(n);
 }
 
+// ------------------------------------------------------------------ pool re-index
+// [P3] CSA2: a "Reindex" layer keeps its indexing inside the candidate pool
+// built by the first layer in Full mode (the layers share the indexer keys).
+// One CTA of 512 threads per sequence: the pool (ascending entry indices,
+// negative = no entry) is copied to shared memory, the pool's keys are
+// gathered and scored (half a warp per bf16 key, a quarter warp per fp4 key)
+// into shared memory as order-preserving codes, and the exact selection runs
+// there: the 12-bit histogram gives the threshold bin, a second 12-bit
+// histogram of that bin the 24-bit prefix, a 256-bin histogram of the
+// entries at the prefix the threshold code, and the entries equal to it are
+// taken in pool order (= entry order, so ties go to the lower entry); an
+// ordered compaction over pool positions writes the result ascending.
+constexpr int kPoolMax = 8192;
+constexpr int kPoolPer = kPoolMax / kSelThreads;  // pool positions per thread
+constexpr size_t kPoolDyn = 2 * size_t(kPoolMax) * sizeof(uint32_t);
+
+// The bin where the descending cumulative count of a 256-bin histogram first
+// reaches `need`; *above = count in higher bins.  Warp 0 scans (8 bins per
+// lane), one block barrier publishes the result.
+__device__ int find_threshold_bin256(const uint32_t* h, uint32_t need, uint32_t* above) {
+  __shared__ int s_bin;
+  __shared__ uint32_t s_above;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int lo = 256 - 8 * (lane + 1);  // lane 0 owns the highest 8 bins
+    uint32_t v[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[i] = h[lo + i];
+      sum += v[i];
+    }
+    const uint32_t incl = warp_inclusive_scan(sum);
+    const uint32_t ex = incl - sum;
+    if (ex < need && ex + sum >= need) {
+      uint32_t c = ex;
+#pragma unroll
+      for (int i = 7; i >= 0; --i) {
+        if (c < need && c + v[i] >= need) {
+          s_bin = lo + i;
+          s_above = c;
+        }
+        c += v[i];
+      }
+    }
+  }
+  __syncthreads();
+  *above = s_above;
+  const int r = s_bin;
+  __syncthreads();
+  return r;
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kSelThreads, 1)
+    index_pool_select(const uint16_t* __restrict__ qidx, const void* __restrict__ codes,
+                      const uint8_t* __restrict__ kscales, int64_t key_rows, int64_t n,
+                      const int32_t* __restrict__ pool, int pool_cap, int k, int32_t* __restrict__ idx_out,
+                      int32_t* __restrict__ count_out, uint32_t* __restrict__ status) {
+  extern __shared__ __align__(16) uint32_t psm[];
+  uint32_t* pcode = psm;              // kPoolMax order-preserving codes (0 = no entry)
+  int32_t* pent = reinterpret_cast<int32_t*>(psm + kPoolMax);  // the pool's entries
+  __shared__ __align__(16) uint32_t sh[kHistBins];
+  __shared__ uint32_t s_cnt;
+  const int b = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int32_t* pb = pool + size_t(b) * pool_cap;
+  for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) sh[i] = 0;
+  if (threadIdx.x == 0) s_cnt = 0;
+  pdl_trigger();
+  pdl_wait();
+  // the pool, and its validity: entries in [0, n), ascending
+  for (int j = threadIdx.x; j < pool_cap; j += kSelThreads) {
+    const int32_t e = pb[j];
+    pent[j] = e;
+    if (e >= n) set_status(status, DSV4KV_DEV_BAD_INDEX);
+    if (e >= 0 && j > 0 && !(pb[j - 1] >= 0 && pb[j - 1] < e)) set_status(status, DSV4KV_DEV_BAD_POOL);
+  }
+  __syncthreads();
+  const uint64_t pol = l2_evict_first_policy();
+  if constexpr (FMT == DSV4KV_BF16) {
+    // half-warp hw scores positions hw, hw + 32, ...; 16 keys in flight per
+    // half-warp.  The loop bound is the same for every thread (positions past
+    // the pool are masked) so that the shuffles always see the whole warp.
+    constexpr int U = 16;
+    const int half = lane >> 4, l16 = lane & 15, hw = 2 * warp + half;
+    float q[8];
+    {
+      const uint4 v = *reinterpret_cast<const uint4*>(qidx + size_t(b) * 128 + 8 * l16);
+      q[0] = bf16lo(v.x); q[1] = bf16hi(v.x); q[2] = bf16lo(v.y); q[3] = bf16hi(v.y);
+      q[4] = bf16lo(v.z); q[5] = bf16hi(v.z); q[6] = bf16lo(v.w); q[7] = bf16hi(v.w);
+    }
+    const uint16_t* kb = static_cast<const uint16_t*>(codes) + size_t(b) * size_t(key_rows) * 128 + 8 * l16;
+    for (int it = 0; it * 32 * U < pool_cap; ++it) {
+      const int j0 = hw + 32 * U * it;
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = j0 + 32 * u;
+        const int32_t e = j < pool_cap ? pent[j] : -1;
+        v[u] = (e >= 0 && e < n) ? ld_once_v4(kb + size_t(e) * 128, pol) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = j0 + 32 * u;
+        float sc = dot8_bf16(v[u], q);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) sc += __shfl_xor_sync(kFull, sc, o);
+        sc += 0.0f;  // -0 -> +0
+        if (l16 == 0 && j < pool_cap) {
+          const int32_t e = pent[j];
+          const bool ok = e >= 0 && e < n;
+          const uint32_t c = ok ? ord_f32(sc) : 0u;
+          pcode[j] = c;
+          if (ok) {
+            atomicAdd(&sh[c >> 20], 1u);
+            atomicAdd(&s_cnt, 1u);
+          }
+        }
+      }
+    }
+  } else {
+    // fp4 keys: a quarter warp per key, lane l4 owns channels [32 l4, 32 l4 + 32);
+    // a loop bound common to all threads, as above
+    constexpr int U = 8;
+    const int quad = threadIdx.x >> 2, l4 = lane & 3;  // 128 quads
+    uint32_t qp[16];
+    {
+      const uint16_t* qb = qidx + size_t(b) * 128 + 32 * l4;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) qp[j] = f32x2_to_f16x2(bf16f(qb[2 * j]), bf16f(qb[2 * j + 1]));
+    }
+    const uint8_t* cb = static_cast<const uint8_t*>(codes) + size_t(b) * size_t(key_rows) * 64 + 16 * l4;
+    const uint8_t* sb = kscales + size_t(b) * size_t(key_rows) * 8 + 2 * l4;
+    for (int it = 0; it * 128 * U < pool_cap; ++it) {
+      const int j0 = quad + 128 * U * it;
+      uint4 v[U];
+      uint32_t s2[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = j0 + 128 * u;
+        const int32_t e = j < pool_cap ? pent[j] : -1;
+        const bool ok = e >= 0 && e < n;
+        v[u] = ok ? ld_once_v4(cb + size_t(e) * 64, pol) : make_uint4(0, 0, 0, 0);
+        s2[u] = ok ? ld_once_u16(sb + size_t(e) * 8, pol) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = j0 + 128 * u;
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        uint32_t acc0 = 0, acc1 = 0;
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+          uint32_t h[4];
+          e2m1x8_unpack(w[wi], h);
+#pragma unroll
+          for (int by = 0; by < 4; ++by) {
+            if (wi < 2) acc0 = hfma2(qp[4 * wi + by], h[by], acc0);
+            else acc1 = hfma2(qp[4 * wi + by], h[by], acc1);
+          }
+        }
+        float sc = f16x2_sum(acc0) * e4m3_to_f32(s2[u] & 0xffu) + f16x2_sum(acc1) * e4m3_to_f32(s2[u] >> 8);
+        sc += __shfl_xor_sync(kFull, sc, 1);
+        sc += __shfl_xor_sync(kFull, sc, 2);
+        sc += 0.0f;
+        if (l4 == 0 && j < pool_cap) {
+          const int32_t e = pent[j];
+          const bool ok = e >= 0 && e < n;
+          const uint32_t c = ok ? ord_f32(sc) : 0u;
+          pcode[j] = c;
+          if (ok) {
+            atomicAdd(&sh[c >> 20], 1u);
+            atomicAdd(&s_cnt, 1u);
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t cnt = s_cnt;
+  const uint32_t kk = min(uint32_t(k), cnt);
+  uint32_t c[kPoolPer];
+#pragma unroll
+  for (int j = 0; j < kPoolPer; ++j) {
+    const int pos = threadIdx.x + j * kSelThreads;
+    c[j] = pos < pool_cap ? pcode[pos] : 0u;
+  }
+  // the threshold code o* and how many entries equal to it are needed
+  uint32_t ostar = 1u, need_eq = 0xffffffffu;  // every valid entry (codes >= 1) when cnt <= k
+  if (cnt > uint32_t(k)) {
+    uint32_t above1, above2, above3;
+    const int bin1 = find_threshold_bin<kSelThreads>(sh, kk, &above1);
+    for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) sh[i] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kPoolPer; ++j)
+      if (c[j] != 0u && int(c[j] >> 20) == bin1) atomicAdd(&sh[(c[j] >> 8) & 0xfffu], 1u);
+    __syncthreads();
+    const int bin2 = find_threshold_bin<kSelThreads>(sh, kk - above1, &above2);
+    const uint32_t prefix = (uint32_t(bin1) << 12) | uint32_t(bin2);
+    for (int i = threadIdx.x; i < 256; i += kSelThreads) sh[i] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kPoolPer; ++j)
+      if (c[j] != 0u && (c[j] >> 8) == prefix) atomicAdd(&sh[c[j] & 0xffu], 1u);
+    __syncthreads();
+    const int bin3 = find_threshold_bin256(sh, kk - above1 - above2, &above3);
+    ostar = (prefix << 8) | uint32_t(bin3);
+    need_eq = kk - above1 - above2 - above3;
+  }
+  // ranks of the entries equal to o*, in pool order
+  uint32_t m[kPoolPer], off[kPoolPer];
+#pragma unroll
+  for (int j = 0; j < kPoolPer; ++j) m[j] = __ballot_sync(kFull, cnt > uint32_t(k) && c[j] == ostar);
+  ordered_offsets<kSelThreads, kPoolPer>(m, off);
+  const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int j = 0; j < kPoolPer; ++j) {
+    const bool eq = (m[j] >> lane) & 1u;
+    const bool keep = cnt > uint32_t(k) ? (c[j] > ostar || (eq && off[j] + __popc(m[j] & lt) < need_eq)) : c[j] != 0u;
+    m[j] = __ballot_sync(kFull, keep);
+  }
+  const uint32_t got = ordered_offsets<kSelThreads, kPoolPer>(m, off);
+  int32_t* out = idx_out + size_t(b) * k;
+#pragma unroll
+  for (int j = 0; j < kPoolPer; ++j) {
+    if ((m[j] >> lane) & 1u) {
+      const uint32_t at = off[j] + __popc(m[j] & lt);
+      if (at < kk) out[at] = pent[threadIdx.x + j * kSelThreads];
+    }
+  }
+  for (int i = int(kk) + threadIdx.x; i < k; i += kSelThreads) out[i] = -1;
+  if (threadIdx.x == 0) {
+    if (count_out) count_out[b] = int32_t(kk);
+    if (got != kk) set_status(status, DSV4KV_DEV_INCONSISTENT);
+  }
+}
+
+dsv4kv_status index_topk_pool_launch(const uint16_t* qidx, const dsv4kv_cache& keys, int batch, int64_t n,
+                                     const int32_t* pool, int pool_cap, int k, int32_t* idx_out, int32_t* count_out,
+                                     void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (ws_bytes < 16) return set_error(DSV4KV_ERR_WORKSPACE, "index_topk_pool: workspace too small");
+  if (pool_cap > kPoolMax)
+    return set_error(DSV4KV_ERR_UNSUPPORTED, "index_topk_pool: pool of %d entries > %d", pool_cap, kPoolMax);
+  uint32_t* status = static_cast<uint32_t*>(ws);
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(index_pool_select<DSV4KV_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(kPoolDyn)) != cudaSuccess ||
+        cudaFuncSetAttribute(index_pool_select<DSV4KV_FP4_E2M1_G16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(kPoolDyn)) != cudaSuccess)
+      return check_launch("index_topk_pool: cudaFuncSetAttribute");
+    attr = true;
+  }
+  if (keys.fmt == DSV4KV_BF16)
+    launch_pdl(index_pool_select<DSV4KV_BF16>, dim3(unsigned(batch)), dim3(kSelThreads), kPoolDyn, stream, qidx,
+               keys.codes, static_cast<const uint8_t*>(keys.scales), keys.rows, n, pool, pool_cap, k, idx_out,
+               count_out, status);
+  else
+    launch_pdl(index_pool_select<DSV4KV_FP4_E2M1_G16>, dim3(unsigned(batch)), dim3(kSelThreads), kPoolDyn, stream,
+               qidx, keys.codes, static_cast<const uint8_t*>(keys.scales), keys.rows, n, pool, pool_cap, k, idx_out,
+               count_out, status);
+  return check_launch("index_pool_select");
+}
+
 // ------------------------------------------------------------------ host side
 struct IndexWs {
   uint32_t* status;

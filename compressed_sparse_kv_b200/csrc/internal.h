@@ -67,6 +67,9 @@ dsv4kv_status index_score_launch(const uint16_t* qidx, const dsv4kv_cache& keys,
                                  void* ws, size_t ws_bytes, cudaStream_t stream);
 dsv4kv_status index_select_launch(int batch, int64_t n, int k, int32_t* idx_out, int32_t* count_out, void* ws,
                                   size_t ws_bytes, cudaStream_t stream);
+dsv4kv_status index_topk_pool_launch(const uint16_t* qidx, const dsv4kv_cache& keys, int batch, int64_t n,
+                                     const int32_t* pool, int pool_cap, int k, int32_t* idx_out, int32_t* count_out,
+                                     void* ws, size_t ws_bytes, cudaStream_t stream);
 dsv4kv_status index_topk_launch(const uint16_t* qidx, const dsv4kv_cache& keys, int batch, int64_t n, int k,
                                 int32_t* idx_out, int32_t* count_out, void* ws, size_t ws_bytes,
                                 cudaStream_t stream);

@@ -49,6 +49,7 @@ typedef enum {
 #define DSV4KV_DEV_BAD_INDEX 0x1u  /* a selected index was outside [0, n): row skipped */
 #define DSV4KV_DEV_TIMEOUT 0x2u    /* a bounded wait gave up: outputs are invalid       */
 #define DSV4KV_DEV_INCONSISTENT 0x4u /* selection counts disagreed: outputs are invalid */
+#define DSV4KV_DEV_BAD_POOL 0x8u     /* a candidate pool was not ascending: ties may differ */
 
 /* Cache row formats.
  *  DSV4KV_BF16:          codes = bf16 [B][rows][dim]; scales = NULL.
@@ -167,6 +168,33 @@ dsv4kv_status dsv4kv_index_score(const void* qidx, const dsv4kv_cache* keys, int
 
 dsv4kv_status dsv4kv_index_select(int32_t batch, int64_t n, int32_t k, int32_t* idx_out,
                                   int32_t* count_out, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Re-index inside a candidate pool.  [P3] "Three mechanisms instead of one
+ * trick", CSA2: layers in Reindex mode keep their indexing inside the
+ * candidate pool built by the first layer in Full mode, and the layers share
+ * the indexer keys.  For sequence b, with pool[b][0..pool_cap) holding entry
+ * indices in ascending order (negative = no entry, e.g. the -1 padding of a
+ * dsv4kv_index_topk output that built the pool):
+ *   idx_out[b] = the first min(k, m) pool entries under (score descending,
+ *   entry index ascending), written in ascending entry order, padded with -1
+ *   (m = number of pool entries); count_out[b] = min(k, m).
+ * score as in dsv4kv_index_topk (this layer's qidx against the shared keys,
+ * bf16 or fp4 keys).  The pool size is the caller's choice (the pages give
+ * none); pool_cap <= 8192.  A pool entry >= n sets DSV4KV_DEV_BAD_INDEX and is
+ * skipped; a pool that is not ascending sets DSV4KV_DEV_BAD_POOL (the set is
+ * still the top-k, but ties then follow pool order).  One CTA per sequence;
+ * the workspace holds only the status word
+ * (dsv4kv_index_topk_pool_workspace_bytes).
+ *   qidx  : bf16 [batch][128];  keys: as for dsv4kv_index_topk
+ *   pool  : int32 [batch][pool_cap];  idx_out: int32 [batch][k];
+ *   count_out: int32 [batch] or NULL
+ * ------------------------------------------------------------------------ */
+size_t dsv4kv_index_topk_pool_workspace_bytes(int32_t batch, int32_t pool_cap, int32_t k);
+
+dsv4kv_status dsv4kv_index_topk_pool(const void* qidx, const dsv4kv_cache* keys, int32_t batch, int64_t n,
+                                     const int32_t* pool, int32_t pool_cap, int32_t k, int32_t* idx_out,
+                                     int32_t* count_out, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * dsv4kv_index_topk without a caller workspace.  The pages have no
