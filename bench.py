@@ -41,6 +41,9 @@ WORKLOADS = {
     "q_c128a_fp4": ("c128a", 64, 262144, 64, 2, 0),
     "q_c4a_fp8rope": ("c4a", 64, 262144, 64, 3, 2),
     "q_c128a_fp8rope": ("c128a", 64, 262144, 64, 3, 0),
+    # a CSA2 Reindex layer: top-512 re-indexed inside the 2048-entry pool a Full
+    # layer built (the pool size is a reading; the pages give none)
+    "c4a_b32_reindex": ("c4a", 32, 131072, 64, 0, 0, 2048),
 }
 FMT_NAME = {0: "bf16", 1: "fp8", 2: "fp4", 3: "fp8+bf16rope"}
 L2_BYTES = 126 * 2 ** 20
@@ -118,28 +121,30 @@ ROW_BYTES = {0: 1024, 1: 516, 2: 288, 3: 580}  # one 512-channel cache row: bf16
 KEY_BYTES = {0: 256, 2: 72}               # one 128-channel indexer key: bf16, fp4 + scales
 
 
-def step_bytes(kind, batch, t, main_fmt, index_fmt, k=512, window=128):
+def step_bytes(kind, batch, t, main_fmt, index_fmt, k=512, window=128, pool=0):
     """Algorithmic bytes one step reads from one cache replica: indexer keys
-    (c4a) + the attended rows.  Queries and outputs are excluded."""
+    (c4a; only the pool's keys for a Reindex layer) + the attended rows.
+    Queries and outputs are excluded."""
     n = (t - window) // (4 if kind == "c4a" else 128)
     rows = (k + window) if kind == "c4a" else (n + window)
     b = batch * rows * ROW_BYTES[main_fmt]
     if kind == "c4a":
-        b += batch * n * KEY_BYTES[index_fmt]
+        b += batch * (pool if pool else n) * KEY_BYTES[index_fmt]
     return b
 
 
-def replicas_for(kind, batch, t, main_fmt, index_fmt, at_least):
+def replicas_for(kind, batch, t, main_fmt, index_fmt, at_least, pool=0):
     """Cache replicas the timed steps cycle through: together they hold at
     least four times the L2, so every step streams its rows from DRAM."""
-    per = step_bytes(kind, batch, t, main_fmt, index_fmt)
+    per = step_bytes(kind, batch, t, main_fmt, index_fmt, pool=pool)
     return max(at_least, -(-4 * L2_BYTES // per))
 
 
 class Layer:
     """One layer's resident caches (R replicas) and per-step buffers on the GPU."""
 
-    def __init__(self, kind, batch, t, heads, seed, replicas, main_fmt=0, index_fmt=0, layer_id=0, shared=None):
+    def __init__(self, kind, batch, t, heads, seed, replicas, main_fmt=0, index_fmt=0, layer_id=0, shared=None,
+                 pool=0):
         import torch
         import compressed_sparse_kv_b200 as K
         import datagen.gpu as G
@@ -148,6 +153,7 @@ class Layer:
         self.kind, self.batch, self.t, self.heads = kind, batch, t, heads
         self.main_fmt, self.index_fmt = main_fmt, index_fmt
         self.window, self.k = 128, 512
+        self.pool = pool  # > 0: a Reindex layer over a pool of this many entries
         stride = 4 if kind == "c4a" else 128
         self.n = (t - self.window) // stride
         dev = "cuda"
@@ -174,6 +180,14 @@ class Layer:
                     G.fp4_index_keys_(codes, scales, keys["kidx_fp4"])
                     rep["kidx"] = K.Cache(2, codes, scales, 128)
             self.reps.append(rep)
+        if pool:
+            # the pool: the top-`pool` entries of each replica's keys under another
+            # layer's query (the Full layer of the group), built once
+            qf = G.int_bf16_(torch.empty(batch, 128, dtype=torch.bfloat16, device=dev),
+                             WL.keys_for(seed, 5000 + layer_id)["qidx"])
+            for rep in self.reps:
+                rep["pool"], _ = K.index_topk(qf, rep["kidx"], self.n, pool)
+            self.ws_pool = K.new_workspace(16)
         keys = WL.keys_for(seed, layer_id)
         self.q = G.normal_bf16_(torch.empty(batch, heads, 512, dtype=torch.bfloat16, device=dev), keys["q"])
         # the inputs are generated on the current stream; the timed work runs on its own stream
@@ -197,27 +211,39 @@ class Layer:
 
     # algorithmic bytes of one step: indexer keys + rows read (queries/outputs excluded)
     def alg_bytes(self):
-        return step_bytes(self.kind, self.batch, self.t, self.main_fmt, self.index_fmt, self.k, self.window)
+        return step_bytes(self.kind, self.batch, self.t, self.main_fmt, self.index_fmt, self.k, self.window, self.pool)
 
     def index_bytes(self):
-        return self.batch * self.n * KEY_BYTES[self.index_fmt] + self.batch * 256
+        return self.batch * (self.pool or self.n) * KEY_BYTES[self.index_fmt] + self.batch * 256
 
     def flops(self):
         rows = (self.k + self.window) if self.kind == "c4a" else (self.n + self.window)
         return self.batch * rows * 4 * self.heads * 512
 
     def launches_per_step(self):
-        return 4 if self.kind == "c4a" else 2
+        if self.kind != "c4a":
+            return 2
+        return 3 if self.pool else 4
 
     def index(self, r):
+        if self.pool:
+            self.index_score(r)
+            return
         self.K.index_topk(self.qidx, self.reps[r]["kidx"], self.n, self.k, idx_out=self.idx, count_out=self.cnt,
                           ws=self.ws_idx)
 
-    # the same call in its two steps (dsv4kv_index_score; dsv4kv_index_select)
+    # the same call in its two steps (dsv4kv_index_score; dsv4kv_index_select);
+    # a Reindex layer's one call (dsv4kv_index_topk_pool) stands in the first
     def index_score(self, r):
+        if self.pool:
+            self.K.index_topk_pool(self.qidx, self.reps[r]["kidx"], self.n, self.reps[r]["pool"], self.k,
+                                   idx_out=self.idx, count_out=self.cnt, ws=self.ws_pool)
+            return
         self.K.index_score(self.qidx, self.reps[r]["kidx"], self.n, self.k, self.ws_idx)
 
     def index_select(self):
+        if self.pool:
+            return
         self.K.index_select(self.batch, self.n, self.k, self.idx, self.cnt, self.ws_idx)
 
     def decode(self, r, q=None, out=None):
@@ -476,7 +502,10 @@ def time_e2e(layer, steps):
         with torch.cuda.stream(s_comp):
             wait(s_comp, ev_in[j])
             wait(s_comp, ev_out[j])              # step i-NB's output has left this buffer
-            if layer.kind == "c4a":
+            if layer.kind == "c4a" and layer.pool:
+                layer.K.index_topk_pool(qi_dev[j], layer.reps[i % R]["kidx"], layer.n, layer.reps[i % R]["pool"],
+                                        layer.k, idx_out=layer.idx, count_out=layer.cnt, ws=layer.ws_pool)
+            elif layer.kind == "c4a":
                 layer.K.index_topk(qi_dev[j], layer.reps[i % R]["kidx"], layer.n, layer.k, idx_out=layer.idx,
                                    count_out=layer.cnt, ws=layer.ws_idx)
             layer.decode(i % R, q=q_dev[j], out=out_dev[j])
@@ -631,7 +660,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="c4a_b32")
     ap.add_argument("--secondary", default="c128a_b8,c128a_b32,q_c4a_fp8,q_c4a_fp4,q_c128a_fp8,q_c128a_fp4,"
-                                           "q_c4a_fp8rope,q_c128a_fp8rope",
+                                           "q_c4a_fp8rope,q_c128a_fp8rope,c4a_b32_reindex",
                     help="extra per-layer-type workloads (comma list, 'none' = none)")
     ap.add_argument("--no-stack", action="store_true", help="skip the 61-layer stack step")
     ap.add_argument("--no-bulk", action="store_true", help="skip compressor/quantiser throughput")
@@ -642,13 +671,16 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
     d = dist_init()
-    kind, batch, t, heads, mfmt, ifmt = WORKLOADS[args.workload]
+    kind, batch, t, heads, mfmt, ifmt = WORKLOADS[args.workload][:6]
+    pool = WORKLOADS[args.workload][6] if len(WORKLOADS[args.workload]) > 6 else 0
 
-    def wl_desc(kind, batch, t, heads, mfmt, ifmt):
+    def wl_desc(kind, batch, t, heads, mfmt, ifmt, pool=0):
         idx = f", {FMT_NAME[ifmt]} indexer" if kind == "c4a" else ""
+        if pool:
+            idx += f", Reindex layer (top-512 inside a {pool}-entry pool)"
         return f"{kind} layer decode B={batch} t={t} H={heads} k=512 W=128 {FMT_NAME[mfmt]} main cache{idx}"
 
-    wl_name = wl_desc(kind, batch, t, heads, mfmt, ifmt)
+    wl_name = wl_desc(kind, batch, t, heads, mfmt, ifmt, pool)
 
     if args.impl == "reference":
         if d["rank"] != 0:
@@ -672,8 +704,8 @@ def main():
     torch.cuda.set_device(d["local"])
     hbm_peak, tf_peak, peak_src = measured_peaks()
     seed = 1234 + d["rank"]
-    reps = replicas_for(kind, batch, t, mfmt, ifmt, args.replicas)
-    layer = Layer(kind, batch, t, heads, seed, reps, mfmt, ifmt)
+    reps = replicas_for(kind, batch, t, mfmt, ifmt, args.replicas, pool)
+    layer = Layer(kind, batch, t, heads, seed, reps, mfmt, ifmt, pool=pool)
     res = time_layer(layer, args.steps, args.warmup, dist_max, d["local"], sample_clocks=(d["rank"] == 0))
     ms = res["total_ms"] / args.steps
     steps_per_s = d["world"] * 1e3 / ms            # whole job: every rank ran `steps` steps
@@ -687,7 +719,7 @@ def main():
     # launch per dsv4kv_index_score call), the dense decode call for c128a
     if kind == "c4a":
         dom_bytes, dom_ms = layer.index_bytes(), res["score_ms"]
-        dom_name = "index_score_bf16" if ifmt == 0 else "index_score_fp4"
+        dom_name = "index_pool_select" if pool else ("index_score_bf16" if ifmt == 0 else "index_score_fp4")
     else:
         dom_bytes, dom_ms, dom_name = alg, res["decode_ms"], "dsv4kv_dense_decode (decode_kernel + decode_combine)"
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
@@ -706,8 +738,9 @@ def main():
                        "median_of_5_ms_per_step": round(dist_max(res["median5_ms"]) / args.steps, 5)}}
     for name in [s for s in args.secondary.split(",") if s and s not in ("none", args.workload)]:
         spec = WORKLOADS[name]
-        r2n = replicas_for(spec[0], spec[1], spec[2], spec[4], spec[5], 2)
-        L2 = Layer(*spec[:4], seed + 99, r2n, spec[4], spec[5])
+        pool2 = spec[6] if len(spec) > 6 else 0
+        r2n = replicas_for(spec[0], spec[1], spec[2], spec[4], spec[5], 2, pool2)
+        L2 = Layer(*spec[:4], seed + 99, r2n, spec[4], spec[5], pool=pool2)
         r2 = time_layer(L2, args.steps, args.warmup, dist_max, d["local"], sample_clocks=False)
         ms2 = r2["total_ms"] / args.steps
         a2 = L2.alg_bytes()

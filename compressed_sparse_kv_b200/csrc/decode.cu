@@ -675,61 +675,62 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           cp_async_wait_all();
         } else if constexpr (FMT == DSV4KV_FP8_E4M3_ROW_ROPE_BF16) {
-          // rows of kDim + 64 bytes: lanes < 28 own 16 fp8 channels (16 code
-          // bytes), lanes 28..31 16 of the 64 bf16 rotary channels (32 bytes),
-          // stored as f16 of value / scale so that the row scale folds into
-          // the softmax weights exactly as for plain fp8 rows; two rounds of
-          // 8 rows keep the loads of a round in flight together
+          // rows of kDim + 64 bytes: 28 chunks of 16 fp8 channels (16 bytes),
+          // then 8 chunks of 8 bf16 rotary channels.  The warp's 16 rows hold
+          // 448 fp8 chunks (14 per lane) and 128 rotary chunks (4 per lane);
+          // all 18 loads of a lane are issued before any is converted, and
+          // each conversion loop has one chunk kind for the whole warp.  The
+          // rotary channels are stored as f16 of value / scale so that the
+          // row scale folds into the softmax weights exactly as for fp8 rows.
+          constexpr int kBodyChunks = (kDim - 64) / 16, kRopeChunks = 64 / 8;
+          constexpr int kPerBody = 16 * kBodyChunks / 32, kPerRope = 16 * kRopeChunks / 32;
           const uint8_t* codes = mine.from_win ? p.win_codes : p.comp_codes;
           const float* scales = static_cast<const float*>(mine.from_win ? p.win_scales : p.comp_scales);
           const float my_scale = (lane < 16 && mine.valid) ? scales[mine.row] : 0.f;
           if (lane < 16) ctl->row_scale[stage][16 * lw + lane] = my_scale;
-          const bool rope_lane = lane >= 28;
-          const int chunk = lane >> 2, u0 = (lane & 3) * 2;  // lane owns channels [16*lane, 16*lane+16)
-          uint8_t* ctile = tile + chunk * kChunkBytes;
+          uint4 rawb[kPerBody], rawr[kPerRope];
 #pragma unroll
-          for (int hb = 0; hb < 2; ++hb) {
-            uint4 ra[8], rb[8];
+          for (int i = 0; i < kPerBody; ++i) {
+            const int g = lane + 32 * i, jr = g / kBodyChunks, cr = g % kBodyChunks;
+            const int64_t row = __shfl_sync(kFull, mine.row, jr);
+            const bool valid = __shfl_sync(kFull, mine.valid, jr);
+            rawb[i] = valid ? ld_stream_v4(codes + size_t(row) * (kDim + 64) + 16 * cr) : make_uint4(0, 0, 0, 0);
+          }
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-              const int j = 8 * hb + jj;
-              const int64_t row = __shfl_sync(kFull, mine.row, j);
-              const bool valid = __shfl_sync(kFull, mine.valid, j);
-              const uint8_t* rp = codes + size_t(row) * (kDim + 64);
-              if (!valid) {
-                ra[jj] = rb[jj] = make_uint4(0, 0, 0, 0);
-              } else if (rope_lane) {
-                const uint8_t* src = rp + (kDim - 64) + 32 * (lane - 28);
-                ra[jj] = ld_stream_v4(src);
-                rb[jj] = ld_stream_v4(src + 16);
-              } else {
-                ra[jj] = ld_stream_v4(rp + 16 * lane);
-                rb[jj] = make_uint4(0, 0, 0, 0);
-              }
+          for (int i = 0; i < kPerRope; ++i) {
+            const int g = lane + 32 * i, jr = g / kRopeChunks, cr = g % kRopeChunks;
+            const int64_t row = __shfl_sync(kFull, mine.row, jr);
+            const bool valid = __shfl_sync(kFull, mine.valid, jr);
+            rawr[i] = valid ? ld_stream_v4(codes + size_t(row) * (kDim + 64) + (kDim - 64) + 16 * cr)
+                            : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int i = 0; i < kPerBody; ++i) {
+            const int g = lane + 32 * i, jr = g / kBodyChunks, cr = g % kBodyChunks;
+            const int r = 16 * lw + jr, ch = 16 * cr, u = (ch & 63) >> 3;
+            const uint32_t w[4] = {rawb[i].x, rawb[i].y, rawb[i].z, rawb[i].w};
+            uint32_t hv[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              hv[2 * e] = e4m3x2_to_f16x2(w[e] & 0xffffu);
+              hv[2 * e + 1] = e4m3x2_to_f16x2(w[e] >> 16);
             }
+            uint8_t* line = tile + (ch >> 6) * kChunkBytes + r * 128;
+            *reinterpret_cast<uint4*>(line + ((u ^ (r & 7)) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+            *reinterpret_cast<uint4*>(line + (((u + 1) ^ (r & 7)) << 4)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+          }
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-              const int j = 8 * hb + jj;
-              const int r = 16 * lw + j;
-              const float s = __shfl_sync(kFull, my_scale, j);
-              uint32_t hv[8];
-              if (rope_lane) {
-                const float inv = s > 0.f ? 1.f / s : 0.f;
-                const uint32_t w[8] = {ra[jj].x, ra[jj].y, ra[jj].z, ra[jj].w, rb[jj].x, rb[jj].y, rb[jj].z, rb[jj].w};
+          for (int i = 0; i < kPerRope; ++i) {
+            const int g = lane + 32 * i, jr = g / kRopeChunks, cr = g % kRopeChunks;
+            const int r = 16 * lw + jr, ch = (kDim - 64) + 8 * cr, u = (ch & 63) >> 3;
+            const float sr = __shfl_sync(kFull, my_scale, jr);
+            const float inv = sr > 0.f ? __frcp_rn(sr) : 0.f;
+            const uint32_t w[4] = {rawr[i].x, rawr[i].y, rawr[i].z, rawr[i].w};
+            uint32_t hv[4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) hv[e] = f32x2_to_f16x2_sat(bf16lo(w[e]) * inv, bf16hi(w[e]) * inv);
-              } else {
-                const uint32_t w[4] = {ra[jj].x, ra[jj].y, ra[jj].z, ra[jj].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  hv[2 * e] = e4m3x2_to_f16x2(w[e] & 0xffffu);
-                  hv[2 * e + 1] = e4m3x2_to_f16x2(w[e] >> 16);
-                }
-              }
-              uint8_t* line = ctile + r * 128;
-              *reinterpret_cast<uint4*>(line + ((u0 ^ (r & 7)) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-              *reinterpret_cast<uint4*>(line + (((u0 + 1) ^ (r & 7)) << 4)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
-            }
+            for (int e = 0; e < 4; ++e) hv[e] = f32x2_to_f16x2_sat(bf16lo(w[e]) * inv, bf16hi(w[e]) * inv);
+            uint8_t* line = tile + (ch >> 6) * kChunkBytes + r * 128;
+            *reinterpret_cast<uint4*>(line + ((u ^ (r & 7)) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
           }
         } else {
           const uint8_t* codes = mine.from_win ? p.win_codes : p.comp_codes;
