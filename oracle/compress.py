@@ -47,3 +47,22 @@ def compress(s_raw, w, stride: int, window: int, pos0: int = 0,
         live = p >= 0
         out[live] += w[j][None, :] * s_raw[p[live]]
     return rope(out, pos0 + stride * i, rope_dim, base)
+
+
+def append_state(s_hist, w, stride: int, window: int, rope_dim: int = 64, base: float = 10000.0):
+    """Incremental maintenance of one layer's caches for a decode step (the
+    steps either side of the path, [P1] "compressor-state blocks"): after the
+    state of position t = len(s_hist) - 1 is appended, the caches hold
+      * the window: rope(S[p], p) for p in [max(0, t + 1 - W), t + 1);
+      * the compressed entries 0 .. n_entries(t + 1, W, s) - 1, each exactly
+        the entry `compress` makes from the whole history.
+    Reading: appending token by token must reach the same caches as
+    compressing the whole history at once; an entry is emitted the step its
+    stride block leaves the window.  s_hist [t+1][D] float64 (unrotated),
+    w [K][D].  Returns (window positions, window rows [.][D], entries [N][D])."""
+    s_hist = np.asarray(s_hist, dtype=np.float64)
+    t1 = s_hist.shape[0]
+    pos = np.arange(max(0, t1 - window), t1)
+    win = np.stack([rope(s_hist[p], int(p), rope_dim, base) for p in pos]) if len(pos) else np.zeros((0, s_hist.shape[1]))
+    ent = compress(s_hist, w, stride, window, 0, rope_dim, base)
+    return pos, win, ent

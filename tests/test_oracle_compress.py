@@ -119,3 +119,35 @@ def test_per_channel_weights_are_not_transposed():
     out = C.compress(raw, w, 4, 128, rope_dim=64)
     # channel 3 of entry 1 = sum_j w[j,3] * raw[j,3] (taps 0..7), plain channel so no rotation
     assert np.isclose(out[1, 3], sum(w[j, 3] * raw[j, 3] for j in range(8)), atol=1e-13)
+
+
+# ------------------------------------------------ incremental maintenance
+@pytest.mark.parametrize("stride,k_taps,window", [(4, 8, 128), (128, 128, 128), (4, 8, 0), (8, 16, 20)])
+def test_append_emits_each_entry_when_its_block_leaves_the_window(stride, k_taps, window):
+    """Entry count grows by one exactly when (t+1-W) reaches a multiple of the
+    stride, and the new entry's taps all lie in the last W + K positions (the
+    raw ring the incremental kernel keeps)."""
+    prev = 0
+    for t in range(0, 6 * stride + window + 3):
+        n1 = C.n_entries(t + 1, window, stride)
+        grew = n1 - prev
+        assert grew in (0, 1)
+        assert grew == (1 if (t + 1 - window) >= stride and (t + 1 - window) % stride == 0 else 0)
+        if grew:
+            taps = C.tap_positions(n1 - 1, stride, k_taps)
+            live = taps[taps >= 0]
+            assert live.min() >= t + 1 - window - k_taps and live.max() <= t - window
+        prev = n1
+
+
+def test_append_state_is_the_whole_history_compressed():
+    rng = np.random.default_rng(12)
+    s = rng.standard_normal((300, 64))
+    w = rng.random((8, 64))
+    pos, win, ent = C.append_state(s, w, 4, 32, rope_dim=16)
+    assert pos.tolist() == list(range(268, 300))
+    assert np.allclose(win[5], R.rope(s[273], 273, 16), rtol=0, atol=1e-12)
+    assert ent.shape == (67, 64)                      # floor((300 - 32) / 4)
+    # entry 10 mixes positions 36..43 (taps 4*10 + 4 - 8 + j), rotated at 40
+    raw = sum(w[j] * s[36 + j] for j in range(8))
+    assert np.allclose(ent[10], R.rope(raw, 40, 16), rtol=0, atol=1e-12)
