@@ -50,6 +50,9 @@ _SIGS = {
                                      _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "dsv4kv_index_score": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.c_int32, _c.c_int64, _c.c_int32,
                                       _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "dsv4kv_append": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_int64, _c.c_int32, _c.c_int32,
+                                 _c.c_int32, _c.c_int32, _c.c_int32, _c.c_double, _c.c_void_p, _c.c_void_p,
+                                 _c.c_void_p, _c.c_int64, _c.c_void_p]),
     "dsv4kv_index_topk_pool_workspace_bytes": (_c.c_size_t, [_c.c_int32, _c.c_int32, _c.c_int32]),
     "dsv4kv_index_topk_pool": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.c_int32, _c.c_int64, _c.c_void_p,
                                           _c.c_int32, _c.c_int32, _c.c_void_p, _c.c_void_p, _c.c_void_p,
@@ -145,6 +148,17 @@ def compress(s_raw: torch.Tensor, w: torch.Tensor, stride: int, window: int, pos
     _check(lib().dsv4kv_compress(_ptr(s_raw), _ptr(w), b, t, d, int(w.shape[0]), stride, window, pos0, rope_dim,
                                  rope_base, int(out_fp32), _ptr(out), _stream(stream)), "dsv4kv_compress")
     return out
+
+
+def append(s_new: torch.Tensor, w: torch.Tensor, t: int, stride: int, window: int, raw_ring: torch.Tensor,
+           win_ring: Optional[torch.Tensor], comp: torch.Tensor, rope_dim: int = 64, rope_base: float = 10000.0,
+           stream=None) -> None:
+    """Append the states s_new bf16 [B][D] of position t: raw ring [B][W+K][D], window ring [B][W][D] and,
+    when an entry's block leaves the window, that entry into comp [B][rows][D] (all bf16)."""
+    b, d = int(s_new.shape[0]), int(s_new.shape[1])
+    _check(lib().dsv4kv_append(_ptr(s_new), _ptr(w), b, t, d, int(w.shape[0]), stride, window, rope_dim, rope_base,
+                               _ptr(raw_ring), _ptr(win_ring) if win_ring is not None else None, _ptr(comp),
+                               int(comp.shape[1]), _stream(stream)), "dsv4kv_append")
 
 
 def quantize(x: torch.Tensor, fmt: int, codes: Optional[torch.Tensor] = None,

@@ -133,6 +133,28 @@ DSV4KV_API dsv4kv_status dsv4kv_compress(const void* s_raw, const float* w, int3
                          static_cast<cudaStream_t>(stream));
 }
 
+DSV4KV_API dsv4kv_status dsv4kv_append(const void* s_new, const float* w, int32_t batch, int64_t t, int32_t dim,
+                                       int32_t k_taps, int32_t stride, int32_t window, int32_t rope_dim,
+                                       double rope_base, void* raw_ring, void* win_ring, void* comp,
+                                       int64_t comp_rows, void* stream) {
+  g_err[0] = 0;
+  if (batch < 0 || t < 0 || k_taps < 1 || stride < 1 || window < 0 || comp_rows < 0)
+    return set_error(DSV4KV_ERR_INVALID_ARG, "append: bad sizes");
+  if (rope_dim < 0 || rope_dim > dim || (rope_dim & 1))
+    return set_error(DSV4KV_ERR_INVALID_ARG, "append: rope_dim must be even and <= dim");
+  if (!(rope_base > 0.0)) return set_error(DSV4KV_ERR_INVALID_ARG, "append: rope_base must be > 0");
+  if (batch == 0) return DSV4KV_OK;
+  if (!s_new || !w || !raw_ring || !aligned16(s_new) || !aligned16(w) || !aligned16(raw_ring))
+    return set_error(DSV4KV_ERR_INVALID_ARG, "append: null or misaligned pointer");
+  if (window > 0 && (!win_ring || !aligned16(win_ring)))
+    return set_error(DSV4KV_ERR_INVALID_ARG, "append: window ring null or misaligned");
+  const int64_t emit = append_emit_entry(t, window, stride);
+  if (emit >= 0 && (!comp || !aligned16(comp) || emit >= comp_rows))
+    return set_error(DSV4KV_ERR_INVALID_ARG, "append: entry %lld does not fit the compressed cache", (long long)emit);
+  return append_launch(s_new, w, batch, t, dim, k_taps, stride, window, rope_dim, rope_base, raw_ring, win_ring, comp,
+                       comp_rows, static_cast<cudaStream_t>(stream));
+}
+
 DSV4KV_API dsv4kv_status dsv4kv_quantize(const void* in, int32_t in_fp32, int64_t rows, int32_t dim, int32_t fmt,
                                          void* codes, void* scales, void* stream) {
   g_err[0] = 0;

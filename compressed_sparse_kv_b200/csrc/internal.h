@@ -65,6 +65,10 @@ size_t index_topk_ws_bytes(int batch, int64_t n, int k);
 size_t index_topk_zero_prefix_bytes(int batch);
 dsv4kv_status index_score_launch(const uint16_t* qidx, const dsv4kv_cache& keys, int batch, int64_t n, int k,
                                  void* ws, size_t ws_bytes, cudaStream_t stream);
+int64_t append_emit_entry(int64_t t, int window, int stride);
+dsv4kv_status append_launch(const void* s_new, const float* w, int batch, int64_t t, int dim, int k_taps, int stride,
+                            int window, int rope_dim, double rope_base, void* raw_ring, void* win_ring, void* comp,
+                            int64_t comp_rows, cudaStream_t stream);
 dsv4kv_status index_select_launch(int batch, int64_t n, int k, int32_t* idx_out, int32_t* count_out, void* ws,
                                   size_t ws_bytes, cudaStream_t stream);
 dsv4kv_status index_topk_pool_launch(const uint16_t* qidx, const dsv4kv_cache& keys, int batch, int64_t n,

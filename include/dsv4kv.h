@@ -111,6 +111,35 @@ dsv4kv_status dsv4kv_compress(const void* s_raw, const float* w, int32_t batch, 
                               int32_t out_fp32, void* out, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Incremental cache maintenance for one decode step ([P1] "compressor-state
+ * blocks": the caches are updated as tokens arrive).  Appends the unrotated
+ * state of position t of every sequence and keeps, per layer:
+ *   raw_ring : bf16 [batch][window + k_taps][dim]; row p % (window + k_taps)
+ *              holds S[p] (unrotated) for the last window + k_taps positions;
+ *   win_ring : bf16 [batch][window][dim]; row p % window holds
+ *              rope(S[p], p) (rotary pairs as in dsv4kv_compress) for the
+ *              last `window` positions -- the window cache the decode calls
+ *              read (row order does not matter to them; before t + 1 >=
+ *              window only rows 0..t are written);
+ *   comp     : bf16 [batch][comp_rows][dim]; entry i, the dsv4kv_compress
+ *              entry of the history (taps s i + s - K + j, rotated at s i), is
+ *              written the step its stride block leaves the window: when
+ *              dsv4kv_compress_entries(t + 1, window, stride) grows, entry
+ *              dsv4kv_compress_entries(t + 1, window, stride) - 1.
+ * Appending positions 0, 1, ..., T-1 one call at a time leaves comp equal to
+ * dsv4kv_compress over the whole history (up to fp32 summation order) and
+ * the window ring equal to the rotated last `window` states.
+ *   s_new : bf16 [batch][dim];  w : float [k_taps][dim]
+ * Requirements: dim in {256, 512, 1024}; rope_dim even, <= dim; t >= 0;
+ * comp_rows > the entry written (else DSV4KV_ERR_INVALID_ARG); win_ring may
+ * be NULL only when window == 0.  Quantised caches are made from these rows
+ * with dsv4kv_quantize.
+ * ------------------------------------------------------------------------ */
+dsv4kv_status dsv4kv_append(const void* s_new, const float* w, int32_t batch, int64_t t, int32_t dim,
+                            int32_t k_taps, int32_t stride, int32_t window, int32_t rope_dim, double rope_base,
+                            void* raw_ring, void* win_ring, void* comp, int64_t comp_rows, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Quantiser.  [P1] quantisation paragraphs (fp8 attention cache, fp4 indexer
  * cache); [P3] fp4 E2M1 main cache with one E4M3 scale per 16 channels.
  *   DSV4KV_FP8_E4M3_ROW: scale = fp32(amax / 448) (1 if amax == 0),
