@@ -322,7 +322,8 @@ def time_stack(steps, warmup, seed, dist_max):
 
 
 def time_bulk(seed):
-    """Bulk throughput of the c4a / c128a compressors and the fp8 / fp4 quantiser."""
+    """Bulk throughput of the c4a / c128a compressors and the fp8 / fp4 quantiser;
+    per-token time of the incremental cache maintenance."""
     import torch
     import compressed_sparse_kv_b200 as K
     import datagen as D
@@ -357,6 +358,35 @@ def time_bulk(seed):
         byts = x.shape[0] * (1024 + rb)
         out[f"quantize_{name}"] = {"workload": f"{x.shape[0]} rows x 512 bf16", "us": round(ms * 1e3, 1),
                                    "gbs": round(byts / (ms * 1e-3) / 1e9, 1)}
+    # incremental maintenance (dsv4kv_append) per decoded token at t = 131072:
+    # B = 32 for c4a (an entry every 4 tokens), B = 8 for c128a (every 128);
+    # the mean over a run of consecutive tokens, one CUDA graph
+    for kind, st, k, bsz in (("c4a", 4, 8, 32), ("c128a", 128, 128, 8)):
+        w = torch.from_numpy(D.compress_weights(seed, 0, k, 512)).cuda()
+        ring = torch.zeros(bsz, 128 + k, 512, dtype=torch.bfloat16, device="cuda")
+        win = torch.zeros(bsz, 128, 512, dtype=torch.bfloat16, device="cuda")
+        comp = torch.zeros(bsz, K.compress_entries(131072 + 256, 128, st) + 1, 512, dtype=torch.bfloat16, device="cuda")
+        x = raw[:, 0].repeat(bsz // 8, 1).contiguous()  # [bsz][512] states
+        t0, steps = 131072, 256
+        stream = torch.cuda.Stream()
+        with torch.cuda.stream(stream):
+            for i in range(steps):
+                K.append(x, w, t0 + i, st, 128, ring, win, comp)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(steps):
+                K.append(x, w, t0 + i, st, 128, ring, win, comp)
+        with torch.cuda.stream(stream):
+            g.replay()
+            s.record(stream)
+            g.replay()
+            e.record(stream)
+        e.synchronize()
+        emits = sum(1 for i in range(steps) if (t0 + i + 1 - 128) % st == 0)
+        out[f"append_{kind}"] = {"workload": f"B={bsz}, {steps} consecutive tokens from t={t0} ({emits} entries emitted)",
+                                 "us_per_token": round(s.elapsed_time(e) * 1e3 / steps, 2)}
+        del g
     del raw
     torch.cuda.empty_cache()
     return out
