@@ -93,3 +93,31 @@ def test_bad_arguments_return_status_codes():
                                   64, 1e4, 0, 16, 16, 1 << 30, z) == 1                        # idx null
     assert L.dsv4kv_sparse_decode(16, ctypes.byref(comp), ctypes.byref(win), 16, 1, 16, 100, 128, 4096, 2048, 0.04,
                                   64, 1e4, 0, 16, 16, 1 << 30, z) == 2                        # k too big
+
+
+def test_new_entry_points_reject_bad_arguments():
+    """dsv4kv_index_topk_pool, dsv4kv_append and the fp8 + bf16-rotary format
+    answer bad arguments with status codes before any launch."""
+    L = K.lib()
+    z = ctypes.c_void_p(0)
+    keys = K.CacheDesc(0, 128, 1000, 16, None)
+    pool_args = lambda k, cap, ws: (16, ctypes.byref(keys), 1, 1000, 16, cap, k, 16, z, 16, ws, z)
+    assert L.dsv4kv_index_topk_pool(*pool_args(0, 64, 16)) == 2              # k = 0
+    assert L.dsv4kv_index_topk_pool(*pool_args(512, 9000, 16)) == 2          # pool beyond 8192
+    assert L.dsv4kv_index_topk_pool(*pool_args(512, 64, 8)) == 3             # workspace too small
+    fp8 = K.CacheDesc(1, 128, 1000, 16, 16)
+    assert L.dsv4kv_index_topk_pool(16, ctypes.byref(fp8), 1, 1000, 16, 64, 512, 16, z, 16, 16, z) == 2
+    assert L.dsv4kv_index_topk_pool(16, ctypes.byref(keys), 0, 1000, 16, 64, 512, 16, z, 16, 16, z) == 0  # no batch
+    assert K.lib().dsv4kv_index_topk_pool_workspace_bytes(4, 2048, 512) == 16
+    # append: bad stride, odd rope_dim, a window ring missing, an entry beyond the cache
+    assert L.dsv4kv_append(16, 16, 1, 0, 512, 8, 0, 128, 64, 1e4, 16, 16, 16, 10, z) == 1
+    assert L.dsv4kv_append(16, 16, 1, 0, 512, 8, 4, 128, 63, 1e4, 16, 16, 16, 10, z) == 1
+    assert L.dsv4kv_append(16, 16, 1, 0, 512, 8, 4, 128, 64, 1e4, 16, z, 16, 10, z) == 1
+    rc, msg = _status(L.dsv4kv_append(16, 16, 1, 135, 512, 8, 4, 128, 64, 1e4, 16, 16, 16, 1, z))
+    assert rc == 1 and "does not fit" in msg
+    assert L.dsv4kv_append(z, z, 0, 5, 512, 8, 4, 128, 64, 1e4, z, z, z, 0, z) == 0   # empty batch
+    # the fp8 + bf16-rotary format needs rope_dim == 64 in the decode calls
+    f3 = K.CacheDesc(3, 512, 100, 16, 16)
+    rc = L.dsv4kv_dense_decode(16, ctypes.byref(f3), ctypes.byref(f3), 1, 64, 100, 100, 4096, 0.044, 32, 1e4, 0,
+                               16, 16, 1 << 30, z)
+    assert rc == 2 and "rope_dim" in K.lib().dsv4kv_last_error().decode()
