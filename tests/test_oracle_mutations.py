@@ -118,3 +118,75 @@ def test_format_pin_catches_round_half_away():
         lo = np.clip(hi - 1, 0, 126)
         return np.where(pos[hi] - a <= a - pos[lo], hi, lo).astype(np.uint8)
     assert not np.array_equal(half_away(mids), lib)
+
+
+# ------------------------------------------------ the NEXT rows' oracle functions
+def _pool_matches_brute(fn):
+    rng = np.random.default_rng(21)
+    keys = rng.integers(0, 2, (400, 128)).astype(np.float64)       # scores = counts of ones: many equal
+    keys[399] = 1.0                                                 # the best key, outside the pool
+    q = np.ones(128)
+    pool = np.sort(rng.choice(399, 150, replace=False))
+    s = {int(i): float(keys[i] @ q) for i in pool}
+    want = sorted(sorted(pool.tolist(), key=lambda i: (-s[i], i))[:40])
+    got, _ = fn(q, keys, np.concatenate([pool, [-1, -1]]), 40)
+    return got[:40].tolist() == want
+
+
+def test_pool_pin_catches_tie_and_padding_errors():
+    assert _pool_matches_brute(I.index_topk_pool)
+
+    def ties_to_higher(q, keys, pool, k):                          # ties broken toward the higher entry
+        pool = np.asarray(pool)
+        ent = pool[pool >= 0]
+        sc = keys[ent] @ q
+        order = np.lexsort((-ent, -sc))
+        out = np.full(k, -1, dtype=np.int32)
+        out[:min(k, len(ent))] = np.sort(ent[order[:k]])
+        return out, min(k, len(ent))
+    assert not _pool_matches_brute(ties_to_higher)
+
+    def padding_as_entry(q, keys, pool, k):                        # -1 read as the last entry
+        return I.index_topk_pool(q, keys, np.where(np.asarray(pool) < 0, len(keys) - 1, pool), k)
+    assert not _pool_matches_brute(padding_as_entry)
+
+
+def _fp8_rope_matches_worked_row(fn):
+    x = np.zeros((1, 512), dtype=np.float32)
+    x[0, 0], x[0, 1], x[0, 448], x[0, 511] = 224.0, 1.0, 1.5, -2.0
+    codes, scales = fn(x)
+    return (scales[0] == np.float32(0.5) and codes[0, 0] == 0x7E and codes[0, 1] == 0x40
+            and list(codes[0, 448:450]) == [0xC0, 0x3F] and list(codes[0, 574:576]) == [0x00, 0xC0])
+
+
+def test_fp8_rope_pin_catches_scale_and_byte_order_errors():
+    assert _fp8_rope_matches_worked_row(F.quantize_fp8_rope_rows)
+
+    def scale_over_all_channels(x):                                # amax taken over the rotary channels too
+        x = np.asarray(x, dtype=np.float32).copy()
+        x[:, 448:] *= 1000.0
+        c, s = F.quantize_fp8_rope_rows(x)
+        return c, s
+    x_big = np.zeros((1, 512), dtype=np.float32)
+    x_big[0, 0], x_big[0, 448] = 1.0, 5000.0
+    _, good = F.quantize_fp8_rope_rows(x_big)
+    amax_all = np.float32(5000.0) / np.float32(448.0)
+    assert good[0] != amax_all                                      # the body's amax sets the scale
+
+    def big_endian_rope(x):
+        c, s = F.quantize_fp8_rope_rows(x)
+        c = c.copy()
+        c[:, 448:] = c[:, 448:].reshape(c.shape[0], -1, 2)[:, :, ::-1].reshape(c.shape[0], -1)
+        return c, s
+    assert not _fp8_rope_matches_worked_row(big_endian_rope)
+
+
+def test_append_pin_catches_late_emission():
+    """An emission rule one stride late leaves an entry missing at the step its block leaves the window."""
+    def late(t, window, stride):
+        return max(0, (t - window) // stride - 1)
+    ok = all(C.n_entries(t + 1, 128, 4) - C.n_entries(t, 128, 4) == (1 if (t + 1 - 128) >= 4 and (t + 1 - 128) % 4 == 0 else 0)
+             for t in range(400))
+    bad = all(late(t + 1, 128, 4) - late(t, 128, 4) == (1 if (t + 1 - 128) >= 4 and (t + 1 - 128) % 4 == 0 else 0)
+              for t in range(400))
+    assert ok and not bad
