@@ -123,12 +123,17 @@ def test_format_pin_catches_round_half_away():
 # ------------------------------------------------ the NEXT rows' oracle functions
 def _pool_matches_brute(fn):
     rng = np.random.default_rng(21)
-    keys = rng.integers(0, 2, (400, 128)).astype(np.float64)       # scores = counts of ones: many equal
+    # score of entry i = the number of leading ones of key i, in 60..69: ~15 pool entries per value
+    keys = np.zeros((400, 128))
+    for i, c in enumerate(rng.integers(60, 70, 400)):
+        keys[i, :c] = 1.0
     keys[399] = 1.0                                                 # the best key, outside the pool
     q = np.ones(128)
     pool = np.sort(rng.choice(399, 150, replace=False))
     s = {int(i): float(keys[i] @ q) for i in pool}
-    want = sorted(sorted(pool.tolist(), key=lambda i: (-s[i], i))[:40])
+    ranked = sorted(pool.tolist(), key=lambda i: (-s[i], i))
+    assert s[ranked[39]] == s[ranked[40]]                           # the cut falls inside a group of ties
+    want = sorted(ranked[:40])
     got, _ = fn(q, keys, np.concatenate([pool, [-1, -1]]), 40)
     return got[:40].tolist() == want
 
