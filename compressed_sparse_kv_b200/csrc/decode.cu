@@ -1112,12 +1112,12 @@ size_t decode_ws_bytes(int batch, int heads, int dim, int64_t rows_per_seq) {
 template <int FMT>
 dsv4kv_status launch_fmt(const CUtensorMap& tq, const CUtensorMap& tc, const CUtensorMap& tw, const Params& p,
                          int grid, cudaStream_t stream) {
-  static bool attr_set = false;  // per instantiation
-  if (!attr_set) {
+  static std::atomic<uint64_t> attr_set{0};  // per instantiation, one bit per device
+  if (!done_on_device(attr_set)) {
     if (cudaFuncSetAttribute(decode_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes)) !=
         cudaSuccess)
       return check_launch("decode: cudaFuncSetAttribute");
-    attr_set = true;
+    mark_done_on_device(attr_set);
   }
   launch_pdl(decode_kernel<FMT>, dim3(grid), dim3(kThreads), kSmemBytes, stream, tq, tc, tw, p);
   return check_launch("decode_kernel");

@@ -1174,14 +1174,14 @@ dsv4kv_status index_topk_pool_launch(const uint16_t* qidx, const dsv4kv_cache& k
   if (pool_cap > kPoolMax)
     return set_error(DSV4KV_ERR_UNSUPPORTED, "index_topk_pool: pool of %d entries > %d", pool_cap, kPoolMax);
   uint32_t* status = static_cast<uint32_t*>(ws);
-  static bool attr = false;
-  if (!attr) {
+  static std::atomic<uint64_t> attr{0};  // one bit per device
+  if (!done_on_device(attr)) {
     if (cudaFuncSetAttribute(index_pool_select<DSV4KV_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(kPoolDyn)) != cudaSuccess ||
         cudaFuncSetAttribute(index_pool_select<DSV4KV_FP4_E2M1_G16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(kPoolDyn)) != cudaSuccess)
       return check_launch("index_topk_pool: cudaFuncSetAttribute");
-    attr = true;
+    mark_done_on_device(attr);
   }
   if (keys.fmt == DSV4KV_BF16)
     launch_pdl(index_pool_select<DSV4KV_BF16>, dim3(unsigned(batch)), dim3(kSelThreads), kPoolDyn, stream, qidx,
@@ -1246,7 +1246,8 @@ dsv4kv_status index_score_launch(const uint16_t* qidx, const dsv4kv_cache& keys,
   const int sms = sm_count();
   if (keys.fmt == DSV4KV_BF16) {
     // one wave (resident CTAs per SM x SMs) over the flattened (sequence, entry) range
-    static int occ = 0;
+    static int occ_dev[64] = {0};  // per device
+    int& occ = occ_dev[current_device()];
     if (occ == 0 &&
         (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, index_score_bf16<8>, 256, 0) != cudaSuccess ||
          occ < 1))
@@ -1262,7 +1263,8 @@ dsv4kv_status index_score_launch(const uint16_t* qidx, const dsv4kv_cache& keys,
                static_cast<const uint16_t*>(keys.codes), keys.rows, n, n_h, batch, per_cta, w.scores, w.hist,
                w.tail_ctr);
   } else {
-    static int occ4 = 0;
+    static int occ4_dev[64] = {0};  // per device
+    int& occ4 = occ4_dev[current_device()];
     if (occ4 == 0 &&
         (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ4, index_score_fp4, 256, 0) != cudaSuccess || occ4 < 1))
       occ4 = 1;
@@ -1283,7 +1285,8 @@ dsv4kv_status index_select_launch(int batch, int64_t n, int k, int32_t* idx_out,
   if (ws_bytes < w.bytes) return set_error(DSV4KV_ERR_WORKSPACE, "index_select: workspace too small");
   const int sms = sm_count();
   // selection: one cluster of C CTAs per sequence, chunks of whole 4096-score batches
-  static int max_cluster = 0;
+  static int max_cluster_dev[64] = {0};  // per device
+  int& max_cluster = max_cluster_dev[current_device()];
   if (max_cluster == 0) {
     if (cudaFuncSetAttribute(index_select, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSelDyn)) != cudaSuccess)
       return check_launch("index_select: cudaFuncSetAttribute");

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <utility>
 #include <cstdint>
 
@@ -52,6 +53,19 @@ cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, 
 }
 dsv4kv_status check_launch(const char* what);
 int sm_count();
+// The current device (0 when it cannot be read or is >= 64).  One-time set-up
+// of a kernel (shared-memory limits, occupancy queries) is kept per device,
+// so a process that drives several GPUs sets every one of them up.
+inline int current_device() {
+  int d = 0;
+  return (cudaGetDevice(&d) == cudaSuccess && d >= 0 && d < 64) ? d : 0;
+}
+inline bool done_on_device(const std::atomic<uint64_t>& mask) {
+  return (mask.load(std::memory_order_acquire) >> current_device()) & 1u;
+}
+inline void mark_done_on_device(std::atomic<uint64_t>& mask) {
+  mask.fetch_or(uint64_t(1) << current_device(), std::memory_order_acq_rel);
+}
 
 // Driver entry point for cuTensorMapEncodeTiled (resolved once through the runtime).
 bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
