@@ -133,11 +133,12 @@ def step_bytes(kind, batch, t, main_fmt, index_fmt, k=512, window=128, pool=0):
     return b
 
 
-def replicas_for(kind, batch, t, main_fmt, index_fmt, at_least, pool=0):
+def replicas_for(kind, batch, t, main_fmt, index_fmt, at_least, pool=0, l2_factor=4):
     """Cache replicas the timed steps cycle through: together they hold at
-    least four times the L2, so every step streams its rows from DRAM."""
+    least `l2_factor` times the L2 (4 for every timed run), so every step
+    streams its rows from DRAM."""
     per = step_bytes(kind, batch, t, main_fmt, index_fmt, pool=pool)
-    return max(at_least, -(-4 * L2_BYTES // per))
+    return max(at_least, -(-l2_factor * L2_BYTES // per))
 
 
 class Layer:
@@ -695,6 +696,8 @@ def main():
     ap.add_argument("--no-stack", action="store_true", help="skip the 61-layer stack step")
     ap.add_argument("--no-bulk", action="store_true", help="skip compressor/quantiser throughput")
     ap.add_argument("--replicas", type=int, default=2, help="minimum cache replicas (raised until they hold 4x L2)")
+    ap.add_argument("--l2-factor", type=int, default=4,
+                    help="replicas hold at least this many L2 sizes (0 only for small profiling runs)")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -734,7 +737,7 @@ def main():
     torch.cuda.set_device(d["local"])
     hbm_peak, tf_peak, peak_src = measured_peaks()
     seed = 1234 + d["rank"]
-    reps = replicas_for(kind, batch, t, mfmt, ifmt, args.replicas, pool)
+    reps = replicas_for(kind, batch, t, mfmt, ifmt, args.replicas, pool, args.l2_factor)
     layer = Layer(kind, batch, t, heads, seed, reps, mfmt, ifmt, pool=pool)
     res = time_layer(layer, args.steps, args.warmup, dist_max, d["local"], sample_clocks=(d["rank"] == 0))
     ms = res["total_ms"] / args.steps
