@@ -933,18 +933,21 @@ __global__ void index_fill_all(int64_t n, int k, int32_t* __restrict__ idx_out, 
 // ------------------------------------------------------------------ pool re-index
 // [P3] CSA2: a "Reindex" layer keeps its indexing inside the candidate pool
 // built by the first layer in Full mode (the layers share the indexer keys).
-// One CTA of 512 threads per sequence: the pool (ascending entry indices,
-// negative = no entry) is copied to shared memory, the pool's keys are
-// gathered and scored (half a warp per bf16 key, a quarter warp per fp4 key)
-// into shared memory as order-preserving codes, and the exact selection runs
-// there: the 12-bit histogram gives the threshold bin, a second 12-bit
+// One thread-block cluster of C <= 4 CTAs (512 threads) per sequence: CTA r
+// gathers and scores the r-th part of the pool (ascending entry indices,
+// negative = no entry; half a warp per bf16 key, a quarter warp per fp4 key)
+// and pushes the order-preserving codes, its 12-bit histogram and its count
+// into the leader's shared memory; after one cluster barrier the leader runs
+// the exact selection: the 12-bit histogram gives the threshold bin, a second 12-bit
 // histogram of that bin the 24-bit prefix, a 256-bin histogram of the
 // entries at the prefix the threshold code, and the entries equal to it are
 // taken in pool order (= entry order, so ties go to the lower entry); an
 // ordered compaction over pool positions writes the result ascending.
 constexpr int kPoolMax = 8192;
 constexpr int kPoolPer = kPoolMax / kSelThreads;  // pool positions per thread
-constexpr size_t kPoolDyn = 2 * size_t(kPoolMax) * sizeof(uint32_t);
+constexpr int kMaxPoolCluster = 4;
+// dynamic shared memory: codes and entries of the pool, the CTAs' histograms (leader)
+constexpr size_t kPoolDyn = (2 * size_t(kPoolMax) + size_t(kMaxPoolCluster) * kHistBins) * sizeof(uint32_t);
 
 // The bin where the descending cumulative count of a 256-bin histogram first
 // reaches `need`; *above = count in higher bins.  Warp 0 scans (8 bins per
@@ -989,23 +992,33 @@ __global__ void __launch_bounds__(kSelThreads, 1)
                       const int32_t* __restrict__ pool, int pool_cap, int k, int32_t* __restrict__ idx_out,
                       int32_t* __restrict__ count_out, uint32_t* __restrict__ status) {
   extern __shared__ __align__(16) uint32_t psm[];
-  uint32_t* pcode = psm;              // kPoolMax order-preserving codes (0 = no entry)
-  int32_t* pent = reinterpret_cast<int32_t*>(psm + kPoolMax);  // the pool's entries
+  uint32_t* pcode = psm;              // leader: kPoolMax order-preserving codes (0 = no entry)
+  int32_t* pent = reinterpret_cast<int32_t*>(psm + kPoolMax);  // the pool's entries (this CTA's part; leader: all)
+  uint32_t* hparts = psm + 2 * kPoolMax;                       // leader: the CTAs' histograms
   __shared__ __align__(16) uint32_t sh[kHistBins];
   __shared__ uint32_t s_cnt;
-  const int b = blockIdx.x;
+  __shared__ uint32_t s_cparts[kMaxPoolCluster];
+  const int b = blockIdx.y;
+  const uint32_t rank = cluster_rank(), csize = gridDim.x;  // one cluster spans the sequence's CTAs
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int32_t* pb = pool + size_t(b) * pool_cap;
+  // this CTA's part of the pool: [c0, c1), whole multiples of 32 positions
+  const int part = ((pool_cap + int(csize) - 1) / int(csize) + 31) / 32 * 32;
+  const int c0 = min(pool_cap, int(rank) * part), c1 = min(pool_cap, c0 + part);
   for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) sh[i] = 0;
   if (threadIdx.x == 0) s_cnt = 0;
   pdl_trigger();
   pdl_wait();
-  // the pool, and its validity: entries in [0, n), ascending
-  for (int j = threadIdx.x; j < pool_cap; j += kSelThreads) {
+  // the pool (the leader reads all of it for the output and checks it: entries
+  // in [0, n), ascending); the other CTAs read their part
+  const int e0 = rank == 0 ? 0 : c0, e1 = rank == 0 ? pool_cap : c1;
+  for (int j = e0 + int(threadIdx.x); j < e1; j += kSelThreads) {
     const int32_t e = pb[j];
     pent[j] = e;
-    if (e >= n) set_status(status, DSV4KV_DEV_BAD_INDEX);
-    if (e >= 0 && j > 0 && !(pb[j - 1] >= 0 && pb[j - 1] < e)) set_status(status, DSV4KV_DEV_BAD_POOL);
+    if (rank == 0) {
+      if (e >= n) set_status(status, DSV4KV_DEV_BAD_INDEX);
+      if (e >= 0 && j > 0 && !(pb[j - 1] >= 0 && pb[j - 1] < e)) set_status(status, DSV4KV_DEV_BAD_POOL);
+    }
   }
   __syncthreads();
   const uint64_t pol = l2_evict_first_policy();
@@ -1022,13 +1035,13 @@ __global__ void __launch_bounds__(kSelThreads, 1)
       q[4] = bf16lo(v.z); q[5] = bf16hi(v.z); q[6] = bf16lo(v.w); q[7] = bf16hi(v.w);
     }
     const uint16_t* kb = static_cast<const uint16_t*>(codes) + size_t(b) * size_t(key_rows) * 128 + 8 * l16;
-    for (int it = 0; it * 32 * U < pool_cap; ++it) {
-      const int j0 = hw + 32 * U * it;
+    for (int it = 0; it * 32 * U < c1 - c0; ++it) {
+      const int j0 = c0 + hw + 32 * U * it;
       uint4 v[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int j = j0 + 32 * u;
-        const int32_t e = j < pool_cap ? pent[j] : -1;
+        const int32_t e = j < c1 ? pent[j] : -1;
         v[u] = (e >= 0 && e < n) ? ld_once_v4(kb + size_t(e) * 128, pol) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
@@ -1038,11 +1051,11 @@ __global__ void __launch_bounds__(kSelThreads, 1)
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) sc += __shfl_xor_sync(kFull, sc, o);
         sc += 0.0f;  // -0 -> +0
-        if (l16 == 0 && j < pool_cap) {
+        if (l16 == 0 && j < c1) {
           const int32_t e = pent[j];
           const bool ok = e >= 0 && e < n;
           const uint32_t c = ok ? ord_f32(sc) : 0u;
-          pcode[j] = c;
+          st_dsmem_u32(dsmem_addr(&pcode[j], 0), c);
           if (ok) {
             atomicAdd(&sh[c >> 20], 1u);
             atomicAdd(&s_cnt, 1u);
@@ -1063,14 +1076,14 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     }
     const uint8_t* cb = static_cast<const uint8_t*>(codes) + size_t(b) * size_t(key_rows) * 64 + 16 * l4;
     const uint8_t* sb = kscales + size_t(b) * size_t(key_rows) * 8 + 2 * l4;
-    for (int it = 0; it * 128 * U < pool_cap; ++it) {
-      const int j0 = quad + 128 * U * it;
+    for (int it = 0; it * 128 * U < c1 - c0; ++it) {
+      const int j0 = c0 + quad + 128 * U * it;
       uint4 v[U];
       uint32_t s2[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int j = j0 + 128 * u;
-        const int32_t e = j < pool_cap ? pent[j] : -1;
+        const int32_t e = j < c1 ? pent[j] : -1;
         const bool ok = e >= 0 && e < n;
         v[u] = ok ? ld_once_v4(cb + size_t(e) * 64, pol) : make_uint4(0, 0, 0, 0);
         s2[u] = ok ? ld_once_u16(sb + size_t(e) * 8, pol) : 0u;
@@ -1094,11 +1107,11 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         sc += __shfl_xor_sync(kFull, sc, 1);
         sc += __shfl_xor_sync(kFull, sc, 2);
         sc += 0.0f;
-        if (l4 == 0 && j < pool_cap) {
+        if (l4 == 0 && j < c1) {
           const int32_t e = pent[j];
           const bool ok = e >= 0 && e < n;
           const uint32_t c = ok ? ord_f32(sc) : 0u;
-          pcode[j] = c;
+          st_dsmem_u32(dsmem_addr(&pcode[j], 0), c);
           if (ok) {
             atomicAdd(&sh[c >> 20], 1u);
             atomicAdd(&s_cnt, 1u);
@@ -1106,6 +1119,25 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         }
       }
     }
+  }
+  __syncthreads();
+  // this CTA's histogram and count into the leader; one cluster barrier
+  {
+    const uint32_t hdst = dsmem_addr(hparts + size_t(rank) * kHistBins, 0);
+    for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) st_dsmem_u32(hdst + 4u * uint32_t(i), sh[i]);
+    if (threadIdx.x == 0) st_dsmem_u32(dsmem_addr(&s_cparts[rank], 0), s_cnt);
+  }
+  cluster_sync();  // every code, histogram and count is in the leader's shared memory
+  if (rank != 0) return;
+  for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) {
+    uint32_t sum = 0;
+    for (uint32_t r = 0; r < csize; ++r) sum += hparts[size_t(r) * kHistBins + i];
+    sh[i] = sum;
+  }
+  if (threadIdx.x == 0) {
+    uint32_t tot = 0;
+    for (uint32_t r = 0; r < csize; ++r) tot += s_cparts[r];
+    s_cnt = tot;
   }
   __syncthreads();
   const uint32_t cnt = s_cnt;
@@ -1183,14 +1215,17 @@ dsv4kv_status index_topk_pool_launch(const uint16_t* qidx, const dsv4kv_cache& k
       return check_launch("index_topk_pool: cudaFuncSetAttribute");
     mark_done_on_device(attr);
   }
+  // C CTAs per sequence, as many as keep the grid within one CTA per SM
+  const int csize = std::max(1, std::min(kMaxPoolCluster, sm_count() / std::max(batch, 1)));
+  const dim3 grid{static_cast<unsigned>(csize), static_cast<unsigned>(batch)};
   if (keys.fmt == DSV4KV_BF16)
-    launch_pdl(index_pool_select<DSV4KV_BF16>, dim3(unsigned(batch)), dim3(kSelThreads), kPoolDyn, stream, qidx,
-               keys.codes, static_cast<const uint8_t*>(keys.scales), keys.rows, n, pool, pool_cap, k, idx_out,
-               count_out, status);
+    launch_pdl_cluster(index_pool_select<DSV4KV_BF16>, grid, dim3(kSelThreads), kPoolDyn, unsigned(csize), stream,
+                       qidx, keys.codes, static_cast<const uint8_t*>(keys.scales), keys.rows, n, pool, pool_cap, k,
+                       idx_out, count_out, status);
   else
-    launch_pdl(index_pool_select<DSV4KV_FP4_E2M1_G16>, dim3(unsigned(batch)), dim3(kSelThreads), kPoolDyn, stream,
-               qidx, keys.codes, static_cast<const uint8_t*>(keys.scales), keys.rows, n, pool, pool_cap, k, idx_out,
-               count_out, status);
+    launch_pdl_cluster(index_pool_select<DSV4KV_FP4_E2M1_G16>, grid, dim3(kSelThreads), kPoolDyn, unsigned(csize),
+                       stream, qidx, keys.codes, static_cast<const uint8_t*>(keys.scales), keys.rows, n, pool,
+                       pool_cap, k, idx_out, count_out, status);
   return check_launch("index_pool_select");
 }
 
