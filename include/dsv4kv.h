@@ -40,7 +40,7 @@ extern "C" {
 typedef enum {
   DSV4KV_OK = 0,
   DSV4KV_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer  */
-  DSV4KV_ERR_UNSUPPORTED = 2,  /* a format or dimension this build lacks      */
+  DSV4KV_ERR_UNSUPPORTED = 2,  /* a format or dimension the library lacks    */
   DSV4KV_ERR_WORKSPACE = 3,    /* workspace null or smaller than required     */
   DSV4KV_ERR_CUDA = 4          /* CUDA runtime/driver error at launch         */
 } dsv4kv_status;
