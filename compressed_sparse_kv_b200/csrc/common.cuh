@@ -72,10 +72,6 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   return r;
 }
 // Every thread of every CTA of the cluster must call it (no early exits before).
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -87,21 +83,11 @@ __device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
                : "r"(uint32_t(__cvta_generic_to_shared(p))), "r"(rank));
   return a;
 }
-__device__ __forceinline__ uint32_t ld_dsmem_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
-}
 __device__ __forceinline__ void st_dsmem_u32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 __device__ __forceinline__ void st_dsmem_u64(uint32_t addr, uint64_t v) {
   asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
-}
-__device__ __forceinline__ uint64_t ld_dsmem_u64(uint32_t addr) {
-  uint64_t v;
-  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
-  return v;
 }
 
 // ----------------------------------------------------------------- programmatic dependent launch
