@@ -67,7 +67,10 @@ typedef enum {
  *                        value = E4M3(code) * scale for channels < dim - 64, the bf16 value
  *                        for the rest.  ([P1] quantisation paragraph: fp8 for most of the
  *                        attention cache, the RoPE dimensions in bf16.)  With this format
- *                        the decode calls require rope_dim == 64.
+ *                        the decode calls require rope_dim == 64; they stage the rotary
+ *                        values as f16 of value / scale, accurate while a row's rotary
+ *                        values stay below 146 x the largest magnitude of its other
+ *                        channels (the f16 range).
  */
 typedef enum {
   DSV4KV_BF16 = 0,
