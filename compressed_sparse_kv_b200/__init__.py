@@ -62,6 +62,7 @@ _SIGS = {
     "dsv4kv_index_topk_noalloc_max_scratch_bytes": (_c.c_size_t, []),
     "dsv4kv_index_topk_noalloc": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.c_int32, _c.c_int64, _c.c_int32,
                                              _c.c_void_p, _c.c_void_p, _c.c_void_p]),
+    "dsv4kv_index_topk_noalloc_status": (_c.c_int, [_c.c_void_p, _c.c_int32, _c.c_void_p]),
     "dsv4kv_sparse_decode_workspace_bytes": (_c.c_size_t, [_c.c_int32, _c.c_int32, _c.c_int32, _c.c_int32,
                                                            _c.c_int32]),
     "dsv4kv_sparse_decode": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.POINTER(CacheDesc), _c.c_void_p,
@@ -250,6 +251,17 @@ def index_topk_noalloc(qidx: torch.Tensor, keys: Cache, n: int, k: int, idx_out:
     _check(lib().dsv4kv_index_topk_noalloc(_ptr(qidx), ctypes.byref(d), b, n, k, _ptr(idx_out), _ptr(count_out),
                                            _stream(stream)), "dsv4kv_index_topk_noalloc")
     return idx_out, count_out
+
+
+def index_topk_noalloc_status(clear: bool = False, stream=None) -> int:
+    """The device status word (DEV_* flags) that the calls of index_topk_noalloc have accumulated in the
+    static scratch since it was last cleared; `clear` zeroes it after reading."""
+    word = torch.zeros(1, dtype=torch.int32).pin_memory()
+    s = torch.cuda.current_stream() if stream is None else stream
+    _check(lib().dsv4kv_index_topk_noalloc_status(_ptr(word), int(clear), _stream(s)),
+           "dsv4kv_index_topk_noalloc_status")
+    s.synchronize()
+    return int(word.item()) & 0xffffffff
 
 
 def sparse_decode_workspace_bytes(batch: int, heads: int, k: int, window: int, dim: int = 512) -> int:

@@ -713,6 +713,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
   const int lane = threadIdx.x & 31;
   pdl_trigger();
   pdl_wait();
+  cluster_arrive_relaxed();  // this CTA has started (waited for before the first remote store)
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *tail_ctr = 0;  // the score kernel's queue, for the next call
 
   // 1) every warp owns a contiguous run of the CTA's chunk; the first
@@ -770,6 +771,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
     over |= tot > regcap;
     const uint32_t mine = min(wc, uint32_t(kWarpCap));
     const uint32_t dst = dsmem_addr(recv + size_t(rank) * regcap, 0);
+    cluster_wait();  // every CTA of the cluster (the leader among them) has started
     if (!over)
       for (uint32_t i = lane; i < mine; i += 32) st_dsmem_u64(dst + 8u * (off + i), wl[i]);
     if (threadIdx.x == 0) st_dsmem_u32(dsmem_addr(&s_rcnt[rank], 0), over ? 0xffffffffu : tot);
@@ -1009,6 +1011,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   if (threadIdx.x == 0) s_cnt = 0;
   pdl_trigger();
   pdl_wait();
+  cluster_arrive_relaxed();  // this CTA has started (waited for before the first remote store)
   // the pool (the leader reads all of it for the output and checks it: entries
   // in [0, n), ascending); the other CTAs read their part
   const int e0 = rank == 0 ? 0 : c0, e1 = rank == 0 ? pool_cap : c1;
@@ -1021,6 +1024,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     }
   }
   __syncthreads();
+  cluster_wait();  // every CTA of the cluster (the leader among them) has started
   const uint64_t pol = l2_evict_first_policy();
   if constexpr (FMT == DSV4KV_BF16) {
     // half-warp hw scores positions hw, hw + 32, ...; 16 keys in flight per
@@ -1281,12 +1285,14 @@ dsv4kv_status index_score_launch(const uint16_t* qidx, const dsv4kv_cache& keys,
   const int sms = sm_count();
   if (keys.fmt == DSV4KV_BF16) {
     // one wave (resident CTAs per SM x SMs) over the flattened (sequence, entry) range
-    static int occ_dev[64] = {0};  // per device
-    int& occ = occ_dev[current_device()];
-    if (occ == 0 &&
-        (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, index_score_bf16<8>, 256, 0) != cudaSuccess ||
-         occ < 1))
-      occ = 1;
+    static std::atomic<int> occ_dev[64];  // per device; 0 = not queried yet
+    std::atomic<int>& occ_slot = occ_dev[current_device()];
+    int occ = occ_slot.load(std::memory_order_relaxed);
+    if (occ == 0) {
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, index_score_bf16<8>, 256, 0) != cudaSuccess || occ < 1)
+        occ = 1;
+      occ_slot.store(occ, std::memory_order_relaxed);
+    }
     // the last kTailPct % of every sequence (whole units) goes to the shared queue
     const int64_t n_tail = std::min<int64_t>(n, (n * kTailPct / 100) / kTailUnit * kTailUnit);
     const int64_t n_h = n - n_tail;
@@ -1298,11 +1304,14 @@ dsv4kv_status index_score_launch(const uint16_t* qidx, const dsv4kv_cache& keys,
                static_cast<const uint16_t*>(keys.codes), keys.rows, n, n_h, batch, per_cta, w.scores, w.hist,
                w.tail_ctr);
   } else {
-    static int occ4_dev[64] = {0};  // per device
-    int& occ4 = occ4_dev[current_device()];
-    if (occ4 == 0 &&
-        (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ4, index_score_fp4, 256, 0) != cudaSuccess || occ4 < 1))
-      occ4 = 1;
+    static std::atomic<int> occ4_dev[64];  // per device; 0 = not queried yet
+    std::atomic<int>& occ4_slot = occ4_dev[current_device()];
+    int occ4 = occ4_slot.load(std::memory_order_relaxed);
+    if (occ4 == 0) {
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ4, index_score_fp4, 256, 0) != cudaSuccess || occ4 < 1)
+        occ4 = 1;
+      occ4_slot.store(occ4, std::memory_order_relaxed);
+    }
     const int64_t total = int64_t(batch) * n;
     const int64_t grid = int64_t(sms) * occ4;
     const int64_t per_cta = std::max<int64_t>(64, (total + grid - 1) / grid);
@@ -1320,8 +1329,9 @@ dsv4kv_status index_select_launch(int batch, int64_t n, int k, int32_t* idx_out,
   if (ws_bytes < w.bytes) return set_error(DSV4KV_ERR_WORKSPACE, "index_select: workspace too small");
   const int sms = sm_count();
   // selection: one cluster of C CTAs per sequence, chunks of whole 4096-score batches
-  static int max_cluster_dev[64] = {0};  // per device
-  int& max_cluster = max_cluster_dev[current_device()];
+  static std::atomic<int> max_cluster_dev[64];  // per device; 0 = not set up yet
+  std::atomic<int>& max_cluster_slot = max_cluster_dev[current_device()];
+  int max_cluster = max_cluster_slot.load(std::memory_order_acquire);
   if (max_cluster == 0) {
     if (cudaFuncSetAttribute(index_select, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSelDyn)) != cudaSuccess)
       return check_launch("index_select: cudaFuncSetAttribute");
@@ -1343,6 +1353,7 @@ dsv4kv_status index_select_launch(int batch, int64_t n, int k, int32_t* idx_out,
         max_cluster = kMaxClusterSel;
     }
     cudaGetLastError();  // a refused query only means the portable size
+    max_cluster_slot.store(max_cluster, std::memory_order_release);
   }
   // at most one CTA per SM in all (the leader's registers allow one per SM)
   const int64_t per_seq = std::max<int64_t>(1, std::min<int64_t>(max_cluster, sms / std::max(batch, 1)));

@@ -11,7 +11,10 @@
  *  - Every pointer argument that names tensor data is DEVICE memory owned by
  *    the caller (for example allocated through PyTorch).  The library keeps
  *    no pointer after a call returns and allocates no device memory on any
- *    call path; scratch memory is the caller's workspace.
+ *    call path; scratch memory is the caller's workspace.  The one exception
+ *    is dsv4kv_index_topk_noalloc, whose scratch is a library-owned static
+ *    device array shared by all its calls (calls to it that overlap on the
+ *    GPU race).
  *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *    NULL = the legacy default stream) and never synchronises the host.
  *  - Tensors are dense and row-major with the shapes given below.
@@ -242,16 +245,26 @@ dsv4kv_status dsv4kv_index_topk_pool(const void* qidx, const dsv4kv_cache* keys,
  * which loads the library holds until the process exits.  A call whose
  * scratch need (dsv4kv_index_topk_workspace_bytes) exceeds it returns
  * DSV4KV_ERR_UNSUPPORTED; batch 32 x 32736 entries with k = 512 fits.  The
- * first call on a device (with that device current) looks up the array's
- * device address; make it before any stream capture.  Each call clears the
- * scratch counters on `stream` first.  All calls share the one array, so
- * calls that overlap on the GPU race.  Nothing here allocates memory.
+ * call looks up the array's device address on the current device; the first
+ * lookup on a device loads the library's device code there, so make the first
+ * call before any stream capture.  Each call clears the scratch counters and
+ * histograms on `stream` first.  All calls share the one array, so calls that
+ * overlap on the GPU race.  Nothing here allocates memory.
+ *
+ * The scratch's status word (the DSV4KV_DEV_* flags a workspace would carry)
+ * is not cleared by the calls: it accumulates the flags of every call on the
+ * device.  dsv4kv_index_topk_noalloc_status copies it into *host_out on
+ * `stream` (with pinned host memory the copy is asynchronous: synchronise the
+ * stream before reading it) and then, if `clear` != 0, zeroes it on `stream`.
+ * A non-zero word means an output since the last clear may be invalid.
  * ------------------------------------------------------------------------ */
 size_t dsv4kv_index_topk_noalloc_max_scratch_bytes(void);
 
 dsv4kv_status dsv4kv_index_topk_noalloc(const void* qidx, const dsv4kv_cache* keys, int32_t batch,
                                         int64_t n, int32_t k, int32_t* idx_out, int32_t* count_out,
                                         void* stream);
+
+dsv4kv_status dsv4kv_index_topk_noalloc_status(uint32_t* host_out, int32_t clear, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Decode attention with shared K/V.  [P2] Step 3: one cached vector S_j is
