@@ -44,6 +44,9 @@ WORKLOADS = {
     # a CSA2 Reindex layer: top-512 re-indexed inside the 2048-entry pool a Full
     # layer built (the pool size is a reading; the pages give none)
     "c4a_b32_reindex": ("c4a", 32, 131072, 64, 0, 0, 2048),
+    # paged caches of a ragged batch: every sequence has its own length (uniform in
+    # [t/2, t], seeded), its caches in 256-row pages of shared pools, pages shuffled
+    "c4a_b32_paged": ("c4a", 32, 131072, 64, 0, 0, 0, "paged"),
 }
 FMT_NAME = {0: "bf16", 1: "fp8", 2: "fp4", 3: "fp8+bf16rope"}
 L2_BYTES = 126 * 2 ** 20
@@ -141,6 +144,103 @@ def replicas_for(kind, batch, t, main_fmt, index_fmt, at_least, pool=0, l2_facto
     return max(at_least, -(-l2_factor * L2_BYTES // per))
 
 
+PAGE_ROWS = 256
+
+
+def ragged_lengths(batch, t, seed):
+    """Per-sequence query positions of the ragged workloads: uniform in [t/2, t]."""
+    rng = np.random.default_rng(seed)
+    return rng.integers(t // 2, t + 1, size=batch).astype(np.int64)
+
+
+class PagedLayer:
+    """A c4a layer over paged caches of a ragged batch (R replicas of pools and
+    shuffled block tables): one step is dsv4kv_index_topk_paged +
+    dsv4kv_sparse_decode_paged."""
+
+    def __init__(self, batch, t, heads, seed, replicas, layer_id=0):
+        import torch
+        import compressed_sparse_kv_b200 as K
+        import datagen.gpu as G
+        from datagen import workloads as WL
+        self.K, self.torch = K, torch
+        self.kind, self.batch, self.t, self.heads = "c4a", batch, t, heads
+        self.main_fmt, self.index_fmt, self.pool = 0, 0, 0
+        self.window, self.k = 128, 512
+        self.t_host = ragged_lengths(batch, t, seed)
+        self.t_max = int(t)
+        self.n_seq = np.maximum(0, (self.t_host - self.window) // 4)
+        self.n = int(self.n_seq.max())
+        dev = "cuda"
+        rng = np.random.default_rng(seed + 1)
+
+        def tables(counts):
+            need = (counts + PAGE_ROWS - 1) // PAGE_ROWS
+            perm = rng.permutation(int(need.sum())).astype(np.int32)
+            tab = np.full((batch, max(1, int(need.max()))), -1, np.int32)
+            o = 0
+            for b, m in enumerate(need):
+                tab[b, :m] = perm[o:o + m]
+                o += m
+            return torch.from_numpy(tab).to(dev), int(need.sum())
+
+        w_seq = np.minimum(self.t_host, self.window)
+        self.reps = []
+        for r in range(replicas):
+            keys = WL.keys_for(seed, 1000 * r + layer_id)
+            ct, cp = tables(self.n_seq)
+            kt, kp = tables(self.n_seq)
+            wt, wp = tables(w_seq)
+            comp = G.normal_bf16_(torch.empty(cp * PAGE_ROWS, 512, dtype=torch.bfloat16, device=dev), keys["comp"])
+            win = G.normal_bf16_(torch.empty(wp * PAGE_ROWS, 512, dtype=torch.bfloat16, device=dev), keys["win"])
+            kidx = G.int_bf16_(torch.empty(kp * PAGE_ROWS, 128, dtype=torch.bfloat16, device=dev), keys["kidx"])
+            self.reps.append({"comp": K.PagedCache(0, comp, ct, PAGE_ROWS), "win": K.PagedCache(0, win, wt, PAGE_ROWS),
+                              "kidx": K.PagedCache(0, kidx, kt, PAGE_ROWS, dim=128)})
+        keys = WL.keys_for(seed, layer_id)
+        self.t_seq = torch.from_numpy(self.t_host).to(dev)
+        self.q = G.normal_bf16_(torch.empty(batch, heads, 512, dtype=torch.bfloat16, device=dev), keys["q"])
+        self.qidx = G.int_bf16_(torch.empty(batch, 128, dtype=torch.bfloat16, device=dev), keys["qidx"])
+        self.idx = torch.empty(batch, self.k, dtype=torch.int32, device=dev)
+        self.cnt = torch.empty(batch, dtype=torch.int32, device=dev)
+        self.out = torch.empty(batch, heads, 512, dtype=torch.bfloat16, device=dev)
+        self.ws_idx = K.new_workspace(K.lib().dsv4kv_index_topk_paged_workspace_bytes(batch, self.t_max, 128, 4, 512))
+        self.ws_dec = K.new_workspace(K.lib().dsv4kv_sparse_decode_paged_workspace_bytes(batch, heads, 512, 512, 128))
+        torch.cuda.synchronize()
+
+    def alg_bytes(self):
+        sel = np.minimum(self.n_seq, self.k)
+        win = np.minimum(self.t_host, self.window)
+        return int((self.n_seq * KEY_BYTES[0]).sum() + ((sel + win) * ROW_BYTES[0]).sum())
+
+    def index_bytes(self):
+        return int((self.n_seq * KEY_BYTES[0]).sum()) + self.batch * 256
+
+    def flops(self):
+        return int(((np.minimum(self.n_seq, self.k) + np.minimum(self.t_host, self.window)) * 4 * self.heads * 512).sum())
+
+    def launches_per_step(self):
+        return 4
+
+    def index(self, r, qidx=None):
+        self.K.index_topk_paged(self.qidx if qidx is None else qidx, self.reps[r]["kidx"], self.t_seq, self.t_max,
+                                self.k, idx_out=self.idx, count_out=self.cnt, ws=self.ws_idx)
+
+    def index_score(self, r):
+        self.index(r)
+
+    def index_select(self):
+        pass
+
+    def decode(self, r, q=None, out=None):
+        rep = self.reps[r]
+        self.K.sparse_decode_paged(self.q if q is None else q, rep["comp"], rep["win"], self.idx, self.t_seq,
+                                   self.t_max, out=self.out if out is None else out, ws=self.ws_dec)
+
+    def step(self, r):
+        self.index(r)
+        self.decode(r)
+
+
 class Layer:
     """One layer's resident caches (R replicas) and per-step buffers on the GPU."""
 
@@ -226,11 +326,13 @@ class Layer:
             return 2
         return 3 if self.pool else 4
 
-    def index(self, r):
+    def index(self, r, qidx=None):
+        qidx = self.qidx if qidx is None else qidx
         if self.pool:
-            self.index_score(r)
+            self.K.index_topk_pool(qidx, self.reps[r]["kidx"], self.n, self.reps[r]["pool"], self.k,
+                                   idx_out=self.idx, count_out=self.cnt, ws=self.ws_pool)
             return
-        self.K.index_topk(self.qidx, self.reps[r]["kidx"], self.n, self.k, idx_out=self.idx, count_out=self.cnt,
+        self.K.index_topk(qidx, self.reps[r]["kidx"], self.n, self.k, idx_out=self.idx, count_out=self.cnt,
                           ws=self.ws_idx)
 
     # the same call in its two steps (dsv4kv_index_score; dsv4kv_index_select);
@@ -533,12 +635,8 @@ def time_e2e(layer, steps):
         with torch.cuda.stream(s_comp):
             wait(s_comp, ev_in[j])
             wait(s_comp, ev_out[j])              # step i-NB's output has left this buffer
-            if layer.kind == "c4a" and layer.pool:
-                layer.K.index_topk_pool(qi_dev[j], layer.reps[i % R]["kidx"], layer.n, layer.reps[i % R]["pool"],
-                                        layer.k, idx_out=layer.idx, count_out=layer.cnt, ws=layer.ws_pool)
-            elif layer.kind == "c4a":
-                layer.K.index_topk(qi_dev[j], layer.reps[i % R]["kidx"], layer.n, layer.k, idx_out=layer.idx,
-                                   count_out=layer.cnt, ws=layer.ws_idx)
+            if layer.kind == "c4a":
+                layer.index(i % R, qidx=qi_dev[j])
             layer.decode(i % R, q=q_dev[j], out=out_dev[j])
             record(ev_comp[j], s_comp)
         with torch.cuda.stream(s_out):
@@ -691,7 +789,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="c4a_b32")
     ap.add_argument("--secondary", default="c128a_b8,c128a_b32,q_c4a_fp8,q_c4a_fp4,q_c128a_fp8,q_c128a_fp4,"
-                                           "q_c4a_fp8rope,q_c128a_fp8rope,c4a_b32_reindex",
+                                           "q_c4a_fp8rope,q_c128a_fp8rope,c4a_b32_reindex,c4a_b32_paged",
                     help="extra per-layer-type workloads (comma list, 'none' = none)")
     ap.add_argument("--no-stack", action="store_true", help="skip the 61-layer stack step")
     ap.add_argument("--no-bulk", action="store_true", help="skip compressor/quantiser throughput")
@@ -706,6 +804,7 @@ def main():
     d = dist_init()
     kind, batch, t, heads, mfmt, ifmt = WORKLOADS[args.workload][:6]
     pool = WORKLOADS[args.workload][6] if len(WORKLOADS[args.workload]) > 6 else 0
+    paged = len(WORKLOADS[args.workload]) > 7 and WORKLOADS[args.workload][7] == "paged"
 
     def wl_desc(kind, batch, t, heads, mfmt, ifmt, pool=0):
         idx = f", {FMT_NAME[ifmt]} indexer" if kind == "c4a" else ""
@@ -737,8 +836,12 @@ def main():
     torch.cuda.set_device(d["local"])
     hbm_peak, tf_peak, peak_src = measured_peaks()
     seed = 1234 + d["rank"]
-    reps = replicas_for(kind, batch, t, mfmt, ifmt, args.replicas, pool, args.l2_factor)
-    layer = Layer(kind, batch, t, heads, seed, reps, mfmt, ifmt, pool=pool)
+    if paged:
+        reps = replicas_for(kind, batch, t // 2, mfmt, ifmt, args.replicas, 0, args.l2_factor)
+        layer = PagedLayer(batch, t, heads, seed, reps)
+    else:
+        reps = replicas_for(kind, batch, t, mfmt, ifmt, args.replicas, pool, args.l2_factor)
+        layer = Layer(kind, batch, t, heads, seed, reps, mfmt, ifmt, pool=pool)
     res = time_layer(layer, args.steps, args.warmup, dist_max, d["local"], sample_clocks=(d["rank"] == 0))
     ms = res["total_ms"] / args.steps
     steps_per_s = d["world"] * 1e3 / ms            # whole job: every rank ran `steps` steps
@@ -752,7 +855,8 @@ def main():
     # launch per dsv4kv_index_score call), the dense decode call for c128a
     if kind == "c4a":
         dom_bytes, dom_ms = layer.index_bytes(), res["score_ms"]
-        dom_name = "index_pool_select" if pool else ("index_score_bf16" if ifmt == 0 else "index_score_fp4")
+        dom_name = ("index_pool_select" if pool else "index_score_paged + index_select" if paged
+                    else "index_score_bf16" if ifmt == 0 else "index_score_fp4")
     else:
         dom_bytes, dom_ms, dom_name = alg, res["decode_ms"], "dsv4kv_dense_decode (decode_kernel + decode_combine)"
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
@@ -772,12 +876,23 @@ def main():
     for name in [s for s in args.secondary.split(",") if s and s not in ("none", args.workload)]:
         spec = WORKLOADS[name]
         pool2 = spec[6] if len(spec) > 6 else 0
-        r2n = replicas_for(spec[0], spec[1], spec[2], spec[4], spec[5], 2, pool2)
-        L2 = Layer(*spec[:4], seed + 99, r2n, spec[4], spec[5], pool=pool2)
+        paged2 = len(spec) > 7 and spec[7] == "paged"
+        if paged2:
+            # every length is >= t/2, so replicas sized at t/2 hold >= 4 x L2
+            r2n = replicas_for(spec[0], spec[1], spec[2] // 2, spec[4], spec[5], 2)
+            L2 = PagedLayer(spec[1], spec[2], spec[3], seed + 99, r2n)
+        else:
+            r2n = replicas_for(spec[0], spec[1], spec[2], spec[4], spec[5], 2, pool2)
+            L2 = Layer(*spec[:4], seed + 99, r2n, spec[4], spec[5], pool=pool2)
         r2 = time_layer(L2, args.steps, args.warmup, dist_max, d["local"], sample_clocks=False)
         ms2 = r2["total_ms"] / args.steps
         a2 = L2.alg_bytes()
-        per_type[name] = {"workload": wl_desc(*spec), "steps_per_s": round(d["world"] * 1e3 / ms2, 1),
+        desc2 = wl_desc(*spec[:7])
+        if paged2:
+            desc2 = (f"c4a layer decode, paged caches ({PAGE_ROWS}-row pages, shuffled), ragged B={spec[1]}: t_b "
+                     f"uniform in [{spec[2] // 2}, {spec[2]}] (mean {L2.t_host.mean():.0f}), H={spec[3]} k=512 "
+                     f"W=128 bf16")
+        per_type[name] = {"workload": desc2, "steps_per_s": round(d["world"] * 1e3 / ms2, 1),
                           "us_per_step": round(ms2 * 1e3, 2), "cache_replicas": r2n,
                           "hbm_gbs": round(a2 / (ms2 * 1e-3) / 1e9, 1),
                           "frac_of_measured_hbm": round(a2 / (ms2 * 1e-3) / 1e9 / hbm_peak, 4),

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libdsv4kv.so")
 
 BF16, FP8_E4M3_ROW, FP4_E2M1_G16, FP8_E4M3_ROW_ROPE_BF16 = 0, 1, 2, 3
 DEV_BAD_INDEX, DEV_TIMEOUT, DEV_INCONSISTENT, DEV_BAD_POOL = 0x1, 0x2, 0x4, 0x8
+DEV_BAD_PAGE, DEV_BAD_LENGTH = 0x10, 0x20
 STATUS_NAMES = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED", 3: "ERR_WORKSPACE", 4: "ERR_CUDA"}
 
 
@@ -30,6 +31,12 @@ class Dsv4kvError(RuntimeError):
 
 class CacheDesc(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("dim", ctypes.c_int32), ("rows", ctypes.c_int64),
+                ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+class PagedDesc(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("dim", ctypes.c_int32), ("page_rows", ctypes.c_int32),
+                ("table_stride", ctypes.c_int32), ("pool_pages", ctypes.c_int64), ("table", ctypes.c_void_p),
                 ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
 
 
@@ -69,6 +76,24 @@ _SIGS = {
                                         _c.c_int32, _c.c_int32, _c.c_int64, _c.c_int32, _c.c_int32, _c.c_int64,
                                         _c.c_float, _c.c_int32, _c.c_double, _c.c_int32, _c.c_void_p,
                                         _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "dsv4kv_index_topk_paged_workspace_bytes": (_c.c_size_t, [_c.c_int32, _c.c_int64, _c.c_int32, _c.c_int32,
+                                                              _c.c_int32]),
+    "dsv4kv_index_topk_paged": (_c.c_int, [_c.c_void_p, _c.POINTER(PagedDesc), _c.c_int32, _c.c_void_p, _c.c_int64,
+                                           _c.c_int32, _c.c_int32, _c.c_int32, _c.c_void_p, _c.c_void_p,
+                                           _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "dsv4kv_sparse_decode_paged_workspace_bytes": (_c.c_size_t, [_c.c_int32, _c.c_int32, _c.c_int32, _c.c_int32,
+                                                                 _c.c_int32]),
+    "dsv4kv_sparse_decode_paged": (_c.c_int, [_c.c_void_p, _c.POINTER(PagedDesc), _c.POINTER(PagedDesc),
+                                              _c.c_void_p, _c.c_int32, _c.c_int32, _c.c_void_p, _c.c_int64,
+                                              _c.c_int32, _c.c_int32, _c.c_int32, _c.c_float, _c.c_int32,
+                                              _c.c_double, _c.c_int32, _c.c_void_p, _c.c_void_p, _c.c_size_t,
+                                              _c.c_void_p]),
+    "dsv4kv_dense_decode_paged_workspace_bytes": (_c.c_size_t, [_c.c_int32, _c.c_int32, _c.c_int32, _c.c_int64,
+                                                                _c.c_int32, _c.c_int32]),
+    "dsv4kv_dense_decode_paged": (_c.c_int, [_c.c_void_p, _c.POINTER(PagedDesc), _c.POINTER(PagedDesc), _c.c_int32,
+                                             _c.c_int32, _c.c_void_p, _c.c_int64, _c.c_int32, _c.c_int32,
+                                             _c.c_float, _c.c_int32, _c.c_double, _c.c_int32, _c.c_void_p,
+                                             _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "dsv4kv_dense_decode_workspace_bytes": (_c.c_size_t, [_c.c_int32, _c.c_int32, _c.c_int32, _c.c_int64,
                                                           _c.c_int32]),
     "dsv4kv_dense_decode": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.POINTER(CacheDesc), _c.c_int32,
@@ -122,6 +147,26 @@ class Cache:
 
     def desc(self) -> CacheDesc:
         return CacheDesc(self.fmt, self.dim, self.rows, _ptr(self.codes), _ptr(self.scales))
+
+
+@dataclass
+class PagedCache:
+    """A paged cache: rows of every sequence in pages of `page_rows` rows of one shared pool.
+    Row i of sequence b is pool row table[b][i // page_rows] * page_rows + i % page_rows."""
+    fmt: int
+    codes: torch.Tensor                      # pool rows: [pool_pages * page_rows][row bytes or channels]
+    table: torch.Tensor                      # int32 [B][table_stride] page numbers
+    page_rows: int
+    scales: Optional[torch.Tensor] = None    # pool scales per row (fp8: f32 [rows], fp4: u8 [rows][dim/16])
+    dim: int = 512
+
+    @property
+    def pool_pages(self) -> int:
+        return int(self.codes.shape[0]) // self.page_rows
+
+    def desc(self) -> PagedDesc:
+        return PagedDesc(self.fmt, self.dim, self.page_rows, int(self.table.shape[1]), self.pool_pages,
+                         _ptr(self.table), _ptr(self.codes), _ptr(self.scales))
 
 
 def new_workspace(nbytes: int, device=None) -> torch.Tensor:
@@ -308,4 +353,67 @@ def dense_decode(q: torch.Tensor, comp: Cache, win: Cache, n: int, window: int, 
     _check(lib().dsv4kv_dense_decode(_ptr(q), ctypes.byref(cd), ctypes.byref(wd), b, h, n, window, t, sm_scale,
                                      rope_dim, rope_base, int(out_fp32), _ptr(out), _ptr(ws), ws.numel(),
                                      _stream(stream)), "dsv4kv_dense_decode")
+    return out
+
+
+def index_topk_paged(qidx: torch.Tensor, keys: PagedCache, t_seq: torch.Tensor, t_max: int, k: int,
+                     window: int = 128, stride: int = 4, idx_out: Optional[torch.Tensor] = None,
+                     count_out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                     stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Ragged, paged top-k: t_seq int64 [B] (device) query positions, sequence b has
+    max(0, (t_b - window) // stride) keys -> (idx int32 [B][k] ascending, -1 padded; count int32 [B])."""
+    b = int(qidx.shape[0])
+    dev = qidx.device
+    if idx_out is None:
+        idx_out = torch.empty((b, k), dtype=torch.int32, device=dev)
+    if count_out is None:
+        count_out = torch.empty((b,), dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = new_workspace(int(lib().dsv4kv_index_topk_paged_workspace_bytes(b, t_max, window, stride, k)), dev)
+    d = keys.desc()
+    _check(lib().dsv4kv_index_topk_paged(_ptr(qidx), ctypes.byref(d), b, _ptr(t_seq), t_max, window, stride, k,
+                                         _ptr(idx_out), _ptr(count_out), _ptr(ws), ws.numel(), _stream(stream)),
+           "dsv4kv_index_topk_paged")
+    return idx_out, count_out
+
+
+def sparse_decode_paged(q: torch.Tensor, comp: PagedCache, win: PagedCache, idx: torch.Tensor, t_seq: torch.Tensor,
+                        t_max: int, window: int = 128, stride: int = 4, sm_scale: Optional[float] = None,
+                        rope_dim: int = 64, rope_base: float = 10000.0, out_fp32: bool = False,
+                        out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                        stream=None) -> torch.Tensor:
+    """Ragged, paged c4a decode: q bf16 [B][H][512], idx int32 [B][k] from index_topk_paged."""
+    b, h, d = q.shape
+    k = int(idx.shape[1])
+    if sm_scale is None:
+        sm_scale = d ** -0.5
+    if out is None:
+        out = torch.empty((b, h, d), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=q.device)
+    if ws is None:
+        ws = new_workspace(int(lib().dsv4kv_sparse_decode_paged_workspace_bytes(b, h, d, k, window)), q.device)
+    cd, wd = comp.desc(), win.desc()
+    _check(lib().dsv4kv_sparse_decode_paged(_ptr(q), ctypes.byref(cd), ctypes.byref(wd), _ptr(idx), b, h, _ptr(t_seq),
+                                            t_max, window, stride, k, sm_scale, rope_dim, rope_base, int(out_fp32),
+                                            _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+           "dsv4kv_sparse_decode_paged")
+    return out
+
+
+def dense_decode_paged(q: torch.Tensor, comp: PagedCache, win: PagedCache, t_seq: torch.Tensor, t_max: int,
+                       window: int = 128, stride: int = 128, sm_scale: Optional[float] = None, rope_dim: int = 64,
+                       rope_base: float = 10000.0, out_fp32: bool = False, out: Optional[torch.Tensor] = None,
+                       ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Ragged, paged c128a decode over every sequence's n_b entries plus its window rows."""
+    b, h, d = q.shape
+    if sm_scale is None:
+        sm_scale = d ** -0.5
+    if out is None:
+        out = torch.empty((b, h, d), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=q.device)
+    if ws is None:
+        ws = new_workspace(int(lib().dsv4kv_dense_decode_paged_workspace_bytes(b, h, d, t_max, window, stride)),
+                           q.device)
+    cd, wd = comp.desc(), win.desc()
+    _check(lib().dsv4kv_dense_decode_paged(_ptr(q), ctypes.byref(cd), ctypes.byref(wd), b, h, _ptr(t_seq), t_max,
+                                           window, stride, sm_scale, rope_dim, rope_base, int(out_fp32), _ptr(out),
+                                           _ptr(ws), ws.numel(), _stream(stream)), "dsv4kv_dense_decode_paged")
     return out

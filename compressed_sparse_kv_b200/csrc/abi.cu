@@ -297,6 +297,152 @@ DSV4KV_API dsv4kv_status dsv4kv_sparse_decode(const void* q, const dsv4kv_cache*
   return decode_launch(a, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
+// ------------------------------------------------------------------ paged, ragged
+// Checks a paged cache whose sequences have at most `max_rows` rows and
+// turns it into the kernels' form (a pool "cache" of pool rows + its pages).
+static dsv4kv_status check_paged(const dsv4kv_paged_cache* c, const char* what, int64_t max_rows, int dim,
+                                 bool keys, dsv4kv_cache* pool, PageDesc* pg) {
+  if (!c) return set_error(DSV4KV_ERR_INVALID_ARG, "%s: paged cache descriptor is null", what);
+  if (c->dim != dim) return set_error(DSV4KV_ERR_UNSUPPORTED, "%s: dim %d, expected %d", what, c->dim, dim);
+  if (keys ? (c->fmt != DSV4KV_BF16 && c->fmt != DSV4KV_FP4_E2M1_G16)
+           : (c->fmt < DSV4KV_BF16 || c->fmt > DSV4KV_FP8_E4M3_ROW_ROPE_BF16))
+    return set_error(DSV4KV_ERR_UNSUPPORTED, "%s: format %d", what, c->fmt);
+  if (c->page_rows <= 0 || c->page_rows % 64 != 0)
+    return set_error(DSV4KV_ERR_INVALID_ARG, "%s: page_rows must be a positive multiple of 64", what);
+  if (c->pool_pages < 1 || c->pool_pages * int64_t(c->page_rows) >= (int64_t(1) << 31))
+    return set_error(DSV4KV_ERR_UNSUPPORTED, "%s: the pool must hold between 1 page and 2^31 rows", what);
+  const int64_t need_pages = (max_rows + c->page_rows - 1) / c->page_rows;
+  if (c->table_stride < need_pages)
+    return set_error(DSV4KV_ERR_INVALID_ARG, "%s: table_stride %d < %lld pages a sequence may need", what,
+                     c->table_stride, (long long)need_pages);
+  if (max_rows > 0 && !c->table) return set_error(DSV4KV_ERR_INVALID_ARG, "%s: block table is null", what);
+  dsv4kv_cache d{c->fmt, c->dim, c->pool_pages * int64_t(c->page_rows), c->codes, c->scales};
+  dsv4kv_status st = check_cache(&d, what, max_rows > 0 ? 1 : 0, dim);
+  if (st != DSV4KV_OK) return st;
+  *pool = d;
+  *pg = PageDesc{c->table, c->page_rows, c->table_stride, c->pool_pages};
+  return DSV4KV_OK;
+}
+
+static dsv4kv_status check_ragged(const char* what, int32_t batch, const int64_t* t_seq, int64_t t_max,
+                                  int32_t window, int32_t stride) {
+  if (batch < 1) return set_error(DSV4KV_ERR_INVALID_ARG, "%s: batch must be >= 1", what);
+  if (!t_seq) return set_error(DSV4KV_ERR_INVALID_ARG, "%s: t_seq is null", what);
+  if (t_max < 0 || window < 0 || stride < 1) return set_error(DSV4KV_ERR_INVALID_ARG, "%s: bad sizes", what);
+  if (t_max >= (int64_t(1) << 40)) return set_error(DSV4KV_ERR_UNSUPPORTED, "%s: t_max too large", what);
+  return DSV4KV_OK;
+}
+
+DSV4KV_API size_t dsv4kv_index_topk_paged_workspace_bytes(int32_t batch, int64_t t_max, int32_t window, int32_t stride,
+                                                          int32_t k) {
+  if (batch < 0 || t_max < 0 || window < 0 || stride < 1 || k < 1) return 0;
+  return index_topk_ws_bytes(batch, dsv4kv_compress_entries(t_max, window, stride), k);
+}
+
+DSV4KV_API dsv4kv_status dsv4kv_index_topk_paged(const void* qidx, const dsv4kv_paged_cache* keys, int32_t batch,
+                                                 const int64_t* t_seq, int64_t t_max, int32_t window, int32_t stride,
+                                                 int32_t k, int32_t* idx_out, int32_t* count_out, void* ws,
+                                                 size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  const char* what = "index_topk_paged";
+  dsv4kv_status st = check_ragged(what, batch, t_seq, t_max, window, stride);
+  if (st != DSV4KV_OK) return st;
+  if (k < 1 || k > 2048) return set_error(DSV4KV_ERR_UNSUPPORTED, "%s: k must be in [1, 2048]", what);
+  if (!idx_out) return set_error(DSV4KV_ERR_INVALID_ARG, "%s: idx_out is null", what);
+  const int64_t n_max = dsv4kv_compress_entries(t_max, window, stride);
+  dsv4kv_cache pool{};
+  PageDesc pg{};
+  st = check_paged(keys, what, n_max, 128, true, &pool, &pg);
+  if (st != DSV4KV_OK) return st;
+  if (n_max > k) {
+    if (!qidx || !aligned16(qidx)) return set_error(DSV4KV_ERR_INVALID_ARG, "%s: qidx null or misaligned", what);
+    if (int64_t(batch) * n_max > (int64_t(1) << 40)) return set_error(DSV4KV_ERR_UNSUPPORTED, "%s: too large", what);
+  }
+  if (!ws || ws_bytes < dsv4kv_index_topk_paged_workspace_bytes(batch, t_max, window, stride, k))
+    return set_error(DSV4KV_ERR_WORKSPACE, "%s: workspace null or too small", what);
+  Ragged rg;
+  rg.t_seq = t_seq;
+  rg.t_max = t_max;
+  rg.window = window;
+  rg.stride = stride;
+  return index_topk_paged_launch(static_cast<const uint16_t*>(qidx), pool, pg, batch, rg, k, idx_out, count_out, ws,
+                                 ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+DSV4KV_API size_t dsv4kv_sparse_decode_paged_workspace_bytes(int32_t batch, int32_t heads, int32_t dim, int32_t k,
+                                                             int32_t window) {
+  return dsv4kv_sparse_decode_workspace_bytes(batch, heads, dim, k, window);
+}
+
+DSV4KV_API size_t dsv4kv_dense_decode_paged_workspace_bytes(int32_t batch, int32_t heads, int32_t dim, int64_t t_max,
+                                                            int32_t window, int32_t stride) {
+  if (stride < 1 || t_max < 0) return 0;
+  return dsv4kv_dense_decode_workspace_bytes(batch, heads, dim, dsv4kv_compress_entries(t_max, window, stride),
+                                             window);
+}
+
+static dsv4kv_status decode_paged(const char* what, const void* q, const dsv4kv_paged_cache* comp,
+                                  const dsv4kv_paged_cache* win, const int32_t* idx, int32_t batch, int32_t heads,
+                                  const int64_t* t_seq, int64_t t_max, int32_t window, int32_t stride, int32_t k,
+                                  float sm_scale, int32_t rope_dim, double rope_base, int32_t out_fp32, void* out,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  dsv4kv_status st = check_ragged(what, batch, t_seq, t_max, window, stride);
+  if (st != DSV4KV_OK) return st;
+  if (heads < 1 || heads > 64) return set_error(DSV4KV_ERR_UNSUPPORTED, "%s: heads must be in [1, 64]", what);
+  if (!q || !aligned16(q) || !out || !aligned16(out))
+    return set_error(DSV4KV_ERR_INVALID_ARG, "%s: q/out null or misaligned", what);
+  if (rope_dim < 0 || rope_dim > 512 || (rope_dim & 1)) return set_error(DSV4KV_ERR_INVALID_ARG, "%s: bad rope_dim", what);
+  const int64_t n_max = dsv4kv_compress_entries(t_max, window, stride);
+  const int32_t w_max = int32_t(std::min<int64_t>(t_max, window));
+  if (n_max > (int64_t(1) << 30)) return set_error(DSV4KV_ERR_UNSUPPORTED, "%s: too many entries", what);
+  dsv4kv_cache cpool{}, wpool{};
+  PageDesc cpg{}, wpg{};
+  st = check_paged(comp, what, n_max, 512, false, &cpool, &cpg);
+  if (st != DSV4KV_OK) return st;
+  st = check_paged(win, what, w_max, 512, false, &wpool, &wpg);
+  if (st != DSV4KV_OK) return st;
+  if (win->fmt != comp->fmt)
+    return set_error(DSV4KV_ERR_UNSUPPORTED, "%s: the window cache must have the compressed cache's format", what);
+  if (idx) {
+    if (k < 0 || k > 2048) return set_error(DSV4KV_ERR_UNSUPPORTED, "%s: k must be in [0, 2048]", what);
+    if (!ws || ws_bytes < dsv4kv_sparse_decode_workspace_bytes(batch, heads, 512, k, window))
+      return set_error(DSV4KV_ERR_WORKSPACE, "%s: workspace null or too small", what);
+  } else if (!ws || ws_bytes < dsv4kv_dense_decode_workspace_bytes(batch, heads, 512, n_max, window)) {
+    return set_error(DSV4KV_ERR_WORKSPACE, "%s: workspace null or too small", what);
+  }
+  DecodeArgs a{q, cpool, wpool, idx, batch, heads, 512, n_max, window, idx ? k : 0, t_max, sm_scale, rope_dim,
+               rope_base, out_fp32, out};
+  a.t_seq = t_seq;
+  a.t_max = t_max;
+  a.stride = stride;
+  a.comp_pg = cpg;
+  a.win_pg = wpg;
+  return decode_launch(a, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+DSV4KV_API dsv4kv_status dsv4kv_sparse_decode_paged(const void* q, const dsv4kv_paged_cache* comp,
+                                                    const dsv4kv_paged_cache* win, const int32_t* idx, int32_t batch,
+                                                    int32_t heads, const int64_t* t_seq, int64_t t_max, int32_t window,
+                                                    int32_t stride, int32_t k, float sm_scale, int32_t rope_dim,
+                                                    double rope_base, int32_t out_fp32, void* out, void* ws,
+                                                    size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  if (!idx) return set_error(DSV4KV_ERR_INVALID_ARG, "sparse_decode_paged: idx is null");
+  return decode_paged("sparse_decode_paged", q, comp, win, idx, batch, heads, t_seq, t_max, window, stride, k,
+                      sm_scale, rope_dim, rope_base, out_fp32, out, ws, ws_bytes, stream);
+}
+
+DSV4KV_API dsv4kv_status dsv4kv_dense_decode_paged(const void* q, const dsv4kv_paged_cache* comp,
+                                                   const dsv4kv_paged_cache* win, int32_t batch, int32_t heads,
+                                                   const int64_t* t_seq, int64_t t_max, int32_t window, int32_t stride,
+                                                   float sm_scale, int32_t rope_dim, double rope_base,
+                                                   int32_t out_fp32, void* out, void* ws, size_t ws_bytes,
+                                                   void* stream) {
+  g_err[0] = 0;
+  return decode_paged("dense_decode_paged", q, comp, win, nullptr, batch, heads, t_seq, t_max, window, stride, 0,
+                      sm_scale, rope_dim, rope_base, out_fp32, out, ws, ws_bytes, stream);
+}
+
 DSV4KV_API dsv4kv_status dsv4kv_dense_decode(const void* q, const dsv4kv_cache* comp, const dsv4kv_cache* win,
                                              int32_t batch, int32_t heads, int64_t n, int32_t window, int64_t t,
                                              float sm_scale, int32_t rope_dim, double rope_base, int32_t out_fp32,

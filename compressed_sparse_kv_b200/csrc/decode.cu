@@ -89,13 +89,26 @@ struct __align__(8) Ctl {
 constexpr size_t kSmemBytes = 1024 + kQBytes + kStages * kTileBytes + 2 * kPBytes + sizeof(Ctl);
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
+// Where the rows of one cache live: a dense [B][rows] layout (table null:
+// row i of sequence b is row b * rows + i) or pages of a shared pool (row i
+// of sequence b is pool row table[b * tstride + i / page] * page + i % page).
+struct RowMap {
+  const int32_t* table;
+  int page, tstride;
+  int64_t rows;   // dense: rows per sequence; paged: rows in the pool
+  int64_t pages;  // paged: pages in the pool
+};
+
 struct Params {
   int heads;
-  int64_t n;
-  int window;
+  int64_t n;    // compressed entries (uniform batch) or the most any sequence has (ragged)
+  int window;   // window rows (uniform) or the window length W (ragged)
   int k;
-  int comp_tiles, tiles, splits, tiles_per_split;
-  int64_t comp_rows, win_rows;  // per-sequence row capacity of each cache
+  int splits;
+  const int64_t* t_seq;  // ragged batch: query position of every sequence; null = uniform
+  int64_t t_max;
+  int stride;
+  RowMap comp_map, win_map;
   const int32_t* idx;           // [B][k] or null (dense)
   const uint8_t* comp_codes;
   const void* comp_scales;
@@ -104,7 +117,7 @@ struct Params {
   float score_scale;  // sm_scale * log2(e)
   float* o_part;      // [B][splits][H][512]
   float* ml_part;     // [B][splits][H][4]: (m_o, m_l, l, 0)
-  float* rope_tab;    // [2][256]: the rotation table for decode_combine (written by CTA 0)
+  float* rope_tab;    // [B][2][256]: the rotation tables for decode_combine (written by split 0)
   uint32_t* status;
   // direct output when splits == 1
   int64_t t;
@@ -158,56 +171,107 @@ __device__ __forceinline__ bool named_bar_or(bool pred) {
 __device__ __forceinline__ void named_bar_sync() { asm volatile("barrier.cta.sync 1, 128;" ::: "memory"); }
 __device__ __forceinline__ void loader_bar_sync() { asm volatile("barrier.cta.sync 2, 128;" ::: "memory"); }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
-// Whether tile T is a run of contiguous rows (TMA tile) rather than a gather.
-__device__ __forceinline__ bool tile_contiguous(const Params& p, int T) {
-  return T >= p.comp_tiles || p.idx == nullptr;
+// The extent of one sequence and the tiles of one CTA.  Tiles 0 ..
+// comp_tiles-1 hold the sequence's compressed rows (selected slots or all
+// entries, 64 per tile), the rest its window rows.
+struct Seq {
+  int64_t t, n;  // query position, compressed entries
+  int w;         // window rows
+  int comp_tiles, tiles, t0, nt;
+};
+
+__device__ __forceinline__ Seq seq_info(const Params& p, int b, int split) {
+  Seq q;
+  if (p.t_seq) {
+    int64_t t = p.t_seq[b];
+    if (t < 0 || t > p.t_max) {
+      set_status(p.status, DSV4KV_DEV_BAD_LENGTH);
+      t = t < 0 ? 0 : p.t_max;
+    }
+    q.t = t;
+    q.n = t > p.window ? min(p.n, (t - p.window) / p.stride) : 0;
+    q.w = int(t < int64_t(p.window) ? t : int64_t(p.window));
+  } else {
+    q.t = p.t;
+    q.n = p.n;
+    q.w = p.window;
+  }
+  const int64_t slots = p.idx ? (int64_t(p.k) < q.n ? int64_t(p.k) : q.n) : q.n;
+  q.comp_tiles = int((slots + kTileRows - 1) / kTileRows);
+  q.tiles = q.comp_tiles + (q.w + kTileRows - 1) / kTileRows;
+  const int per = (q.tiles + p.splits - 1) / p.splits;
+  q.t0 = split * per;
+  q.nt = max(0, min(q.tiles, q.t0 + per) - q.t0);
+  return q;
 }
 
-// Source of row `r` of tile T: global row (b * rows + i) of the compressed
-// cache (from_win = false) or of the window cache; valid = false for padding
-// slots and rejected indices (the row then reads row 0 of the sequence, which
-// is finite, and is masked in the softmax).
+// Global row of logical row i of sequence b; ok = false (and row 0) when its
+// page number is outside the pool.
+__device__ __forceinline__ int64_t map_row(const RowMap& m, int b, int64_t i, bool& ok, uint32_t* status) {
+  if (!m.table) return int64_t(b) * m.rows + i;
+  const int32_t pg = __ldg(m.table + size_t(b) * m.tstride + size_t(i / m.page));
+  if (pg < 0 || pg >= m.pages) {
+    set_status(status, DSV4KV_DEV_BAD_PAGE);
+    ok = false;
+    return 0;
+  }
+  return int64_t(pg) * m.page + i % m.page;
+}
+
+// Rows of tile T that exist: the first n - 64T compressed rows (dense) or
+// w - 64(T - comp_tiles) window rows.
+__device__ __forceinline__ int64_t tile_rows(const Seq& q, int T) {
+  return T < q.comp_tiles ? q.n - int64_t(T) * kTileRows : int64_t(q.w) - int64_t(T - q.comp_tiles) * kTileRows;
+}
+
+// Whether tile T is loaded by TMA: 64 rows that exist and lie consecutively
+// in memory (dense compressed rows or window rows; a page holds whole tiles,
+// and its page number is in the pool).  Partial tiles, tiles of bad pages and
+// gathered (selected) rows go through the loader warps, which zero-fill what
+// does not exist, so no row past a sequence's end is read.
+__device__ __forceinline__ bool tile_tma(const Params& p, const Seq& q, int b, int T) {
+  if (!((T >= q.comp_tiles || p.idx == nullptr) && tile_rows(q, T) >= kTileRows)) return false;
+  const bool win = T >= q.comp_tiles;
+  const RowMap& m = win ? p.win_map : p.comp_map;
+  if (!m.table) return true;
+  const int64_t i0 = int64_t(win ? T - q.comp_tiles : T) * kTileRows;
+  const int32_t pg = __ldg(m.table + size_t(b) * m.tstride + size_t(i0 / m.page));
+  return pg >= 0 && pg < m.pages;
+}
+
+// Source of row `r` of tile T: global row of the compressed cache (from_win =
+// false) or of the window cache; valid = false for padding slots, rejected
+// indices and rows of bad pages (such rows are zero-filled and masked).
 struct RowSrc {
   int64_t row;
   bool valid, from_win;
 };
-__device__ __forceinline__ RowSrc row_source(const Params& p, int b, int T, int r, const int32_t* idx_s = nullptr,
-                                             int slot0 = 0) {
+__device__ __forceinline__ RowSrc row_source(const Params& p, const Seq& q, int b, int T, int r,
+                                             const int32_t* idx_s = nullptr, int slot0 = 0) {
   RowSrc s{0, false, false};
-  if (T < p.comp_tiles) {
+  if (T < q.comp_tiles) {
     const int slot = T * kTileRows + r;
     int64_t i = -1;
     if (p.idx) {
       const int32_t v = slot >= p.k ? -1 : (idx_s ? idx_s[slot - slot0] : p.idx[size_t(b) * p.k + slot]);
-      if (v >= p.n) set_status(p.status, DSV4KV_DEV_BAD_INDEX);
+      if (v >= q.n) set_status(p.status, DSV4KV_DEV_BAD_INDEX);
       i = v;
-    } else if (slot < p.n) {
+    } else if (slot < q.n) {
       i = slot;
     }
-    s.valid = i >= 0 && i < p.n;
-    s.row = int64_t(b) * p.comp_rows + (s.valid ? i : 0);
+    s.valid = i >= 0 && i < q.n;
+    if (s.valid) s.row = map_row(p.comp_map, b, i, s.valid, p.status);
   } else {
-    const int wr = (T - p.comp_tiles) * kTileRows + r;
+    const int wr = (T - q.comp_tiles) * kTileRows + r;
     s.from_win = true;
-    s.valid = wr < p.window;
-    s.row = int64_t(b) * p.win_rows + (s.valid ? wr : 0);
+    s.valid = wr < q.w;
+    if (s.valid) s.row = map_row(p.win_map, b, wr, s.valid, p.status);
   }
   return s;
-}
-
-// Row validity of a contiguous tile: the first n - 64T compressed rows, or
-// the first window - 64(T - comp_tiles) window rows.
-__device__ __forceinline__ uint64_t contiguous_mask(const Params& p, int T) {
-  const int64_t lim = T < p.comp_tiles ? p.n - int64_t(T) * kTileRows
-                                       : int64_t(p.window) - int64_t(T - p.comp_tiles) * kTileRows;
-  return lim >= kTileRows ? ~0ull : (lim <= 0 ? 0ull : ((1ull << lim) - 1ull));
 }
 
 // cos / sin of the inverse-RoPE angle -t * rope_base^(-2m/rope_dim): the
@@ -284,8 +348,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x / p.splits, split = blockIdx.x % p.splits;
-  const int t0 = split * p.tiles_per_split;
-  const int nt = max(0, min(p.tiles, t0 + p.tiles_per_split) - t0);
   pdl_trigger();
 
   if (threadIdx.x == 0) {
@@ -321,6 +383,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
   pdl_wait();  // everything above touched only shared memory, TMEM and the tensor maps
+  const Seq sq = seq_info(p, b, split);  // (the lengths of a ragged batch may come from the previous kernel)
+  const int t0 = sq.t0, nt = sq.nt;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA: Q and contiguous tiles
@@ -331,11 +395,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < nt; ++i) {
         const int T = t0 + i, stage = i % kStages;
         if (i >= kStages && !wait_or_abort(&ctl->empty[stage], ((i / kStages) - 1) & 1, ctl)) break;
-        if (!C::kQuant && tile_contiguous(p, T)) {
-          const RowSrc s0 = row_source(p, b, T, 0);  // first row of the run
+        if (!C::kQuant && tile_tma(p, sq, b, T)) {
+          const RowSrc s0 = row_source(p, sq, b, T, 0);  // first row of the run
           const CUtensorMap* tm = s0.from_win ? &tm_win : &tm_comp;
-          const int32_t row0 = int32_t(s0.from_win ? int64_t(b) * p.win_rows + (T - p.comp_tiles) * kTileRows
-                                                   : int64_t(b) * p.comp_rows + int64_t(T) * kTileRows);
+          const int32_t row0 = int32_t(s0.row);
           mbar_arrive_expect_tx(&ctl->full[stage], kTileBytes);
           uint8_t* dst = sR + stage * kTileBytes;
           for (int c = 0; c < kChunks; ++c) tma_load_2d(dst + c * kChunkBytes, tm, &ctl->full[stage], c * 64, row0);
@@ -427,19 +490,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the inverse-RoPE table, while the first tile is still in flight
     for (int m = threadIdx.x - 64; m < p.rope_dim / 2; m += 128) {
       float cs, sn;
-      inv_rope_rotation(p.t, m, p.rope_dim, p.rope_base, &cs, &sn);
+      inv_rope_rotation(sq.t, m, p.rope_dim, p.rope_base, &cs, &sn);
       ctl->rope_cs[m] = cs;
       ctl->rope_sn[m] = sn;
-      if (p.splits > 1 && blockIdx.x == 0) {
-        p.rope_tab[m] = cs;
-        p.rope_tab[kDim / 2 + m] = sn;
+      if (p.splits > 1 && split == 0) {
+        p.rope_tab[size_t(b) * kDim + m] = cs;
+        p.rope_tab[size_t(b) * kDim + kDim / 2 + m] = sn;
       }
     }
     float m_o[2] = {-INFINITY, -INFINITY}, m_l[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
     bool dead = false;
     for (int i = 0; i < nt; ++i) {
       const int T = t0 + i, sb = i & 1, stage = i % kStages;
-      const bool gathered = C::kQuant || !tile_contiguous(p, T);
+      const bool gathered = C::kQuant || !tile_tma(p, sq, b, T);
       if (!dead) dead = !warp_wait(&ctl->s_full[sb], (i >> 1) & 1, ctl, lane);
       // the loaders' row mask and row scales (complete: the MMA already consumed this tile)
       if ((gathered || C::kRowScale) && !dead) dead = !warp_wait(&ctl->full[stage], (i / kStages) & 1, ctl, lane);
@@ -455,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&ctl->s_free[sb]);
         const uint64_t vm = gathered ? (uint64_t(ctl->vmask[stage][0]) | (uint64_t(ctl->vmask[stage][1]) << 16) |
                                         (uint64_t(ctl->vmask[stage][2]) << 32) | (uint64_t(ctl->vmask[stage][3]) << 48))
-                                     : contiguous_mask(p, T);
+                                     : ~0ull;  // a TMA tile: 64 rows that exist
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
 #pragma unroll
@@ -611,7 +674,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const int hh = 32 * half + e;
-              float v = __uint_as_float(o[e]) * ctl->fin[hh];
+              // (fin == 0: no rows, or a wait gave up; the accumulator was never written)
+              float v = ctl->fin[hh] != 0.f ? __uint_as_float(o[e]) * ctl->fin[hh] : 0.f;
               const float partner = __shfl_xor_sync(kFull, v, 1);  // channel c ^ 1 of the same head
               if (rot) v = (c & 1) ? partner * sn + v * cs : v * cs - partner * sn;
               if (hh < p.heads) {
@@ -651,26 +715,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int T = t0 + i, stage = i % kStages;
       if (i >= kStages && !warp_wait(&ctl->empty[stage], ((i / kStages) - 1) & 1, ctl, lane)) break;
       uint8_t* tile = sR + stage * kTileBytes;
-      if (!C::kQuant && tile_contiguous(p, T)) {
+      if (!C::kQuant && tile_tma(p, sq, b, T)) {
         // warp 0 brings this tile by TMA
       } else {
         // lane j < 16 resolves row 16*lw + j; every lane reads all 16 answers
-        const RowSrc mine = row_source(p, b, T, 16 * lw + (lane & 15), ctl->idx_s, slot0);
+        const RowSrc mine = row_source(p, sq, b, T, 16 * lw + (lane & 15), ctl->idx_s, slot0);
         const uint32_t vb = __ballot_sync(kFull, mine.valid) & 0xffffu;
         if (lane == 0) ctl->vmask[stage][lw] = vb;
         if (!C::kQuant) {
           // gathered bf16 rows: 16-byte cp.async into the 128-byte-swizzled tile
+          // (rows that do not exist are zero-filled without a read)
           const uint8_t* base = static_cast<const uint8_t*>(mine.from_win ? p.win_codes : p.comp_codes);
 #pragma unroll 4
           for (int j = 0; j < 16; ++j) {
             const int r = 16 * lw + j;
             const int64_t row = __shfl_sync(kFull, mine.row, j);
+            const uint32_t bytes = (vb >> j) & 1u ? 16u : 0u;
             const uint8_t* src = base + size_t(row) * (kDim * 2);
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
               const int u_all = 32 * hh + lane;  // 16-byte unit of the 1 KB row
               const int c = u_all >> 3, u = u_all & 7;
-              cp_async16(tile + c * kChunkBytes + r * 128 + ((u ^ (r & 7)) << 4), src + 16 * u_all);
+              cp_async16_zfill(tile + c * kChunkBytes + r * 128 + ((u ^ (r & 7)) << 4), src + 16 * u_all, bytes);
             }
           }
           cp_async_wait_all();
@@ -825,6 +891,7 @@ __global__ void __launch_bounds__(32 * kCombWarps) decode_combine(const float* _
   const size_t ml_stride = size_t(heads) * 4, o_stride = size_t(heads) * kDim;
   const float* mlb = ml_part + (size_t(b) * splits * heads + h) * 4;
   const float* ob = o_part + (size_t(b) * splits * heads + h) * kDim + 4 * lane;
+  rope_tab += size_t(b) * kDim;  // this sequence's rotation
   // the rotation of this lane's rotary pairs (channels 128q + 4 lane + {0, 2}), read up front
   const int r0 = kDim - rope_dim;
   float cs[4][2], sn[4][2];
@@ -1047,7 +1114,8 @@ __global__ void __launch_bounds__(32 * kWideWarps, CB == 1 ? 4 : 2) decode_combi
   const int r0 = kDim - rope_dim;
   if (c >= r0) {
     const int m = (c - r0) >> 1;
-    const float cs = __ldcg(rope_tab + m), sn = __ldcg(rope_tab + kDim / 2 + m);
+    const float* rt = rope_tab + size_t(b) * kDim;  // this sequence's rotation
+    const float cs = __ldcg(rt + m), sn = __ldcg(rt + kDim / 2 + m);
     const float x = v0, y = v1;
     v0 = x * cs - y * sn;
     v1 = x * sn + y * cs;
@@ -1093,7 +1161,7 @@ DecodeWs decode_ws_layout(char* base, int batch, int heads, const Plan& pl) {
   w.status = reinterpret_cast<uint32_t*>(take(16));
   w.o_part = reinterpret_cast<float*>(take(sizeof(float) * size_t(batch) * pl.splits * heads * kDim));
   w.ml_part = reinterpret_cast<float*>(take(sizeof(float) * size_t(batch) * pl.splits * heads * 4));
-  w.rope_tab = reinterpret_cast<float*>(take(sizeof(float) * kDim));
+  w.rope_tab = reinterpret_cast<float*>(take(sizeof(float) * size_t(batch) * kDim));
   w.bytes = off;
   return w;
 }
@@ -1133,8 +1201,8 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
     return set_error(DSV4KV_ERR_UNSUPPORTED, "decode: unknown cache format %d", fmt);
   if (fmt == DSV4KV_FP8_E4M3_ROW_ROPE_BF16 && a.rope_dim != 64)
     return set_error(DSV4KV_ERR_UNSUPPORTED, "decode: fp8 rows with bf16 rotary channels need rope_dim == 64");
-  const int slots = a.idx ? a.k : int(a.n);
-  const int comp_tiles = (a.n > 0 && slots > 0) ? (slots + kTileRows - 1) / kTileRows : 0;
+  const int64_t slots = a.idx ? std::min<int64_t>(a.k, a.n) : a.n;
+  const int comp_tiles = int((slots + kTileRows - 1) / kTileRows);
   const int win_tiles = (a.window + kTileRows - 1) / kTileRows;
   if (comp_tiles + win_tiles == 0) return set_error(DSV4KV_ERR_INVALID_ARG, "decode: no rows to attend");
   const Plan pl = make_plan(a.batch, comp_tiles, win_tiles);
@@ -1146,17 +1214,20 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
                       uint64_t(kDim) * 2, uint64_t(a.heads) * kDim * 2, 64, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B))
     return set_error(DSV4KV_ERR_INVALID_ARG, "decode: cannot encode the query tensor map");
   const dsv4kv_cache& cc = a.comp;
+  // rows a tensor map spans: the batch of dense caches, or a pool
+  auto total_rows = [&](const dsv4kv_cache& c, const PageDesc& pg) -> uint64_t {
+    const int64_t r = pg.table ? c.rows : int64_t(a.batch) * std::max<int64_t>(c.rows, 1);
+    return std::max<uint64_t>(1, uint64_t(r));
+  };
   if (fmt == DSV4KV_BF16) {
     // contiguous row runs: boxes of 64 channels x 64 rows, 128-byte swizzle
     const void* comp_base = cc.codes ? cc.codes : a.win.codes;
-    const uint64_t comp_rows_total = std::max<uint64_t>(1, uint64_t(a.batch) * uint64_t(std::max<int64_t>(cc.rows, 1)));
-    if (!encode_tmap_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, comp_base, kDim, comp_rows_total, uint64_t(kDim) * 2,
-                        64, kTileRows, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!encode_tmap_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, comp_base, kDim, total_rows(cc, a.comp_pg),
+                        uint64_t(kDim) * 2, 64, kTileRows, CU_TENSOR_MAP_SWIZZLE_128B))
       return set_error(DSV4KV_ERR_INVALID_ARG, "decode: cannot encode the compressed-cache tensor map");
     const void* win_base = a.win.codes ? a.win.codes : comp_base;
-    const uint64_t win_rows_total = std::max<uint64_t>(1, uint64_t(a.batch) * uint64_t(std::max<int64_t>(a.win.rows, 1)));
-    if (!encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, win_base, kDim, win_rows_total, uint64_t(kDim) * 2, 64,
-                        kTileRows, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, win_base, kDim, total_rows(a.win, a.win_pg),
+                        uint64_t(kDim) * 2, 64, kTileRows, CU_TENSOR_MAP_SWIZZLE_128B))
       return set_error(DSV4KV_ERR_INVALID_ARG, "decode: cannot encode the window tensor map");
   } else {
     tc = tq;  // unused: quantised rows are loaded by the loader warps
@@ -1168,12 +1239,14 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
   p.n = a.n;
   p.window = a.window;
   p.k = a.idx ? a.k : 0;
-  p.comp_tiles = pl.comp_tiles;
-  p.tiles = pl.tiles;
   p.splits = pl.splits;
-  p.tiles_per_split = pl.tiles_per_split;
-  p.comp_rows = cc.rows;
-  p.win_rows = a.win.rows;
+  p.t_seq = a.t_seq;
+  p.t_max = a.t_max;
+  p.stride = std::max(1, a.stride);
+  p.comp_map = RowMap{a.comp_pg.table, std::max(1, a.comp_pg.page_rows), a.comp_pg.table_stride,
+                      cc.rows, a.comp_pg.pool_pages};
+  p.win_map = RowMap{a.win_pg.table, std::max(1, a.win_pg.page_rows), a.win_pg.table_stride, a.win.rows,
+                     a.win_pg.pool_pages};
   p.idx = a.idx;
   p.comp_codes = static_cast<const uint8_t*>(cc.codes);
   p.comp_scales = cc.scales;

@@ -688,12 +688,267 @@ __device__ void select_by_scan(const float* __restrict__ sc, int64_t n, uint32_t
   if (threadIdx.x == 0 && s_gt_seen + min(s_eq_seen, r_eq) != kk) set_status(status, DSV4KV_DEV_INCONSISTENT);
 }
 
-__global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __restrict__ scores, int64_t n, int k,
+// ------------------------------------------------------------------ paged, ragged scoring
+// Sequence b of a ragged batch has n_b = max(0, floor((t_b - window) /
+// stride)) keys, stored in pages of a pool: key i is pool row table[b][i /
+// page] * page + i % page.  Its keys are cut into units of kPagedUnit
+// consecutive keys (a page holds whole units); the units of all sequences
+// are numbered sequence after sequence (a sequence with n_b <= k has none: it
+// needs no scores) and handed out one per warp claim from one counter, the
+// next claim issued while the current unit is scored, as in the tail queue of
+// the dense-layout kernel.  Scores go to the sequence's score row, histogram
+// counts straight to its global histogram.  Keys of a page number outside the
+// pool score -inf (and flag DSV4KV_DEV_BAD_PAGE).
+constexpr int kPagedUnit = 32;
+constexpr int kMaxPagedBatch = 1024;
+
+__device__ __forceinline__ int64_t ragged_entries(const int64_t* t_seq, int b, int64_t t_max, int window, int stride,
+                                                  int64_t n_max, uint32_t* status) {
+  int64_t t = t_seq[b];
+  if (t < 0 || t > t_max) {
+    set_status(status, DSV4KV_DEV_BAD_LENGTH);
+    t = t < 0 ? 0 : t_max;
+  }
+  return t > window ? min(n_max, (t - window) / stride) : 0;
+}
+
+struct PagedKeys {
+  const void* codes;       // pool rows: bf16 [rows][128] or fp4 codes [rows][64]
+  const uint8_t* scales;   // fp4: [rows][8]
+  const int32_t* table;
+  int page, tstride;
+  int64_t pages;
+};
+
+template <int FMT>
+__global__ void __launch_bounds__(256) index_score_paged(const uint16_t* __restrict__ qidx, const PagedKeys pk,
+                                                         const int64_t* __restrict__ t_seq, int64_t t_max, int window,
+                                                         int stride, int64_t n_max, int k, int batch,
+                                                         float* __restrict__ scores, uint32_t* __restrict__ hist,
+                                                         uint32_t* __restrict__ claim, uint32_t* __restrict__ status) {
+  __shared__ uint32_t s_upre[kMaxPagedBatch + 1];  // first unit of every sequence; [batch] = all units
+  pdl_trigger();
+  pdl_wait();
+  {
+    constexpr int PER = kMaxPagedBatch / 256;
+    uint32_t c[PER], sum = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int b = PER * threadIdx.x + j;
+      const int64_t n_b = b < batch ? ragged_entries(t_seq, b, t_max, window, stride, n_max, nullptr) : 0;
+      c[j] = n_b > k ? uint32_t((n_b + kPagedUnit - 1) / kPagedUnit) : 0u;
+      sum += c[j];
+    }
+    uint32_t total;
+    uint32_t run = block_exclusive_scan<256>(sum, &total);
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int b = PER * threadIdx.x + j;
+      if (b < batch) s_upre[b] = run;
+      run += c[j];
+    }
+    if (threadIdx.x == 0) s_upre[batch] = total;
+  }
+  __syncthreads();
+  const uint32_t units = s_upre[batch];
+  const uint64_t pol = l2_evict_first_policy();  // keys are read once
+  const int lane = threadIdx.x & 31;
+  const size_t srow = size_t(score_stride(n_max));
+  // the unit's sequence: the last b with s_upre[b] <= u (binary search)
+  auto locate = [&](uint32_t u, int& b, int64_t& i0) {
+    int lo = 0, hi = batch - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_upre[mid] <= u) lo = mid;
+      else hi = mid - 1;
+    }
+    b = lo;
+    i0 = int64_t(u - s_upre[lo]) * kPagedUnit;
+  };
+  // pool row of key i0 of sequence b (-1: bad page)
+  auto unit_row = [&](int b, int64_t i0) -> int64_t {
+    const int32_t pg = __ldg(pk.table + size_t(b) * pk.tstride + size_t(i0 / pk.page));
+    if (pg < 0 || pg >= pk.pages) return -1;
+    return int64_t(pg) * pk.page + i0 % pk.page;
+  };
+  uint32_t raw = 0;
+  auto claim_next = [&]() {
+    if (lane == 0) raw = atomicAdd(claim, 1u);
+  };
+  auto resolve = [&]() -> int64_t {
+    const uint32_t u = __shfl_sync(kFull, raw, 0);
+    return u < units ? int64_t(u) : -1;
+  };
+  claim_next();
+  int64_t cur = resolve();
+  if (cur < 0) return;
+  if constexpr (FMT == DSV4KV_BF16) {
+    // half a warp per key; a unit is two groups of 16 keys (8 per half-warp)
+    constexpr int U = 8;
+    const int half = lane >> 4, l16 = lane & 15, my_key = (l16 >> 1) & 7;
+    const bool writer = !(lane & 1);
+    const uint16_t* keys = static_cast<const uint16_t*>(pk.codes);
+    float q[8];
+    int bq = -1;
+    auto load_group = [&](int64_t row0, int64_t left, int g, uint4 (&v)[U]) {
+      const uint16_t* kb = keys + size_t(row0 < 0 ? 0 : row0) * 128 + 8 * l16;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int key = 16 * g + U * half + u;
+        v[u] = (row0 >= 0 && key < left) ? ld_once_v4(kb + size_t(key) * 128, pol) : make_uint4(0, 0, 0, 0);
+      }
+    };
+    auto process = [&](int b, int64_t i0, int64_t row0, int64_t left, int g, const uint4 (&v)[U]) {
+      float pr[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) pr[u] = dot8_bf16(v[u], q);
+      float sc = reduce16_transposed<U>(pr, l16) + 0.0f;  // -0 -> +0
+      if (row0 < 0) sc = -INFINITY;
+      const int key = 16 * g + U * half + my_key;
+      if (writer && key < left) {
+        scores[size_t(b) * srow + size_t(i0 + key)] = sc;
+        atomicAdd(&hist[size_t(b) * kHistBins + (ord_f32(sc) >> 20)], 1u);
+      }
+    };
+    int b;
+    int64_t i0;
+    locate(uint32_t(cur), b, i0);
+    int64_t n_b = ragged_entries(t_seq, b, t_max, window, stride, n_max, status);
+    int64_t row0 = unit_row(b, i0);
+    if (row0 < 0) set_status(status, DSV4KV_DEV_BAD_PAGE);
+    uint4 va[U], vb[U];
+    load_group(row0, n_b - i0, 0, va);
+    claim_next();
+    while (true) {
+      load_group(row0, n_b - i0, 1, vb);
+      if (b != bq) {
+        const uint4 x = *reinterpret_cast<const uint4*>(qidx + size_t(b) * 128 + 8 * l16);
+        q[0] = bf16lo(x.x); q[1] = bf16hi(x.x); q[2] = bf16lo(x.y); q[3] = bf16hi(x.y);
+        q[4] = bf16lo(x.z); q[5] = bf16hi(x.z); q[6] = bf16lo(x.w); q[7] = bf16hi(x.w);
+        bq = b;
+      }
+      process(b, i0, row0, n_b - i0, 0, va);
+      const int64_t nxt = resolve();
+      int nb = b;
+      int64_t ni0 = 0, nn = n_b, nrow = row0;
+      if (nxt >= 0) {
+        locate(uint32_t(nxt), nb, ni0);
+        if (nb != b) nn = ragged_entries(t_seq, nb, t_max, window, stride, n_max, status);
+        nrow = unit_row(nb, ni0);
+        if (nrow < 0) set_status(status, DSV4KV_DEV_BAD_PAGE);
+        load_group(nrow, nn - ni0, 0, va);
+        claim_next();
+      }
+      process(b, i0, row0, n_b - i0, 1, vb);
+      if (nxt < 0) break;
+      b = nb;
+      i0 = ni0;
+      n_b = nn;
+      row0 = nrow;
+    }
+  } else {
+    // fp4 keys: a quarter warp per key (lane l4 owns channels [32 l4, 32 l4 + 32)),
+    // a unit is one warp iteration of 8 quads x 4 keys
+    constexpr int U = 4;
+    const int quad = lane >> 2, l4 = lane & 3;
+    const uint8_t* codes = static_cast<const uint8_t*>(pk.codes);
+    uint32_t qp[16];
+    int bq = -1;
+    auto load_unit = [&](int64_t row0, int64_t left, uint4 (&v)[U], uint32_t (&s2)[U]) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int key = 8 * u + quad;
+        const bool ok = row0 >= 0 && key < left;
+        const size_t r = size_t(ok ? row0 + key : 0);
+        v[u] = ok ? ld_once_v4(codes + r * 64 + 16 * l4, pol) : make_uint4(0, 0, 0, 0);
+        s2[u] = ok ? ld_once_u16(pk.scales + r * 8 + 2 * l4, pol) : 0u;
+      }
+    };
+    auto process = [&](int b, int64_t i0, int64_t row0, int64_t left, const uint4 (&v)[U], const uint32_t (&s2)[U]) {
+      float pr[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        uint32_t acc0 = 0, acc1 = 0;
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+          uint32_t h[4];
+          e2m1x8_unpack(w[wi], h);
+#pragma unroll
+          for (int by = 0; by < 4; ++by) {
+            if (wi < 2) acc0 = hfma2(qp[4 * wi + by], h[by], acc0);
+            else acc1 = hfma2(qp[4 * wi + by], h[by], acc1);
+          }
+        }
+        pr[u] = f16x2_sum(acc0) * e4m3_to_f32(s2[u] & 0xffu) + f16x2_sum(acc1) * e4m3_to_f32(s2[u] >> 8);
+      }
+      const bool bb1 = l4 & 2, bb0 = l4 & 1;
+      float k2[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) k2[i] = (bb1 ? pr[2 + i] : pr[i]) + __shfl_xor_sync(kFull, bb1 ? pr[i] : pr[2 + i], 2);
+      float sc = (bb0 ? k2[1] : k2[0]) + __shfl_xor_sync(kFull, bb0 ? k2[0] : k2[1], 1) + 0.0f;
+      if (row0 < 0) sc = -INFINITY;
+      const int key = 8 * l4 + quad;  // lane l4 ends with key u = l4
+      if (key < left) {
+        scores[size_t(b) * srow + size_t(i0 + key)] = sc;
+        atomicAdd(&hist[size_t(b) * kHistBins + (ord_f32(sc) >> 20)], 1u);
+      }
+    };
+    int b;
+    int64_t i0;
+    locate(uint32_t(cur), b, i0);
+    int64_t n_b = ragged_entries(t_seq, b, t_max, window, stride, n_max, status);
+    int64_t row0 = unit_row(b, i0);
+    if (row0 < 0) set_status(status, DSV4KV_DEV_BAD_PAGE);
+    uint4 va[U];
+    uint32_t sa[U];
+    load_unit(row0, n_b - i0, va, sa);
+    claim_next();
+    while (true) {
+      if (b != bq) {
+        const uint16_t* qb = qidx + size_t(b) * 128 + 32 * l4;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) qp[j] = f32x2_to_f16x2(bf16f(qb[2 * j]), bf16f(qb[2 * j + 1]));
+        bq = b;
+      }
+      const int64_t nxt = resolve();
+      int nb = b;
+      int64_t ni0 = 0, nn = n_b, nrow = row0;
+      uint4 vb[U];
+      uint32_t sb2[U];
+      if (nxt >= 0) {
+        locate(uint32_t(nxt), nb, ni0);
+        if (nb != b) nn = ragged_entries(t_seq, nb, t_max, window, stride, n_max, status);
+        nrow = unit_row(nb, ni0);
+        if (nrow < 0) set_status(status, DSV4KV_DEV_BAD_PAGE);
+        load_unit(nrow, nn - ni0, vb, sb2);
+        claim_next();
+      }
+      process(b, i0, row0, n_b - i0, va, sa);
+      if (nxt < 0) break;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        va[u] = vb[u];
+        sa[u] = sb2[u];
+      }
+      b = nb;
+      i0 = ni0;
+      n_b = nn;
+      row0 = nrow;
+    }
+  }
+}
+
+// (t_seq != null: a ragged batch, sequence b selects among its own n_b <=
+// n_max entries; the score rows keep the stride of n_max.)
+__global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __restrict__ scores, int64_t n_max, int k,
                                                             int64_t chunk, uint32_t* __restrict__ hist,
                                                             int32_t* __restrict__ idx_out,
                                                             int32_t* __restrict__ count_out,
                                                             uint32_t* __restrict__ status,
-                                                            uint32_t* __restrict__ tail_ctr) {
+                                                            uint32_t* __restrict__ tail_ctr,
+                                                            const int64_t* __restrict__ t_seq, int64_t t_max,
+                                                            int window, int stride) {
   extern __shared__ __align__(16) uint64_t stage[];  // the tie list; kSelWarps lists of kWarpCap (the
                                                      // warps' runs); the leader's receive buffer
   __shared__ uint32_t s_wcnt[kSelWarps];
@@ -706,15 +961,27 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
   const int b = blockIdx.y;
   const uint32_t rank = cluster_rank();
   const uint32_t csize = gridDim.x;  // one cluster spans the sequence's CTAs
-  const uint32_t kk = uint32_t(int64_t(k) < n ? int64_t(k) : n);
   uint32_t* hb = hist + size_t(b) * kHistBins;
-  const float* sc = scores + size_t(b) * size_t(score_stride(n));
-  const int64_t n0 = int64_t(rank) * chunk, n1 = min(n, n0 + chunk);
+  const float* sc = scores + size_t(b) * size_t(score_stride(n_max));
   const int lane = threadIdx.x & 31;
   pdl_trigger();
   pdl_wait();
-  cluster_arrive_relaxed();  // this CTA has started (waited for before the first remote store)
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *tail_ctr = 0;  // the score kernel's queue, for the next call
+  const int64_t n = t_seq ? ragged_entries(t_seq, b, t_max, window, stride, n_max, nullptr) : n_max;
+  if (n <= k) {
+    // a ragged sequence with no more entries than k: all of them (the score
+    // kernel left its histogram untouched).  The whole cluster takes this
+    // branch, before any cluster barrier.
+    if (rank == 0) {
+      int32_t* out = idx_out + size_t(b) * k;
+      for (int i = threadIdx.x; i < k; i += kSelThreads) out[i] = i < n ? i : -1;
+      if (threadIdx.x == 0 && count_out) count_out[b] = int32_t(n);
+    }
+    return;
+  }
+  const uint32_t kk = uint32_t(k);
+  const int64_t n0 = min(n, int64_t(rank) * chunk), n1 = min(n, n0 + chunk);
+  cluster_arrive_relaxed();  // this CTA has started (waited for before the first remote store)
 
   // 1) every warp owns a contiguous run of the CTA's chunk; the first
   //    batches of its run are in flight while the histogram is read
@@ -923,10 +1190,13 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
     for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) hb[i] = 0;
 }
 
-__global__ void index_fill_all(int64_t n, int k, int32_t* __restrict__ idx_out, int32_t* __restrict__ count_out) {
+__global__ void index_fill_all(int64_t n_max, int k, int32_t* __restrict__ idx_out, int32_t* __restrict__ count_out,
+                               const int64_t* __restrict__ t_seq, int64_t t_max, int window, int stride,
+                               uint32_t* __restrict__ status) {
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.y;
+  const int64_t n = t_seq ? ragged_entries(t_seq, b, t_max, window, stride, n_max, status) : n_max;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < k; i += gridDim.x * blockDim.x)
     idx_out[size_t(b) * k + i] = i < n ? i : -1;
   if (count_out && blockIdx.x == 0 && threadIdx.x == 0) count_out[b] = int32_t(n);
@@ -1271,9 +1541,10 @@ size_t index_topk_zero_prefix_bytes(int batch) {
 }
 
 static dsv4kv_status index_fill_launch(int batch, int64_t n, int k, int32_t* idx_out, int32_t* count_out,
-                                       cudaStream_t stream) {
+                                       cudaStream_t stream, const Ragged& rg, uint32_t* status) {
   const dim3 grid((unsigned)((k + 255) / 256), (unsigned)batch);
-  launch_pdl(index_fill_all, grid, dim3(256), 0, stream, n, k, idx_out, count_out);
+  launch_pdl(index_fill_all, grid, dim3(256), 0, stream, n, k, idx_out, count_out, rg.t_seq, rg.t_max, rg.window,
+             rg.stride, status);
   return check_launch("index_fill_all");
 }
 
@@ -1323,8 +1594,10 @@ dsv4kv_status index_score_launch(const uint16_t* qidx, const dsv4kv_cache& keys,
 }
 
 dsv4kv_status index_select_launch(int batch, int64_t n, int k, int32_t* idx_out, int32_t* count_out, void* ws,
-                                  size_t ws_bytes, cudaStream_t stream) {
-  if (n <= k) return index_fill_launch(batch, n, k, idx_out, count_out, stream);
+                                  size_t ws_bytes, cudaStream_t stream, const Ragged& rg) {
+  if (n <= k)
+    return index_fill_launch(batch, n, k, idx_out, count_out, stream, rg,
+                             ws_bytes >= 16 ? static_cast<uint32_t*>(ws) : nullptr);
   const IndexWs w = index_ws_layout(static_cast<char*>(ws), batch, n, k);
   if (ws_bytes < w.bytes) return set_error(DSV4KV_ERR_WORKSPACE, "index_select: workspace too small");
   const int sms = sm_count();
@@ -1361,7 +1634,8 @@ dsv4kv_status index_select_launch(int batch, int64_t n, int k, int32_t* idx_out,
   const int64_t chunk = units_per_cta * kSelChunkUnit;
   const unsigned ctas = unsigned((n + chunk - 1) / chunk);
   launch_pdl_cluster(index_select, dim3(ctas, unsigned(batch)), dim3(kSelThreads), kSelDyn, ctas, stream,
-                     (const float*)w.scores, n, k, chunk, w.hist, idx_out, count_out, w.status, w.tail_ctr);
+                     (const float*)w.scores, n, k, chunk, w.hist, idx_out, count_out, w.status, w.tail_ctr, rg.t_seq,
+                     rg.t_max, rg.window, rg.stride);
   return check_launch("index_select");
 }
 
@@ -1371,7 +1645,35 @@ dsv4kv_status index_topk_launch(const uint16_t* qidx, const dsv4kv_cache& keys, 
                                 cudaStream_t stream) {
   const dsv4kv_status st = index_score_launch(qidx, keys, batch, n, k, ws, ws_bytes, stream);
   if (st != DSV4KV_OK) return st;
-  return index_select_launch(batch, n, k, idx_out, count_out, ws, ws_bytes, stream);
+  return index_select_launch(batch, n, k, idx_out, count_out, ws, ws_bytes, stream, Ragged{});
+}
+
+dsv4kv_status index_topk_paged_launch(const uint16_t* qidx, const dsv4kv_cache& pool, const PageDesc& pg, int batch,
+                                      const Ragged& rg, int k, int32_t* idx_out, int32_t* count_out, void* ws,
+                                      size_t ws_bytes, cudaStream_t stream) {
+  const int64_t n_max = rg.t_max > rg.window ? (rg.t_max - rg.window) / rg.stride : 0;
+  if (batch > kMaxPagedBatch)
+    return set_error(DSV4KV_ERR_UNSUPPORTED, "index_topk_paged: batch %d > %d", batch, kMaxPagedBatch);
+  if (n_max > k) {
+    const IndexWs w = index_ws_layout(static_cast<char*>(ws), batch, n_max, k);
+    if (ws_bytes < w.bytes) return set_error(DSV4KV_ERR_WORKSPACE, "index_topk_paged: workspace too small");
+    const PagedKeys pk{pool.codes, static_cast<const uint8_t*>(pool.scales), pg.table, pg.page_rows, pg.table_stride,
+                       pg.pool_pages};
+    // one wave of persistent CTAs draining the unit queue
+    auto kern = pool.fmt == DSV4KV_BF16 ? index_score_paged<DSV4KV_BF16> : index_score_paged<DSV4KV_FP4_E2M1_G16>;
+    static std::atomic<int> occ_dev[2][64];  // per format and device; 0 = not queried yet
+    std::atomic<int>& slot = occ_dev[pool.fmt == DSV4KV_BF16 ? 0 : 1][current_device()];
+    int occ = slot.load(std::memory_order_relaxed);
+    if (occ == 0) {
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 256, 0) != cudaSuccess || occ < 1) occ = 1;
+      slot.store(occ, std::memory_order_relaxed);
+    }
+    launch_pdl(kern, dim3(unsigned(sm_count() * occ)), dim3(256), 0, stream, qidx, pk, rg.t_seq, rg.t_max, rg.window,
+               rg.stride, n_max, k, batch, w.scores, w.hist, w.tail_ctr, w.status);
+    const dsv4kv_status st = check_launch("index_score_paged");
+    if (st != DSV4KV_OK) return st;
+  }
+  return index_select_launch(batch, n_max, k, idx_out, count_out, ws, ws_bytes, stream, rg);
 }
 
 }  // namespace dsv4kv

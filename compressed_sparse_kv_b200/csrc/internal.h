@@ -83,8 +83,23 @@ int64_t append_emit_entry(int64_t t, int window, int stride);
 dsv4kv_status append_launch(const void* s_new, const float* w, int batch, int64_t t, int dim, int k_taps, int stride,
                             int window, int rope_dim, double rope_base, void* raw_ring, void* win_ring, void* comp,
                             int64_t comp_rows, cudaStream_t stream);
+// A ragged batch (t_seq null: every sequence has the call's n entries).
+struct Ragged {
+  const int64_t* t_seq = nullptr;
+  int64_t t_max = 0;
+  int window = 0, stride = 1;
+};
+// Pages of a paged cache (table null: the dense [B][rows] layout of a dsv4kv_cache).
+struct PageDesc {
+  const int32_t* table;
+  int page_rows, table_stride;
+  int64_t pool_pages;
+};
 dsv4kv_status index_select_launch(int batch, int64_t n, int k, int32_t* idx_out, int32_t* count_out, void* ws,
-                                  size_t ws_bytes, cudaStream_t stream);
+                                  size_t ws_bytes, cudaStream_t stream, const Ragged& rg = Ragged{});
+dsv4kv_status index_topk_paged_launch(const uint16_t* qidx, const dsv4kv_cache& pool, const PageDesc& pg, int batch,
+                                      const Ragged& rg, int k, int32_t* idx_out, int32_t* count_out, void* ws,
+                                      size_t ws_bytes, cudaStream_t stream);
 dsv4kv_status index_topk_pool_launch(const uint16_t* qidx, const dsv4kv_cache& keys, int batch, int64_t n,
                                      const int32_t* pool, int pool_cap, int k, int32_t* idx_out, int32_t* count_out,
                                      void* ws, size_t ws_bytes, cudaStream_t stream);
@@ -94,19 +109,24 @@ dsv4kv_status index_topk_launch(const uint16_t* qidx, const dsv4kv_cache& keys, 
 
 struct DecodeArgs {
   const void* q;
-  dsv4kv_cache comp;
+  dsv4kv_cache comp;   // paged: codes / scales are the pools, rows = pool rows
   dsv4kv_cache win;
   const int32_t* idx;  // null for dense
   int batch, heads, dim;
-  int64_t n;
-  int window;
-  int k;  // sparse only
+  int64_t n;           // uniform: entries; ragged: the most any sequence has
+  int window;          // uniform: window rows; ragged: the window length W
+  int k;               // sparse only
   int64_t t;
   float sm_scale;
   int rope_dim;
   double rope_base;
   int out_fp32;
   void* out;
+  // ragged batch (t_seq null: uniform)
+  const int64_t* t_seq = nullptr;
+  int64_t t_max = 0;
+  int stride = 1;
+  PageDesc comp_pg{}, win_pg{};
 };
 size_t decode_ws_bytes(int batch, int heads, int dim, int64_t rows_per_seq);
 dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream);

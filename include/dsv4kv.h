@@ -53,6 +53,8 @@ typedef enum {
 #define DSV4KV_DEV_TIMEOUT 0x2u    /* a bounded wait gave up: outputs are invalid       */
 #define DSV4KV_DEV_INCONSISTENT 0x4u /* selection counts disagreed: outputs are invalid */
 #define DSV4KV_DEV_BAD_POOL 0x8u     /* a candidate pool was not ascending: ties may differ */
+#define DSV4KV_DEV_BAD_PAGE 0x10u    /* a block-table page number was outside the pool: its rows skipped */
+#define DSV4KV_DEV_BAD_LENGTH 0x20u  /* a sequence length was < 0 or > t_max: clamped into [0, t_max] */
 
 /* Cache row formats.
  *  DSV4KV_BF16:          codes = bf16 [B][rows][dim]; scales = NULL.
@@ -303,6 +305,75 @@ dsv4kv_status dsv4kv_dense_decode(const void* q, const dsv4kv_cache* comp,
                                   int64_t n, int32_t window, int64_t t, float sm_scale,
                                   int32_t rope_dim, double rope_base, int32_t out_fp32,
                                   void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Paged and ragged caches.  [P1] hybrid KV cache manager paragraph: the
+ * caches are kept in blocks drawn from a shared block pool (window and
+ * compressor-state blocks of a constant size per request).
+ *
+ * A paged cache keeps the rows of every sequence in pages of `page_rows` rows
+ * inside one pool that the whole batch shares; row i of sequence b is pool row
+ *   table[b * table_stride + i / page_rows] * page_rows + i % page_rows.
+ * A ragged batch gives every sequence its own length: t_seq[b] (device int64
+ * [batch]) is the position of its decode query, so that it has
+ *   n_b = max(0, floor((t_b - window) / stride)) compressed entries and
+ *   w_b = min(t_b, window) window rows (logical rows 0 .. w_b - 1 of its
+ *   window pages, in any order of positions),
+ * its own top-k over its own n_b entries and its own output rotation by -t_b.
+ * The calls below are the per-sequence steps of the dense-layout calls above
+ * on the rows the tables point to.  t_max (host) must be >= every t_b; it
+ * sizes the workspaces and the grids.  A t_b outside [0, t_max] is clamped
+ * into it and flags DSV4KV_DEV_BAD_LENGTH; a page number outside
+ * [0, pool_pages) flags DSV4KV_DEV_BAD_PAGE and the rows of that page are
+ * skipped.  Rows of a page past a sequence's last row are never read.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int32_t fmt;            /* dsv4kv_format */
+  int32_t dim;            /* channels per row */
+  int32_t page_rows;      /* rows per page: a positive multiple of 64 */
+  int32_t table_stride;   /* page numbers per sequence in `table` (its row pitch) */
+  int64_t pool_pages;     /* pages in the pool */
+  const int32_t* table;   /* device int32 [batch][table_stride] page numbers */
+  const void* codes;      /* device pool [pool_pages * page_rows][row bytes of fmt], 16-byte aligned */
+  const void* scales;     /* device pool of the format's scales per row, or NULL for bf16 */
+} dsv4kv_paged_cache;
+
+/* dsv4kv_index_topk over paged indexer keys (bf16 or fp4, dim 128) of a
+ * ragged batch: sequence b scores its n_b keys and keeps the first
+ * min(k, n_b) under (score descending, index ascending), written ascending
+ * to idx_out[b], padded with -1; count_out[b] = min(k, n_b). */
+size_t dsv4kv_index_topk_paged_workspace_bytes(int32_t batch, int64_t t_max, int32_t window, int32_t stride,
+                                               int32_t k);
+
+dsv4kv_status dsv4kv_index_topk_paged(const void* qidx, const dsv4kv_paged_cache* keys, int32_t batch,
+                                      const int64_t* t_seq, int64_t t_max, int32_t window, int32_t stride,
+                                      int32_t k, int32_t* idx_out, int32_t* count_out, void* ws,
+                                      size_t ws_bytes, void* stream);
+
+/* dsv4kv_sparse_decode over paged compressed and window caches of a ragged
+ * batch: sequence b attends to its selected entries (idx[b], indices in
+ * [0, n_b), as dsv4kv_index_topk_paged writes them) and its w_b window rows,
+ * and its output is rotated by -t_b. */
+size_t dsv4kv_sparse_decode_paged_workspace_bytes(int32_t batch, int32_t heads, int32_t dim, int32_t k,
+                                                  int32_t window);
+
+dsv4kv_status dsv4kv_sparse_decode_paged(const void* q, const dsv4kv_paged_cache* comp,
+                                         const dsv4kv_paged_cache* win, const int32_t* idx, int32_t batch,
+                                         int32_t heads, const int64_t* t_seq, int64_t t_max, int32_t window,
+                                         int32_t stride, int32_t k, float sm_scale, int32_t rope_dim,
+                                         double rope_base, int32_t out_fp32, void* out, void* ws,
+                                         size_t ws_bytes, void* stream);
+
+/* dsv4kv_dense_decode over paged caches of a ragged batch: sequence b attends
+ * to all its n_b compressed entries and its w_b window rows. */
+size_t dsv4kv_dense_decode_paged_workspace_bytes(int32_t batch, int32_t heads, int32_t dim, int64_t t_max,
+                                                 int32_t window, int32_t stride);
+
+dsv4kv_status dsv4kv_dense_decode_paged(const void* q, const dsv4kv_paged_cache* comp,
+                                        const dsv4kv_paged_cache* win, int32_t batch, int32_t heads,
+                                        const int64_t* t_seq, int64_t t_max, int32_t window, int32_t stride,
+                                        float sm_scale, int32_t rope_dim, double rope_base, int32_t out_fp32,
+                                        void* out, void* ws, size_t ws_bytes, void* stream);
 
 /* Text of the last error on the calling host thread ("" if none). */
 const char* dsv4kv_last_error(void);

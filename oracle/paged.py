@@ -52,3 +52,20 @@ def ragged_c4a_step(q, qidx, key_pool, key_tables, comp_pool, comp_tables, win_p
         cnt.append(c)
         out.append(shared_kv_decode(q[b], rows, scale, int(t[b]), rope_dim, base))
     return np.stack(idx), np.array(cnt), np.stack(out)
+
+
+def ragged_c128a_step(q, comp_pool, comp_tables, win_pool, win_tables, t, page: int, window: int = 128,
+                      stride: int = 128, scale: float = 512 ** -0.5, rope_dim: int = 64,
+                      base: float = 10000.0) -> np.ndarray:
+    """One c128a layer step of a ragged, paged batch: per sequence b, one
+    softmax over all its n_b compressed entries and its min(t_b, W) window
+    rows, rotated by -t_b ([P1] "c128a": full attention over the compressed
+    entries).  Returns out [B][H][D]."""
+    out = []
+    for b in range(len(q)):
+        n_b = n_entries(int(t[b]), window, stride)
+        w_b = min(int(t[b]), window)
+        rows = np.concatenate([paged_rows(comp_pool, comp_tables[b], n_b, page),
+                               paged_rows(win_pool, win_tables[b], w_b, page)], axis=0)
+        out.append(shared_kv_decode(q[b], rows, scale, int(t[b]), rope_dim, base))
+    return np.stack(out)

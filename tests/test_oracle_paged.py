@@ -79,3 +79,41 @@ def test_ragged_lengths_are_independent_sequences():
     win = P.paged_rows(wp, wt[2], 90, 64)
     ref = A.shared_kv_decode(q[2], win, 512 ** -0.5, 90)
     assert np.allclose(out[2], ref, rtol=0, atol=1e-12)
+
+
+def test_ragged_c128a_with_equal_lengths_is_the_uniform_dense_step():
+    rng = np.random.default_rng(5)
+    b, t, page = 2, 128 * 40 + 128, 64               # 40 entries each
+    n = C.n_entries(t, 128, 128)
+    cpool = rng.standard_normal((b * page, 512))
+    wpool = rng.standard_normal((2 * b * page, 512))
+    ct = [np.array([1]), np.array([0])]               # sequence 0 in page 1, sequence 1 in page 0
+    wt = [np.array([3, 2]), np.array([0, 1])]
+    q = rng.standard_normal((b, 4, 512))
+    out = P.ragged_c128a_step(q, cpool, ct, wpool, wt, [t, t], page)
+    comp = np.stack([cpool[page:page + n], cpool[:n]])
+    win = np.stack([np.concatenate([wpool[3 * page:4 * page], wpool[2 * page:3 * page]])[:128],
+                    wpool[:2 * page][:128]])
+    ref = A.dense_decode(q, comp, win, t, 512 ** -0.5)
+    assert np.allclose(out, ref, rtol=0, atol=1e-12)
+
+
+def test_ragged_c128a_short_sequences_are_window_only_attention():
+    """t_b < W: no compressed entries, t_b window rows, textbook softmax attention."""
+    rng = np.random.default_rng(6)
+    wpool = rng.standard_normal((3 * 64, 512))
+    q = rng.standard_normal((2, 4, 512))
+    t = [100, 37]
+    out = P.ragged_c128a_step(q, np.zeros((64, 512)), [np.array([0]), np.array([0])], wpool,
+                              [np.array([2, 0]), np.array([1])], t, 64)
+    for s, (tb, rows) in enumerate([(100, np.concatenate([wpool[128:192], wpool[:64]])[:100]),
+                                    (37, wpool[64:101])]):
+        sc = q[s] @ rows.T * 512 ** -0.5
+        p = np.exp(sc - sc.max(axis=1, keepdims=True))
+        o = (p / p.sum(axis=1, keepdims=True)) @ rows
+        # inverse rotation by -t_b of the last 64 channels (interleaved pairs), written out
+        ang = -tb * 10000.0 ** (-np.arange(32) / 32.0)
+        x, y = o[:, 448::2].copy(), o[:, 449::2].copy()
+        o[:, 448::2] = x * np.cos(ang) - y * np.sin(ang)
+        o[:, 449::2] = x * np.sin(ang) + y * np.cos(ang)
+        assert np.allclose(out[s], o, rtol=0, atol=1e-12)
