@@ -147,6 +147,11 @@ def replicas_for(kind, batch, t, main_fmt, index_fmt, at_least, pool=0, l2_facto
 PAGE_ROWS = 256
 
 
+def torch_empty_like(t):
+    import torch
+    return torch.empty_like(t)
+
+
 def ragged_lengths(batch, t, seed):
     """Per-sequence query positions of the ragged workloads: uniform in [t/2, t]."""
     rng = np.random.default_rng(seed)
@@ -206,6 +211,14 @@ class PagedLayer:
         self.ws_idx = K.new_workspace(K.lib().dsv4kv_index_topk_paged_workspace_bytes(batch, self.t_max, 128, 4, 512))
         self.ws_dec = K.new_workspace(K.lib().dsv4kv_sparse_decode_paged_workspace_bytes(batch, heads, 512, 512, 128))
         torch.cuda.synchronize()
+
+    def twin(self):
+        """The same layer (same caches) with its own per-step buffers and workspaces."""
+        import copy
+        t = copy.copy(self)
+        t.idx, t.cnt, t.out = torch_empty_like(self.idx), torch_empty_like(self.cnt), torch_empty_like(self.out)
+        t.ws_idx, t.ws_dec = self.K.new_workspace(self.ws_idx.numel()), self.K.new_workspace(self.ws_dec.numel())
+        return t
 
     def alg_bytes(self):
         sel = np.minimum(self.n_seq, self.k)
@@ -309,6 +322,18 @@ class Layer:
             sh["ws_dec"] = K.new_workspace(need_d)
         self.ws_dec = sh["ws_dec"]
         torch.cuda.synchronize()  # inputs and zeroed workspaces are complete before any other stream uses them
+
+    def twin(self):
+        """The same layer (same caches) with its own per-step buffers and workspaces."""
+        import copy
+        t = copy.copy(self)
+        t.idx, t.cnt, t.out = torch_empty_like(self.idx), torch_empty_like(self.cnt), torch_empty_like(self.out)
+        t.ws_dec = self.K.new_workspace(self.ws_dec.numel())
+        if self.kind == "c4a":
+            t.ws_idx = self.K.new_workspace(self.ws_idx.numel())
+        if self.pool:
+            t.ws_pool = self.K.new_workspace(self.ws_pool.numel())
+        return t
 
     # algorithmic bytes of one step: indexer keys + rows read (queries/outputs excluded)
     def alg_bytes(self):
@@ -589,134 +614,142 @@ def time_layer(layer, steps, warmup, dist_max, dev_index, sample_clocks):
 
 def time_e2e(layer, steps):
     """Same steps through the public API with host buffers: every step copies
-    its queries from pinned host memory to the device, makes the calls and
-    copies its outputs back to pinned host memory, all inside the timed
-    region.  Steps are independent, so they are pipelined over three streams
-    (upload, compute, download) with double-buffered device and host buffers:
-    step i's copies overlap the compute of its neighbours, and events order
-    every buffer reuse.  The steps run twice: issued eagerly from Python, and
-    captured once (calls and copies) into a CUDA graph that is replayed, the
-    way a serving loop issues its decode steps.  Returns (graph ms, eager ms,
-    H2D bytes per step, D2H bytes per step)."""
+    its queries (and, for c4a, its indexer query) from pinned host memory to
+    the device, makes the library calls and copies its output back to pinned
+    host memory, all inside the timed region.
+
+    Steps alternate between two streams, each with its own device buffers,
+    workspaces and pinned host buffers, so step i+1's upload and step i-1's
+    download overlap step i's calls (and two steps' kernels may share the
+    GPU).  Each (stream, cache replica) pair replays a CUDA graph of its
+    [upload -> calls -> download], captured once, the way a serving loop
+    issues its decode steps; the same steps issued eagerly from Python give
+    the eager figure.  Returns (graph ms, eager ms, H2D bytes per step, D2H
+    bytes per step)."""
     torch = layer.torch
     R = len(layer.reps)
     NB = 2
+    lanes = [layer.twin() for _ in range(NB)]             # own buffers and workspaces per stream
     q_host = [layer.q.cpu().pin_memory() for _ in range(NB)]
     qi_host = [layer.qidx.cpu().pin_memory() for _ in range(NB)]
     out_host = [torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory() for _ in range(NB)]
     q_dev = [torch.empty_like(layer.q) for _ in range(NB)]
     qi_dev = [torch.empty_like(layer.qidx) for _ in range(NB)]
-    out_dev = [torch.empty_like(layer.out) for _ in range(NB)]
-    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    ev_in = [torch.cuda.Event() for _ in range(NB)]
-    ev_comp = [torch.cuda.Event() for _ in range(NB)]
-    ev_out = [torch.cuda.Event() for _ in range(NB)]
+    streams = [torch.cuda.Stream() for _ in range(NB)]
     torch.cuda.synchronize()
 
-    def step(i, recorded=None):
-        # recorded: during a capture, the events recorded so far in it (only those can be waited on)
-        j = i % NB
+    def body(i):
+        j, r = i % NB, i % R
+        L = lanes[j]
+        q_dev[j].copy_(q_host[j], non_blocking=True)
+        if L.kind == "c4a":
+            qi_dev[j].copy_(qi_host[j], non_blocking=True)
+            L.index(r, qidx=qi_dev[j])
+        L.decode(r, q=q_dev[j])
+        out_host[j].copy_(L.out, non_blocking=True)
 
-        def wait(s, e):
-            if recorded is None or id(e) in recorded:
-                s.wait_event(e)
-
-        def record(e, s):
-            e.record(s)
-            if recorded is not None:
-                recorded.add(id(e))
-
-        with torch.cuda.stream(s_in):
-            wait(s_in, ev_comp[j])               # step i-NB has consumed this input buffer
-            q_dev[j].copy_(q_host[j], non_blocking=True)
-            if layer.kind == "c4a":
-                qi_dev[j].copy_(qi_host[j], non_blocking=True)
-            record(ev_in[j], s_in)
-        with torch.cuda.stream(s_comp):
-            wait(s_comp, ev_in[j])
-            wait(s_comp, ev_out[j])              # step i-NB's output has left this buffer
-            if layer.kind == "c4a":
-                layer.index(i % R, qidx=qi_dev[j])
-            layer.decode(i % R, q=q_dev[j], out=out_dev[j])
-            record(ev_comp[j], s_comp)
-        with torch.cuda.stream(s_out):
-            wait(s_out, ev_comp[j])
-            out_host[j].copy_(out_dev[j], non_blocking=True)
-            record(ev_out[j], s_out)
-
-    for i in range(2 * NB):
-        step(i)
-    torch.cuda.synchronize()
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(s_in)
-    for i in range(steps):
-        step(i)
-    stop.record(s_out)                              # after the last download (s_out is last in every step)
-    stop.synchronize()
-    eager_ms = start.elapsed_time(stop)
-
-    cap = torch.cuda.Stream()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=cap):
-        fork = torch.cuda.Event()
-        fork.record(cap)
-        for s_ in (s_in, s_comp, s_out):
-            s_.wait_event(fork)
-        rec = set()
+    def run(issue):
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        start.record(streams[0])
+        for s_ in streams[1:]:
+            s_.wait_event(start)
         for i in range(steps):
-            step(i, rec)
-        for s_ in (s_in, s_comp, s_out):
+            with torch.cuda.stream(streams[i % NB]):
+                issue(i)
+        for s_ in streams[1:]:
             e = torch.cuda.Event()
             e.record(s_)
-            cap.wait_event(e)
-    with torch.cuda.stream(cap):
-        g.replay()                                  # warm-up replay
+            streams[0].wait_event(e)
+        stop.record(streams[0])
+        stop.synchronize()
+        return start.elapsed_time(stop)
+
+    for i in range(2 * NB):                          # warm-up, eager
+        with torch.cuda.stream(streams[i % NB]):
+            body(i)
     torch.cuda.synchronize()
-    with torch.cuda.stream(cap):
-        start.record(cap)
-        g.replay()
-        stop.record(cap)
-    stop.synchronize()
-    graph_ms = start.elapsed_time(stop)
-    del g
+    eager_ms = run(body)
+    # one graph per (stream, replica) pair of a step index
+    M = R if R % NB == 0 else NB * R
+    graphs = []
+    for m in range(M):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=streams[m % NB]):
+            body(m)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    for i in range(M):                               # every graph launched once before timing
+        with torch.cuda.stream(streams[i % NB]):
+            graphs[i].replay()
+    graph_ms = run(lambda i: graphs[i % M].replay())
+    del graphs
     h2d = layer.q.numel() * 2 + (layer.qidx.numel() * 2 if layer.kind == "c4a" else 0)
     return graph_ms, eager_ms, h2d, layer.out.numel() * 2
 
 
 # ------------------------------------------------------------------ oracle arm
-def oracle_sample(kind, batch, t, heads, budget_s=12.0, seed=7):
-    """Seconds per sequence of the float64 oracle on one layer step (one
-    sequence of the batch, repeated within a time budget)."""
-    import datagen as D
-    from datagen import workloads as WL
-    from oracle import attention as OA
-    from oracle import formats as OF
-    from oracle import indexer as OI
-    window, k = 128, 512
-    n = (t - window) // (4 if kind == "c4a" else 128)
-    keys = WL.keys_for(seed, 0)
-    q = OF.bf16_bits_to_f64(D.rows_normal_bf16(keys["q"], np.arange(heads), 512))
-    win = OF.bf16_bits_to_f64(D.rows_normal_bf16(keys["win"], np.arange(window), 512))
-    if kind == "c4a":
-        kr = OF.bf16_bits_to_f64(D.rows_int_bf16(keys["kidx"], np.arange(n), 128))
-        qi = OF.bf16_bits_to_f64(D.rows_int_bf16(keys["qidx"], np.array([0]), 128)[0])
-        comp = None
-    else:
-        comp = OF.bf16_bits_to_f64(D.rows_normal_bf16(keys["comp"], np.arange(n), 512))
-    reps, t0 = 0, time.perf_counter()
-    while True:
-        if kind == "c4a":
-            idx, cnt = OI.index_topk(qi, kr, k)
-            sel = OF.bf16_bits_to_f64(D.rows_normal_bf16(keys["comp"], idx[:cnt].astype(np.uint64), 512))
-            rows = np.concatenate([sel, win])
-            OA.shared_kv_decode(q, rows, 512 ** -0.5, t)
-        else:
-            OA.dense_decode(q[None], comp[None], win[None], t, 512 ** -0.5)
-        reps += 1
-        el = time.perf_counter() - t0
-        if el > budget_s or reps >= 200:
-            break
-    return el / reps, reps
+class OracleStep:
+    """The float64 oracle on one layer step of a workload, sequence by
+    sequence, with every input generated before any timing: the queries,
+    window rows and indexer keys of each sequence, and the compressed rows
+    the step reads (all of them for c128a; for c4a the rows its top-k picks,
+    found by one untimed top-k, as a resident cache would hold them).  A
+    timed sequence runs the oracle's top-k over all its keys, gathers the
+    selected rows and runs its attention."""
+
+    def __init__(self, kind, batch, t, heads, seqs, seed=7, t_seq=None):
+        import datagen as D
+        from datagen import workloads as WL
+        from oracle import formats as OF
+        from oracle import indexer as OI
+        self.kind, self.batch, self.heads, self.window, self.k = kind, batch, heads, 128, 512
+        self.seqs = list(seqs)
+        stride = 4 if kind == "c4a" else 128
+        keys = WL.keys_for(seed, 0)
+        self.inp = {}
+        for b in self.seqs:
+            tb = int(t if t_seq is None else t_seq[b])
+            n = max(0, (tb - self.window) // stride)
+            w = min(tb, self.window)
+            q = OF.bf16_bits_to_f64(D.rows_normal_bf16(keys["q"], np.arange(b * heads, (b + 1) * heads), 512))
+            win = OF.bf16_bits_to_f64(D.rows_normal_bf16(keys["win"], np.arange(b * 128, b * 128 + w), 512))
+            e = {"t": tb, "q": q, "win": win}
+            if kind == "c4a":
+                kr = OF.bf16_bits_to_f64(D.rows_int_bf16(keys["kidx"], np.arange(b * n, (b + 1) * n), 128))
+                qi = OF.bf16_bits_to_f64(D.rows_int_bf16(keys["qidx"], np.array([b]), 128)[0])
+                idx, cnt = OI.index_topk(qi, kr, self.k)
+                sel = idx[:cnt].astype(np.int64)
+                e.update(keys=kr, qidx=qi, sel=sel,
+                         rows=OF.bf16_bits_to_f64(D.rows_normal_bf16(keys["comp"], b * n + sel, 512)))
+            else:
+                e["comp"] = OF.bf16_bits_to_f64(D.rows_normal_bf16(keys["comp"], np.arange(b * n, (b + 1) * n), 512))
+            self.inp[b] = e
+
+    def run(self, b):
+        from oracle import attention as OA
+        from oracle import indexer as OI
+        e = self.inp[b]
+        if self.kind == "c4a":
+            idx, cnt = OI.index_topk(e["qidx"], e["keys"], self.k)
+            rows = e["rows"][np.searchsorted(e["sel"], idx[:cnt])]          # the selected rows of the cache
+            return OA.shared_kv_decode(e["q"], np.concatenate([rows, e["win"]]), 512 ** -0.5, e["t"])
+        return OA.dense_decode(e["q"][None], e["comp"][None], e["win"][None], e["t"], 512 ** -0.5)[0]
+
+
+def oracle_per_seq(kind, batch, t, heads, budget_s=12.0, t_seq=None):
+    """(seconds per sequence, sequences timed) of the oracle: the first
+    sequences of the batch, each once, until the budget is used."""
+    first = OracleStep(kind, batch, t, heads, [0], t_seq=t_seq)
+    t0 = time.perf_counter()
+    first.run(0)
+    one = time.perf_counter() - t0
+    m = int(max(1, min(batch, budget_s / max(one, 1e-6))))
+    st = OracleStep(kind, batch, t, heads, range(m), t_seq=t_seq)
+    t0 = time.perf_counter()
+    for b in range(m):
+        st.run(b)
+    return (time.perf_counter() - t0) / m, m
 
 
 def blas_threads():
@@ -728,21 +761,58 @@ def blas_threads():
         return 1
 
 
-def cpu_baseline(kind, batch, t, heads, budget_s):
+def cpu_baseline(kind, batch, t, heads, budget_s, t_seq=None):
     """The oracle on the host: with all the BLAS threads it starts with, and
     again limited to one thread."""
-    per_seq, reps = oracle_sample(kind, batch, t, heads, budget_s)
+    per_seq, m = oracle_per_seq(kind, batch, t, heads, budget_s, t_seq)
     out = {"value": 1.0 / (per_seq * batch), "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
-           "sample": f"{reps} x one sequence of the {batch}-sequence step (float64 NumPy oracle), scaled to a step"}
+           "sample": f"{m} of the {batch} sequences of one step (float64 NumPy oracle, inputs generated before "
+                     f"timing), scaled to the whole step"}
     try:
         from threadpoolctl import threadpool_limits
         with threadpool_limits(limits=1):
-            per1, reps1 = oracle_sample(kind, batch, t, heads, budget_s / 2)
+            per1, m1 = oracle_per_seq(kind, batch, t, heads, budget_s / 2, t_seq)
         out["value_1core"] = 1.0 / (per1 * batch)
-        out["sample_1core"] = f"{reps1} x one sequence, one BLAS thread"
+        out["sample_1core"] = f"{m1} sequences, one BLAS thread"
     except ImportError:
         pass
     return out
+
+
+def reference_arm(args, kind, batch, t, heads, config, wl_name, t_seq=None, budget_s=150.0):
+    """--impl reference: the oracle times `warmup` untimed and `steps` timed
+    steps on the host cores.  A step is the whole batch when all the steps
+    fit the budget; otherwise each step is a sample of S sequences (the next
+    S of the batch, cycling), and value counts whole steps (S / batch each)."""
+    probe = OracleStep(kind, batch, t, heads, [0], t_seq=t_seq)
+    t0 = time.perf_counter()
+    probe.run(0)
+    per_seq = time.perf_counter() - t0
+    total = args.steps + args.warmup
+    S = batch if total * batch * per_seq <= budget_s else int(max(1, budget_s / (total * per_seq)))
+    seqs = sorted({(i * S + j) % batch for i in range(total) for j in range(S)})
+    st = OracleStep(kind, batch, t, heads, seqs, t_seq=t_seq)
+
+    def one_step(i):
+        for j in range(S):
+            st.run((i * S + j) % batch)
+
+    for i in range(args.warmup):
+        one_step(i)
+    t0 = time.perf_counter()
+    for i in range(args.warmup, total):
+        one_step(i)
+    el = time.perf_counter() - t0
+    v = args.steps * S / batch / el
+    sample = (f"whole steps ({batch} sequences each)" if S == batch else
+              f"each step {S} of the {batch} sequences (cycling through the batch), counted as {S}/{batch} of a step")
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
+            "sequences_per_step": S, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "config": config,
+            "cpu_baseline": {"value": v, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample + "; float64 NumPy oracle, inputs generated before timing"},
+            "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 # ------------------------------------------------------------------ distributed plumbing
@@ -814,20 +884,29 @@ def main():
 
     wl_name = wl_desc(kind, batch, t, heads, mfmt, ifmt, pool)
 
+    # the workload's cache replicas and bytes per step, from the shapes alone, so
+    # that both arms print the same config
+    seed = 1234 + d["rank"]
+    if paged:
+        reps = replicas_for(kind, batch, t // 2, mfmt, ifmt, args.replicas, 0, args.l2_factor)
+        t_seq = ragged_lengths(batch, t, seed)
+        n_seq = np.maximum(0, (t_seq - 128) // 4)
+        alg = int((n_seq * KEY_BYTES[0]).sum() + ((np.minimum(n_seq, 512) + np.minimum(t_seq, 128)) * ROW_BYTES[0]).sum())
+        wl_name = (f"c4a layer decode, paged caches ({PAGE_ROWS}-row pages, shuffled), ragged B={batch}: t_b uniform "
+                   f"in [{t // 2}, {t}], H={heads} k=512 W=128 bf16")
+    else:
+        reps = replicas_for(kind, batch, t, mfmt, ifmt, args.replicas, pool, args.l2_factor)
+        t_seq = None
+        alg = step_bytes(kind, batch, t, mfmt, ifmt, pool=pool)
+    config = {"workload": wl_name, "batch_per_gpu": batch, "context": t, "heads": heads,
+              "parallelism": f"dp{d['world']}",
+              "l2": f"inputs larger than L2: {reps} cache replicas cycle, {alg / 1e6:.0f} MB read per step, "
+                    f"{reps * alg / 1e6:.0f} MB in all (>= 4 x the 126 MB L2)"}
+
     if args.impl == "reference":
         if d["rank"] != 0:
             return
-        per_seq, reps = oracle_sample(kind, batch, t, heads, budget_s=max(5.0, args.cpu_budget))  # bf16 rows
-        v = 1.0 / (per_seq * batch)
-        cb = {"value": v, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
-              "sample": f"{reps} x one sequence of the {batch}-sequence step, scaled to a step"}
-        print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": args.gpus,
-                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / v,
-                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                          "data": "synthetic", "config": {"workload": wl_name, "parallelism": f"dp{args.gpus}"},
-                          "cpu_baseline": cb,
-                          "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
-              flush=True)
+        print(json.dumps(reference_arm(args, kind, batch, t, heads, config, wl_name, t_seq)), flush=True)
         return
 
     import torch
@@ -835,17 +914,14 @@ def main():
     K.lib()
     torch.cuda.set_device(d["local"])
     hbm_peak, tf_peak, peak_src = measured_peaks()
-    seed = 1234 + d["rank"]
     if paged:
-        reps = replicas_for(kind, batch, t // 2, mfmt, ifmt, args.replicas, 0, args.l2_factor)
         layer = PagedLayer(batch, t, heads, seed, reps)
     else:
-        reps = replicas_for(kind, batch, t, mfmt, ifmt, args.replicas, pool, args.l2_factor)
         layer = Layer(kind, batch, t, heads, seed, reps, mfmt, ifmt, pool=pool)
+    assert layer.alg_bytes() == alg
     res = time_layer(layer, args.steps, args.warmup, dist_max, d["local"], sample_clocks=(d["rank"] == 0))
     ms = res["total_ms"] / args.steps
     steps_per_s = d["world"] * 1e3 / ms            # whole job: every rank ran `steps` steps
-    alg = layer.alg_bytes()
     e2e_ms, e2e_eager_ms, h2d, d2h = time_e2e(layer, args.steps)
     e2e_ms, e2e_eager_ms = dist_max(e2e_ms), dist_max(e2e_eager_ms)
     e2e_v = d["world"] * args.steps * 1e3 / e2e_ms
@@ -911,19 +987,15 @@ def main():
     line = {"metric": METRIC, "value": round(steps_per_s, 2), "unit": "steps/s", "n_gpus": d["world"],
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": FMT_NAME[mfmt], "data": "synthetic",
-            "config": {"workload": wl_name, "batch_per_gpu": batch, "context": t, "heads": heads,
-                       "parallelism": f"dp{d['world']}",
-                       "l2": f"inputs larger than L2: {reps} cache replicas cycle, {alg / 1e6:.0f} MB read per step, "
-                             f"{reps * alg / 1e6:.0f} MB in all (>= 4 x the 126 MB L2)"},
+            "config": config,
             "hbm_gbs": round(alg / (ms * 1e-3) / 1e9, 1), "alg_bytes_per_step": alg,
             "per_layer_type": per_type, "roofline": roof,
             "e2e": {"value": round(e2e_v, 2), "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "eager_value": round(e2e_eager_v, 2),
-                    "method": "public API (dsv4kv_index_topk + dsv4kv_sparse/dense_decode) on pinned host buffers; "
-                              "per step an H2D of the queries and a D2H of the outputs, pipelined over upload / "
-                              "compute / download streams with double buffers; the calls and copies of all steps "
-                              "captured once into a CUDA graph and replayed (eager_value: the same steps issued "
-                              "from Python)"},
+                    "method": "public API (the layer's index and decode calls) on pinned host buffers; per "
+                              "step an H2D of the queries and a D2H of the outputs; steps alternate between two "
+                              "streams with their own buffers and workspaces, each replaying a CUDA graph of "
+                              "[H2D -> calls -> D2H] (eager_value: the same steps issued from Python)"},
             "gpu_launches": layer.launches_per_step() * args.steps,
             "clocks": res["clocks"]}
     if stack:
@@ -931,7 +1003,7 @@ def main():
     if bulk:
         line["bulk"] = bulk
     if d["rank"] == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(kind, batch, t, heads, args.cpu_budget)
+        line["cpu_baseline"] = cpu_baseline(kind, batch, t, heads, args.cpu_budget, t_seq)
     if d["rank"] == 0:
         print(json.dumps(line), flush=True)
     if _dist["on"]:
