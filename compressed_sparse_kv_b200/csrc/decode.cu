@@ -73,13 +73,14 @@ struct __align__(8) Ctl {
   uint64_t s_full[2];
   uint64_t s_free[2];
   uint64_t p_full[2];
-  uint64_t pv_done;
+  uint64_t pv_done[2];  // PV of the tiles that used P buffer 0 / 1
   uint64_t o_done;
   uint32_t tmem_base;
   volatile int abort;
   float alpha[64];
   float fin[64];
   float row_scale[kStages][kTileRows];
+  float row_ls[kStages][kTileRows];  // log2 of the row scale (-inf: no row)
   uint32_t vmask[kStages][4];  // row validity of a gathered tile, 16 rows per loader warp
   int32_t idx_s[kIdxSmem];     // the selected indices of this CTA's compressed tiles
   float rope_cs[kDim / 2];  // inverse-RoPE rotation of pair m: cos / sin of -t * theta_m
@@ -362,7 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ctl->s_free[s], 4);
       mbar_init(&ctl->p_full[s], 4);
     }
-    mbar_init(&ctl->pv_done, 1);
+    mbar_init(&ctl->pv_done[0], 1);
+    mbar_init(&ctl->pv_done[1], 1);
     mbar_init(&ctl->o_done, 1);
     ctl->abort = 0;
     fence_mbar_init();
@@ -436,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           mma_commit(&ctl->empty[stage]);
-          mma_commit(&ctl->pv_done);
+          mma_commit(&ctl->pv_done[pb]);
           ++next_pv;
           progressed = true;
         } else if (next_qk < nt && next_qk < next_pv + 2) {
@@ -528,9 +530,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             float ls = 0.f;
             bool sok = true;
             if (C::kRowScale) {
-              const float s = ctl->row_scale[stage][r];
-              sok = s > 0.f;
-              ls = sok ? __log2f(s) : 0.f;
+              sok = ctl->row_scale[stage][r] > 0.f;
+              ls = ctl->row_ls[stage][r];
             }
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
@@ -554,7 +555,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!C::kRowScale) ymax[hh] = tmax[hh];
         }
-        if (i >= 1) dead = !warp_wait(&ctl->pv_done, (i - 1) & 1, ctl, lane);
       }
       bool need = false;
       float alpha[2] = {1.f, 1.f};
@@ -571,6 +571,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (i >= 1 && named_bar_or(need)) {
+        // the accumulator is rescaled: PV(i-1) must have finished adding to it
+        if (!dead) dead = !warp_wait(&ctl->pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, ctl, lane);
         if (!dead && c2 == 0) {
           ctl->alpha[hd[0]] = alpha[0];
           ctl->alpha[hd[1]] = alpha[1];
@@ -596,6 +598,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         named_bar_sync();  // alpha[] is rewritten only after everyone read it
       }
+      // P buffer sb was last read by PV(i-2)
+      if (i >= 2 && !dead) dead = !warp_wait(&ctl->pv_done[sb], ((i - 2) >> 1) & 1, ctl, lane);
       if (dead) continue;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
@@ -606,9 +610,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int r = 8 * j + 2 * c2;
           float ya = x[hh][2 * j], yb = x[hh][2 * j + 1];
           if (C::kRowScale) {  // y = x + log2(s_r): the weight of the stored row carries its scale
-            const float sa = ctl->row_scale[stage][r], sb2 = ctl->row_scale[stage][r + 1];
-            ya = sa > 0.f ? ya + __log2f(sa) : -INFINITY;
-            yb = sb2 > 0.f ? yb + __log2f(sb2) : -INFINITY;
+            ya += ctl->row_ls[stage][r];
+            yb += ctl->row_ls[stage][r + 1];
           }
           const float wa = (m_o[hh] == -INFINITY) ? 0.f : fast_exp2(ya - m_o[hh]);
           const float wb = (m_o[hh] == -INFINITY) ? 0.f : fast_exp2(yb - m_o[hh]);
@@ -753,7 +756,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint8_t* codes = mine.from_win ? p.win_codes : p.comp_codes;
           const float* scales = static_cast<const float*>(mine.from_win ? p.win_scales : p.comp_scales);
           const float my_scale = (lane < 16 && mine.valid) ? scales[mine.row] : 0.f;
-          if (lane < 16) ctl->row_scale[stage][16 * lw + lane] = my_scale;
+          if (lane < 16) {
+            ctl->row_scale[stage][16 * lw + lane] = my_scale;
+            ctl->row_ls[stage][16 * lw + lane] = my_scale > 0.f ? __log2f(my_scale) : -INFINITY;
+          }
           uint4 rawb[kPerBody], rawr[kPerRope];
 #pragma unroll
           for (int i = 0; i < kPerBody; ++i) {
@@ -801,8 +807,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const uint8_t* codes = mine.from_win ? p.win_codes : p.comp_codes;
           const void* scales = mine.from_win ? p.win_scales : p.comp_scales;
-          if (C::kRowScale && lane < 16)
-            ctl->row_scale[stage][16 * lw + lane] = mine.valid ? static_cast<const float*>(scales)[mine.row] : 0.f;
+          if (C::kRowScale && lane < 16) {
+            const float sr = mine.valid ? static_cast<const float*>(scales)[mine.row] : 0.f;
+            ctl->row_scale[stage][16 * lw + lane] = sr;
+            ctl->row_ls[stage][16 * lw + lane] = sr > 0.f ? __log2f(sr) : -INFINITY;
+          }
           const int chunk = lane >> 2, u0 = (lane & 3) * 2;  // lane owns channels [16*lane, 16*lane+16)
           uint4 raw[16];
           uint32_t sgrp[16];
@@ -858,6 +867,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       store_partial(p, b, split, tmem, warp & 3, lane, kDim / 256, kDim / 128);
     }
   }
+  // every lane of a warp arrives together (lanes 1-31 of the TMA and MMA
+  // warps would otherwise reach the barrier ahead of their lane 0, and the
+  // warp count as arrived), so TMEM is freed only after all its users are done
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -1509,6 +1509,7 @@ struct IndexWs {
   uint32_t* hist;
   uint32_t* tail_ctr;  // claim counter of the bf16 score kernel's tail queue
   float* scores;
+  size_t scores_off;   // byte offset of the scores: everything before must be zero between calls
   size_t bytes;
 };
 
@@ -1526,6 +1527,7 @@ static IndexWs index_ws_layout(char* base, int batch, int64_t n, int k) {
   w.status = reinterpret_cast<uint32_t*>(take(16));
   w.hist = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * kHistBins * size_t(batch)));
   w.tail_ctr = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t)));
+  w.scores_off = off;
   w.scores = reinterpret_cast<float*>(take(sizeof(float) * size_t(batch) * size_t(score_stride(n))));
   w.bytes = off;
   return w;
@@ -1535,10 +1537,7 @@ size_t index_topk_ws_bytes(int batch, int64_t n, int k) { return index_ws_layout
 
 // Bytes at the start of the workspace that must be zero before a call (status
 // word, counters, histograms): everything before the scores.
-size_t index_topk_zero_prefix_bytes(int batch) {
-  const IndexWs w = index_ws_layout(nullptr, batch, 1, 1);
-  return size_t(reinterpret_cast<char*>(w.scores) - static_cast<char*>(nullptr));
-}
+size_t index_topk_zero_prefix_bytes(int batch) { return index_ws_layout(nullptr, batch, 1, 1).scores_off; }
 
 static dsv4kv_status index_fill_launch(int batch, int64_t n, int k, int32_t* idx_out, int32_t* count_out,
                                        cudaStream_t stream, const Ragged& rg, uint32_t* status) {

@@ -73,6 +73,8 @@ extern "C" __attribute__((visibility("default"))) dsv4kv_status dsv4kv_index_top
     // the score kernel's claim counter; a successful call leaves them zero,
     // but one that gave up may not have, so clear them.
     const size_t zero_bytes = index_topk_zero_prefix_bytes(batch);
+    if (zero_bytes <= kStatusBytes || zero_bytes > need)
+      return set_error(DSV4KV_ERR_UNSUPPORTED, "index_topk_noalloc: bad scratch layout (%zu bytes to clear)", zero_bytes);
     const cudaError_t e = cudaMemsetAsync(static_cast<char*>(ws) + kStatusBytes, 0, zero_bytes - kStatusBytes,
                                           static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess)
