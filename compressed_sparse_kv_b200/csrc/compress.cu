@@ -11,6 +11,10 @@
 // channels (two 16-byte bf16 loads per tap row), so a tap row is one fully
 // coalesced 1 KB read.  The K tap loads are unrolled by 4 to keep several
 // rows in flight; c4a entries overlap by 4 rows, which the L1/L2 absorb.
+// The rotation: the block computes rope_base^(-2m/rope_dim) / pi once per
+// pair m (shared memory); per entry, lane m computes the cos / sin of pair m
+// (the angle in units of pi reduced exactly modulo 2 in fp64, then sincospi)
+// and the lanes that own rotary channels take theirs by shuffles.
 #include <cmath>
 #include <cstdint>
 
@@ -22,6 +26,7 @@ namespace dsv4kv {
 namespace {
 
 constexpr int kWarpsPerBlock = 8;
+constexpr int kMaxRopePairs = 512;  // rope_dim <= 1024
 
 template <int PER>  // channels per lane (dim / 32)
 __global__ void __launch_bounds__(32 * kWarpsPerBlock)
@@ -29,6 +34,10 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock)
                     int stride, int64_t n_entries, int64_t pos0, int rope_dim, double rope_base, int out_fp32,
                     void* __restrict__ out) {
   constexpr int D = 32 * PER;
+  __shared__ double theta_pi[kMaxRopePairs];  // rope_base^(-2m/rope_dim) / pi
+  for (int m = threadIdx.x; m < rope_dim / 2; m += blockDim.x)
+    theta_pi[m] = pow(rope_base, -2.0 * double(m) / double(rope_dim)) / 3.141592653589793;
+  __syncthreads();
   const int lane = threadIdx.x & 31;
   const int b = blockIdx.y;
   const int64_t i = int64_t(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5);
@@ -59,21 +68,41 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock)
       acc[8 * v + 7] = fmaf(wb.w, bf16hi(x.w), acc[8 * v + 7]);
     }
   }
-  // RoPE at the block's first position (fp64 angle; the pair index m of
-  // channel c is (c - (D - rope_dim)) / 2).
+  // RoPE at the block's first position.  The pair index m of channel c is
+  // (c - (D - rope_dim)) / 2; the angle pos * theta_m in units of pi is
+  // reduced exactly modulo 2 (fp64) before sincospi.
   const int r0 = D - rope_dim;
-  if (c0 + PER > r0) {
-    const double pos = double(pos0 + int64_t(stride) * i);
+  const int pairs = rope_dim / 2;
+  const double pos = double(pos0 + int64_t(stride) * i);
+  auto rotation = [&](int m, float* cs, float* sn) {
+    const double ang = pos * theta_pi[m];
+    double sd, cd;
+    sincospi(ang - 2.0 * rint(0.5 * ang), &sd, &cd);
+    *cs = float(cd);
+    *sn = float(sd);
+  };
+  if (pairs <= 32) {
+    // lane m computes pair m; the owners of rotary channels fetch theirs
+    float cs_m = 1.f, sn_m = 0.f;
+    if (lane < pairs) rotation(lane, &cs_m, &sn_m);
+#pragma unroll
+    for (int e = 0; e < PER; e += 2) {
+      const int c = c0 + e;
+      const int m = c >= r0 ? (c - r0) >> 1 : 0;
+      const float cs = __shfl_sync(kFull, cs_m, m & 31), sn = __shfl_sync(kFull, sn_m, m & 31);
+      if (c >= r0) {
+        const float x = acc[e], y = acc[e + 1];
+        acc[e] = float(double(x) * cs - double(y) * sn);
+        acc[e + 1] = float(double(x) * sn + double(y) * cs);
+      }
+    }
+  } else if (c0 + PER > r0) {
 #pragma unroll
     for (int e = 0; e < PER; e += 2) {
       const int c = c0 + e;
       if (c >= r0) {
-        const int m = (c - r0) >> 1;
-        // angle pos*theta in units of pi, reduced exactly modulo 2 before sincospi
-        const double ang = pos * (pow(rope_base, -2.0 * double(m) / double(rope_dim)) / 3.141592653589793);
-        const double xr = ang - 2.0 * rint(0.5 * ang);
-        double sn, cs;
-        sincospi(xr, &sn, &cs);
+        float cs, sn;
+        rotation((c - r0) >> 1, &cs, &sn);
         const float x = acc[e], y = acc[e + 1];
         acc[e] = float(double(x) * cs - double(y) * sn);
         acc[e + 1] = float(double(x) * sn + double(y) * cs);

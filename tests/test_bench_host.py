@@ -31,3 +31,22 @@ def test_replicas_hold_four_l2():
 
 def test_flops_and_launch_counts():
     assert B.FMT_NAME[3] == "fp8+bf16rope" and B.ROW_BYTES[3] == 576 + 4
+
+
+def test_ragged_lengths_are_seeded_and_bounded():
+    a, b = B.ragged_lengths(32, 131072, 7), B.ragged_lengths(32, 131072, 7)
+    assert (a == b).all() and a.min() >= 65536 and a.max() <= 131072
+
+
+def test_reference_arm_times_the_steps_it_reports():
+    """The oracle arm runs `warmup` + `steps` steps of the given workload (here
+    a small one, whole steps) and prints the config it was handed unchanged."""
+    import argparse
+    args = argparse.Namespace(steps=2, warmup=1, gpus=1)
+    cfg = {"workload": "tiny", "batch_per_gpu": 2}
+    line = B.reference_arm(args, "c4a", 2, 4224, 4, cfg, "tiny")
+    assert line["impl"] == "reference" and line["config"] is cfg
+    assert line["steps"] == 2 and line["warmup"] == 1 and line["sequences_per_step"] == 2
+    assert line["value"] > 0 and abs(line["ms_per_step"] * line["value"] - 1e3) < 1e-6 * 1e3
+    dense = B.reference_arm(args, "c128a", 2, 128 * 40, 4, cfg, "tiny")
+    assert dense["value"] > 0
