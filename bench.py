@@ -179,10 +179,11 @@ class PagedLayer:
         dev = "cuda"
         rng = np.random.default_rng(seed + 1)
 
-        def tables(counts):
+        def tables(counts, most):
+            # `most`: the rows a sequence of length t_max may have (the table's row pitch covers them)
             need = (counts + PAGE_ROWS - 1) // PAGE_ROWS
             perm = rng.permutation(int(need.sum())).astype(np.int32)
-            tab = np.full((batch, max(1, int(need.max()))), -1, np.int32)
+            tab = np.full((batch, max(1, (most + PAGE_ROWS - 1) // PAGE_ROWS)), -1, np.int32)
             o = 0
             for b, m in enumerate(need):
                 tab[b, :m] = perm[o:o + m]
@@ -193,9 +194,10 @@ class PagedLayer:
         self.reps = []
         for r in range(replicas):
             keys = WL.keys_for(seed, 1000 * r + layer_id)
-            ct, cp = tables(self.n_seq)
-            kt, kp = tables(self.n_seq)
-            wt, wp = tables(w_seq)
+            n_most = max(0, (self.t_max - self.window) // 4)
+            ct, cp = tables(self.n_seq, n_most)
+            kt, kp = tables(self.n_seq, n_most)
+            wt, wp = tables(w_seq, self.window)
             comp = G.normal_bf16_(torch.empty(cp * PAGE_ROWS, 512, dtype=torch.bfloat16, device=dev), keys["comp"])
             win = G.normal_bf16_(torch.empty(wp * PAGE_ROWS, 512, dtype=torch.bfloat16, device=dev), keys["win"])
             kidx = G.int_bf16_(torch.empty(kp * PAGE_ROWS, 128, dtype=torch.bfloat16, device=dev), keys["kidx"])
@@ -863,6 +865,8 @@ def main():
                     help="extra per-layer-type workloads (comma list, 'none' = none)")
     ap.add_argument("--no-stack", action="store_true", help="skip the 61-layer stack step")
     ap.add_argument("--no-bulk", action="store_true", help="skip compressor/quantiser throughput")
+    ap.add_argument("--stack-only", action="store_true",
+                    help="time only the 61-layer stack step (--steps replays) and print its figures")
     ap.add_argument("--replicas", type=int, default=2, help="minimum cache replicas (raised until they hold 4x L2)")
     ap.add_argument("--l2-factor", type=int, default=4,
                     help="replicas hold at least this many L2 sizes (0 only for small profiling runs)")
@@ -913,6 +917,11 @@ def main():
     import compressed_sparse_kv_b200 as K
     K.lib()
     torch.cuda.set_device(d["local"])
+    if args.stack_only:
+        st = time_stack(args.steps, args.warmup, seed + 7, dist_max)
+        if d["rank"] == 0:
+            print(json.dumps({"stack": st}), flush=True)
+        return
     hbm_peak, tf_peak, peak_src = measured_peaks()
     if paged:
         layer = PagedLayer(batch, t, heads, seed, reps)

@@ -80,7 +80,8 @@ struct __align__(8) Ctl {
   float alpha[64];
   float fin[64];
   float row_scale[kStages][kTileRows];
-  float row_ls[kStages][kTileRows];  // log2 of the row scale (-inf: no row)
+  float row_ls[kStages][kTileRows];   // log2 of the row scale (-inf: no row)
+  float row_inv[kStages][kTileRows];  // 1 / row scale (0: no row)
   uint32_t vmask[kStages][4];  // row validity of a gathered tile, 16 rows per loader warp
   int32_t idx_s[kIdxSmem];     // the selected indices of this CTA's compressed tiles
   float rope_cs[kDim / 2];  // inverse-RoPE rotation of pair m: cos / sin of -t * theta_m
@@ -334,6 +335,137 @@ __device__ __forceinline__ void store_partial(const Params& p, int b, int split,
     }
   }
 }
+
+// The loader warps' part of one quantised tile: warp lw owns rows 16 lw ..
+// 16 lw + 15.  fetch() resolves the rows and issues every global load of the
+// warp's part into registers; put() (once the stage is free) stores the row
+// mask and scales and the rows dequantised to f16 into the 128-byte-swizzled
+// tile.  The loaders fetch tile i + 1 right after putting tile i, so its
+// loads are in flight while the stage it needs is still in use.
+template <int FMT>
+struct QuantLoad {
+  static constexpr bool kRowScale = Cfg<FMT>::kRowScale;
+  static constexpr bool kRope = FMT == DSV4KV_FP8_E4M3_ROW_ROPE_BF16;
+  // fp8 rows with bf16 rotary channels: rows of kDim + 64 bytes, 28 chunks of
+  // 16 fp8 channels then 8 chunks of 8 bf16 rotary channels; the warp's 16
+  // rows hold 448 fp8 chunks (14 per lane) and 128 rotary chunks (4 per lane)
+  static constexpr int kBodyChunks = (kDim - 64) / 16, kRopeChunks = 64 / 8;
+  static constexpr int kPerBody = 16 * kBodyChunks / 32, kPerRope = 16 * kRopeChunks / 32;
+  static constexpr int kRaw = kRope ? kPerBody + kPerRope : 16;
+  uint4 raw[kRaw];
+  uint32_t sgrp[16];  // fp4: the E4M3 scale of this lane's 16-channel group, per row
+  float my_scale;     // row-scale formats: the scale of row 16 lw + lane (lanes < 16)
+  uint32_t vb;        // rows of the warp's part that exist
+
+  __device__ __forceinline__ void fetch(const Params& p, const Seq& q, int b, int T, int lw, int lane,
+                                        const int32_t* idx_s, int slot0) {
+    const RowSrc mine = row_source(p, q, b, T, 16 * lw + (lane & 15), idx_s, slot0);
+    vb = __ballot_sync(kFull, mine.valid) & 0xffffu;
+    const uint8_t* codes = mine.from_win ? p.win_codes : p.comp_codes;
+    const void* scales = mine.from_win ? p.win_scales : p.comp_scales;
+    my_scale = 0.f;
+    if (kRowScale && lane < 16 && mine.valid) my_scale = static_cast<const float*>(scales)[mine.row];
+    if constexpr (kRope) {
+#pragma unroll
+      for (int i = 0; i < kPerBody; ++i) {
+        const int g = lane + 32 * i, jr = g / kBodyChunks, cr = g % kBodyChunks;
+        const int64_t row = __shfl_sync(kFull, mine.row, jr);
+        raw[i] = (vb >> jr) & 1u ? ld_stream_v4(codes + size_t(row) * (kDim + 64) + 16 * cr) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int i = 0; i < kPerRope; ++i) {
+        const int g = lane + 32 * i, jr = g / kRopeChunks, cr = g % kRopeChunks;
+        const int64_t row = __shfl_sync(kFull, mine.row, jr);
+        raw[kPerBody + i] = (vb >> jr) & 1u ? ld_stream_v4(codes + size_t(row) * (kDim + 64) + (kDim - 64) + 16 * cr)
+                                            : make_uint4(0, 0, 0, 0);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int64_t row = __shfl_sync(kFull, mine.row, j);
+        const bool valid = (vb >> j) & 1u;
+        if (kRowScale) {  // lane owns channels [16 lane, 16 lane + 16)
+          raw[j] = valid ? ld_stream_v4(codes + size_t(row) * kDim + 16 * lane) : make_uint4(0, 0, 0, 0);
+        } else if (valid) {
+          const uint2 c8 = *reinterpret_cast<const uint2*>(codes + size_t(row) * (kDim / 2) + 8 * lane);
+          raw[j] = make_uint4(c8.x, c8.y, 0, 0);
+          sgrp[j] = static_cast<const uint8_t*>(scales)[size_t(row) * (kDim / 16) + lane];
+        } else {
+          raw[j] = make_uint4(0, 0, 0, 0);
+          sgrp[j] = 0;
+        }
+      }
+    }
+  }
+
+  __device__ __forceinline__ void put(Ctl* ctl, int stage, uint8_t* tile, int lw, int lane) const {
+    if (lane == 0) ctl->vmask[stage][lw] = vb;
+    if (kRowScale && lane < 16) {
+      const float sr = my_scale;
+      ctl->row_scale[stage][16 * lw + lane] = sr;
+      ctl->row_ls[stage][16 * lw + lane] = sr > 0.f ? __log2f(sr) : -INFINITY;
+      ctl->row_inv[stage][16 * lw + lane] = sr > 0.f ? __frcp_rn(sr) : 0.f;
+    }
+    if constexpr (kRope) {
+      // one conversion loop per chunk kind for the whole warp; the rotary
+      // channels are stored as f16 of value / scale so that the row scale
+      // folds into the softmax weights exactly as for fp8 rows
+#pragma unroll
+      for (int i = 0; i < kPerBody; ++i) {
+        const int g = lane + 32 * i, jr = g / kBodyChunks, cr = g % kBodyChunks;
+        const int r = 16 * lw + jr, ch = 16 * cr, u = (ch & 63) >> 3;
+        const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+        uint32_t hv[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          hv[2 * e] = e4m3x2_to_f16x2(w[e] & 0xffffu);
+          hv[2 * e + 1] = e4m3x2_to_f16x2(w[e] >> 16);
+        }
+        uint8_t* line = tile + (ch >> 6) * kChunkBytes + r * 128;
+        *reinterpret_cast<uint4*>(line + ((u ^ (r & 7)) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        *reinterpret_cast<uint4*>(line + (((u + 1) ^ (r & 7)) << 4)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+      }
+#pragma unroll
+      for (int i = 0; i < kPerRope; ++i) {
+        const int g = lane + 32 * i, jr = g / kRopeChunks, cr = g % kRopeChunks;
+        const int r = 16 * lw + jr, ch = (kDim - 64) + 8 * cr, u = (ch & 63) >> 3;
+        const float sr = __shfl_sync(kFull, my_scale, jr);
+        const float inv = sr > 0.f ? __frcp_rn(sr) : 0.f;
+        const uint4 x = raw[kPerBody + i];
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t hv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) hv[e] = f32x2_to_f16x2_sat(bf16lo(w[e]) * inv, bf16hi(w[e]) * inv);
+        uint8_t* line = tile + (ch >> 6) * kChunkBytes + r * 128;
+        *reinterpret_cast<uint4*>(line + ((u ^ (r & 7)) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+      }
+    } else {
+      const int chunk = lane >> 2, u0 = (lane & 3) * 2;  // lane owns channels [16 lane, 16 lane + 16)
+      uint8_t* ctile = tile + chunk * kChunkBytes;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int r = 16 * lw + j;
+        uint32_t hv[8];
+        if (kRowScale) {
+          const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            hv[2 * e] = e4m3x2_to_f16x2(w[e] & 0xffffu);
+            hv[2 * e + 1] = e4m3x2_to_f16x2(w[e] >> 16);
+          }
+        } else {
+          const uint32_t s2 = e4m3x2_to_f16x2(sgrp[j] | (sgrp[j] << 8));  // (scale, scale) as f16x2
+          const uint32_t w[2] = {raw[j].x, raw[j].y};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) hv[e] = hmul2(e2m1x2_to_f16x2((w[e >> 2] >> (8 * (e & 3))) & 0xffu), s2);
+        }
+        uint8_t* line = ctile + r * 128;
+        *reinterpret_cast<uint4*>(line + ((u0 ^ (r & 7)) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        *reinterpret_cast<uint4*>(line + (((u0 + 1) ^ (r & 7)) << 4)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+      }
+    }
+  }
+};
 
 template <int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -605,6 +737,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int hh = 0; hh < 2; ++hh) {
         const int h = hd[hh];
         uint8_t* prow = sP + sb * kPBytes + (h >> 3) * 1024 + (h & 7) * 128 + 4 * c2;
+        // row-scale formats: sum_r w_r / s_r = sum_r 2^(x_r - m_o), so the
+        // denominator's terms 2^(x_r - m_l) need no exponential of their own
+        float lw_sum = 0.f;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int r = 8 * j + 2 * c2;
@@ -617,13 +752,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float wb = (m_o[hh] == -INFINITY) ? 0.f : fast_exp2(yb - m_o[hh]);
           const uint32_t packed = pack_p(wa, wb, C::kQuant);
           if (C::kRowScale) {
-            if (m_l[hh] != -INFINITY) l[hh] += fast_exp2(x[hh][2 * j] - m_l[hh]) + fast_exp2(x[hh][2 * j + 1] - m_l[hh]);
+            lw_sum = fmaf(wa, ctl->row_inv[stage][r], fmaf(wb, ctl->row_inv[stage][r + 1], lw_sum));
           } else {
             l[hh] += p_lo(packed, C::kQuant) + p_hi(packed, C::kQuant);  // the weights the MMA uses
           }
           // rows 8j .. 8j+7 form 16-byte chunk j of the head's 128-byte row (128-byte swizzle)
           *reinterpret_cast<uint32_t*>(prow + ((j ^ (h & 7)) << 4)) = packed;
         }
+        if (C::kRowScale && lw_sum > 0.f) l[hh] += lw_sum * fast_exp2(m_o[hh] - m_l[hh]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -699,7 +835,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nslots = p.idx ? min(max(0, min(p.k, (t0 + nt) * kTileRows) - slot0), kIdxSmem) : 0;
     for (int i = threadIdx.x - 192; i < nslots; i += 128) ctl->idx_s[i] = __ldg(p.idx + size_t(b) * p.k + slot0 + i);
     loader_bar_sync();
-    if (C::kQuant) {
+    if constexpr (C::kQuant) {
+      // the first tile's loads go out before Q's conversion waits for Q
+      QuantLoad<FMT> ql;
+      if (nt > 0) ql.fetch(p, sq, b, t0, lw, lane, ctl->idx_s, slot0);
       // Q: bf16 -> f16 in place (saturating), once per CTA
       if (warp_wait(&ctl->q_full, 0, ctl, lane)) {
         for (int v = threadIdx.x - 192; v < kQBytes / 16; v += 128) {
@@ -712,20 +851,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->q_ready);
       }
-    }
-    // rows: warp lw covers rows 16*lw .. 16*lw+15 of every tile
-    for (int i = 0; i < nt; ++i) {
-      const int T = t0 + i, stage = i % kStages;
-      if (i >= kStages && !warp_wait(&ctl->empty[stage], ((i / kStages) - 1) & 1, ctl, lane)) break;
-      uint8_t* tile = sR + stage * kTileBytes;
-      if (!C::kQuant && tile_tma(p, sq, b, T)) {
-        // warp 0 brings this tile by TMA
-      } else {
-        // lane j < 16 resolves row 16*lw + j; every lane reads all 16 answers
-        const RowSrc mine = row_source(p, sq, b, T, 16 * lw + (lane & 15), ctl->idx_s, slot0);
-        const uint32_t vb = __ballot_sync(kFull, mine.valid) & 0xffffu;
-        if (lane == 0) ctl->vmask[stage][lw] = vb;
-        if (!C::kQuant) {
+      for (int i = 0; i < nt; ++i) {
+        const int stage = i % kStages;
+        if (i >= kStages && !warp_wait(&ctl->empty[stage], ((i / kStages) - 1) & 1, ctl, lane)) break;
+        ql.put(ctl, stage, sR + stage * kTileBytes, lw, lane);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->full[stage]);
+        if (i + 1 < nt) ql.fetch(p, sq, b, t0 + i + 1, lw, lane, ctl->idx_s, slot0);
+      }
+    } else {
+      // rows: warp lw covers rows 16*lw .. 16*lw+15 of every tile
+      for (int i = 0; i < nt; ++i) {
+        const int T = t0 + i, stage = i % kStages;
+        if (i >= kStages && !warp_wait(&ctl->empty[stage], ((i / kStages) - 1) & 1, ctl, lane)) break;
+        uint8_t* tile = sR + stage * kTileBytes;
+        if (!tile_tma(p, sq, b, T)) {
+          // lane j < 16 resolves row 16*lw + j; every lane reads all 16 answers
+          const RowSrc mine = row_source(p, sq, b, T, 16 * lw + (lane & 15), ctl->idx_s, slot0);
+          const uint32_t vb = __ballot_sync(kFull, mine.valid) & 0xffffu;
+          if (lane == 0) ctl->vmask[stage][lw] = vb;
           // gathered bf16 rows: 16-byte cp.async into the 128-byte-swizzled tile
           // (rows that do not exist are zero-filled without a read)
           const uint8_t* base = static_cast<const uint8_t*>(mine.from_win ? p.win_codes : p.comp_codes);
@@ -743,123 +888,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           cp_async_wait_all();
-        } else if constexpr (FMT == DSV4KV_FP8_E4M3_ROW_ROPE_BF16) {
-          // rows of kDim + 64 bytes: 28 chunks of 16 fp8 channels (16 bytes),
-          // then 8 chunks of 8 bf16 rotary channels.  The warp's 16 rows hold
-          // 448 fp8 chunks (14 per lane) and 128 rotary chunks (4 per lane);
-          // all 18 loads of a lane are issued before any is converted, and
-          // each conversion loop has one chunk kind for the whole warp.  The
-          // rotary channels are stored as f16 of value / scale so that the
-          // row scale folds into the softmax weights exactly as for fp8 rows.
-          constexpr int kBodyChunks = (kDim - 64) / 16, kRopeChunks = 64 / 8;
-          constexpr int kPerBody = 16 * kBodyChunks / 32, kPerRope = 16 * kRopeChunks / 32;
-          const uint8_t* codes = mine.from_win ? p.win_codes : p.comp_codes;
-          const float* scales = static_cast<const float*>(mine.from_win ? p.win_scales : p.comp_scales);
-          const float my_scale = (lane < 16 && mine.valid) ? scales[mine.row] : 0.f;
-          if (lane < 16) {
-            ctl->row_scale[stage][16 * lw + lane] = my_scale;
-            ctl->row_ls[stage][16 * lw + lane] = my_scale > 0.f ? __log2f(my_scale) : -INFINITY;
-          }
-          uint4 rawb[kPerBody], rawr[kPerRope];
-#pragma unroll
-          for (int i = 0; i < kPerBody; ++i) {
-            const int g = lane + 32 * i, jr = g / kBodyChunks, cr = g % kBodyChunks;
-            const int64_t row = __shfl_sync(kFull, mine.row, jr);
-            const bool valid = __shfl_sync(kFull, mine.valid, jr);
-            rawb[i] = valid ? ld_stream_v4(codes + size_t(row) * (kDim + 64) + 16 * cr) : make_uint4(0, 0, 0, 0);
-          }
-#pragma unroll
-          for (int i = 0; i < kPerRope; ++i) {
-            const int g = lane + 32 * i, jr = g / kRopeChunks, cr = g % kRopeChunks;
-            const int64_t row = __shfl_sync(kFull, mine.row, jr);
-            const bool valid = __shfl_sync(kFull, mine.valid, jr);
-            rawr[i] = valid ? ld_stream_v4(codes + size_t(row) * (kDim + 64) + (kDim - 64) + 16 * cr)
-                            : make_uint4(0, 0, 0, 0);
-          }
-#pragma unroll
-          for (int i = 0; i < kPerBody; ++i) {
-            const int g = lane + 32 * i, jr = g / kBodyChunks, cr = g % kBodyChunks;
-            const int r = 16 * lw + jr, ch = 16 * cr, u = (ch & 63) >> 3;
-            const uint32_t w[4] = {rawb[i].x, rawb[i].y, rawb[i].z, rawb[i].w};
-            uint32_t hv[8];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              hv[2 * e] = e4m3x2_to_f16x2(w[e] & 0xffffu);
-              hv[2 * e + 1] = e4m3x2_to_f16x2(w[e] >> 16);
-            }
-            uint8_t* line = tile + (ch >> 6) * kChunkBytes + r * 128;
-            *reinterpret_cast<uint4*>(line + ((u ^ (r & 7)) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-            *reinterpret_cast<uint4*>(line + (((u + 1) ^ (r & 7)) << 4)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
-          }
-#pragma unroll
-          for (int i = 0; i < kPerRope; ++i) {
-            const int g = lane + 32 * i, jr = g / kRopeChunks, cr = g % kRopeChunks;
-            const int r = 16 * lw + jr, ch = (kDim - 64) + 8 * cr, u = (ch & 63) >> 3;
-            const float sr = __shfl_sync(kFull, my_scale, jr);
-            const float inv = sr > 0.f ? __frcp_rn(sr) : 0.f;
-            const uint32_t w[4] = {rawr[i].x, rawr[i].y, rawr[i].z, rawr[i].w};
-            uint32_t hv[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) hv[e] = f32x2_to_f16x2_sat(bf16lo(w[e]) * inv, bf16hi(w[e]) * inv);
-            uint8_t* line = tile + (ch >> 6) * kChunkBytes + r * 128;
-            *reinterpret_cast<uint4*>(line + ((u ^ (r & 7)) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-          }
-        } else {
-          const uint8_t* codes = mine.from_win ? p.win_codes : p.comp_codes;
-          const void* scales = mine.from_win ? p.win_scales : p.comp_scales;
-          if (C::kRowScale && lane < 16) {
-            const float sr = mine.valid ? static_cast<const float*>(scales)[mine.row] : 0.f;
-            ctl->row_scale[stage][16 * lw + lane] = sr;
-            ctl->row_ls[stage][16 * lw + lane] = sr > 0.f ? __log2f(sr) : -INFINITY;
-          }
-          const int chunk = lane >> 2, u0 = (lane & 3) * 2;  // lane owns channels [16*lane, 16*lane+16)
-          uint4 raw[16];
-          uint32_t sgrp[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int64_t row = __shfl_sync(kFull, mine.row, j);
-            const bool valid = __shfl_sync(kFull, mine.valid, j);
-            if (C::kRowScale) {
-              raw[j] = valid ? ld_stream_v4(codes + size_t(row) * kDim + 16 * lane) : make_uint4(0, 0, 0, 0);
-              sgrp[j] = 0;
-            } else {
-              if (valid) {
-                const uint2 c8 = *reinterpret_cast<const uint2*>(codes + size_t(row) * (kDim / 2) + 8 * lane);
-                raw[j] = make_uint4(c8.x, c8.y, 0, 0);
-                sgrp[j] = static_cast<const uint8_t*>(scales)[size_t(row) * (kDim / 16) + lane];
-              } else {
-                raw[j] = make_uint4(0, 0, 0, 0);
-                sgrp[j] = 0;
-              }
-            }
-          }
-          uint8_t* ctile = tile + chunk * kChunkBytes;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int r = 16 * lw + j;
-            uint32_t hv[8];
-            if (C::kRowScale) {
-              const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                hv[2 * e] = e4m3x2_to_f16x2(w[e] & 0xffffu);
-                hv[2 * e + 1] = e4m3x2_to_f16x2(w[e] >> 16);
-              }
-            } else {
-              const uint32_t s2 = e4m3x2_to_f16x2(sgrp[j] | (sgrp[j] << 8));  // (scale, scale) as f16x2
-              const uint32_t w[2] = {raw[j].x, raw[j].y};
-#pragma unroll
-              for (int e = 0; e < 8; ++e) hv[e] = hmul2(e2m1x2_to_f16x2((w[e >> 2] >> (8 * (e & 3))) & 0xffu), s2);
-            }
-            uint8_t* line = ctile + r * 128;
-            *reinterpret_cast<uint4*>(line + ((u0 ^ (r & 7)) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-            *reinterpret_cast<uint4*>(line + (((u0 + 1) ^ (r & 7)) << 4)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
-          }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
+        // (a TMA tile is brought by warp 0)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->full[stage]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->full[stage]);
     }
     // the other half of the partial O^T (this warp's TMEM lane quarter is warp % 4)
     if (p.splits > 1 && warp_wait(&ctl->o_done, 0, ctl, lane)) {

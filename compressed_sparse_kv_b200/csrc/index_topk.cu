@@ -285,25 +285,31 @@ __device__ __forceinline__ void e2m1x8_unpack(uint32_t w, uint32_t (&h)[4]) {
       : "r"(w));
 }
 
-__device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
-  // exact: E4M3 bits placed in a binary32 with the exponent rebased by 2^120
-  const uint32_t mag = (c & 0x7fu) << 20;
-  const float v = __uint_as_float(mag) * 0x1p120f;
-  return (c & 0x80u) ? -v : v;
-}
-
 __device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t d;
   asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
-__device__ __forceinline__ float f16x2_sum(uint32_t h) {
-  float lo, hi;
+// sum_g scale_g * (even_g + odd_g) over the two 16-channel groups of a lane:
+// acc0 / acc1 are the f16x2 (even, odd) channel sums of groups 0 / 1 and s2
+// their two E4M3 scale bytes (group 0 in the low byte).  The halves are added
+// in f16 (exact while the sums are multiples of 0.5 below 1024, as for the
+// integer-valued keys of the indexer), the scales converted by one cvt, the
+// products taken in fp32.
+__device__ __forceinline__ float scaled_group_sums(uint32_t acc0, uint32_t acc1, uint32_t s2) {
+  uint32_t ev, od, t, sc;
+  asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(ev) : "r"(acc0), "r"(acc1));  // (even0, even1)
+  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(od) : "r"(acc0), "r"(acc1));  // (odd0, odd1)
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(t) : "r"(ev), "r"(od));
+  asm("{\n\t.reg .b16 b;\n\tcvt.u16.u32 b, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, b;\n\t}" : "=r"(sc) : "r"(s2));
+  float t0, t1, s0, s1;
   asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
-      : "=f"(lo), "=f"(hi)
-      : "r"(h));
-  return lo + hi;
+      : "=f"(t0), "=f"(t1) : "r"(t));
+  asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+      : "=f"(s0), "=f"(s1) : "r"(sc));
+  return fmaf(t1, s1, t0 * s0);
 }
+
 __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
   uint32_t d;
   asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(d) : "f"(lo), "f"(hi));
@@ -357,7 +363,7 @@ __device__ __forceinline__ void score_segment_fp4(const uint16_t* __restrict__ q
           else acc1 = hfma2(qp[4 * wi + by], h[by], acc1);
         }
       }
-      p[u] = f16x2_sum(acc0) * e4m3_to_f32(s2[u] & 0xffu) + f16x2_sum(acc1) * e4m3_to_f32(s2[u] >> 8);
+      p[u] = scaled_group_sums(acc0, acc1, s2[u]);
     }
     // reduce over the 4 lanes of the quad: 4 values -> transposing butterfly
     const bool bb1 = l4 & 2, bb0 = l4 & 1;
@@ -880,7 +886,7 @@ __global__ void __launch_bounds__(256) index_score_paged(const uint16_t* __restr
             else acc1 = hfma2(qp[4 * wi + by], h[by], acc1);
           }
         }
-        pr[u] = f16x2_sum(acc0) * e4m3_to_f32(s2[u] & 0xffu) + f16x2_sum(acc1) * e4m3_to_f32(s2[u] >> 8);
+        pr[u] = scaled_group_sums(acc0, acc1, s2[u]);
       }
       const bool bb1 = l4 & 2, bb0 = l4 & 1;
       float k2[2];
@@ -1377,7 +1383,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
             else acc1 = hfma2(qp[4 * wi + by], h[by], acc1);
           }
         }
-        float sc = f16x2_sum(acc0) * e4m3_to_f32(s2[u] & 0xffu) + f16x2_sum(acc1) * e4m3_to_f32(s2[u] >> 8);
+        float sc = scaled_group_sums(acc0, acc1, s2[u]);
         sc += __shfl_xor_sync(kFull, sc, 1);
         sc += __shfl_xor_sync(kFull, sc, 2);
         sc += 0.0f;
