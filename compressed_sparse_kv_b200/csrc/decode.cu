@@ -524,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ TMA: Q and contiguous tiles
     if (lane == 0) {
       mbar_arrive_expect_tx(&ctl->q_full, kQBytes);
-      for (int c = 0; c < kChunks; ++c) tma_load_3d(sQ + c * kChunkBytes, &tm_q, &ctl->q_full, c * 64, 0, b);
+      tma_load_4d(sQ, &tm_q, &ctl->q_full, 0, 0, 0, b);  // all 8 channel chunks in one box
       int issued = 0;
       for (int i = 0; i < nt; ++i) {
         const int T = t0 + i, stage = i % kStages;
@@ -535,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int32_t row0 = int32_t(s0.row);
           mbar_arrive_expect_tx(&ctl->full[stage], kTileBytes);
           uint8_t* dst = sR + stage * kTileBytes;
-          for (int c = 0; c < kChunks; ++c) tma_load_2d(dst + c * kChunkBytes, tm, &ctl->full[stage], c * 64, row0);
+          tma_load_3d(dst, tm, &ctl->full[stage], 0, row0, 0);  // 64 rows x all 8 channel chunks
         } else {
           mbar_arrive(&ctl->full[stage]);
         }
@@ -1257,9 +1257,16 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
   if (ws_bytes < w.bytes) return set_error(DSV4KV_ERR_WORKSPACE, "decode: workspace too small");
 
   CUtensorMap tq, tc, tw;
-  if (!encode_tmap_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.q, kDim, uint64_t(a.heads), uint64_t(a.batch),
-                      uint64_t(kDim) * 2, uint64_t(a.heads) * kDim * 2, 64, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B))
-    return set_error(DSV4KV_ERR_INVALID_ARG, "decode: cannot encode the query tensor map");
+  // One box brings a whole operand in the layout the MMAs read: dimensions
+  // (64 channels, rows, 8 channel chunks[, sequence]) land chunk-major, 64
+  // rows x 128 bytes (128-byte swizzle) per chunk.
+  {
+    const uint64_t dims[4] = {64, uint64_t(a.heads), uint64_t(kChunks), uint64_t(a.batch)};
+    const uint64_t strides[3] = {uint64_t(kDim) * 2, 128, uint64_t(a.heads) * kDim * 2};
+    const uint32_t box[4] = {64, 64, uint32_t(kChunks), 1};
+    if (!encode_tmap_nd(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return set_error(DSV4KV_ERR_INVALID_ARG, "decode: cannot encode the query tensor map");
+  }
   const dsv4kv_cache& cc = a.comp;
   // rows a tensor map spans: the batch of dense caches, or a pool
   auto total_rows = [&](const dsv4kv_cache& c, const PageDesc& pg) -> uint64_t {
@@ -1268,13 +1275,17 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
   };
   if (fmt == DSV4KV_BF16) {
     // contiguous row runs: boxes of 64 channels x 64 rows, 128-byte swizzle
+    auto rows_map = [&](CUtensorMap* m, const void* base, uint64_t rows) {
+      const uint64_t dims[3] = {64, rows, uint64_t(kChunks)};
+      const uint64_t strides[2] = {uint64_t(kDim) * 2, 128};
+      const uint32_t box[3] = {64, uint32_t(kTileRows), uint32_t(kChunks)};
+      return encode_tmap_nd(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    };
     const void* comp_base = cc.codes ? cc.codes : a.win.codes;
-    if (!encode_tmap_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, comp_base, kDim, total_rows(cc, a.comp_pg),
-                        uint64_t(kDim) * 2, 64, kTileRows, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!rows_map(&tc, comp_base, total_rows(cc, a.comp_pg)))
       return set_error(DSV4KV_ERR_INVALID_ARG, "decode: cannot encode the compressed-cache tensor map");
     const void* win_base = a.win.codes ? a.win.codes : comp_base;
-    if (!encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, win_base, kDim, total_rows(a.win, a.win_pg),
-                        uint64_t(kDim) * 2, 64, kTileRows, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!rows_map(&tw, win_base, total_rows(a.win, a.win_pg)))
       return set_error(DSV4KV_ERR_INVALID_ARG, "decode: cannot encode the window tensor map");
   } else {
     tc = tq;  // unused: quantised rows are loaded by the loader warps

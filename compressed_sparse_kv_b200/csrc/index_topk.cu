@@ -161,6 +161,7 @@ constexpr int kTailUnit = 32;  // two groups of 16 keys (8 per half-warp)
 // the c4a B=32 step (per-call score time / whole step): 0 % 49.1 / 93.7 us,
 // 8 % 47.5 / 94.1, 15 % 47.1 / 92.1, 25 % 48.5 / 90.0, 35 % 49.7 / 91.1.
 constexpr int kTailPct = 25;
+constexpr int kTailMinBatch = 16;
 
 __device__ __forceinline__ void score_tail_bf16(const uint16_t* __restrict__ qidx, const uint16_t* __restrict__ keys,
                                                 int64_t key_rows, int64_t n, int64_t n_h, int batch,
@@ -697,16 +698,17 @@ __device__ void select_by_scan(const float* __restrict__ sc, int64_t n, uint32_t
 // ------------------------------------------------------------------ paged, ragged scoring
 // Sequence b of a ragged batch has n_b = max(0, floor((t_b - window) /
 // stride)) keys, stored in pages of a pool: key i is pool row table[b][i /
-// page] * page + i % page.  Its keys are cut into units of kPagedUnit
-// consecutive keys (a page holds whole units); the units of all sequences
-// are numbered sequence after sequence (a sequence with n_b <= k has none: it
-// needs no scores) and handed out one per warp claim from one counter, the
-// next claim issued while the current unit is scored, as in the tail queue of
-// the dense-layout kernel.  Scores go to the sequence's score row, histogram
-// counts straight to its global histogram.  Keys of a page number outside the
-// pool score -inf (and flag DSV4KV_DEV_BAD_PAGE).
-constexpr int kPagedUnit = 32;
+// page] * page + i % page.  Only sequences with n_b > k need scores.  Their
+// keys are laid end to end, each sequence padded to a multiple of 64 keys
+// (the padding is masked), and the whole range is split evenly over one wave
+// of CTAs, as in the dense-layout kernel: a CTA walks its range one sequence
+// segment at a time with a shared-memory histogram flushed per segment.
+// Segments start at multiples of 64 keys of their sequence and pages hold
+// multiples of 64 rows, so a group of 16 keys never straddles two pages: each
+// group resolves its page with one table load.  Keys of a page number outside
+// the pool score -inf (and flag DSV4KV_DEV_BAD_PAGE).
 constexpr int kMaxPagedBatch = 1024;
+constexpr int kPagedAlign = 64;
 
 __device__ __forceinline__ int64_t ragged_entries(const int64_t* t_seq, int b, int64_t t_max, int window, int stride,
                                                   int64_t n_max, uint32_t* status) {
@@ -726,223 +728,221 @@ struct PagedKeys {
   int64_t pages;
 };
 
+// Pool row of key i of sequence b (-1: a page number outside the pool).
+__device__ __forceinline__ int64_t paged_key_row(const PagedKeys& pk, int b, int64_t i) {
+  const int32_t pg = __ldg(pk.table + size_t(b) * pk.tstride + size_t(i / pk.page));
+  if (pg < 0 || pg >= pk.pages) return -1;
+  return int64_t(pg) * pk.page + i % pk.page;
+}
+
+// bf16 keys [i0, i0 + cnt) of sequence b (i0 a multiple of 64; keys >= n_b
+// masked): the loop of score_segment_bf16 with a page lookup per group of 16.
+template <int U>
+__device__ __forceinline__ void score_segment_paged_bf16(const uint16_t* __restrict__ qrow, const PagedKeys& pk,
+                                                         int b, int64_t i0, int64_t cnt, int64_t n_b, float* sc,
+                                                         uint32_t* sh, uint64_t pol, uint32_t* status) {
+  static_assert(U == 8, "two half-warps of 8 keys: a group of 16 keys");
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int half = lane >> 4, l16 = lane & 15;
+  const int my_key = (l16 >> 1) & 7;
+  const bool writer = !(lane & 1);
+  const uint16_t* keys = static_cast<const uint16_t*>(pk.codes) + 8 * l16;
+  float q[8];
+  {
+    const uint4 v = *reinterpret_cast<const uint4*>(qrow + 8 * l16);
+    q[0] = bf16lo(v.x); q[1] = bf16hi(v.x); q[2] = bf16lo(v.y); q[3] = bf16hi(v.y);
+    q[4] = bf16lo(v.z); q[5] = bf16hi(v.z); q[6] = bf16lo(v.w); q[7] = bf16hi(v.w);
+  }
+  const int64_t valid = min(cnt, n_b - i0);  // keys of the segment that exist
+  auto load = [&](int64_t j, uint4 (&v)[U], int64_t& row0) {
+    row0 = paged_key_row(pk, b, i0 + 16 * j);
+    if (row0 < 0) set_status(status, DSV4KV_DEV_BAD_PAGE);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t key = 16 * j + U * half + u;
+      v[u] = (row0 >= 0 && key < valid) ? ld_once_v4(keys + size_t(row0 + U * half + u) * 128, pol)
+                                        : make_uint4(0, 0, 0, 0);
+    }
+  };
+  auto process = [&](int64_t j, const uint4 (&v)[U], int64_t row0) {
+    float p[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) p[u] = dot8_bf16(v[u], q);
+    float s = reduce16_transposed<U>(p, l16) + 0.0f;  // -0 -> +0
+    if (row0 < 0) s = -INFINITY;
+    const int64_t key = 16 * j + U * half + my_key;
+    if (writer && key < valid) {
+      sc[key] = s;
+      atomicAdd(&sh[ord_f32(s) >> 20], 1u);
+    }
+  };
+  const int64_t ngroups = (cnt + 15) / 16;
+  uint4 va[U], vb[U];
+  int64_t ra = 0, rb = 0;
+  int64_t j = warp;
+  if (j < ngroups) load(j, va, ra);
+  while (j < ngroups) {
+    if (j + nwarps < ngroups) load(j + nwarps, vb, rb);
+    process(j, va, ra);
+    j += nwarps;
+    if (j >= ngroups) break;
+    if (j + nwarps < ngroups) load(j + nwarps, va, ra);
+    process(j, vb, rb);
+    j += nwarps;
+  }
+}
+
+// fp4 keys: a quarter warp per key (lane l4 owns channels [32 l4, 32 l4 + 32)),
+// 4 keys per quad and 32 per warp iteration (two iterations per group of 64
+// are within one page).
+__device__ __forceinline__ void score_segment_paged_fp4(const uint16_t* __restrict__ qrow, const PagedKeys& pk, int b,
+                                                        int64_t i0, int64_t cnt, int64_t n_b, float* sc,
+                                                        uint32_t* sh, uint64_t pol, uint32_t* status) {
+  constexpr int U = 4;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int quad = lane >> 2, l4 = lane & 3;
+  uint32_t qp[16];
+  {
+    const uint16_t* qb = qrow + 32 * l4;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) qp[j] = f32x2_to_f16x2(bf16f(qb[2 * j]), bf16f(qb[2 * j + 1]));
+  }
+  const uint8_t* codes = static_cast<const uint8_t*>(pk.codes) + 16 * l4;
+  const uint8_t* scales = pk.scales + 2 * l4;
+  const int64_t valid = min(cnt, n_b - i0);
+  auto load = [&](int64_t j, uint4 (&v)[U], uint32_t (&s2)[U], int64_t& row0) {
+    row0 = paged_key_row(pk, b, i0 + 32 * j);
+    if (row0 < 0) set_status(status, DSV4KV_DEV_BAD_PAGE);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t key = 32 * j + 8 * u + quad;
+      const bool ok = row0 >= 0 && key < valid;
+      const size_t r = size_t(ok ? row0 + 8 * u + quad : 0);
+      v[u] = ok ? ld_once_v4(codes + r * 64, pol) : make_uint4(0, 0, 0, 0);
+      s2[u] = ok ? ld_once_u16(scales + r * 8, pol) : 0u;
+    }
+  };
+  auto process = [&](int64_t j, const uint4 (&v)[U], const uint32_t (&s2)[U], int64_t row0) {
+    float pr[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      uint32_t acc0 = 0, acc1 = 0;
+#pragma unroll
+      for (int wi = 0; wi < 4; ++wi) {
+        uint32_t h[4];
+        e2m1x8_unpack(w[wi], h);
+#pragma unroll
+        for (int by = 0; by < 4; ++by) {
+          if (wi < 2) acc0 = hfma2(qp[4 * wi + by], h[by], acc0);
+          else acc1 = hfma2(qp[4 * wi + by], h[by], acc1);
+        }
+      }
+      pr[u] = scaled_group_sums(acc0, acc1, s2[u]);
+    }
+    const bool bb1 = l4 & 2, bb0 = l4 & 1;
+    float k2[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) k2[i] = (bb1 ? pr[2 + i] : pr[i]) + __shfl_xor_sync(kFull, bb1 ? pr[i] : pr[2 + i], 2);
+    float s = (bb0 ? k2[1] : k2[0]) + __shfl_xor_sync(kFull, bb0 ? k2[0] : k2[1], 1) + 0.0f;
+    if (row0 < 0) s = -INFINITY;
+    const int64_t key = 32 * j + 8 * l4 + quad;  // lane l4 ends with key u = l4
+    if (key < valid) {
+      sc[key] = s;
+      atomicAdd(&sh[ord_f32(s) >> 20], 1u);
+    }
+  };
+  const int64_t ngroups = (cnt + 31) / 32;
+  uint4 va[U], vb[U];
+  uint32_t sa[U], sb2[U];
+  int64_t ra = 0, rb = 0;
+  int64_t j = warp;
+  if (j < ngroups) load(j, va, sa, ra);
+  while (j < ngroups) {
+    if (j + nwarps < ngroups) load(j + nwarps, vb, sb2, rb);
+    process(j, va, sa, ra);
+    j += nwarps;
+    if (j >= ngroups) break;
+    if (j + nwarps < ngroups) load(j + nwarps, va, sa, ra);
+    process(j, vb, sb2, rb);
+    j += nwarps;
+  }
+}
+
 template <int FMT>
 __global__ void __launch_bounds__(256) index_score_paged(const uint16_t* __restrict__ qidx, const PagedKeys pk,
                                                          const int64_t* __restrict__ t_seq, int64_t t_max, int window,
                                                          int stride, int64_t n_max, int k, int batch,
                                                          float* __restrict__ scores, uint32_t* __restrict__ hist,
-                                                         uint32_t* __restrict__ claim, uint32_t* __restrict__ status) {
-  __shared__ uint32_t s_upre[kMaxPagedBatch + 1];  // first unit of every sequence; [batch] = all units
+                                                         uint32_t* __restrict__ status) {
+  __shared__ uint32_t sh[kHistBins];
+  __shared__ int64_t s_pre[kMaxPagedBatch + 1];  // flattened start of every sequence; [batch] = the total
   pdl_trigger();
   pdl_wait();
   {
     constexpr int PER = kMaxPagedBatch / 256;
-    uint32_t c[PER], sum = 0;
+    int64_t c[PER], sum = 0;
 #pragma unroll
     for (int j = 0; j < PER; ++j) {
       const int b = PER * threadIdx.x + j;
       const int64_t n_b = b < batch ? ragged_entries(t_seq, b, t_max, window, stride, n_max, nullptr) : 0;
-      c[j] = n_b > k ? uint32_t((n_b + kPagedUnit - 1) / kPagedUnit) : 0u;
+      c[j] = n_b > k ? (n_b + kPagedAlign - 1) / kPagedAlign * kPagedAlign : 0;
       sum += c[j];
     }
+    // exclusive scan of the per-thread sums (in units of kPagedAlign keys, which fit 32 bits)
     uint32_t total;
-    uint32_t run = block_exclusive_scan<256>(sum, &total);
+    int64_t run = int64_t(block_exclusive_scan<256>(uint32_t(sum / kPagedAlign), &total)) * kPagedAlign;
 #pragma unroll
     for (int j = 0; j < PER; ++j) {
       const int b = PER * threadIdx.x + j;
-      if (b < batch) s_upre[b] = run;
+      if (b < batch) s_pre[b] = run;
       run += c[j];
     }
-    if (threadIdx.x == 0) s_upre[batch] = total;
+    if (threadIdx.x == 0) s_pre[batch] = int64_t(total) * kPagedAlign;
   }
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0;
   __syncthreads();
-  const uint32_t units = s_upre[batch];
+  const int64_t total = s_pre[batch];
+  // the CTA's range: whole multiples of kPagedAlign keys
+  const int64_t units = total / kPagedAlign;
+  const int64_t per = (units + gridDim.x - 1) / gridDim.x * kPagedAlign;
+  const int64_t g0 = min(total, int64_t(blockIdx.x) * per), g1 = min(total, g0 + per);
   const uint64_t pol = l2_evict_first_policy();  // keys are read once
-  const int lane = threadIdx.x & 31;
   const size_t srow = size_t(score_stride(n_max));
-  // the unit's sequence: the last b with s_upre[b] <= u (binary search)
-  auto locate = [&](uint32_t u, int& b, int64_t& i0) {
+  int b = 0;
+  {  // the sequence holding g0: the last b with s_pre[b] <= g0
     int lo = 0, hi = batch - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (s_upre[mid] <= u) lo = mid;
+      if (s_pre[mid] <= g0) lo = mid;
       else hi = mid - 1;
     }
     b = lo;
-    i0 = int64_t(u - s_upre[lo]) * kPagedUnit;
-  };
-  // pool row of key i0 of sequence b (-1: bad page)
-  auto unit_row = [&](int b, int64_t i0) -> int64_t {
-    const int32_t pg = __ldg(pk.table + size_t(b) * pk.tstride + size_t(i0 / pk.page));
-    if (pg < 0 || pg >= pk.pages) return -1;
-    return int64_t(pg) * pk.page + i0 % pk.page;
-  };
-  uint32_t raw = 0;
-  auto claim_next = [&]() {
-    if (lane == 0) raw = atomicAdd(claim, 1u);
-  };
-  auto resolve = [&]() -> int64_t {
-    const uint32_t u = __shfl_sync(kFull, raw, 0);
-    return u < units ? int64_t(u) : -1;
-  };
-  claim_next();
-  int64_t cur = resolve();
-  if (cur < 0) return;
-  if constexpr (FMT == DSV4KV_BF16) {
-    // half a warp per key; a unit is two groups of 16 keys (8 per half-warp)
-    constexpr int U = 8;
-    const int half = lane >> 4, l16 = lane & 15, my_key = (l16 >> 1) & 7;
-    const bool writer = !(lane & 1);
-    const uint16_t* keys = static_cast<const uint16_t*>(pk.codes);
-    float q[8];
-    int bq = -1;
-    auto load_group = [&](int64_t row0, int64_t left, int g, uint4 (&v)[U]) {
-      const uint16_t* kb = keys + size_t(row0 < 0 ? 0 : row0) * 128 + 8 * l16;
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int key = 16 * g + U * half + u;
-        v[u] = (row0 >= 0 && key < left) ? ld_once_v4(kb + size_t(key) * 128, pol) : make_uint4(0, 0, 0, 0);
-      }
-    };
-    auto process = [&](int b, int64_t i0, int64_t row0, int64_t left, int g, const uint4 (&v)[U]) {
-      float pr[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) pr[u] = dot8_bf16(v[u], q);
-      float sc = reduce16_transposed<U>(pr, l16) + 0.0f;  // -0 -> +0
-      if (row0 < 0) sc = -INFINITY;
-      const int key = 16 * g + U * half + my_key;
-      if (writer && key < left) {
-        scores[size_t(b) * srow + size_t(i0 + key)] = sc;
-        atomicAdd(&hist[size_t(b) * kHistBins + (ord_f32(sc) >> 20)], 1u);
-      }
-    };
-    int b;
-    int64_t i0;
-    locate(uint32_t(cur), b, i0);
-    int64_t n_b = ragged_entries(t_seq, b, t_max, window, stride, n_max, status);
-    int64_t row0 = unit_row(b, i0);
-    if (row0 < 0) set_status(status, DSV4KV_DEV_BAD_PAGE);
-    uint4 va[U], vb[U];
-    load_group(row0, n_b - i0, 0, va);
-    claim_next();
-    while (true) {
-      load_group(row0, n_b - i0, 1, vb);
-      if (b != bq) {
-        const uint4 x = *reinterpret_cast<const uint4*>(qidx + size_t(b) * 128 + 8 * l16);
-        q[0] = bf16lo(x.x); q[1] = bf16hi(x.x); q[2] = bf16lo(x.y); q[3] = bf16hi(x.y);
-        q[4] = bf16lo(x.z); q[5] = bf16hi(x.z); q[6] = bf16lo(x.w); q[7] = bf16hi(x.w);
-        bq = b;
-      }
-      process(b, i0, row0, n_b - i0, 0, va);
-      const int64_t nxt = resolve();
-      int nb = b;
-      int64_t ni0 = 0, nn = n_b, nrow = row0;
-      if (nxt >= 0) {
-        locate(uint32_t(nxt), nb, ni0);
-        if (nb != b) nn = ragged_entries(t_seq, nb, t_max, window, stride, n_max, status);
-        nrow = unit_row(nb, ni0);
-        if (nrow < 0) set_status(status, DSV4KV_DEV_BAD_PAGE);
-        load_group(nrow, nn - ni0, 0, va);
-        claim_next();
-      }
-      process(b, i0, row0, n_b - i0, 1, vb);
-      if (nxt < 0) break;
-      b = nb;
-      i0 = ni0;
-      n_b = nn;
-      row0 = nrow;
-    }
-  } else {
-    // fp4 keys: a quarter warp per key (lane l4 owns channels [32 l4, 32 l4 + 32)),
-    // a unit is one warp iteration of 8 quads x 4 keys
-    constexpr int U = 4;
-    const int quad = lane >> 2, l4 = lane & 3;
-    const uint8_t* codes = static_cast<const uint8_t*>(pk.codes);
-    uint32_t qp[16];
-    int bq = -1;
-    auto load_unit = [&](int64_t row0, int64_t left, uint4 (&v)[U], uint32_t (&s2)[U]) {
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int key = 8 * u + quad;
-        const bool ok = row0 >= 0 && key < left;
-        const size_t r = size_t(ok ? row0 + key : 0);
-        v[u] = ok ? ld_once_v4(codes + r * 64 + 16 * l4, pol) : make_uint4(0, 0, 0, 0);
-        s2[u] = ok ? ld_once_u16(pk.scales + r * 8 + 2 * l4, pol) : 0u;
-      }
-    };
-    auto process = [&](int b, int64_t i0, int64_t row0, int64_t left, const uint4 (&v)[U], const uint32_t (&s2)[U]) {
-      float pr[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-        uint32_t acc0 = 0, acc1 = 0;
-#pragma unroll
-        for (int wi = 0; wi < 4; ++wi) {
-          uint32_t h[4];
-          e2m1x8_unpack(w[wi], h);
-#pragma unroll
-          for (int by = 0; by < 4; ++by) {
-            if (wi < 2) acc0 = hfma2(qp[4 * wi + by], h[by], acc0);
-            else acc1 = hfma2(qp[4 * wi + by], h[by], acc1);
-          }
-        }
-        pr[u] = scaled_group_sums(acc0, acc1, s2[u]);
-      }
-      const bool bb1 = l4 & 2, bb0 = l4 & 1;
-      float k2[2];
-#pragma unroll
-      for (int i = 0; i < 2; ++i) k2[i] = (bb1 ? pr[2 + i] : pr[i]) + __shfl_xor_sync(kFull, bb1 ? pr[i] : pr[2 + i], 2);
-      float sc = (bb0 ? k2[1] : k2[0]) + __shfl_xor_sync(kFull, bb0 ? k2[0] : k2[1], 1) + 0.0f;
-      if (row0 < 0) sc = -INFINITY;
-      const int key = 8 * l4 + quad;  // lane l4 ends with key u = l4
-      if (key < left) {
-        scores[size_t(b) * srow + size_t(i0 + key)] = sc;
-        atomicAdd(&hist[size_t(b) * kHistBins + (ord_f32(sc) >> 20)], 1u);
-      }
-    };
-    int b;
-    int64_t i0;
-    locate(uint32_t(cur), b, i0);
-    int64_t n_b = ragged_entries(t_seq, b, t_max, window, stride, n_max, status);
-    int64_t row0 = unit_row(b, i0);
-    if (row0 < 0) set_status(status, DSV4KV_DEV_BAD_PAGE);
-    uint4 va[U];
-    uint32_t sa[U];
-    load_unit(row0, n_b - i0, va, sa);
-    claim_next();
-    while (true) {
-      if (b != bq) {
-        const uint16_t* qb = qidx + size_t(b) * 128 + 32 * l4;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) qp[j] = f32x2_to_f16x2(bf16f(qb[2 * j]), bf16f(qb[2 * j + 1]));
-        bq = b;
-      }
-      const int64_t nxt = resolve();
-      int nb = b;
-      int64_t ni0 = 0, nn = n_b, nrow = row0;
-      uint4 vb[U];
-      uint32_t sb2[U];
-      if (nxt >= 0) {
-        locate(uint32_t(nxt), nb, ni0);
-        if (nb != b) nn = ragged_entries(t_seq, nb, t_max, window, stride, n_max, status);
-        nrow = unit_row(nb, ni0);
-        if (nrow < 0) set_status(status, DSV4KV_DEV_BAD_PAGE);
-        load_unit(nrow, nn - ni0, vb, sb2);
-        claim_next();
-      }
-      process(b, i0, row0, n_b - i0, va, sa);
-      if (nxt < 0) break;
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        va[u] = vb[u];
-        sa[u] = sb2[u];
-      }
-      b = nb;
-      i0 = ni0;
-      n_b = nn;
-      row0 = nrow;
-    }
   }
+  int b_last = -1;
+  for (int64_t s0 = g0; s0 < g1 && b < batch;) {
+    const int64_t e = s_pre[b + 1];
+    if (e <= s0) {  // an empty (or finished) sequence
+      ++b;
+      continue;
+    }
+    const int64_t s1 = min(g1, e);
+    const int64_t i0 = s0 - s_pre[b];
+    const int64_t n_b = ragged_entries(t_seq, b, t_max, window, stride, n_max, status);
+    if (b_last >= 0) {
+      flush_histogram(sh, hist + size_t(b_last) * kHistBins);
+      __syncthreads();
+    }
+    if constexpr (FMT == DSV4KV_BF16)
+      score_segment_paged_bf16<8>(qidx + size_t(b) * 128, pk, b, i0, s1 - s0, n_b, scores + size_t(b) * srow + i0, sh,
+                                  pol, status);
+    else
+      score_segment_paged_fp4(qidx + size_t(b) * 128, pk, b, i0, s1 - s0, n_b, scores + size_t(b) * srow + i0, sh, pol,
+                              status);
+    b_last = b;
+    s0 = s1;
+  }
+  if (b_last >= 0) flush_histogram(sh, hist + size_t(b_last) * kHistBins);
 }
 
 // (t_seq != null: a ragged batch, sequence b selects among its own n_b <=
@@ -1569,8 +1569,12 @@ dsv4kv_status index_score_launch(const uint16_t* qidx, const dsv4kv_cache& keys,
         occ = 1;
       occ_slot.store(occ, std::memory_order_relaxed);
     }
-    // the last kTailPct % of every sequence (whole units) goes to the shared queue
-    const int64_t n_tail = std::min<int64_t>(n, (n * kTailPct / 100) / kTailUnit * kTailUnit);
+    // the last kTailPct % of every sequence (whole units) goes to the shared
+    // queue.  Its histogram counts go straight to global memory, one atomic
+    // per key, so with few sequences they would pile onto the few bins that
+    // hold most scores of one histogram: small batches use the even split alone.
+    const int64_t n_tail =
+        batch >= kTailMinBatch ? std::min<int64_t>(n, (n * kTailPct / 100) / kTailUnit * kTailUnit) : 0;
     const int64_t n_h = n - n_tail;
     const int64_t total = int64_t(batch) * n_h;
     const int64_t grid = int64_t(sms) * occ;
@@ -1674,7 +1678,7 @@ dsv4kv_status index_topk_paged_launch(const uint16_t* qidx, const dsv4kv_cache& 
       slot.store(occ, std::memory_order_relaxed);
     }
     launch_pdl(kern, dim3(unsigned(sm_count() * occ)), dim3(256), 0, stream, qidx, pk, rg.t_seq, rg.t_max, rg.window,
-               rg.stride, n_max, k, batch, w.scores, w.hist, w.tail_ctr, w.status);
+               rg.stride, n_max, k, batch, w.scores, w.hist, w.status);
     const dsv4kv_status st = check_launch("index_score_paged");
     if (st != DSV4KV_OK) return st;
   }
