@@ -620,71 +620,83 @@ def time_e2e(layer, steps):
     the device, makes the library calls and copies its output back to pinned
     host memory, all inside the timed region.
 
-    Steps alternate between two streams, each with its own device buffers,
-    workspaces and pinned host buffers, so step i+1's upload and step i-1's
-    download overlap step i's calls (and two steps' kernels may share the
-    GPU).  Each (stream, cache replica) pair replays a CUDA graph of its
-    [upload -> calls -> download], captured once, the way a serving loop
-    issues its decode steps; the same steps issued eagerly from Python give
-    the eager figure.  Returns (graph ms, eager ms, H2D bytes per step, D2H
-    bytes per step)."""
+    The steps run as a three-stage pipeline over three streams (upload,
+    compute, download) with NB sets of device and pinned host buffers: step
+    i's upload and step i-1's download overlap step i-1's / i's calls, and
+    events order every reuse of a buffer.  The calls of a step are one CUDA
+    graph per (buffer set, cache replica), captured once and replayed, the way
+    a serving loop issues its decode steps; the copies and event waits are
+    issued from Python.  The eager figure issues the calls themselves instead
+    of the graphs.  Returns (graph ms, eager ms, H2D bytes per step, D2H bytes
+    per step)."""
     torch = layer.torch
     R = len(layer.reps)
-    NB = 2
-    lanes = [layer.twin() for _ in range(NB)]             # own buffers and workspaces per stream
+    NB = 3
+    lanes = [layer.twin() for _ in range(NB)]             # own output buffers and workspaces per set
     q_host = [layer.q.cpu().pin_memory() for _ in range(NB)]
     qi_host = [layer.qidx.cpu().pin_memory() for _ in range(NB)]
     out_host = [torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory() for _ in range(NB)]
     q_dev = [torch.empty_like(layer.q) for _ in range(NB)]
     qi_dev = [torch.empty_like(layer.qidx) for _ in range(NB)]
-    streams = [torch.cuda.Stream() for _ in range(NB)]
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(NB)]
+    ev_comp = [torch.cuda.Event() for _ in range(NB)]
+    ev_out = [torch.cuda.Event() for _ in range(NB)]
+    for e in ev_comp + ev_out:
+        e.record(s_comp)                               # nothing to wait for before the first use
     torch.cuda.synchronize()
 
-    def body(i):
-        j, r = i % NB, i % R
+    def calls(j, r):
         L = lanes[j]
-        q_dev[j].copy_(q_host[j], non_blocking=True)
         if L.kind == "c4a":
-            qi_dev[j].copy_(qi_host[j], non_blocking=True)
             L.index(r, qidx=qi_dev[j])
         L.decode(r, q=q_dev[j])
-        out_host[j].copy_(L.out, non_blocking=True)
 
-    def run(issue):
+    graphs = {}
+    for j in range(NB):
+        for r in range(R):
+            with torch.cuda.stream(s_comp):
+                calls(j, r)                            # warm the buffers before capture
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s_comp):
+                calls(j, r)
+            graphs[(j, r)] = g
+    torch.cuda.synchronize()
+
+    def run(use_graphs):
         start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
-        start.record(streams[0])
-        for s_ in streams[1:]:
-            s_.wait_event(start)
+        start.record(s_in)
+        s_comp.wait_event(start)
+        s_out.wait_event(start)
         for i in range(steps):
-            with torch.cuda.stream(streams[i % NB]):
-                issue(i)
-        for s_ in streams[1:]:
-            e = torch.cuda.Event()
-            e.record(s_)
-            streams[0].wait_event(e)
-        stop.record(streams[0])
+            j, r = i % NB, i % R
+            s_in.wait_event(ev_comp[j])                # step i - NB's calls have read this input set
+            with torch.cuda.stream(s_in):
+                q_dev[j].copy_(q_host[j], non_blocking=True)
+                if layer.kind == "c4a":
+                    qi_dev[j].copy_(qi_host[j], non_blocking=True)
+            ev_in[j].record(s_in)
+            s_comp.wait_event(ev_in[j])
+            s_comp.wait_event(ev_out[j])               # step i - NB's output has left this set
+            with torch.cuda.stream(s_comp):
+                if use_graphs:
+                    graphs[(j, r)].replay()
+                else:
+                    calls(j, r)
+            ev_comp[j].record(s_comp)
+            s_out.wait_event(ev_comp[j])
+            with torch.cuda.stream(s_out):
+                out_host[j].copy_(lanes[j].out, non_blocking=True)
+            ev_out[j].record(s_out)
+        stop.record(s_out)                             # after the last download
         stop.synchronize()
         return start.elapsed_time(stop)
 
-    for i in range(2 * NB):                          # warm-up, eager
-        with torch.cuda.stream(streams[i % NB]):
-            body(i)
-    torch.cuda.synchronize()
-    eager_ms = run(body)
-    # one graph per (stream, replica) pair of a step index
-    M = R if R % NB == 0 else NB * R
-    graphs = []
-    for m in range(M):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=streams[m % NB]):
-            body(m)
-        graphs.append(g)
-    torch.cuda.synchronize()
-    for i in range(M):                               # every graph launched once before timing
-        with torch.cuda.stream(streams[i % NB]):
-            graphs[i].replay()
-    graph_ms = run(lambda i: graphs[i % M].replay())
+    run(True)                                          # warm-up pass (every graph launched once)
+    eager_ms = run(False)
+    graph_ms = run(True)
     del graphs
     h2d = layer.q.numel() * 2 + (layer.qidx.numel() * 2 if layer.kind == "c4a" else 0)
     return graph_ms, eager_ms, h2d, layer.out.numel() * 2
@@ -1002,9 +1014,10 @@ def main():
             "e2e": {"value": round(e2e_v, 2), "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "eager_value": round(e2e_eager_v, 2),
                     "method": "public API (the layer's index and decode calls) on pinned host buffers; per "
-                              "step an H2D of the queries and a D2H of the outputs; steps alternate between two "
-                              "streams with their own buffers and workspaces, each replaying a CUDA graph of "
-                              "[H2D -> calls -> D2H] (eager_value: the same steps issued from Python)"},
+                              "step an H2D of the queries and a D2H of the outputs, pipelined over upload / "
+                              "compute / download streams with three buffer sets; the calls of a step replayed "
+                              "as one CUDA graph per (buffer set, cache replica) (eager_value: the calls "
+                              "issued from Python)"},
             "gpu_launches": layer.launches_per_step() * args.steps,
             "clocks": res["clocks"]}
     if stack:

@@ -642,6 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if ((gathered || C::kRowScale) && !dead) dead = !warp_wait(&ctl->full[stage], (i / kStages) & 1, ctl, lane);
       float x[2][16];
       float tmax[2] = {-INFINITY, -INFINITY}, ymax[2] = {-INFINITY, -INFINITY};
+      float2 rsc[C::kRowScale ? 8 : 1], rls[C::kRowScale ? 8 : 1], rinv[C::kRowScale ? 8 : 1];
       if (!dead) {
         tc_fence_after();
         uint32_t sc[32];
@@ -653,23 +654,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t vm = gathered ? (uint64_t(ctl->vmask[stage][0]) | (uint64_t(ctl->vmask[stage][1]) << 16) |
                                         (uint64_t(ctl->vmask[stage][2]) << 32) | (uint64_t(ctl->vmask[stage][3]) << 48))
                                      : ~0ull;  // a TMA tile: 64 rows that exist
+        if (C::kRowScale) {  // this thread's rows 8j + 2 c2 + {0, 1}: their scale terms, up front
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            rsc[j] = *reinterpret_cast<const float2*>(&ctl->row_scale[stage][8 * j + 2 * c2]);
+            rls[j] = *reinterpret_cast<const float2*>(&ctl->row_ls[stage][8 * j + 2 * c2]);
+            rinv[j] = *reinterpret_cast<const float2*>(&ctl->row_inv[stage][8 * j + 2 * c2]);
+          }
+        }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int r = 8 * j + 2 * c2 + e;
             const bool v = (vm >> r) & 1;
-            float ls = 0.f;
+            float ls = 0.f, rs = 1.f;
             bool sok = true;
             if (C::kRowScale) {
-              sok = ctl->row_scale[stage][r] > 0.f;
-              ls = ctl->row_ls[stage][r];
+              rs = e ? rsc[j].y : rsc[j].x;
+              ls = e ? rls[j].y : rls[j].x;
+              sok = rs > 0.f;
             }
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
               float xv = v ? __uint_as_float(sc[4 * j + 2 * hh + e]) * p.score_scale : -INFINITY;
               if (C::kRowScale) {
-                xv = v ? xv * ctl->row_scale[stage][r] : -INFINITY;
+                xv = v ? xv * rs : -INFINITY;
                 ymax[hh] = fmaxf(ymax[hh], (v && sok) ? xv + ls : -INFINITY);
               }
               x[hh][2 * j + e] = xv;
@@ -742,17 +752,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         float lw_sum = 0.f;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const int r = 8 * j + 2 * c2;
           float ya = x[hh][2 * j], yb = x[hh][2 * j + 1];
           if (C::kRowScale) {  // y = x + log2(s_r): the weight of the stored row carries its scale
-            ya += ctl->row_ls[stage][r];
-            yb += ctl->row_ls[stage][r + 1];
+            ya += rls[j].x;
+            yb += rls[j].y;
           }
           const float wa = (m_o[hh] == -INFINITY) ? 0.f : fast_exp2(ya - m_o[hh]);
           const float wb = (m_o[hh] == -INFINITY) ? 0.f : fast_exp2(yb - m_o[hh]);
           const uint32_t packed = pack_p(wa, wb, C::kQuant);
           if (C::kRowScale) {
-            lw_sum = fmaf(wa, ctl->row_inv[stage][r], fmaf(wb, ctl->row_inv[stage][r + 1], lw_sum));
+            lw_sum = fmaf(wa, rinv[j].x, fmaf(wb, rinv[j].y, lw_sum));
           } else {
             l[hh] += p_lo(packed, C::kQuant) + p_hi(packed, C::kQuant);  // the weights the MMA uses
           }

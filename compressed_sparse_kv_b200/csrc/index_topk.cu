@@ -728,9 +728,15 @@ struct PagedKeys {
   int64_t pages;
 };
 
-// Pool row of key i of sequence b (-1: a page number outside the pool).
-__device__ __forceinline__ int64_t paged_key_row(const PagedKeys& pk, int b, int64_t i) {
-  const int32_t pg = __ldg(pk.table + size_t(b) * pk.tstride + size_t(i / pk.page));
+// Pool row of key i of sequence b (-1: a page number outside the pool).  The
+// page numbers of the segment being scored are staged in shared memory
+// (pg_s[j] = the table entry of page pg0 + j) when they fit, else read from
+// the table.
+constexpr int kPageStage = 512;
+__device__ __forceinline__ int64_t paged_key_row(const PagedKeys& pk, int b, int64_t i, const int32_t* pg_s,
+                                                 int64_t pg0) {
+  const int64_t pi = i / pk.page;
+  const int32_t pg = pg_s ? pg_s[pi - pg0] : __ldg(pk.table + size_t(b) * pk.tstride + size_t(pi));
   if (pg < 0 || pg >= pk.pages) return -1;
   return int64_t(pg) * pk.page + i % pk.page;
 }
@@ -740,7 +746,8 @@ __device__ __forceinline__ int64_t paged_key_row(const PagedKeys& pk, int b, int
 template <int U>
 __device__ __forceinline__ void score_segment_paged_bf16(const uint16_t* __restrict__ qrow, const PagedKeys& pk,
                                                          int b, int64_t i0, int64_t cnt, int64_t n_b, float* sc,
-                                                         uint32_t* sh, uint64_t pol, uint32_t* status) {
+                                                         uint32_t* sh, uint64_t pol, uint32_t* status,
+                                                         const int32_t* pg_s, int64_t pg0) {
   static_assert(U == 8, "two half-warps of 8 keys: a group of 16 keys");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int half = lane >> 4, l16 = lane & 15;
@@ -755,7 +762,8 @@ __device__ __forceinline__ void score_segment_paged_bf16(const uint16_t* __restr
   }
   const int64_t valid = min(cnt, n_b - i0);  // keys of the segment that exist
   auto load = [&](int64_t j, uint4 (&v)[U], int64_t& row0) {
-    row0 = paged_key_row(pk, b, i0 + 16 * j);
+    // (a group of padding keys past the sequence's end looks up no page)
+    row0 = 16 * j < valid ? paged_key_row(pk, b, i0 + 16 * j, pg_s, pg0) : 0;
     if (row0 < 0) set_status(status, DSV4KV_DEV_BAD_PAGE);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -797,7 +805,8 @@ __device__ __forceinline__ void score_segment_paged_bf16(const uint16_t* __restr
 // are within one page).
 __device__ __forceinline__ void score_segment_paged_fp4(const uint16_t* __restrict__ qrow, const PagedKeys& pk, int b,
                                                         int64_t i0, int64_t cnt, int64_t n_b, float* sc,
-                                                        uint32_t* sh, uint64_t pol, uint32_t* status) {
+                                                        uint32_t* sh, uint64_t pol, uint32_t* status,
+                                                        const int32_t* pg_s, int64_t pg0) {
   constexpr int U = 4;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int quad = lane >> 2, l4 = lane & 3;
@@ -811,7 +820,8 @@ __device__ __forceinline__ void score_segment_paged_fp4(const uint16_t* __restri
   const uint8_t* scales = pk.scales + 2 * l4;
   const int64_t valid = min(cnt, n_b - i0);
   auto load = [&](int64_t j, uint4 (&v)[U], uint32_t (&s2)[U], int64_t& row0) {
-    row0 = paged_key_row(pk, b, i0 + 32 * j);
+    // (a group of padding keys past the sequence's end looks up no page)
+    row0 = 32 * j < valid ? paged_key_row(pk, b, i0 + 32 * j, pg_s, pg0) : 0;
     if (row0 < 0) set_status(status, DSV4KV_DEV_BAD_PAGE);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -877,6 +887,7 @@ __global__ void __launch_bounds__(256) index_score_paged(const uint16_t* __restr
                                                          uint32_t* __restrict__ status) {
   __shared__ uint32_t sh[kHistBins];
   __shared__ int64_t s_pre[kMaxPagedBatch + 1];  // flattened start of every sequence; [batch] = the total
+  __shared__ int32_t s_pg[kPageStage];           // the page numbers of the segment being scored
   pdl_trigger();
   pdl_wait();
   {
@@ -929,16 +940,24 @@ __global__ void __launch_bounds__(256) index_score_paged(const uint16_t* __restr
     const int64_t s1 = min(g1, e);
     const int64_t i0 = s0 - s_pre[b];
     const int64_t n_b = ragged_entries(t_seq, b, t_max, window, stride, n_max, status);
-    if (b_last >= 0) {
-      flush_histogram(sh, hist + size_t(b_last) * kHistBins);
-      __syncthreads();
-    }
+    if (b_last >= 0) flush_histogram(sh, hist + size_t(b_last) * kHistBins);  // (starts with a block barrier)
+    // stage the segment's page numbers (the keys that exist) in shared memory
+    const int64_t pg0 = i0 / pk.page;
+    const int64_t last = min(s1 - s0, n_b - i0);
+    const int64_t npg = last > 0 ? (i0 + last - 1) / pk.page - pg0 + 1 : 0;
+    const bool staged = npg <= kPageStage;
+    if (staged)
+      for (int64_t j = threadIdx.x; j < npg; j += blockDim.x)
+        s_pg[j] = __ldg(pk.table + size_t(b) * pk.tstride + size_t(pg0 + j));
+    __syncthreads();
+    const int32_t* pg_s = staged ? s_pg : nullptr;
     if constexpr (FMT == DSV4KV_BF16)
       score_segment_paged_bf16<8>(qidx + size_t(b) * 128, pk, b, i0, s1 - s0, n_b, scores + size_t(b) * srow + i0, sh,
-                                  pol, status);
+                                  pol, status, pg_s, pg0);
     else
       score_segment_paged_fp4(qidx + size_t(b) * 128, pk, b, i0, s1 - s0, n_b, scores + size_t(b) * srow + i0, sh, pol,
-                              status);
+                              status, pg_s, pg0);
+    __syncthreads();  // s_pg is rewritten for the next segment only after every warp used it
     b_last = b;
     s0 = s1;
   }
