@@ -555,7 +555,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint64_t idle_since = 0;
       while (ok && next_pv < nt) {
         bool progressed = false;
-        if (next_pv < next_qk && mbar_try_wait(&ctl->p_full[next_pv & 1], (next_pv >> 1) & 1)) {
+        // both products are polled with non-blocking tests, so that one that is
+        // not ready never holds up the other
+        if (next_pv < next_qk && mbar_test_wait(&ctl->p_full[next_pv & 1], (next_pv >> 1) & 1)) {
           const int j = next_pv, stage = j % kStages, pb = j & 1;
           tc_fence_after();
           const uint32_t r_addr = smem_u32(sR + stage * kTileBytes);
@@ -575,8 +577,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           progressed = true;
         } else if (next_qk < nt && next_qk < next_pv + 2) {
           const int i = next_qk, stage = i % kStages, sb = i & 1;
-          if (mbar_try_wait(&ctl->full[stage], (i / kStages) & 1) &&
-              (i < 2 || mbar_try_wait(&ctl->s_free[sb], ((i - 2) >> 1) & 1))) {
+          if (mbar_test_wait(&ctl->full[stage], (i / kStages) & 1) &&
+              (i < 2 || mbar_test_wait(&ctl->s_free[sb], ((i - 2) >> 1) & 1))) {
             tc_fence_after();
             const uint64_t rd = smem_desc_sw128(smem_u32(sR + stage * kTileBytes), 16, 1024);
             const uint32_t d = tmem + kColS + 64 * sb;

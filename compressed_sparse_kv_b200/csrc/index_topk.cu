@@ -447,6 +447,7 @@ constexpr int kCandCap = 8192;                         // candidates per sequenc
 constexpr int kResPer = kCandCap / kSelThreads;        // candidates per leader thread
 constexpr int kTieCap = 2048;
 constexpr int kMaxClusterSel = 16;
+constexpr int64_t kSelOneCtaMax = 65536;
 constexpr int kWarpCap = kSelStage / kSelWarps;       // candidates a warp's list can hold
 // Every warp streams its run of scores through its own ring of kRing slots
 // of one warp batch (256 fp32 = 1 KB) in shared memory, filled by 16-byte
@@ -1657,7 +1658,12 @@ dsv4kv_status index_select_launch(int batch, int64_t n, int k, int32_t* idx_out,
     max_cluster_slot.store(max_cluster, std::memory_order_release);
   }
   // at most one CTA per SM in all (the leader's registers allow one per SM)
-  const int64_t per_seq = std::max<int64_t>(1, std::min<int64_t>(max_cluster, sms / std::max(batch, 1)));
+  // (a sequence of up to kSelOneCtaMax scores is selected by one CTA: below
+  // that the cluster's push, barrier and gather cost more than the filter
+  // they spread)
+  const int64_t per_seq = n <= kSelOneCtaMax
+                              ? 1
+                              : std::max<int64_t>(1, std::min<int64_t>(max_cluster, sms / std::max(batch, 1)));
   const int64_t units_per_cta = std::max<int64_t>(1, (n + per_seq * kSelChunkUnit - 1) / (per_seq * kSelChunkUnit));
   const int64_t chunk = units_per_cta * kSelChunkUnit;
   const unsigned ctas = unsigned((n + chunk - 1) / chunk);
