@@ -27,6 +27,14 @@ namespace dsv4kv {
 
 constexpr int kHistBins = 4096;  // 12-bit digits
 
+// The global histograms keep bin i at position ((i & 31) << 7) | (i >> 5):
+// neighbouring bins sit 512 bytes apart, in different L2 lines.  Most scores
+// fall into a few neighbouring bins, and with many CTAs adding into one
+// sequence's histogram (small batches), atomics that all hit the same few
+// lines would queue behind each other.
+__host__ __device__ __forceinline__ int hist_pos(int bin) { return ((bin & 31) << 7) | (bin >> 5); }
+__host__ __device__ __forceinline__ int hist_bin(int pos) { return ((pos & 127) << 5) | (pos >> 7); }
+
 // Row stride of the fp32 score rows in the workspace: n rounded up to 4, so
 // every row starts on a 16-byte boundary.
 __host__ __device__ __forceinline__ int64_t score_stride(int64_t n) { return (n + 3) & ~int64_t(3); }
@@ -143,7 +151,7 @@ __device__ __forceinline__ void flush_histogram(uint32_t* sh, uint32_t* hb) {
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
     const uint32_t c = sh[i];
     if (c) {
-      atomicAdd(&hb[i], c);
+      atomicAdd(&hb[hist_pos(i)], c);
       sh[i] = 0;
     }
   }
@@ -200,7 +208,7 @@ __device__ __forceinline__ void score_tail_bf16(const uint16_t* __restrict__ qid
     const int64_t key = i0 + 16 * g + U * half + my_key;
     if (writer && key < n) {
       scores[size_t(b) * size_t(score_stride(n)) + size_t(key)] = sc;
-      atomicAdd(&hist[size_t(b) * kHistBins + (ord_f32(sc) >> 20)], 1u);
+      atomicAdd(&hist[size_t(b) * kHistBins + hist_pos(int(ord_f32(sc) >> 20))], 1u);
     }
   };
   claim();
@@ -447,7 +455,6 @@ constexpr int kCandCap = 8192;                         // candidates per sequenc
 constexpr int kResPer = kCandCap / kSelThreads;        // candidates per leader thread
 constexpr int kTieCap = 2048;
 constexpr int kMaxClusterSel = 16;
-constexpr int64_t kSelOneCtaMax = 65536;
 constexpr int kWarpCap = kSelStage / kSelWarps;       // candidates a warp's list can hold
 // Every warp streams its run of scores through its own ring of kRing slots
 // of one warp batch (256 fp32 = 1 KB) in shared memory, filled by 16-byte
@@ -587,16 +594,26 @@ __device__ uint32_t ordered_offsets(const uint32_t (&m)[BATCH], uint32_t (&off)[
 }
 
 // Copies a sequence's 4096-bin histogram from the workspace (L2) into shared
-// memory with every load of a thread issued before its stores.
+// memory in bin order, with every load of a thread issued before its stores.
+// Lane l of warp w takes the 16-byte group q = 32 l + (w + j NW) of
+// positions (iteration j): the four bins of a group are 32 apart and the
+// lanes' bins fall in 32 different banks.
 template <int NT>
 __device__ __forceinline__ void load_histogram(const uint32_t* __restrict__ hb, uint32_t* sh) {
-  constexpr int V = kHistBins / 4 / NT;  // uint4 per thread
-  static_assert(V * 4 * NT == kHistBins, "histogram split");
+  constexpr int NW = NT / 32, V = 32 / NW;  // uint4 per thread
+  static_assert(V * NW == 32 && V * 4 * NT == kHistBins, "histogram split");
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint4 v[V];
 #pragma unroll
-  for (int j = 0; j < V; ++j) v[j] = __ldcg(reinterpret_cast<const uint4*>(hb) + threadIdx.x + j * NT);
+  for (int j = 0; j < V; ++j) v[j] = __ldcg(reinterpret_cast<const uint4*>(hb) + 32 * lane + warp + j * NW);
 #pragma unroll
-  for (int j = 0; j < V; ++j) reinterpret_cast<uint4*>(sh)[threadIdx.x + j * NT] = v[j];
+  for (int j = 0; j < V; ++j) {
+    const int p = 4 * (32 * lane + warp + j * NW);  // positions p .. p + 3
+    sh[hist_bin(p)] = v[j].x;
+    sh[hist_bin(p + 1)] = v[j].y;
+    sh[hist_bin(p + 2)] = v[j].z;
+    sh[hist_bin(p + 3)] = v[j].w;
+  }
 }
 
 // Issues the copy of one warp batch (scores [base, base + 256) of the row,
@@ -1658,12 +1675,7 @@ dsv4kv_status index_select_launch(int batch, int64_t n, int k, int32_t* idx_out,
     max_cluster_slot.store(max_cluster, std::memory_order_release);
   }
   // at most one CTA per SM in all (the leader's registers allow one per SM)
-  // (a sequence of up to kSelOneCtaMax scores is selected by one CTA: below
-  // that the cluster's push, barrier and gather cost more than the filter
-  // they spread)
-  const int64_t per_seq = n <= kSelOneCtaMax
-                              ? 1
-                              : std::max<int64_t>(1, std::min<int64_t>(max_cluster, sms / std::max(batch, 1)));
+  const int64_t per_seq = std::max<int64_t>(1, std::min<int64_t>(max_cluster, sms / std::max(batch, 1)));
   const int64_t units_per_cta = std::max<int64_t>(1, (n + per_seq * kSelChunkUnit - 1) / (per_seq * kSelChunkUnit));
   const int64_t chunk = units_per_cta * kSelChunkUnit;
   const unsigned ctas = unsigned((n + chunk - 1) / chunk);
