@@ -117,7 +117,7 @@ struct Params {
   const uint8_t* win_codes;
   const void* win_scales;
   float score_scale;  // sm_scale * log2(e)
-  float* o_part;      // [B][splits][H][512]
+  uint16_t* o_part;   // [B][splits][H][512] bf16 (the split's unnormalised output)
   float* ml_part;     // [B][splits][H][4]: (m_o, m_l, l, 0)
   float* rope_tab;    // [B][2][256]: the rotation tables for decode_combine (written by split 0)
   uint32_t* status;
@@ -318,7 +318,7 @@ __device__ __forceinline__ float p_hi(uint32_t v, bool f16) {
 __device__ __forceinline__ void store_partial(const Params& p, int b, int split, uint32_t tmem, int wq, int lane,
                                               int ct0, int ct1) {
   const uint32_t lane_base = uint32_t(32 * wq) << 16;
-  float* op = p.o_part + (size_t(b) * p.splits + split) * size_t(p.heads) * kDim;
+  uint16_t* op = p.o_part + (size_t(b) * p.splits + split) * size_t(p.heads) * kDim;
 #pragma unroll 1
   for (int ct = ct0; ct < ct1; ++ct) {
     const int c = 128 * ct + 32 * wq + lane;
@@ -330,7 +330,7 @@ __device__ __forceinline__ void store_partial(const Params& p, int b, int split,
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         const int hh = 32 * half + e;
-        if (hh < p.heads) op[size_t(hh) * kDim + c] = __uint_as_float(o[e]);
+        if (hh < p.heads) op[size_t(hh) * kDim + c] = f2bf(__uint_as_float(o[e]));
       }
     }
   }
@@ -935,7 +935,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr int kCombWarps = 4;
 constexpr int kCombFast = 4;  // splits up to which a warp issues all its loads at once
 
-__global__ void __launch_bounds__(32 * kCombWarps) decode_combine(const float* __restrict__ o_part,
+// The partial outputs are bf16 (half the bytes the decode CTAs write and the
+// merges read); 4 channels of a split are one 8-byte load.
+__device__ __forceinline__ float4 ld_bf16x4(const uint16_t* p) {
+  const uint2 v = __ldcg(reinterpret_cast<const uint2*>(p));
+  return make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
+}
+
+__global__ void __launch_bounds__(32 * kCombWarps) decode_combine(const uint16_t* __restrict__ o_part,
                                                                   const float* __restrict__ ml_part,
                                                                   const float* __restrict__ rope_tab, int splits,
                                                                   int heads, int bh_total, int rope_dim, int out_fp32,
@@ -948,7 +955,7 @@ __global__ void __launch_bounds__(32 * kCombWarps) decode_combine(const float* _
   const int b = bh / heads, h = bh % heads;
   const size_t ml_stride = size_t(heads) * 4, o_stride = size_t(heads) * kDim;
   const float* mlb = ml_part + (size_t(b) * splits * heads + h) * 4;
-  const float* ob = o_part + (size_t(b) * splits * heads + h) * kDim + 4 * lane;
+  const uint16_t* ob = o_part + (size_t(b) * splits * heads + h) * kDim + 4 * lane;
   rope_tab += size_t(b) * kDim;  // this sequence's rotation
   // the rotation of this lane's rotary pairs (channels 128q + 4 lane + {0, 2}), read up front
   const int r0 = kDim - rope_dim;
@@ -976,8 +983,7 @@ __global__ void __launch_bounds__(32 * kCombWarps) decode_combine(const float* _
     for (int s = 0; s < kCombFast; ++s)
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        x[s][q] = s < splits ? __ldcg(reinterpret_cast<const float4*>(ob + size_t(s) * o_stride + 128 * q))
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[s][q] = s < splits ? ld_bf16x4(ob + size_t(s) * o_stride + 128 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
     mo = v.x;
     ml = v.y;
 #pragma unroll
@@ -1022,10 +1028,10 @@ __global__ void __launch_bounds__(32 * kCombWarps) decode_combine(const float* _
 #pragma unroll 4
       for (int j = 0; j < cnt; ++j) {
         const float wj = __shfl_sync(kFull, w, j);
-        const float* os = ob + size_t(s0 + j) * o_stride;
+        const uint16_t* os = ob + size_t(s0 + j) * o_stride;
         float4 v[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) v[q] = __ldcg(reinterpret_cast<const float4*>(os + 128 * q));
+        for (int q = 0; q < 4; ++q) v[q] = ld_bf16x4(os + 128 * q);
         if (wj != 0.f) {  // an empty partial's O is never read
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -1072,7 +1078,7 @@ __global__ void __launch_bounds__(32 * kCombWarps) decode_combine(const float* _
 constexpr int kWideWarps = 8;
 
 template <int CB>
-__global__ void __launch_bounds__(32 * kWideWarps, CB == 1 ? 4 : 2) decode_combine_wide(const float* __restrict__ o_part,
+__global__ void __launch_bounds__(32 * kWideWarps, CB == 1 ? 4 : 2) decode_combine_wide(const uint16_t* __restrict__ o_part,
                                                                        const float* __restrict__ ml_part,
                                                                        const float* __restrict__ rope_tab, int splits,
                                                                        int heads, int rope_dim, int out_fp32,
@@ -1089,7 +1095,7 @@ __global__ void __launch_bounds__(32 * kWideWarps, CB == 1 ? 4 : 2) decode_combi
   const int b = bh / heads, h = bh % heads;
   const size_t ml_stride = size_t(heads) * 4, o_stride = size_t(heads) * kDim;
   const float* mlb = ml_part + (size_t(b) * splits * heads + h) * 4;
-  const float* ob = o_part + (size_t(b) * splits * heads + h) * kDim + CW * cb + 4 * lane;
+  const uint16_t* ob = o_part + (size_t(b) * splits * heads + h) * kDim + CW * cb + 4 * lane;
   // maxima over all splits
   float mo = -INFINITY, ml = -INFINITY;
   for (int s = threadIdx.x; s < splits; s += 32 * kWideWarps) {
@@ -1132,8 +1138,7 @@ __global__ void __launch_bounds__(32 * kWideWarps, CB == 1 ? 4 : 2) decode_combi
       const int s = s0 + u * kWideWarps;
 #pragma unroll
       for (int q = 0; q < Q; ++q)
-        x[u][q] = s < splits ? __ldcg(reinterpret_cast<const float4*>(ob + size_t(s) * o_stride + 128 * q))
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[u][q] = s < splits ? ld_bf16x4(ob + size_t(s) * o_stride + 128 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -1202,7 +1207,7 @@ Plan make_plan(int batch, int comp_tiles, int win_tiles) {
 
 struct DecodeWs {
   uint32_t* status;
-  float* o_part;
+  uint16_t* o_part;
   float* ml_part;
   float* rope_tab;
   size_t bytes;
@@ -1217,7 +1222,7 @@ DecodeWs decode_ws_layout(char* base, int batch, int heads, const Plan& pl) {
     return p;
   };
   w.status = reinterpret_cast<uint32_t*>(take(16));
-  w.o_part = reinterpret_cast<float*>(take(sizeof(float) * size_t(batch) * pl.splits * heads * kDim));
+  w.o_part = reinterpret_cast<uint16_t*>(take(sizeof(uint16_t) * size_t(batch) * pl.splits * heads * kDim));
   w.ml_part = reinterpret_cast<float*>(take(sizeof(float) * size_t(batch) * pl.splits * heads * 4));
   w.rope_tab = reinterpret_cast<float*>(take(sizeof(float) * size_t(batch) * kDim));
   w.bytes = off;
@@ -1346,14 +1351,14 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
   const int bh_total = a.batch * a.heads;
   if (pl.splits <= kCombFast)
     launch_pdl(decode_combine, dim3((bh_total + kCombWarps - 1) / kCombWarps), dim3(32 * kCombWarps), 0, stream,
-               (const float*)w.o_part, (const float*)w.ml_part, (const float*)w.rope_tab, pl.splits, a.heads,
+               (const uint16_t*)w.o_part, (const float*)w.ml_part, (const float*)w.rope_tab, pl.splits, a.heads,
                bh_total, a.rope_dim, a.out_fp32, a.out);
   else {
     // channel blocks per (sequence, head): as many as keep the grid within ~3 blocks per SM
     const int sms = sm_count();
     const int cb = bh_total * 4 <= 3 * sms ? 4 : (bh_total * 2 <= 3 * sms ? 2 : 1);
     auto kern = cb == 4 ? decode_combine_wide<4> : (cb == 2 ? decode_combine_wide<2> : decode_combine_wide<1>);
-    launch_pdl(kern, dim3(bh_total * cb), dim3(32 * kWideWarps), 0, stream, (const float*)w.o_part,
+    launch_pdl(kern, dim3(bh_total * cb), dim3(32 * kWideWarps), 0, stream, (const uint16_t*)w.o_part,
                (const float*)w.ml_part, (const float*)w.rope_tab, pl.splits, a.heads, a.rope_dim, a.out_fp32,
                a.out);
   }
