@@ -44,6 +44,9 @@ WORKLOADS = {
     # a CSA2 Reindex layer: top-512 re-indexed inside the 2048-entry pool a Full
     # layer built (the pool size is a reading; the pages give none)
     "c4a_b32_reindex": ("c4a", 32, 131072, 64, 0, 0, 2048),
+    # one c4a layer of the 61-layer stack on its own (one 1M-token sequence)
+    "c4a_b1_t1m": ("c4a", 1, 1 << 20, 64, 0, 0),
+    "c128a_b1_t1m": ("c128a", 1, 1 << 20, 64, 0, 0),
     # paged caches of a ragged batch: every sequence has its own length (uniform in
     # [t/2, t], seeded), its caches in 256-row pages of shared pools, pages shuffled
     "c4a_b32_paged": ("c4a", 32, 131072, 64, 0, 0, 0, "paged"),

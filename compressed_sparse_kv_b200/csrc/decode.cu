@@ -51,7 +51,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;    // O^T: 4 channel tiles x 64 heads
 constexpr uint32_t kColS = 256;  // scores: 2 buffers x 64 columns
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kIdxSmem = 2048;             // selected indices a CTA keeps in shared memory (k <= 2048)
 
 // Per-format configuration.  bf16 rows feed kind::f16 MMAs with bf16 inputs.
 // Quantised rows are dequantised in the load path; every E4M3 value and every
@@ -83,7 +82,6 @@ struct __align__(8) Ctl {
   float row_ls[kStages][kTileRows];   // log2 of the row scale (-inf: no row)
   float row_inv[kStages][kTileRows];  // 1 / row scale (0: no row)
   uint32_t vmask[kStages][4];  // row validity of a gathered tile, 16 rows per loader warp
-  int32_t idx_s[kIdxSmem];     // the selected indices of this CTA's compressed tiles
   float rope_cs[kDim / 2];  // inverse-RoPE rotation of pair m: cos / sin of -t * theta_m
   float rope_sn[kDim / 2];
 };
@@ -171,7 +169,6 @@ __device__ __forceinline__ bool named_bar_or(bool pred) {
   return r != 0;
 }
 __device__ __forceinline__ void named_bar_sync() { asm volatile("barrier.cta.sync 1, 128;" ::: "memory"); }
-__device__ __forceinline__ void loader_bar_sync() { asm volatile("barrier.cta.sync 2, 128;" ::: "memory"); }
 
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
@@ -252,14 +249,13 @@ struct RowSrc {
   int64_t row;
   bool valid, from_win;
 };
-__device__ __forceinline__ RowSrc row_source(const Params& p, const Seq& q, int b, int T, int r,
-                                             const int32_t* idx_s = nullptr, int slot0 = 0) {
+__device__ __forceinline__ RowSrc row_source(const Params& p, const Seq& q, int b, int T, int r) {
   RowSrc s{0, false, false};
   if (T < q.comp_tiles) {
     const int slot = T * kTileRows + r;
     int64_t i = -1;
     if (p.idx) {
-      const int32_t v = slot >= p.k ? -1 : (idx_s ? idx_s[slot - slot0] : p.idx[size_t(b) * p.k + slot]);
+      const int32_t v = slot >= p.k ? -1 : __ldg(p.idx + size_t(b) * p.k + slot);
       if (v >= q.n) set_status(p.status, DSV4KV_DEV_BAD_INDEX);
       i = v;
     } else if (slot < q.n) {
@@ -357,9 +353,8 @@ struct QuantLoad {
   float my_scale;     // row-scale formats: the scale of row 16 lw + lane (lanes < 16)
   uint32_t vb;        // rows of the warp's part that exist
 
-  __device__ __forceinline__ void fetch(const Params& p, const Seq& q, int b, int T, int lw, int lane,
-                                        const int32_t* idx_s, int slot0) {
-    const RowSrc mine = row_source(p, q, b, T, 16 * lw + (lane & 15), idx_s, slot0);
+  __device__ __forceinline__ void fetch(const Params& p, const Seq& q, int b, int T, int lw, int lane) {
+    const RowSrc mine = row_source(p, q, b, T, 16 * lw + (lane & 15));
     vb = __ballot_sync(kFull, mine.valid) & 0xffffu;
     const uint8_t* codes = mine.from_win ? p.win_codes : p.comp_codes;
     const void* scales = mine.from_win ? p.win_scales : p.comp_scales;
@@ -842,14 +837,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ loaders (warps 6..9)
     const int lw = warp - 6;
     // the CTA's selected indices, once, into shared memory
-    const int slot0 = t0 * kTileRows;
-    const int nslots = p.idx ? min(max(0, min(p.k, (t0 + nt) * kTileRows) - slot0), kIdxSmem) : 0;
-    for (int i = threadIdx.x - 192; i < nslots; i += 128) ctl->idx_s[i] = __ldg(p.idx + size_t(b) * p.k + slot0 + i);
-    loader_bar_sync();
+    // (a lane reads the index of its row straight from idx: one load per tile)
     if constexpr (C::kQuant) {
       // the first tile's loads go out before Q's conversion waits for Q
       QuantLoad<FMT> ql;
-      if (nt > 0) ql.fetch(p, sq, b, t0, lw, lane, ctl->idx_s, slot0);
+      if (nt > 0) ql.fetch(p, sq, b, t0, lw, lane);
       // Q: bf16 -> f16 in place (saturating), once per CTA
       if (warp_wait(&ctl->q_full, 0, ctl, lane)) {
         for (int v = threadIdx.x - 192; v < kQBytes / 16; v += 128) {
@@ -869,7 +861,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->full[stage]);
-        if (i + 1 < nt) ql.fetch(p, sq, b, t0 + i + 1, lw, lane, ctl->idx_s, slot0);
+        if (i + 1 < nt) ql.fetch(p, sq, b, t0 + i + 1, lw, lane);
       }
     } else {
       // rows: warp lw covers rows 16*lw .. 16*lw+15 of every tile
@@ -879,7 +871,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* tile = sR + stage * kTileBytes;
         if (!tile_tma(p, sq, b, T)) {
           // lane j < 16 resolves row 16*lw + j; every lane reads all 16 answers
-          const RowSrc mine = row_source(p, sq, b, T, 16 * lw + (lane & 15), ctl->idx_s, slot0);
+          const RowSrc mine = row_source(p, sq, b, T, 16 * lw + (lane & 15));
           const uint32_t vb = __ballot_sync(kFull, mine.valid) & 0xffffu;
           if (lane == 0) ctl->vmask[stage][lw] = vb;
           // gathered bf16 rows: 16-byte cp.async into the 128-byte-swizzled tile
