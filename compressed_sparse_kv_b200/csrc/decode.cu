@@ -318,17 +318,17 @@ __device__ __forceinline__ void store_partial(const Params& p, int b, int split,
 #pragma unroll 1
   for (int ct = ct0; ct < ct1; ++ct) {
     const int c = 128 * ct + 32 * wq + lane;
-#pragma unroll 1
-    for (int half = 0; half < 2; ++half) {
-      uint32_t o[32];
-      tmem_ld32(tmem + lane_base + kColO + 64 * ct + 32 * half, o);
-      tmem_wait_ld();
+    uint32_t o[2][32];  // both halves of the channel tile's 64 heads behind one wait
+    tmem_ld32(tmem + lane_base + kColO + 64 * ct, o[0]);
+    tmem_ld32(tmem + lane_base + kColO + 64 * ct + 32, o[1]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int half = 0; half < 2; ++half)
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         const int hh = 32 * half + e;
-        if (hh < p.heads) op[size_t(hh) * kDim + c] = f2bf(__uint_as_float(o[e]));
+        if (hh < p.heads) op[size_t(hh) * kDim + c] = f2bf(__uint_as_float(o[half][e]));
       }
-    }
   }
 }
 
@@ -618,17 +618,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = uint32_t(32 * wq) << 16;
     const int g = lane >> 2, c2 = lane & 3;
     const int hd[2] = {16 * wq + g, 16 * wq + 8 + g};
-    // the inverse-RoPE table, while the first tile is still in flight
-    for (int m = threadIdx.x - 64; m < p.rope_dim / 2; m += 128) {
-      float cs, sn;
-      inv_rope_rotation(sq.t, m, p.rope_dim, p.rope_base, &cs, &sn);
-      ctl->rope_cs[m] = cs;
-      ctl->rope_sn[m] = sn;
-      if (p.splits > 1 && split == 0) {
-        p.rope_tab[size_t(b) * kDim + m] = cs;
-        p.rope_tab[size_t(b) * kDim + kDim / 2 + m] = sn;
-      }
-    }
     float m_o[2] = {-INFINITY, -INFINITY}, m_l[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
     bool dead = false;
     for (int i = 0; i < nt; ++i) {
@@ -771,6 +760,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->p_full[sb]);
+    }
+    // the inverse-RoPE table (fp64 angles), while the last PV finishes
+    for (int m = threadIdx.x - 64; m < p.rope_dim / 2; m += 128) {
+      float cs, sn;
+      inv_rope_rotation(sq.t, m, p.rope_dim, p.rope_base, &cs, &sn);
+      ctl->rope_cs[m] = cs;
+      ctl->rope_sn[m] = sn;
+      if (p.splits > 1 && split == 0) {
+        p.rope_tab[size_t(b) * kDim + m] = cs;
+        p.rope_tab[size_t(b) * kDim + kDim / 2 + m] = sn;
+      }
     }
     if (!dead) dead = !warp_wait(&ctl->o_done, 0, ctl, lane);
     float l_tot[2];
