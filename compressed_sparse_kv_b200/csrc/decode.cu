@@ -74,6 +74,7 @@ struct __align__(8) Ctl {
   uint64_t p_full[2];
   uint64_t pv_done[2];  // PV of the tiles that used P buffer 0 / 1
   uint64_t o_done;
+  uint64_t retire;  // one arrival per warp once it is done with TMEM and shared memory
   uint32_t tmem_base;
   volatile int abort;
   float alpha[64];
@@ -153,6 +154,15 @@ __device__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ctl* ctl) {
 }
 
 // Warp-uniform bounded wait: lane 0 polls, the result is broadcast.
+// The retire wait: unlike wait_or_abort it does not stop at the abort flag
+// (every other wait is bounded, so every warp arrives in the end); it gives
+// up only after twice the per-wait limit, and TMEM is freed either way.
+__device__ void retire_wait(uint64_t* bar) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, 0))
+    if (globaltimer() - t0 > 2 * kWaitLimitNs) return;
+}
+
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Ctl* ctl, int lane) {
   bool ok = true;
   if (lane == 0) ok = wait_or_abort(bar, parity, ctl);
@@ -493,6 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&ctl->pv_done[0], 1);
     mbar_init(&ctl->pv_done[1], 1);
     mbar_init(&ctl->o_done, 1);
+    mbar_init(&ctl->retire, kThreads / 32);
     ctl->abort = 0;
     fence_mbar_init();
   }
@@ -904,17 +915,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       store_partial(p, b, split, tmem, warp & 3, lane, kDim / 256, kDim / 128);
     }
   }
-  // every lane of a warp arrives together (lanes 1-31 of the TMA and MMA
-  // warps would otherwise reach the barrier ahead of their lane 0, and the
-  // warp count as arrived), so TMEM is freed only after all its users are done
-  __syncwarp();
+  // Retire: lane 0 of every warp arrives once the warp's own work is done
+  // (in the TMA and MMA warps only lane 0 works), and warp 1 frees TMEM after
+  // all ten arrivals.  A CTA-wide bar.sync here is not enough: its warps are
+  // diverged (lanes 1-31 of warps 0 and 1 reach the end long before lane 0),
+  // and such a barrier was seen to let warp 1 through before the epilogue
+  // warps had finished reading TMEM.
   tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&ctl->retire);
   if (warp == 1) {
+    if (lane == 0) retire_wait(&ctl->retire);
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+    if (lane == 0 && ctl->abort) set_status(p.status, DSV4KV_DEV_TIMEOUT);
   }
-  if (threadIdx.x == 0 && ctl->abort) set_status(p.status, DSV4KV_DEV_TIMEOUT);
 }
 
 // Merge split partials, normalise, inverse RoPE.  Per split: O_s (weights
