@@ -11,10 +11,11 @@
 //     entry to the workspace and builds a per-sequence histogram of the top
 //     12 bits of the order-preserving score code.
 //  2. index_select: several CTAs per sequence filter the scores against the
-//     threshold bin of that histogram into a candidate list; the last of them
-//     resolves the exact selection from the candidates (second-level
-//     histogram, ranked ties, index-ordered output) and re-zeroes the
-//     sequence's counters.
+//     threshold bin of that histogram into a candidate list; the first of
+//     them resolves the exact selection from the candidates (two more
+//     histogram levels down to the exact threshold code, the lowest indices
+//     among equal scores, index-ordered output) and the sequence's histogram
+//     is re-zeroed.
 //  (only when n <= k) index_fill_all writes 0..n-1 directly.
 // The order (score desc, index asc) is a total order, so the result is the
 // same for every split of the entries (exact, not approximate).
@@ -440,11 +441,13 @@ __global__ void __launch_bounds__(256) index_score_fp4(const uint16_t* __restric
 // leader CTA reads every CTA's list through distributed shared memory, in
 // chunk order, so the candidates arrive sorted by index; the other CTAs wait
 // at a second barrier until it has, then exit.  The leader resolves the exact
-// selection from the candidates alone: the second-level histogram of the
-// entries in b1 gives the 24-bit threshold prefix; entries above it are in;
-// the entries at it are ranked by (score desc, index asc) and the best fill
-// what is missing; an ordered compaction writes the result in ascending index
-// order.  It re-zeroes the sequence's histogram for the next call.
+// selection from the candidates alone: the histogram of bits 8-19 of the
+// codes in b1 gives the 24-bit threshold prefix, the histogram of bits 0-7 of
+// the codes at that prefix the exact threshold code T; every code above T is
+// in, and of the codes equal to T (equal scores) the earliest positions
+// (lowest indices) fill what is missing, found by an ordered scan; an ordered
+// compaction writes the result in ascending index order.  The sequence's
+// histogram is re-zeroed for the next call.
 constexpr int kSelThreads = 512;
 constexpr int kSelBatch = 8;                           // scores per lane and warp batch
 constexpr int kSelWarps = kSelThreads / 32;
@@ -453,7 +456,6 @@ constexpr int kSelChunkUnit = 4096;                    // CTA chunks are multipl
 constexpr int kSelStage = 4096;                        // candidates a CTA can hold
 constexpr int kCandCap = 8192;                         // candidates per sequence the leader can resolve
 constexpr int kResPer = kCandCap / kSelThreads;        // candidates per leader thread
-constexpr int kTieCap = 2048;
 constexpr int kMaxClusterSel = 16;
 constexpr int kWarpCap = kSelStage / kSelWarps;       // candidates a warp's list can hold
 // Every warp streams its run of scores through its own ring of kRing slots
@@ -461,12 +463,10 @@ constexpr int kWarpCap = kSelStage / kSelWarps;       // candidates a warp's lis
 // cp.async copies kRing - 1 batches ahead of the one it filters.
 constexpr int kRing = 4;
 constexpr size_t kRingBytes = size_t(kSelWarps) * kRing * kSelWarpSpan * sizeof(float);  // 64 KB
-// dynamic shared memory: the rings (whose first bytes the leader's tie list
-// reuses after the filter), the warps' lists (kSelStage u64), and the
+// dynamic shared memory: the rings, the warps' lists (kSelStage u64), and the
 // leader's receive buffer (kCandCap): CTA r of the cluster pushes its list
 // into region r (kCandCap / C entries)
 constexpr size_t kSelDyn = kRingBytes + (size_t(kSelStage) + kCandCap) * sizeof(uint64_t);
-static_assert(kTieCap * (sizeof(uint64_t) + sizeof(uint32_t)) <= kRingBytes, "the tie list fits the ring area");
 
 // Block-wide exclusive prefix sum of one value per thread (NT threads).
 template <int NT>
@@ -503,6 +503,15 @@ __device__ __forceinline__ uint32_t warp_inclusive_scan(uint32_t v) {
   return v;
 }
 
+// Adds 1 to bin `bin` of the shared histogram h for every active lane, one
+// atomic per distinct bin of the warp: lanes with equal bins (common when
+// many scores are equal) are counted by their lowest lane.
+__device__ __forceinline__ void hist_add_warp(uint32_t* h, bool active, uint32_t bin) {
+  if (!__any_sync(kFull, active)) return;
+  const uint32_t peers = __match_any_sync(kFull, active ? bin : 0xffffffffu);
+  if (active && __ffs(peers) - 1 == int(threadIdx.x & 31)) atomicAdd(&h[bin], uint32_t(__popc(peers)));
+}
+
 // The bin where the descending cumulative count of the 4096-bin histogram h
 // (shared memory, 16-byte aligned) first reaches `need` (1 <= need <= sum h);
 // *above = count in higher bins.  Warp w owns the S = 4096/warps highest bins
@@ -533,7 +542,8 @@ __device__ int find_threshold_bin(const uint32_t* h, uint32_t need, uint32_t* ab
   if (lane == 31) s_wtot[warp] = incl;
   __syncthreads();
   uint32_t before = 0;
-  for (int w = 0; w < warp; ++w) before += s_wtot[w];
+#pragma unroll
+  for (int w = 0; w < NW; ++w) before += w < warp ? s_wtot[w] : 0u;  // independent loads, no chain
   const uint32_t ex = before + incl - sum;  // entries in higher bins than this run
   if (ex < need && ex + sum >= need) {      // exactly one lane: walk its run from the top
     uint32_t c = ex;
@@ -593,19 +603,67 @@ __device__ uint32_t ordered_offsets(const uint32_t (&m)[BATCH], uint32_t (&off)[
   return total;
 }
 
+// ordered_offsets for two predicates at once: off[j] receives (count of a
+// before lane 0 of (j, warp)) << 16 | (count of e before it); returns the
+// totals packed the same way.  Every count must stay below 2^16.
+template <int NT, int BATCH>
+__device__ uint32_t ordered_offsets_pair(const uint32_t (&a)[BATCH], const uint32_t (&e)[BATCH],
+                                         uint32_t (&off)[BATCH]) {
+  constexpr int NW = NT / 32, E = BATCH * NW, PER = E / 32;
+  static_assert(PER * 32 == E, "entries per lane");
+  __shared__ uint32_t s_c[E];
+  __shared__ uint32_t s_total;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) {
+#pragma unroll
+    for (int j = 0; j < BATCH; ++j) s_c[j * NW + warp] = (uint32_t(__popc(a[j])) << 16) | uint32_t(__popc(e[j]));
+  }
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t x[PER], loc = 0;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      x[q] = s_c[PER * lane + q];
+      loc += x[q];
+    }
+    const uint32_t incl = warp_inclusive_scan(loc);
+    uint32_t run = incl - loc;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      s_c[PER * lane + q] = run;
+      run += x[q];
+    }
+    if (lane == 31) s_total = incl;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < BATCH; ++j) off[j] = s_c[j * NW + warp];
+  const uint32_t total = s_total;
+  __syncthreads();  // s_c is rewritten by the next call
+  return total;
+}
+
 // Copies a sequence's 4096-bin histogram from the workspace (L2) into shared
-// memory in bin order, with every load of a thread issued before its stores.
+// memory in bin order: fetch() issues a thread's loads, store() writes them.
 // Lane l of warp w takes the 16-byte group q = 32 l + (w + j NW) of
 // positions (iteration j): the four bins of a group are 32 apart and the
 // lanes' bins fall in 32 different banks.
 template <int NT>
-__device__ __forceinline__ void load_histogram(const uint32_t* __restrict__ hb, uint32_t* sh) {
-  constexpr int NW = NT / 32, V = 32 / NW;  // uint4 per thread
+struct HistLoad {
+  static constexpr int NW = NT / 32, V = 32 / NW;  // uint4 per thread
   static_assert(V * NW == 32 && V * 4 * NT == kHistBins, "histogram split");
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint4 v[V];
+  // the loads (issued before anything else the thread asks of memory)
+  __device__ __forceinline__ void fetch(const uint32_t* __restrict__ hb) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-  for (int j = 0; j < V; ++j) v[j] = __ldcg(reinterpret_cast<const uint4*>(hb) + 32 * lane + warp + j * NW);
+    for (int j = 0; j < V; ++j) v[j] = __ldcg(reinterpret_cast<const uint4*>(hb) + 32 * lane + warp + j * NW);
+  }
+  __device__ __forceinline__ void store(uint32_t* sh) const;
+};
+template <int NT>
+__device__ __forceinline__ void HistLoad<NT>::store(uint32_t* sh) const {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int j = 0; j < V; ++j) {
     const int p = 4 * (32 * lane + warp + j * NW);  // positions p .. p + 3
@@ -662,8 +720,8 @@ __device__ __forceinline__ uint32_t warp_stage_batch(const uint32_t (&o)[kSelBat
   return count;
 }
 
-// Exact selection with no candidate list (overflow, or more than kTieCap
-// entries at the prefix): the threshold code o* from the low 8 bits of the
+// Exact selection with no candidate list (the candidates overflowed the
+// leader's buffer): the threshold code o* from the low 8 bits of the
 // entries at the 24-bit prefix, then one ordered scan of all scores keeps
 // codes > o* and the first r codes == o* (the lowest indices), in index order.
 template <int NT>
@@ -997,8 +1055,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
   __shared__ uint32_t s_wcnt[kSelWarps];
   __shared__ uint32_t s_rcnt[kMaxClusterSel];  // leader: the count each CTA pushed (~0u: overflow)
   __shared__ __align__(16) uint32_t sh[kHistBins];
-  __shared__ uint32_t s_ntie;
-  __shared__ uint32_t s_keep[kCandCap / 32];  // tie verdicts by candidate position
+  __shared__ uint32_t s_h3[256];  // leader: histogram of the low 8 code bits at the 24-bit prefix
+  __shared__ uint32_t s_low, s_above3;
   __shared__ uint32_t s_pre[kMaxClusterSel + 1];
 
   const int b = blockIdx.y;
@@ -1033,12 +1091,14 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
   const int64_t w0 = min(n1, n0 + int64_t(warp) * wspan), w1 = min(n1, w0 + wspan);
   const int64_t nbat = (w1 - w0 + kSelWarpSpan - 1) / kSelWarpSpan;
   float* ring = reinterpret_cast<float*>(stage) + size_t(warp) * kRing * kSelWarpSpan;
+  HistLoad<kSelThreads> hl;
+  hl.fetch(hb);  // first: the threshold waits for it, the batches are needed only after
 #pragma unroll
   for (int t = 0; t < kRing - 1; ++t) {
     if (t < nbat) warp_issue_batch(sc, w0 + int64_t(t) * kSelWarpSpan, w1, ring + t * kSelWarpSpan);
     cp_async_commit();
   }
-  load_histogram<kSelThreads>(hb, sh);
+  hl.store(sh);
   __syncthreads();
   uint32_t above1;
   const int bin1 = find_threshold_bin<kSelThreads>(sh, kk, &above1);
@@ -1088,8 +1148,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
   }
   if (rank == 0) {  // the leader's resolve state, cleared while the other CTAs finish
     for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) sh[i] = 0;
-    for (int i = threadIdx.x; i < kCandCap / 32; i += kSelThreads) s_keep[i] = 0;
-    if (threadIdx.x == 0) s_ntie = 0;
+    for (int i = threadIdx.x; i < 256; i += kSelThreads) s_h3[i] = 0;
   }
   cluster_sync();  // every list is in the leader's shared memory
   if (rank != 0) {
@@ -1113,6 +1172,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
   __syncthreads();
   total = s_pre[csize];
   fits = total <= uint32_t(kCandCap);
+  const int J = int((total + kSelThreads - 1) / kSelThreads);  // candidate rounds in use (block-uniform)
   if (fits) {
     // the region of every position (offsets in registers, a branch-free
     // search: offsets are non-decreasing, the last one <= g holds g)
@@ -1121,6 +1181,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
     for (int i = 0; i < kMaxClusterSel; ++i) pre[i] = i < int(csize) ? s_pre[i] : 0xffffffffu;
 #pragma unroll
     for (int j = 0; j < kResPer; ++j) {
+      c[j] = 0ull;
+      if (j >= J) continue;
       const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
       uint32_t r = 0, base = 0;
 #pragma unroll
@@ -1129,84 +1191,87 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
         r = past ? uint32_t(i) : r;
         base = past ? pre[i] : base;
       }
-      c[j] = g < total ? recv[size_t(r) * regcap + (g - base)] : 0ull;
+      if (g < total) c[j] = recv[size_t(r) * regcap + (g - base)];
     }
   }
 
-  // 5) resolve
+  // 5) resolve: the exact threshold code T from two more histogram levels
+  //    over the candidates; codes above T are kept, and of the codes equal to
+  //    T (equal scores) the first need_eq by position (= by index)
   int32_t* out = idx_out + size_t(b) * k;
   const uint32_t need1 = kk - above1;  // still needed from bin1 (>= 1)
-  uint64_t* ties = stage;              // the leader's list is in registers now
+  const uint32_t lt = (1u << lane) - 1u;
   bool ok = false;
   uint32_t prefix = 0, need_tie = 0;
   if (fits) {
-    // second-level histogram of bin1 (every entry of bin1 is a candidate)
+    // bits 8-19 of the codes in bin1 (every entry of bin1 is a candidate)
 #pragma unroll
     for (int j = 0; j < kResPer; ++j) {
       const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
       const uint32_t o = uint32_t(c[j] >> 32);
-      if (g < total && int(o >> 20) == bin1) atomicAdd(&sh[(o >> 8) & 0xfffu], 1u);
+      if (j < J) hist_add_warp(sh, g < total && int(o >> 20) == bin1, (o >> 8) & 0xfffu);
     }
     __syncthreads();
     uint32_t above2;
     const int bin2 = find_threshold_bin<kSelThreads>(sh, need1, &above2);
     prefix = (uint32_t(bin1) << 12) | uint32_t(bin2);  // 24-bit threshold prefix
     need_tie = need1 - above2;                          // >= 1
-    // every entry at the prefix is needed (the usual case: one entry at a
-    // 24-bit prefix) -> no ranking; else rank the entries at the prefix
-    const bool all_at = sh[bin2] == need_tie;
-    if (!all_at) {
-      // the entries at the prefix: (key, position) into the tie list
+    // bits 0-7 of the codes at the prefix
 #pragma unroll
-      for (int j = 0; j < kResPer; ++j) {
-        const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
-        if (g < total && uint32_t(c[j] >> 40) == prefix) {
-          const uint32_t slot = atomicAdd(&s_ntie, 1u);
-          if (slot < uint32_t(kTieCap)) {
-            ties[slot] = c[j];
-            reinterpret_cast<uint32_t*>(ties + kTieCap)[slot] = g;
-          }
-        }
-      }
-      __syncthreads();
+    for (int j = 0; j < kResPer; ++j) {
+      const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
+      const uint32_t o = uint32_t(c[j] >> 32);
+      if (j < J) hist_add_warp(s_h3, g < total && (o >> 8) == prefix, o & 0xffu);
     }
-    const uint32_t n_tie = all_at ? 0u : s_ntie;
-    if (n_tie <= uint32_t(kTieCap)) {
-      ok = true;
-      // a tie is kept when fewer than need_tie keys (score desc, index asc) exceed its own
-      if (!all_at) {
-        for (uint32_t t = threadIdx.x; t < n_tie; t += kSelThreads) {
-          const uint64_t key = ties[t];
-          uint32_t r = 0;
-          for (uint32_t u = 0; u < n_tie; ++u) r += ties[u] > key ? 1u : 0u;
-          if (r < need_tie) {
-            const uint32_t g = reinterpret_cast<const uint32_t*>(ties + kTieCap)[t];
-            atomicOr(&s_keep[g >> 5], 1u << (g & 31));
+    __syncthreads();
+    if (warp == 0) {  // lane l owns bins 255 - 8l - 7 .. 255 - 8l (descending lane order)
+      uint32_t v[8], sum = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[i] = s_h3[255 - 8 * lane - i];
+        sum += v[i];
+      }
+      const uint32_t incl = warp_inclusive_scan(sum);
+      uint32_t cnt = incl - sum;
+      if (cnt < need_tie && incl >= need_tie) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (cnt < need_tie && cnt + v[i] >= need_tie) {
+            s_low = uint32_t(255 - 8 * lane - i);
+            s_above3 = cnt;
           }
-        }
-        __syncthreads();
-      }
-      // ordered compaction of the kept candidates
-      uint32_t m[kResPer], off[kResPer];
-#pragma unroll
-      for (int j = 0; j < kResPer; ++j) {
-        const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
-        const uint32_t pre = uint32_t(c[j] >> 40);
-        const bool keep =
-            g < total && (pre > prefix || (pre == prefix && (all_at || ((s_keep[g >> 5] >> (g & 31)) & 1u))));
-        m[j] = __ballot_sync(kFull, keep);
-      }
-      const uint32_t got = ordered_offsets<kSelThreads, kResPer>(m, off);
-      const uint32_t lt = (1u << lane) - 1u;
-#pragma unroll
-      for (int j = 0; j < kResPer; ++j) {
-        if ((m[j] >> lane) & 1u) {
-          const uint32_t at = off[j] + __popc(m[j] & lt);
-          if (at < kk) out[at] = int32_t(0xffffffffu - uint32_t(c[j]));
+          cnt += v[i];
         }
       }
-      if (threadIdx.x == 0 && got != kk) set_status(status, DSV4KV_DEV_INCONSISTENT);
     }
+    __syncthreads();
+    const uint32_t tcode = (prefix << 8) | s_low;
+    const uint32_t need_eq = need_tie - s_above3;  // codes equal to T to keep (>= 1)
+    // one ordered scan counts, before every position, the codes above T and
+    // the codes equal to T; an entry's output slot is (above before) +
+    // min(equal before, need_eq), so the kept entries come out in index order
+    uint32_t mg[kResPer], me[kResPer], off[kResPer];
+#pragma unroll
+    for (int j = 0; j < kResPer; ++j) {
+      const uint32_t g = threadIdx.x + uint32_t(j) * kSelThreads;
+      const uint32_t o = uint32_t(c[j] >> 32);
+      mg[j] = j < J ? __ballot_sync(kFull, g < total && o > tcode) : 0u;
+      me[j] = j < J ? __ballot_sync(kFull, g < total && o == tcode) : 0u;
+    }
+    const uint32_t tot = ordered_offsets_pair<kSelThreads, kResPer>(mg, me, off);
+    const uint32_t got = (tot >> 16) + min(tot & 0xffffu, need_eq);
+#pragma unroll
+    for (int j = 0; j < kResPer; ++j) {
+      const uint32_t gt_before = (off[j] >> 16) + __popc(mg[j] & lt);
+      const uint32_t eq_before = (off[j] & 0xffffu) + __popc(me[j] & lt);
+      const bool gt = (mg[j] >> lane) & 1u, eq = (me[j] >> lane) & 1u;
+      if (gt || (eq && eq_before < need_eq)) {
+        const uint32_t at = gt_before + min(eq_before, need_eq);
+        if (at < kk) out[at] = int32_t(0xffffffffu - uint32_t(c[j]));
+      }
+    }
+    if (threadIdx.x == 0 && got != kk) set_status(status, DSV4KV_DEV_INCONSISTENT);
+    ok = true;
   }
   __syncthreads();
   if (!ok) {
