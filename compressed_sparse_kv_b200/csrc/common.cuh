@@ -97,6 +97,29 @@ __device__ __forceinline__ void st_dsmem_u32(uint32_t addr, uint32_t v) {
 __device__ __forceinline__ void st_dsmem_u64(uint32_t addr, uint64_t v) {
   asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
 }
+__device__ __forceinline__ void st_dsmem_f4(uint32_t addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+// A cluster barrier for warp-specialised kernels whose warps may be diverged
+// when they reach it (no .aligned): release / acquire order every earlier
+// shared-memory and global access of the arriving thread before every later
+// one of the waiting threads.
+__device__ __forceinline__ void cluster_arrive_release_div() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire_div() {
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
 
 // ----------------------------------------------------------------- programmatic dependent launch
 // Every kernel of the library is launched with programmatic stream

@@ -30,6 +30,7 @@
 // workspace and decode_combine merges them with log-sum-exp weights.
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 
 #include "common.cuh"
 #include "internal.h"
@@ -64,7 +65,7 @@ struct Cfg {
   static constexpr uint32_t kIdescPV = kQuant ? idesc_f16(128, 64, 1, 0) : idesc_bf16(128, 64, 1, 0);
 };
 
-struct __align__(8) Ctl {
+struct __align__(16) Ctl {
   uint64_t q_full;
   uint64_t q_ready;
   uint64_t full[kStages];
@@ -85,6 +86,11 @@ struct __align__(8) Ctl {
   uint32_t vmask[kStages][4];  // row validity of a gathered tile, 16 rows per loader warp
   float rope_cs[kDim / 2];  // inverse-RoPE rotation of pair m: cos / sin of -t * theta_m
   float rope_sn[kDim / 2];
+  // in-cluster merge: this split's (m_o, m_l, l) per head, read by every CTA
+  // of the cluster; the merged statistics; this split's weight per head
+  float4 st[64];
+  float4 gst[64];
+  float a_self[64];
 };
 
 constexpr size_t kSmemBytes = 1024 + kQBytes + kStages * kTileBytes + 2 * kPBytes + sizeof(Ctl);
@@ -119,6 +125,7 @@ struct Params {
   uint16_t* o_part;   // [B][splits][H][512] bf16 (the split's unnormalised output)
   float* ml_part;     // [B][splits][H][4]: (m_o, m_l, l, 0)
   float* rope_tab;    // [B][2][256]: the rotation tables for decode_combine (written by split 0)
+  int cluster;        // CTAs per thread-block cluster (consecutive splits), merged in the kernel; 1 = none
   uint32_t* status;
   // direct output when splits == 1
   int64_t t;
@@ -472,6 +479,162 @@ struct QuantLoad {
   }
 };
 
+// In-cluster merge of a sequence's splits.  The C CTAs of a cluster (C a
+// power of two <= 16) hold consecutive splits; each holds its unnormalised
+// O^T in TMEM and its per-head (m_o, m_l, l) in ctl->st.  The 512 channels
+// form 16 units of 32 (channel tile ct, lane quarter wq; unit 4 ct + wq) and
+// CTA r owns units [16 r / C, 16 (r + 1) / C).  After a cluster barrier
+// (every split's statistics are final and every CTA is done with its tiles,
+// whose shared memory becomes the receive buffer) each CTA forms the merged
+// statistics, scales its O^T by its weight 2^(m_o - M_o) and stores every
+// unit it does not own into the owner's buffer (distributed shared memory,
+// 16-byte stores); after a second barrier each owner adds its own TMEM part
+// to what it received.  When the cluster spans all splits the owner
+// normalises (2^(M_o - M_l) / L), applies the inverse RoPE and writes the
+// output; otherwise it writes one merged partial per cluster (group) for
+// decode_combine.  Receive buffer (floats): [sender][unit][head / 4][32
+// channels][4 heads], 8 KB per (sender, unit), 128 KB in all.
+__device__ __forceinline__ void named_bar_sync_256() { asm volatile("barrier.cta.sync 2, 256;" ::: "memory"); }
+
+__device__ __forceinline__ void cluster_merge(const Params& p, const Seq& sq, Ctl* ctl, float* buf, uint32_t tmem, int b,
+                                           int split, int warp, int lane) {
+  const int C = p.cluster, U = 16 / C;
+  const int self = int(cluster_rank());
+  const bool final_out = C == p.splits;
+  // 1) every CTA's statistics are published and its tiles consumed
+  __syncwarp();
+  cluster_arrive_release_div();
+  cluster_wait_acquire_div();
+  // this CTA has an accumulator (it ran tiles, and no wait gave up)
+  const bool own = sq.nt > 0 && !ctl->abort;
+  if (warp >= 2) {
+    tc_fence_after();
+    if (warp < 4) {  // one thread per head: the merged statistics
+      const int h = threadIdx.x - 64;
+      // running (M_o, M_l, L) over the splits' terms (L relative to 2^M_l)
+      float mo = -INFINITY, ml = -INFINITY, L = 0.f, mine = -INFINITY;
+#pragma unroll 1
+      for (int r = 0; r < C; ++r) {
+        const float4 v = ld_dsmem_f4(dsmem_addr(&ctl->st[h], uint32_t(r)));
+        mo = fmaxf(mo, v.x);
+        if (r == self) mine = v.x;
+        if (v.y != -INFINITY) {
+          if (v.y > ml) {
+            L = (ml == -INFINITY ? 0.f : L * fast_exp2(ml - v.y)) + v.z;
+            ml = v.y;
+          } else {
+            L += v.z * fast_exp2(v.y - ml);
+          }
+        }
+      }
+      ctl->a_self[h] = (own && mine != -INFINITY) ? fast_exp2(mine - mo) : 0.f;
+      ctl->fin[h] = (mo == -INFINITY || !(L > 0.f)) ? 0.f : fast_exp2(mo - ml) / L;
+      ctl->gst[h] = make_float4(mo, ml, L, 0.f);
+    }
+    named_bar_sync_256();
+    // 2) scaled O^T of the units this CTA does not own, to their owners
+    const int wq = warp & 3, half = warp >= 6 ? 1 : 0;
+    const uint32_t lane_base = uint32_t(32 * wq) << 16;
+#pragma unroll 1
+    for (int ct = 0; ct < kDim / 128; ++ct) {
+      const int u = 4 * ct + wq, owner = u / U;
+      if (owner == self) continue;
+      uint32_t o[32];
+      if (own) {
+        tmem_ld32(tmem + lane_base + kColO + 64 * ct + 32 * half, o);
+        tmem_wait_ld();
+      }
+      const uint32_t dst =
+          dsmem_addr(buf + size_t((self * U + (u - owner * U)) * 16 + 8 * half) * 128 + 4 * lane, uint32_t(owner));
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        float w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float a = ctl->a_self[32 * half + 4 * q + k];
+          w[k] = (own && a != 0.f) ? __uint_as_float(o[4 * q + k]) * a : 0.f;
+        }
+        st_dsmem_f4(dst + uint32_t(q) * 512u, make_float4(w[0], w[1], w[2], w[3]));
+      }
+    }
+  }
+  // 3) every contribution is in its owner's buffer
+  __syncwarp();
+  cluster_arrive_release_div();
+  cluster_wait_acquire_div();
+  if (warp < 2) return;
+  const int wq = warp & 3, half = warp >= 6 ? 1 : 0;
+  const uint32_t lane_base = uint32_t(32 * wq) << 16;
+  const int r0 = kDim - p.rope_dim, groups = p.splits / C, g = split / C;
+#pragma unroll 1
+  for (int ct = 0; ct < kDim / 128; ++ct) {
+    const int u = 4 * ct + wq;
+    if (u / U != self) continue;
+    const int ul = u - self * U;
+    float acc[32];
+    {
+      uint32_t o[32];
+      if (own) {
+        tmem_ld32(tmem + lane_base + kColO + 64 * ct + 32 * half, o);
+        tmem_wait_ld();
+      }
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float a = ctl->a_self[32 * half + e];
+        acc[e] = (own && a != 0.f) ? __uint_as_float(o[e]) * a : 0.f;
+      }
+    }
+#pragma unroll 1
+    for (int s = 0; s < C; ++s) {
+      if (s == self) continue;
+      const float* src = buf + size_t((s * U + ul) * 16 + 8 * half) * 128 + 4 * lane;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 v = *reinterpret_cast<const float4*>(src + 128 * q);
+        acc[4 * q] += v.x;
+        acc[4 * q + 1] += v.y;
+        acc[4 * q + 2] += v.z;
+        acc[4 * q + 3] += v.w;
+      }
+    }
+    const int c = 128 * ct + 32 * wq + lane;
+    if (final_out) {
+      const bool rot = c >= r0;
+      const float cs = rot ? ctl->rope_cs[(c - r0) >> 1] : 1.f;
+      const float sn = rot ? ctl->rope_sn[(c - r0) >> 1] : 0.f;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int hh = 32 * half + e;
+        const float f = ctl->fin[hh];
+        float v = f != 0.f ? acc[e] * f : 0.f;
+        const float partner = __shfl_xor_sync(kFull, v, 1);  // channel c ^ 1 of the same head
+        if (rot) v = (c & 1) ? partner * sn + v * cs : v * cs - partner * sn;
+        if (hh < p.heads) {
+          const size_t oi = (size_t(b) * p.heads + hh) * kDim + c;
+          if (p.out_fp32) static_cast<float*>(p.out)[oi] = v;
+          else static_cast<uint16_t*>(p.out)[oi] = f2bf(v);
+        }
+      }
+    } else {
+      uint16_t* op = p.o_part + (size_t(b) * groups + g) * size_t(p.heads) * kDim + c;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int hh = 32 * half + e;
+        if (hh < p.heads) op[size_t(hh) * kDim] = f2bf(acc[e]);
+      }
+    }
+  }
+  // the group's merged statistics (one CTA writes them)
+  if (!final_out && self == 0 && warp >= 2 && warp < 4) {
+    const int h = threadIdx.x - 64;
+    if (h < p.heads) {
+      const float4 gs = ctl->gst[h];
+      *reinterpret_cast<float4*>(p.ml_part + ((size_t(b) * groups + g) * p.heads + h) * 4) =
+          gs.x == -INFINITY ? make_float4(-INFINITY, -INFINITY, 0.f, 0.f) : gs;
+    }
+  }
+}
+
 template <int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_comp,
@@ -778,7 +941,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       inv_rope_rotation(sq.t, m, p.rope_dim, p.rope_base, &cs, &sn);
       ctl->rope_cs[m] = cs;
       ctl->rope_sn[m] = sn;
-      if (p.splits > 1 && split == 0) {
+      if (p.splits > p.cluster && split == 0) {  // (decode_combine reads it)
         p.rope_tab[size_t(b) * kDim + m] = cs;
         p.rope_tab[size_t(b) * kDim + kDim / 2 + m] = sn;
       }
@@ -790,7 +953,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       l_tot[hh] = l[hh] + __shfl_xor_sync(kFull, l[hh], 1);
       l_tot[hh] += __shfl_xor_sync(kFull, l_tot[hh], 2);
     }
-    if (p.splits > 1) {
+    if (p.cluster > 1) {
+      // the cluster merges the splits (cluster_merge, below): publish this split's statistics
+      if (c2 == 0) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          ctl->st[hd[hh]] = dead ? make_float4(-INFINITY, -INFINITY, 0.f, 0.f)  // an empty split
+                                 : make_float4(m_o[hh], m_l[hh], l_tot[hh], 0.f);
+      }
+    } else if (p.splits > 1) {
       if (!dead) {  // channel tiles 0-1; the loader warp of the same lane quarter writes 2-3
         tc_fence_after();
         store_partial(p, b, split, tmem, wq, lane, 0, kDim / 256);
@@ -910,11 +1081,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     // the other half of the partial O^T (this warp's TMEM lane quarter is warp % 4)
-    if (p.splits > 1 && warp_wait(&ctl->o_done, 0, ctl, lane)) {
+    if (p.cluster == 1 && p.splits > 1 && warp_wait(&ctl->o_done, 0, ctl, lane)) {
       tc_fence_after();
       store_partial(p, b, split, tmem, warp & 3, lane, kDim / 256, kDim / 128);
     }
   }
+  if (p.cluster > 1) cluster_merge(p, sq, ctl, reinterpret_cast<float*>(smem), tmem, b, split, warp, lane);
   // Retire: lane 0 of every warp arrives once the warp's own work is done
   // (in the TMA and MMA warps only lane 0 works), and warp 1 frees TMEM after
   // all ten arrivals.  A CTA-wide bar.sync here is not enough: its warps are
@@ -1248,18 +1420,102 @@ size_t decode_ws_bytes(int batch, int heads, int dim, int64_t rows_per_seq) {
   return decode_ws_layout(nullptr, batch, heads, pl).bytes;
 }
 
+// Shared-memory limit and cluster permission of decode_kernel<FMT>, once per device.
+template <int FMT>
+bool setup_fmt() {
+  static std::atomic<uint64_t> attr_set{0};  // per instantiation, one bit per device
+  if (done_on_device(attr_set)) return true;
+  if (cudaFuncSetAttribute(decode_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes)) !=
+      cudaSuccess)
+    return false;
+  // clusters of 16 are beyond the portable size; without the permission the
+  // occupancy query below answers 0 for them and they are not used
+  cudaFuncSetAttribute(decode_kernel<FMT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaGetLastError();
+  mark_done_on_device(attr_set);
+  return true;
+}
+
+// How many clusters of C decode CTAs the device runs at once (0: none).
+template <int FMT>
+int active_clusters(int c) {
+  static std::atomic<int> cache[5][64];  // [log2 C][device]; 0 = not queried, -1 = none
+  int lc = 0;
+  while ((1 << lc) < c) ++lc;
+  std::atomic<int>& slot = cache[lc][current_device()];
+  int n = slot.load(std::memory_order_relaxed);
+  if (n == 0) {
+    n = -1;
+    if (setup_fmt<FMT>()) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(unsigned(c));
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = kSmemBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = unsigned(c);
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int got = 0;
+      if (cudaOccupancyMaxActiveClusters(&got, decode_kernel<FMT>, &cfg) == cudaSuccess && got > 0) n = got;
+      cudaGetLastError();
+    }
+    slot.store(n, std::memory_order_relaxed);
+  }
+  return n > 0 ? n : 0;
+}
+
 template <int FMT>
 dsv4kv_status launch_fmt(const CUtensorMap& tq, const CUtensorMap& tc, const CUtensorMap& tw, const Params& p,
                          int grid, cudaStream_t stream) {
-  static std::atomic<uint64_t> attr_set{0};  // per instantiation, one bit per device
-  if (!done_on_device(attr_set)) {
-    if (cudaFuncSetAttribute(decode_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes)) !=
-        cudaSuccess)
-      return check_launch("decode: cudaFuncSetAttribute");
-    mark_done_on_device(attr_set);
-  }
-  launch_pdl(decode_kernel<FMT>, dim3(grid), dim3(kThreads), kSmemBytes, stream, tq, tc, tw, p);
+  if (!setup_fmt<FMT>()) return check_launch("decode: cudaFuncSetAttribute");
+  if (p.cluster > 1)
+    launch_pdl_cluster(decode_kernel<FMT>, dim3(grid), dim3(kThreads), kSmemBytes, unsigned(p.cluster), stream, tq,
+                       tc, tw, p);
+  else
+    launch_pdl(decode_kernel<FMT>, dim3(grid), dim3(kThreads), kSmemBytes, stream, tq, tc, tw, p);
   return check_launch("decode_kernel");
+}
+
+// The cluster size for a batch whose plan has s0 splits per sequence: the
+// smallest power of two C >= s0 (C <= 16) whose clusters all run at once
+// merges every sequence inside the kernel (no combine launch, splits = C);
+// else the largest C that divides the split count rounded up to it, with one
+// wave of clusters and at most one CTA per SM, merges groups of C splits; 1 = none.
+// The environment variable DSV4KV_DECODE_MAX_CLUSTER (1, 2, 4, 8 or 16; read
+// at every call) caps C.  The default is 1, the plain split-and-combine path:
+// on B200, with the decode launched behind the selection kernel, the merge in
+// clusters measured slower for every workload tried (c4a B=32 decode 26.9 us
+// -> 32.7 us with C = 2, 34.4 us with C = 4; c128a B=1 t=2^20 17.4 -> 22.6 us),
+// although it saves the combine launch and the partials' round trip.
+template <int FMT>
+void choose_cluster(int batch, int s0, int* cluster, int* splits) {
+  *cluster = 1;
+  *splits = s0;
+  if (s0 <= 1) return;
+  int cmax = 1;
+  if (const char* e = std::getenv("DSV4KV_DECODE_MAX_CLUSTER")) {
+    const int v = std::atoi(e);
+    cmax = v >= 16 ? 16 : (v >= 8 ? 8 : (v >= 4 ? 4 : (v >= 2 ? 2 : 1)));
+  }
+  const int sms = sm_count();
+  for (int c = 2; c <= cmax; c *= 2)
+    if (c >= s0 && int64_t(batch) * c <= sms && active_clusters<FMT>(c) >= batch) {
+      *cluster = c;
+      *splits = c;
+      return;
+    }
+  for (int c = cmax; c >= 2; c /= 2) {
+    const int sp = (s0 + c - 1) / c * c;
+    if (sp < 2 * c || int64_t(batch) * sp > sms) continue;
+    if (int64_t(active_clusters<FMT>(c)) >= int64_t(batch) * (sp / c)) {
+      *cluster = c;
+      *splits = sp;
+      return;
+    }
+  }
 }
 
 dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream) {
@@ -1321,7 +1577,17 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
   p.n = a.n;
   p.window = a.window;
   p.k = a.idx ? a.k : 0;
-  p.splits = pl.splits;
+  int cluster = 1, splits = pl.splits;
+  switch (fmt) {
+    case DSV4KV_BF16: choose_cluster<DSV4KV_BF16>(a.batch, pl.splits, &cluster, &splits); break;
+    case DSV4KV_FP8_E4M3_ROW: choose_cluster<DSV4KV_FP8_E4M3_ROW>(a.batch, pl.splits, &cluster, &splits); break;
+    case DSV4KV_FP8_E4M3_ROW_ROPE_BF16:
+      choose_cluster<DSV4KV_FP8_E4M3_ROW_ROPE_BF16>(a.batch, pl.splits, &cluster, &splits);
+      break;
+    default: choose_cluster<DSV4KV_FP4_E2M1_G16>(a.batch, pl.splits, &cluster, &splits); break;
+  }
+  p.splits = splits;
+  p.cluster = cluster;
   p.t_seq = a.t_seq;
   p.t_max = a.t_max;
   p.stride = std::max(1, a.stride);
@@ -1345,7 +1611,7 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
   p.out_fp32 = a.out_fp32;
   p.out = a.out;
 
-  const int grid = a.batch * pl.splits;
+  const int grid = a.batch * splits;
   dsv4kv_status st;
   switch (fmt) {
     case DSV4KV_BF16: st = launch_fmt<DSV4KV_BF16>(tq, tc, tw, p, grid, stream); break;
@@ -1355,11 +1621,13 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
       break;
     default: st = launch_fmt<DSV4KV_FP4_E2M1_G16>(tq, tc, tw, p, grid, stream); break;
   }
-  if (st != DSV4KV_OK || pl.splits == 1) return st;  // one split: the decode kernel stored the output
+  // one split, or one cluster per sequence: the decode kernel stored the output
+  if (st != DSV4KV_OK || splits == 1 || cluster == splits) return st;
+  const int parts = splits / cluster;  // partials per sequence left to merge
   const int bh_total = a.batch * a.heads;
-  if (pl.splits <= kCombFast)
+  if (parts <= kCombFast)
     launch_pdl(decode_combine, dim3((bh_total + kCombWarps - 1) / kCombWarps), dim3(32 * kCombWarps), 0, stream,
-               (const uint16_t*)w.o_part, (const float*)w.ml_part, (const float*)w.rope_tab, pl.splits, a.heads,
+               (const uint16_t*)w.o_part, (const float*)w.ml_part, (const float*)w.rope_tab, parts, a.heads,
                bh_total, a.rope_dim, a.out_fp32, a.out);
   else {
     // channel blocks per (sequence, head): as many as keep the grid within ~3 blocks per SM
@@ -1367,7 +1635,7 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
     const int cb = bh_total * 4 <= 3 * sms ? 4 : (bh_total * 2 <= 3 * sms ? 2 : 1);
     auto kern = cb == 4 ? decode_combine_wide<4> : (cb == 2 ? decode_combine_wide<2> : decode_combine_wide<1>);
     launch_pdl(kern, dim3(bh_total * cb), dim3(32 * kWideWarps), 0, stream, (const uint16_t*)w.o_part,
-               (const float*)w.ml_part, (const float*)w.rope_tab, pl.splits, a.heads, a.rope_dim, a.out_fp32,
+               (const float*)w.ml_part, (const float*)w.rope_tab, parts, a.heads, a.rope_dim, a.out_fp32,
                a.out);
   }
   return check_launch("decode_combine");

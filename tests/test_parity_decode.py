@@ -140,3 +140,40 @@ def test_sparse_equals_dense_when_everything_is_selected():
     sp = K.sparse_decode(q, K.Cache(0, comp), K.Cache(0, win), idx, n, window, t, SCALE, out_fp32=True)
     de = K.dense_decode(q, K.Cache(0, comp), K.Cache(0, win), n, window, t, SCALE, out_fp32=True)
     assert_close(to_f64(sp), to_f64(de), max_abs=1e-5, rel_l2=1e-5)
+
+
+@pytest.mark.parametrize("max_cluster", ["1", "2", "16"])
+@pytest.mark.parametrize("kind,b,n,t", [
+    ("dense", 1, 8191, 1048576),   # c128a B=1: 130 tiles, merged in groups, then decode_combine(_wide)
+    ("dense", 2, 1500, 262144),    # 26 tiles per sequence
+    ("sparse", 1, 262112, 1048576),  # c4a B=1: 10 tiles, empty splits padded into one cluster
+    ("sparse", 32, 32736, 131072),   # c4a B=32: 4 splits per sequence
+])
+def test_split_merge_paths(monkeypatch, max_cluster, kind, b, n, t):
+    """The same outputs whether the splits of a sequence are merged inside the
+    decode kernel (one thread-block cluster per sequence, or per group of
+    splits followed by decode_combine) or only by decode_combine."""
+    monkeypatch.setenv("DSV4KV_DECODE_MAX_CLUSTER", max_cluster)
+    h, window, k = 64, 128, 512
+    rows = n if kind == "sparse" else n + 3
+    q, comp, win, (kq, kc, kw) = _inputs(5000 + b + n, b, h, rows, window)
+    if kind == "dense":
+        out = K.dense_decode(q, K.Cache(0, comp), K.Cache(0, win), n, window, t, SCALE, out_fp32=True)
+    else:
+        rng = np.random.default_rng(b + n)
+        idx = np.stack([_sorted_choice(rng, n, k, k) for _ in range(b)])
+        out = K.sparse_decode(q, K.Cache(0, comp), K.Cache(0, win), torch.from_numpy(idx).cuda(), n, window, t,
+                              SCALE, out_fp32=True)
+    torch.cuda.synchronize()
+    got = to_f64(out)
+    for s in ((0,) if b == 1 else (0, b - 1)):
+        win_rows = _rows(kw, np.arange(s * window, (s + 1) * window))
+        if kind == "dense":
+            comp_rows = _rows(kc, np.arange(s * rows, s * rows + n))
+            ref = OA.dense_decode(_q_host(kq, s, h)[None], comp_rows[None], win_rows[None], t, SCALE)[0]
+        else:
+            # only the selected rows, renumbered 0..k-1 (the attention is over the set)
+            sel_rows = _rows(kc, s * rows + idx[s])
+            ref = OA.sparse_decode(_q_host(kq, s, h)[None], sel_rows[None], win_rows[None],
+                                   np.arange(k, dtype=np.int32)[None], t, SCALE)[0]
+        assert_close(got[s], ref, what=f"seq {s} (max cluster {max_cluster})")
