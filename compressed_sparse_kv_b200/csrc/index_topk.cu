@@ -6,8 +6,9 @@
 // indexer scores compressed blocks and the query reads the selected ones.
 //
 // Two launches per call (both on the caller's stream):
-//  1. index_score_*: streams the keys once (16-byte vector loads, half a warp
-//     per bf16 key / a quarter warp per fp4 key), writes one fp32 score per
+//  1. index_score_*: streams the keys once (bulk copies into shared memory,
+//     half a warp per bf16 key; 16-byte vector loads, a quarter warp per fp4
+//     key), writes one fp32 score per
 //     entry to the workspace and builds a per-sequence histogram of the top
 //     12 bits of the order-preserving score code.
 //  2. index_select: several CTAs per sequence filter the scores against the
@@ -91,61 +92,6 @@ __device__ __forceinline__ float dot8_bf16(const uint4& v, const float (&q)[8]) 
   return fmaf(q[7], bf16hi(v.w), a);
 }
 
-// bf16 keys, dim 128: a key is 256 B = 16 lanes x 16 B.  score_segment_bf16
-// scores the keys [0, cnt) of one sequence segment (kb: the segment's first
-// key, this lane's 16 bytes): a warp iteration covers 2U keys, half-warp h
-// reading keys 2U*j + U*h + u (u < U), U independent 16-byte loads per lane;
-// the next iteration's loads are issued before the current one is reduced,
-// so loads stay in flight.  Scores go to sc (global) and, when ssc is not
-// null, to shared memory; the top-12-bit histogram of the codes to sh.
-template <int U>
-__device__ __forceinline__ void score_segment_bf16(const uint16_t* __restrict__ qrow, const uint16_t* kb,
-                                                   int64_t cnt, float* sc, float* ssc, uint32_t* sh, uint64_t pol) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int half = lane >> 4, l16 = lane & 15;
-  const int my_key = U == 16 ? l16 : (U == 8 ? ((l16 >> 1) & 7) : ((l16 >> 2) & 3));
-  const bool writer = U == 16 || (U == 8 ? !(lane & 1) : !(lane & 3));
-  float q[8];
-  {
-    const uint4 v = *reinterpret_cast<const uint4*>(qrow + 8 * l16);
-    q[0] = bf16lo(v.x); q[1] = bf16hi(v.x); q[2] = bf16lo(v.y); q[3] = bf16hi(v.y);
-    q[4] = bf16lo(v.z); q[5] = bf16hi(v.z); q[6] = bf16lo(v.w); q[7] = bf16hi(v.w);
-  }
-  kb += 8 * l16;
-  auto load = [&](int64_t j, uint4 (&v)[U]) {
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t key = 2 * U * j + U * half + u;
-      v[u] = key < cnt ? ld_once_v4(kb + key * 128, pol) : make_uint4(0, 0, 0, 0);
-    }
-  };
-  auto process = [&](int64_t j, const uint4 (&v)[U]) {
-    float p[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) p[u] = dot8_bf16(v[u], q);
-    const float s = reduce16_transposed<U>(p, l16) + 0.0f;  // -0 -> +0
-    const int64_t key = 2 * U * j + U * half + my_key;
-    if (writer && key < cnt) {
-      sc[key] = s;
-      if (ssc) ssc[key] = s;
-      atomicAdd(&sh[ord_f32(s) >> 20], 1u);
-    }
-  };
-  const int64_t ngroups = (cnt + 2 * U - 1) / (2 * U);
-  uint4 va[U], vb[U];
-  int64_t j = warp;
-  if (j < ngroups) load(j, va);
-  while (j < ngroups) {
-    if (j + nwarps < ngroups) load(j + nwarps, vb);
-    process(j, va);
-    j += nwarps;
-    if (j >= ngroups) break;
-    if (j + nwarps < ngroups) load(j + nwarps, va);
-    process(j, vb);
-    j += nwarps;
-  }
-}
-
 // Adds the CTA's histogram sh to the sequence's global histogram and clears it.
 __device__ __forceinline__ void flush_histogram(uint32_t* sh, uint32_t* hb) {
   __syncthreads();
@@ -158,130 +104,200 @@ __device__ __forceinline__ void flush_histogram(uint32_t* sh, uint32_t* hb) {
   }
 }
 
-// The tail of the bf16 score kernel: the last n - n_h keys of every
-// sequence, in units of kTailUnit keys (unit u: sequence u / tups, keys
-// n_h + (u % tups) * kTailUnit ...), handed out one unit per warp claim from
-// a single counter.  A warp claims its next unit one unit ahead (the atomic's
-// round trip hides behind the current unit) and keeps the next unit's first
-// loads in flight while it reduces the current one.  Histogram counts go
-// straight to the sequence's global histogram.
-constexpr int kTailUnit = 32;  // two groups of 16 keys (8 per half-warp)
-// Share of every sequence's keys scored from the shared queue.  Measured on
-// the c4a B=32 step (per-call score time / whole step): 0 % 49.1 / 93.7 us,
-// 8 % 47.5 / 94.1, 15 % 47.1 / 92.1, 25 % 48.5 / 90.0, 35 % 49.7 / 91.1.
+// Share of every sequence's keys scored from the shared queue of the bf16
+// score kernel, and the smallest batch that uses it.
 constexpr int kTailPct = 25;
 constexpr int kTailMinBatch = 16;
 
-__device__ __forceinline__ void score_tail_bf16(const uint16_t* __restrict__ qidx, const uint16_t* __restrict__ keys,
-                                                int64_t key_rows, int64_t n, int64_t n_h, int batch,
-                                                float* __restrict__ scores, uint32_t* __restrict__ hist,
-                                                uint32_t* __restrict__ tail_ctr, uint64_t pol) {
-  constexpr int U = 8;
-  const int lane = threadIdx.x & 31, half = lane >> 4, l16 = lane & 15;
-  const int my_key = (l16 >> 1) & 7;
-  const bool writer = !(lane & 1);
-  const int64_t tups = (n - n_h + kTailUnit - 1) / kTailUnit;
-  const int64_t TU = int64_t(batch) * tups;
-  uint32_t raw = 0;
-  auto claim = [&]() {
-    if (lane == 0) raw = atomicAdd(tail_ctr, 1u);
-  };
-  auto resolve = [&]() -> int64_t {
-    const int64_t u = int64_t(__shfl_sync(kFull, raw, 0));
-    return u < TU ? u : -1;
-  };
-  float q[8];
-  uint4 qn = make_uint4(0, 0, 0, 0);
-  int bq = -1;
-  auto load_group = [&](int b, int64_t i0, int g, uint4 (&v)[U]) {
-    const uint16_t* kb = keys + (size_t(b) * size_t(key_rows) + size_t(i0)) * 128 + 8 * l16;
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t key = 16 * g + U * half + u;
-      v[u] = i0 + key < n ? ld_once_v4(kb + key * 128, pol) : make_uint4(0, 0, 0, 0);
+// index_score_stream: the bf16 score kernel with the keys streamed into
+// shared memory by bulk copies.  One CTA per SM: a producer thread (warp 8)
+// feeds a ring of kStreamStages stages of up to 128 keys (32 KB) plus the
+// sequence's query (256 B), each completing on its own mbarrier; 8 consumer
+// warps score every stage (a warp 16 keys, half a warp per key as in
+// score_segment_bf16) and free it as soon as its keys are in registers.  The
+// producer walks the CTA's even share of the first n_h keys of every
+// sequence (flattened over the batch; stages never straddle two sequences),
+// then claims 128-key units of the sequences' tails from the shared counter
+// (batches of kTailMinBatch or more), so the CTAs that stream faster take
+// more of the tail.  Histogram counts of the even share go to one of two
+// shared-memory histograms (the CTA's first two sequences; an even share
+// spans at most two when it is shorter than n_h) and are flushed once at
+// the end; tail counts and those of further sequences go straight to global
+// memory.  Every wait is bounded; a wait that gives up flags
+// DSV4KV_DEV_TIMEOUT and ends the CTA's loop.
+constexpr int kStreamKeys = 128;
+constexpr int kStreamStages = 5;
+constexpr int kStreamConsumers = 8;  // warps
+constexpr int kStreamThreads = 32 * (kStreamConsumers + 1);
+constexpr uint32_t kStreamKeyBytes = kStreamKeys * 256;
+constexpr uint32_t kStreamStageBytes = kStreamKeyBytes + 256;  // keys, then the query
+struct StreamMeta {
+  int32_t b, cnt;  // cnt < 0: no more stages
+  int64_t i0;
+  int32_t tail, pad;
+};
+struct StreamCtl {
+  uint64_t full[kStreamStages];
+  uint64_t empty[kStreamStages];
+  StreamMeta meta[kStreamStages];
+  int abort;
+};
+constexpr size_t kStreamSmem =
+    size_t(kStreamStages) * kStreamStageBytes + 2 * kHistBins * sizeof(uint32_t) + sizeof(StreamCtl) + 128;
+static_assert(kStreamSmem <= 232448, "shared memory per CTA");
+constexpr uint64_t kStreamWaitNs = 1000000000ull;
+
+__device__ __forceinline__ uint64_t stream_now() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait on one phase of an mbarrier (every calling thread polls).
+__device__ __forceinline__ bool stream_wait(uint64_t* bar, uint32_t parity, StreamCtl* ctl) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = stream_now();
+  while (!mbar_try_wait(bar, parity)) {
+    if (ctl->abort || stream_now() - t0 > kStreamWaitNs) {
+      ctl->abort = 1;
+      return false;
     }
-  };
-  auto process = [&](int b, int64_t i0, int g, const uint4 (&v)[U]) {
-    float p[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) p[u] = dot8_bf16(v[u], q);
-    const float sc = reduce16_transposed<U>(p, l16) + 0.0f;  // -0 -> +0
-    const int64_t key = i0 + 16 * g + U * half + my_key;
-    if (writer && key < n) {
-      scores[size_t(b) * size_t(score_stride(n)) + size_t(key)] = sc;
-      atomicAdd(&hist[size_t(b) * kHistBins + hist_pos(int(ord_f32(sc) >> 20))], 1u);
-    }
-  };
-  claim();
-  int64_t cur = resolve();
-  if (cur < 0) return;
-  uint4 va[U], vb[U];
-  int b = int(cur / tups);
-  int64_t i0 = n_h + (cur % tups) * kTailUnit;
-  qn = *reinterpret_cast<const uint4*>(qidx + size_t(b) * 128 + 8 * l16);
-  load_group(b, i0, 0, va);
-  claim();
-  while (true) {
-    load_group(b, i0, 1, vb);
-    if (b != bq) {
-      q[0] = bf16lo(qn.x); q[1] = bf16hi(qn.x); q[2] = bf16lo(qn.y); q[3] = bf16hi(qn.y);
-      q[4] = bf16lo(qn.z); q[5] = bf16hi(qn.z); q[6] = bf16lo(qn.w); q[7] = bf16hi(qn.w);
-      bq = b;
-    }
-    process(b, i0, 0, va);
-    const int64_t nxt = resolve();
-    int nb = b;
-    int64_t ni0 = 0;
-    if (nxt >= 0) {
-      nb = int(nxt / tups);
-      ni0 = n_h + (nxt % tups) * kTailUnit;
-      if (nb != b) qn = *reinterpret_cast<const uint4*>(qidx + size_t(nb) * 128 + 8 * l16);
-      load_group(nb, ni0, 0, va);
-      claim();
-    }
-    process(b, i0, 1, vb);
-    if (nxt < 0) break;
-    b = nb;
-    i0 = ni0;
   }
+  return true;
 }
 
-// index_score_bf16: the first n_h keys of every sequence (flattened over the
-// batch) split evenly over one wave of CTAs, a CTA walking its range one
-// sequence segment at a time with a shared-memory histogram; then every warp
-// turns to the shared queue of the remaining keys (score_tail_bf16), so the
-// CTAs that stream faster take more of the tail and the wave ends together.
-template <int U>
-__global__ void __launch_bounds__(256) index_score_bf16(const uint16_t* __restrict__ qidx,
-                                                        const uint16_t* __restrict__ keys, int64_t key_rows,
-                                                        int64_t n, int64_t n_h, int batch, int64_t per_cta,
-                                                        float* __restrict__ scores, uint32_t* __restrict__ hist,
-                                                        uint32_t* __restrict__ tail_ctr) {
-  __shared__ uint32_t sh[kHistBins];
+__global__ void __launch_bounds__(kStreamThreads, 1)
+    index_score_stream(const uint16_t* __restrict__ qidx, const uint16_t* __restrict__ keys, int64_t key_rows,
+                       int64_t n, int64_t n_h, int batch, int64_t per_cta, float* __restrict__ scores,
+                       uint32_t* __restrict__ hist, uint32_t* __restrict__ tail_ctr, uint32_t* __restrict__ status) {
+  extern __shared__ __align__(128) uint8_t sraw[];
+  uint8_t* stage = sraw;
+  uint32_t* sh = reinterpret_cast<uint32_t*>(sraw + size_t(kStreamStages) * kStreamStageBytes);  // [2][kHistBins]
+  StreamCtl* ctl = reinterpret_cast<StreamCtl*>(sh + 2 * kHistBins);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
-  const int64_t total = int64_t(batch) * n_h;
-  const int64_t g0 = min(total, int64_t(blockIdx.x) * per_cta);
-  const int64_t g1 = min(total, g0 + per_cta);
-  pdl_wait();
-  const uint64_t pol = l2_evict_first_policy();  // keys are read once
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0;
-  __syncthreads();
-  int b_last = -1;
-  for (int64_t s0 = g0; s0 < g1;) {
-    const int b = int(s0 / n_h);
-    const int64_t s1 = min(g1, int64_t(b + 1) * n_h);
-    const int64_t i0 = s0 - int64_t(b) * n_h;
-    if (b_last >= 0) {
-      flush_histogram(sh, hist + size_t(b_last) * kHistBins);
-      __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStreamStages; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], kStreamConsumers);
     }
-    score_segment_bf16<U>(qidx + size_t(b) * 128, keys + (size_t(b) * size_t(key_rows) + size_t(i0)) * 128, s1 - s0,
-                          scores + size_t(b) * size_t(score_stride(n)) + size_t(i0), nullptr, sh, pol);
-    b_last = b;
-    s0 = s1;
+    ctl->abort = 0;
+    fence_mbar_init();
   }
-  if (n_h < n) score_tail_bf16(qidx, keys, key_rows, n, n_h, batch, scores, hist, tail_ctr, pol);
-  if (b_last >= 0) flush_histogram(sh, hist + size_t(b_last) * kHistBins);
+  for (int i = threadIdx.x; i < 2 * kHistBins; i += kStreamThreads) sh[i] = 0;
+  __syncthreads();
+  pdl_wait();
+  const int64_t total = int64_t(batch) * n_h;
+  const int64_t g0 = min(total, int64_t(blockIdx.x) * per_cta), g1 = min(total, g0 + per_cta);
+  const int64_t tups = (n - n_h + kStreamKeys - 1) / kStreamKeys;  // tail units per sequence
+  const int64_t TU = n_h < n ? int64_t(batch) * tups : 0;
+  volatile int* abort = &ctl->abort;
+
+  if (warp == kStreamConsumers) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      const uint64_t pol = l2_evict_first_policy();  // keys are read once
+      int64_t pos = g0;
+      uint32_t claimed = TU > 0 ? atomicAdd(tail_ctr, 1u) : 0u;  // one claim ahead
+      int it = 0;
+      bool ok = true;
+      for (;; ++it) {
+        int b, cnt, tail;
+        int64_t i0;
+        if (pos < g1) {
+          b = int(pos / n_h);
+          i0 = pos - int64_t(b) * n_h;
+          const int64_t end = min(g1, int64_t(b + 1) * n_h);
+          cnt = int(min(int64_t(kStreamKeys), end - pos));
+          pos += cnt;
+          tail = 0;
+        } else if (int64_t(claimed) < TU) {
+          b = int(int64_t(claimed) / tups);
+          i0 = n_h + (int64_t(claimed) % tups) * kStreamKeys;
+          cnt = int(min(int64_t(kStreamKeys), n - i0));
+          tail = 1;
+          claimed = atomicAdd(tail_ctr, 1u);
+        } else {
+          break;
+        }
+        const int s = it % kStreamStages;
+        if (it >= kStreamStages && !stream_wait(&ctl->empty[s], ((it / kStreamStages) - 1) & 1, ctl)) {
+          ok = false;
+          break;
+        }
+        ctl->meta[s] = StreamMeta{b, cnt, i0, tail, 0};
+        uint8_t* dst = stage + size_t(s) * kStreamStageBytes;
+        mbar_arrive_expect_tx(&ctl->full[s], uint32_t(cnt) * 256u + 256u);
+        bulk_load(dst, keys + (size_t(b) * size_t(key_rows) + size_t(i0)) * 128, uint32_t(cnt) * 256u, &ctl->full[s],
+                  pol);
+        bulk_load_plain(dst + kStreamKeyBytes, qidx + size_t(b) * 128, 256u, &ctl->full[s]);
+      }
+      bool marked = false;
+      if (ok) {  // the end marker
+        const int s = it % kStreamStages;
+        if (it < kStreamStages || stream_wait(&ctl->empty[s], ((it / kStreamStages) - 1) & 1, ctl)) {
+          ctl->meta[s] = StreamMeta{0, -1, 0, 0, 0};
+          mbar_arrive(&ctl->full[s]);
+          marked = true;
+        }
+      }
+      // Normally the consumers wait for every copy before they finish.  After
+      // a wait that gave up, never leave with copies in flight: wait (bounded)
+      // for the last phase of each stage still armed (none was re-armed by a
+      // marker on this path).
+      if (!marked) {
+        const uint64_t t0 = stream_now();
+        for (int j = max(0, it - kStreamStages); j < it; ++j)
+          while (!mbar_try_wait(&ctl->full[j % kStreamStages], (j / kStreamStages) & 1))
+            if (stream_now() - t0 > kStreamWaitNs) break;
+      }
+      if (*abort) set_status(status, DSV4KV_DEV_TIMEOUT);
+    }
+    return;
+  }
+  // ------------------------------------------------------------------ consumers (warps 0-7)
+  const int half = lane >> 4, l16 = lane & 15;
+  const int my_key = (l16 >> 1) & 7;  // reduce16_transposed<8>: lanes 2i, 2i+1 end with key i
+  const bool writer = !(lane & 1);
+  const int b0 = n_h > 0 ? int(g0 / n_h) : 0;  // the even share's first sequence: shared histogram 0
+  for (int it = 0;; ++it) {
+    const int s = it % kStreamStages;
+    bool ok = true;
+    if (lane == 0) ok = stream_wait(&ctl->full[s], (it / kStreamStages) & 1, ctl);
+    if (!__shfl_sync(kFull, ok, 0)) break;
+    const StreamMeta m = ctl->meta[s];
+    if (m.cnt < 0) break;
+    const uint8_t* st = stage + size_t(s) * kStreamStageBytes;
+    float q[8];
+    {
+      const uint4 v = *reinterpret_cast<const uint4*>(st + kStreamKeyBytes + 16 * l16);
+      q[0] = bf16lo(v.x); q[1] = bf16hi(v.x); q[2] = bf16lo(v.y); q[3] = bf16hi(v.y);
+      q[4] = bf16lo(v.z); q[5] = bf16hi(v.z); q[6] = bf16lo(v.w); q[7] = bf16hi(v.w);
+    }
+    const int k0 = 16 * warp + 8 * half;  // this half-warp's first key of the stage
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = *reinterpret_cast<const uint4*>(st + (k0 + u) * 256 + 16 * l16);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ctl->empty[s]);  // the warp's keys are in registers
+    float p[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) p[u] = dot8_bf16(v[u], q);  // (keys past cnt: stale data, never written)
+    const float sc = reduce16_transposed<8>(p, l16) + 0.0f;  // -0 -> +0
+    const int key = k0 + my_key;
+    if (writer && key < m.cnt) {
+      scores[size_t(m.b) * size_t(score_stride(n)) + size_t(m.i0 + key)] = sc;
+      const int bin = int(ord_f32(sc) >> 20), slot = m.b - b0;
+      if (!m.tail && slot >= 0 && slot < 2) atomicAdd(&sh[slot * kHistBins + bin], 1u);
+      else atomicAdd(&hist[size_t(m.b) * kHistBins + hist_pos(bin)], 1u);
+    }
+  }
+  // flush the two shared histograms (every consumer warp ends its loop: the waits are bounded)
+  asm volatile("barrier.cta.sync 1, %0;" ::"n"(32 * kStreamConsumers) : "memory");
+  for (int i = threadIdx.x; i < 2 * kHistBins; i += 32 * kStreamConsumers) {
+    const uint32_t c = sh[i];
+    const int bb = b0 + i / kHistBins;
+    if (c && bb < batch) atomicAdd(&hist[size_t(bb) * kHistBins + hist_pos(i % kHistBins)], c);
+  }
 }
 
 // The four code bytes of w (byte 0 = lowest) decoded to four f16x2 pairs by
@@ -1662,29 +1678,28 @@ dsv4kv_status index_score_launch(const uint16_t* qidx, const dsv4kv_cache& keys,
   if (ws_bytes < w.bytes) return set_error(DSV4KV_ERR_WORKSPACE, "index_score: workspace too small");
   const int sms = sm_count();
   if (keys.fmt == DSV4KV_BF16) {
-    // one wave (resident CTAs per SM x SMs) over the flattened (sequence, entry) range
-    static std::atomic<int> occ_dev[64];  // per device; 0 = not queried yet
-    std::atomic<int>& occ_slot = occ_dev[current_device()];
-    int occ = occ_slot.load(std::memory_order_relaxed);
-    if (occ == 0) {
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, index_score_bf16<8>, 256, 0) != cudaSuccess || occ < 1)
-        occ = 1;
-      occ_slot.store(occ, std::memory_order_relaxed);
+    // one CTA per SM streaming through shared memory; the last kTailPct % of
+    // every sequence (whole 128-key units) goes to the shared queue, whose
+    // histogram counts go straight to global memory: with few sequences they
+    // would pile onto the few bins that hold most scores of one histogram,
+    // so small batches use the even split alone
+    static std::atomic<uint64_t> attr_set{0};
+    if (!done_on_device(attr_set)) {
+      if (cudaFuncSetAttribute(index_score_stream, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kStreamSmem)) !=
+          cudaSuccess)
+        return check_launch("index_score: cudaFuncSetAttribute");
+      mark_done_on_device(attr_set);
     }
-    // the last kTailPct % of every sequence (whole units) goes to the shared
-    // queue.  Its histogram counts go straight to global memory, one atomic
-    // per key, so with few sequences they would pile onto the few bins that
-    // hold most scores of one histogram: small batches use the even split alone.
+    if ((reinterpret_cast<uintptr_t>(qidx) | reinterpret_cast<uintptr_t>(keys.codes)) & 15)
+      return set_error(DSV4KV_ERR_INVALID_ARG, "index_score: query and key rows must be 16-byte aligned");
     const int64_t n_tail =
-        batch >= kTailMinBatch ? std::min<int64_t>(n, (n * kTailPct / 100) / kTailUnit * kTailUnit) : 0;
+        batch >= kTailMinBatch ? std::min<int64_t>(n, (n * kTailPct / 100) / kStreamKeys * kStreamKeys) : 0;
     const int64_t n_h = n - n_tail;
     const int64_t total = int64_t(batch) * n_h;
-    const int64_t grid = int64_t(sms) * occ;
-    const int64_t per_cta = std::max<int64_t>(64, (total + grid - 1) / grid);
-    const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>(grid, (total + per_cta - 1) / per_cta));
-    launch_pdl(index_score_bf16<8>, dim3(unsigned(n_h > 0 ? ctas : grid)), dim3(256), 0, stream, qidx,
+    const int64_t per_cta = std::max<int64_t>(kStreamKeys, (total + sms - 1) / sms);
+    launch_pdl(index_score_stream, dim3(unsigned(sms)), dim3(kStreamThreads), kStreamSmem, stream, qidx,
                static_cast<const uint16_t*>(keys.codes), keys.rows, n, n_h, batch, per_cta, w.scores, w.hist,
-               w.tail_ctr);
+               w.tail_ctr, w.status);
   } else {
     static std::atomic<int> occ4_dev[64];  // per device; 0 = not queried yet
     std::atomic<int>& occ4_slot = occ4_dev[current_device()];
