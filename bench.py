@@ -56,7 +56,7 @@ L2_BYTES = 126 * 2 ** 20
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
 # capture of that kernel in this workload (profiles/ holds the summary and the
 # command); cleared whenever the kernel changes
-TRAFFIC = {("c4a_b32", "index_score_stream"): 274427392}
+TRAFFIC = {("c4a_b32", "index_score_stream<bf16>"): 274427392}
 
 
 def measured_peaks():
@@ -971,7 +971,7 @@ def main():
     if kind == "c4a":
         dom_bytes, dom_ms = layer.index_bytes(), res["score_ms"]
         dom_name = ("index_pool_select" if pool else "index_score_paged + index_select" if paged
-                    else "index_score_stream" if ifmt == 0 else "index_score_fp4")
+                    else "index_score_stream<bf16>" if ifmt == 0 else "index_score_stream<fp4>")
     else:
         dom_bytes, dom_ms, dom_name = alg, res["decode_ms"], "dsv4kv_dense_decode (decode_kernel + decode_combine)"
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9

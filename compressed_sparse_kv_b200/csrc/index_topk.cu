@@ -109,197 +109,6 @@ __device__ __forceinline__ void flush_histogram(uint32_t* sh, uint32_t* hb) {
 constexpr int kTailPct = 25;
 constexpr int kTailMinBatch = 16;
 
-// index_score_stream: the bf16 score kernel with the keys streamed into
-// shared memory by bulk copies.  One CTA per SM: a producer thread (warp 8)
-// feeds a ring of kStreamStages stages of up to 128 keys (32 KB) plus the
-// sequence's query (256 B), each completing on its own mbarrier; 8 consumer
-// warps score every stage (a warp 16 keys, half a warp per key as in
-// score_segment_bf16) and free it as soon as its keys are in registers.  The
-// producer walks the CTA's even share of the first n_h keys of every
-// sequence (flattened over the batch; stages never straddle two sequences),
-// then claims 128-key units of the sequences' tails from the shared counter
-// (batches of kTailMinBatch or more), so the CTAs that stream faster take
-// more of the tail.  Histogram counts of the even share go to one of two
-// shared-memory histograms (the CTA's first two sequences; an even share
-// spans at most two when it is shorter than n_h) and are flushed once at
-// the end; tail counts and those of further sequences go straight to global
-// memory.  Every wait is bounded; a wait that gives up flags
-// DSV4KV_DEV_TIMEOUT and ends the CTA's loop.
-constexpr int kStreamKeys = 128;
-constexpr int kStreamStages = 5;
-constexpr int kStreamConsumers = 8;  // warps
-constexpr int kStreamThreads = 32 * (kStreamConsumers + 1);
-constexpr uint32_t kStreamKeyBytes = kStreamKeys * 256;
-constexpr uint32_t kStreamStageBytes = kStreamKeyBytes + 256;  // keys, then the query
-struct StreamMeta {
-  int32_t b, cnt;  // cnt < 0: no more stages
-  int64_t i0;
-  int32_t tail, pad;
-};
-struct StreamCtl {
-  uint64_t full[kStreamStages];
-  uint64_t empty[kStreamStages];
-  StreamMeta meta[kStreamStages];
-  int abort;
-};
-constexpr size_t kStreamSmem =
-    size_t(kStreamStages) * kStreamStageBytes + 2 * kHistBins * sizeof(uint32_t) + sizeof(StreamCtl) + 128;
-static_assert(kStreamSmem <= 232448, "shared memory per CTA");
-constexpr uint64_t kStreamWaitNs = 1000000000ull;
-
-__device__ __forceinline__ uint64_t stream_now() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
-// Bounded wait on one phase of an mbarrier (every calling thread polls).
-__device__ __forceinline__ bool stream_wait(uint64_t* bar, uint32_t parity, StreamCtl* ctl) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = stream_now();
-  while (!mbar_try_wait(bar, parity)) {
-    if (ctl->abort || stream_now() - t0 > kStreamWaitNs) {
-      ctl->abort = 1;
-      return false;
-    }
-  }
-  return true;
-}
-
-__global__ void __launch_bounds__(kStreamThreads, 1)
-    index_score_stream(const uint16_t* __restrict__ qidx, const uint16_t* __restrict__ keys, int64_t key_rows,
-                       int64_t n, int64_t n_h, int batch, int64_t per_cta, float* __restrict__ scores,
-                       uint32_t* __restrict__ hist, uint32_t* __restrict__ tail_ctr, uint32_t* __restrict__ status) {
-  extern __shared__ __align__(128) uint8_t sraw[];
-  uint8_t* stage = sraw;
-  uint32_t* sh = reinterpret_cast<uint32_t*>(sraw + size_t(kStreamStages) * kStreamStageBytes);  // [2][kHistBins]
-  StreamCtl* ctl = reinterpret_cast<StreamCtl*>(sh + 2 * kHistBins);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_trigger();
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStreamStages; ++s) {
-      mbar_init(&ctl->full[s], 1);
-      mbar_init(&ctl->empty[s], kStreamConsumers);
-    }
-    ctl->abort = 0;
-    fence_mbar_init();
-  }
-  for (int i = threadIdx.x; i < 2 * kHistBins; i += kStreamThreads) sh[i] = 0;
-  __syncthreads();
-  pdl_wait();
-  const int64_t total = int64_t(batch) * n_h;
-  const int64_t g0 = min(total, int64_t(blockIdx.x) * per_cta), g1 = min(total, g0 + per_cta);
-  const int64_t tups = (n - n_h + kStreamKeys - 1) / kStreamKeys;  // tail units per sequence
-  const int64_t TU = n_h < n ? int64_t(batch) * tups : 0;
-  volatile int* abort = &ctl->abort;
-
-  if (warp == kStreamConsumers) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      const uint64_t pol = l2_evict_first_policy();  // keys are read once
-      int64_t pos = g0;
-      uint32_t claimed = TU > 0 ? atomicAdd(tail_ctr, 1u) : 0u;  // one claim ahead
-      int it = 0;
-      bool ok = true;
-      for (;; ++it) {
-        int b, cnt, tail;
-        int64_t i0;
-        if (pos < g1) {
-          b = int(pos / n_h);
-          i0 = pos - int64_t(b) * n_h;
-          const int64_t end = min(g1, int64_t(b + 1) * n_h);
-          cnt = int(min(int64_t(kStreamKeys), end - pos));
-          pos += cnt;
-          tail = 0;
-        } else if (int64_t(claimed) < TU) {
-          b = int(int64_t(claimed) / tups);
-          i0 = n_h + (int64_t(claimed) % tups) * kStreamKeys;
-          cnt = int(min(int64_t(kStreamKeys), n - i0));
-          tail = 1;
-          claimed = atomicAdd(tail_ctr, 1u);
-        } else {
-          break;
-        }
-        const int s = it % kStreamStages;
-        if (it >= kStreamStages && !stream_wait(&ctl->empty[s], ((it / kStreamStages) - 1) & 1, ctl)) {
-          ok = false;
-          break;
-        }
-        ctl->meta[s] = StreamMeta{b, cnt, i0, tail, 0};
-        uint8_t* dst = stage + size_t(s) * kStreamStageBytes;
-        mbar_arrive_expect_tx(&ctl->full[s], uint32_t(cnt) * 256u + 256u);
-        bulk_load(dst, keys + (size_t(b) * size_t(key_rows) + size_t(i0)) * 128, uint32_t(cnt) * 256u, &ctl->full[s],
-                  pol);
-        bulk_load_plain(dst + kStreamKeyBytes, qidx + size_t(b) * 128, 256u, &ctl->full[s]);
-      }
-      bool marked = false;
-      if (ok) {  // the end marker
-        const int s = it % kStreamStages;
-        if (it < kStreamStages || stream_wait(&ctl->empty[s], ((it / kStreamStages) - 1) & 1, ctl)) {
-          ctl->meta[s] = StreamMeta{0, -1, 0, 0, 0};
-          mbar_arrive(&ctl->full[s]);
-          marked = true;
-        }
-      }
-      // Normally the consumers wait for every copy before they finish.  After
-      // a wait that gave up, never leave with copies in flight: wait (bounded)
-      // for the last phase of each stage still armed (none was re-armed by a
-      // marker on this path).
-      if (!marked) {
-        const uint64_t t0 = stream_now();
-        for (int j = max(0, it - kStreamStages); j < it; ++j)
-          while (!mbar_try_wait(&ctl->full[j % kStreamStages], (j / kStreamStages) & 1))
-            if (stream_now() - t0 > kStreamWaitNs) break;
-      }
-      if (*abort) set_status(status, DSV4KV_DEV_TIMEOUT);
-    }
-    return;
-  }
-  // ------------------------------------------------------------------ consumers (warps 0-7)
-  const int half = lane >> 4, l16 = lane & 15;
-  const int my_key = (l16 >> 1) & 7;  // reduce16_transposed<8>: lanes 2i, 2i+1 end with key i
-  const bool writer = !(lane & 1);
-  const int b0 = n_h > 0 ? int(g0 / n_h) : 0;  // the even share's first sequence: shared histogram 0
-  for (int it = 0;; ++it) {
-    const int s = it % kStreamStages;
-    bool ok = true;
-    if (lane == 0) ok = stream_wait(&ctl->full[s], (it / kStreamStages) & 1, ctl);
-    if (!__shfl_sync(kFull, ok, 0)) break;
-    const StreamMeta m = ctl->meta[s];
-    if (m.cnt < 0) break;
-    const uint8_t* st = stage + size_t(s) * kStreamStageBytes;
-    float q[8];
-    {
-      const uint4 v = *reinterpret_cast<const uint4*>(st + kStreamKeyBytes + 16 * l16);
-      q[0] = bf16lo(v.x); q[1] = bf16hi(v.x); q[2] = bf16lo(v.y); q[3] = bf16hi(v.y);
-      q[4] = bf16lo(v.z); q[5] = bf16hi(v.z); q[6] = bf16lo(v.w); q[7] = bf16hi(v.w);
-    }
-    const int k0 = 16 * warp + 8 * half;  // this half-warp's first key of the stage
-    uint4 v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = *reinterpret_cast<const uint4*>(st + (k0 + u) * 256 + 16 * l16);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&ctl->empty[s]);  // the warp's keys are in registers
-    float p[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) p[u] = dot8_bf16(v[u], q);  // (keys past cnt: stale data, never written)
-    const float sc = reduce16_transposed<8>(p, l16) + 0.0f;  // -0 -> +0
-    const int key = k0 + my_key;
-    if (writer && key < m.cnt) {
-      scores[size_t(m.b) * size_t(score_stride(n)) + size_t(m.i0 + key)] = sc;
-      const int bin = int(ord_f32(sc) >> 20), slot = m.b - b0;
-      if (!m.tail && slot >= 0 && slot < 2) atomicAdd(&sh[slot * kHistBins + bin], 1u);
-      else atomicAdd(&hist[size_t(m.b) * kHistBins + hist_pos(bin)], 1u);
-    }
-  }
-  // flush the two shared histograms (every consumer warp ends its loop: the waits are bounded)
-  asm volatile("barrier.cta.sync 1, %0;" ::"n"(32 * kStreamConsumers) : "memory");
-  for (int i = threadIdx.x; i < 2 * kHistBins; i += 32 * kStreamConsumers) {
-    const uint32_t c = sh[i];
-    const int bb = b0 + i / kHistBins;
-    if (c && bb < batch) atomicAdd(&hist[size_t(bb) * kHistBins + hist_pos(i % kHistBins)], c);
-  }
-}
-
 // The four code bytes of w (byte 0 = lowest) decoded to four f16x2 pairs by
 // cvt.rn.f16x2.e2m1x2 straight from the unpacked bytes (no shifts or masks);
 // each pair holds (low nibble, high nibble) = (even, odd) channel.
@@ -344,39 +153,159 @@ __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
 
 // fp4 keys, dim 128: 64 B of codes + 8 E4M3 scale bytes per key.  A quarter
 // warp (4 lanes x 16 B) covers one key; lane l4 holds channels
-// [32*l4, 32*l4+32) = two 16-channel scale groups.  Same segment structure as
-// the bf16 path; each warp iteration covers 32 keys (U = 4 per quad).  Each
-// code byte is decoded to a packed f16 pair with cvt.rn.f16x2.e2m1x2 and
-// accumulated with packed f16 FMAs per group (exact for integer queries:
-// |partial| <= 8*8*6 per half at a resolution of 0.5), then scaled by the
-// group's E4M3 scale in fp32.
-__device__ __forceinline__ void score_segment_fp4(const uint16_t* __restrict__ qrow, const uint8_t* cb,
-                                                  const uint8_t* sb, int64_t cnt, float* sc, float* ssc,
-                                                  uint32_t* sh, uint64_t pol) {
-  constexpr int U = 4;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int quad = lane >> 2, l4 = lane & 3;
-  uint32_t qp[16];  // (q[2j], q[2j+1]) as f16x2 for this lane's 32 channels
-  {
-    const uint16_t* qb = qrow + 32 * l4;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) qp[j] = f32x2_to_f16x2(bf16f(qb[2 * j]), bf16f(qb[2 * j + 1]));
-  }
-  cb += 16 * l4;
-  sb += 2 * l4;
-  auto load = [&](int64_t j, uint4 (&v)[U], uint32_t (&s2)[U]) {
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t key = 8 * U * j + 8 * u + quad;
-      const bool ok = key < cnt;
-      v[u] = ok ? ld_once_v4(cb + key * 64, pol) : make_uint4(0, 0, 0, 0);
-      s2[u] = ok ? ld_once_u16(sb + key * 8, pol) : 0u;
+// [32*l4, 32*l4+32) = two 16-channel scale groups; a warp takes 32 keys (4
+// per quad).  Each code byte is decoded to a packed f16 pair with
+// cvt.rn.f16x2.e2m1x2 and accumulated with packed f16 FMAs per group (exact
+// for integer queries: |partial| <= 8*8*6 per half at a resolution of 0.5),
+// then scaled by the group's E4M3 scale in fp32 (StreamConsumer<StreamFp4>).
+
+// index_score_stream<F>: the score kernel with the keys streamed into shared
+// memory by bulk copies.  One CTA per SM: a producer thread (the last warp)
+// feeds a ring of F::kStages stages of up to F::kKeys keys (codes, the fp4
+// keys' group scales, and the sequence's query), each completing on its own
+// mbarrier; F::kConsumers consumer warps score every stage and free it as
+// soon as its keys are in their registers.  The producer walks the CTA's
+// even share of the first n_h keys of every sequence (flattened over the
+// batch; stages never straddle two sequences), then claims F::kKeys-key
+// units of the sequences' tails from the shared counter (batches of
+// kTailMinBatch or more), so the CTAs that stream faster take more of the
+// tail.  Histogram counts of the even share go to one of two shared-memory
+// histograms (the CTA's first two sequences; an even share spans at most two
+// when it is shorter than n_h) flushed once at the end; tail counts and
+// those of further sequences go straight to global memory.  Every wait is
+// bounded; a wait that gives up flags DSV4KV_DEV_TIMEOUT and ends the loop.
+//
+// bf16 keys: 128 keys (32 KB) per stage, 8 consumer warps, a warp 16 keys,
+// half a warp per key (as the bf16 scoring elsewhere in this file).  fp4
+// keys: 512 keys (32 KB of codes + 4 KB of scales) per stage, 16 consumer
+// warps, a warp 32 keys, a quarter warp per key (see the fp4 note above).
+struct StreamBf16 {
+  static constexpr int kKeys = 128, kConsumers = 8, kStages = 5;
+  static constexpr uint32_t kCodeBytes = 256, kScaleBytes = 0;  // per key
+};
+struct StreamFp4 {
+  static constexpr int kKeys = 512, kConsumers = 16, kStages = 5;
+  static constexpr uint32_t kCodeBytes = 64, kScaleBytes = 8;
+};
+template <class F>
+struct StreamLayout {
+  static constexpr uint32_t kCodes = F::kKeys * F::kCodeBytes;
+  // the scale rows are copied from an even row on (a bulk copy moves whole
+  // 16-byte units), so a stage holds up to two more of them
+  static constexpr uint32_t kScales = F::kScaleBytes ? (F::kKeys + 2) * F::kScaleBytes : 0;
+  static constexpr uint32_t kStage = kCodes + kScales + 256;  // codes, scales, the query
+  static constexpr int kThreads = 32 * (F::kConsumers + 1);
+};
+struct StreamMeta {
+  int32_t b, cnt;  // cnt < 0: no more stages
+  int64_t i0;
+  int32_t tail;
+  int32_t soff;  // key 0's row among the stage's scale rows (0 or 1)
+};
+template <class F>
+struct StreamCtl {
+  uint64_t full[F::kStages];
+  uint64_t empty[F::kStages];
+  StreamMeta meta[F::kStages];
+  int abort;
+};
+template <class F>
+constexpr size_t stream_smem() {
+  return size_t(F::kStages) * StreamLayout<F>::kStage + 2 * kHistBins * sizeof(uint32_t) + sizeof(StreamCtl<F>) + 128;
+}
+static_assert(stream_smem<StreamBf16>() <= 232448 && stream_smem<StreamFp4>() <= 232448, "shared memory per CTA");
+constexpr uint64_t kStreamWaitNs = 1000000000ull;
+
+__device__ __forceinline__ uint64_t stream_now() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait on one phase of an mbarrier (the calling thread polls).
+template <class F>
+__device__ __forceinline__ bool stream_wait(uint64_t* bar, uint32_t parity, StreamCtl<F>* ctl) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = stream_now();
+  while (!mbar_try_wait(bar, parity)) {
+    if (ctl->abort || stream_now() - t0 > kStreamWaitNs) {
+      ctl->abort = 1;
+      return false;
     }
-  };
-  auto process = [&](int64_t j, const uint4 (&v)[U], const uint32_t (&s2)[U]) {
-    float p[U];
+  }
+  return true;
+}
+
+// Where a consumer finds what a stage does not hold: the scale row of the
+// last key row when the rows total is odd (bulk copies move whole 16-byte
+// units, two scale rows).
+struct StreamEdge {
+  const uint8_t* scales;
+  int64_t key_rows, last_odd_row;  // last_odd_row < 0: none
+};
+
+// A consumer warp's part of one stage: load() brings the warp's keys and the
+// query into registers (after it the stage may be refilled); score() leaves
+// on each lane the score of key `key` of the stage, to be stored by the
+// lanes with `writer` set.
+template <class F>
+struct StreamConsumer;
+
+template <>
+struct StreamConsumer<StreamBf16> {
+  uint4 v[8];
+  float q[8];
+  __device__ __forceinline__ void load(const uint8_t* st, const StreamMeta&, const StreamEdge&, int warp, int lane) {
+    const int half = lane >> 4, l16 = lane & 15;
+    const uint4 x = *reinterpret_cast<const uint4*>(st + StreamLayout<StreamBf16>::kCodes + 16 * l16);
+    q[0] = bf16lo(x.x); q[1] = bf16hi(x.x); q[2] = bf16lo(x.y); q[3] = bf16hi(x.y);
+    q[4] = bf16lo(x.z); q[5] = bf16hi(x.z); q[6] = bf16lo(x.w); q[7] = bf16hi(x.w);
+    const int k0 = 16 * warp + 8 * half;  // this half-warp's first key of the stage
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
+    for (int u = 0; u < 8; ++u) v[u] = *reinterpret_cast<const uint4*>(st + (k0 + u) * 256 + 16 * l16);
+  }
+  __device__ __forceinline__ float score(int warp, int lane, int* key, bool* writer) const {
+    const int half = lane >> 4, l16 = lane & 15;
+    float p[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) p[u] = dot8_bf16(v[u], q);  // (keys past cnt: stale data, never stored)
+    *key = 16 * warp + 8 * half + ((l16 >> 1) & 7);  // reduce16_transposed<8>: lanes 2i, 2i+1 hold key i
+    *writer = !(lane & 1);
+    return reduce16_transposed<8>(p, l16) + 0.0f;  // -0 -> +0
+  }
+};
+
+template <>
+struct StreamConsumer<StreamFp4> {
+  uint4 v[4];
+  uint32_t s2[4];
+  uint32_t qp[16];  // (q[2j], q[2j+1]) as f16x2 for this lane's 32 channels
+  __device__ __forceinline__ void load(const uint8_t* st, const StreamMeta& m, const StreamEdge& e, int warp,
+                                       int lane) {
+    using Lay = StreamLayout<StreamFp4>;
+    const int quad = lane >> 2, l4 = lane & 3;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 x = *reinterpret_cast<const uint4*>(st + Lay::kCodes + Lay::kScales + 64 * l4 + 16 * i);
+      qp[4 * i] = f32x2_to_f16x2(bf16lo(x.x), bf16hi(x.x));
+      qp[4 * i + 1] = f32x2_to_f16x2(bf16lo(x.y), bf16hi(x.y));
+      qp[4 * i + 2] = f32x2_to_f16x2(bf16lo(x.z), bf16hi(x.z));
+      qp[4 * i + 3] = f32x2_to_f16x2(bf16lo(x.w), bf16hi(x.w));
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int key = 32 * warp + 8 * u + quad;
+      v[u] = *reinterpret_cast<const uint4*>(st + key * 64 + 16 * l4);
+      const int64_t row = int64_t(m.b) * e.key_rows + m.i0 + key;
+      s2[u] = row == e.last_odd_row && key < m.cnt
+                  ? uint32_t(*reinterpret_cast<const uint16_t*>(e.scales + row * 8 + 2 * l4))
+                  : uint32_t(*reinterpret_cast<const uint16_t*>(st + Lay::kCodes + (m.soff + key) * 8 + 2 * l4));
+    }
+  }
+  __device__ __forceinline__ float score(int warp, int lane, int* key, bool* writer) const {
+    const int quad = lane >> 2, l4 = lane & 3;
+    float p[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
       const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
       uint32_t acc0 = 0, acc1 = 0;  // f16x2 sums of group 0 (words 0, 1) and group 1 (words 2, 3)
 #pragma unroll
@@ -396,55 +325,147 @@ __device__ __forceinline__ void score_segment_fp4(const uint16_t* __restrict__ q
     float k2[2];
 #pragma unroll
     for (int i = 0; i < 2; ++i) k2[i] = (bb1 ? p[2 + i] : p[i]) + __shfl_xor_sync(kFull, bb1 ? p[i] : p[2 + i], 2);
-    const float s = (bb0 ? k2[1] : k2[0]) + __shfl_xor_sync(kFull, bb0 ? k2[0] : k2[1], 1) + 0.0f;
-    const int64_t key = 8 * U * j + 8 * l4 + quad;  // lane l4 ends with key u = l4
-    if (key < cnt) {
-      sc[key] = s;
-      if (ssc) ssc[key] = s;
-      atomicAdd(&sh[ord_f32(s) >> 20], 1u);
-    }
-  };
-  const int64_t ngroups = (cnt + 8 * U - 1) / (8 * U);
-  uint4 va[U], vb[U];
-  uint32_t sa[U], sb2[U];
-  int64_t j = warp;
-  if (j < ngroups) load(j, va, sa);
-  while (j < ngroups) {
-    if (j + nwarps < ngroups) load(j + nwarps, vb, sb2);
-    process(j, va, sa);
-    j += nwarps;
-    if (j >= ngroups) break;
-    if (j + nwarps < ngroups) load(j + nwarps, va, sa);
-    process(j, vb, sb2);
-    j += nwarps;
+    *key = 32 * warp + 8 * l4 + quad;  // lane l4 ends with key u = l4
+    *writer = true;
+    return (bb0 ? k2[1] : k2[0]) + __shfl_xor_sync(kFull, bb0 ? k2[0] : k2[1], 1) + 0.0f;
   }
-}
+};
 
-__global__ void __launch_bounds__(256) index_score_fp4(const uint16_t* __restrict__ qidx,
-                                                       const uint8_t* __restrict__ codes,
-                                                       const uint8_t* __restrict__ scales, int64_t key_rows,
-                                                       int64_t n, int batch, int64_t per_cta,
-                                                       float* __restrict__ scores, uint32_t* __restrict__ hist) {
-  __shared__ uint32_t sh[kHistBins];
+template <class F>
+__global__ void __launch_bounds__(StreamLayout<F>::kThreads, 1)
+    index_score_stream(const uint16_t* __restrict__ qidx, const uint8_t* __restrict__ codes,
+                       const uint8_t* __restrict__ scales, int64_t key_rows, int64_t n, int64_t n_h, int batch,
+                       int64_t per_cta, float* __restrict__ scores, uint32_t* __restrict__ hist,
+                       uint32_t* __restrict__ tail_ctr, uint32_t* __restrict__ status) {
+  using Lay = StreamLayout<F>;
+  constexpr int S = F::kStages;
+  extern __shared__ __align__(128) uint8_t sraw[];
+  uint8_t* stage = sraw;
+  uint32_t* sh = reinterpret_cast<uint32_t*>(sraw + size_t(S) * Lay::kStage);  // [2][kHistBins]
+  StreamCtl<F>* ctl = reinterpret_cast<StreamCtl<F>*>(sh + 2 * kHistBins);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
-  const int64_t total = int64_t(batch) * n;
-  const int64_t g0 = int64_t(blockIdx.x) * per_cta;
-  const int64_t g1 = min(total, g0 + per_cta);
-  if (g0 >= g1) return;
-  pdl_wait();
-  const uint64_t pol = l2_evict_first_policy();  // keys are read once
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], F::kConsumers);
+    }
+    ctl->abort = 0;
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < 2 * kHistBins; i += Lay::kThreads) sh[i] = 0;
   __syncthreads();
-  for (int64_t s0 = g0; s0 < g1;) {
-    const int b = int(s0 / n);
-    const int64_t s1 = min(g1, int64_t(b + 1) * n);
-    const int64_t i0 = s0 - int64_t(b) * n;
-    const size_t r0 = size_t(b) * size_t(key_rows) + size_t(i0);
-    score_segment_fp4(qidx + size_t(b) * 128, codes + r0 * 64, scales + r0 * 8, s1 - s0,
-                      scores + size_t(b) * size_t(score_stride(n)) + size_t(i0), nullptr, sh, pol);
-    flush_histogram(sh, hist + size_t(b) * kHistBins);
-    __syncthreads();
-    s0 = s1;
+  pdl_wait();
+  const int64_t total = int64_t(batch) * n_h;
+  const int64_t g0 = min(total, int64_t(blockIdx.x) * per_cta), g1 = min(total, g0 + per_cta);
+  const int64_t tups = (n - n_h + F::kKeys - 1) / F::kKeys;  // tail units per sequence
+  const int64_t rows_total = int64_t(batch) * key_rows;      // rows of the key (and scale) arrays
+  const int64_t TU = n_h < n ? int64_t(batch) * tups : 0;
+
+  if (warp == F::kConsumers) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      const uint64_t pol = l2_evict_first_policy();  // keys are read once
+      int64_t pos = g0;
+      uint32_t claimed = TU > 0 ? atomicAdd(tail_ctr, 1u) : 0u;  // one claim ahead
+      int it = 0;
+      bool ok = true;
+      for (;; ++it) {
+        int b, cnt, tail;
+        int64_t i0;
+        if (pos < g1) {
+          b = int(pos / n_h);
+          i0 = pos - int64_t(b) * n_h;
+          const int64_t end = min(g1, int64_t(b + 1) * n_h);
+          cnt = int(min(int64_t(F::kKeys), end - pos));
+          pos += cnt;
+          tail = 0;
+        } else if (int64_t(claimed) < TU) {
+          b = int(int64_t(claimed) / tups);
+          i0 = n_h + (int64_t(claimed) % tups) * F::kKeys;
+          cnt = int(min(int64_t(F::kKeys), n - i0));
+          tail = 1;
+          claimed = atomicAdd(tail_ctr, 1u);
+        } else {
+          break;
+        }
+        const int s = it % S;
+        if (it >= S && !stream_wait(&ctl->empty[s], ((it / S) - 1) & 1, ctl)) {
+          ok = false;
+          break;
+        }
+        uint8_t* dst = stage + size_t(s) * Lay::kStage;
+        const int64_t row = int64_t(b) * key_rows + i0;
+        const uint32_t cbytes = uint32_t(cnt) * F::kCodeBytes;
+        // scale rows [r0, r1): from the even row at or below the first key to
+        // the even row at or above the end, but never past the last even row
+        // of the array (an odd total's last row is read by the consumers)
+        int64_t r0 = row, r1 = row;
+        if constexpr (F::kScaleBytes > 0) {
+          r0 = row & ~int64_t(1);
+          r1 = min((row + cnt + 1) & ~int64_t(1), rows_total & ~int64_t(1));
+        }
+        const uint32_t sbytes = uint32_t(r1 - r0) * F::kScaleBytes;
+        ctl->meta[s] = StreamMeta{b, cnt, i0, tail, int32_t(row - r0)};
+        mbar_arrive_expect_tx(&ctl->full[s], cbytes + sbytes + 256u);
+        bulk_load(dst, codes + size_t(row) * F::kCodeBytes, cbytes, &ctl->full[s], pol);
+        if (sbytes > 0) bulk_load(dst + Lay::kCodes, scales + size_t(r0) * F::kScaleBytes, sbytes, &ctl->full[s], pol);
+        bulk_load_plain(dst + Lay::kCodes + Lay::kScales, qidx + size_t(b) * 128, 256u, &ctl->full[s]);
+      }
+      bool marked = false;
+      if (ok) {  // the end marker
+        const int s = it % S;
+        if (it < S || stream_wait(&ctl->empty[s], ((it / S) - 1) & 1, ctl)) {
+          ctl->meta[s] = StreamMeta{0, -1, 0, 0, 0};
+          mbar_arrive(&ctl->full[s]);
+          marked = true;
+        }
+      }
+      // Normally the consumers wait for every copy before they finish.  After
+      // a wait that gave up, never leave with copies in flight: wait (bounded)
+      // for the last phase of each stage still armed (none was re-armed by a
+      // marker on this path).
+      if (!marked) {
+        const uint64_t t0 = stream_now();
+        for (int j = max(0, it - S); j < it; ++j)
+          while (!mbar_try_wait(&ctl->full[j % S], (j / S) & 1))
+            if (stream_now() - t0 > kStreamWaitNs) break;
+      }
+      if (ctl->abort) set_status(status, DSV4KV_DEV_TIMEOUT);
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------------ consumers
+  const int b0 = n_h > 0 ? int(g0 / n_h) : 0;  // the even share's first sequence: shared histogram 0
+  const StreamEdge edge{scales, key_rows, (rows_total & 1) ? rows_total - 1 : -1};
+  for (int it = 0;; ++it) {
+    const int s = it % S;
+    bool ok = true;
+    if (lane == 0) ok = stream_wait(&ctl->full[s], (it / S) & 1, ctl);
+    if (!__shfl_sync(kFull, ok, 0)) break;
+    const StreamMeta m = ctl->meta[s];
+    if (m.cnt < 0) break;
+    StreamConsumer<F> c;
+    c.load(stage + size_t(s) * Lay::kStage, m, edge, warp, lane);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ctl->empty[s]);  // the warp's keys are in registers
+    int key;
+    bool writer;
+    const float sc = c.score(warp, lane, &key, &writer);
+    if (writer && key < m.cnt) {
+      scores[size_t(m.b) * size_t(score_stride(n)) + size_t(m.i0 + key)] = sc;
+      const int bin = int(ord_f32(sc) >> 20), slot = m.b - b0;
+      if (!m.tail && slot >= 0 && slot < 2) atomicAdd(&sh[slot * kHistBins + bin], 1u);
+      else atomicAdd(&hist[size_t(m.b) * kHistBins + hist_pos(bin)], 1u);
+    }
+  }
+  // flush the two shared histograms (every consumer warp ends its loop: the waits are bounded)
+  asm volatile("barrier.cta.sync 1, %0;" ::"n"(32 * F::kConsumers) : "memory");
+  for (int i = threadIdx.x; i < 2 * kHistBins; i += 32 * F::kConsumers) {
+    const uint32_t c = sh[i];
+    const int bb = b0 + i / kHistBins;
+    if (c && bb < batch) atomicAdd(&hist[size_t(bb) * kHistBins + hist_pos(i % kHistBins)], c);
   }
 }
 
@@ -1677,45 +1698,38 @@ dsv4kv_status index_score_launch(const uint16_t* qidx, const dsv4kv_cache& keys,
   const IndexWs w = index_ws_layout(static_cast<char*>(ws), batch, n, k);
   if (ws_bytes < w.bytes) return set_error(DSV4KV_ERR_WORKSPACE, "index_score: workspace too small");
   const int sms = sm_count();
-  if (keys.fmt == DSV4KV_BF16) {
-    // one CTA per SM streaming through shared memory; the last kTailPct % of
-    // every sequence (whole 128-key units) goes to the shared queue, whose
-    // histogram counts go straight to global memory: with few sequences they
-    // would pile onto the few bins that hold most scores of one histogram,
-    // so small batches use the even split alone
-    static std::atomic<uint64_t> attr_set{0};
+  // one CTA per SM streaming the keys through shared memory; the last
+  // kTailPct % of every sequence (whole units of a stage's keys) goes to the
+  // shared queue, whose histogram counts go straight to global memory: with
+  // few sequences they would pile onto the few bins that hold most scores of
+  // one histogram, so small batches use the even split alone
+  if ((reinterpret_cast<uintptr_t>(qidx) | reinterpret_cast<uintptr_t>(keys.codes) |
+       reinterpret_cast<uintptr_t>(keys.scales)) & 15)
+    return set_error(DSV4KV_ERR_INVALID_ARG, "index_score: queries, codes and scales must be 16-byte aligned");
+  auto launch = [&](auto traits, void (*kern)(const uint16_t*, const uint8_t*, const uint8_t*, int64_t, int64_t,
+                                              int64_t, int, int64_t, float*, uint32_t*, uint32_t*, uint32_t*),
+                    std::atomic<uint64_t>& attr_set) -> dsv4kv_status {
+    using F = decltype(traits);
     if (!done_on_device(attr_set)) {
-      if (cudaFuncSetAttribute(index_score_stream, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kStreamSmem)) !=
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(stream_smem<F>())) !=
           cudaSuccess)
         return check_launch("index_score: cudaFuncSetAttribute");
       mark_done_on_device(attr_set);
     }
-    if ((reinterpret_cast<uintptr_t>(qidx) | reinterpret_cast<uintptr_t>(keys.codes)) & 15)
-      return set_error(DSV4KV_ERR_INVALID_ARG, "index_score: query and key rows must be 16-byte aligned");
-    const int64_t n_tail =
-        batch >= kTailMinBatch ? std::min<int64_t>(n, (n * kTailPct / 100) / kStreamKeys * kStreamKeys) : 0;
+    const int64_t n_tail = batch >= kTailMinBatch ? std::min<int64_t>(n, (n * kTailPct / 100) / F::kKeys * F::kKeys) : 0;
     const int64_t n_h = n - n_tail;
     const int64_t total = int64_t(batch) * n_h;
-    const int64_t per_cta = std::max<int64_t>(kStreamKeys, (total + sms - 1) / sms);
-    launch_pdl(index_score_stream, dim3(unsigned(sms)), dim3(kStreamThreads), kStreamSmem, stream, qidx,
-               static_cast<const uint16_t*>(keys.codes), keys.rows, n, n_h, batch, per_cta, w.scores, w.hist,
-               w.tail_ctr, w.status);
-  } else {
-    static std::atomic<int> occ4_dev[64];  // per device; 0 = not queried yet
-    std::atomic<int>& occ4_slot = occ4_dev[current_device()];
-    int occ4 = occ4_slot.load(std::memory_order_relaxed);
-    if (occ4 == 0) {
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ4, index_score_fp4, 256, 0) != cudaSuccess || occ4 < 1)
-        occ4 = 1;
-      occ4_slot.store(occ4, std::memory_order_relaxed);
-    }
-    const int64_t total = int64_t(batch) * n;
-    const int64_t grid = int64_t(sms) * occ4;
-    const int64_t per_cta = std::max<int64_t>(64, (total + grid - 1) / grid);
-    launch_pdl(index_score_fp4, dim3(unsigned((total + per_cta - 1) / per_cta)), dim3(256), 0, stream, qidx,
-               static_cast<const uint8_t*>(keys.codes), static_cast<const uint8_t*>(keys.scales), keys.rows, n,
-               batch, per_cta, w.scores, w.hist);
-  }
+    const int64_t per_cta = std::max<int64_t>(F::kKeys, (total + sms - 1) / sms);
+    launch_pdl(kern, dim3(unsigned(sms)), dim3(StreamLayout<F>::kThreads), stream_smem<F>(), stream, qidx,
+               static_cast<const uint8_t*>(keys.codes), static_cast<const uint8_t*>(keys.scales), keys.rows, n, n_h,
+               batch, per_cta, w.scores, w.hist, w.tail_ctr, w.status);
+    return DSV4KV_OK;
+  };
+  static std::atomic<uint64_t> attr_bf16{0}, attr_fp4{0};
+  const dsv4kv_status st = keys.fmt == DSV4KV_BF16
+                               ? launch(StreamBf16{}, index_score_stream<StreamBf16>, attr_bf16)
+                               : launch(StreamFp4{}, index_score_stream<StreamFp4>, attr_fp4);
+  if (st != DSV4KV_OK) return st;
   return check_launch("index_score");
 }
 
