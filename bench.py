@@ -983,7 +983,7 @@ def main():
     per_type = {kind: {"workload": wl_name, "steps_per_s": round(steps_per_s, 1),
                        "tokens_per_s": round(steps_per_s * batch, 1),
                        "hbm_gbs": round(alg / (ms * 1e-3) / 1e9, 1),
-                       "frac_of_measured_hbm": round(alg / (ms * 1e-3) / 1e9 / hbm_peak, 4),
+                       "frac_of_peak_hbm": round(alg / (ms * 1e-3) / 1e9 / hbm_peak, 4),
                        "frac_of_8tbs": round(alg / (ms * 1e-3) / 8e12, 4),
                        "index_ms": round(res["index_ms"], 5), "score_ms": round(res["score_ms"], 5),
                        "select_ms": round(res["select_ms"], 5), "decode_ms": round(res["decode_ms"], 5),
@@ -1010,9 +1010,9 @@ def main():
         per_type[name] = {"workload": desc2, "steps_per_s": round(d["world"] * 1e3 / ms2, 1),
                           "us_per_step": round(ms2 * 1e3, 2), "cache_replicas": r2n,
                           "hbm_gbs": round(a2 / (ms2 * 1e-3) / 1e9, 1),
-                          "frac_of_measured_hbm": round(a2 / (ms2 * 1e-3) / 1e9 / hbm_peak, 4),
+                          "frac_of_peak_hbm": round(a2 / (ms2 * 1e-3) / 1e9 / hbm_peak, 4),
                           "tflops": round(L2.flops() / (ms2 * 1e-3) / 1e12, 1),
-                          "frac_of_measured_bf16": round(L2.flops() / (ms2 * 1e-3) / 1e12 / tf_peak, 4)}
+                          "frac_of_peak_bf16": round(L2.flops() / (ms2 * 1e-3) / 1e12 / tf_peak, 4)}
         if spec[0] == "c4a":
             per_type[name]["index_us"] = round(r2["index_ms"] * 1e3, 2)
             per_type[name]["score_us"] = round(r2["score_ms"] * 1e3, 2)
