@@ -64,19 +64,29 @@ def test_index_topk_heavy_ties(lo, hi, n):
         assert np.array_equal(idx[s], ref)
 
 
-def test_index_topk_fp4_keys():
+@pytest.mark.parametrize("b,n,rows", [
+    (3, 20000, 20000),
+    (1, 5001, 5001),      # an odd number of rows: the last key's scale row is not in a 16-byte unit of its own
+    (3, 4999, 5003),      # sequences start on odd rows
+    (17, 3001, 3001),     # batch >= 16: the shared tail queue, odd total
+    (150, 1000, 1001),    # many short sequences per CTA
+])
+def test_index_topk_fp4_keys(b, n, rows):
     import datagen.gpu as G
-    b, n, k = 3, 20000, 512
-    kf = D.stream_key(5, D.TID_KIDX_FP4, 0)
-    kq = D.stream_key(5, D.TID_QIDX, 0)
-    codes = torch.empty(b, n, 64, dtype=torch.uint8, device="cuda")
-    scales = torch.empty(b, n, 8, dtype=torch.uint8, device="cuda")
+    k = 512
+    kf = D.stream_key(5 + n, D.TID_KIDX_FP4, 0)
+    kq = D.stream_key(5 + n, D.TID_QIDX, 0)
+    codes = torch.empty(b, rows, 64, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(b, rows, 8, dtype=torch.uint8, device="cuda")
     G.fp4_index_keys_(codes, scales, kf)
     q = G.int_bf16_(torch.empty(b, 128, dtype=torch.bfloat16, device="cuda"), kq)
-    idx, cnt = K.index_topk(q, K.Cache(2, codes, scales, 128), n, k)
+    ws = K.new_workspace(K.index_topk_workspace_bytes(b, n, k))
+    idx, cnt = K.index_topk(q, K.Cache(2, codes, scales, 128), n, k, ws=ws)
+    torch.cuda.synchronize()
+    assert K.workspace_status(ws) == 0
     idx = idx.cpu().numpy()
-    for s in range(b):
-        hc, hs = D.fp4_index_keys_rows(kf, np.arange(s * n, (s + 1) * n), 128)
+    for s in (range(b) if b <= 17 else (0, 77, b - 1)):
+        hc, hs = D.fp4_index_keys_rows(kf, np.arange(s * rows, s * rows + n), 128)
         kr = OF.dequant_fp4_rows(hc, hs)
         qr = OF.bf16_bits_to_f64(D.rows_int_bf16(kq, np.array([s]), 128)[0])
         ref, c = OI.index_topk(qr, kr, k)
