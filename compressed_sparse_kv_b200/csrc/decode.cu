@@ -9,12 +9,13 @@
 // One CTA per (sequence, split) walks a contiguous range of 64-row tiles of
 // the sequence's row list (selected or all compressed rows, then the window
 // rows).  Roles (10 warps):
-//   * warp 0 loads Q (TMA, 128-byte swizzle) and every tile whose rows are
-//     contiguous in HBM (dense compressed rows, window rows) with 2D TMA
-//     tiles: 8 copies of 64 rows x 64 channels per tile;
+//   * warp 0 loads Q (one 4-D TMA box, 128-byte swizzle) and every tile whose
+//     rows are contiguous in HBM (dense compressed rows, window rows) as one
+//     3-D TMA box of 64 rows x 8 chunks of 64 channels;
 //   * warps 6-9 load the tiles that are not: gathered bf16 rows with 16-byte
-//     cp.async straight into the swizzled tile, and quantised rows
-//     (fp8 / fp4) with 16-byte loads and hardware cvt to f16 (exact);
+//     cp.async straight into the swizzled tile (each lane reading its row's
+//     index from the selection), and quantised rows (fp8 / fp4) with 16-byte
+//     loads one tile ahead and hardware cvt to f16 (exact);
 //   * warp 1 (one thread) issues tcgen05.mma: S = Q . R^T (M = 64 heads,
 //     N = 64 rows, 32 K-steps of 16 channels; head h lands in TMEM lane
 //     32*(h/16) + h%16, row r in column r), and O^T += R^T . P^T
@@ -27,7 +28,10 @@
 //     TMEM only when a head's running max grows by > 2^8.
 // With one split per sequence the CTA normalises, applies the inverse RoPE
 // and stores the output itself; otherwise partial (O, m, l) go to the
-// workspace and decode_combine merges them with log-sum-exp weights.
+// workspace (O as bf16) and decode_combine merges them with log-sum-exp
+// weights (or, when enabled, the splits of a thread-block cluster merge over
+// distributed shared memory: cluster_merge).  TMEM is freed after every
+// warp has arrived on a retire barrier.
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
