@@ -70,6 +70,7 @@ _SIGS = {
     "dsv4kv_index_topk_noalloc": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.c_int32, _c.c_int64, _c.c_int32,
                                              _c.c_void_p, _c.c_void_p, _c.c_void_p]),
     "dsv4kv_index_topk_noalloc_status": (_c.c_int, [_c.c_void_p, _c.c_int32, _c.c_void_p]),
+    "dsv4kv_selftest_wait_timeout": (_c.c_int, [_c.c_void_p, _c.c_void_p]),
     "dsv4kv_sparse_decode_workspace_bytes": (_c.c_size_t, [_c.c_int32, _c.c_int32, _c.c_int32, _c.c_int32,
                                                            _c.c_int32]),
     "dsv4kv_sparse_decode": (_c.c_int, [_c.c_void_p, _c.POINTER(CacheDesc), _c.POINTER(CacheDesc), _c.c_void_p,
@@ -307,6 +308,12 @@ def index_topk_noalloc_status(clear: bool = False, stream=None) -> int:
            "dsv4kv_index_topk_noalloc_status")
     s.synchronize()
     return int(word.item()) & 0xffffffff
+
+
+def selftest_wait_timeout(status: torch.Tensor, stream=None) -> None:
+    """Launch the library's bounded-wait self-test: after about one second on the GPU it ORs DEV_TIMEOUT
+    into `status` (one int32 on the device)."""
+    _check(lib().dsv4kv_selftest_wait_timeout(_ptr(status), _stream(stream)), "dsv4kv_selftest_wait_timeout")
 
 
 def sparse_decode_workspace_bytes(batch: int, heads: int, k: int, window: int, dim: int = 512) -> int:

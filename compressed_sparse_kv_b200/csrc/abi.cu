@@ -126,6 +126,11 @@ DSV4KV_API const char* dsv4kv_last_error(void) { return g_err; }
 
 DSV4KV_API const char* dsv4kv_version(void) { return "dsv4kv 0.1 (sm_100a)"; }
 
+DSV4KV_API dsv4kv_status dsv4kv_selftest_wait_timeout(uint32_t* status, void* stream) {
+  if (!status) return set_error(DSV4KV_ERR_INVALID_ARG, "selftest_wait_timeout: status is null");
+  return selftest_wait_timeout_launch(status, static_cast<cudaStream_t>(stream));
+}
+
 DSV4KV_API int64_t dsv4kv_compress_entries(int64_t t, int32_t window, int32_t stride) {
   if (stride <= 0 || t < window) return 0;
   return (t - window) / stride;

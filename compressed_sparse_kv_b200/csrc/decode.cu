@@ -1413,7 +1413,27 @@ DecodeWs decode_ws_layout(char* base, int batch, int heads, const Plan& pl) {
   return w;
 }
 
+// Self-test of the bounded waits: one thread waits with wait_or_abort (as
+// every wait of decode_kernel does) on an mbarrier that no thread arrives on,
+// gives up after kWaitLimitNs, and flags DSV4KV_DEV_TIMEOUT.
+__global__ void wait_timeout_probe(uint32_t* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ Ctl ctl;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    ctl.abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !wait_or_abort(&bar, 0, &ctl)) set_status(status, DSV4KV_DEV_TIMEOUT);
+}
+
 }  // namespace
+
+dsv4kv_status selftest_wait_timeout_launch(uint32_t* status, cudaStream_t stream) {
+  wait_timeout_probe<<<1, 32, 0, stream>>>(status);
+  return check_launch("selftest_wait_timeout");
+}
 
 size_t decode_ws_bytes(int batch, int heads, int dim, int64_t rows_per_seq) {
   (void)dim;

@@ -52,6 +52,7 @@ cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, 
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 dsv4kv_status check_launch(const char* what);
+dsv4kv_status selftest_wait_timeout_launch(uint32_t* status, cudaStream_t stream);
 int sm_count();
 // The current device (0 when it cannot be read or is >= 64).  One-time set-up
 // of a kernel (shared-memory limits, occupancy queries) is kept per device,

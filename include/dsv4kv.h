@@ -381,6 +381,16 @@ const char* dsv4kv_last_error(void);
 /* Library version string. */
 const char* dsv4kv_version(void);
 
+/* Self-test of the device-side failure path (no passage of the pages: it
+ * checks the library's own error reporting).  Launches one thread that waits
+ * on a barrier no thread completes, with the same bounded wait as every wait
+ * in the library's kernels; after the one-second limit it gives up and ORs
+ * DSV4KV_DEV_TIMEOUT into *status.  status: one uint32 in device memory,
+ * owned by the caller (not cleared).  Asynchronous on `stream`; the context
+ * stays usable.  Errors: DSV4KV_ERR_INVALID_ARG (null status),
+ * DSV4KV_ERR_CUDA (launch). */
+dsv4kv_status dsv4kv_selftest_wait_timeout(uint32_t* status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

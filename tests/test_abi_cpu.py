@@ -121,3 +121,10 @@ def test_new_entry_points_reject_bad_arguments():
     rc = L.dsv4kv_dense_decode(16, ctypes.byref(f3), ctypes.byref(f3), 1, 64, 100, 100, 4096, 0.044, 32, 1e4, 0,
                                16, 16, 1 << 30, z)
     assert rc == 2 and "rope_dim" in K.lib().dsv4kv_last_error().decode()
+
+
+def test_selftest_rejects_a_null_status():
+    """The bounded-wait self-test validates its argument on the host (nothing launched)."""
+    z = ctypes.c_void_p(0)
+    rc, msg = _status(K.lib().dsv4kv_selftest_wait_timeout(z, z))
+    assert rc == 1 and "status" in msg
