@@ -7,9 +7,10 @@
 // K taps mixes positions s*i + s - K + j (j < K; positions < 0 contribute 0),
 // per channel, then rotates its rotary channel pairs at position pos0 + s*i.
 //
-// Layout of the work: one warp per entry, each lane owns 16 consecutive
-// channels (two 16-byte bf16 loads per tap row), so a tap row is one fully
-// coalesced 1 KB read.  The K tap loads are unrolled by 4 to keep several
+// Layout of the work (compress_kernel; c4a at dim 512 uses compress_c4_kernel
+// below): one warp per entry, each lane owns 16 consecutive channels (two
+// 16-byte bf16 loads per tap row), so a tap row is one fully coalesced 1 KB
+// read.  The K tap loads are unrolled by 4 to keep several
 // rows in flight; c4a entries overlap by 4 rows, which the L1/L2 absorb.
 // The rotation: the block computes rope_base^(-2m/rope_dim) / pi once per
 // pair m (shared memory); per entry, lane m computes the cos / sin of pair m
@@ -125,6 +126,102 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock)
   }
 }
 
+
+// c4a-shaped compression (K taps at stride S = K / 2, dim 512), with each
+// warp emitting consecutive entries: entry i mixes rows [S(i-1), S(i+1)), so
+// row r feeds entry floor(r / S) (taps S..K-1) and the next one (taps
+// 0..S-1).  A CTA of four warps takes kC4Entries consecutive entries of one
+// sequence; warp w owns channels [128 w, 128 w + 128), 4 per lane, whose K x 4
+// weights stay in registers.  The warp walks its rows once, block by block of
+// S rows (the next block's loads issued before the current one is used),
+// keeping two accumulators: the entry being completed and the next one.  The
+// taps of an entry are added in ascending order, as in compress_kernel, so
+// the results are the same bit for bit.
+constexpr int kC4Entries = 32;
+
+template <int K>
+__global__ void __launch_bounds__(128) compress_c4_kernel(const uint16_t* __restrict__ s_raw,
+                                                          const float* __restrict__ w, int64_t t, int64_t n_entries,
+                                                          int64_t pos0, int rope_dim, double rope_base, int out_fp32,
+                                                          void* __restrict__ out) {
+  constexpr int S = K / 2, D = 512;
+  __shared__ double theta_pi[kMaxRopePairs];  // rope_base^(-2m/rope_dim) / pi
+  for (int m = threadIdx.x; m < rope_dim / 2; m += blockDim.x)
+    theta_pi[m] = pow(rope_base, -2.0 * double(m) / double(rope_dim)) / 3.141592653589793;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.y;
+  const int64_t i0 = int64_t(blockIdx.x) * kC4Entries;
+  const int64_t i1 = min(n_entries, i0 + kC4Entries);
+  if (i0 >= i1) return;
+  const int c = 128 * warp + 4 * lane;  // this lane's 4 channels
+  float wr[K][4];
+#pragma unroll
+  for (int j = 0; j < K; ++j) {
+    const float4 x = *reinterpret_cast<const float4*>(w + size_t(j) * D + c);
+    wr[j][0] = x.x;
+    wr[j][1] = x.y;
+    wr[j][2] = x.z;
+    wr[j][3] = x.w;
+  }
+  const uint16_t* sb = s_raw + size_t(b) * size_t(t) * D + c;
+  auto load_block = [&](int64_t q, uint2 (&v)[S]) {
+#pragma unroll
+    for (int u = 0; u < S; ++u) {
+      const int64_t r = S * q + u;
+      v[u] = r >= 0 ? *reinterpret_cast<const uint2*>(sb + size_t(r) * D) : make_uint2(0, 0);
+    }
+  };
+  const int r0 = D - rope_dim;
+  float acc_a[4] = {0.f, 0.f, 0.f, 0.f}, acc_b[4] = {0.f, 0.f, 0.f, 0.f};
+  uint2 cur[S], nxt[S] = {};
+  int64_t q = i0 - 1;  // block q = rows [S q, S q + S): taps S.. of entry q, taps 0.. of entry q + 1
+  load_block(q, cur);
+  for (; q < i1; ++q) {
+    if (q + 1 < i1) load_block(q + 1, nxt);
+#pragma unroll
+    for (int u = 0; u < S; ++u) {
+      if (S * q + u < 0) continue;  // positions before 0 contribute nothing
+      const float x[4] = {bf16lo(cur[u].x), bf16hi(cur[u].x), bf16lo(cur[u].y), bf16hi(cur[u].y)};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc_a[e] = fmaf(wr[S + u][e], x[e], acc_a[e]);
+        acc_b[e] = fmaf(wr[u][e], x[e], acc_b[e]);
+      }
+    }
+    if (q >= i0) {  // entry q is complete: rotate its rotary pairs at position pos0 + S q, store
+      if (c + 4 > r0) {
+        const double pos = double(pos0 + int64_t(S) * q);
+#pragma unroll
+        for (int e = 0; e < 4; e += 2) {
+          if (c + e >= r0) {
+            const double ang = pos * theta_pi[(c + e - r0) >> 1];
+            double sd, cd;
+            sincospi(ang - 2.0 * rint(0.5 * ang), &sd, &cd);
+            const float cs = float(cd), sn = float(sd);
+            const float xa = acc_a[e], ya = acc_a[e + 1];
+            acc_a[e] = float(double(xa) * cs - double(ya) * sn);
+            acc_a[e + 1] = float(double(xa) * sn + double(ya) * cs);
+          }
+        }
+      }
+      const size_t o = (size_t(b) * size_t(n_entries) + size_t(q)) * D + c;
+      if (out_fp32)
+        *reinterpret_cast<float4*>(static_cast<float*>(out) + o) = make_float4(acc_a[0], acc_a[1], acc_a[2], acc_a[3]);
+      else
+        *reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + o) =
+            make_uint2(pack_bf16x2(acc_a[0], acc_a[1]), pack_bf16x2(acc_a[2], acc_a[3]));
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc_a[e] = acc_b[e];
+      acc_b[e] = 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < S; ++u) cur[u] = nxt[u];
+  }
+}
+
 }  // namespace
 
 dsv4kv_status compress_launch(const void* s_raw, const float* w, int batch, int64_t t, int dim, int k_taps,
@@ -132,8 +229,13 @@ dsv4kv_status compress_launch(const void* s_raw, const float* w, int batch, int6
                               int out_fp32, void* out, cudaStream_t stream) {
   const int64_t n = std::max<int64_t>(0, (t - window) / stride);
   if (n == 0) return DSV4KV_OK;
-  dim3 grid(unsigned((n + kWarpsPerBlock - 1) / kWarpsPerBlock), unsigned(batch));
   const uint16_t* s = static_cast<const uint16_t*>(s_raw);
+  if (dim == 512 && k_taps == 8 && stride == 4) {  // c4a: consecutive entries per warp
+    dim3 grid(unsigned((n + kC4Entries - 1) / kC4Entries), unsigned(batch));
+    compress_c4_kernel<8><<<grid, 128, 0, stream>>>(s, w, t, n, pos0, rope_dim, rope_base, out_fp32, out);
+    return check_launch("compress_c4_kernel");
+  }
+  dim3 grid(unsigned((n + kWarpsPerBlock - 1) / kWarpsPerBlock), unsigned(batch));
   switch (dim) {
     case 256:
       compress_kernel<8><<<grid, 32 * kWarpsPerBlock, 0, stream>>>(s, w, t, k_taps, stride, n, pos0, rope_dim,

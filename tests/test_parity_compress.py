@@ -22,6 +22,7 @@ def _raw(seed, b, t, d=512):
     ("c4a", 1, 2048, 128, 0),          # tiny c4a: 480 entries
     ("c4a", 2, 1000 + 3, 128, 0),      # ragged t
     ("c4a", 1, 4096, 0, 1 << 20),      # no window, large positions
+    ("c4a", 2, 131072, 128, 12345),    # c4a t=131072: 32736 entries, 1023 blocks of 32 per sequence
     ("c128a", 2, 128 * 20 + 128 + 50, 128, 0),
     ("c128a", 1, 131072, 128, 0),      # c128a t=131072: 1023 entries
 ])
