@@ -7,8 +7,8 @@
 // K taps mixes positions s*i + s - K + j (j < K; positions < 0 contribute 0),
 // per channel, then rotates its rotary channel pairs at position pos0 + s*i.
 //
-// Layout of the work (compress_kernel; c4a at dim 512 uses compress_c4_kernel
-// below): one warp per entry, each lane owns 16 consecutive channels (two
+// Layout of the work (compress_kernel; at dim 512, c4a uses compress_c4_kernel
+// and c128a compress_c128_kernel, below): one warp per entry, each lane owns 16 consecutive channels (two
 // 16-byte bf16 loads per tap row), so a tap row is one fully coalesced 1 KB
 // read.  The K tap loads are unrolled by 4 to keep several
 // rows in flight; c4a entries overlap by 4 rows, which the L1/L2 absorb.
@@ -222,6 +222,96 @@ __global__ void __launch_bounds__(128) compress_c4_kernel(const uint16_t* __rest
   }
 }
 
+
+// c128a-shaped compression (K taps at stride S = K, K a multiple of 16, dim
+// 512): entries do not share rows, and the K x 512 fp32 weights (256 KB for
+// K = 128) are what every entry re-reads.  A CTA of four warps takes
+// kC128Entries consecutive entries of one sequence; warp w owns channels
+// [128 w, 128 w + 128), 4 per lane, and keeps the accumulators of all its
+// entries in registers.  The weights come through shared memory 16 taps
+// (32 KB) at a time, so each weight is read from L2 once per CTA instead of
+// once per entry; the rows stream with 16 loads in flight per lane.  (Bulk
+// c128a, B=8 t=131072: 16 entries and 16-tap chunks 288 us; 8 entries and
+// 32-tap chunks 459 us; one warp per entry with the weights from L2 387 us.)
+// Taps are added in ascending order, as in compress_kernel, so the results
+// are the same bit for bit.
+constexpr int kC128Entries = 16;
+constexpr int kC128Chunk = 16;  // taps per staged weight chunk (the rows go in batches of 16 taps)
+static_assert(kC128Chunk % 16 == 0, "whole batches of 16 taps per chunk");
+
+__global__ void __launch_bounds__(128) compress_c128_kernel(const uint16_t* __restrict__ s_raw,
+                                                            const float* __restrict__ w, int64_t t, int k_taps,
+                                                            int64_t n_entries, int64_t pos0, int rope_dim,
+                                                            double rope_base, int out_fp32, void* __restrict__ out) {
+  constexpr int D = 512, E = kC128Entries, J = kC128Chunk;
+  extern __shared__ __align__(16) float w_s[];  // [J][D]
+  __shared__ double theta_pi[kMaxRopePairs];
+  for (int m = threadIdx.x; m < rope_dim / 2; m += blockDim.x)
+    theta_pi[m] = pow(rope_base, -2.0 * double(m) / double(rope_dim)) / 3.141592653589793;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.y;
+  const int64_t i0 = int64_t(blockIdx.x) * E;
+  const int ne = int(min(int64_t(E), n_entries - i0));
+  const int c = 128 * warp + 4 * lane;
+  const int S = k_taps;
+  const uint16_t* sb = s_raw + size_t(b) * size_t(t) * D + c;
+  float acc[E][4];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e][0] = acc[e][1] = acc[e][2] = acc[e][3] = 0.f;
+  for (int jc = 0; jc < k_taps; jc += J) {
+    __syncthreads();  // the previous chunk's weights have been used
+    for (int v = threadIdx.x; v < J * D / 4; v += blockDim.x)
+      reinterpret_cast<float4*>(w_s)[v] = reinterpret_cast<const float4*>(w + size_t(jc) * D)[v];
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      if (e >= ne) continue;
+      const uint16_t* rows = sb + (size_t(S) * size_t(i0 + e) + size_t(jc)) * D;  // tap jc of entry i0 + e
+#pragma unroll
+      for (int h = 0; h < J; h += 16) {
+        uint2 x[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) x[u] = *reinterpret_cast<const uint2*>(rows + size_t(h + u) * D);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const float4 wv = *reinterpret_cast<const float4*>(w_s + (h + u) * D + c);
+          acc[e][0] = fmaf(wv.x, bf16lo(x[u].x), acc[e][0]);
+          acc[e][1] = fmaf(wv.y, bf16hi(x[u].x), acc[e][1]);
+          acc[e][2] = fmaf(wv.z, bf16lo(x[u].y), acc[e][2]);
+          acc[e][3] = fmaf(wv.w, bf16hi(x[u].y), acc[e][3]);
+        }
+      }
+    }
+  }
+  const int r0 = D - rope_dim;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    if (e >= ne) continue;
+    const int64_t i = i0 + e;
+    if (c + 4 > r0) {  // rotate the rotary pairs at position pos0 + S i
+      const double pos = double(pos0 + int64_t(S) * i);
+#pragma unroll
+      for (int q = 0; q < 4; q += 2) {
+        if (c + q >= r0) {
+          const double ang = pos * theta_pi[(c + q - r0) >> 1];
+          double sd, cd;
+          sincospi(ang - 2.0 * rint(0.5 * ang), &sd, &cd);
+          const float cs = float(cd), sn = float(sd);
+          const float xa = acc[e][q], ya = acc[e][q + 1];
+          acc[e][q] = float(double(xa) * cs - double(ya) * sn);
+          acc[e][q + 1] = float(double(xa) * sn + double(ya) * cs);
+        }
+      }
+    }
+    const size_t o = (size_t(b) * size_t(n_entries) + size_t(i)) * D + c;
+    if (out_fp32)
+      *reinterpret_cast<float4*>(static_cast<float*>(out) + o) = make_float4(acc[e][0], acc[e][1], acc[e][2], acc[e][3]);
+    else
+      *reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + o) =
+          make_uint2(pack_bf16x2(acc[e][0], acc[e][1]), pack_bf16x2(acc[e][2], acc[e][3]));
+  }
+}
+
 }  // namespace
 
 dsv4kv_status compress_launch(const void* s_raw, const float* w, int batch, int64_t t, int dim, int k_taps,
@@ -234,6 +324,19 @@ dsv4kv_status compress_launch(const void* s_raw, const float* w, int batch, int6
     dim3 grid(unsigned((n + kC4Entries - 1) / kC4Entries), unsigned(batch));
     compress_c4_kernel<8><<<grid, 128, 0, stream>>>(s, w, t, n, pos0, rope_dim, rope_base, out_fp32, out);
     return check_launch("compress_c4_kernel");
+  }
+  if (dim == 512 && k_taps == stride && k_taps % kC128Chunk == 0) {  // c128a: weights staged per CTA
+    static std::atomic<uint64_t> attr_set{0};
+    constexpr int kSmem = kC128Chunk * 512 * int(sizeof(float));
+    if (!done_on_device(attr_set)) {
+      if (cudaFuncSetAttribute(compress_c128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
+          cudaSuccess)
+        return check_launch("compress: cudaFuncSetAttribute");
+      mark_done_on_device(attr_set);
+    }
+    dim3 grid(unsigned((n + kC128Entries - 1) / kC128Entries), unsigned(batch));
+    compress_c128_kernel<<<grid, 128, kSmem, stream>>>(s, w, t, k_taps, n, pos0, rope_dim, rope_base, out_fp32, out);
+    return check_launch("compress_c128_kernel");
   }
   dim3 grid(unsigned((n + kWarpsPerBlock - 1) / kWarpsPerBlock), unsigned(batch));
   switch (dim) {
