@@ -56,3 +56,26 @@ def test_window_rows_are_one_tap_compression():
     from oracle import rope as OR
     ref = OR.rope(r[t - W:], np.arange(t - W, t))
     assert_close(to_f64(win)[0], ref, max_abs=1e-5, rel_l2=1e-6)
+
+
+@pytest.mark.parametrize("d,k,s,rope_dim", [
+    (256, 8, 4, 64),       # c4a shape at dim 256 (one warp per entry)
+    (1024, 8, 4, 128),     # dim 1024, a wider rotary part
+    (512, 6, 4, 64),       # taps that are not 2 x stride
+    (512, 40, 40, 64),     # stride = taps, not a multiple of 16 (one warp per entry)
+    (512, 96, 96, 64),     # stride = taps = 96: the staged-weight kernel with 6 chunks
+    (512, 128, 128, 0),    # c128a shape without rotary channels
+])
+def test_compress_other_shapes(d, k, s, rope_dim):
+    """Shapes beside the two bench shapes: the one-warp-per-entry kernel and the staged-weight kernel at
+    other tap counts."""
+    b, t, window, pos0 = 2, 3 * 128 + 200, 128, 777
+    raw, key = _raw(11 + d + k, b, t, d)
+    w = D.compress_weights(9, 0, k, d)
+    out = K.compress(raw, torch.from_numpy(w).cuda(), s, window, pos0=pos0, rope_dim=rope_dim, out_fp32=True)
+    got = to_f64(out)
+    for bb in range(b):
+        r = OF.bf16_bits_to_f64(D.normal_bf16(key, t * d, offset=bb * t * d).reshape(t, d))
+        ref = OC.compress(r, w.astype(np.float64), s, window, pos0=pos0, rope_dim=rope_dim)
+        assert got[bb].shape == ref.shape
+        assert np.abs(got[bb] - ref).max() < 1e-4
