@@ -236,23 +236,24 @@ __global__ void __launch_bounds__(128) compress_c4_kernel(const uint16_t* __rest
 // Taps are added in ascending order, as in compress_kernel, so the results
 // are the same bit for bit.
 constexpr int kC128Entries = 16;
+constexpr int kC128Groups = 2;  // groups of four warps, each taking kC128Entries / kC128Groups of the entries
 constexpr int kC128Chunk = 16;  // taps per staged weight chunk (the rows go in batches of 16 taps)
 static_assert(kC128Chunk % 16 == 0, "whole batches of 16 taps per chunk");
 
-__global__ void __launch_bounds__(128) compress_c128_kernel(const uint16_t* __restrict__ s_raw,
+__global__ void __launch_bounds__(128 * kC128Groups) compress_c128_kernel(const uint16_t* __restrict__ s_raw,
                                                             const float* __restrict__ w, int64_t t, int k_taps,
                                                             int64_t n_entries, int64_t pos0, int rope_dim,
                                                             double rope_base, int out_fp32, void* __restrict__ out) {
-  constexpr int D = 512, E = kC128Entries, J = kC128Chunk;
+  constexpr int D = 512, E = kC128Entries / kC128Groups, J = kC128Chunk;
   extern __shared__ __align__(16) float w_s[];  // [J][D]
   __shared__ double theta_pi[kMaxRopePairs];
   for (int m = threadIdx.x; m < rope_dim / 2; m += blockDim.x)
     theta_pi[m] = pow(rope_base, -2.0 * double(m) / double(rope_dim)) / 3.141592653589793;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
-  const int64_t i0 = int64_t(blockIdx.x) * E;
-  const int ne = int(min(int64_t(E), n_entries - i0));
-  const int c = 128 * warp + 4 * lane;
+  const int64_t i0 = int64_t(blockIdx.x) * kC128Entries + int64_t(warp >> 2) * E;  // this warp's entries
+  const int ne = int(max(int64_t(0), min(int64_t(E), n_entries - i0)));
+  const int c = 128 * (warp & 3) + 4 * lane;
   const int S = k_taps;
   const uint16_t* sb = s_raw + size_t(b) * size_t(t) * D + c;
   float acc[E][4];
@@ -335,7 +336,8 @@ dsv4kv_status compress_launch(const void* s_raw, const float* w, int batch, int6
       mark_done_on_device(attr_set);
     }
     dim3 grid(unsigned((n + kC128Entries - 1) / kC128Entries), unsigned(batch));
-    compress_c128_kernel<<<grid, 128, kSmem, stream>>>(s, w, t, k_taps, n, pos0, rope_dim, rope_base, out_fp32, out);
+    compress_c128_kernel<<<grid, 128 * kC128Groups, kSmem, stream>>>(s, w, t, k_taps, n, pos0, rope_dim, rope_base,
+                                                                    out_fp32, out);
     return check_launch("compress_c128_kernel");
   }
   dim3 grid(unsigned((n + kWarpsPerBlock - 1) / kWarpsPerBlock), unsigned(batch));
