@@ -225,18 +225,20 @@ __global__ void __launch_bounds__(128) compress_c4_kernel(const uint16_t* __rest
 
 // c128a-shaped compression (K taps at stride S = K, K a multiple of 16, dim
 // 512): entries do not share rows, and the K x 512 fp32 weights (256 KB for
-// K = 128) are what every entry re-reads.  A CTA of four warps takes
-// kC128Entries consecutive entries of one sequence; warp w owns channels
-// [128 w, 128 w + 128), 4 per lane, and keeps the accumulators of all its
-// entries in registers.  The weights come through shared memory 16 taps
-// (32 KB) at a time, so each weight is read from L2 once per CTA instead of
-// once per entry; the rows stream with 16 loads in flight per lane.  (Bulk
-// c128a, B=8 t=131072: 16 entries and 16-tap chunks 288 us; 8 entries and
-// 32-tap chunks 459 us; one warp per entry with the weights from L2 387 us.)
+// K = 128) are what every entry re-reads.  A CTA of kC128Groups groups of
+// four warps takes kC128Entries consecutive entries of one sequence, each
+// group a quarter of them; warp w of a group owns channels [128 w, 128 w +
+// 128), 4 per lane, and keeps the accumulators of its entries in registers.
+// The weights come through shared memory 16 taps (32 KB) at a time, so each
+// weight is read from L2 once per CTA instead of once per entry; the rows
+// stream with 16 loads in flight per lane.  (Bulk c128a, B=8 t=131072, 16
+// entries and 16-tap chunks: 182 us with four groups, 226 with two, 230 with
+// eight, 288 with one; 211 us with four groups of 8 entries; one warp per
+// entry with the weights from L2 387 us.)
 // Taps are added in ascending order, as in compress_kernel, so the results
 // are the same bit for bit.
 constexpr int kC128Entries = 16;
-constexpr int kC128Groups = 2;  // groups of four warps, each taking kC128Entries / kC128Groups of the entries
+constexpr int kC128Groups = 4;  // groups of four warps, each taking kC128Entries / kC128Groups of the entries
 constexpr int kC128Chunk = 16;  // taps per staged weight chunk (the rows go in batches of 16 taps)
 static_assert(kC128Chunk % 16 == 0, "whole batches of 16 taps per chunk");
 
