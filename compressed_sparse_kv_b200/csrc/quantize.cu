@@ -13,8 +13,16 @@
 //             the fp8 row rule over the first D - 64 channels (amax over
 //             those only), then the last 64 channels as bf16 (nearest even);
 //             a row is D - 64 code bytes followed by the 64 bf16 values.
-// Divisions are IEEE round-to-nearest (__fdiv_rn); conversions use the
-// hardware cvt.rn.satfinite instructions.  One warp per row.
+// Divisions are IEEE round-to-nearest: by a row's (or group's) scale s they
+// use Markstein's method (P. Markstein, "Computation of elementary functions
+// on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): with
+// y = RN(1/s), q0 = RN(x y), the remainder r = x - s q0 is exact in one FMA
+// and RN(q0 + r y) = RN(x / s), which holds while nothing under- or
+// overflows: the quotients here are at most 448 in magnitude, scales outside
+// [2^-64, 2^64] take __fdiv_rn instead (so y is a normal number), and
+// quotients small enough for r to underflow round to a zero code either way.
+// The sign of a zero quotient is restored after the correction.  Conversions use the hardware
+// cvt.rn.satfinite instructions.  One warp per row.
 #include <cstdint>
 
 #include "common.cuh"
@@ -40,6 +48,27 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float hi, float lo) {
       : "f"(hi), "f"(lo));
   return r & 0xffu;  // lo in bits 0..3, hi in bits 4..7
 }
+// x / s rounded to nearest for every x of a row or group that shares s.
+struct RnDivider {
+  float s, y;  // the divisor and RN(1 / s)
+  bool fast;
+  __device__ __forceinline__ float operator()(float x) const {
+    if (!fast) return __fdiv_rn(x, s);
+    const float q0 = x * y;
+    const float r = fmaf(-q0, s, x);
+    // The correction turns a quotient of -0 into +0; the sign of x / s is
+    // the sign of q0 (s > 0), so it is put back.
+    return copysignf(fmaf(r, y, q0), q0);
+  }
+};
+__device__ __forceinline__ RnDivider rn_divider(float s) {
+  RnDivider d;
+  d.s = s;
+  d.y = __frcp_rn(s);
+  d.fast = s >= 0x1p-64f && s <= 0x1p64f;  // false for NaN
+  return d;
+}
+
 __device__ __forceinline__ float e4m3_value(uint32_t c) {
   const float v = __uint_as_float((c & 0x7fu) << 20) * 0x1p120f;
   return (c & 0x80u) ? -v : v;
@@ -86,13 +115,14 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
     const float scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    const RnDivider div = rn_divider(scale);
     uint8_t* row_dst = codes + size_t(row) * (D + 64);
     if (body) {
       uint32_t packed[PER / 4];
 #pragma unroll
       for (int v = 0; v < PER / 4; ++v) {
-        const uint32_t lo = cvt_e4m3x2(__fdiv_rn(x[4 * v + 1], scale), __fdiv_rn(x[4 * v], scale));
-        const uint32_t hi = cvt_e4m3x2(__fdiv_rn(x[4 * v + 3], scale), __fdiv_rn(x[4 * v + 2], scale));
+        const uint32_t lo = cvt_e4m3x2(div(x[4 * v + 1]), div(x[4 * v]));
+        const uint32_t hi = cvt_e4m3x2(div(x[4 * v + 3]), div(x[4 * v + 2]));
         packed[v] = lo | (hi << 16);
       }
 #pragma unroll
@@ -111,11 +141,12 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
     const float scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    const RnDivider div = rn_divider(scale);
     uint32_t packed[PER / 4];
 #pragma unroll
     for (int v = 0; v < PER / 4; ++v) {
-      const uint32_t lo = cvt_e4m3x2(__fdiv_rn(x[4 * v + 1], scale), __fdiv_rn(x[4 * v], scale));
-      const uint32_t hi = cvt_e4m3x2(__fdiv_rn(x[4 * v + 3], scale), __fdiv_rn(x[4 * v + 2], scale));
+      const uint32_t lo = cvt_e4m3x2(div(x[4 * v + 1]), div(x[4 * v]));
+      const uint32_t hi = cvt_e4m3x2(div(x[4 * v + 3]), div(x[4 * v + 2]));
       packed[v] = lo | (hi << 16);
     }
     uint8_t* dst = codes + size_t(row) * D + PER * lane;
@@ -139,6 +170,9 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock)
       s_code[g] = cvt_e4m3x2(0.f, __fdiv_rn(amax, 6.f)) & 0xffu;
       s_val[g] = e4m3_value(s_code[g]);
     }
+    RnDivider divs[NG];
+#pragma unroll
+    for (int g = 0; g < NG; ++g) divs[g] = rn_divider(s_val[g] > 0.f ? s_val[g] : 1.f);
     uint8_t* dst = codes + size_t(row) * (D / 2) + (PER / 2) * lane;
     uint32_t packed[PER / 8 > 0 ? PER / 8 : 1];
 #pragma unroll
@@ -146,7 +180,8 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock)
 #pragma unroll
     for (int e = 0; e < PER; e += 2) {
       const float s = s_val[e / G];
-      const uint32_t byte = s > 0.f ? cvt_e2m1x2(__fdiv_rn(x[e + 1], s), __fdiv_rn(x[e], s)) : 0u;
+      const RnDivider& div = divs[e / G];
+      const uint32_t byte = s > 0.f ? cvt_e2m1x2(div(x[e + 1]), div(x[e])) : 0u;
       packed[e / 8] |= byte << (8 * ((e / 2) & 3));
     }
     if (PER >= 8) {

@@ -66,3 +66,27 @@ def test_quantize_full_size_rows():
         assert np.array_equal(codes[sample].cpu().numpy(), rc)
         got_s = scales[sample].cpu().numpy()
         assert np.array_equal(got_s.view(np.uint8), np.asarray(rs).view(np.uint8))
+
+
+@pytest.mark.parametrize("fmt", [K.FP8_E4M3_ROW, K.FP4_E2M1_G16, K.FP8_E4M3_ROW_ROPE_BF16])
+def test_quantize_bit_exact_across_magnitudes(fmt):
+    """fp32 rows of uniform values whose magnitudes span 2^-100 .. 2^60, so that the row scales run
+    from far below 2^-64 (where a reciprocal of the scale would overflow) to far above 1, and the
+    quotients by the scale land everywhere between grid points: a quotient off the correctly
+    rounded x / scale by one unit in the last place changes a code about once in 2^20 values."""
+    rng = np.random.default_rng(5)
+    rows, d = 20000, 512
+    mag = np.exp2(rng.uniform(-100, 60, size=(rows, 1)))
+    x32 = (rng.uniform(-1, 1, size=(rows, d)) * mag).astype(np.float32)
+    codes, scales = K.quantize(torch.from_numpy(x32).cuda(), fmt)
+    if fmt == K.FP8_E4M3_ROW:
+        rc, rs = OF.quantize_fp8_rows(x32)
+        assert np.array_equal(scales.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    elif fmt == K.FP8_E4M3_ROW_ROPE_BF16:
+        rc, rs = OF.quantize_fp8_rope_rows(x32)
+        assert np.array_equal(scales.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    else:
+        rc, rs = OF.quantize_fp4_rows(x32)
+        assert np.array_equal(scales.cpu().numpy(), rs)
+    got = codes.cpu().numpy()
+    assert np.array_equal(got, rc), f"{int((got != rc).sum())} codes differ"
