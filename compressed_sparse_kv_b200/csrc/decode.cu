@@ -798,6 +798,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int hd[2] = {16 * wq + g, 16 * wq + 8 + g};
     float m_o[2] = {-INFINITY, -INFINITY}, m_l[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
     bool dead = false;
+    // the inverse-RoPE table (fp64 angles, ~1 us of dependent double-precision
+    // work), while the first tile loads and its QK runs
+    for (int m = threadIdx.x - 64; m < p.rope_dim / 2; m += 128) {
+      float cs, sn;
+      inv_rope_rotation(sq.t, m, p.rope_dim, p.rope_base, &cs, &sn);
+      ctl->rope_cs[m] = cs;
+      ctl->rope_sn[m] = sn;
+      if (p.splits > p.cluster && split == 0) {  // (decode_combine reads it)
+        p.rope_tab[size_t(b) * kDim + m] = cs;
+        p.rope_tab[size_t(b) * kDim + kDim / 2 + m] = sn;
+      }
+    }
     for (int i = 0; i < nt; ++i) {
       const int T = t0 + i, sb = i & 1, stage = i % kStages;
       const bool gathered = C::kQuant || !tile_tma(p, sq, b, T);
@@ -938,17 +950,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->p_full[sb]);
-    }
-    // the inverse-RoPE table (fp64 angles), while the last PV finishes
-    for (int m = threadIdx.x - 64; m < p.rope_dim / 2; m += 128) {
-      float cs, sn;
-      inv_rope_rotation(sq.t, m, p.rope_dim, p.rope_base, &cs, &sn);
-      ctl->rope_cs[m] = cs;
-      ctl->rope_sn[m] = sn;
-      if (p.splits > p.cluster && split == 0) {  // (decode_combine reads it)
-        p.rope_tab[size_t(b) * kDim + m] = cs;
-        p.rope_tab[size_t(b) * kDim + kDim / 2 + m] = sn;
-      }
     }
     if (!dead) dead = !warp_wait(&ctl->o_done, 0, ctl, lane);
     float l_tot[2];
