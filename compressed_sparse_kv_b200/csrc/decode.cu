@@ -1257,9 +1257,11 @@ __global__ void __launch_bounds__(32 * kCombWarps) decode_combine(const uint16_t
 // lane l of every warp owns channels cb D/CB + 128 q + 4l .. + 3 (float4s,
 // q < 4/CB; both channels of a rotary pair sit in one float4), warp w the
 // splits s = w mod kWideWarps, taken 2 CB at a time (one when CB = 1) with all their loads in
-// flight before any is used.  The maxima come first from one pass over the
-// (m, l) terms; the warps' sums meet in shared memory.  CB is chosen per
-// launch so that the grid stays within a few blocks per SM.
+// flight before any is used.  Each warp keeps running maxima of the (m, l)
+// terms it has seen, rescaling its sums when one grows (no separate pass
+// over the maxima); the warps' sums, scaled to the block's maxima, meet in
+// shared memory.  CB is chosen per launch so that the grid stays within a
+// few blocks per SM.
 constexpr int kWideWarps = 8;
 
 template <int CB>
@@ -1281,35 +1283,12 @@ __global__ void __launch_bounds__(32 * kWideWarps, CB == 1 ? 4 : 2) decode_combi
   const size_t ml_stride = size_t(heads) * 4, o_stride = size_t(heads) * kDim;
   const float* mlb = ml_part + (size_t(b) * splits * heads + h) * 4;
   const uint16_t* ob = o_part + (size_t(b) * splits * heads + h) * kDim + CW * cb + 4 * lane;
-  // maxima over all splits
-  float mo = -INFINITY, ml = -INFINITY;
-  for (int s = threadIdx.x; s < splits; s += 32 * kWideWarps) {
-    const float4 v = __ldcg(reinterpret_cast<const float4*>(mlb + s * ml_stride));
-    mo = fmaxf(mo, v.x);
-    ml = fmaxf(ml, v.y);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    mo = fmaxf(mo, __shfl_xor_sync(kFull, mo, o));
-    ml = fmaxf(ml, __shfl_xor_sync(kFull, ml, o));
-  }
-  if (lane == 0) {
-    s_mo[warp] = mo;
-    s_ml[warp] = ml;
-  }
-  __syncthreads();
-  mo = s_mo[0];
-  ml = s_ml[0];
-#pragma unroll
-  for (int w = 1; w < kWideWarps; ++w) {
-    mo = fmaxf(mo, s_mo[w]);
-    ml = fmaxf(ml, s_ml[w]);
-  }
-  // this warp's splits, U per round
+  // this warp's splits, U per round, with running maxima (the warp's loads
+  // are identical across its lanes, so every branch below is warp-uniform)
   float4 acc[Q];
 #pragma unroll
   for (int q = 0; q < Q; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-  float L = 0.f;
+  float L = 0.f, mo = -INFINITY, ml = -INFINITY;
   for (int s0 = warp; s0 < splits; s0 += kWideWarps * U) {
     float4 v[U], x[U][Q];
 #pragma unroll
@@ -1324,6 +1303,27 @@ __global__ void __launch_bounds__(32 * kWideWarps, CB == 1 ? 4 : 2) decode_combi
 #pragma unroll
       for (int q = 0; q < Q; ++q)
         x[u][q] = s < splits ? ld_bf16x4(ob + size_t(s) * o_stride + 128 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float rmo = mo, rml = ml;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      rmo = fmaxf(rmo, v[u].x);
+      rml = fmaxf(rml, v[u].y);
+    }
+    if (rmo > mo) {  // rescale what the warp has summed so far to the new maximum
+      const float a = mo == -INFINITY ? 0.f : exp2f(mo - rmo);
+#pragma unroll
+      for (int q = 0; q < Q; ++q) {
+        acc[q].x *= a;
+        acc[q].y *= a;
+        acc[q].z *= a;
+        acc[q].w *= a;
+      }
+      mo = rmo;
+    }
+    if (rml > ml) {
+      L *= ml == -INFINITY ? 0.f : exp2f(ml - rml);
+      ml = rml;
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -1342,20 +1342,33 @@ __global__ void __launch_bounds__(32 * kWideWarps, CB == 1 ? 4 : 2) decode_combi
   }
 #pragma unroll
   for (int q = 0; q < Q; ++q) *reinterpret_cast<float4*>(&red[warp][128 * q + 4 * lane]) = acc[q];
-  if (lane == 0) s_l[warp] = L;  // every lane carries the same L
+  if (lane == 0) {  // every lane carries the same maxima and L
+    s_mo[warp] = mo;
+    s_ml[warp] = ml;
+    s_l[warp] = L;
+  }
   __syncthreads();
   if (threadIdx.x >= CW / 2) return;
+  float mo_all = -INFINITY, ml_all = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kWideWarps; ++w) {
+    mo_all = fmaxf(mo_all, s_mo[w]);
+    ml_all = fmaxf(ml_all, s_ml[w]);
+  }
   float Lt = 0.f;
 #pragma unroll
-  for (int w = 0; w < kWideWarps; ++w) Lt += s_l[w];
-  const float inv = (mo == -INFINITY || Lt <= 0.f) ? 0.f : exp2f(mo - ml) / Lt;
+  for (int w = 0; w < kWideWarps; ++w)
+    if (s_ml[w] != -INFINITY) Lt += s_l[w] * exp2f(s_ml[w] - ml_all);
+  const float inv = (mo_all == -INFINITY || Lt <= 0.f) ? 0.f : exp2f(mo_all - ml_all) / Lt;
   const int cl = 2 * threadIdx.x, c = CW * cb + cl;  // CW/2 threads x 2 channels
   float v0 = 0.f, v1 = 0.f;
 #pragma unroll
   for (int w = 0; w < kWideWarps; ++w) {
+    if (s_mo[w] == -INFINITY) continue;  // a warp without a used partial
+    const float a = exp2f(s_mo[w] - mo_all);
     const float2 x = *reinterpret_cast<const float2*>(&red[w][cl]);
-    v0 += x.x;
-    v1 += x.y;
+    v0 = fmaf(a, x.x, v0);
+    v1 = fmaf(a, x.y, v1);
   }
   v0 *= inv;
   v1 *= inv;
