@@ -410,23 +410,39 @@ def time_stack(steps, warmup, seed, dist_max):
                 L.step(0)
     stream.synchronize()
     ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * len(layers) + 1)]
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        ev[0].record(stream)
-        for i, L in enumerate(layers):
-            if L.kind == "c4a":
-                L.index(0)
-            ev[2 * i + 1].record(stream)
-            L.decode(0)
-            ev[2 * i + 2].record(stream)
+
+    def capture(events):
+        # events: event nodes around every layer's calls (each one costs the
+        # programmatic-launch overlap at its boundary), for the per-call times
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            if events:
+                ev[0].record(stream)
+            for i, L in enumerate(layers):
+                if L.kind == "c4a":
+                    L.index(0)
+                if events:
+                    ev[2 * i + 1].record(stream)
+                L.decode(0)
+                if events:
+                    ev[2 * i + 2].record(stream)
+        return g
+
+    g = capture(False)       # the timed step
+    g_inst = capture(True)   # the same step with event nodes, for the breakdown
     with torch.cuda.stream(stream):
         for _ in range(3):
             g.replay()
+        g_inst.replay()
     stream.synchronize()
-    # one replay for the per-call breakdown
+    # one instrumented replay for the per-call breakdown
+    inst_start, inst_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
-        g.replay()
+        inst_start.record(stream)
+        g_inst.replay()
+        inst_stop.record(stream)
     stream.synchronize()
+    inst_ms = inst_start.elapsed_time(inst_stop)
     idx_ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i, L in enumerate(layers) if L.kind == "c4a")
     c4a_dec = sum(ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i, L in enumerate(layers) if L.kind == "c4a")
     c128a_ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 2]) for i, L in enumerate(layers) if L.kind == "c128a")
@@ -448,8 +464,10 @@ def time_stack(steps, warmup, seed, dist_max):
            "c4a_layer_us": round((idx_ms + c4a_dec) / n4 * 1e3, 2),
            "c4a_index_us": round(idx_ms / n4 * 1e3, 2),
            "c128a_layer_us": round(c128a_ms / (len(layers) - n4) * 1e3, 2),
+           "breakdown_note": "per-layer times from a replay with event nodes between the calls "
+                             f"({round(inst_ms, 4)} ms per step); the timed step has none",
            "launches_per_step": sum(L.launches_per_step() for L in layers)}
-    del g, layers
+    del g, g_inst, layers
     torch.cuda.empty_cache()
     return res
 
