@@ -1408,7 +1408,10 @@ __device__ int find_threshold_bin256(const uint32_t* h, uint32_t need, uint32_t*
   return r;
 }
 
-template <int FMT>
+// PER: pool positions per thread (PER x 512 >= the pool's capacity).  The
+// kernel is latency-bound and its loops over the positions are unrolled, so
+// pools of up to 2048 entries take PER = 4 (a quarter of the code of PER = 16).
+template <int FMT, int PER>
 __global__ void __launch_bounds__(kSelThreads, 1)
     index_pool_select(const uint16_t* __restrict__ qidx, const void* __restrict__ codes,
                       const uint8_t* __restrict__ kscales, int64_t key_rows, int64_t n,
@@ -1567,9 +1570,9 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   __syncthreads();
   const uint32_t cnt = s_cnt;
   const uint32_t kk = min(uint32_t(k), cnt);
-  uint32_t c[kPoolPer];
+  uint32_t c[PER];
 #pragma unroll
-  for (int j = 0; j < kPoolPer; ++j) {
+  for (int j = 0; j < PER; ++j) {
     const int pos = threadIdx.x + j * kSelThreads;
     c[j] = pos < pool_cap ? pcode[pos] : 0u;
   }
@@ -1581,7 +1584,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) sh[i] = 0;
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < kPoolPer; ++j)
+    for (int j = 0; j < PER; ++j)
       if (c[j] != 0u && int(c[j] >> 20) == bin1) atomicAdd(&sh[(c[j] >> 8) & 0xfffu], 1u);
     __syncthreads();
     const int bin2 = find_threshold_bin<kSelThreads>(sh, kk - above1, &above2);
@@ -1589,7 +1592,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     for (int i = threadIdx.x; i < 256; i += kSelThreads) sh[i] = 0;
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < kPoolPer; ++j)
+    for (int j = 0; j < PER; ++j)
       if (c[j] != 0u && (c[j] >> 8) == prefix) atomicAdd(&sh[c[j] & 0xffu], 1u);
     __syncthreads();
     const int bin3 = find_threshold_bin256(sh, kk - above1 - above2, &above3);
@@ -1597,21 +1600,21 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     need_eq = kk - above1 - above2 - above3;
   }
   // ranks of the entries equal to o*, in pool order
-  uint32_t m[kPoolPer], off[kPoolPer];
+  uint32_t m[PER], off[PER];
 #pragma unroll
-  for (int j = 0; j < kPoolPer; ++j) m[j] = __ballot_sync(kFull, cnt > uint32_t(k) && c[j] == ostar);
-  ordered_offsets<kSelThreads, kPoolPer>(m, off);
+  for (int j = 0; j < PER; ++j) m[j] = __ballot_sync(kFull, cnt > uint32_t(k) && c[j] == ostar);
+  ordered_offsets<kSelThreads, PER>(m, off);
   const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll
-  for (int j = 0; j < kPoolPer; ++j) {
+  for (int j = 0; j < PER; ++j) {
     const bool eq = (m[j] >> lane) & 1u;
     const bool keep = cnt > uint32_t(k) ? (c[j] > ostar || (eq && off[j] + __popc(m[j] & lt) < need_eq)) : c[j] != 0u;
     m[j] = __ballot_sync(kFull, keep);
   }
-  const uint32_t got = ordered_offsets<kSelThreads, kPoolPer>(m, off);
+  const uint32_t got = ordered_offsets<kSelThreads, PER>(m, off);
   int32_t* out = idx_out + size_t(b) * k;
 #pragma unroll
-  for (int j = 0; j < kPoolPer; ++j) {
+  for (int j = 0; j < PER; ++j) {
     if ((m[j] >> lane) & 1u) {
       const uint32_t at = off[j] + __popc(m[j] & lt);
       if (at < kk) out[at] = pent[threadIdx.x + j * kSelThreads];
@@ -1633,24 +1636,39 @@ dsv4kv_status index_topk_pool_launch(const uint16_t* qidx, const dsv4kv_cache& k
   uint32_t* status = static_cast<uint32_t*>(ws);
   static std::atomic<uint64_t> attr{0};  // one bit per device
   if (!done_on_device(attr)) {
-    if (cudaFuncSetAttribute(index_pool_select<DSV4KV_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(index_pool_select<DSV4KV_BF16, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(kPoolDyn)) != cudaSuccess ||
-        cudaFuncSetAttribute(index_pool_select<DSV4KV_FP4_E2M1_G16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(kPoolDyn)) != cudaSuccess)
+        cudaFuncSetAttribute(index_pool_select<DSV4KV_BF16, kPoolPer>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(kPoolDyn)) != cudaSuccess ||
+        cudaFuncSetAttribute(index_pool_select<DSV4KV_FP4_E2M1_G16, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(kPoolDyn)) != cudaSuccess ||
+        cudaFuncSetAttribute(index_pool_select<DSV4KV_FP4_E2M1_G16, kPoolPer>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(kPoolDyn)) != cudaSuccess)
       return check_launch("index_topk_pool: cudaFuncSetAttribute");
     mark_done_on_device(attr);
   }
   // C CTAs per sequence, as many as keep the grid within one CTA per SM
   const int csize = std::max(1, std::min(kMaxPoolCluster, sm_count() / std::max(batch, 1)));
   const dim3 grid{static_cast<unsigned>(csize), static_cast<unsigned>(batch)};
-  if (keys.fmt == DSV4KV_BF16)
-    launch_pdl_cluster(index_pool_select<DSV4KV_BF16>, grid, dim3(kSelThreads), kPoolDyn, unsigned(csize), stream,
-                       qidx, keys.codes, static_cast<const uint8_t*>(keys.scales), keys.rows, n, pool, pool_cap, k,
-                       idx_out, count_out, status);
-  else
-    launch_pdl_cluster(index_pool_select<DSV4KV_FP4_E2M1_G16>, grid, dim3(kSelThreads), kPoolDyn, unsigned(csize),
-                       stream, qidx, keys.codes, static_cast<const uint8_t*>(keys.scales), keys.rows, n, pool,
-                       pool_cap, k, idx_out, count_out, status);
+  const bool small = pool_cap <= 4 * kSelThreads;
+  const void* kc = keys.codes;
+  const uint8_t* ks = static_cast<const uint8_t*>(keys.scales);
+  if (keys.fmt == DSV4KV_BF16) {
+    if (small)
+      launch_pdl_cluster(index_pool_select<DSV4KV_BF16, 4>, grid, dim3(kSelThreads), kPoolDyn, unsigned(csize), stream,
+                         qidx, kc, ks, keys.rows, n, pool, pool_cap, k, idx_out, count_out, status);
+    else
+      launch_pdl_cluster(index_pool_select<DSV4KV_BF16, kPoolPer>, grid, dim3(kSelThreads), kPoolDyn, unsigned(csize),
+                         stream, qidx, kc, ks, keys.rows, n, pool, pool_cap, k, idx_out, count_out, status);
+  } else {
+    if (small)
+      launch_pdl_cluster(index_pool_select<DSV4KV_FP4_E2M1_G16, 4>, grid, dim3(kSelThreads), kPoolDyn, unsigned(csize),
+                         stream, qidx, kc, ks, keys.rows, n, pool, pool_cap, k, idx_out, count_out, status);
+    else
+      launch_pdl_cluster(index_pool_select<DSV4KV_FP4_E2M1_G16, kPoolPer>, grid, dim3(kSelThreads), kPoolDyn,
+                         unsigned(csize), stream, qidx, kc, ks, keys.rows, n, pool, pool_cap, k, idx_out, count_out,
+                         status);
+  }
   return check_launch("index_pool_select");
 }
 
