@@ -20,7 +20,11 @@
 // is due, warp w sums the taps j = w, w + 8, ... and the warps' sums are
 // added in warp order through shared memory before the rotation.  The
 // rotation uses an fp64 angle reduced exactly modulo 2 pi (as the batch
-// compressor).
+// compressor); the cos / sin of every rotary pair at the window row's and at
+// the entry's position are computed once per CTA, one pair per lane, by
+// warps 1 and 2 while warp 0 copies the raw row (each is a dependent chain of
+// double-precision work; the lanes that own the rotary channels would
+// otherwise run 8 of them one after another).
 #include <cstdint>
 
 #include "common.cuh"
@@ -32,9 +36,21 @@ namespace {
 
 constexpr int kAppendWarps = 8;
 
+// cos / sin of the angle pos * rope_base^(-2m / rope_dim) of every rotary
+// pair m, the angle in units of pi reduced exactly modulo 2; lane l takes
+// pairs l, l + 32, ...
+__device__ __forceinline__ void rope_table(double* cs, double* sn, int rope_dim, double rope_base, double pos,
+                                           int lane) {
+  for (int m = lane; m < rope_dim / 2; m += 32) {
+    const double ang = pos * (pow(rope_base, -2.0 * double(m) / double(rope_dim)) / 3.141592653589793);
+    const double xr = ang - 2.0 * rint(0.5 * ang);
+    sincospi(xr, &sn[m], &cs[m]);
+  }
+}
+
 template <int PER>
-__device__ __forceinline__ void rope_pairs(float (&v)[PER], int c0, int dim, int rope_dim, double rope_base,
-                                           double pos) {
+__device__ __forceinline__ void rope_pairs(float (&v)[PER], int c0, int dim, int rope_dim, const double* cs,
+                                           const double* sn) {
   const int r0 = dim - rope_dim;
   if (c0 + PER <= r0) return;
 #pragma unroll
@@ -42,13 +58,9 @@ __device__ __forceinline__ void rope_pairs(float (&v)[PER], int c0, int dim, int
     const int c = c0 + e;
     if (c >= r0) {
       const int m = (c - r0) >> 1;
-      const double ang = pos * (pow(rope_base, -2.0 * double(m) / double(rope_dim)) / 3.141592653589793);
-      const double xr = ang - 2.0 * rint(0.5 * ang);
-      double sn, cs;
-      sincospi(xr, &sn, &cs);
       const float x = v[e], y = v[e + 1];
-      v[e] = float(double(x) * cs - double(y) * sn);
-      v[e + 1] = float(double(x) * sn + double(y) * cs);
+      v[e] = float(double(x) * cs[m] - double(y) * sn[m]);
+      v[e + 1] = float(double(x) * sn[m] + double(y) * cs[m]);
     }
   }
 }
@@ -69,6 +81,12 @@ __global__ void __launch_bounds__(32 * kAppendWarps)
                   uint16_t* __restrict__ win_ring, uint16_t* __restrict__ comp, int64_t comp_rows, int64_t emit) {
   constexpr int D = 32 * PER;
   __shared__ __align__(16) float red[kAppendWarps][D];
+  extern __shared__ double rtab[];  // cos, sin at the window row's position; cos, sin at the entry's
+  const int np = rope_dim / 2;
+  double* w_cs = rtab;
+  double* w_sn = rtab + np;
+  double* e_cs = rtab + 2 * np;
+  double* e_sn = rtab + 3 * np;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x;
   const int c0 = PER * lane;
@@ -76,13 +94,18 @@ __global__ void __launch_bounds__(32 * kAppendWarps)
   const uint16_t* xs = s_new + size_t(b) * D + c0;
   pdl_trigger();
   pdl_wait();
+  uint4 raw[PER / 8];
   if (warp == 0) {
-    uint4 raw[PER / 8];
 #pragma unroll
     for (int q = 0; q < PER / 8; ++q) raw[q] = *reinterpret_cast<const uint4*>(xs + 8 * q);
     uint16_t* rr = raw_ring + (size_t(b) * size_t(ring) + size_t(t % ring)) * D + c0;
 #pragma unroll
     for (int q = 0; q < PER / 8; ++q) *reinterpret_cast<uint4*>(rr + 8 * q) = raw[q];
+  }
+  if (warp == 1 && window > 0) rope_table(w_cs, w_sn, rope_dim, rope_base, double(t), lane);
+  if (warp == 2 && emit >= 0) rope_table(e_cs, e_sn, rope_dim, rope_base, double(int64_t(stride) * emit), lane);
+  __syncthreads();
+  if (warp == 0) {
     if (window > 0) {
       float v[PER];
 #pragma unroll
@@ -92,7 +115,7 @@ __global__ void __launch_bounds__(32 * kAppendWarps)
         v[8 * q + 4] = bf16lo(raw[q].z); v[8 * q + 5] = bf16hi(raw[q].z);
         v[8 * q + 6] = bf16lo(raw[q].w); v[8 * q + 7] = bf16hi(raw[q].w);
       }
-      rope_pairs<PER>(v, c0, D, rope_dim, rope_base, double(t));
+      rope_pairs<PER>(v, c0, D, rope_dim, w_cs, w_sn);
       store_bf16_row<PER>(win_ring + (size_t(b) * size_t(window) + size_t(t % window)) * D + c0, v);
     }
   }
@@ -136,7 +159,7 @@ __global__ void __launch_bounds__(32 * kAppendWarps)
     for (int ww = 1; ww < kAppendWarps; ++ww) sum += red[ww][c0 + e];
     v[e] = sum;
   }
-  rope_pairs<PER>(v, c0, D, rope_dim, rope_base, double(int64_t(stride) * emit));
+  rope_pairs<PER>(v, c0, D, rope_dim, e_cs, e_sn);
   store_bf16_row<PER>(comp + (size_t(b) * size_t(comp_rows) + size_t(emit)) * D + c0, v);
 }
 
@@ -157,17 +180,18 @@ dsv4kv_status append_launch(const void* s_new, const float* w, int batch, int64_
   uint16_t* wr = static_cast<uint16_t*>(win_ring);
   uint16_t* cp = static_cast<uint16_t*>(comp);
   const dim3 grid{static_cast<unsigned>(batch)}, block{32 * kAppendWarps};
+  const size_t tab = size_t(rope_dim / 2) * 4 * sizeof(double);  // two positions x (cos, sin) per rotary pair
   switch (dim) {
     case 256:
-      launch_pdl(append_kernel<8>, grid, block, 0, stream, s, w, t, k_taps, stride, window, rope_dim, rope_base, rr,
+      launch_pdl(append_kernel<8>, grid, block, tab, stream, s, w, t, k_taps, stride, window, rope_dim, rope_base, rr,
                  wr, cp, comp_rows, emit);
       break;
     case 512:
-      launch_pdl(append_kernel<16>, grid, block, 0, stream, s, w, t, k_taps, stride, window, rope_dim, rope_base, rr,
+      launch_pdl(append_kernel<16>, grid, block, tab, stream, s, w, t, k_taps, stride, window, rope_dim, rope_base, rr,
                  wr, cp, comp_rows, emit);
       break;
     case 1024:
-      launch_pdl(append_kernel<32>, grid, block, 0, stream, s, w, t, k_taps, stride, window, rope_dim, rope_base, rr,
+      launch_pdl(append_kernel<32>, grid, block, tab, stream, s, w, t, k_taps, stride, window, rope_dim, rope_base, rr,
                  wr, cp, comp_rows, emit);
       break;
     default:
