@@ -1573,6 +1573,8 @@ dsv4kv_status decode_launch(const DecodeArgs& a, void* ws, size_t ws_bytes, cuda
   const Plan pl = make_plan(a.batch, comp_tiles, win_tiles);
   const DecodeWs w = decode_ws_layout(static_cast<char*>(ws), a.batch, a.heads, pl);
   if (ws_bytes < w.bytes) return set_error(DSV4KV_ERR_WORKSPACE, "decode: workspace too small");
+  if (reinterpret_cast<uintptr_t>(ws) % 16 != 0)  // (the split statistics are 16-byte stores)
+    return set_error(DSV4KV_ERR_INVALID_ARG, "decode: workspace not 16-byte aligned");
 
   CUtensorMap tq, tc, tw;
   // One box brings a whole operand in the layout the MMAs read: dimensions

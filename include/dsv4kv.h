@@ -22,7 +22,9 @@
  *  - Return value: DSV4KV_OK or an error code; on an error nothing was
  *    launched (DSV4KV_ERR_CUDA: a launch failed — the text is in
  *    dsv4kv_last_error(), and the workspace must be zero-filled again).
- *  - Workspaces: `*_workspace_bytes` gives the size; a workspace must be
+ *  - Workspaces: `*_workspace_bytes` gives the size; a workspace is 16-byte
+ *    aligned (as every cudaMalloc'd block is; the decode calls return
+ *    DSV4KV_ERR_INVALID_ARG otherwise), and it must be
  *    zero-filled once before its first use and is left in that state by every
  *    successful call, so it can be reused by the next call on the same stream.
  *    Calls that run concurrently need separate workspaces.  The first 4 bytes

@@ -177,3 +177,19 @@ def test_split_merge_paths(monkeypatch, max_cluster, kind, b, n, t):
             ref = OA.sparse_decode(_q_host(kq, s, h)[None], sel_rows[None], win_rows[None],
                                    np.arange(k, dtype=np.int32)[None], t, SCALE)[0]
         assert_close(got[s], ref, what=f"seq {s} (max cluster {max_cluster})")
+
+
+def test_unaligned_workspace_is_rejected():
+    """A workspace that is not 16-byte aligned is refused on the host (its
+    16-byte statistics stores would otherwise fault); nothing is launched."""
+    q, comp, win, _ = _inputs(3, 2, 64, 300, 128)
+    n, t = 300, 300 * 128 + 128
+    need = K.dense_decode_workspace_bytes(2, 64, n, 128)
+    ws = K.new_workspace(need + 32)[8:8 + need + 16]
+    assert ws.data_ptr() % 16 == 8
+    with pytest.raises(K.Dsv4kvError) as e:
+        K.dense_decode(q, K.Cache(0, comp), K.Cache(0, win), n, 128, t, ws=ws)
+    assert e.value.status == 1
+    # the same call on an aligned workspace runs
+    out = K.dense_decode(q, K.Cache(0, comp), K.Cache(0, win), n, 128, t)
+    assert torch.isfinite(out.float()).all()
