@@ -17,6 +17,27 @@ def scaled_max_abs(ref) -> float:
     return MAX_ABS * max(1.0, float(np.max(np.abs(np.asarray(ref, dtype=np.float64)))))
 
 
+def bf16_half_ulp(x) -> np.ndarray:
+    """Half the spacing of bf16 values (8 significand bits) in the binade of |x|."""
+    ax = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.maximum(ax, 2.0 ** -126)))
+    return np.exp2(e - 8)
+
+
+def assert_bf16_rounding_of(got, ref, what="", acc_rel=1e-5):
+    """Outputs stored in bf16 from an fp32 computation: each is a bf16
+    rounding of a value within acc_rel x max(1, |ref|) of the exact ref, so it
+    lies within half a bf16 ulp of ref plus that.  (Comparing with the bf16
+    rounding of ref itself fails by one ulp wherever ref and the fp32 value
+    straddle a rounding midpoint.)"""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    err = np.abs(got - ref)
+    bad = err > bf16_half_ulp(ref) + acc_rel * np.maximum(1.0, np.abs(ref))
+    assert not bad.any(), f"{what}: {int(bad.sum())} outputs beyond half a bf16 ulp, worst error {err[bad].max():.3e}"
+
+
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 

@@ -1,4 +1,6 @@
 """dsv4kv_compress against the oracle (c4a and c128a, bf16 and fp32 outputs)."""
+import zlib
+
 import numpy as np
 import pytest
 import torch
@@ -7,7 +9,7 @@ import compressed_sparse_kv_b200 as K
 import datagen as D
 from oracle import compress as OC
 from oracle import formats as OF
-from tests._util import assert_close, to_f64
+from tests._util import assert_bf16_rounding_of, assert_close, scaled_max_abs, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -29,7 +31,7 @@ def _raw(seed, b, t, d=512):
 @pytest.mark.parametrize("out_fp32", [True, False])
 def test_compress(kind, b, t, window, pos0, out_fp32):
     s, k = (4, 8) if kind == "c4a" else (128, 128)
-    raw, key = _raw(hash((kind, t)) % 1000, b, t)
+    raw, key = _raw(zlib.crc32(f"{kind}-{t}".encode()) % 1000, b, t)  # (a fixed seed per case)
     w = D.compress_weights(5, 0, k, 512)
     out = K.compress(raw, torch.from_numpy(w).cuda(), s, window, pos0=pos0, out_fp32=out_fp32)
     n = OC.n_entries(t, window, s)
@@ -38,12 +40,14 @@ def test_compress(kind, b, t, window, pos0, out_fp32):
     for bb in range(b):
         r = OF.bf16_bits_to_f64(D.normal_bf16(key, t * 512, offset=bb * t * 512).reshape(t, 512))
         ref = OC.compress(r, w.astype(np.float64), s, window, pos0=pos0)
-        if not out_fp32:
-            ref_stored = OF.round_bf16(ref)
-            assert_close(got[bb], ref_stored, what=f"{kind} seq {bb}")
-        assert_close(got[bb], ref, what=f"{kind} seq {bb}")
         if out_fp32:
+            assert_close(got[bb], ref, what=f"{kind} seq {bb}")
             assert np.abs(got[bb] - ref).max() < 1e-4       # fp32 accumulation of <= 128 taps
+        else:
+            # every stored value is a bf16 rounding of the fp32 entry; the
+            # entries reach |x| ~ 5, where half a bf16 ulp exceeds 1e-2
+            assert_bf16_rounding_of(got[bb], ref, what=f"{kind} seq {bb}")
+            assert_close(got[bb], ref, max_abs=scaled_max_abs(ref), what=f"{kind} seq {bb}")
 
 
 def test_window_rows_are_one_tap_compression():
