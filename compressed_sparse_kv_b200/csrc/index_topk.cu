@@ -498,6 +498,10 @@ constexpr int kSelStage = 4096;                        // candidates a CTA can h
 // that code cost more than the rare fallback saves (16 per thread: the
 // selection 17.3 -> 14.3 us per call at B = 32).
 constexpr int kCandCap = 2048;
+// entries of the leader's receive buffer: CTA r of a C-CTA cluster pushes its
+// list into region r (kRecvCap / C entries), so the candidates of one part of
+// a sequence (scores that cluster by position) fit as well as spread ones
+constexpr int kRecvCap = 8192;
 constexpr int kResPer = kCandCap / kSelThreads;        // candidates per leader thread
 constexpr int kMaxClusterSel = 16;
 constexpr int kWarpCap = kSelStage / kSelWarps;       // candidates a warp's list can hold
@@ -507,9 +511,8 @@ constexpr int kWarpCap = kSelStage / kSelWarps;       // candidates a warp's lis
 constexpr int kRing = 4;
 constexpr size_t kRingBytes = size_t(kSelWarps) * kRing * kSelWarpSpan * sizeof(float);  // 64 KB
 // dynamic shared memory: the rings, the warps' lists (kSelStage u64), and the
-// leader's receive buffer (kCandCap): CTA r of the cluster pushes its list
-// into region r (kCandCap / C entries)
-constexpr size_t kSelDyn = kRingBytes + (size_t(kSelStage) + kCandCap) * sizeof(uint64_t);
+// leader's receive buffer (kRecvCap u64)
+constexpr size_t kSelDyn = kRingBytes + (size_t(kSelStage) + kRecvCap) * sizeof(uint64_t);
 
 // Block-wide exclusive prefix sum of one value per thread (NT threads).
 template <int NT>
@@ -1169,7 +1172,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select(const float* __re
   //    its region of the leader's receive buffer (remote shared-memory stores),
   //    and its count; a list or region that overflowed sends the sequence to
   //    the exact fallback
-  const uint32_t regcap = uint32_t(kCandCap) / csize;
+  const uint32_t regcap = uint32_t(kRecvCap) / csize;
   uint64_t* recv = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(stage) + kRingBytes) + kSelStage;
   {
     uint32_t off = 0, tot = 0;
