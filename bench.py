@@ -642,17 +642,22 @@ def time_e2e(layer, steps):
     host memory, all inside the timed region.
 
     The steps run as a three-stage pipeline over three streams (upload,
-    compute, download) with NB sets of device and pinned host buffers: step
-    i's upload and step i-1's download overlap step i-1's / i's calls, and
-    events order every reuse of a buffer.  The whole pipeline of `steps`
-    steps (copies, calls and event dependencies) is captured once into one
-    CUDA graph and replayed, the way a serving loop launches its decode
+    compute, download), in chunks of C steps with two sets of C device and
+    pinned host buffers: the uploads of chunk c (one copy per step) overlap
+    the calls of chunk c-1, every step's download follows its calls, and
+    events order every reuse of a buffer.  The compute stream waits on the
+    other streams once per chunk: a cross-stream dependency in front of a
+    step's first kernel costs the programmatic-launch overlap with the
+    previous step's last kernel.  The whole pipeline of `steps` steps
+    (copies, calls and event dependencies) is captured once into one CUDA
+    graph and replayed, the way a serving loop launches its decode
     iterations without a host round trip per kernel.  The eager figure issues
     the same copies and calls from Python step by step.  Returns (graph ms,
     eager ms, H2D bytes per step, D2H bytes per step)."""
     torch = layer.torch
     R = len(layer.reps)
-    NB = 3
+    C = 3                                                  # steps per chunk
+    NB = 2 * C                                             # buffer sets: two chunks' worth
     lanes = [layer.twin() for _ in range(NB)]             # own output buffers and workspaces per set
     q_host = [layer.q.cpu().pin_memory() for _ in range(NB)]
     qi_host = [layer.qidx.cpu().pin_memory() for _ in range(NB)]
@@ -660,9 +665,10 @@ def time_e2e(layer, steps):
     q_dev = [torch.empty_like(layer.q) for _ in range(NB)]
     qi_dev = [torch.empty_like(layer.qidx) for _ in range(NB)]
     s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    ev_in = [torch.cuda.Event() for _ in range(NB)]
-    ev_comp = [torch.cuda.Event() for _ in range(NB)]
-    ev_out = [torch.cuda.Event() for _ in range(NB)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]       # per chunk parity: the chunk's inputs are up
+    ev_comp = [torch.cuda.Event() for _ in range(2)]     # the chunk's calls are done (its inputs read)
+    ev_out = [torch.cuda.Event() for _ in range(2)]      # the chunk's outputs are down
+    ev_step = [torch.cuda.Event() for _ in range(NB)]    # one step's calls are done
 
     def calls(j, r):
         L = lanes[j]
@@ -682,25 +688,31 @@ def time_e2e(layer, steps):
         fork.record(head)
         for s in (s_in, s_comp, s_out):
             s.wait_event(fork)
-        for i in range(steps):
-            j, r = i % NB, i % R
-            if i >= NB:
-                s_in.wait_event(ev_comp[j])            # step i - NB's calls have read this input set
+        for c in range((steps + C - 1) // C):
+            cp = c % 2
+            chunk = range(c * C, min(steps, (c + 1) * C))
+            if c >= 2:
+                s_in.wait_event(ev_comp[cp])           # chunk c - 2's calls have read these input sets
             with torch.cuda.stream(s_in):
-                q_dev[j].copy_(q_host[j], non_blocking=True)
-                if layer.kind == "c4a":
-                    qi_dev[j].copy_(qi_host[j], non_blocking=True)
-            ev_in[j].record(s_in)
-            s_comp.wait_event(ev_in[j])
-            if i >= NB:
-                s_comp.wait_event(ev_out[j])           # step i - NB's output has left this set
-            with torch.cuda.stream(s_comp):
-                calls(j, r)
-            ev_comp[j].record(s_comp)
-            s_out.wait_event(ev_comp[j])
-            with torch.cuda.stream(s_out):
-                out_host[j].copy_(lanes[j].out, non_blocking=True)
-            ev_out[j].record(s_out)
+                for i in chunk:
+                    j = cp * C + i % C
+                    q_dev[j].copy_(q_host[j], non_blocking=True)
+                    if layer.kind == "c4a":
+                        qi_dev[j].copy_(qi_host[j], non_blocking=True)
+            ev_in[cp].record(s_in)
+            s_comp.wait_event(ev_in[cp])
+            if c >= 2:
+                s_comp.wait_event(ev_out[cp])          # chunk c - 2's outputs have left these sets
+            for i in chunk:
+                j, r = cp * C + i % C, i % R
+                with torch.cuda.stream(s_comp):
+                    calls(j, r)
+                ev_step[j].record(s_comp)
+                s_out.wait_event(ev_step[j])
+                with torch.cuda.stream(s_out):
+                    out_host[j].copy_(lanes[j].out, non_blocking=True)
+            ev_comp[cp].record(s_comp)
+            ev_out[cp].record(s_out)
         for s in (s_in, s_comp, s_out):                # join every stream back into the head
             e = torch.cuda.Event()
             e.record(s)
